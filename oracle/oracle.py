@@ -1,0 +1,201 @@
+"""ctypes front end for the plain-C oracle (oracle/vq_oracle.c).
+
+TEST INFRASTRUCTURE ONLY: imported by tests/, by __graft_entry__.smoke() and by
+bench.py's cpu_baseline / reference arm.  The product library never imports it.
+
+All arrays are numpy arrays; fp16/bf16 data are uint16 bit patterns.  Results are
+fp64 numpy arrays (or uint16 bits for rounded weights).
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+SRC = os.path.join(HERE, "vq_oracle.c")
+LIB = os.path.join(HERE, "liboracle.so")
+
+FMT_RVQ12, FMT_RVQ12_4, FMT_VQ16 = 1, 2, 3
+DT_F16, DT_BF16 = 0, 1
+
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile vq_oracle.c into liboracle.so with gcc (strict IEEE: no contraction, no fast-math)."""
+    if force or not os.path.exists(LIB) or os.path.getmtime(LIB) < os.path.getmtime(SRC):
+        tmp = LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math",
+                               "-shared", "-fPIC", "-o", tmp, SRC, "-lm"])
+        os.replace(tmp, LIB)
+    return LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = ctypes.CDLL(LIB)
+            P = ctypes.c_void_p
+            I = ctypes.c_int
+            lib.vqo_f16_to_f64.restype = ctypes.c_double
+            lib.vqo_f16_to_f64.argtypes = [ctypes.c_uint16]
+            lib.vqo_bf16_to_f64.restype = ctypes.c_double
+            lib.vqo_bf16_to_f64.argtypes = [ctypes.c_uint16]
+            lib.vqo_f64_to_f16.restype = ctypes.c_uint16
+            lib.vqo_f64_to_f16.argtypes = [ctypes.c_double]
+            lib.vqo_f64_to_bf16.restype = ctypes.c_uint16
+            lib.vqo_f64_to_bf16.argtypes = [ctypes.c_double]
+            lib.vqo_fl32.restype = ctypes.c_double
+            lib.vqo_fl32.argtypes = [ctypes.c_double]
+            lib.vqo_decode_array.restype = None
+            lib.vqo_decode_array.argtypes = [P, ctypes.c_int64, I, P]
+            lib.vqo_rht_f64.restype = I
+            lib.vqo_rht_f64.argtypes = [I, I, P, P, P]
+            lib.vqo_round_array.restype = None
+            lib.vqo_round_array.argtypes = [P, ctypes.c_int64, I, P]
+            lib.vqo_unpack.restype = I
+            lib.vqo_unpack.argtypes = [I, I, I, P, P, P, P, P, P]
+            lib.vqo_dequant.restype = I
+            lib.vqo_dequant.argtypes = [I, I, I, P, P, P, P, P, P, P, I, P, P, I]
+            lib.vqo_forward.restype = I
+            lib.vqo_forward.argtypes = [I, I, I, I, P, I, P, P, P, P, P, P, P, I, P]
+            lib.vqo_rht.restype = I
+            lib.vqo_rht.argtypes = [I, I, P, I, P, P]
+            _lib = lib
+    return _lib
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype):
+    return None if a is None else np.ascontiguousarray(a, dtype=dtype)
+
+
+def decode(bits, dt: int) -> np.ndarray:
+    """fp16 (dt=0) or bf16 (dt=1) bit patterns -> fp64 values."""
+    lib = _load()
+    b = _c(bits, np.uint16)
+    out = np.empty(b.shape, dtype=np.float64)
+    lib.vqo_decode_array(_p(b), b.size, dt, _p(out))
+    return out
+
+
+def f16_to_f64(bits) -> np.ndarray:
+    return decode(bits, DT_F16)
+
+
+def bf16_to_f64(bits) -> np.ndarray:
+    return decode(bits, DT_BF16)
+
+
+def round_to(values, dt: int) -> np.ndarray:
+    """Round fp64 values to fp16 (dt=0) or bf16 (dt=1) bits, ties to even."""
+    lib = _load()
+    v = _c(values, np.float64)
+    out = np.empty(v.shape, dtype=np.uint16)
+    lib.vqo_round_array(_p(v), v.size, dt, _p(out))
+    return out
+
+
+def fl32(v: float) -> float:
+    return _load().vqo_fl32(float(v))
+
+
+def _planes(layer):
+    return (_c(layer.get("lo"), np.uint8), _c(layer.get("hi4"), np.uint8), _c(layer.get("s2"), np.uint8),
+            _c(layer.get("idx16"), np.uint16))
+
+
+def unpack(layer) -> tuple[np.ndarray, np.ndarray]:
+    """Return (i1 uint32 [N,G], i2 uint8 [N,G]) for a layer dict from ``synth.make_layer``."""
+    lib = _load()
+    spec = layer["spec"]
+    lo, hi4, s2, idx16 = _planes(layer)
+    i1 = np.empty((spec.N, spec.G), dtype=np.uint32)
+    i2 = np.empty((spec.N, spec.G), dtype=np.uint8)
+    rc = lib.vqo_unpack(spec.fmt, spec.N, spec.K, _p(lo), _p(hi4), _p(s2), _p(idx16), _p(i1), _p(i2))
+    if rc:
+        raise ValueError(f"vqo_unpack failed rc={rc}")
+    return i1, i2
+
+
+def dequant(layer, wdt: int = DT_F16) -> tuple[np.ndarray, np.ndarray]:
+    """Return (W exact fp64 [N,K], W materialised fp16/bf16 bits [N,K])."""
+    lib = _load()
+    spec = layer["spec"]
+    lo, hi4, s2, idx16 = _planes(layer)
+    cb1, cb2, sc = _c(layer["cb1"], np.uint16), _c(layer.get("cb2"), np.uint16), _c(layer["scales"], np.uint16)
+    w = np.empty((spec.N, spec.K), dtype=np.float64)
+    wb = np.empty((spec.N, spec.K), dtype=np.uint16)
+    rc = lib.vqo_dequant(spec.fmt, spec.N, spec.K, _p(lo), _p(hi4), _p(s2), _p(idx16), _p(cb1), _p(cb2),
+                         _p(sc), spec.scale_group, _p(w), _p(wb), wdt)
+    if rc:
+        raise ValueError(f"vqo_dequant failed rc={rc}")
+    return w, wb
+
+
+def forward(layer, x_bits, xdt: int) -> np.ndarray:
+    """y[m][n] = sum_k x[m][k] W[n][k] in fp64 (x given as fp16/bf16 bits [M,K])."""
+    lib = _load()
+    spec = layer["spec"]
+    x = _c(x_bits, np.uint16)
+    M = x.shape[0]
+    if x.shape[1] != spec.K:
+        raise ValueError("x has the wrong K")
+    lo, hi4, s2, idx16 = _planes(layer)
+    cb1, cb2, sc = _c(layer["cb1"], np.uint16), _c(layer.get("cb2"), np.uint16), _c(layer["scales"], np.uint16)
+    y = np.empty((M, spec.N), dtype=np.float64)
+    rc = lib.vqo_forward(spec.fmt, M, spec.N, spec.K, _p(x), xdt, _p(lo), _p(hi4), _p(s2), _p(idx16), _p(cb1),
+                         _p(cb2), _p(sc), spec.scale_group, _p(y))
+    if rc:
+        raise ValueError(f"vqo_forward failed rc={rc}")
+    return y
+
+
+def rht(x_bits, xdt: int, signs) -> np.ndarray:
+    """Rotated activations (1/sqrt K) H (signs * x) in fp64, x given as bits [M,K]."""
+    lib = _load()
+    x = _c(x_bits, np.uint16)
+    sg = _c(signs, np.int8)
+    M, K = x.shape
+    out = np.empty((M, K), dtype=np.float64)
+    rc = lib.vqo_rht(M, K, _p(x), xdt, _p(sg), _p(out))
+    if rc:
+        raise ValueError(f"vqo_rht failed rc={rc}")
+    return out
+
+
+def rht_f64(x, signs) -> np.ndarray:
+    """Rotation of fp64 activations [M,K]: (1/sqrt K) H (signs * x)."""
+    lib = _load()
+    xd = _c(x, np.float64)
+    sg = _c(signs, np.int8)
+    M, K = xd.shape
+    out = np.empty((M, K), dtype=np.float64)
+    rc = lib.vqo_rht_f64(M, K, _p(xd), _p(sg), _p(out))
+    if rc:
+        raise ValueError(f"vqo_rht_f64 failed rc={rc}")
+    return out
+
+
+def tolerance(x_bits, xdt: int, w_exact: np.ndarray, coeff: float = 2e-3) -> np.ndarray:
+    """Per-token bound coeff * ||x_m||_2 * max|w| used for the y comparison, shape [M, 1]."""
+    xd = widen(np.asarray(x_bits, dtype=np.uint16), xdt)
+    return coeff * np.sqrt((xd * xd).sum(axis=1, keepdims=True)) * np.abs(w_exact).max()
+
+
+def widen(bits: np.ndarray, xdt: int) -> np.ndarray:
+    """fp16/bf16 bits -> fp64 through numpy widening (exact); used to size tolerances."""
+    if xdt == DT_F16:
+        return bits.view(np.float16).astype(np.float64)
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)

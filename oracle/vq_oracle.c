@@ -1,0 +1,290 @@
+/*
+ * vq_oracle.c -- plain, slow CPU oracle for the codebook-VQ linear layer.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may link, load or call
+ * this file: it is used by tests/, by __graft_entry__.smoke() (to check one tiny
+ * GPU call) and by bench.py's cpu_baseline / reference arm.  It shares no code,
+ * header, table or helper with the CUDA library.
+ *
+ * What it computes, and where the pages define it:
+ *   - orka README, "How it works": every group of 8 consecutive weights is one
+ *     codebook index; indices are stored as 12-bit bit-planes (a low-byte plane
+ *     plus a packed high plane); decode is scale x sum over stages of
+ *     codebook_s[index_s].  "rvq-12-4" is a 12-bit stage 1 plus a 4-bit stage 2.
+ *   - GLQ README, "How it works" (E8 lattice codebooks): one 16-bit index per group
+ *     of 8 into a 65,536-entry table; "Randomized Hadamard Transform": random sign
+ *     flips followed by a fast Walsh-Hadamard transform.
+ *   - GLQ README, "Inference kernels": Y = X . dequant(W)^T without materialising W.
+ *
+ * Readings taken where the pages are silent (all fixed here, by construction):
+ *   - groups run along K (the input dimension); planes are row-major [N][G], G=K/8;
+ *   - "packed hi": two 4-bit fields per byte, group 2t in bits 0..3, 2t+1 in 4..7;
+ *     the 4-bit stage-2 plane is packed the same way;
+ *   - the 16-bit index plane is one little-endian uint16 per group;
+ *   - stages are summed with no residual scale (any such scale is folded into
+ *     the stage-2 codebook);
+ *   - scales are per 64-weight block along K within a row, or one per row
+ *     (scale_group == K);
+ *   - materialised weights are rounded at two points: c = fl32(cb1 + cb2),
+ *     p = fl32(s * c), then round-to-nearest-even to fp16 or bf16;
+ *   - the rotation is x' = (1/sqrt K) H_K (sigma .* x) with the Sylvester
+ *     Hadamard matrix H[k][j] = (-1)^popcount(k & j), signs applied first.
+ *
+ * Every floating-point value is handled in fp64.  fp16 / bf16 / fp32 values are
+ * decoded and rounded with converters written from the IEEE-754 binary formats
+ * (round to nearest, ties to even), not with library conversions.
+ *
+ * Parity is pinned for every function here by tests/test_oracle_pins.py.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define VQO_FMT_RVQ12 1
+#define VQO_FMT_RVQ12_4 2
+#define VQO_FMT_VQ16 3
+
+#define VQO_DT_F16 0
+#define VQO_DT_BF16 1
+#define VQO_DT_F32 2
+
+/* ---------------------------------------------------------------------------
+ * Binary floating-point formats with `ebits` exponent bits and `mbits`
+ * fraction bits (binary16: 5/10, bfloat16: 8/7, binary32: 8/23).
+ * ------------------------------------------------------------------------- */
+
+/* Value of a bit pattern of the format (IEEE-754 interpretation). */
+static double vqo_decode_bits(uint32_t bits, int ebits, int mbits) {
+  const int bias = (1 << (ebits - 1)) - 1;
+  const uint32_t emax_field = (1u << ebits) - 1u;
+  const uint32_t sign = (bits >> (ebits + mbits)) & 1u;
+  const uint32_t efield = (bits >> mbits) & emax_field;
+  const uint32_t frac = bits & ((1u << mbits) - 1u);
+  double v;
+  if (efield == 0) {
+    v = ldexp((double)frac, 1 - bias - mbits); /* zero or subnormal */
+  } else if (efield == emax_field) {
+    v = frac ? NAN : INFINITY;
+  } else {
+    v = ldexp((double)((1u << mbits) | frac), (int)efield - bias - mbits);
+  }
+  return sign ? -v : v;
+}
+
+/* Round half to even of a non-negative double q (q is an exact scaled value). */
+static double vqo_rne(double q) {
+  double r = floor(q);
+  double f = q - r;
+  if (f > 0.5 || (f == 0.5 && fmod(r, 2.0) != 0.0)) r += 1.0;
+  return r;
+}
+
+/* Round v to the nearest value of the format, ties to even; return the bits. */
+static uint32_t vqo_round_bits(double v, int ebits, int mbits) {
+  const int bias = (1 << (ebits - 1)) - 1;
+  const int emin = 1 - bias, emax = bias;
+  const uint32_t sign = signbit(v) ? (1u << (ebits + mbits)) : 0u;
+  const uint32_t inf = ((1u << ebits) - 1u) << mbits;
+  if (isnan(v)) return inf | (1u << (mbits - 1)); /* quiet NaN */
+  double a = fabs(v);
+  if (isinf(a)) return sign | inf;
+  if (a == 0.0) return sign;
+  int ex;
+  frexp(a, &ex);      /* a = f * 2^ex, f in [0.5, 1) */
+  int e = ex - 1;     /* a in [2^e, 2^(e+1)) */
+  if (e < emin) e = emin; /* subnormal range: fixed spacing 2^(emin - mbits) */
+  double q = ldexp(a, mbits - e); /* exact: scaling by a power of two */
+  double r = vqo_rne(q);
+  const double one = ldexp(1.0, mbits); /* implicit leading bit */
+  if (r >= 2.0 * one) { r = one; e += 1; }
+  if (r >= one) {
+    if (e > emax) return sign | inf;
+    return sign | ((uint32_t)(e + bias) << mbits) | (uint32_t)(r - one);
+  }
+  return sign | (uint32_t)r; /* subnormal, biased exponent 0 */
+}
+
+double vqo_f16_to_f64(uint16_t h) { return vqo_decode_bits(h, 5, 10); }
+double vqo_bf16_to_f64(uint16_t b) { return vqo_decode_bits(b, 8, 7); }
+uint16_t vqo_f64_to_f16(double v) { return (uint16_t)vqo_round_bits(v, 5, 10); }
+uint16_t vqo_f64_to_bf16(double v) { return (uint16_t)vqo_round_bits(v, 8, 7); }
+/* fl32(v): v rounded to binary32, returned as an fp64 value. */
+double vqo_fl32(double v) { return vqo_decode_bits(vqo_round_bits(v, 8, 23), 8, 23); }
+
+static double vqo_act_to_f64(uint16_t bits, int dt) {
+  return dt == VQO_DT_BF16 ? vqo_bf16_to_f64(bits) : vqo_f16_to_f64(bits);
+}
+
+/* Decode an array of fp16 or bf16 bit patterns to fp64. */
+void vqo_decode_array(const uint16_t* in, int64_t n, int dt, double* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = vqo_act_to_f64(in[i], dt);
+}
+
+/* Round an array of fp64 values to fp16 or bf16 bits. */
+void vqo_round_array(const double* in, int64_t n, int dt, uint16_t* out) {
+  for (int64_t i = 0; i < n; ++i)
+    out[i] = dt == VQO_DT_BF16 ? vqo_f64_to_bf16(in[i]) : vqo_f64_to_f16(in[i]);
+}
+
+/* ---------------------------------------------------------------------------
+ * Unpack (orka README, "How it works": 12-bit bit-planes, lo byte + packed hi;
+ * GLQ README: one 16-bit index per 8-weight group).
+ * i1[n][g] is the stage-1 (or 16-bit) index, i2[n][g] the stage-2 index (0 if
+ * the format has no second stage).
+ * ------------------------------------------------------------------------- */
+static int vqo_nibble(uint8_t byte, int g) { return (g & 1) ? (byte >> 4) : (byte & 15); }
+
+int vqo_unpack(int fmt, int N, int K, const uint8_t* lo, const uint8_t* hi4, const uint8_t* s2,
+               const uint16_t* idx16, uint32_t* i1, uint8_t* i2) {
+  if (N < 0 || K <= 0 || K % 16 != 0) return 1;
+  const int G = K / 8;
+  for (int n = 0; n < N; ++n) {
+    for (int g = 0; g < G; ++g) {
+      uint32_t a = 0;
+      int b = 0;
+      if (fmt == VQO_FMT_VQ16) {
+        a = idx16[(int64_t)n * G + g];
+      } else if (fmt == VQO_FMT_RVQ12 || fmt == VQO_FMT_RVQ12_4) {
+        uint32_t low = lo[(int64_t)n * G + g];
+        uint32_t high = (uint32_t)vqo_nibble(hi4[(int64_t)n * (G / 2) + g / 2], g);
+        a = low + 256u * high;
+        if (fmt == VQO_FMT_RVQ12_4) b = vqo_nibble(s2[(int64_t)n * (G / 2) + g / 2], g);
+      } else {
+        return 2;
+      }
+      i1[(int64_t)n * G + g] = a;
+      i2[(int64_t)n * G + g] = (uint8_t)b;
+    }
+  }
+  return 0;
+}
+
+/* ---------------------------------------------------------------------------
+ * Decode (orka README, "How it works": scale x sum(codebook[index])).
+ * For weight (n, k): group g = k / 8, position j = k % 8, scale block
+ * k / scale_group.  w_exact is the exact fp64 value s * (c1 + c2); w_bits is
+ * the materialised weight RN(fl32(s * fl32(c1 + c2))) in fp16 or bf16.
+ * ------------------------------------------------------------------------- */
+static double vqo_weight_exact(int fmt, int n, int k, int K, const uint32_t* i1, const uint8_t* i2,
+                               const uint16_t* cb1, const uint16_t* cb2, const uint16_t* scales,
+                               int scale_group, double* c_out, double* s_out) {
+  const int G = K / 8, g = k / 8, j = k % 8;
+  double c = vqo_f16_to_f64(cb1[(int64_t)i1[(int64_t)n * G + g] * 8 + j]);
+  if (fmt == VQO_FMT_RVQ12_4) c += vqo_f16_to_f64(cb2[(int64_t)i2[(int64_t)n * G + g] * 8 + j]);
+  const int nblk = K / scale_group;
+  double s = vqo_f16_to_f64(scales[(int64_t)n * nblk + k / scale_group]);
+  *c_out = c;
+  *s_out = s;
+  return s * c;
+}
+
+static int vqo_check(int fmt, int N, int K, int scale_group) {
+  if (N < 0 || K <= 0 || K % 16 != 0) return 1;
+  if (scale_group <= 0 || scale_group % 8 != 0 || K % scale_group != 0) return 1;
+  if (fmt != VQO_FMT_RVQ12 && fmt != VQO_FMT_RVQ12_4 && fmt != VQO_FMT_VQ16) return 2;
+  return 0;
+}
+
+int vqo_dequant(int fmt, int N, int K, const uint8_t* lo, const uint8_t* hi4, const uint8_t* s2,
+                const uint16_t* idx16, const uint16_t* cb1, const uint16_t* cb2, const uint16_t* scales,
+                int scale_group, double* w_exact, uint16_t* w_bits, int wdt) {
+  int rc = vqo_check(fmt, N, K, scale_group);
+  if (rc) return rc;
+  const int G = K / 8;
+  uint32_t* i1 = (uint32_t*)malloc(sizeof(uint32_t) * (size_t)N * G + 1);
+  uint8_t* i2 = (uint8_t*)malloc((size_t)N * G + 1);
+  if (!i1 || !i2) { free(i1); free(i2); return 3; }
+  rc = vqo_unpack(fmt, N, K, lo, hi4, s2, idx16, i1, i2);
+  for (int n = 0; rc == 0 && n < N; ++n) {
+    for (int k = 0; k < K; ++k) {
+      double c, s;
+      double w = vqo_weight_exact(fmt, n, k, K, i1, i2, cb1, cb2, scales, scale_group, &c, &s);
+      if (w_exact) w_exact[(int64_t)n * K + k] = w;
+      if (w_bits) {
+        double c32 = vqo_fl32(c);      /* stage sum rounded to fp32 */
+        double p32 = vqo_fl32(s * c32); /* exact product of two fp32-representable values, rounded */
+        w_bits[(int64_t)n * K + k] = wdt == VQO_DT_BF16 ? vqo_f64_to_bf16(p32) : vqo_f64_to_f16(p32);
+      }
+    }
+  }
+  free(i1);
+  free(i2);
+  return rc;
+}
+
+/* ---------------------------------------------------------------------------
+ * Forward (GLQ README, "Inference kernels": Y = X . dequant(W)^T).
+ * y[m][n] = sum_k x[m][k] * W[n][k], with W the exact fp64 decode, x taken
+ * exactly from its fp16/bf16 bits, a naive loop over k in order.
+ * ------------------------------------------------------------------------- */
+int vqo_forward(int fmt, int M, int N, int K, const uint16_t* x, int xdt, const uint8_t* lo,
+                const uint8_t* hi4, const uint8_t* s2, const uint16_t* idx16, const uint16_t* cb1,
+                const uint16_t* cb2, const uint16_t* scales, int scale_group, double* y) {
+  int rc = vqo_check(fmt, N, K, scale_group);
+  if (rc || M < 0) return rc ? rc : 1;
+  const int G = K / 8;
+  uint32_t* i1 = (uint32_t*)malloc(sizeof(uint32_t) * (size_t)N * G + 1);
+  uint8_t* i2 = (uint8_t*)malloc((size_t)N * G + 1);
+  double* wrow = (double*)malloc(sizeof(double) * (size_t)K);
+  double* xd = (double*)malloc(sizeof(double) * (size_t)M * K + 1);
+  if (!i1 || !i2 || !wrow || !xd) { free(i1); free(i2); free(wrow); free(xd); return 3; }
+  rc = vqo_unpack(fmt, N, K, lo, hi4, s2, idx16, i1, i2);
+  for (int64_t t = 0; rc == 0 && t < (int64_t)M * K; ++t) xd[t] = vqo_act_to_f64(x[t], xdt);
+  for (int n = 0; rc == 0 && n < N; ++n) {
+    for (int k = 0; k < K; ++k) {
+      double c, s;
+      wrow[k] = vqo_weight_exact(fmt, n, k, K, i1, i2, cb1, cb2, scales, scale_group, &c, &s);
+    }
+    for (int m = 0; m < M; ++m) {
+      double acc = 0.0;
+      for (int k = 0; k < K; ++k) acc += xd[(int64_t)m * K + k] * wrow[k];
+      y[(int64_t)m * N + n] = acc;
+    }
+  }
+  free(i1);
+  free(i2);
+  free(wrow);
+  free(xd);
+  return rc;
+}
+
+/* ---------------------------------------------------------------------------
+ * Input rotation (GLQ README, "How it works", Randomized Hadamard Transform:
+ * random sign flips followed by a Walsh-Hadamard transform).  Written as the
+ * explicit O(K^2) matrix-vector product with the Sylvester matrix, not as a
+ * butterfly: out[m][k] = (1/sqrt K) sum_j (-1)^popcount(k & j) sigma_j x[m][j].
+ * ------------------------------------------------------------------------- */
+static int vqo_parity(uint32_t v) {
+  int p = 0;
+  while (v) { p ^= 1; v &= v - 1; }
+  return p;
+}
+
+int vqo_rht_f64(int M, int K, const double* x, const int8_t* signs, double* out) {
+  if (M < 0 || K <= 0 || (K & (K - 1)) != 0) return 1;
+  double* row = (double*)malloc(sizeof(double) * (size_t)K);
+  if (!row) return 3;
+  const double inv_sqrt_k = 1.0 / sqrt((double)K);
+  for (int m = 0; m < M; ++m) {
+    for (int j = 0; j < K; ++j) row[j] = (double)signs[j] * x[(int64_t)m * K + j];
+    for (int k = 0; k < K; ++k) {
+      double acc = 0.0;
+      for (int j = 0; j < K; ++j) acc += vqo_parity((uint32_t)(k & j)) ? -row[j] : row[j];
+      out[(int64_t)m * K + k] = acc * inv_sqrt_k;
+    }
+  }
+  free(row);
+  return 0;
+}
+
+/* Same rotation with x given as fp16 / bf16 bits (taken exactly). */
+int vqo_rht(int M, int K, const uint16_t* x, int xdt, const int8_t* signs, double* out) {
+  if (M < 0 || K <= 0 || (K & (K - 1)) != 0) return 1;
+  double* xd = (double*)malloc(sizeof(double) * (size_t)M * K + 1);
+  if (!xd) return 3;
+  vqo_decode_array(x, (int64_t)M * K, xdt, xd);
+  int rc = vqo_rht_f64(M, K, xd, signs, out);
+  free(xd);
+  return rc;
+}

@@ -1,0 +1,300 @@
+"""Pins for the CPU oracle against facts that do not come from the oracle itself.
+
+Each test fixes one part of the oracle to something independent: an exhaustive
+comparison with numpy/torch IEEE conversions, hand-worked golden values, a
+brute-force dense matmul written separately here, the Sylvester Hadamard matrix
+from scipy, or an algebraic identity (one-hot columns, linearity, involution).
+"""
+
+import json
+import os
+
+import numpy as np
+import pytest
+import scipy.linalg
+import torch
+
+from synth import FMT_RVQ12, FMT_RVQ12_4, FMT_VQ16, DT_BF16, DT_F16, LayerSpec, make_layer, make_x
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# --------------------------------------------------------------------------- converters
+
+def test_f16_decode_exhaustive(oracle):
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    ours = oracle.decode(bits, DT_F16)
+    ref = bits.view(np.float16).astype(np.float64)
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(ours), nan)
+    assert np.array_equal(ours[~nan], ref[~nan])
+    # signed zeros keep their sign
+    assert np.array_equal(np.signbit(ours[~nan]), np.signbit(ref[~nan]))
+
+
+def test_f16_round_trip_exhaustive(oracle):
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    vals = bits.view(np.float16).astype(np.float64)
+    keep = ~np.isnan(vals)
+    assert np.array_equal(oracle.round_to(vals[keep], DT_F16), bits[keep])
+
+
+def test_f16_round_matches_numpy_on_doubles(oracle):
+    rng = np.random.default_rng(1)
+    mag = np.exp2(rng.uniform(-30, 17, size=200_000))
+    v = mag * rng.choice([-1.0, 1.0], size=mag.size)
+    v = np.concatenate([v, rng.standard_normal(50_000) * 1e-6])
+    ours = oracle.round_to(v, DT_F16)
+    ref = v.astype(np.float16).view(np.uint16)  # numpy rounds double -> half directly (RN-even)
+    assert np.array_equal(ours, ref)
+
+
+def test_f16_ties_and_limits_by_hand(oracle):
+    cases = {
+        1.0 + 2.0 ** -11: 0x3C00,         # halfway between 1 and 1+2^-10 -> even (1.0)
+        1.0 + 3 * 2.0 ** -11: 0x3C02,     # halfway between 1+2^-10 and 1+2^-9 -> even
+        65504.0: 0x7BFF,                  # largest finite
+        65519.99: 0x7BFF,
+        65520.0: 0x7C00,                  # halfway to 2^16 rounds to even = inf
+        2.0 ** -24: 0x0001,               # smallest subnormal
+        2.0 ** -25: 0x0000,               # halfway to zero -> even (0)
+        3 * 2.0 ** -25: 0x0002,           # halfway between 1 and 2 subnormal steps -> even
+        -2.0 ** -14: 0x8400,              # smallest normal, negative
+        -0.0: 0x8000,
+    }
+    got = oracle.round_to(np.array(list(cases.keys())), DT_F16)
+    assert [int(g) for g in got] == list(cases.values())
+
+
+def test_bf16_decode_exhaustive(oracle):
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    ours = oracle.decode(bits, DT_BF16)
+    ref = (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(ours), nan)
+    assert np.array_equal(ours[~nan], ref[~nan])
+
+
+def test_bf16_round_matches_torch(oracle):
+    rng = np.random.default_rng(2)
+    f = (np.exp2(rng.uniform(-130, 127, size=200_000)) * rng.choice([-1.0, 1.0], size=200_000)).astype(np.float32)
+    f = np.concatenate([f, rng.standard_normal(50_000).astype(np.float32)])
+    ours = oracle.round_to(f.astype(np.float64), DT_BF16)
+    ref = torch.from_numpy(f).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(ours, ref)
+
+
+def test_fl32_matches_numpy(oracle):
+    rng = np.random.default_rng(3)
+    v = np.exp2(rng.uniform(-140, 120, size=2000)) * rng.choice([-1.0, 1.0], size=2000)
+    for a in v:
+        assert oracle.fl32(a) == float(np.float32(a))
+
+
+# --------------------------------------------------------------------------- unpack
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def test_unpack_golden_layout(oracle):
+    g = _golden("unpack_layout.json")
+    spec = LayerSpec(g["N"], g["K"], FMT_RVQ12_4, 32)
+    layer = {"spec": spec, "lo": np.array(g["lo"], np.uint8), "hi4": np.array(g["hi4"], np.uint8),
+             "s2": np.array(g["s2"], np.uint8)}
+    i1, i2 = oracle.unpack(layer)
+    assert i1.tolist() == g["i1"]
+    assert i2.tolist() == g["i2"]
+
+
+def _pack12(i1, i2=None):
+    """Pack indices into the plane layout (written here from the layout description)."""
+    N, G = i1.shape
+    lo = (i1 & 0xFF).astype(np.uint8)
+    hi = (i1 >> 8).astype(np.uint8)
+    hi4 = (hi[:, 0::2] | (hi[:, 1::2] << 4)).astype(np.uint8)
+    out = {"lo": lo, "hi4": hi4}
+    if i2 is not None:
+        out["s2"] = (i2[:, 0::2] | (i2[:, 1::2] << 4)).astype(np.uint8)
+    return out
+
+
+def test_unpack_round_trip_all_12bit_values_both_parities(oracle):
+    vals = np.arange(4096, dtype=np.uint32)
+    G = 64
+    # every value at an even group and at an odd group
+    i1 = np.concatenate([vals.reshape(-1, G), np.roll(vals, 1).reshape(-1, G)])
+    i2 = ((np.arange(i1.size, dtype=np.uint32) // 2) % 16).reshape(i1.shape)
+    layer = {"spec": LayerSpec(i1.shape[0], G * 8, FMT_RVQ12_4, 64), **_pack12(i1, i2)}
+    o1, o2 = oracle.unpack(layer)
+    assert np.array_equal(o1, i1)
+    assert np.array_equal(o2, i2)
+    # every stage-2 value at both parities
+    assert set(map(int, o2[:, 0::2].ravel())) == set(range(16))
+    assert set(map(int, o2[:, 1::2].ravel())) == set(range(16))
+
+
+def test_unpack_round_trip_all_16bit_values(oracle):
+    vals = np.arange(65536, dtype=np.uint32).astype(np.uint16).reshape(-1, 256)
+    layer = {"spec": LayerSpec(vals.shape[0], 256 * 8, FMT_VQ16, 2048), "idx16": vals}
+    o1, o2 = oracle.unpack(layer)
+    assert np.array_equal(o1, vals.astype(np.uint32))
+    assert not o2.any()
+
+
+# --------------------------------------------------------------------------- decode
+
+def _tiny_layer_from_golden(g):
+    cb1 = np.zeros((4096, 8), np.float16)
+    for k, row in g["cb1_rows"].items():
+        cb1[int(k)] = row
+    cb2 = np.zeros((16, 8), np.float16)
+    for k, row in g["cb2_rows"].items():
+        cb2[int(k)] = row
+    i1 = np.array([g["i1"]], np.uint32)
+    i2 = np.array([g["i2"]], np.uint32)
+    spec = LayerSpec(g["N"], g["K"], g["fmt"], g["scale_group"])
+    return {"spec": spec, "cb1": cb1.view(np.uint16), "cb2": cb2.view(np.uint16),
+            "scales": np.array([g["scales"]], np.float16).view(np.uint16), **_pack12(i1, i2)}
+
+
+def test_decode_golden_tiny_codebooks(oracle):
+    g = _golden("decode_tiny.json")
+    layer = _tiny_layer_from_golden(g)
+    w, wb = oracle.dequant(layer, DT_F16)
+    assert w[0].tolist() == g["w"]
+    # every golden weight is exact in fp16, so the materialised weights are those values
+    assert wb[0].view(np.float16).astype(np.float64).tolist() == g["w"]
+
+
+def _one_group_layer(c1, c2, s, fmt=FMT_RVQ12_4):
+    cb1 = np.zeros((4096, 8), np.float16)
+    cb2 = np.zeros((16, 8), np.float16)
+    cb1[5, 0] = c1
+    cb2[7, 0] = c2
+    i1 = np.array([[5, 5]], np.uint32)
+    i2 = np.array([[7, 7]], np.uint32)
+    return {"spec": LayerSpec(1, 16, fmt, 16), "cb1": cb1.view(np.uint16), "cb2": cb2.view(np.uint16),
+            "scales": np.array([[s]], np.float16).view(np.uint16), **_pack12(i1, i2)}
+
+
+@pytest.mark.parametrize("c1,c2,s,dt,expect", [
+    (2048.0, 2.0 ** -14, 1.0, DT_F16, 0x6800),             # fl32(2048 + 2^-14) = 2048
+    (1.0, 2.0 ** -11, 1.0, DT_F16, 0x3C00),                # 1 + 2^-11 ties to even in fp16
+    (1.0, 3 * 2.0 ** -11, 1.0, DT_F16, 0x3C02),            # 1 + 3*2^-11 ties to even (up)
+    (1.0, 2.0 ** -8, 1.0, DT_BF16, 0x3F80),                # 1 + 2^-8 ties to even in bf16
+    (1.0, 3 * 2.0 ** -8, 1.0, DT_BF16, 0x3F82),
+    (3.0, 0.0, -0.5, DT_F16, 0xBE00),                      # scale applied after the stage sum
+    (1024.0, 1.0, 2.0 ** -10, DT_F16, 0x3C01),             # (1025) * 2^-10 = 1 + 2^-10
+])
+def test_decode_rounding_points_by_hand(oracle, c1, c2, s, dt, expect):
+    w, wb = oracle.dequant(_one_group_layer(c1, c2, s), dt)
+    assert int(wb[0, 0]) == expect
+    assert w[0, 0] == s * (c1 + c2)
+
+
+# --------------------------------------------------------------------------- forward
+
+def _dense_numpy(layer):
+    """Brute-force dense W, built here independently with numpy fancy indexing."""
+    spec = layer["spec"]
+    cb1 = layer["cb1"].view(np.float16).astype(np.float64)
+    if spec.fmt == FMT_VQ16:
+        i1 = layer["idx16"].astype(np.int64)
+    else:
+        hi = np.empty((spec.N, spec.G), np.int64)
+        hi[:, 0::2] = layer["hi4"] & 15
+        hi[:, 1::2] = layer["hi4"] >> 4
+        i1 = layer["lo"].astype(np.int64) + 256 * hi
+    W = cb1[i1]  # [N, G, 8]
+    if spec.fmt == FMT_RVQ12_4:
+        i2 = np.empty((spec.N, spec.G), np.int64)
+        i2[:, 0::2] = layer["s2"] & 15
+        i2[:, 1::2] = layer["s2"] >> 4
+        W = W + layer["cb2"].view(np.float16).astype(np.float64)[i2]
+    W = W.reshape(spec.N, spec.K)
+    sc = layer["scales"].view(np.float16).astype(np.float64)
+    return W * np.repeat(sc, spec.scale_group, axis=1)
+
+
+@pytest.mark.parametrize("fmt,sg", [(FMT_RVQ12, 8), (FMT_RVQ12_4, 16), (FMT_VQ16, 16), (FMT_RVQ12_4, 8)])
+@pytest.mark.parametrize("xdt", [DT_F16, DT_BF16])
+def test_forward_brute_force_16x16(oracle, fmt, sg, xdt):
+    layer = make_layer(LayerSpec(16, 16, fmt, sg), cfg_id=99, tensor_id=fmt * 10 + sg)
+    x = make_x(5, 16, xdt, cfg_id=99)
+    W = _dense_numpy(layer)
+    xd = x.view(np.float16).astype(np.float64) if xdt == DT_F16 else \
+        (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    ref = xd @ W.T
+    y = oracle.forward(layer, x, xdt)
+    assert np.allclose(y, ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
+    w, _ = oracle.dequant(layer)
+    assert np.array_equal(w, W)
+
+
+def test_forward_one_hot_returns_columns(oracle):
+    spec = LayerSpec(24, 64, FMT_RVQ12_4, 64)
+    layer = make_layer(spec, cfg_id=98)
+    w, _ = oracle.dequant(layer)
+    ks = [0, 7, 8, 33, 63]
+    x = np.zeros((len(ks), spec.K), np.float16)
+    for r, k in enumerate(ks):
+        x[r, k] = 1.0
+    y = oracle.forward(layer, x.view(np.uint16), DT_F16)
+    for r, k in enumerate(ks):
+        assert np.array_equal(y[r], w[:, k])
+
+
+def test_forward_linearity(oracle):
+    spec = LayerSpec(32, 128, FMT_RVQ12_4, 64)
+    layer = make_layer(spec, cfg_id=97)
+    rng = np.random.default_rng(4)
+    x1 = rng.integers(-8, 9, size=(3, spec.K)).astype(np.float16)
+    x2 = rng.integers(-8, 9, size=(3, spec.K)).astype(np.float16)
+    x3 = (2 * x1.astype(np.float64) - 3 * x2.astype(np.float64)).astype(np.float16)  # exact small integers
+    y1, y2, y3 = (oracle.forward(layer, v.view(np.uint16), DT_F16) for v in (x1, x2, x3))
+    assert np.allclose(y3, 2 * y1 - 3 * y2, rtol=1e-12, atol=1e-12 * np.abs(y3).max())
+
+
+# --------------------------------------------------------------------------- rotation
+
+@pytest.mark.parametrize("K", [1, 2, 4, 8, 64, 256])
+def test_rht_matches_sylvester_hadamard(oracle, K):
+    rng = np.random.default_rng(K)
+    x = rng.standard_normal((3, K))
+    signs = rng.choice([-1, 1], size=K).astype(np.int8)
+    ref = (scipy.linalg.hadamard(K).astype(np.float64) @ (signs * x).T).T / np.sqrt(K)
+    assert np.allclose(oracle.rht_f64(x, signs), ref, rtol=1e-13, atol=1e-13)
+
+
+def test_rht_small_cases_by_hand(oracle):
+    out = oracle.rht_f64(np.array([[3.0]]), np.array([-1], np.int8))
+    assert out.tolist() == [[-3.0]]
+    a, b = 5.0, 2.0
+    out = oracle.rht_f64(np.array([[a, b]]), np.array([1, -1], np.int8))
+    r = 1 / np.sqrt(2)
+    assert np.allclose(out, [[(a - b) * r, (a + b) * r]], rtol=1e-15)
+
+
+def test_rht_identities(oracle):
+    K = 128
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((4, K))
+    ones = np.ones(K, np.int8)
+    assert np.allclose(oracle.rht_f64(oracle.rht_f64(x, ones), ones), x, atol=1e-13)  # H/sqrt(K) is an involution
+    signs = rng.choice([-1, 1], size=K).astype(np.int8)
+    y = oracle.rht_f64(x, signs)
+    assert np.allclose(np.linalg.norm(y, axis=1), np.linalg.norm(x, axis=1), rtol=1e-13)  # orthogonal
+    assert np.allclose(y @ y.T, x @ x.T, atol=1e-12)
+    e0 = np.zeros((1, K))
+    e0[0, 0] = 1.0
+    assert np.allclose(oracle.rht_f64(e0, ones), np.full((1, K), 1 / np.sqrt(K)), rtol=1e-15)
+
+
+def test_rht_bits_entry_matches_f64(oracle):
+    K = 64
+    x = make_x(2, K, DT_BF16, cfg_id=96)
+    signs = np.where(np.arange(K) % 3 == 0, -1, 1).astype(np.int8)
+    xd = (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    assert np.array_equal(oracle.rht(x, DT_BF16, signs), oracle.rht_f64(xd, signs))
