@@ -1,0 +1,171 @@
+"""ctypes binding of libvqlinear's C ABI (include/vqlinear.h).
+
+Argument marshalling only: every function here passes plain pointers and sizes
+to the library of the same name and turns a non-OK status into ``VQError``.
+Tensors are torch CUDA tensors (device memory and streams come from PyTorch);
+their ``data_ptr()`` is what crosses the ABI.  There is no fallback: if the
+shared library is missing or fails to load, ``load()`` raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libvqlinear.so")
+
+VQ_OK, VQ_ERR_INVALID_ARG, VQ_ERR_UNSUPPORTED, VQ_ERR_CUDA, VQ_ERR_NOMEM, VQ_ERR_TIMEOUT = range(6)
+VQ_FMT_RVQ12, VQ_FMT_RVQ12_4, VQ_FMT_VQ16 = 1, 2, 3
+VQ_F16, VQ_BF16 = 0, 1
+VQ_PATH_AUTO, VQ_PATH_LUT, VQ_PATH_GEMV, VQ_PATH_TC = 0, 1, 2, 3
+
+STATUS_NAMES = {0: "VQ_OK", 1: "VQ_ERR_INVALID_ARG", 2: "VQ_ERR_UNSUPPORTED", 3: "VQ_ERR_CUDA",
+                4: "VQ_ERR_NOMEM", 5: "VQ_ERR_TIMEOUT"}
+
+# Every entry point the header declares (checked by the tests against the .so).
+EXPORTS = ("vq_abi_version", "vq_linear_create", "vq_linear_destroy", "vq_linear_set_path", "vq_linear_forward",
+           "vq_linear_launches", "vq_rht_apply", "vq_linear_check", "vq_last_error", "vq_debug_unpack",
+           "vq_debug_dequant")
+
+
+class VQError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+class vq_linear_desc(ctypes.Structure):
+    _fields_ = [("N", ctypes.c_int32), ("K", ctypes.c_int32), ("fmt", ctypes.c_int32),
+                ("scale_group", ctypes.c_int32), ("act_dtype", ctypes.c_int32), ("max_M", ctypes.c_int32),
+                ("rht", ctypes.c_int32)]
+
+
+class vq_planes(ctypes.Structure):
+    _fields_ = [("lo", ctypes.c_void_p), ("hi4", ctypes.c_void_p), ("s2", ctypes.c_void_p),
+                ("idx16", ctypes.c_void_p)]
+
+
+class vq_codebooks(ctypes.Structure):
+    _fields_ = [("cb1", ctypes.c_void_p), ("cb2", ctypes.c_void_p)]
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def load(path: str | None = None):
+    """Load libvqlinear.so and declare its signatures (raises if it is missing)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        p = path or LIB_PATH
+        if not os.path.exists(p):
+            raise ImportError(f"{p} is missing: build it with compressed_index_matmul_b200.build.build()")
+        lib = ctypes.CDLL(p)
+        P, I32 = ctypes.c_void_p, ctypes.c_int32
+        st = ctypes.c_int
+        lib.vq_abi_version.restype = I32
+        lib.vq_abi_version.argtypes = []
+        lib.vq_last_error.restype = ctypes.c_char_p
+        lib.vq_last_error.argtypes = []
+        lib.vq_linear_create.restype = st
+        lib.vq_linear_create.argtypes = [ctypes.POINTER(vq_linear_desc), ctypes.POINTER(P)]
+        lib.vq_linear_destroy.restype = st
+        lib.vq_linear_destroy.argtypes = [P]
+        lib.vq_linear_set_path.restype = st
+        lib.vq_linear_set_path.argtypes = [P, I32]
+        lib.vq_linear_forward.restype = st
+        lib.vq_linear_forward.argtypes = [P, P, ctypes.POINTER(vq_planes), ctypes.POINTER(vq_codebooks), P, P,
+                                          I32, I32, I32, P]
+        lib.vq_linear_launches.restype = I32
+        lib.vq_linear_launches.argtypes = [P, I32]
+        lib.vq_rht_apply.restype = st
+        lib.vq_rht_apply.argtypes = [P, P, P, I32, I32, I32, P]
+        lib.vq_linear_check.restype = st
+        lib.vq_linear_check.argtypes = [P, P]
+        lib.vq_debug_unpack.restype = st
+        lib.vq_debug_unpack.argtypes = [P, ctypes.POINTER(vq_planes), P, P, P]
+        lib.vq_debug_dequant.restype = st
+        lib.vq_debug_dequant.argtypes = [P, ctypes.POINTER(vq_planes), ctypes.POINTER(vq_codebooks), P, P, I32, P]
+        _lib = lib
+        return lib
+
+
+def _check(status: int):
+    if status != VQ_OK:
+        raise VQError(status, load().vq_last_error().decode(errors="replace"))
+
+
+def _ptr(t) -> int | None:
+    """Device address of a tensor (or an int address, or None)."""
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        import torch
+
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def make_planes(lo=None, hi4=None, s2=None, idx16=None) -> vq_planes:
+    return vq_planes(_ptr(lo), _ptr(hi4), _ptr(s2), _ptr(idx16))
+
+
+def make_codebooks(cb1, cb2=None) -> vq_codebooks:
+    return vq_codebooks(_ptr(cb1), _ptr(cb2))
+
+
+def vq_abi_version() -> int:
+    return load().vq_abi_version()
+
+
+def vq_linear_create(N, K, fmt, scale_group, act_dtype, max_M, rht=0) -> int:
+    d = vq_linear_desc(N, K, fmt, scale_group, act_dtype, max_M, rht)
+    h = ctypes.c_void_p()
+    _check(load().vq_linear_create(ctypes.byref(d), ctypes.byref(h)))
+    return h.value
+
+
+def vq_linear_destroy(h) -> None:
+    _check(load().vq_linear_destroy(h))
+
+
+def vq_linear_set_path(h, path: int) -> None:
+    _check(load().vq_linear_set_path(h, path))
+
+
+def vq_linear_launches(h, M: int) -> int:
+    return load().vq_linear_launches(h, M)
+
+
+def vq_linear_forward(h, x, planes: vq_planes, codebooks: vq_codebooks, scales, y, M, N, K, stream=None) -> None:
+    _check(load().vq_linear_forward(h, _ptr(x), ctypes.byref(planes), ctypes.byref(codebooks), _ptr(scales),
+                                    _ptr(y), M, N, K, _stream(stream)))
+
+
+def vq_rht_apply(x, x_out, signs, M, K, dtype, stream=None) -> None:
+    _check(load().vq_rht_apply(_ptr(x), _ptr(x_out), _ptr(signs), M, K, dtype, _stream(stream)))
+
+
+def vq_linear_check(h, stream=None) -> None:
+    _check(load().vq_linear_check(h, _stream(stream)))
+
+
+def vq_debug_unpack(h, planes: vq_planes, i1_out, i2_out=None, stream=None) -> None:
+    _check(load().vq_debug_unpack(h, ctypes.byref(planes), _ptr(i1_out), _ptr(i2_out), _stream(stream)))
+
+
+def vq_debug_dequant(h, planes: vq_planes, codebooks: vq_codebooks, scales, w_out, wdt, stream=None) -> None:
+    _check(load().vq_debug_dequant(h, ctypes.byref(planes), ctypes.byref(codebooks), _ptr(scales), _ptr(w_out),
+                                   wdt, _stream(stream)))

@@ -1,0 +1,346 @@
+// C ABI front end of libvqlinear: argument validation, handle management, the
+// per-forward plan and kernel dispatch.  Every argument problem is caught here,
+// on the host, before anything is enqueued.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "internal.h"
+#include "vqlinear.h"
+
+#define VQ_API extern "C" __attribute__((visibility("default")))
+
+namespace vq {
+void plan_gemv(const vq_linear_desc& d, const DeviceInfo& dev, int M, Plan* p);
+bool plan_lut(const vq_linear_desc& d, const DeviceInfo& dev, int M, Plan* p);
+bool plan_tc(const vq_linear_desc& d, const DeviceInfo& dev, int M, Plan* p);
+}  // namespace vq
+
+struct vq_linear_s {
+  vq_linear_desc d;
+  vq::DeviceInfo dev;
+  int path;
+  float* scratch;
+  size_t scratch_bytes;
+  uint32_t* tickets;  // completion counters, zeroed at create, left zero by every forward
+  int num_tickets;
+  uint32_t* err;      // device word, set by bounded waits that gave up
+};
+
+namespace {
+
+thread_local std::string t_err;
+
+vq_status fail(vq_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  t_err = buf;
+  return st;
+}
+
+vq_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(VQ_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+vq_status check_ptr(const void* p, const char* name) {
+  if (p == nullptr) return fail(VQ_ERR_INVALID_ARG, "%s is NULL", name);
+  if (!aligned16(p)) return fail(VQ_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+  return VQ_OK;
+}
+
+vq_status validate_desc(const vq_linear_desc* d) {
+  if (d == nullptr) return fail(VQ_ERR_INVALID_ARG, "desc is NULL");
+  if (d->N <= 0 || d->K <= 0) return fail(VQ_ERR_INVALID_ARG, "N=%d and K=%d must be positive", d->N, d->K);
+  if (d->K % 16 != 0) return fail(VQ_ERR_INVALID_ARG, "K=%d is not a multiple of 16 (two groups of 8)", d->K);
+  if (d->K % 64 != 0) return fail(VQ_ERR_UNSUPPORTED, "K=%d: this library needs K to be a multiple of 64", d->K);
+  if (d->N > (1 << 24) || d->K > (1 << 24))
+    return fail(VQ_ERR_UNSUPPORTED, "N=%d / K=%d exceed the supported 2^24", d->N, d->K);
+  if (d->fmt != VQ_FMT_RVQ12 && d->fmt != VQ_FMT_RVQ12_4 && d->fmt != VQ_FMT_VQ16)
+    return fail(VQ_ERR_INVALID_ARG, "fmt=%d is not a VQ_FMT_* value", d->fmt);
+  if (d->scale_group <= 0 || d->scale_group % 8 != 0 || d->K % d->scale_group != 0)
+    return fail(VQ_ERR_INVALID_ARG, "scale_group=%d must be a positive multiple of 8 dividing K", d->scale_group);
+  if (d->scale_group != 64 && d->scale_group != d->K)
+    return fail(VQ_ERR_UNSUPPORTED, "scale_group=%d: only 64 or K (per row) are implemented", d->scale_group);
+  if (d->act_dtype != VQ_F16 && d->act_dtype != VQ_BF16)
+    return fail(VQ_ERR_INVALID_ARG, "act_dtype=%d is not VQ_F16 or VQ_BF16", d->act_dtype);
+  if (d->max_M <= 0 || d->max_M > (1 << 20))
+    return fail(VQ_ERR_INVALID_ARG, "max_M=%d must be in [1, 2^20]", d->max_M);
+  return VQ_OK;
+}
+
+vq_status validate_planes(const vq_linear_desc& d, const vq_planes* p) {
+  if (p == nullptr) return fail(VQ_ERR_INVALID_ARG, "planes is NULL");
+  vq_status st;
+  if (d.fmt == VQ_FMT_VQ16) {
+    if ((st = check_ptr(p->idx16, "planes->idx16"))) return st;
+  } else {
+    if ((st = check_ptr(p->lo, "planes->lo"))) return st;
+    if ((st = check_ptr(p->hi4, "planes->hi4"))) return st;
+    if (d.fmt == VQ_FMT_RVQ12_4 && (st = check_ptr(p->s2, "planes->s2"))) return st;
+  }
+  return VQ_OK;
+}
+
+vq_status validate_codebooks(const vq_linear_desc& d, const vq_codebooks* cb, const void* scales) {
+  if (cb == nullptr) return fail(VQ_ERR_INVALID_ARG, "codebooks is NULL");
+  vq_status st;
+  if ((st = check_ptr(cb->cb1, "codebooks->cb1"))) return st;
+  if (d.fmt == VQ_FMT_RVQ12_4 && (st = check_ptr(cb->cb2, "codebooks->cb2"))) return st;
+  if ((st = check_ptr(scales, "scales"))) return st;
+  return VQ_OK;
+}
+
+vq_status check_device(const vq_linear_s* h) {
+  int cur = -1;
+  cudaError_t e = cudaGetDevice(&cur);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (cur != h->dev.device)
+    return fail(VQ_ERR_INVALID_ARG, "current device %d differs from the handle's device %d", cur, h->dev.device);
+  return VQ_OK;
+}
+
+vq::LayerArgs make_args(const vq_linear_desc& d, const vq_planes* p, const vq_codebooks* cb, const void* scales) {
+  vq::LayerArgs a{};
+  a.lo = p ? p->lo : nullptr;
+  a.hi4 = p ? p->hi4 : nullptr;
+  a.s2 = p ? p->s2 : nullptr;
+  a.idx16 = p ? p->idx16 : nullptr;
+  a.cb1 = cb ? static_cast<const uint16_t*>(cb->cb1) : nullptr;
+  a.cb2 = cb ? static_cast<const uint16_t*>(cb->cb2) : nullptr;
+  a.scales = static_cast<const uint16_t*>(scales);
+  a.N = d.N;
+  a.K = d.K;
+  a.fmt = d.fmt;
+  a.scale_group = d.scale_group;
+  a.act = d.act_dtype;
+  return a;
+}
+
+}  // namespace
+
+namespace vq {
+
+bool plan_forward(const vq_linear_desc& d, const DeviceInfo& dev, int M, int forced_path, Plan* out) {
+  int path = forced_path;
+  if (path == VQ_PATH_AUTO) path = (M == 1) ? VQ_PATH_LUT : (M <= 16 ? VQ_PATH_GEMV : VQ_PATH_TC);
+  switch (path) {
+    case VQ_PATH_LUT:
+      if (plan_lut(d, dev, M, out)) return true;
+      if (forced_path != VQ_PATH_AUTO) return false;
+      path = VQ_PATH_GEMV;
+      [[fallthrough]];
+    case VQ_PATH_GEMV:
+      if (M < 1 || M > 16) {
+        if (forced_path != VQ_PATH_AUTO) return false;
+        return plan_tc(d, dev, M, out);
+      }
+      plan_gemv(d, dev, M, out);
+      return true;
+    case VQ_PATH_TC:
+      if (plan_tc(d, dev, M, out)) return true;
+      if (forced_path != VQ_PATH_AUTO || M > 16) return false;
+      plan_gemv(d, dev, M, out);
+      return true;
+    default:
+      return false;
+  }
+}
+
+}  // namespace vq
+
+VQ_API int32_t vq_abi_version(void) { return 1; }
+
+VQ_API const char* vq_last_error(void) { return t_err.c_str(); }
+
+VQ_API vq_status vq_linear_create(const vq_linear_desc* desc, vq_linear_t* out) {
+  if (out == nullptr) return fail(VQ_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  vq_status st = validate_desc(desc);
+  if (st) return st;
+  vq::DeviceInfo dev{};
+  cudaError_t e = cudaGetDevice(&dev.device);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  int major = 0, minor = 0;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev.device);
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev.device);
+  if (major != 10 || minor != 0)
+    return fail(VQ_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a only", dev.device,
+                major, minor);
+  cudaDeviceGetAttribute(&dev.num_sms, cudaDevAttrMultiProcessorCount, dev.device);
+  cudaDeviceGetAttribute(&dev.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev.device);
+
+  // Scratch: the largest any path may need for any M <= max_M.
+  size_t need = 0;
+  int tickets = 0;
+  for (int M = 1; M <= desc->max_M; ++M) {
+    const int paths[3] = {VQ_PATH_LUT, VQ_PATH_GEMV, VQ_PATH_TC};
+    for (int pth : paths) {
+      vq::Plan p{};
+      if (!vq::plan_forward(*desc, dev, M, pth, &p)) continue;
+      if (p.scratch_bytes > need) need = p.scratch_bytes;
+      if (p.tickets > tickets) tickets = p.tickets;
+    }
+  }
+  vq_linear_s* h = new (std::nothrow) vq_linear_s{};
+  if (!h) return fail(VQ_ERR_NOMEM, "host allocation of the handle failed");
+  h->d = *desc;
+  h->dev = dev;
+  h->path = VQ_PATH_AUTO;
+  h->scratch_bytes = need;
+  if (need) {
+    e = cudaMalloc(&h->scratch, need);
+    if (e != cudaSuccess) {
+      delete h;
+      cudaGetLastError();
+      return fail(VQ_ERR_NOMEM, "cudaMalloc of %zu scratch bytes failed: %s", need, cudaGetErrorString(e));
+    }
+  }
+  h->num_tickets = tickets;
+  const size_t small = sizeof(uint32_t) * (size_t)(1 + tickets);
+  uint32_t* words = nullptr;
+  e = cudaMalloc(&words, small);
+  if (e == cudaSuccess) e = cudaMemset(words, 0, small);
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();  // the zeroing is complete before any forward
+  h->err = words;
+  h->tickets = tickets ? words + 1 : nullptr;
+  if (e != cudaSuccess) {
+    cudaFree(h->scratch);
+    cudaFree(words);
+    delete h;
+    cudaGetLastError();
+    return fail(VQ_ERR_NOMEM, "cudaMalloc of the error word failed: %s", cudaGetErrorString(e));
+  }
+  *out = h;
+  return VQ_OK;
+}
+
+VQ_API vq_status vq_linear_destroy(vq_linear_t h) {
+  if (h == nullptr) return VQ_OK;
+  cudaError_t e1 = cudaSuccess, e2 = cudaSuccess;
+  if (h->scratch) e1 = cudaFree(h->scratch);
+  if (h->err) e2 = cudaFree(h->err);  // also frees the tickets (one allocation)
+  delete h;
+  if (e1 != cudaSuccess) return cuda_fail(e1, "cudaFree(scratch)");
+  if (e2 != cudaSuccess) return cuda_fail(e2, "cudaFree(err)");
+  return VQ_OK;
+}
+
+VQ_API vq_status vq_linear_set_path(vq_linear_t h, int32_t path) {
+  if (h == nullptr) return fail(VQ_ERR_INVALID_ARG, "handle is NULL");
+  if (path < VQ_PATH_AUTO || path > VQ_PATH_TC) return fail(VQ_ERR_INVALID_ARG, "path=%d is not a VQ_PATH_*", path);
+  h->path = path;
+  return VQ_OK;
+}
+
+VQ_API int32_t vq_linear_launches(vq_linear_t h, int32_t M) {
+  if (h == nullptr || M < 0 || M > h->d.max_M) return -1;
+  if (M == 0) return 0;
+  vq::Plan p{};
+  if (!vq::plan_forward(h->d, h->dev, M, h->path, &p)) return -1;
+  return p.launches;
+}
+
+VQ_API vq_status vq_linear_forward(vq_linear_t h, const void* x, const vq_planes* planes,
+                                   const vq_codebooks* codebooks, const void* scales, void* y, int32_t M,
+                                   int32_t N, int32_t K, void* stream) {
+  if (h == nullptr) return fail(VQ_ERR_INVALID_ARG, "handle is NULL");
+  const vq_linear_desc& d = h->d;
+  if (N != d.N || K != d.K)
+    return fail(VQ_ERR_INVALID_ARG, "N=%d, K=%d do not match the handle's N=%d, K=%d", N, K, d.N, d.K);
+  if (M < 0 || M > d.max_M) return fail(VQ_ERR_INVALID_ARG, "M=%d outside [0, max_M=%d]", M, d.max_M);
+  vq_status st;
+  if ((st = check_ptr(x, "x")) || (st = check_ptr(y, "y")) || (st = validate_planes(d, planes)) ||
+      (st = validate_codebooks(d, codebooks, scales)))
+    return st;
+  if (x == y) return fail(VQ_ERR_INVALID_ARG, "y must not alias x");
+  if (M == 0) return VQ_OK;
+  if ((st = check_device(h))) return st;
+  vq::Plan p{};
+  if (!vq::plan_forward(d, h->dev, M, h->path, &p))
+    return fail(VQ_ERR_UNSUPPORTED, "path %d cannot run M=%d", h->path, M);
+  if (p.scratch_bytes > h->scratch_bytes || p.tickets > h->num_tickets)
+    return fail(VQ_ERR_UNSUPPORTED, "plan needs %zu scratch bytes / %d tickets, handle has %zu / %d",
+                p.scratch_bytes, p.tickets, h->scratch_bytes, h->num_tickets);
+  vq::LayerArgs a = make_args(d, planes, codebooks, scales);
+  a.x = x;
+  a.y = y;
+  a.M = M;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  switch (p.path) {
+    case VQ_PATH_LUT: e = vq::launch_lut(a, p, h->scratch, h->tickets, s); break;
+    case VQ_PATH_TC: e = vq::launch_tc(a, p, h->scratch, h->err, s); break;
+    default: e = vq::launch_gemv(a, p, h->scratch, h->tickets, s); break;
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "vq_linear_forward launch");
+  return VQ_OK;
+}
+
+VQ_API vq_status vq_rht_apply(const void* x, void* x_out, const int8_t* signs, int32_t M, int32_t K, int32_t dtype,
+                              void* stream) {
+  if (K < 64 || K > 32768 || (K & (K - 1)) != 0)
+    return fail(VQ_ERR_INVALID_ARG, "K=%d must be a power of two in [64, 32768]", K);
+  if (M < 0) return fail(VQ_ERR_INVALID_ARG, "M=%d is negative", M);
+  if (dtype != VQ_F16 && dtype != VQ_BF16) return fail(VQ_ERR_INVALID_ARG, "dtype=%d", dtype);
+  vq_status st;
+  if ((st = check_ptr(x, "x")) || (st = check_ptr(x_out, "x_out"))) return st;
+  if (signs == nullptr) return fail(VQ_ERR_INVALID_ARG, "signs is NULL");
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(x), b0 = reinterpret_cast<uintptr_t>(x_out);
+  const uintptr_t bytes = (uintptr_t)M * K * 2;
+  if (a0 != b0 && a0 < b0 + bytes && b0 < a0 + bytes)
+    return fail(VQ_ERR_INVALID_ARG, "x_out partially overlaps x");
+  if (M == 0) return VQ_OK;
+  cudaError_t e = vq::launch_rht(x, x_out, signs, M, K, dtype, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "vq_rht_apply launch");
+  return VQ_OK;
+}
+
+VQ_API vq_status vq_linear_check(vq_linear_t h, void* stream) {
+  if (h == nullptr) return fail(VQ_ERR_INVALID_ARG, "handle is NULL");
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  uint32_t flag = 0;
+  e = cudaMemcpy(&flag, h->err, sizeof flag, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the error word");
+  if (flag) {
+    cudaMemset(h->err, 0, sizeof(uint32_t));
+    return fail(VQ_ERR_TIMEOUT, "a bounded device wait gave up (flag 0x%x)", flag);
+  }
+  return VQ_OK;
+}
+
+VQ_API vq_status vq_debug_unpack(vq_linear_t h, const vq_planes* planes, uint16_t* i1_out, uint8_t* i2_out,
+                                 void* stream) {
+  if (h == nullptr) return fail(VQ_ERR_INVALID_ARG, "handle is NULL");
+  vq_status st;
+  if ((st = validate_planes(h->d, planes)) || (st = check_ptr(i1_out, "i1_out"))) return st;
+  if ((st = check_device(h))) return st;
+  vq::LayerArgs a = make_args(h->d, planes, nullptr, nullptr);
+  cudaError_t e = vq::launch_debug_unpack(a, i1_out, i2_out, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "vq_debug_unpack launch");
+  return VQ_OK;
+}
+
+VQ_API vq_status vq_debug_dequant(vq_linear_t h, const vq_planes* planes, const vq_codebooks* codebooks,
+                                  const void* scales, void* w_out, int32_t wdt, void* stream) {
+  if (h == nullptr) return fail(VQ_ERR_INVALID_ARG, "handle is NULL");
+  if (wdt != VQ_F16 && wdt != VQ_BF16) return fail(VQ_ERR_INVALID_ARG, "wdt=%d", wdt);
+  vq_status st;
+  if ((st = validate_planes(h->d, planes)) || (st = validate_codebooks(h->d, codebooks, scales)) ||
+      (st = check_ptr(w_out, "w_out")))
+    return st;
+  if ((st = check_device(h))) return st;
+  vq::LayerArgs a = make_args(h->d, planes, codebooks, scales);
+  cudaError_t e = vq::launch_debug_dequant(a, w_out, wdt, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "vq_debug_dequant launch");
+  return VQ_OK;
+}

@@ -1,0 +1,166 @@
+// Small kernels of libvqlinear: the fixed-order split-K reduction, the input
+// rotation (sign flip + fast Walsh-Hadamard transform), and the debug exports
+// that materialise unpacked indices / decoded weights into caller buffers.
+#include "common.cuh"
+#include "internal.h"
+
+namespace vq {
+
+// ---------------------------------------------------------------- split reduce
+//
+// y[m][n] = RN( sum_{s=0..S-1} partial[s][m][n] ), summed in increasing s so the
+// result does not depend on which split finished first (GLQ README, "Inference
+// kernels": fixed-order scratch-buffer split-K instead of atomics).
+template <typename T>
+__global__ void split_reduce_kernel(const float* __restrict__ partial, uint16_t* __restrict__ y, int splits,
+                                    int64_t MN) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < MN; i += (int64_t)gridDim.x * blockDim.x) {
+    float acc = 0.f;
+    for (int s = 0; s < splits; ++s) acc += partial[s * MN + i];
+    y[i] = Elt<T>::from_f32(acc);
+  }
+}
+
+cudaError_t launch_split_reduce(const float* partial, void* y, int splits, int M, int N, int act, cudaStream_t s) {
+  const int64_t MN = (int64_t)M * N;
+  const int threads = 256;
+  int blocks = (int)((MN + threads - 1) / threads);
+  if (blocks > 4096) blocks = 4096;
+  if (act == VQ_BF16)
+    split_reduce_kernel<__nv_bfloat16><<<blocks, threads, 0, s>>>(partial, (uint16_t*)y, splits, MN);
+  else
+    split_reduce_kernel<__half><<<blocks, threads, 0, s>>>(partial, (uint16_t*)y, splits, MN);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------- rotation
+//
+// GLQ README, "How it works": Randomized Hadamard Transform = random sign flips
+// followed by a fast Walsh-Hadamard transform.  One CTA per token row: the row is
+// loaded into shared memory as fp32 with the signs applied, transformed with
+// in-place radix-2 butterflies in natural (Sylvester) order, scaled by 1/sqrt(K)
+// and rounded to the element type.  The five lowest stages (pairs inside 32
+// consecutive elements) run on registers with warp shuffles; the rest in shared
+// memory.  Each CTA reads its whole row before writing it, so x_out may be x.
+template <typename T>
+__global__ void __launch_bounds__(1024) rht_kernel(const uint16_t* __restrict__ x, uint16_t* __restrict__ xo,
+                                                   const int8_t* __restrict__ signs, int K, float scale) {
+  extern __shared__ float buf[];
+  const int64_t row = blockIdx.x;
+  const uint16_t* xr = x + row * K;
+  const int lane = threadIdx.x & 31;
+  // Stages h = 1..16 on registers: element i = 32*w + lane of each 32-chunk.
+  for (int base = (threadIdx.x & ~31); base < K; base += blockDim.x) {
+    const int i = base + lane;
+    float v = Elt<T>::to_f32(xr[i]) * (float)signs[i];
+#pragma unroll
+    for (int h = 1; h < 32; h <<= 1) {
+      const float o = __shfl_xor_sync(0xffffffffu, v, h);
+      v = (lane & h) ? (o - v) : (v + o);
+    }
+    buf[i] = v;
+  }
+  __syncthreads();
+  for (int h = 32; h < K; h <<= 1) {
+    for (int t = threadIdx.x; t < K / 2; t += blockDim.x) {
+      const int i = (t / h) * (2 * h) + (t % h);
+      const float a = buf[i], b = buf[i + h];
+      buf[i] = a + b;
+      buf[i + h] = a - b;
+    }
+    __syncthreads();
+  }
+  uint16_t* orow = xo + row * K;
+  for (int i = threadIdx.x; i < K; i += blockDim.x) orow[i] = Elt<T>::from_f32(buf[i] * scale);
+}
+
+cudaError_t launch_rht(const void* x, void* x_out, const int8_t* signs, int M, int K, int dtype, cudaStream_t s) {
+  const int threads = K < 1024 ? K : 1024;
+  const size_t smem = (size_t)K * sizeof(float);
+  const float scale = (float)(1.0 / __builtin_sqrt((double)K));
+  cudaError_t e;
+  if (dtype == VQ_BF16) {
+    e = cudaFuncSetAttribute(rht_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    rht_kernel<__nv_bfloat16><<<M, threads, smem, s>>>((const uint16_t*)x, (uint16_t*)x_out, signs, K, scale);
+  } else {
+    e = cudaFuncSetAttribute(rht_kernel<__half>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    rht_kernel<__half><<<M, threads, smem, s>>>((const uint16_t*)x, (uint16_t*)x_out, signs, K, scale);
+  }
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ debug exports
+
+__device__ __forceinline__ void unpack_one(const LayerArgs& a, int n, int g, uint32_t* i1, uint32_t* i2) {
+  const int G = a.K / 8;
+  if (a.fmt == kFmtVq16) {
+    *i1 = a.idx16[(int64_t)n * G + g];
+    *i2 = 0;
+    return;
+  }
+  const uint32_t hb = a.hi4[(int64_t)n * (G / 2) + g / 2];
+  *i1 = a.lo[(int64_t)n * G + g] | (((g & 1) ? (hb >> 4) : (hb & 15u)) << 8);
+  if (a.fmt == kFmtRvq12_4) {
+    const uint32_t sb = a.s2[(int64_t)n * (G / 2) + g / 2];
+    *i2 = (g & 1) ? (sb >> 4) : (sb & 15u);
+  } else {
+    *i2 = 0;
+  }
+}
+
+__global__ void debug_unpack_kernel(LayerArgs a, uint16_t* __restrict__ i1o, uint8_t* __restrict__ i2o) {
+  const int G = a.K / 8;
+  const int64_t total = (int64_t)a.N * G;
+  for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < total; t += (int64_t)gridDim.x * blockDim.x) {
+    uint32_t i1, i2;
+    unpack_one(a, (int)(t / G), (int)(t % G), &i1, &i2);
+    i1o[t] = (uint16_t)i1;
+    if (i2o) i2o[t] = (uint8_t)i2;
+  }
+}
+
+template <typename W>
+__global__ void debug_dequant_kernel(LayerArgs a, uint16_t* __restrict__ w) {
+  const int G = a.K / 8;
+  const int nblk = a.K / a.scale_group;
+  const int64_t total = (int64_t)a.N * G;
+  for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < total; t += (int64_t)gridDim.x * blockDim.x) {
+    const int n = (int)(t / G), g = (int)(t % G);
+    uint32_t i1, i2;
+    unpack_one(a, n, g, &i1, &i2);
+    const float s = f16_bits_to_f32(a.scales[(int64_t)n * nblk + (8 * g) / a.scale_group]);
+    const uint4 c1 = reinterpret_cast<const uint4*>(a.cb1)[i1];
+    uint32_t out[4];
+    if (a.fmt == kFmtRvq12_4) {
+      const uint4 c2 = reinterpret_cast<const uint4*>(a.cb2)[i2];
+      decode_group_packed<W, true>(c1, c2, s, out);
+    } else {
+      decode_group_packed<W, false>(c1, c1, s, out);
+    }
+    reinterpret_cast<uint4*>(w)[t] = make_uint4(out[0], out[1], out[2], out[3]);
+  }
+}
+
+static int grid_for(int64_t total, int threads) {
+  int64_t b = (total + threads - 1) / threads;
+  return (int)(b > 65535 ? 65535 : (b < 1 ? 1 : b));
+}
+
+cudaError_t launch_debug_unpack(const LayerArgs& a, uint16_t* i1, uint8_t* i2, cudaStream_t s) {
+  const int64_t total = (int64_t)a.N * (a.K / 8);
+  debug_unpack_kernel<<<grid_for(total, 256), 256, 0, s>>>(a, i1, i2);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_debug_dequant(const LayerArgs& a, void* w, int wdt, cudaStream_t s) {
+  const int64_t total = (int64_t)a.N * (a.K / 8);
+  if (wdt == VQ_BF16)
+    debug_dequant_kernel<__nv_bfloat16><<<grid_for(total, 256), 256, 0, s>>>(a, (uint16_t*)w);
+  else
+    debug_dequant_kernel<__half><<<grid_for(total, 256), 256, 0, s>>>(a, (uint16_t*)w);
+  return cudaGetLastError();
+}
+
+}  // namespace vq

@@ -1,0 +1,61 @@
+// Host-side internals of libvqlinear shared between the API front end and the
+// kernel launchers.  Not part of the ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "vqlinear.h"
+
+namespace vq {
+
+// Everything a forward kernel needs, as plain pointers and sizes.
+struct LayerArgs {
+  const void* x;        // [M][K] act dtype
+  void* y;              // [M][N] act dtype
+  const uint8_t* lo;    // [N][G]
+  const uint8_t* hi4;   // [N][G/2]
+  const uint8_t* s2;    // [N][G/2]
+  const uint16_t* idx16;
+  const uint16_t* cb1;  // fp16 bits
+  const uint16_t* cb2;
+  const uint16_t* scales;
+  int M, N, K;
+  int fmt;
+  int scale_group;
+  int act;              // VQ_F16 / VQ_BF16
+};
+
+// Work split chosen for one forward.
+struct Plan {
+  int path;          // VQ_PATH_LUT / GEMV / TC
+  int splits;        // K splits (1 = the kernel writes y directly)
+  int k_per_split;   // multiple of 64
+  int launches;      // kernels enqueued
+  size_t scratch_bytes;
+  int tickets;       // completion counters needed (zero between forwards)
+};
+
+struct DeviceInfo {
+  int device;
+  int num_sms;
+  int smem_optin;
+};
+
+// Planning (deterministic in its inputs, so the same M always takes the same path).
+bool plan_forward(const vq_linear_desc& d, const DeviceInfo& dev, int M, int forced_path, Plan* out);
+
+// Launchers: return cudaSuccess or the launch error.
+// `tickets` are per-launch completion counters: zero before every forward, and
+// every forward leaves them zero again.
+cudaError_t launch_gemv(const LayerArgs& a, const Plan& p, float* scratch, uint32_t* tickets, cudaStream_t s);
+cudaError_t launch_lut(const LayerArgs& a, const Plan& p, float* scratch, uint32_t* tickets, cudaStream_t s);
+cudaError_t launch_tc(const LayerArgs& a, const Plan& p, float* scratch, uint32_t* err_flag, cudaStream_t s);
+cudaError_t launch_split_reduce(const float* partial, void* y, int splits, int M, int N, int act, cudaStream_t s);
+cudaError_t launch_rht(const void* x, void* x_out, const int8_t* signs, int M, int K, int dtype,
+                       cudaStream_t s);
+cudaError_t launch_debug_unpack(const LayerArgs& a, uint16_t* i1, uint8_t* i2, cudaStream_t s);
+cudaError_t launch_debug_dequant(const LayerArgs& a, void* w, int wdt, cudaStream_t s);
+
+}  // namespace vq

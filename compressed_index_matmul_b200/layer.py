@@ -1,0 +1,72 @@
+"""VQLinear: one compressed layer resident on the GPU plus its library handle."""
+
+from __future__ import annotations
+
+import numpy as np
+
+from . import _binding as B
+
+
+def _dev(a: np.ndarray, device):
+    import torch
+
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.uint16:
+        a = a.view(np.int16)  # same bits; int16 is torch's portable 16-bit container
+    return torch.from_numpy(a).to(device)
+
+
+class VQLinear:
+    """Holds the planes, codebooks and scales of one layer in device memory.
+
+    ``arrays`` is a dict with numpy arrays named as in include/vqlinear.h
+    (lo, hi4, s2, idx16, cb1, cb2, scales; fp16 as uint16 bits) and the layer shape
+    (N, K, fmt, scale_group).  ``forward(x)`` calls vq_linear_forward.
+    """
+
+    def __init__(self, N, K, fmt, scale_group, act_dtype, max_M, arrays: dict, device="cuda", rht=0):
+        import torch
+
+        self.N, self.K, self.fmt, self.scale_group, self.act_dtype, self.max_M = N, K, fmt, scale_group, act_dtype, max_M
+        self.device = torch.device(device)
+        self.t = {k: _dev(v, self.device) for k, v in arrays.items() if v is not None and k in
+                  ("lo", "hi4", "s2", "idx16", "cb1", "cb2", "scales")}
+        self.planes = B.make_planes(self.t.get("lo"), self.t.get("hi4"), self.t.get("s2"), self.t.get("idx16"))
+        self.codebooks = B.make_codebooks(self.t["cb1"], self.t.get("cb2"))
+        with torch.cuda.device(self.device):
+            self.handle = B.vq_linear_create(N, K, fmt, scale_group, act_dtype, max_M, rht)
+
+    @property
+    def torch_dtype(self):
+        import torch
+
+        return torch.bfloat16 if self.act_dtype == B.VQ_BF16 else torch.float16
+
+    def forward(self, x, y=None, stream=None):
+        import torch
+
+        M = x.shape[0]
+        if y is None:
+            y = torch.empty((M, self.N), dtype=self.torch_dtype, device=self.device)
+        B.vq_linear_forward(self.handle, x, self.planes, self.codebooks, self.t["scales"], y, M, self.N, self.K,
+                            stream)
+        return y
+
+    __call__ = forward
+
+    def set_path(self, path: int):
+        B.vq_linear_set_path(self.handle, path)
+
+    def launches(self, M: int) -> int:
+        return B.vq_linear_launches(self.handle, M)
+
+    def close(self):
+        if getattr(self, "handle", None):
+            B.vq_linear_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

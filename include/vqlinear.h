@@ -1,0 +1,186 @@
+/*
+ * vqlinear.h -- C ABI of libvqlinear, a linear layer y = x . W^T computed on an
+ * NVIDIA B200 (sm_100a) directly from codebook-quantised weights.  The dense W is
+ * never written to device memory by the forward path.
+ *
+ * Where the operations are defined:
+ *   - orka README, "How it works": each group of 8 consecutive weights is replaced
+ *     by a codebook index; indices are stored as 12-bit bit-planes (a low-byte
+ *     plane plus a packed high plane); "rvq-12-4" adds a 4-bit second (residual)
+ *     stage; decode is scale x sum over stages of codebook_s[index_s]; scales come
+ *     from "block-max" normalisation.
+ *   - GLQ README, "How it works" (E8 lattice codebooks): one 16-bit index per
+ *     8-weight group into a 65,536-entry codebook; "Randomized Hadamard Transform":
+ *     random sign flips followed by a fast Walsh-Hadamard transform.
+ *   - GLQ README, "Inference kernels": Y = X . dequant(W)^T computed against the
+ *     compressed indices; partial sums reduced in a fixed order (no atomics), so
+ *     results are bit-identical from run to run.
+ *
+ * Storage format (all arrays row-major, contiguous, no padding; W is N x K,
+ * G = K / 8 groups per row; every pointer is a DEVICE pointer unless stated):
+ *   lo    uint8  [N][G]     low 8 bits of the 12-bit stage-1 index of each group
+ *   hi4   uint8  [N][G/2]   high 4 bits of the stage-1 index: group 2t in bits 0..3,
+ *                           group 2t+1 in bits 4..7
+ *   s2    uint8  [N][G/2]   4-bit stage-2 index, packed like hi4 (VQ_FMT_RVQ12_4 only)
+ *   idx16 uint16 [N][G]     16-bit index (VQ_FMT_VQ16 only), little endian
+ *   cb1   fp16   [4096][8]  stage-1 codebook (or [65536][8] for VQ_FMT_VQ16)
+ *   cb2   fp16   [16][8]    stage-2 codebook (VQ_FMT_RVQ12_4 only)
+ *   scales fp16  [N][K/scale_group]   scale_group is 64 or K (one scale per row)
+ *   x     fp16 or bf16 [M][K]          y  same dtype [M][N]
+ * Weight (n, k) with g = k/8, j = k%8 decodes to
+ *   scales[n][k/scale_group] * (cb1[i1(n,g)][j] + cb2[i2(n,g)][j]),
+ * with i1 = lo[n][g] | hi_nibble(n,g) << 8 and i2 = s2 nibble (or i1 = idx16[n][g]).
+ *
+ * Conventions shared by every entry point:
+ *   - Errors: every call returns a vq_status.  Argument problems are detected on
+ *     the host before anything is launched and return VQ_ERR_INVALID_ARG or
+ *     VQ_ERR_UNSUPPORTED; a CUDA launch/runtime failure returns VQ_ERR_CUDA.  The
+ *     message for the last non-OK status of the calling thread is available from
+ *     vq_last_error().  No C++ exception crosses this ABI.
+ *   - Streams: `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Calls only enqueue work on it and never synchronise, except the
+ *     ones documented as synchronising.
+ *   - Ownership: the caller owns every buffer passed in.  A handle owns host state
+ *     and one device scratch buffer (split-K partial sums), allocated by
+ *     vq_linear_create and freed by vq_linear_destroy.
+ *   - Concurrency: one handle must not run two calls at the same time on different
+ *     streams (they share the scratch buffer).  Different handles are independent.
+ *   - Alignment: every device pointer must be 16-byte aligned.
+ */
+#ifndef VQLINEAR_H
+#define VQLINEAR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  VQ_OK = 0,
+  VQ_ERR_INVALID_ARG = 1, /* null/misaligned pointer, shape mismatch, bad enum */
+  VQ_ERR_UNSUPPORTED = 2, /* valid request this library does not implement */
+  VQ_ERR_CUDA = 3,        /* a CUDA runtime call or kernel launch failed */
+  VQ_ERR_NOMEM = 4,       /* device or host allocation failed */
+  VQ_ERR_TIMEOUT = 5      /* a bounded device-side wait gave up (see vq_linear_check) */
+} vq_status;
+
+/* Index formats. */
+enum {
+  VQ_FMT_RVQ12 = 1,   /* one 12-bit stage: lo + hi4 planes, 4096 x 8 codebook */
+  VQ_FMT_RVQ12_4 = 2, /* 12-bit stage 1 + 4-bit stage 2: lo + hi4 + s2, cb1 + cb2 */
+  VQ_FMT_VQ16 = 3     /* one 16-bit stage: idx16 plane, 65,536 x 8 codebook */
+};
+
+/* Element types of x / y / materialised weights. */
+enum { VQ_F16 = 0, VQ_BF16 = 1 };
+
+/* Kernel choice for vq_linear_set_path (VQ_PATH_AUTO picks by M). */
+enum {
+  VQ_PATH_AUTO = 0,
+  VQ_PATH_LUT = 1,    /* M == 1 only: per-group x.codebook tables in shared memory */
+  VQ_PATH_GEMV = 2,   /* 1 <= M <= 16: decode to registers, warp MMA, split-K */
+  VQ_PATH_TC = 3      /* any M: decode to shared memory, tcgen05 MMA into TMEM */
+};
+
+typedef struct {
+  int32_t N;           /* output features (rows of W), >= 1 */
+  int32_t K;           /* input features, multiple of 64 */
+  int32_t fmt;         /* VQ_FMT_* */
+  int32_t scale_group; /* 64 (block scales along K) or K (one scale per row) */
+  int32_t act_dtype;   /* VQ_F16 or VQ_BF16: dtype of x and y */
+  int32_t max_M;       /* largest token count a forward will be given, >= 1 */
+  int32_t rht;         /* informational: 1 if the planes encode W . R^T for a
+                          rotated input (the caller applies vq_rht_apply to x) */
+} vq_linear_desc;
+
+typedef struct {
+  const uint8_t* lo;     /* [N][K/8]   (RVQ12, RVQ12_4), else NULL */
+  const uint8_t* hi4;    /* [N][K/16]  (RVQ12, RVQ12_4), else NULL */
+  const uint8_t* s2;     /* [N][K/16]  (RVQ12_4), else NULL */
+  const uint16_t* idx16; /* [N][K/8]   (VQ16), else NULL */
+} vq_planes;
+
+typedef struct {
+  const void* cb1; /* fp16 [4096][8], or [65536][8] for VQ_FMT_VQ16 */
+  const void* cb2; /* fp16 [16][8] for VQ_FMT_RVQ12_4, else NULL */
+} vq_codebooks;
+
+typedef struct vq_linear_s* vq_linear_t;
+
+/* Version of this ABI (increments on any incompatible change). */
+int32_t vq_abi_version(void);
+
+/* Create a handle for one layer shape.  Validates `desc`, queries the current
+ * device and allocates the split-K scratch buffer (sized from max_M and N) on it.
+ * Synchronous.  On error *out is set to NULL. */
+vq_status vq_linear_create(const vq_linear_desc* desc, vq_linear_t* out);
+
+/* Free the handle and its scratch.  Synchronises the device first so that no
+ * enqueued forward still uses the scratch.  NULL is accepted (no-op). */
+vq_status vq_linear_destroy(vq_linear_t h);
+
+/* Force a kernel (VQ_PATH_*) for later forwards of this handle; VQ_PATH_AUTO
+ * restores the default choice.  A forward whose M the forced path cannot take
+ * returns VQ_ERR_UNSUPPORTED. */
+vq_status vq_linear_set_path(vq_linear_t h, int32_t path);
+
+/* y = x . W^T with W decoded on the fly from planes / codebooks / scales
+ * (GLQ README, "Inference kernels"; orka README, "How it works" for the decode).
+ *   x [M][K] and y [M][N] have the handle's act_dtype; y is overwritten (no bias,
+ *   no accumulation into y) and must not overlap x or any input.
+ *   N and K must equal the handle's; 0 <= M <= max_M; M == 0 returns VQ_OK
+ *   without launching.  Accumulation is fp32; the result is rounded to nearest
+ *   even into y.  For a given handle, path and M the result is bit-identical from
+ *   run to run (fixed-order reductions, no atomics).
+ * Enqueues 1 or 2 kernels on `stream` (see vq_linear_launches) and returns. */
+vq_status vq_linear_forward(vq_linear_t h, const void* x, const vq_planes* planes,
+                            const vq_codebooks* codebooks, const void* scales, void* y,
+                            int32_t M, int32_t N, int32_t K, void* stream);
+
+/* Number of kernels vq_linear_forward enqueues for this M (0 for M == 0), or -1
+ * if M is out of range. */
+int32_t vq_linear_launches(vq_linear_t h, int32_t M);
+
+/* Randomised Hadamard rotation of the input (GLQ README, "How it works",
+ * Randomized Hadamard Transform): for every row m,
+ *   x_out[m][k] = (1/sqrt K) * sum_j (-1)^popcount(k & j) * signs[j] * x[m][j],
+ * i.e. sign flips first, then the Walsh-Hadamard transform in natural (Sylvester)
+ * order, orthonormal scaling.  Computed in fp32 and rounded to nearest even into
+ * x_out.  K must be a power of two, 16 <= K <= 32768; dtype is VQ_F16 or
+ * VQ_BF16 for both x and x_out; signs is a device int8 array of +1/-1 [K].
+ * x_out may be the same buffer as x (in place); partial overlap is invalid.
+ * One kernel launch on `stream`. */
+vq_status vq_rht_apply(const void* x, void* x_out, const int8_t* signs, int32_t M, int32_t K,
+                       int32_t dtype, void* stream);
+
+/* Synchronise `stream` and report (then clear) any error flag a bounded
+ * device-side wait of this handle's kernels raised: VQ_ERR_TIMEOUT if one gave
+ * up, else VQ_OK.  Synchronous. */
+vq_status vq_linear_check(vq_linear_t h, void* stream);
+
+/* Message for the calling thread's last non-OK status ("" if none).  The
+ * pointer stays valid until the thread's next failing call. */
+const char* vq_last_error(void);
+
+/* ---- test and debugging entry points (materialise data into caller buffers) ---- */
+
+/* Unpacked indices: i1_out uint16 [N][K/8] (stage-1 or 16-bit index), i2_out
+ * uint8 [N][K/8] (stage-2 index, 0 when the format has none; may be NULL).
+ * One kernel launch. */
+vq_status vq_debug_unpack(vq_linear_t h, const vq_planes* planes, uint16_t* i1_out, uint8_t* i2_out,
+                          void* stream);
+
+/* Materialised weights w_out [N][K] in fp16 (wdt = VQ_F16) or bf16 (VQ_BF16),
+ * each rounded exactly as  RN(fl32(fl32(s) * fl32(cb1 + cb2)))  -- the stage sum
+ * and the scaled value are rounded to fp32, then to nearest even in wdt.
+ * One kernel launch.  The forward path never calls this. */
+vq_status vq_debug_dequant(vq_linear_t h, const vq_planes* planes, const vq_codebooks* codebooks,
+                           const void* scales, void* w_out, int32_t wdt, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VQLINEAR_H */

@@ -1,0 +1,73 @@
+"""Helpers shared by the GPU parity tests (device upload, comparisons)."""
+
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import compressed_index_matmul_b200 as vq
+from compressed_index_matmul_b200 import build as libbuild
+from synth import DT_BF16, DT_F16
+
+
+def require_gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    libbuild.build()
+    vq.load()
+
+
+def dev(a):
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.uint16:
+        a = a.view(np.int16)  # same bits; torch's int16 is the portable 16-bit container
+    return torch.from_numpy(a).cuda()
+
+
+def host_bits(t) -> np.ndarray:
+    return t.view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def layer_on_gpu(layer, act, max_M):
+    s = layer["spec"]
+    return vq.VQLinear(s.N, s.K, s.fmt, s.scale_group, act, max_M, layer)
+
+
+def run_forward(L, x_bits, act, path=vq.VQ_PATH_AUTO):
+    L.set_path(path)
+    x = dev(x_bits).view(torch.bfloat16 if act == DT_BF16 else torch.float16)
+    y = L.forward(x)
+    torch.cuda.synchronize()
+    return host_bits(y)
+
+
+def widen(bits, dt):
+    bits = np.asarray(bits, dtype=np.uint16)
+    if dt == DT_F16:
+        return bits.view(np.float16).astype(np.float64)
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def assert_y_within(y_bits, dt, y_ref, tol, what=""):
+    """max|y_gpu - y_ref| <= tol per element (tol broadcast per token row)."""
+    y = widen(y_bits, dt)
+    err = np.abs(y - y_ref)
+    bad = ~(err <= tol)
+    if bad.any():
+        m, n = np.argwhere(bad)[0]
+        raise AssertionError(f"{what}: {bad.sum()} of {bad.size} outside tolerance; first at (m={m}, n={n}): "
+                             f"gpu={y[m, n]!r} ref={y_ref[m, n]!r} tol={np.broadcast_to(tol, y.shape)[m, n]!r}; "
+                             f"max err/tol={np.max(err / tol):.3g}")
+    return float(np.max(err / tol))
+
+
+def sub_layer(layer, rows):
+    """The same layer restricted to the given output rows (rows are independent)."""
+    out = {"spec": type(layer["spec"])(len(rows), layer["spec"].K, layer["spec"].fmt, layer["spec"].scale_group)}
+    for k, v in layer.items():
+        if k in ("lo", "hi4", "s2", "idx16", "scales"):
+            out[k] = np.ascontiguousarray(v[rows])
+        elif k in ("cb1", "cb2"):
+            out[k] = v
+    return out

@@ -1,0 +1,99 @@
+"""C-ABI checks that need no GPU: the library builds, loads, exports every entry
+point include/vqlinear.h declares, and rejects bad arguments on the host before
+touching CUDA."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from compressed_index_matmul_b200 import _binding as B
+from compressed_index_matmul_b200 import build as libbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "vqlinear.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    libbuild.build()
+    return B.load()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(vq_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_binding_exports():
+    assert declared_functions() == sorted(B.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert lib.vq_abi_version() == 1
+
+
+def test_no_symbols_beyond_the_abi(lib):
+    import subprocess
+
+    out = subprocess.run(["nm", "-D", "--defined-only", B.LIB_PATH], capture_output=True, text=True).stdout
+    syms = {ln.split()[-1] for ln in out.splitlines() if ln.strip()}
+    ours = {s for s in syms if s.startswith("vq_")}
+    assert ours == set(B.EXPORTS)
+
+
+def _create(**kw):
+    d = dict(N=64, K=256, fmt=B.VQ_FMT_RVQ12_4, scale_group=64, act_dtype=B.VQ_F16, max_M=4, rht=0)
+    d.update(kw)
+    return B.vq_linear_create(**d)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(N=0), B.VQ_ERR_INVALID_ARG),
+    (dict(K=-64), B.VQ_ERR_INVALID_ARG),
+    (dict(K=72), B.VQ_ERR_INVALID_ARG),         # not a multiple of 16
+    (dict(K=80), B.VQ_ERR_UNSUPPORTED),         # multiple of 16, not of 64
+    (dict(fmt=7), B.VQ_ERR_INVALID_ARG),
+    (dict(scale_group=12), B.VQ_ERR_INVALID_ARG),
+    (dict(scale_group=128), B.VQ_ERR_UNSUPPORTED),
+    (dict(act_dtype=5), B.VQ_ERR_INVALID_ARG),
+    (dict(max_M=0), B.VQ_ERR_INVALID_ARG),
+])
+def test_create_rejects_bad_descriptors(lib, kw, status):
+    with pytest.raises(B.VQError) as ei:
+        _create(**kw)
+    assert ei.value.status == status
+    assert lib.vq_last_error()
+
+
+def test_null_arguments_are_rejected(lib):
+    assert lib.vq_linear_create(None, None) == B.VQ_ERR_INVALID_ARG
+    assert lib.vq_linear_forward(None, None, None, None, None, None, 1, 1, 1, None) == B.VQ_ERR_INVALID_ARG
+    assert lib.vq_linear_set_path(None, 0) == B.VQ_ERR_INVALID_ARG
+    assert lib.vq_linear_launches(None, 1) == -1
+    assert lib.vq_linear_destroy(None) == B.VQ_OK
+    assert lib.vq_linear_check(None, None) == B.VQ_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("M,K,dt,x,xo,signs", [
+    (1, 100, 0, 16, 16, 16),      # K not a power of two
+    (1, 32, 0, 16, 16, 16),       # K below 64
+    (1, 65536, 0, 16, 16, 16),    # K above 32768
+    (-1, 64, 0, 16, 16, 16),
+    (1, 64, 3, 16, 16, 16),       # bad dtype
+    (1, 64, 0, 0, 16, 16),        # NULL x
+    (1, 64, 0, 24, 16, 16),       # misaligned x
+    (1, 64, 0, 16, 16, 0),        # NULL signs
+    (2, 64, 0, 1024, 1024 + 64, 16),  # partial overlap
+])
+def test_rht_rejects_bad_arguments_without_a_gpu(lib, M, K, dt, x, xo, signs):
+    assert lib.vq_rht_apply(x or None, xo or None, signs or None, M, K, dt, None) == B.VQ_ERR_INVALID_ARG
+
+
+def test_python_binding_raises_with_message(lib):
+    with pytest.raises(B.VQError, match="power of two"):
+        B.vq_rht_apply(16, 16, 16, 1, 100, 0, stream=0)
