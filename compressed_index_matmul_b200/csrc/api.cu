@@ -278,7 +278,7 @@ VQ_API vq_status vq_linear_forward(vq_linear_t h, const void* x, const vq_planes
   cudaError_t e;
   switch (p.path) {
     case VQ_PATH_LUT: e = vq::launch_lut(a, p, h->scratch, h->tickets, s); break;
-    case VQ_PATH_TC: e = vq::launch_tc(a, p, h->scratch, h->err, s); break;
+    case VQ_PATH_TC: e = vq::launch_tc(a, p, h->scratch, h->tickets, h->err, s); break;
     default: e = vq::launch_gemv(a, p, h->scratch, h->tickets, s); break;
   }
   if (e != cudaSuccess) return cuda_fail(e, "vq_linear_forward launch");

@@ -3,55 +3,121 @@
 // split-K partial sums go to a scratch buffer and are reduced in a fixed order).
 //
 // Work layout
-//   CTA    = 8 warps, 128 output rows x one K-split (k_per_split, multiple of 64)
-//   warp   = one 16-row tile of W; loops over its K-split in 64-wide blocks
-//   lane   = (g = lane/4, c = lane%4): rows g and g+8 of the tile, groups 2c and
-//            2c+1 of the current 64-wide block -> 4 codewords per block
-// Each lane decodes its 4 codewords into registers (stage-1 codebook staged in
-// shared memory, stage-2 codebook too; the 65,536-entry table is read through
-// L2) and feeds them straight into mma.sync m16n8k16 as the A operand (W rows x
-// k), with x as the B operand (k x 8 tokens, one or two token tiles).
+//   CTA    = 8 warps, 128 output rows x one K-split (k_per_split, multiple of 256)
+//   warp   = one 16-row tile of W; loops over its K-split in 256-wide blocks
+//   lane   = (g = lane/4, c = lane%4): rows g and g+8 of the tile and groups
+//            8c .. 8c+7 of the current 256-wide block (one 64-weight scale
+//            block) -> 16 codewords per block, fed by 8 small vector loads that
+//            are issued one block ahead
+// Each lane decodes its codewords into registers (12-bit codebooks staged in
+// shared memory by one bulk copy; the 65,536-entry table read through L2) and
+// feeds them straight into mma.sync m16n8k16 as the A operand (W rows x k), with
+// x as the B operand (k x 8 tokens, one or two token tiles).
 //
-// k permutation: an MMA's reduction order is irrelevant to the result's
-// definition, so MMA j of a block uses pair j (elements 2j, 2j+1) of every
-// codeword: fragment slot "k-pair c" holds group 2c and slot "k-pair c+4" holds
-// group 2c+1.  The matching x elements for lane (g, c) are then
-// x[g][16c + 2j .. +1] and x[g][16c + 8 + 2j .. +1], i.e. word j of two 16-byte
-// loads -- no shuffles are needed on either operand.
+// k permutation: the MMA's reduction order does not change the result's
+// definition, so for codeword q of the lane (group 8c+q) MMA 2q+h uses elements
+// 4h..4h+1 in fragment slot "k-pair c" and 4h+2..4h+3 in slot "k-pair c+4".  The
+// matching x elements are then x[g][64c + 8q + 4h .. +3], i.e. half of a 16-byte
+// shared-memory load -- no shuffles on either operand.
 //
 // Decoded weights use the materialised-weight rounding (stage sum and scaled
 // value rounded to fp32, then to the activation type), so every product the MMA
 // forms is of exactly the weights vq_debug_dequant exports.
+//
+// Split-K reduction: each split writes fp32 partials; the CTA that completes a
+// row tile last (atomic ticket) sums the splits in increasing order and writes
+// y, so a forward is one launch and the result does not depend on scheduling.
+// The kernel is launched with programmatic dependent launch: it stages the
+// codebooks and fetches its first indices before waiting for the previous
+// kernel in the stream, and reads x / writes y only after that wait.
 #include "common.cuh"
 #include "internal.h"
+#include "tc_ptx.cuh"
 
 namespace vq {
 
 constexpr int kGemvWarps = 8;
 constexpr int kGemvRows = 16 * kGemvWarps;
-constexpr int kGemvMaxKc = 1024;  // x slice staged per CTA: 16 tokens x 1024 x 2 B
+constexpr int kGemvBlk = 256;     // k per block (32 groups)
+constexpr int kGemvMaxKc = 2048;  // x slice staged per CTA: 16 tokens x 2048 x 2 B
+
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dependents_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <int FMT>
+struct BlockIdx {
+  uint32_t w[2][4];  // per row: lo (2 words) + hi4 (1) + s2 (1), or idx16 (4 words)
+  uint32_t sc;       // two fp16 scales (rows g, g+8)
+};
+
+template <int FMT>
+__device__ __forceinline__ void load_block(const LayerArgs& a, const int rows[2], const bool valid[2], int gbase,
+                                           int k, BlockIdx<FMT>& b) {
+  const int G = a.K / 8;
+  const int nblk = a.K / a.scale_group;
+  uint32_t s16[2] = {0, 0};
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    b.w[r][0] = b.w[r][1] = b.w[r][2] = b.w[r][3] = 0;
+    if (!valid[r]) continue;
+    const int64_t rowoff = (int64_t)rows[r] * G + gbase;
+    if (FMT == kFmtVq16) {
+      const uint4 v = *reinterpret_cast<const uint4*>(a.idx16 + rowoff);
+      b.w[r][0] = v.x; b.w[r][1] = v.y; b.w[r][2] = v.z; b.w[r][3] = v.w;
+    } else {
+      const uint2 lo = *reinterpret_cast<const uint2*>(a.lo + rowoff);
+      b.w[r][0] = lo.x;
+      b.w[r][1] = lo.y;
+      b.w[r][2] = *reinterpret_cast<const uint32_t*>(a.hi4 + rowoff / 2);
+      if (FMT == kFmtRvq12_4) b.w[r][3] = *reinterpret_cast<const uint32_t*>(a.s2 + rowoff / 2);
+    }
+    s16[r] = a.scales[(int64_t)rows[r] * nblk + k / a.scale_group];
+  }
+  b.sc = s16[0] | (s16[1] << 16);
+}
 
 template <int FMT, typename T, int NT>
-__global__ void __launch_bounds__(256) gemv_kernel(LayerArgs a, int k_per_split, float* __restrict__ partial) {
-  extern __shared__ __align__(16) unsigned char smem[];
+__global__ void __launch_bounds__(256) gemv_kernel(LayerArgs a, int k_per_split, int splits, float* __restrict__ partial,
+                                                   uint32_t* __restrict__ tickets) {
+  extern __shared__ __align__(128) unsigned char smem[];
   constexpr bool kSmemCb = (FMT != kFmtVq16);
   constexpr bool kTwo = (FMT == kFmtRvq12_4);
-  uint4* cb1s = reinterpret_cast<uint4*>(smem);                               // 4096 entries
-  uint4* cb2s = cb1s + (kSmemCb ? 4096 : 0);                                  // 16 entries
-  uint16_t* xs = reinterpret_cast<uint16_t*>(cb2s + (kTwo ? 16 : 0));
+  uint4* cb1s = reinterpret_cast<uint4*>(smem);                                // 4096 entries
+  uint4* cb2s = cb1s + (kSmemCb ? 4096 : 0);                                   // 16 entries
+  uint64_t* bar = reinterpret_cast<uint64_t*>(cb2s + (kTwo ? 16 : 0));         // codebook barrier
+  int* flag = reinterpret_cast<int*>(bar + 1);
+  uint16_t* xs = reinterpret_cast<uint16_t*>(bar + 2);
 
-  const int K = a.K, G = K / 8, M = a.M, N = a.N;
+  const int K = a.K, M = a.M, N = a.N;
   const int split = blockIdx.y;
   const int k0 = split * k_per_split;
   const int kc = min(k_per_split, K - k0);
   const int xstride = kc + 8;  // elements; +16 B breaks the 8-token bank alignment
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, c = lane & 3;
+  const int r0 = blockIdx.x * kGemvRows + warp * 16;
+  const int rows[2] = {r0 + g, r0 + g + 8};
+  const bool valid[2] = {rows[0] < N, rows[1] < N};
 
-  // Stage the codebooks and this split's x slice (zeros for tokens >= M).
-  if (kSmemCb) {
-    const uint4* g1 = reinterpret_cast<const uint4*>(a.cb1);
-    for (int i = threadIdx.x; i < 4096; i += blockDim.x) cb1s[i] = g1[i];
-    if (kTwo && threadIdx.x < 16) cb2s[threadIdx.x] = reinterpret_cast<const uint4*>(a.cb2)[threadIdx.x];
+  // Prologue, independent of the previous kernel: codebooks + first indices.
+  if (kSmemCb && threadIdx.x == 0) {
+    const uint32_t b = smem_u32(bar);
+    ptx::mbar_init(b, 1);
+    ptx::fence_barrier_init();
+    ptx::mbar_arrive_expect_tx(b, 65536u + (kTwo ? 256u : 0u));
+    ptx::bulk_load(smem_u32(cb1s), a.cb1, 65536u, b);
+    if (kTwo) ptx::bulk_load(smem_u32(cb2s), a.cb2, 256u, b);
   }
+  BlockIdx<FMT> cur, nxt;
+  {
+    const int kb = 0, kblock = k0 + kb + 64 * c;
+    const bool act[2] = {valid[0] && kblock < k0 + kc, valid[1] && kblock < k0 + kc};
+    load_block<FMT>(a, rows, act, kblock / 8, kblock, cur);
+  }
+
+  grid_dependency_wait();  // x and y (and scratch) may be touched from here on
   {
     const uint16_t* xg = static_cast<const uint16_t*>(a.x);
     const int vec_per_row = kc / 8;
@@ -63,14 +129,9 @@ __global__ void __launch_bounds__(256) gemv_kernel(LayerArgs a, int k_per_split,
     }
   }
   __syncthreads();
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = lane >> 2, c = lane & 3;
-  const int r0 = blockIdx.x * kGemvRows + warp * 16;
-  if (r0 >= N) return;
-  const int rows[2] = {r0 + g, r0 + g + 8};
-  const bool valid[2] = {rows[0] < N, rows[1] < N};
-  const int nblk = K / a.scale_group;
+  // Bounded wait for the codebooks.  Past the bound (never on a healthy device)
+  // the kernel still runs to completion so the split-K tickets stay consistent.
+  if (kSmemCb) ptx::mbar_wait(smem_u32(bar), 0, nullptr);
 
   float acc[NT][4];
 #pragma unroll
@@ -78,115 +139,129 @@ __global__ void __launch_bounds__(256) gemv_kernel(LayerArgs a, int k_per_split,
 #pragma unroll
     for (int i = 0; i < 4; ++i) acc[t][i] = 0.f;
 
-  for (int kb = 0; kb < kc; kb += 64) {
-    const int gA = (k0 + kb) / 8 + 2 * c;  // this lane's first group (even)
-    uint32_t w[2][2][4];                   // [row][codeword A/B][pair]
+  for (int kb = 0; kb < kc; kb += kGemvBlk) {
+    // Prefetch the next block's indices while this one is decoded.
+    if (kb + kGemvBlk < kc) {
+      const int kblock = k0 + kb + kGemvBlk + 64 * c;
+      const bool act[2] = {valid[0] && kblock < k0 + kc, valid[1] && kblock < k0 + kc};
+      load_block<FMT>(a, rows, act, kblock / 8, kblock, nxt);
+    }
+    const bool active = (kb + 64 * c) < kc;  // lanes past a ragged end contribute zeros
+    const float2 sc = f16x2_to_f32x2(cur.sc);
+    const float s[2] = {sc.x, sc.y};
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      uint32_t i1a = 0, i1b = 0, i2a = 0, i2b = 0;
-      float s = 0.f;
-      if (valid[r]) {
-        const int64_t rowoff = (int64_t)rows[r] * G;
+    for (int q = 0; q < 8; ++q) {
+      uint32_t wq[2][4];  // [row][pair]
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        uint32_t i1, i2 = 0;
         if (FMT == kFmtVq16) {
-          const uint32_t v = *reinterpret_cast<const uint32_t*>(a.idx16 + rowoff + gA);
-          i1a = v & 0xFFFFu;
-          i1b = v >> 16;
+          i1 = (cur.w[r][q >> 1] >> (16 * (q & 1))) & 0xFFFFu;
         } else {
-          const uint32_t lo2 = *reinterpret_cast<const uint16_t*>(a.lo + rowoff + gA);
-          const uint32_t hb = a.hi4[rowoff / 2 + gA / 2];
-          i1a = (lo2 & 0xFFu) | ((hb & 15u) << 8);
-          i1b = (lo2 >> 8) | ((hb >> 4) << 8);
-          if (kTwo) {
-            const uint32_t sb = a.s2[rowoff / 2 + gA / 2];
-            i2a = sb & 15u;
-            i2b = sb >> 4;
-          }
+          i1 = ((cur.w[r][q >> 2] >> (8 * (q & 3))) & 0xFFu) | (((cur.w[r][2] >> (4 * q)) & 15u) << 8);
+          if (kTwo) i2 = (cur.w[r][3] >> (4 * q)) & 15u;
         }
-        s = f16_bits_to_f32(a.scales[(int64_t)rows[r] * nblk + (k0 + kb) / a.scale_group]);
+        const uint4 c1 = kSmemCb ? cb1s[i1] : __ldg(reinterpret_cast<const uint4*>(a.cb1) + i1);
+        const uint4 c2 = kTwo ? cb2s[i2] : c1;
+        decode_group_packed<T, kTwo>(c1, c2, active ? s[r] : 0.f, wq[r]);
       }
-      uint4 c1a, c1b, c2a = make_uint4(0, 0, 0, 0), c2b = make_uint4(0, 0, 0, 0);
-      if (kSmemCb) {
-        c1a = cb1s[i1a];
-        c1b = cb1s[i1b];
-      } else {
-        c1a = __ldg(reinterpret_cast<const uint4*>(a.cb1) + i1a);
-        c1b = __ldg(reinterpret_cast<const uint4*>(a.cb1) + i1b);
-      }
-      if (kTwo) {
-        c2a = cb2s[i2a];
-        c2b = cb2s[i2b];
-      }
-      decode_group_packed<T, kTwo>(c1a, c2a, s, w[r][0]);
-      decode_group_packed<T, kTwo>(c1b, c2b, s, w[r][1]);
-    }
 #pragma unroll
-    for (int t = 0; t < NT; ++t) {
-      const uint16_t* xr = xs + (8 * t + g) * xstride + kb + 16 * c;
-      const uint4 q0 = *reinterpret_cast<const uint4*>(xr);
-      const uint4 q1 = *reinterpret_cast<const uint4*>(xr + 8);
-      const uint32_t b0[4] = {q0.x, q0.y, q0.z, q0.w};
-      const uint32_t b1[4] = {q1.x, q1.y, q1.z, q1.w};
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const uint32_t af[4] = {w[0][0][j], w[1][0][j], w[0][1][j], w[1][1][j]};
-        Mma16816<T>::run(acc[t], af, b0[j], b1[j]);
+      for (int t = 0; t < NT; ++t) {
+        uint4 xq = make_uint4(0, 0, 0, 0);
+        if (active) xq = *reinterpret_cast<const uint4*>(xs + (8 * t + g) * xstride + kb + 64 * c + 8 * q);
+        const uint32_t af0[4] = {wq[0][0], wq[1][0], wq[0][1], wq[1][1]};
+        const uint32_t af1[4] = {wq[0][2], wq[1][2], wq[0][3], wq[1][3]};
+        Mma16816<T>::run(acc[t], af0, xq.x, xq.y);
+        Mma16816<T>::run(acc[t], af1, xq.z, xq.w);
       }
     }
+    cur = nxt;
   }
+  grid_dependents_launch();
 
   // Accumulator layout: acc[t][0..1] = (row g, tokens 8t+2c, +1), acc[t][2..3] = row g+8.
+  uint16_t* y = static_cast<uint16_t*>(a.y);
+  if (splits == 1) {
 #pragma unroll
-  for (int t = 0; t < NT; ++t) {
+    for (int t = 0; t < NT; ++t)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int m = 8 * t + 2 * c + (i & 1);
+        const int r = rows[i >> 1];
+        if (m < M && r < N) y[(int64_t)m * N + r] = Elt<T>::from_f32(acc[t][i]);
+      }
+    return;
+  }
+#pragma unroll
+  for (int t = 0; t < NT; ++t)
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int m = 8 * t + 2 * c + (i & 1);
       const int r = rows[i >> 1];
-      if (m >= M || r >= N) continue;
-      if (partial == nullptr)
-        static_cast<uint16_t*>(a.y)[(int64_t)m * N + r] = Elt<T>::from_f32(acc[t][i]);
-      else
-        partial[((int64_t)split * M + m) * N + r] = acc[t][i];
+      if (m < M && r < N) partial[((int64_t)split * M + m) * N + r] = acc[t][i];
     }
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) *flag = (atomicAdd(&tickets[blockIdx.x], 1u) == (uint32_t)(splits - 1));
+  __syncthreads();
+  if (!*flag) return;
+  __threadfence();
+  const int rbeg = blockIdx.x * kGemvRows;
+  const int nrows = min(kGemvRows, N - rbeg);
+  for (int i = threadIdx.x; i < nrows * M; i += blockDim.x) {
+    const int m = i / nrows, r = rbeg + i % nrows;
+    float sum = 0.f;
+    for (int k = 0; k < splits; ++k) sum += __ldcg(partial + ((int64_t)k * M + m) * N + r);
+    y[(int64_t)m * N + r] = Elt<T>::from_f32(sum);
   }
+  if (threadIdx.x == 0) tickets[blockIdx.x] = 0u;  // ready for the next forward
 }
 
 template <int FMT, typename T, int NT>
-static cudaError_t launch_one(const LayerArgs& a, const Plan& p, float* scratch, cudaStream_t s) {
+static cudaError_t launch_one(const LayerArgs& a, const Plan& p, float* scratch, uint32_t* tickets, cudaStream_t s) {
   const int kc = p.k_per_split;
-  const size_t smem = (FMT != kFmtVq16 ? 4096 * 16 : 0) + (FMT == kFmtRvq12_4 ? 256 : 0) +
+  const size_t smem = (FMT != kFmtVq16 ? 4096 * 16 : 0) + (FMT == kFmtRvq12_4 ? 256 : 0) + 16 +
                       (size_t)8 * NT * (kc + 8) * 2;
-  cudaError_t e = cudaFuncSetAttribute(gemv_kernel<FMT, T, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  auto kern = gemv_kernel<FMT, T, NT>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((a.N + kGemvRows - 1) / kGemvRows, p.splits);
-  gemv_kernel<FMT, T, NT><<<grid, 256, smem, s>>>(a, kc, p.splits > 1 ? scratch : nullptr);
-  e = cudaGetLastError();
-  if (e != cudaSuccess || p.splits == 1) return e;
-  return launch_split_reduce(scratch, a.y, p.splits, a.M, a.N, a.act, s);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((a.N + kGemvRows - 1) / kGemvRows, p.splits);
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, a, kc, p.splits, p.splits > 1 ? scratch : nullptr,
+                            p.splits > 1 ? tickets : nullptr);
 }
 
 template <int FMT, typename T>
-static cudaError_t launch_nt(const LayerArgs& a, const Plan& p, float* scratch, cudaStream_t s) {
-  return a.M <= 8 ? launch_one<FMT, T, 1>(a, p, scratch, s) : launch_one<FMT, T, 2>(a, p, scratch, s);
+static cudaError_t launch_nt(const LayerArgs& a, const Plan& p, float* scratch, uint32_t* tickets, cudaStream_t s) {
+  return a.M <= 8 ? launch_one<FMT, T, 1>(a, p, scratch, tickets, s) : launch_one<FMT, T, 2>(a, p, scratch, tickets, s);
 }
 
 template <typename T>
-static cudaError_t launch_fmt(const LayerArgs& a, const Plan& p, float* scratch, cudaStream_t s) {
+static cudaError_t launch_fmt(const LayerArgs& a, const Plan& p, float* scratch, uint32_t* tickets, cudaStream_t s) {
   switch (a.fmt) {
-    case kFmtRvq12: return launch_nt<kFmtRvq12, T>(a, p, scratch, s);
-    case kFmtRvq12_4: return launch_nt<kFmtRvq12_4, T>(a, p, scratch, s);
-    default: return launch_nt<kFmtVq16, T>(a, p, scratch, s);
+    case kFmtRvq12: return launch_nt<kFmtRvq12, T>(a, p, scratch, tickets, s);
+    case kFmtRvq12_4: return launch_nt<kFmtRvq12_4, T>(a, p, scratch, tickets, s);
+    default: return launch_nt<kFmtVq16, T>(a, p, scratch, tickets, s);
   }
 }
 
-cudaError_t launch_gemv(const LayerArgs& a, const Plan& p, float* scratch, uint32_t* /*tickets*/, cudaStream_t s) {
-  return a.act == VQ_BF16 ? launch_fmt<__nv_bfloat16>(a, p, scratch, s) : launch_fmt<__half>(a, p, scratch, s);
+cudaError_t launch_gemv(const LayerArgs& a, const Plan& p, float* scratch, uint32_t* tickets, cudaStream_t s) {
+  return a.act == VQ_BF16 ? launch_fmt<__nv_bfloat16>(a, p, scratch, tickets, s)
+                          : launch_fmt<__half>(a, p, scratch, tickets, s);
 }
 
 // Split choice: enough CTAs to cover the SMs about twice, each K-split a multiple
-// of 64 and at most kGemvMaxKc wide (bounds the staged x slice).
+// of 256 (the last may be ragged) and at most kGemvMaxKc wide.
 void plan_gemv(const vq_linear_desc& d, const DeviceInfo& dev, int M, Plan* p) {
-  const int nb = d.K / 64;
+  const int nb = (d.K + kGemvBlk - 1) / kGemvBlk;
   const int row_tiles = (d.N + kGemvRows - 1) / kGemvRows;
   const int s_min = (d.K + kGemvMaxKc - 1) / kGemvMaxKc;
   const int target = 2 * dev.num_sms;
@@ -197,10 +272,10 @@ void plan_gemv(const vq_linear_desc& d, const DeviceInfo& dev, int M, Plan* p) {
   S = (nb + bps - 1) / bps;
   p->path = VQ_PATH_GEMV;
   p->splits = S;
-  p->k_per_split = bps * 64;
-  p->launches = S > 1 ? 2 : 1;
+  p->k_per_split = bps * kGemvBlk;
+  p->launches = 1;
   p->scratch_bytes = S > 1 ? (size_t)S * M * d.N * sizeof(float) : 0;
-  p->tickets = 0;
+  p->tickets = S > 1 ? row_tiles : 0;
 }
 
 }  // namespace vq

@@ -51,7 +51,8 @@ bool plan_forward(const vq_linear_desc& d, const DeviceInfo& dev, int M, int for
 // every forward leaves them zero again.
 cudaError_t launch_gemv(const LayerArgs& a, const Plan& p, float* scratch, uint32_t* tickets, cudaStream_t s);
 cudaError_t launch_lut(const LayerArgs& a, const Plan& p, float* scratch, uint32_t* tickets, cudaStream_t s);
-cudaError_t launch_tc(const LayerArgs& a, const Plan& p, float* scratch, uint32_t* err_flag, cudaStream_t s);
+cudaError_t launch_tc(const LayerArgs& a, const Plan& p, float* scratch, uint32_t* tickets, uint32_t* err_flag,
+                      cudaStream_t s);
 cudaError_t launch_split_reduce(const float* partial, void* y, int splits, int M, int N, int act, cudaStream_t s);
 cudaError_t launch_rht(const void* x, void* x_out, const int8_t* signs, int M, int K, int dtype,
                        cudaStream_t s);

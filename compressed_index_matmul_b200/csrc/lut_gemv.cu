@@ -1,4 +1,4 @@
-// Batch-1 GEMV by per-group lookup tables (M == 1, 12-bit formats).
+// Batch-1 GEMV by per-group lookup tables (M == 1, 12-bit formats, K % 128 == 0).
 //
 // For one token x and one group g of 8 inputs, every weight group of row n
 // contributes s * (x_g . cb1[i1] + x_g . cb2[i2]) (orka README, "How it works":
@@ -8,30 +8,42 @@
 //   T2[g][e] = x_g . cb2[e]   (16 x 16 entries, fp32, shared memory)
 // and then sweeps many rows with one table lookup per group and stage instead of
 // gathering and decoding 8-wide codewords.  T1 is a small matrix product
-// (16 groups x 8 dims times 8 dims x 4096 codewords) and is built on the tensor
-// cores with mma.sync m16n8k8 (fp16 in, fp32 accumulate).
+// (16 groups x 8 dims times 8 dims x 4096 codewords) built on the tensor cores
+// with mma.sync m16n8k8 (fp16 in, fp32 accumulate).  The codebook operand of
+// those MMAs does not depend on x, so each warp loads its share of it into
+// registers once and every rebuild is only MMAs and stores.
 //
 // Work distribution: units are (K-slice s, 256-row chunk c) in slice-major order;
-// a persistent grid of one CTA per SM takes a contiguous run of units, rebuilding
-// the tables only when its slice changes.  Each unit writes fp32 partial sums
-// partial[s][rows]; the CTA that completes a chunk last (an atomic ticket per
-// chunk) sums the chunk's partials in increasing s and writes y, so the result
-// is independent of scheduling (GLQ README, "Inference kernels": fixed-order
-// split-K reduction, no floating-point atomics).  One launch per forward.
+// a persistent grid of one CTA per SM takes a contiguous run of units.  Thread t
+// handles row t of every unit; its rows' index bytes stream through a private
+// ring of cp.async stages in shared memory, several units ahead, so the loop
+// never waits on DRAM latency.  Each unit writes an fp32 partial sum per row.
+// When a CTA has finished all its units it takes one ticket per unit; the CTA
+// that completes a chunk's last slice sums that chunk's partials in increasing
+// slice order (GLQ README, "Inference kernels": fixed-order split-K reduction, no
+// floating-point atomics) and writes y.  One launch per forward.
 //
-// bf16 activations are scaled by a power of two per slice before they enter the
-// fp16 MMA (so any bf16 magnitude fits), and the partial sum is scaled back; the
-// scaling is exact.
+// Activations are scaled by a power of two per slice so that every value fits the
+// fp16 MMA whatever the activation type; the partial sum is scaled back exactly.
 #include "common.cuh"
 #include "internal.h"
 
 namespace vq {
 
-constexpr int kLutGroups = 16;                    // groups per K-slice (128 inputs)
-constexpr int kLutThreads = 256;                  // one row per thread per unit
-constexpr int kLutTableBytes = 4096 * 2 + 64;     // one group's T1 (bf16) + pad (bank spread)
-constexpr int kLutSmem = kLutGroups * kLutTableBytes + kLutGroups * 16 * 4 + kLutGroups * 8 * 2 +
-                         kLutGroups * 8 * 4 + 64;
+constexpr int kLutGroups = 16;                 // groups per K-slice (128 inputs)
+constexpr int kLutThreads = 256;               // one row per thread per unit
+constexpr int kLutTableBytes = 4096 * 2 + 64;  // one group's T1 (bf16) + pad (bank spread)
+constexpr int kLutStages = 6;                  // cp.async ring depth (units in flight)
+constexpr int kLutRecord = 48;                 // bytes per thread per stage: lo16 hi8 s2 8 scales4 pad
+constexpr int kLutMaxX = 4;                    // x slices preloaded per CTA
+constexpr int kLutOffT2 = kLutGroups * kLutTableBytes;
+constexpr int kLutOffXh = kLutOffT2 + kLutGroups * 16 * 4;
+constexpr int kLutOffXf = kLutOffXh + kLutGroups * 8 * 2;
+constexpr int kLutOffRed = kLutOffXf + kLutGroups * 8 * 4;
+constexpr int kLutOffList = kLutOffRed + 64;
+constexpr int kLutMaxList = 256;
+constexpr int kLutOffRing = kLutOffList + 4 * kLutMaxList + 16;
+constexpr int kLutSmem = kLutOffRing + kLutStages * kLutThreads * kLutRecord;
 
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   uint32_t r;
@@ -57,99 +69,162 @@ __device__ __forceinline__ float lds_f32(uint32_t addr) {
   return v;
 }
 
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async8(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 template <int FMT, typename T>
 __global__ void __launch_bounds__(kLutThreads, 1)
     lut_gemv_kernel(LayerArgs a, float* __restrict__ partial, uint32_t* __restrict__ tickets, int S, int C) {
   extern __shared__ __align__(128) unsigned char smem[];
   constexpr bool kTwo = (FMT == kFmtRvq12_4);
-  unsigned char* t1 = smem;                                                   // [16][kLutTableBytes]
-  float* t2 = reinterpret_cast<float*>(smem + kLutGroups * kLutTableBytes);   // [16][16]
-  uint32_t* xh = reinterpret_cast<uint32_t*>(t2 + kLutGroups * 16);           // [16][4] half2 (MMA A)
-  float* xf = reinterpret_cast<float*>(xh + kLutGroups * 4);                  // [16][8]
-  float* red = xf + kLutGroups * 8;                                           // misc scalars
-  int* flag = reinterpret_cast<int*>(red + 8);
+  unsigned char* t1 = smem;
+  float* t2 = reinterpret_cast<float*>(smem + kLutOffT2);
+  uint32_t* xh = reinterpret_cast<uint32_t*>(smem + kLutOffXh);
+  float* xf = reinterpret_cast<float*>(smem + kLutOffXf);
+  float* red = reinterpret_cast<float*>(smem + kLutOffRed);
+  int* list = reinterpret_cast<int*>(smem + kLutOffList);
+  int* nlist = reinterpret_cast<int*>(smem + kLutOffRed + 48);
+  const uint32_t t1_base = smem_u32(t1), t2_base = smem_u32(t2), ring = smem_u32(smem + kLutOffRing);
 
   const int K = a.K, G = K / 8, N = a.N;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nblk = K / a.scale_group;
+  const bool block_scales = (a.scale_group == 64);
   const int64_t U = (int64_t)S * C;
   const int64_t u0 = U * blockIdx.x / gridDim.x, u1 = U * (blockIdx.x + 1) / gridDim.x;
   const uint16_t* xg = static_cast<const uint16_t*>(a.x);
-  const uint32_t t1_base = smem_u32(t1), t2_base = smem_u32(t2);
-  const int nblk = K / a.scale_group;
+
+  // Row records for unit u go to stage (u - u0) % kLutStages of this thread's ring.
+  auto issue = [&](int64_t u) {
+    const int s = (int)(u / C), r = (int)(u % C) * kLutThreads + tid;
+    if (r < N) {
+      const uint32_t dst = ring + (((int)((u - u0) % kLutStages)) * kLutThreads + tid) * kLutRecord;
+      const int64_t rowoff = (int64_t)r * G + s * kLutGroups;
+      cp_async16(dst, a.lo + rowoff);
+      cp_async8(dst + 16, a.hi4 + rowoff / 2);
+      if (kTwo) cp_async8(dst + 24, a.s2 + rowoff / 2);
+      if (block_scales) cp_async4(dst + 32, a.scales + (int64_t)r * nblk + 2 * s);
+    }
+  };
+  for (int i = 0; i < kLutStages - 1; ++i) {
+    if (u0 + i < u1) issue(u0 + i);
+    cp_async_commit();
+  }
+
+  // Codebook operand of the table MMAs, held for the whole kernel: warp w covers
+  // codewords 512w .. 512w+511 in 16 blocks of 32; see the build below.
+  const int g = lane >> 2, c = lane & 3;
+  uint32_t bfrag[16][4];
+  {
+    const uint32_t* cbw = reinterpret_cast<const uint32_t*>(a.cb1);
+#pragma unroll
+    for (int it = 0; it < 16; ++it)
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        bfrag[it][j] = __ldg(cbw + (size_t)(warp * 512 + it * 32 + 8 * (g >> 1) + 2 * j + (g & 1)) * 4 + c);
+  }
+  float c2v[8];
+  if (kTwo) {
+    const uint4 q = reinterpret_cast<const uint4*>(a.cb2)[tid & 15];
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      const float2 v = f16x2_to_f32x2(w[p]);
+      c2v[2 * p] = v.x;
+      c2v[2 * p + 1] = v.y;
+    }
+  }
+  // Everything above reads only the layer's constant inputs; x, y and the scratch
+  // are touched only after the previous kernel in the stream has completed.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  // x of the first kLutMaxX slices this CTA touches.
+  const int s_first = (int)(u0 / C);
+  float xpre[kLutMaxX];
+#pragma unroll
+  for (int i = 0; i < kLutMaxX; ++i) {
+    const int s = s_first + i;
+    xpre[i] = (tid < 128 && s < S) ? Elt<T>::to_f32(xg[(int64_t)s * 128 + tid]) : 0.f;
+  }
 
   int cur = -1;
   float inv_xscale = 1.f;
   for (int64_t u = u0; u < u1; ++u) {
     const int s = (int)(u / C), ch = (int)(u % C);
-    const int gs = s * kLutGroups;
-    const int gc = min(kLutGroups, G - gs);  // 16, or 8 for a ragged last slice
+    if (u + kLutStages - 1 < u1) issue(u + kLutStages - 1);
+    cp_async_commit();
     if (s != cur) {
       // ------------------------------------------------------------ build
-      __syncthreads();  // everyone is done reading the previous tables
+      __syncthreads();  // everyone is done with the previous tables
       float xv = 0.f;
-      if (tid < 8 * gc) xv = Elt<T>::to_f32(xg[8 * gs + tid]);
-      // Power-of-two scale so the slice's largest |x| lands in [2^14, 2^15): every
-      // value then fits fp16 for the MMA, whatever the activation type.
-      float xs;
-      {
-        float m = fabsf(xv);
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        if (lane == 0) red[warp] = m;
-        __syncthreads();
-        m = red[0];
+      if (tid < 128) {
+        const int i = s - s_first;
+        if (i < kLutMaxX) {
 #pragma unroll
-        for (int w = 1; w < kLutThreads / 32; ++w) m = fmaxf(m, red[w]);
-        int e = 0;
-        if (m > 0.f && isfinite(m)) {
-          frexpf(m, &e);  // m in [2^(e-1), 2^e)
-          e = min(100, max(-100, 15 - e));
+          for (int k = 0; k < kLutMaxX; ++k)
+            if (k == i) xv = xpre[k];
+        } else {
+          xv = Elt<T>::to_f32(xg[(int64_t)s * 128 + tid]);
         }
-        xs = ldexpf(1.f, e);
-        inv_xscale = ldexpf(1.f, -e);
       }
-      const float xsv = xv * xs;
-      if (tid < kLutGroups * 8) {
-        xf[tid] = xsv;  // zeros past gc groups
-        reinterpret_cast<__half*>(xh)[tid] = __float2half_rn(xsv);
+      float m = fabsf(xv);
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      if (lane == 0) red[warp] = m;
+      __syncthreads();
+      m = red[0];
+#pragma unroll
+      for (int w = 1; w < kLutThreads / 32; ++w) m = fmaxf(m, red[w]);
+      int e = 0;
+      if (m > 0.f && isfinite(m)) {
+        frexpf(m, &e);  // m in [2^(e-1), 2^e): scale the slice's max into [2^14, 2^15)
+        e = min(100, max(-100, 15 - e));
+      }
+      const float xs = ldexpf(1.f, e);
+      inv_xscale = ldexpf(1.f, -e);
+      if (tid < 128) {
+        xf[tid] = xv * xs;
+        reinterpret_cast<__half*>(xh)[tid] = __float2half_rn(xv * xs);
       }
       __syncthreads();
       if (kTwo) {
-        const int g = tid >> 4, e = tid & 15;
-        const uint4 c2 = reinterpret_cast<const uint4*>(a.cb2)[e];
-        const uint32_t w[4] = {c2.x, c2.y, c2.z, c2.w};
+        const int gg = tid >> 4;
         float acc = 0.f;
 #pragma unroll
-        for (int p = 0; p < 4; ++p) {
-          const float2 v = f16x2_to_f32x2(w[p]);
-          acc = fmaf(xf[8 * g + 2 * p], v.x, acc);
-          acc = fmaf(xf[8 * g + 2 * p + 1], v.y, acc);
-        }
-        t2[g * 16 + e] = acc;
+        for (int d = 0; d < 8; ++d) acc = fmaf(xf[8 * gg + d], c2v[d], acc);
+        t2[tid] = acc;  // T2[gg][tid & 15]
       }
       {
-        // T1 on the tensor cores.  A = x slice (16 groups x 8 dims), B = 8 codewords
-        // x 8 dims.  Four MMAs cover 32 codewords with column n of MMA j mapped to
-        // codeword base + 8*(n/2) + 2j + (n%2), so lane (g, c) ends up holding
+        // A = x slice (16 groups x 8 dims, fp16).  Column n of MMA j in block `it`
+        // is codeword base + 8*(n/2) + 2j + (n%2), so lane (g, c) ends with
         // codewords base+8c .. base+8c+7 of groups g and g+8: one 16-byte store each.
-        const int g = lane >> 2, c = lane & 3;
         const uint32_t a0 = xh[g * 4 + c], a1 = xh[(g + 8) * 4 + c];
-        const uint32_t* cbw = reinterpret_cast<const uint32_t*>(a.cb1);
-        for (int base = warp * 512; base < warp * 512 + 512; base += 32) {
-          float d[4][4];
-          uint32_t b[4];
 #pragma unroll
-          for (int j = 0; j < 4; ++j) b[j] = __ldg(cbw + (size_t)(base + 8 * (g >> 1) + 2 * j + (g & 1)) * 4 + c);
+        for (int it = 0; it < 16; ++it) {
+          const int base = warp * 512 + it * 32;
+          float d[4][4];
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             d[j][0] = d[j][1] = d[j][2] = d[j][3] = 0.f;
-            mma_16808_f16(d[j], a0, a1, b[j]);
+            mma_16808_f16(d[j], a0, a1, bfrag[it][j]);
           }
-          const uint4 lo = make_uint4(Elt<__nv_bfloat16>::pack(d[0][0], d[0][1]), Elt<__nv_bfloat16>::pack(d[1][0], d[1][1]),
-                                      Elt<__nv_bfloat16>::pack(d[2][0], d[2][1]), Elt<__nv_bfloat16>::pack(d[3][0], d[3][1]));
-          const uint4 hi = make_uint4(Elt<__nv_bfloat16>::pack(d[0][2], d[0][3]), Elt<__nv_bfloat16>::pack(d[1][2], d[1][3]),
-                                      Elt<__nv_bfloat16>::pack(d[2][2], d[2][3]), Elt<__nv_bfloat16>::pack(d[3][2], d[3][3]));
+          typedef Elt<__nv_bfloat16> B16;
+          const uint4 lo = make_uint4(B16::pack(d[0][0], d[0][1]), B16::pack(d[1][0], d[1][1]),
+                                      B16::pack(d[2][0], d[2][1]), B16::pack(d[3][0], d[3][1]));
+          const uint4 hi = make_uint4(B16::pack(d[0][2], d[0][3]), B16::pack(d[1][2], d[1][3]),
+                                      B16::pack(d[2][2], d[2][3]), B16::pack(d[3][2], d[3][3]));
           *reinterpret_cast<uint4*>(t1 + g * kLutTableBytes + (base + 8 * c) * 2) = lo;
-          if (g + 8 < gc) *reinterpret_cast<uint4*>(t1 + (g + 8) * kLutTableBytes + (base + 8 * c) * 2) = hi;
+          *reinterpret_cast<uint4*>(t1 + (g + 8) * kLutTableBytes + (base + 8 * c) * 2) = hi;
         }
       }
       __syncthreads();
@@ -157,39 +232,25 @@ __global__ void __launch_bounds__(kLutThreads, 1)
     }
 
     // -------------------------------------------------------------- lookups
+    cp_async_wait<kLutStages - 1>();  // this thread's records for unit u have landed
     const int r = ch * kLutThreads + tid;
-    float acc = 0.f;
     if (r < N) {
-      const int64_t rowoff = (int64_t)r * G + gs;
-      uint32_t low[4], hiw[2], s2w[2] = {0, 0};
-      if (gc == kLutGroups && (G % 16) == 0) {
-        const uint4 l = *reinterpret_cast<const uint4*>(a.lo + rowoff);
-        low[0] = l.x; low[1] = l.y; low[2] = l.z; low[3] = l.w;
-        const uint2 h = *reinterpret_cast<const uint2*>(a.hi4 + rowoff / 2);
-        hiw[0] = h.x; hiw[1] = h.y;
-        if (kTwo) {
-          const uint2 q = *reinterpret_cast<const uint2*>(a.s2 + rowoff / 2);
-          s2w[0] = q.x; s2w[1] = q.y;
-        }
-      } else {
-        // 8-byte aligned rows (G % 8 == 0): two halves, the second only for full slices
-        const uint2 l0 = *reinterpret_cast<const uint2*>(a.lo + rowoff);
-        low[0] = l0.x; low[1] = l0.y;
-        hiw[0] = *reinterpret_cast<const uint32_t*>(a.hi4 + rowoff / 2);
-        if (kTwo) s2w[0] = *reinterpret_cast<const uint32_t*>(a.s2 + rowoff / 2);
-        if (gc == kLutGroups) {
-          const uint2 l1 = *reinterpret_cast<const uint2*>(a.lo + rowoff + 8);
-          low[2] = l1.x; low[3] = l1.y;
-          hiw[1] = *reinterpret_cast<const uint32_t*>(a.hi4 + rowoff / 2 + 4);
-          if (kTwo) s2w[1] = *reinterpret_cast<const uint32_t*>(a.s2 + rowoff / 2 + 4);
-        } else {
-          low[2] = low[3] = 0; hiw[1] = 0; s2w[1] = 0;
-        }
-      }
+      const uint32_t rec = ring + (((int)((u - u0) % kLutStages)) * kLutThreads + tid) * kLutRecord;
+      uint4 lo4, hs;
+      uint32_t scw = 0;
+      asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                   : "=r"(lo4.x), "=r"(lo4.y), "=r"(lo4.z), "=r"(lo4.w)
+                   : "r"(rec));
+      asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                   : "=r"(hs.x), "=r"(hs.y), "=r"(hs.z), "=r"(hs.w)
+                   : "r"(rec + 16));
+      if (block_scales) asm volatile("ld.shared.u32 %0, [%1];" : "=r"(scw) : "r"(rec + 32));
+      const uint32_t low[4] = {lo4.x, lo4.y, lo4.z, lo4.w};
+      const uint32_t hiw[2] = {hs.x, hs.y};
+      const uint32_t s2w[2] = {hs.z, hs.w};
       float blk[2] = {0.f, 0.f};
 #pragma unroll
       for (int w = 0; w < 2; ++w) {
-        if (w == 1 && gc < kLutGroups) break;
         const uint32_t hE = hiw[w] & 0x0F0F0F0Fu, hO = (hiw[w] >> 4) & 0x0F0F0F0Fu;
         const uint32_t sE = (s2w[w] & 0x0F0F0F0Fu) << 2, sO = ((s2w[w] >> 4) & 0x0F0F0F0Fu) << 2;
 #pragma unroll
@@ -201,43 +262,67 @@ __global__ void __launch_bounds__(kLutThreads, 1)
           const uint32_t i1 = prmt(low[t >> 2], (q & 1) ? hO : hE, sel);
           float v = lds_bf16(t1_base + t * kLutTableBytes + i1 * 2);
           if (kTwo) {
-            const uint32_t bsel = (q >> 1) | (8u | (q >> 1)) << 4 | (8u | (q >> 1)) << 8 | (8u | (q >> 1)) << 12;
-            const uint32_t e4 = prmt((q & 1) ? sO : sE, 0, bsel);
-            v += lds_f32(t2_base + t * 64 + e4);
+            const uint32_t b = q >> 1;
+            const uint32_t bsel = b | ((8u | b) << 4) | ((8u | b) << 8) | ((8u | b) << 12);
+            v += lds_f32(t2_base + t * 64 + prmt((q & 1) ? sO : sE, 0, bsel));
           }
           blk[w] += v;
         }
       }
-      if (a.scale_group == 64) {
-        const int b0 = 2 * s;
-        acc = blk[0] * f16_bits_to_f32(a.scales[(int64_t)r * nblk + b0]);
-        if (gc == kLutGroups) acc = fmaf(blk[1], f16_bits_to_f32(a.scales[(int64_t)r * nblk + b0 + 1]), acc);
+      float acc;
+      if (block_scales) {
+        const float2 sc = f16x2_to_f32x2(scw);
+        acc = fmaf(blk[1], sc.y, blk[0] * sc.x);
       } else {
-        acc = (blk[0] + blk[1]) * f16_bits_to_f32(a.scales[r]);
+        acc = blk[0] + blk[1];  // the per-row scale is applied once, at the reduction
       }
       acc *= inv_xscale;
-    }
-
-    // --------------------------------------------------- fixed-order reduce
-    if (S == 1) {
-      if (r < N) static_cast<uint16_t*>(a.y)[r] = Elt<T>::from_f32(acc);
-      continue;
-    }
-    if (r < N) partial[(int64_t)s * N + r] = acc;
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) *flag = (atomicAdd(&tickets[ch], 1u) == (uint32_t)(S - 1));
-    __syncthreads();
-    if (*flag) {
-      __threadfence();
-      if (r < N) {
-        float sum = 0.f;
-        for (int k = 0; k < S; ++k) sum += __ldcg(partial + (int64_t)k * N + r);
-        static_cast<uint16_t*>(a.y)[r] = Elt<T>::from_f32(sum);
+      if (S == 1) {
+        if (!block_scales) acc *= f16_bits_to_f32(a.scales[r]);
+        static_cast<uint16_t*>(a.y)[r] = Elt<T>::from_f32(acc);
+      } else {
+        partial[(int64_t)s * N + r] = acc;
       }
-      if (tid == 0) tickets[ch] = 0u;  // ready for the next forward
     }
   }
+  cp_async_wait<0>();
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  if (S == 1) return;
+
+  // ------------------------------------------------------ fixed-order reduce
+  // One ticket per unit, all taken at once (thread i takes unit u0 + i).
+  __threadfence();
+  if (tid == 0) *nlist = 0;
+  __syncthreads();
+  if (tid < u1 - u0) {
+    const int ch = (int)((u0 + tid) % C);
+    if (atomicAdd(&tickets[ch], 1u) == (uint32_t)(S - 1)) list[atomicAdd(nlist, 1)] = ch;
+  }
+  __syncthreads();
+  const int n = *nlist;
+  if (n == 0) return;
+  __threadfence();
+  // Rows of the completed chunks; every split's partial of a row is loaded before
+  // the sum, which then runs in increasing split order.
+  constexpr int kBatch = 16;
+  for (int i = tid; i < n * kLutThreads; i += kLutThreads) {
+    const int ch = list[i / kLutThreads];
+    const int r = ch * kLutThreads + i % kLutThreads;
+    if (r >= N) continue;
+    float sum = 0.f;
+    for (int k0 = 0; k0 < S; k0 += kBatch) {
+      float v[kBatch];
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j) v[j] = (k0 + j < S) ? __ldcg(partial + (int64_t)(k0 + j) * N + r) : 0.f;
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j)
+        if (k0 + j < S) sum += v[j];
+    }
+    if (!block_scales) sum *= f16_bits_to_f32(a.scales[r]);
+    static_cast<uint16_t*>(a.y)[r] = Elt<T>::from_f32(sum);
+  }
+  __syncthreads();
+  if (tid < n) tickets[list[tid]] = 0u;  // ready for the next forward
 }
 
 struct LutGeom {
@@ -246,8 +331,7 @@ struct LutGeom {
 
 static LutGeom lut_geom(int N, int K, int num_sms) {
   LutGeom g;
-  const int G = K / 8;
-  g.S = (G + kLutGroups - 1) / kLutGroups;
+  g.S = K / (8 * kLutGroups);
   g.C = (N + kLutThreads - 1) / kLutThreads;
   const int64_t U = (int64_t)g.S * g.C;
   g.grid = (int)(U < num_sms ? U : num_sms);
@@ -255,8 +339,10 @@ static LutGeom lut_geom(int N, int K, int num_sms) {
 }
 
 bool plan_lut(const vq_linear_desc& d, const DeviceInfo& dev, int M, Plan* p) {
-  if (M != 1 || d.fmt == VQ_FMT_VQ16 || dev.smem_optin < kLutSmem) return false;
+  if (M != 1 || d.fmt == VQ_FMT_VQ16 || d.K % (8 * kLutGroups) != 0 || dev.smem_optin < kLutSmem) return false;
   const LutGeom g = lut_geom(d.N, d.K, dev.num_sms);
+  // Every CTA's units fit its completion list (units per CTA <= kLutMaxList).
+  if (((int64_t)g.S * g.C + g.grid - 1) / g.grid > kLutMaxList) return false;
   p->path = VQ_PATH_LUT;
   p->splits = g.S;
   p->k_per_split = kLutGroups * 8;
@@ -267,26 +353,33 @@ bool plan_lut(const vq_linear_desc& d, const DeviceInfo& dev, int M, Plan* p) {
 }
 
 template <int FMT, typename T>
-static cudaError_t launch_lut_t(const LayerArgs& a, const Plan& p, float* scratch, uint32_t* tickets_buf,
-                                cudaStream_t s) {
+static cudaError_t launch_lut_t(const LayerArgs& a, float* scratch, uint32_t* tickets, cudaStream_t s) {
   int dev = 0, sms = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const LutGeom g = lut_geom(a.N, a.K, sms);
-  cudaError_t e = cudaFuncSetAttribute(lut_gemv_kernel<FMT, T>, cudaFuncAttributeMaxDynamicSharedMemorySize, kLutSmem);
+  auto kern = lut_gemv_kernel<FMT, T>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kLutSmem);
   if (e != cudaSuccess) return e;
-  float* partial = g.S > 1 ? scratch : nullptr;
-  uint32_t* tickets = g.S > 1 ? tickets_buf : nullptr;
-  lut_gemv_kernel<FMT, T><<<g.grid, kLutThreads, kLutSmem, s>>>(a, partial, tickets, g.S, g.C);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(g.grid);
+  cfg.blockDim = dim3(kLutThreads);
+  cfg.dynamicSmemBytes = kLutSmem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // prologue overlaps the previous kernel
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, a, g.S > 1 ? scratch : nullptr, g.S > 1 ? tickets : nullptr, g.S, g.C);
 }
 
-cudaError_t launch_lut(const LayerArgs& a, const Plan& p, float* scratch, uint32_t* tickets, cudaStream_t s) {
+cudaError_t launch_lut(const LayerArgs& a, const Plan&, float* scratch, uint32_t* tickets, cudaStream_t s) {
   if (a.fmt == kFmtRvq12_4)
-    return a.act == VQ_BF16 ? launch_lut_t<kFmtRvq12_4, __nv_bfloat16>(a, p, scratch, tickets, s)
-                            : launch_lut_t<kFmtRvq12_4, __half>(a, p, scratch, tickets, s);
-  return a.act == VQ_BF16 ? launch_lut_t<kFmtRvq12, __nv_bfloat16>(a, p, scratch, tickets, s)
-                          : launch_lut_t<kFmtRvq12, __half>(a, p, scratch, tickets, s);
+    return a.act == VQ_BF16 ? launch_lut_t<kFmtRvq12_4, __nv_bfloat16>(a, scratch, tickets, s)
+                            : launch_lut_t<kFmtRvq12_4, __half>(a, scratch, tickets, s);
+  return a.act == VQ_BF16 ? launch_lut_t<kFmtRvq12, __nv_bfloat16>(a, scratch, tickets, s)
+                          : launch_lut_t<kFmtRvq12, __half>(a, scratch, tickets, s);
 }
 
 }  // namespace vq

@@ -84,7 +84,7 @@ def test_gemv_forward_matches_oracle(oracle, shape, M):
     _check_forward(oracle, layer, act, M, vq.VQ_PATH_GEMV)
 
 
-LUT_SHAPES = [s for s in SHAPES if s[2] != FMT_VQ16] + [
+LUT_SHAPES = [s for s in SHAPES if s[2] != FMT_VQ16 and s[1] % 128 == 0] + [
     (1000, 4096, FMT_RVQ12_4, 64, DT_BF16),   # several 256-row chunks, many K-slices
     (2050, 2048, FMT_RVQ12, 2048, DT_F16),    # ragged last chunk, per-row scales
 ]
@@ -96,6 +96,17 @@ def test_lut_forward_matches_oracle(oracle, shape):
     layer = make_layer(LayerSpec(N, K, fmt, sg), cfg_id=58, tensor_id=N)
     for seed in (0, 1):
         _check_forward(oracle, layer, act, 1, vq.VQ_PATH_LUT, seed=seed)
+
+
+def test_lut_rejects_k_not_multiple_of_128():
+    layer = make_layer(LayerSpec(64, 576, FMT_RVQ12_4, 64), cfg_id=58)
+    L = layer_on_gpu(layer, DT_F16, 1)
+    L.set_path(vq.VQ_PATH_LUT)
+    with pytest.raises(vq.VQError) as ei:
+        L.forward(torch.zeros((1, 576), dtype=torch.float16, device="cuda"))
+    assert ei.value.status == vq._binding.VQ_ERR_UNSUPPORTED
+    L.set_path(vq.VQ_PATH_AUTO)  # AUTO falls back to the warp-MMA kernel
+    assert L.launches(1) >= 1
 
 
 def test_lut_handles_extreme_activation_scales(oracle):

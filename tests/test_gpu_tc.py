@@ -1,0 +1,62 @@
+"""GPU parity of the tensor-core path (decode to shared memory + tcgen05 MMA) against the oracle."""
+
+import numpy as np
+import pytest
+
+import compressed_index_matmul_b200 as vq
+from synth import DT_BF16, DT_F16, FMT_RVQ12, FMT_RVQ12_4, FMT_VQ16, CONFIGS, LayerSpec, make_layer, make_x
+from tests.gpu_util import assert_y_within, layer_on_gpu, require_gpu, run_forward, sub_layer
+
+pytestmark = pytest.mark.gpu
+TOL = 2e-3
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    require_gpu()
+
+
+def _check(oracle, layer, act, M, seed=0):
+    L = layer_on_gpu(layer, act, M)
+    x = make_x(M, layer["spec"].K, act, cfg_id=80, seed=seed)
+    y = run_forward(L, x, act, vq.VQ_PATH_TC)
+    vq.vq_linear_check(L.handle)
+    y_ref = oracle.forward(layer, x, act)
+    w, _ = oracle.dequant(layer)
+    r = assert_y_within(y, act, y_ref, oracle.tolerance(x, act, w, TOL), what=f"tc M={M}")
+    y2 = run_forward(L, x, act, vq.VQ_PATH_TC)
+    assert np.array_equal(y, y2), "not bit-identical run to run"
+    return r
+
+
+TC_CASES = [
+    # (N, K, fmt, scale_group, act, M): ragged rows (N % 128), ragged tokens (M % 16), few/many k blocks
+    (256, 512, FMT_RVQ12_4, 64, DT_BF16, 64),
+    (200, 576, FMT_RVQ12_4, 64, DT_F16, 17),
+    (130, 4096, FMT_VQ16, 4096, DT_F16, 40),
+    (384, 1024, FMT_RVQ12, 64, DT_BF16, 256),
+    (128, 2048, FMT_RVQ12_4, 64, DT_BF16, 300),   # two token tiles, the second ragged
+    (96, 1536, FMT_RVQ12_4, 64, DT_F16, 1),
+]
+
+
+@pytest.mark.parametrize("case", TC_CASES, ids=lambda c: f"{c[0]}x{c[1]}f{c[2]}a{c[4]}M{c[5]}")
+def test_tc_forward_matches_oracle(oracle, case):
+    N, K, fmt, sg, act, M = case
+    layer = make_layer(LayerSpec(N, K, fmt, sg), cfg_id=81, tensor_id=N + M)
+    _check(oracle, layer, act, M)
+
+
+@pytest.mark.parametrize("M", [64, 256])
+def test_prefill_8192_sampled(oracle, M):
+    spec = CONFIGS[5]["tensors"][0][1]
+    layer = make_layer(spec, cfg_id=5)
+    L = layer_on_gpu(layer, DT_BF16, M)
+    x = make_x(M, spec.K, DT_BF16, cfg_id=5)
+    y = run_forward(L, x, DT_BF16, vq.VQ_PATH_AUTO)
+    vq.vq_linear_check(L.handle)
+    rows = np.sort(np.random.default_rng(M).choice(spec.N, size=96, replace=False))
+    sub = sub_layer(layer, rows)
+    y_ref = oracle.forward(sub, x, DT_BF16)
+    w, _ = oracle.dequant(sub)
+    assert_y_within(y[:, rows], DT_BF16, y_ref, oracle.tolerance(x, DT_BF16, w, TOL), what=f"prefill M={M}")
