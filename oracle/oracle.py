@@ -64,9 +64,9 @@ def _load():
             lib.vqo_unpack.restype = I
             lib.vqo_unpack.argtypes = [I, I, I, P, P, P, P, P, P]
             lib.vqo_dequant.restype = I
-            lib.vqo_dequant.argtypes = [I, I, I, P, P, P, P, P, P, P, I, P, P, I]
+            lib.vqo_dequant.argtypes = [I, I, I, P, P, P, P, P, P, P, I, P, I, P, P, I]
             lib.vqo_forward.restype = I
-            lib.vqo_forward.argtypes = [I, I, I, I, P, I, P, P, P, P, P, P, P, I, P]
+            lib.vqo_forward.argtypes = [I, I, I, I, P, I, P, P, P, P, P, P, P, I, P, I, P]
             lib.vqo_rht.restype = I
             lib.vqo_rht.argtypes = [I, I, P, I, P, P]
             _lib = lib
@@ -129,23 +129,32 @@ def unpack(layer) -> tuple[np.ndarray, np.ndarray]:
     return i1, i2
 
 
-def dequant(layer, wdt: int = DT_F16) -> tuple[np.ndarray, np.ndarray]:
-    """Return (W exact fp64 [N,K], W materialised fp16/bf16 bits [N,K])."""
+def _rows(rows):
+    if rows is None:
+        return None, 0
+    r = np.ascontiguousarray(rows, dtype=np.int32)
+    return r, int(r.size)
+
+
+def dequant(layer, wdt: int = DT_F16, rows=None) -> tuple[np.ndarray, np.ndarray]:
+    """Return (W exact fp64 [n,K], W materialised fp16/bf16 bits [n,K]) for `rows` (default: all)."""
     lib = _load()
     spec = layer["spec"]
     lo, hi4, s2, idx16 = _planes(layer)
     cb1, cb2, sc = _c(layer["cb1"], np.uint16), _c(layer.get("cb2"), np.uint16), _c(layer["scales"], np.uint16)
-    w = np.empty((spec.N, spec.K), dtype=np.float64)
-    wb = np.empty((spec.N, spec.K), dtype=np.uint16)
+    r, nr = _rows(rows)
+    n = spec.N if r is None else nr
+    w = np.empty((n, spec.K), dtype=np.float64)
+    wb = np.empty((n, spec.K), dtype=np.uint16)
     rc = lib.vqo_dequant(spec.fmt, spec.N, spec.K, _p(lo), _p(hi4), _p(s2), _p(idx16), _p(cb1), _p(cb2),
-                         _p(sc), spec.scale_group, _p(w), _p(wb), wdt)
+                         _p(sc), spec.scale_group, _p(r), nr, _p(w), _p(wb), wdt)
     if rc:
         raise ValueError(f"vqo_dequant failed rc={rc}")
     return w, wb
 
 
-def forward(layer, x_bits, xdt: int) -> np.ndarray:
-    """y[m][n] = sum_k x[m][k] W[n][k] in fp64 (x given as fp16/bf16 bits [M,K])."""
+def forward(layer, x_bits, xdt: int, rows=None) -> np.ndarray:
+    """y[m][t] = sum_k x[m][k] W[rows[t]][k] in fp64 (x as fp16/bf16 bits [M,K]; rows default: all)."""
     lib = _load()
     spec = layer["spec"]
     x = _c(x_bits, np.uint16)
@@ -154,9 +163,11 @@ def forward(layer, x_bits, xdt: int) -> np.ndarray:
         raise ValueError("x has the wrong K")
     lo, hi4, s2, idx16 = _planes(layer)
     cb1, cb2, sc = _c(layer["cb1"], np.uint16), _c(layer.get("cb2"), np.uint16), _c(layer["scales"], np.uint16)
-    y = np.empty((M, spec.N), dtype=np.float64)
+    r, nr = _rows(rows)
+    n = spec.N if r is None else nr
+    y = np.empty((M, n), dtype=np.float64)
     rc = lib.vqo_forward(spec.fmt, M, spec.N, spec.K, _p(x), xdt, _p(lo), _p(hi4), _p(s2), _p(idx16), _p(cb1),
-                         _p(cb2), _p(sc), spec.scale_group, _p(y))
+                         _p(cb2), _p(sc), spec.scale_group, _p(r), nr, _p(y))
     if rc:
         raise ValueError(f"vqo_forward failed rc={rc}")
     return y

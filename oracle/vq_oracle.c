@@ -17,10 +17,16 @@
  *   - GLQ README, "Inference kernels": Y = X . dequant(W)^T without materialising W.
  *
  * Readings taken where the pages are silent (all fixed here, by construction):
- *   - groups run along K (the input dimension); planes are row-major [N][G], G=K/8;
- *   - "packed hi": two 4-bit fields per byte, group 2t in bits 0..3, 2t+1 in 4..7;
- *     the 4-bit stage-2 plane is packed the same way;
- *   - the 16-bit index plane is one little-endian uint16 per group;
+ *   - groups run along K (the input dimension), G = K/8 groups per row;
+ *   - planes are stored K-slice-major: K is cut into slices of 16 groups (128
+ *     inputs); slice s holds w_s = min(16, G - 16 s) groups; inside a slice the
+ *     rows' entries are contiguous, one row after another (row n's w_s entries
+ *     start at entry 16 s N + n w_s), so consecutive output rows are adjacent in
+ *     memory for every K-slice;
+ *   - "packed hi": two 4-bit fields per byte, group 2t in bits 0..3, 2t+1 in 4..7
+ *     (within a row's slice entries); the 4-bit stage-2 plane is packed the same way;
+ *   - the 16-bit index plane is one little-endian uint16 per group, same layout;
+ *   - scales are stored block-major, scales[b][n] with b = k / scale_group;
  *   - stages are summed with no residual scale (any such scale is folded into
  *     the stage-2 codebook);
  *   - scales are per 64-weight block along K within a row, or one per row
@@ -135,27 +141,45 @@ void vqo_round_array(const double* in, int64_t n, int dt, uint16_t* out) {
  * ------------------------------------------------------------------------- */
 static int vqo_nibble(uint8_t byte, int g) { return (g & 1) ? (byte >> 4) : (byte & 15); }
 
+/* Position, in entries, of group g of row n in a K-slice-major plane with one
+ * entry per group (lo, idx16).  The packed 4-bit planes use half of it. */
+static int64_t vqo_slice_entry(int n, int g, int N, int G) {
+  const int s = g / 16;
+  const int w = (G - 16 * s) < 16 ? (G - 16 * s) : 16;
+  return (int64_t)16 * s * N + (int64_t)n * w + (g - 16 * s);
+}
+
+/* Indices of one row: i1[g] (stage-1 or 16-bit), i2[g] (stage 2, 0 if none). */
+static int vqo_unpack_row(int fmt, int n, int N, int K, const uint8_t* lo, const uint8_t* hi4, const uint8_t* s2,
+                          const uint16_t* idx16, uint32_t* i1, uint8_t* i2) {
+  const int G = K / 8;
+  for (int g = 0; g < G; ++g) {
+    uint32_t a = 0;
+    int b = 0;
+    const int64_t e = vqo_slice_entry(n, g, N, G); /* even for even g: slice widths are even */
+    if (fmt == VQO_FMT_VQ16) {
+      a = idx16[e];
+    } else if (fmt == VQO_FMT_RVQ12 || fmt == VQO_FMT_RVQ12_4) {
+      uint32_t low = lo[e];
+      uint32_t high = (uint32_t)vqo_nibble(hi4[e / 2], g);
+      a = low + 256u * high;
+      if (fmt == VQO_FMT_RVQ12_4) b = vqo_nibble(s2[e / 2], g);
+    } else {
+      return 2;
+    }
+    i1[g] = a;
+    i2[g] = (uint8_t)b;
+  }
+  return 0;
+}
+
 int vqo_unpack(int fmt, int N, int K, const uint8_t* lo, const uint8_t* hi4, const uint8_t* s2,
                const uint16_t* idx16, uint32_t* i1, uint8_t* i2) {
   if (N < 0 || K <= 0 || K % 16 != 0) return 1;
   const int G = K / 8;
   for (int n = 0; n < N; ++n) {
-    for (int g = 0; g < G; ++g) {
-      uint32_t a = 0;
-      int b = 0;
-      if (fmt == VQO_FMT_VQ16) {
-        a = idx16[(int64_t)n * G + g];
-      } else if (fmt == VQO_FMT_RVQ12 || fmt == VQO_FMT_RVQ12_4) {
-        uint32_t low = lo[(int64_t)n * G + g];
-        uint32_t high = (uint32_t)vqo_nibble(hi4[(int64_t)n * (G / 2) + g / 2], g);
-        a = low + 256u * high;
-        if (fmt == VQO_FMT_RVQ12_4) b = vqo_nibble(s2[(int64_t)n * (G / 2) + g / 2], g);
-      } else {
-        return 2;
-      }
-      i1[(int64_t)n * G + g] = a;
-      i2[(int64_t)n * G + g] = (uint8_t)b;
-    }
+    int rc = vqo_unpack_row(fmt, n, N, K, lo, hi4, s2, idx16, i1 + (int64_t)n * G, i2 + (int64_t)n * G);
+    if (rc) return rc;
   }
   return 0;
 }
@@ -166,14 +190,13 @@ int vqo_unpack(int fmt, int N, int K, const uint8_t* lo, const uint8_t* hi4, con
  * k / scale_group.  w_exact is the exact fp64 value s * (c1 + c2); w_bits is
  * the materialised weight RN(fl32(s * fl32(c1 + c2))) in fp16 or bf16.
  * ------------------------------------------------------------------------- */
-static double vqo_weight_exact(int fmt, int n, int k, int K, const uint32_t* i1, const uint8_t* i2,
+static double vqo_weight_exact(int fmt, int n, int k, int N, const uint32_t* i1row, const uint8_t* i2row,
                                const uint16_t* cb1, const uint16_t* cb2, const uint16_t* scales,
                                int scale_group, double* c_out, double* s_out) {
-  const int G = K / 8, g = k / 8, j = k % 8;
-  double c = vqo_f16_to_f64(cb1[(int64_t)i1[(int64_t)n * G + g] * 8 + j]);
-  if (fmt == VQO_FMT_RVQ12_4) c += vqo_f16_to_f64(cb2[(int64_t)i2[(int64_t)n * G + g] * 8 + j]);
-  const int nblk = K / scale_group;
-  double s = vqo_f16_to_f64(scales[(int64_t)n * nblk + k / scale_group]);
+  const int g = k / 8, j = k % 8;
+  double c = vqo_f16_to_f64(cb1[(int64_t)i1row[g] * 8 + j]);
+  if (fmt == VQO_FMT_RVQ12_4) c += vqo_f16_to_f64(cb2[(int64_t)i2row[g] * 8 + j]);
+  double s = vqo_f16_to_f64(scales[(int64_t)(k / scale_group) * N + n]); /* block-major scales[b][n] */
   *c_out = c;
   *s_out = s;
   return s * c;
@@ -186,25 +209,29 @@ static int vqo_check(int fmt, int N, int K, int scale_group) {
   return 0;
 }
 
+/* rows: the output rows to decode (NULL = all N); outputs are [nrows][K]. */
 int vqo_dequant(int fmt, int N, int K, const uint8_t* lo, const uint8_t* hi4, const uint8_t* s2,
                 const uint16_t* idx16, const uint16_t* cb1, const uint16_t* cb2, const uint16_t* scales,
-                int scale_group, double* w_exact, uint16_t* w_bits, int wdt) {
+                int scale_group, const int32_t* rows, int nrows, double* w_exact, uint16_t* w_bits, int wdt) {
   int rc = vqo_check(fmt, N, K, scale_group);
   if (rc) return rc;
+  if (!rows) nrows = N;
   const int G = K / 8;
-  uint32_t* i1 = (uint32_t*)malloc(sizeof(uint32_t) * (size_t)N * G + 1);
-  uint8_t* i2 = (uint8_t*)malloc((size_t)N * G + 1);
+  uint32_t* i1 = (uint32_t*)malloc(sizeof(uint32_t) * (size_t)G);
+  uint8_t* i2 = (uint8_t*)malloc((size_t)G);
   if (!i1 || !i2) { free(i1); free(i2); return 3; }
-  rc = vqo_unpack(fmt, N, K, lo, hi4, s2, idx16, i1, i2);
-  for (int n = 0; rc == 0 && n < N; ++n) {
-    for (int k = 0; k < K; ++k) {
+  for (int t = 0; rc == 0 && t < nrows; ++t) {
+    const int n = rows ? rows[t] : t;
+    if (n < 0 || n >= N) { rc = 1; break; }
+    rc = vqo_unpack_row(fmt, n, N, K, lo, hi4, s2, idx16, i1, i2);
+    for (int k = 0; rc == 0 && k < K; ++k) {
       double c, s;
-      double w = vqo_weight_exact(fmt, n, k, K, i1, i2, cb1, cb2, scales, scale_group, &c, &s);
-      if (w_exact) w_exact[(int64_t)n * K + k] = w;
+      double w = vqo_weight_exact(fmt, n, k, N, i1, i2, cb1, cb2, scales, scale_group, &c, &s);
+      if (w_exact) w_exact[(int64_t)t * K + k] = w;
       if (w_bits) {
-        double c32 = vqo_fl32(c);      /* stage sum rounded to fp32 */
+        double c32 = vqo_fl32(c);       /* stage sum rounded to fp32 */
         double p32 = vqo_fl32(s * c32); /* exact product of two fp32-representable values, rounded */
-        w_bits[(int64_t)n * K + k] = wdt == VQO_DT_BF16 ? vqo_f64_to_bf16(p32) : vqo_f64_to_f16(p32);
+        w_bits[(int64_t)t * K + k] = wdt == VQO_DT_BF16 ? vqo_f64_to_bf16(p32) : vqo_f64_to_f16(p32);
       }
     }
   }
@@ -215,31 +242,36 @@ int vqo_dequant(int fmt, int N, int K, const uint8_t* lo, const uint8_t* hi4, co
 
 /* ---------------------------------------------------------------------------
  * Forward (GLQ README, "Inference kernels": Y = X . dequant(W)^T).
- * y[m][n] = sum_k x[m][k] * W[n][k], with W the exact fp64 decode, x taken
- * exactly from its fp16/bf16 bits, a naive loop over k in order.
+ * y[m][t] = sum_k x[m][k] * W[rows[t]][k], with W the exact fp64 decode, x taken
+ * exactly from its fp16/bf16 bits, a naive loop over k in order.  rows == NULL
+ * means every row (nrows = N); y is [M][nrows].
  * ------------------------------------------------------------------------- */
 int vqo_forward(int fmt, int M, int N, int K, const uint16_t* x, int xdt, const uint8_t* lo,
                 const uint8_t* hi4, const uint8_t* s2, const uint16_t* idx16, const uint16_t* cb1,
-                const uint16_t* cb2, const uint16_t* scales, int scale_group, double* y) {
+                const uint16_t* cb2, const uint16_t* scales, int scale_group, const int32_t* rows, int nrows,
+                double* y) {
   int rc = vqo_check(fmt, N, K, scale_group);
   if (rc || M < 0) return rc ? rc : 1;
+  if (!rows) nrows = N;
   const int G = K / 8;
-  uint32_t* i1 = (uint32_t*)malloc(sizeof(uint32_t) * (size_t)N * G + 1);
-  uint8_t* i2 = (uint8_t*)malloc((size_t)N * G + 1);
+  uint32_t* i1 = (uint32_t*)malloc(sizeof(uint32_t) * (size_t)G);
+  uint8_t* i2 = (uint8_t*)malloc((size_t)G);
   double* wrow = (double*)malloc(sizeof(double) * (size_t)K);
   double* xd = (double*)malloc(sizeof(double) * (size_t)M * K + 1);
   if (!i1 || !i2 || !wrow || !xd) { free(i1); free(i2); free(wrow); free(xd); return 3; }
-  rc = vqo_unpack(fmt, N, K, lo, hi4, s2, idx16, i1, i2);
-  for (int64_t t = 0; rc == 0 && t < (int64_t)M * K; ++t) xd[t] = vqo_act_to_f64(x[t], xdt);
-  for (int n = 0; rc == 0 && n < N; ++n) {
-    for (int k = 0; k < K; ++k) {
+  for (int64_t t = 0; t < (int64_t)M * K; ++t) xd[t] = vqo_act_to_f64(x[t], xdt);
+  for (int t = 0; rc == 0 && t < nrows; ++t) {
+    const int n = rows ? rows[t] : t;
+    if (n < 0 || n >= N) { rc = 1; break; }
+    rc = vqo_unpack_row(fmt, n, N, K, lo, hi4, s2, idx16, i1, i2);
+    for (int k = 0; rc == 0 && k < K; ++k) {
       double c, s;
-      wrow[k] = vqo_weight_exact(fmt, n, k, K, i1, i2, cb1, cb2, scales, scale_group, &c, &s);
+      wrow[k] = vqo_weight_exact(fmt, n, k, N, i1, i2, cb1, cb2, scales, scale_group, &c, &s);
     }
-    for (int m = 0; m < M; ++m) {
+    for (int m = 0; rc == 0 && m < M; ++m) {
       double acc = 0.0;
       for (int k = 0; k < K; ++k) acc += xd[(int64_t)m * K + k] * wrow[k];
-      y[(int64_t)m * N + n] = acc;
+      y[(int64_t)m * nrows + t] = acc;
     }
   }
   free(i1);

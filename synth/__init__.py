@@ -11,14 +11,18 @@ Storage format (the encoder's output, consumed by both implementations):
 * weights W are N x K (out x in); each run of 8 consecutive weights along K is
   one group, G = K // 8 groups per row (orka README, "How it works": each group
   of 8 values is replaced by one codebook index).
-* ``lo``  uint8  [N, G]      low 8 bits of the 12-bit stage-1 index
-* ``hi4`` uint8  [N, G//2]   high 4 bits of the stage-1 index, two groups per
-  byte: group 2t in bits 0..3, group 2t+1 in bits 4..7
-* ``s2``  uint8  [N, G//2]   4-bit stage-2 index, packed like ``hi4``
-* ``idx16`` uint16 [N, G]    16-bit single-stage index (GLQ README, "How it
+* planes are flat arrays in K-slice-major order: K is cut into slices of 16
+  groups (128 inputs); slice s holds w_s = min(16, G - 16 s) groups; inside a
+  slice the rows' entries are contiguous, one row after another.
+* ``lo``  uint8  [N*G]      low 8 bits of the 12-bit stage-1 index
+* ``hi4`` uint8  [N*G/2]    high 4 bits of the stage-1 index, two groups per
+  byte within a row's slice entries: group 2t in bits 0..3, group 2t+1 in 4..7
+* ``s2``  uint8  [N*G/2]    4-bit stage-2 index, packed like ``hi4``
+* ``idx16`` uint16 [N*G]    16-bit single-stage index (GLQ README, "How it
   works", E8 lattice codebooks: one 16-bit index per group of 8)
 * ``cb1`` fp16 [4096, 8] (or [65536, 8] for 16-bit indices), ``cb2`` fp16 [16, 8]
-* ``scales`` fp16 [N, K // scale_group]; ``scale_group == K`` is one scale per row
+* ``scales`` fp16 [K // scale_group, N] (block-major); ``scale_group == K`` is
+  one scale per row
 * ``x`` fp16 or bf16 [M, K]; ``signs`` int8 [K] of +-1 for the input rotation
 
 fp16/bf16 arrays are returned as raw uint16 bit patterns.

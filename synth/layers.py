@@ -62,18 +62,21 @@ def make_layer(spec: LayerSpec, cfg_id: int = 0, layer: int = 0, tensor_id: int 
         raise ValueError(f"K={K} must be a multiple of 16 and of scale_group={spec.scale_group}")
     r = _rng(cfg_id, layer, tensor_id, seed)
     out: dict = {"spec": spec}
+    # Planes are flat arrays (their element order is the K-slice-major storage order;
+    # the values are iid uniform, so the generator needs no layout arithmetic).
     if spec.fmt == FMT_VQ16:
         out["cb1"] = f32_to_f16_bits(r.standard_normal((65536, 8), dtype=np.float32))
-        out["idx16"] = r.integers(0, 65536, size=(N, G), dtype=np.uint16)
+        out["idx16"] = r.integers(0, 65536, size=N * G, dtype=np.uint16)
     else:
         out["cb1"] = f32_to_f16_bits(r.standard_normal((4096, 8), dtype=np.float32))
-        out["lo"] = r.integers(0, 256, size=(N, G), dtype=np.uint8)
-        out["hi4"] = r.integers(0, 256, size=(N, G // 2), dtype=np.uint8)
+        out["lo"] = r.integers(0, 256, size=N * G, dtype=np.uint8)
+        out["hi4"] = r.integers(0, 256, size=N * G // 2, dtype=np.uint8)
         if spec.fmt == FMT_RVQ12_4:
             out["cb2"] = f32_to_f16_bits(r.standard_normal((16, 8), dtype=np.float32))
-            out["s2"] = r.integers(0, 256, size=(N, G // 2), dtype=np.uint8)
+            out["s2"] = r.integers(0, 256, size=N * G // 2, dtype=np.uint8)
     nblk = K // spec.scale_group
-    out["scales"] = f32_to_f16_bits(r.lognormal(-4.0, 0.5, size=(N, nblk)).astype(np.float32))
+    # block-major: scales[b][n]
+    out["scales"] = f32_to_f16_bits(r.lognormal(-4.0, 0.5, size=(nblk, N)).astype(np.float32))
     return out
 
 

@@ -99,25 +99,74 @@ def _golden(name):
 
 
 def test_unpack_golden_layout(oracle):
+    # K=32: a single slice, so the sliced order equals the row-major order of the fixture
     g = _golden("unpack_layout.json")
     spec = LayerSpec(g["N"], g["K"], FMT_RVQ12_4, 32)
-    layer = {"spec": spec, "lo": np.array(g["lo"], np.uint8), "hi4": np.array(g["hi4"], np.uint8),
-             "s2": np.array(g["s2"], np.uint8)}
+    layer = {"spec": spec, "lo": np.array(g["lo"], np.uint8).ravel(), "hi4": np.array(g["hi4"], np.uint8).ravel(),
+             "s2": np.array(g["s2"], np.uint8).ravel()}
     i1, i2 = oracle.unpack(layer)
     assert i1.tolist() == g["i1"]
     assert i2.tolist() == g["i2"]
 
 
+def _slices(G):
+    """(first group, width) of every 16-group slice of a row of G groups."""
+    return [(g0, min(16, G - g0)) for g0 in range(0, G, 16)]
+
+
+def to_sliced(a2d: np.ndarray, per_group: float) -> np.ndarray:
+    """Row-major [N][G*per_group] -> flat K-slice-major order (written from the layout description)."""
+    N, E = a2d.shape
+    G = int(round(E / per_group))
+    out = []
+    for g0, w in _slices(G):
+        e0, e1 = int(g0 * per_group), int((g0 + w) * per_group)
+        out.append(a2d[:, e0:e1].reshape(-1))
+    return np.concatenate(out)
+
+
+def from_sliced(flat: np.ndarray, N: int, G: int, per_group: float) -> np.ndarray:
+    """Inverse of to_sliced."""
+    cols = []
+    pos = 0
+    for g0, w in _slices(G):
+        e = int(w * per_group)
+        cols.append(flat[pos:pos + N * e].reshape(N, e))
+        pos += N * e
+    return np.concatenate(cols, axis=1)
+
+
 def _pack12(i1, i2=None):
-    """Pack indices into the plane layout (written here from the layout description)."""
+    """Pack indices [N][G] into the plane format (written here from the layout description)."""
     N, G = i1.shape
     lo = (i1 & 0xFF).astype(np.uint8)
     hi = (i1 >> 8).astype(np.uint8)
     hi4 = (hi[:, 0::2] | (hi[:, 1::2] << 4)).astype(np.uint8)
-    out = {"lo": lo, "hi4": hi4}
+    out = {"lo": to_sliced(lo, 1), "hi4": to_sliced(hi4, 0.5)}
     if i2 is not None:
-        out["s2"] = (i2[:, 0::2] | (i2[:, 1::2] << 4)).astype(np.uint8)
+        out["s2"] = to_sliced((i2[:, 0::2] | (i2[:, 1::2] << 4)).astype(np.uint8), 0.5)
     return out
+
+
+def test_slice_layout_golden(oracle):
+    g = _golden("slice_layout.json")
+    for case in g["cases"]:
+        N, K = case["N"], case["K"]
+        G = K // 8
+        layer = {"spec": LayerSpec(N, K, FMT_RVQ12, K), "lo": (np.arange(N * G) % 256).astype(np.uint8),
+                 "hi4": (np.arange(N * G // 2) % 256).astype(np.uint8)}
+        i1, _ = oracle.unpack(layer)
+        for n, grp, expect in case["checks"]:
+            assert int(i1[n, grp]) == expect, (K, n, grp)
+
+
+def test_layout_helpers_round_trip():
+    rng = np.random.default_rng(9)
+    for N, G in ((3, 16), (5, 48), (4, 24), (2, 8)):
+        a = rng.integers(0, 256, size=(N, G), dtype=np.uint8)
+        assert np.array_equal(from_sliced(to_sliced(a, 1), N, G, 1), a)
+        h = rng.integers(0, 256, size=(N, G // 2), dtype=np.uint8)
+        assert np.array_equal(from_sliced(to_sliced(h, 0.5), N, G, 0.5), h)
 
 
 def test_unpack_round_trip_all_12bit_values_both_parities(oracle):
@@ -137,7 +186,7 @@ def test_unpack_round_trip_all_12bit_values_both_parities(oracle):
 
 def test_unpack_round_trip_all_16bit_values(oracle):
     vals = np.arange(65536, dtype=np.uint32).astype(np.uint16).reshape(-1, 256)
-    layer = {"spec": LayerSpec(vals.shape[0], 256 * 8, FMT_VQ16, 2048), "idx16": vals}
+    layer = {"spec": LayerSpec(vals.shape[0], 256 * 8, FMT_VQ16, 2048), "idx16": to_sliced(vals, 1)}
     o1, o2 = oracle.unpack(layer)
     assert np.array_equal(o1, vals.astype(np.uint32))
     assert not o2.any()
@@ -155,8 +204,9 @@ def _tiny_layer_from_golden(g):
     i1 = np.array([g["i1"]], np.uint32)
     i2 = np.array([g["i2"]], np.uint32)
     spec = LayerSpec(g["N"], g["K"], g["fmt"], g["scale_group"])
+    # one row: block-major scales [blocks][1]
     return {"spec": spec, "cb1": cb1.view(np.uint16), "cb2": cb2.view(np.uint16),
-            "scales": np.array([g["scales"]], np.float16).view(np.uint16), **_pack12(i1, i2)}
+            "scales": np.array(g["scales"], np.float16).reshape(-1, 1).view(np.uint16), **_pack12(i1, i2)}
 
 
 def test_decode_golden_tiny_codebooks(oracle):
@@ -199,30 +249,36 @@ def test_decode_rounding_points_by_hand(oracle, c1, c2, s, dt, expect):
 def _dense_numpy(layer):
     """Brute-force dense W, built here independently with numpy fancy indexing."""
     spec = layer["spec"]
+    N, G = spec.N, spec.G
     cb1 = layer["cb1"].view(np.float16).astype(np.float64)
     if spec.fmt == FMT_VQ16:
-        i1 = layer["idx16"].astype(np.int64)
+        i1 = from_sliced(layer["idx16"], N, G, 1).astype(np.int64)
     else:
-        hi = np.empty((spec.N, spec.G), np.int64)
-        hi[:, 0::2] = layer["hi4"] & 15
-        hi[:, 1::2] = layer["hi4"] >> 4
-        i1 = layer["lo"].astype(np.int64) + 256 * hi
+        h4 = from_sliced(layer["hi4"], N, G, 0.5)
+        hi = np.empty((N, G), np.int64)
+        hi[:, 0::2] = h4 & 15
+        hi[:, 1::2] = h4 >> 4
+        i1 = from_sliced(layer["lo"], N, G, 1).astype(np.int64) + 256 * hi
     W = cb1[i1]  # [N, G, 8]
     if spec.fmt == FMT_RVQ12_4:
-        i2 = np.empty((spec.N, spec.G), np.int64)
-        i2[:, 0::2] = layer["s2"] & 15
-        i2[:, 1::2] = layer["s2"] >> 4
+        s2 = from_sliced(layer["s2"], N, G, 0.5)
+        i2 = np.empty((N, G), np.int64)
+        i2[:, 0::2] = s2 & 15
+        i2[:, 1::2] = s2 >> 4
         W = W + layer["cb2"].view(np.float16).astype(np.float64)[i2]
-    W = W.reshape(spec.N, spec.K)
-    sc = layer["scales"].view(np.float16).astype(np.float64)
-    return W * np.repeat(sc, spec.scale_group, axis=1)
+    W = W.reshape(N, spec.K)
+    sc = layer["scales"].view(np.float16).astype(np.float64).reshape(-1, N)  # [blocks][N]
+    return W * np.repeat(sc.T, spec.scale_group, axis=1)
 
 
-@pytest.mark.parametrize("fmt,sg", [(FMT_RVQ12, 8), (FMT_RVQ12_4, 16), (FMT_VQ16, 16), (FMT_RVQ12_4, 8)])
+@pytest.mark.parametrize("fmt,sg,K", [(FMT_RVQ12, 8, 16), (FMT_RVQ12_4, 16, 16), (FMT_VQ16, 16, 16),
+                                      (FMT_RVQ12_4, 8, 16), (FMT_RVQ12_4, 64, 384), (FMT_RVQ12, 192, 192),
+                                      (FMT_VQ16, 64, 320)])
 @pytest.mark.parametrize("xdt", [DT_F16, DT_BF16])
-def test_forward_brute_force_16x16(oracle, fmt, sg, xdt):
-    layer = make_layer(LayerSpec(16, 16, fmt, sg), cfg_id=99, tensor_id=fmt * 10 + sg)
-    x = make_x(5, 16, xdt, cfg_id=99)
+def test_forward_brute_force_16x16(oracle, fmt, sg, K, xdt):
+    # 16 rows; K=16 (one slice) and K=384 / 192 / 320 (several slices, some ragged)
+    layer = make_layer(LayerSpec(16, K, fmt, sg), cfg_id=99, tensor_id=fmt * 10 + sg)
+    x = make_x(5, K, xdt, cfg_id=99)
     W = _dense_numpy(layer)
     xd = x.view(np.float16).astype(np.float64) if xdt == DT_F16 else \
         (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
@@ -231,6 +287,9 @@ def test_forward_brute_force_16x16(oracle, fmt, sg, xdt):
     assert np.allclose(y, ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
     w, _ = oracle.dequant(layer)
     assert np.array_equal(w, W)
+    rows = [15, 0, 7]
+    assert np.array_equal(oracle.forward(layer, x, xdt, rows=rows), y[:, rows])
+    assert np.array_equal(oracle.dequant(layer, rows=rows)[0], W[rows])
 
 
 def test_forward_one_hot_returns_columns(oracle):
