@@ -26,7 +26,9 @@
  *   - "packed hi": two 4-bit fields per byte, group 2t in bits 0..3, 2t+1 in 4..7
  *     (within a row's slice entries); the 4-bit stage-2 plane is packed the same way;
  *   - the 16-bit index plane is one little-endian uint16 per group, same layout;
- *   - scales are stored block-major, scales[b][n] with b = k / scale_group;
+ *   - block scales (scale_group dividing 64) are stored K-slice-major like the
+ *     planes, with 128 / scale_group entries per full slice (row n's scales of
+ *     slice s are adjacent); one scale per row (scale_group == K) is scales[n];
  *   - stages are summed with no residual scale (any such scale is folded into
  *     the stage-2 codebook);
  *   - scales are per 64-weight block along K within a row, or one per row
@@ -149,6 +151,16 @@ static int64_t vqo_slice_entry(int n, int g, int N, int G) {
   return (int64_t)16 * s * N + (int64_t)n * w + (g - 16 * s);
 }
 
+/* Position of the scale of weight (n, k).  One per row: scales[n].  Block scales:
+ * K-slice-major, each row holding w_s * 8 / scale_group entries of slice s. */
+static int64_t vqo_scale_index(int n, int k, int N, int K, int scale_group) {
+  if (scale_group == K) return n;
+  const int G = K / 8, s = k / 128;
+  const int w = (G - 16 * s) < 16 ? (G - 16 * s) : 16;
+  const int per_row = w * 8 / scale_group;
+  return (int64_t)(128 / scale_group) * s * N + (int64_t)n * per_row + (k - 128 * s) / scale_group;
+}
+
 /* Indices of one row: i1[g] (stage-1 or 16-bit), i2[g] (stage 2, 0 if none). */
 static int vqo_unpack_row(int fmt, int n, int N, int K, const uint8_t* lo, const uint8_t* hi4, const uint8_t* s2,
                           const uint16_t* idx16, uint32_t* i1, uint8_t* i2) {
@@ -190,13 +202,13 @@ int vqo_unpack(int fmt, int N, int K, const uint8_t* lo, const uint8_t* hi4, con
  * k / scale_group.  w_exact is the exact fp64 value s * (c1 + c2); w_bits is
  * the materialised weight RN(fl32(s * fl32(c1 + c2))) in fp16 or bf16.
  * ------------------------------------------------------------------------- */
-static double vqo_weight_exact(int fmt, int n, int k, int N, const uint32_t* i1row, const uint8_t* i2row,
+static double vqo_weight_exact(int fmt, int n, int k, int N, int K, const uint32_t* i1row, const uint8_t* i2row,
                                const uint16_t* cb1, const uint16_t* cb2, const uint16_t* scales,
                                int scale_group, double* c_out, double* s_out) {
   const int g = k / 8, j = k % 8;
   double c = vqo_f16_to_f64(cb1[(int64_t)i1row[g] * 8 + j]);
   if (fmt == VQO_FMT_RVQ12_4) c += vqo_f16_to_f64(cb2[(int64_t)i2row[g] * 8 + j]);
-  double s = vqo_f16_to_f64(scales[(int64_t)(k / scale_group) * N + n]); /* block-major scales[b][n] */
+  double s = vqo_f16_to_f64(scales[vqo_scale_index(n, k, N, K, scale_group)]);
   *c_out = c;
   *s_out = s;
   return s * c;
@@ -205,6 +217,7 @@ static double vqo_weight_exact(int fmt, int n, int k, int N, const uint32_t* i1r
 static int vqo_check(int fmt, int N, int K, int scale_group) {
   if (N < 0 || K <= 0 || K % 16 != 0) return 1;
   if (scale_group <= 0 || scale_group % 8 != 0 || K % scale_group != 0) return 1;
+  if (scale_group != K && 64 % scale_group != 0) return 1; /* blocks must tile every slice */
   if (fmt != VQO_FMT_RVQ12 && fmt != VQO_FMT_RVQ12_4 && fmt != VQO_FMT_VQ16) return 2;
   return 0;
 }
@@ -226,7 +239,7 @@ int vqo_dequant(int fmt, int N, int K, const uint8_t* lo, const uint8_t* hi4, co
     rc = vqo_unpack_row(fmt, n, N, K, lo, hi4, s2, idx16, i1, i2);
     for (int k = 0; rc == 0 && k < K; ++k) {
       double c, s;
-      double w = vqo_weight_exact(fmt, n, k, N, i1, i2, cb1, cb2, scales, scale_group, &c, &s);
+      double w = vqo_weight_exact(fmt, n, k, N, K, i1, i2, cb1, cb2, scales, scale_group, &c, &s);
       if (w_exact) w_exact[(int64_t)t * K + k] = w;
       if (w_bits) {
         double c32 = vqo_fl32(c);       /* stage sum rounded to fp32 */
@@ -266,7 +279,7 @@ int vqo_forward(int fmt, int M, int N, int K, const uint16_t* x, int xdt, const 
     rc = vqo_unpack_row(fmt, n, N, K, lo, hi4, s2, idx16, i1, i2);
     for (int k = 0; rc == 0 && k < K; ++k) {
       double c, s;
-      wrow[k] = vqo_weight_exact(fmt, n, k, N, i1, i2, cb1, cb2, scales, scale_group, &c, &s);
+      wrow[k] = vqo_weight_exact(fmt, n, k, N, K, i1, i2, cb1, cb2, scales, scale_group, &c, &s);
     }
     for (int m = 0; rc == 0 && m < M; ++m) {
       double acc = 0.0;

@@ -21,8 +21,9 @@ Storage format (the encoder's output, consumed by both implementations):
 * ``idx16`` uint16 [N*G]    16-bit single-stage index (GLQ README, "How it
   works", E8 lattice codebooks: one 16-bit index per group of 8)
 * ``cb1`` fp16 [4096, 8] (or [65536, 8] for 16-bit indices), ``cb2`` fp16 [16, 8]
-* ``scales`` fp16 [K // scale_group, N] (block-major); ``scale_group == K`` is
-  one scale per row
+* ``scales`` fp16 [N * K // scale_group]: block scales (scale_group dividing 64)
+  in K-slice-major order like the planes (a row's scales of one slice are
+  adjacent); ``scale_group == K`` is one scale per row, [N]
 * ``x`` fp16 or bf16 [M, K]; ``signs`` int8 [K] of +-1 for the input rotation
 
 fp16/bf16 arrays are returned as raw uint16 bit patterns.

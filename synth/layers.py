@@ -75,8 +75,8 @@ def make_layer(spec: LayerSpec, cfg_id: int = 0, layer: int = 0, tensor_id: int 
             out["cb2"] = f32_to_f16_bits(r.standard_normal((16, 8), dtype=np.float32))
             out["s2"] = r.integers(0, 256, size=N * G // 2, dtype=np.uint8)
     nblk = K // spec.scale_group
-    # block-major: scales[b][n]
-    out["scales"] = f32_to_f16_bits(r.lognormal(-4.0, 0.5, size=(nblk, N)).astype(np.float32))
+    # flat, in the scales' storage order (K-slice-major for block scales, [N] per row)
+    out["scales"] = f32_to_f16_bits(r.lognormal(-4.0, 0.5, size=N * nblk).astype(np.float32))
     return out
 
 

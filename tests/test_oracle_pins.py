@@ -160,6 +160,23 @@ def test_slice_layout_golden(oracle):
             assert int(i1[n, grp]) == expect, (K, n, grp)
 
 
+def test_scale_layout_by_hand(oracle):
+    """Block scales follow the planes' slice order: K=192 (slices of 16 and 8 groups), N=2,
+    scale_group=64 -> per row 2 scales in slice 0 and 1 in slice 1; storage order
+    [r0b0, r0b1, r1b0, r1b1, r0b2, r1b2].  With cb1 entry 0 = all ones and index 0
+    everywhere, W[n][k] equals the scale of (n, k)."""
+    N, K = 2, 192
+    vals = np.array([1, 2, 3, 4, 5, 6], np.float16)
+    cb1 = np.zeros((4096, 8), np.float16)
+    cb1[0] = 1
+    layer = {"spec": LayerSpec(N, K, FMT_RVQ12, 64), "lo": np.zeros(N * K // 8, np.uint8),
+             "hi4": np.zeros(N * K // 16, np.uint8), "cb1": cb1.view(np.uint16), "scales": vals.view(np.uint16)}
+    w, _ = oracle.dequant(layer)
+    expect = {(0, 0): 1, (0, 64): 2, (1, 0): 3, (1, 127): 4, (0, 128): 5, (1, 191): 6}
+    for (n, k), v in expect.items():
+        assert w[n, k] == v, (n, k)
+
+
 def test_layout_helpers_round_trip():
     rng = np.random.default_rng(9)
     for N, G in ((3, 16), (5, 48), (4, 24), (2, 8)):
@@ -204,9 +221,9 @@ def _tiny_layer_from_golden(g):
     i1 = np.array([g["i1"]], np.uint32)
     i2 = np.array([g["i2"]], np.uint32)
     spec = LayerSpec(g["N"], g["K"], g["fmt"], g["scale_group"])
-    # one row: block-major scales [blocks][1]
+    # one row, one slice: the row's block scales in order
     return {"spec": spec, "cb1": cb1.view(np.uint16), "cb2": cb2.view(np.uint16),
-            "scales": np.array(g["scales"], np.float16).reshape(-1, 1).view(np.uint16), **_pack12(i1, i2)}
+            "scales": np.array(g["scales"], np.float16).view(np.uint16), **_pack12(i1, i2)}
 
 
 def test_decode_golden_tiny_codebooks(oracle):
@@ -267,13 +284,17 @@ def _dense_numpy(layer):
         i2[:, 1::2] = s2 >> 4
         W = W + layer["cb2"].view(np.float16).astype(np.float64)[i2]
     W = W.reshape(N, spec.K)
-    sc = layer["scales"].view(np.float16).astype(np.float64).reshape(-1, N)  # [blocks][N]
-    return W * np.repeat(sc.T, spec.scale_group, axis=1)
+    sc = layer["scales"].view(np.float16).astype(np.float64)
+    if spec.scale_group == spec.K:
+        scm = sc.reshape(N, 1)
+    else:  # K-slice-major with 8 / scale_group entries per group
+        scm = from_sliced(sc, N, G, 8 / spec.scale_group)
+    return W * np.repeat(scm, spec.scale_group, axis=1)
 
 
 @pytest.mark.parametrize("fmt,sg,K", [(FMT_RVQ12, 8, 16), (FMT_RVQ12_4, 16, 16), (FMT_VQ16, 16, 16),
                                       (FMT_RVQ12_4, 8, 16), (FMT_RVQ12_4, 64, 384), (FMT_RVQ12, 192, 192),
-                                      (FMT_VQ16, 64, 320)])
+                                      (FMT_VQ16, 64, 320), (FMT_RVQ12_4, 32, 192)])
 @pytest.mark.parametrize("xdt", [DT_F16, DT_BF16])
 def test_forward_brute_force_16x16(oracle, fmt, sg, K, xdt):
     # 16 rows; K=16 (one slice) and K=384 / 192 / 320 (several slices, some ragged)
