@@ -15,8 +15,9 @@ and reported under "detail" (the SmolLM-135M-shaped 30-layer stack at M=1 and
 
 Timing: W untimed warm-up steps; then exactly K steps, each a replay of a CUDA
 graph of the step's forwards, bracketed by CUDA events on the launching stream;
-the L2 cache is flushed (a 512 MiB buffer is overwritten) between timed steps,
-outside the events.  Barrier + synchronize before and after; the max over ranks
+the L2 cache is flushed between timed steps, outside the events, by writing a
+512 MiB buffer and then reading it back (so L2 is left holding clean lines and
+the timed kernels pay no write-back of the flush).  Barrier + synchronize before and after; the max over ranks
 is reported.  With --gpus N (torchrun) every rank runs an independent replica
 (the layer does not shard here) and ``value`` aggregates all ranks' layers.
 
@@ -210,10 +211,21 @@ class Workload:
         return sum(2.0 * M * spec.N * spec.K for _, spec, _ in self.layers)
 
 
-def _flush_buffer():
-    import torch
+class _Flush:
+    """Evicts L2: write a 512 MiB buffer, then read it (leaving clean lines in L2)."""
 
-    return torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
+    def __init__(self):
+        import torch
+
+        self.buf = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
+
+    def zero_(self):
+        self.buf.zero_()
+        self.buf.sum()
+
+
+def _flush_buffer():
+    return _Flush()
 
 
 def time_graph(wl, M, steps, warmup, flush, per_kernel=False):
@@ -356,14 +368,8 @@ def gpu_arm(args):
     torch.cuda.synchronize()
     del g
     step_ms = [start[k].elapsed_time(end[k]) for k in range(args.steps)]
-    total_ms = float(sum(step_ms))
-    if world > 1:
-        t = torch.tensor([total_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
-    ms_per_step = total_ms / args.steps
     layers = len(wl.layers)
-    us_per_layer = 1e3 * ms_per_step / (layers * world)
+    ms_per_step, us_per_layer = aggregate_over_ranks(float(sum(step_ms)), args.steps, layers, world)
 
     # ------------------------------------------------ per-kernel roofline (same stream, graph nodes)
     _, per_fwd = time_graph(wl, M, min(args.steps, 200), 3, flush, per_kernel=True)
@@ -392,7 +398,8 @@ def gpu_arm(args):
         "config": {"workload": args.workload, "M": M, "layers_per_step": layers,
                    "shapes": [[spec.N, spec.K] for _, spec, _ in wl.layers[:7]],
                    "format": "rvq12_4 block-64" if args.workload != "vq16-4096-rht" else "vq16 per-row",
-                   "parallelism": f"replicas x{world}", "l2": "flushed between timed steps (512 MiB write)",
+                   "parallelism": f"replicas x{world}",
+                   "l2": "flushed between timed steps (512 MiB write then read)",
                    "layer": "one vq_linear_forward (one weight matrix)",
                    "hbm_gbs": round(sum(bytes_per_fwd) / (ms_per_step * 1e-3) / 1e9, 1)},
         "roofline": roofline,
@@ -409,6 +416,29 @@ def gpu_arm(args):
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(out), flush=True)
+
+
+def max_over_ranks(value: float, world: int) -> float:
+    """Max of a per-rank value over all ranks (identity on one rank)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_over_ranks(total_ms_local: float, steps: int, layers_per_step: int, world: int):
+    """Whole-job timing: the slowest rank's time; every rank ran `layers_per_step` layers per step.
+
+    Returns (ms_per_step, us_per_layer) where us_per_layer divides by the layers all ranks ran.
+    """
+    total_ms = max_over_ranks(total_ms_local, world)
+    ms_per_step = total_ms / steps
+    return ms_per_step, 1e3 * ms_per_step / (layers_per_step * world)
 
 
 def lookup_traffic(kernel, workload, M):

@@ -95,15 +95,16 @@ cudaError_t launch_rht(const void* x, void* x_out, const int8_t* signs, int M, i
 
 __device__ __forceinline__ void unpack_one(const LayerArgs& a, int n, int g, uint32_t* i1, uint32_t* i2) {
   const int G = a.K / 8;
+  const int64_t e = slice_entry(n, g, a.N, G);  // even for even g (slice widths are even)
   if (a.fmt == kFmtVq16) {
-    *i1 = a.idx16[(int64_t)n * G + g];
+    *i1 = a.idx16[e];
     *i2 = 0;
     return;
   }
-  const uint32_t hb = a.hi4[(int64_t)n * (G / 2) + g / 2];
-  *i1 = a.lo[(int64_t)n * G + g] | (((g & 1) ? (hb >> 4) : (hb & 15u)) << 8);
+  const uint32_t hb = a.hi4[e >> 1];
+  *i1 = a.lo[e] | (((g & 1) ? (hb >> 4) : (hb & 15u)) << 8);
   if (a.fmt == kFmtRvq12_4) {
-    const uint32_t sb = a.s2[(int64_t)n * (G / 2) + g / 2];
+    const uint32_t sb = a.s2[e >> 1];
     *i2 = (g & 1) ? (sb >> 4) : (sb & 15u);
   } else {
     *i2 = 0;
@@ -124,13 +125,12 @@ __global__ void debug_unpack_kernel(LayerArgs a, uint16_t* __restrict__ i1o, uin
 template <typename W>
 __global__ void debug_dequant_kernel(LayerArgs a, uint16_t* __restrict__ w) {
   const int G = a.K / 8;
-  const int nblk = a.K / a.scale_group;
   const int64_t total = (int64_t)a.N * G;
   for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < total; t += (int64_t)gridDim.x * blockDim.x) {
     const int n = (int)(t / G), g = (int)(t % G);
     uint32_t i1, i2;
     unpack_one(a, n, g, &i1, &i2);
-    const float s = f16_bits_to_f32(a.scales[(int64_t)n * nblk + (8 * g) / a.scale_group]);
+    const float s = f16_bits_to_f32(a.scales[scale_index(n, 8 * g, a.N, a.K, a.scale_group)]);
     const uint4 c1 = reinterpret_cast<const uint4*>(a.cb1)[i1];
     uint32_t out[4];
     if (a.fmt == kFmtRvq12_4) {

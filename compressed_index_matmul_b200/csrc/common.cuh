@@ -2,10 +2,10 @@
 //
 // Storage format (orka README, "How it works"; GLQ README, "How it works"):
 // W is N x K, one codebook index per group of 8 consecutive weights along K,
-// G = K/8 groups per row.  The 12-bit stage-1 index of group g is
-// lo[n][g] | hi_nibble << 8, where the hi4 byte t holds group 2t in bits 0..3 and
-// group 2t+1 in bits 4..7; the 4-bit stage-2 index comes from the s2 plane packed
-// the same way; the 16-bit format stores one uint16 per group.
+// G = K/8 groups per row.  The 12-bit stage-1 index of a group is its lo byte |
+// its hi nibble << 8 (two groups per hi4 byte, the even group in bits 0..3); the
+// 4-bit stage-2 index comes from the s2 plane packed the same way; the 16-bit
+// format stores one uint16 per group.  The storage order is below.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -24,6 +24,32 @@ constexpr uint32_t kErrTimeout = 1u;
 // Iteration cap for every spin-wait on an mbarrier (each try_wait may suspend
 // the thread for a while, so this bounds the wait to well under a second).
 constexpr uint32_t kWaitSpinLimit = 1u << 22;
+
+// ------------------------------------------------------------------ storage order
+//
+// Index planes are K-slice-major: K is cut into slices of 16 groups (128 inputs);
+// slice s holds w = min(16, G - 16 s) groups, and row n's entries of slice s
+// start at entry 16 s N + n w (entries are bytes of lo, uint16 of idx16; the
+// packed 4-bit planes hi4 / s2 use half of every count, two groups per byte with
+// the even group in the low nibble).  Consecutive output rows are therefore
+// adjacent in memory for every slice, so loads across rows coalesce.
+// Block scales (one per 64 inputs) follow the same order with 2 entries per full
+// slice; one scale per row is scales[n].
+
+__host__ __device__ __forceinline__ int slice_width(int s, int G) { return (G - 16 * s) < 16 ? (G - 16 * s) : 16; }
+
+// Entry index of group g of row n (lo / idx16; halve it for hi4 / s2).
+__device__ __forceinline__ int64_t slice_entry(int n, int g, int N, int G) {
+  const int s = g >> 4;
+  return (int64_t)16 * s * N + (int64_t)n * slice_width(s, G) + (g & 15);
+}
+
+// Index of the scale that covers input k of row n (scale_group is 64 or K).
+__device__ __forceinline__ int64_t scale_index(int n, int k, int N, int K, int scale_group) {
+  if (scale_group == K) return n;
+  const int s = k >> 7;
+  return (int64_t)2 * s * N + (int64_t)n * (slice_width(s, K / 8) >> 3) + ((k & 127) >> 6);
+}
 
 // ------------------------------------------------------------------ element types
 

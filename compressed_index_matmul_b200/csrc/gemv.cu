@@ -52,28 +52,30 @@ struct BlockIdx {
   uint32_t sc;       // two fp16 scales (rows g, g+8)
 };
 
+// Index bytes of one 64-wide k block (8 groups, starting at group gbase) for rows
+// g and g+8 of the lane, plus their scales.
 template <int FMT>
 __device__ __forceinline__ void load_block(const LayerArgs& a, const int rows[2], const bool valid[2], int gbase,
                                            int k, BlockIdx<FMT>& b) {
   const int G = a.K / 8;
-  const int nblk = a.K / a.scale_group;
+  const int s = gbase >> 4, w = slice_width(s, G), o = gbase & 15;  // o is 0 or 8
   uint32_t s16[2] = {0, 0};
 #pragma unroll
   for (int r = 0; r < 2; ++r) {
     b.w[r][0] = b.w[r][1] = b.w[r][2] = b.w[r][3] = 0;
     if (!valid[r]) continue;
-    const int64_t rowoff = (int64_t)rows[r] * G + gbase;
+    const int64_t e = (int64_t)16 * s * a.N + (int64_t)rows[r] * w + o;
     if (FMT == kFmtVq16) {
-      const uint4 v = *reinterpret_cast<const uint4*>(a.idx16 + rowoff);
+      const uint4 v = *reinterpret_cast<const uint4*>(a.idx16 + e);
       b.w[r][0] = v.x; b.w[r][1] = v.y; b.w[r][2] = v.z; b.w[r][3] = v.w;
     } else {
-      const uint2 lo = *reinterpret_cast<const uint2*>(a.lo + rowoff);
+      const uint2 lo = *reinterpret_cast<const uint2*>(a.lo + e);
       b.w[r][0] = lo.x;
       b.w[r][1] = lo.y;
-      b.w[r][2] = *reinterpret_cast<const uint32_t*>(a.hi4 + rowoff / 2);
-      if (FMT == kFmtRvq12_4) b.w[r][3] = *reinterpret_cast<const uint32_t*>(a.s2 + rowoff / 2);
+      b.w[r][2] = *reinterpret_cast<const uint32_t*>(a.hi4 + e / 2);
+      if (FMT == kFmtRvq12_4) b.w[r][3] = *reinterpret_cast<const uint32_t*>(a.s2 + e / 2);
     }
-    s16[r] = a.scales[(int64_t)rows[r] * nblk + k / a.scale_group];
+    s16[r] = a.scales[scale_index(rows[r], k, a.N, a.K, a.scale_group)];
   }
   b.sc = s16[0] | (s16[1] << 16);
 }

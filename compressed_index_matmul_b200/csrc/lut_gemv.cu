@@ -98,9 +98,8 @@ __global__ void __launch_bounds__(kLutThreads, 1)
   int* nlist = reinterpret_cast<int*>(smem + kLutOffRed + 48);
   const uint32_t t1_base = smem_u32(t1), t2_base = smem_u32(t2), ring = smem_u32(smem + kLutOffRing);
 
-  const int K = a.K, G = K / 8, N = a.N;
+  const int N = a.N;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int nblk = K / a.scale_group;
   const bool block_scales = (a.scale_group == 64);
   const int64_t U = (int64_t)S * C;
   const int64_t u0 = U * blockIdx.x / gridDim.x, u1 = U * (blockIdx.x + 1) / gridDim.x;
@@ -110,12 +109,14 @@ __global__ void __launch_bounds__(kLutThreads, 1)
   auto issue = [&](int64_t u) {
     const int s = (int)(u / C), r = (int)(u % C) * kLutThreads + tid;
     if (r < N) {
+      // K-slice-major planes: this row's 16 groups of slice s are adjacent to the
+      // next row's, so the warp's copies are contiguous.
       const uint32_t dst = ring + (((int)((u - u0) % kLutStages)) * kLutThreads + tid) * kLutRecord;
-      const int64_t rowoff = (int64_t)r * G + s * kLutGroups;
-      cp_async16(dst, a.lo + rowoff);
-      cp_async8(dst + 16, a.hi4 + rowoff / 2);
-      if (kTwo) cp_async8(dst + 24, a.s2 + rowoff / 2);
-      if (block_scales) cp_async4(dst + 32, a.scales + (int64_t)r * nblk + 2 * s);
+      const int64_t e = (int64_t)16 * s * N + (int64_t)16 * r;
+      cp_async16(dst, a.lo + e);
+      cp_async8(dst + 16, a.hi4 + e / 2);
+      if (kTwo) cp_async8(dst + 24, a.s2 + e / 2);
+      if (block_scales) cp_async4(dst + 32, a.scales + e / 8);  // 2 scales per row per slice
     }
   };
   for (int i = 0; i < kLutStages - 1; ++i) {

@@ -167,9 +167,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
     const int dr = 32 * q + lane;      // row within the tile == TMEM lane
     const int r = row0 + dr;
     const bool valid = r < N;
-    const int nblk = K / a.scale_group;
     const uint4* cbg = reinterpret_cast<const uint4*>(a.cb1);
-    const int64_t rowoff = (int64_t)(valid ? r : 0) * G;
     struct Rec {
       uint32_t w[4];  // lo (2 words) + hi4 + s2, or idx16 (4 words) of this thread's 4 groups
       uint32_t sc;
@@ -179,16 +177,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
       rc.sc = 0;
       if (!valid || kb >= nkb) return;
       const int g0 = (kbeg / 8) + kb * 8 + 4 * half;  // first of this thread's 4 groups
+      const int s = g0 >> 4;
+      const int64_t e = (int64_t)16 * s * N + (int64_t)r * slice_width(s, G) + (g0 & 15);
       if (FMT == kFmtVq16) {
-        const uint2 v = *reinterpret_cast<const uint2*>(a.idx16 + rowoff + g0);
+        const uint2 v = *reinterpret_cast<const uint2*>(a.idx16 + e);
         rc.w[0] = v.x;
         rc.w[1] = v.y;
       } else {
-        rc.w[0] = *reinterpret_cast<const uint32_t*>(a.lo + rowoff + g0);
-        rc.w[1] = *reinterpret_cast<const uint16_t*>(a.hi4 + rowoff / 2 + g0 / 2);
-        if (kTwo) rc.w[2] = *reinterpret_cast<const uint16_t*>(a.s2 + rowoff / 2 + g0 / 2);
+        rc.w[0] = *reinterpret_cast<const uint32_t*>(a.lo + e);
+        rc.w[1] = *reinterpret_cast<const uint16_t*>(a.hi4 + e / 2);
+        if (kTwo) rc.w[2] = *reinterpret_cast<const uint16_t*>(a.s2 + e / 2);
       }
-      rc.sc = a.scales[(int64_t)r * nblk + (8 * g0) / a.scale_group];
+      rc.sc = a.scales[scale_index(r, 8 * g0, N, K, a.scale_group)];
     };
     bool ok = true;
     Rec rec[kTcAhead];

@@ -16,20 +16,28 @@
  *     compressed indices; partial sums reduced in a fixed order (no atomics), so
  *     results are bit-identical from run to run.
  *
- * Storage format (all arrays row-major, contiguous, no padding; W is N x K,
- * G = K / 8 groups per row; every pointer is a DEVICE pointer unless stated):
- *   lo    uint8  [N][G]     low 8 bits of the 12-bit stage-1 index of each group
- *   hi4   uint8  [N][G/2]   high 4 bits of the stage-1 index: group 2t in bits 0..3,
- *                           group 2t+1 in bits 4..7
- *   s2    uint8  [N][G/2]   4-bit stage-2 index, packed like hi4 (VQ_FMT_RVQ12_4 only)
- *   idx16 uint16 [N][G]     16-bit index (VQ_FMT_VQ16 only), little endian
+ * Storage format (W is N x K, G = K / 8 groups of 8 weights per row; every
+ * pointer is a DEVICE pointer unless stated; no padding anywhere):
+ *   Index planes are K-slice-major.  K is cut into slices of 16 groups (128
+ *   inputs); slice s holds w_s = min(16, G - 16 s) groups.  Inside a slice the
+ *   rows' entries are contiguous, row after row: row n's w_s entries of slice s
+ *   start at entry 16 s N + n w_s.  So for every slice the output rows are
+ *   adjacent, and 128-bit loads by consecutive rows coalesce.
+ *   lo    uint8  [N*G]     low 8 bits of the 12-bit stage-1 index, one entry per group
+ *   hi4   uint8  [N*G/2]   high 4 bits of the stage-1 index, half an entry per group:
+ *                          within a row's slice entries group 2t is in bits 0..3 of
+ *                          byte t and group 2t+1 in bits 4..7
+ *   s2    uint8  [N*G/2]   4-bit stage-2 index, packed like hi4 (VQ_FMT_RVQ12_4 only)
+ *   idx16 uint16 [N*G]     16-bit index, one entry per group (VQ_FMT_VQ16 only)
+ *   scales fp16            scale_group == 64: one per 64 inputs, in the same
+ *                          K-slice-major order (2 entries per row per full slice,
+ *                          1 in a 64-wide last slice); scale_group == K: [N]
  *   cb1   fp16   [4096][8]  stage-1 codebook (or [65536][8] for VQ_FMT_VQ16)
  *   cb2   fp16   [16][8]    stage-2 codebook (VQ_FMT_RVQ12_4 only)
- *   scales fp16  [N][K/scale_group]   scale_group is 64 or K (one scale per row)
- *   x     fp16 or bf16 [M][K]          y  same dtype [M][N]
+ *   x     fp16 or bf16 [M][K] row-major;   y  same dtype [M][N] row-major
  * Weight (n, k) with g = k/8, j = k%8 decodes to
- *   scales[n][k/scale_group] * (cb1[i1(n,g)][j] + cb2[i2(n,g)][j]),
- * with i1 = lo[n][g] | hi_nibble(n,g) << 8 and i2 = s2 nibble (or i1 = idx16[n][g]).
+ *   scale(n, k) * (cb1[i1(n,g)][j] + cb2[i2(n,g)][j]),
+ * with i1 = lo byte | hi nibble << 8 and i2 the s2 nibble (or i1 = idx16 entry).
  *
  * Conventions shared by every entry point:
  *   - Errors: every call returns a vq_status.  Argument problems are detected on
@@ -40,9 +48,10 @@
  *   - Streams: `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *     stream).  Calls only enqueue work on it and never synchronise, except the
  *     ones documented as synchronising.
- *   - Ownership: the caller owns every buffer passed in.  A handle owns host state
- *     and one device scratch buffer (split-K partial sums), allocated by
- *     vq_linear_create and freed by vq_linear_destroy.
+ *   - Ownership: the caller owns every buffer passed in.  A handle owns host state,
+ *     one device scratch buffer (split-K partial sums) and a small device array of
+ *     completion counters (zero between forwards), allocated by vq_linear_create
+ *     and freed by vq_linear_destroy.
  *   - Concurrency: one handle must not run two calls at the same time on different
  *     streams (they share the scratch buffer).  Different handles are independent.
  *   - Alignment: every device pointer must be 16-byte aligned.
@@ -96,10 +105,10 @@ typedef struct {
 } vq_linear_desc;
 
 typedef struct {
-  const uint8_t* lo;     /* [N][K/8]   (RVQ12, RVQ12_4), else NULL */
-  const uint8_t* hi4;    /* [N][K/16]  (RVQ12, RVQ12_4), else NULL */
-  const uint8_t* s2;     /* [N][K/16]  (RVQ12_4), else NULL */
-  const uint16_t* idx16; /* [N][K/8]   (VQ16), else NULL */
+  const uint8_t* lo;     /* N*K/8 bytes, K-slice-major (RVQ12, RVQ12_4), else NULL */
+  const uint8_t* hi4;    /* N*K/16 bytes, K-slice-major (RVQ12, RVQ12_4), else NULL */
+  const uint8_t* s2;     /* N*K/16 bytes, K-slice-major (RVQ12_4), else NULL */
+  const uint16_t* idx16; /* N*K/8 entries, K-slice-major (VQ16), else NULL */
 } vq_planes;
 
 typedef struct {
@@ -133,8 +142,11 @@ vq_status vq_linear_set_path(vq_linear_t h, int32_t path);
  *   N and K must equal the handle's; 0 <= M <= max_M; M == 0 returns VQ_OK
  *   without launching.  Accumulation is fp32; the result is rounded to nearest
  *   even into y.  For a given handle, path and M the result is bit-identical from
- *   run to run (fixed-order reductions, no atomics).
- * Enqueues 1 or 2 kernels on `stream` (see vq_linear_launches) and returns. */
+ *   run to run: split-K partials are summed in a fixed order (an integer atomic
+ *   only picks which CTA does the sum; no floating-point atomics).
+ * Enqueues one kernel on `stream` (see vq_linear_launches) and returns.  The
+ * kernel may start its prologue (reading the constant layer inputs) while the
+ * previous kernel in the stream finishes; it reads x and writes y only after it. */
 vq_status vq_linear_forward(vq_linear_t h, const void* x, const vq_planes* planes,
                             const vq_codebooks* codebooks, const void* scales, void* y,
                             int32_t M, int32_t N, int32_t K, void* stream);
@@ -166,8 +178,8 @@ const char* vq_last_error(void);
 
 /* ---- test and debugging entry points (materialise data into caller buffers) ---- */
 
-/* Unpacked indices: i1_out uint16 [N][K/8] (stage-1 or 16-bit index), i2_out
- * uint8 [N][K/8] (stage-2 index, 0 when the format has none; may be NULL).
+/* Unpacked indices, row-major: i1_out uint16 [N][K/8] (stage-1 or 16-bit index),
+ * i2_out uint8 [N][K/8] (stage-2 index, 0 when the format has none; may be NULL).
  * One kernel launch. */
 vq_status vq_debug_unpack(vq_linear_t h, const vq_planes* planes, uint16_t* i1_out, uint8_t* i2_out,
                           void* stream);

@@ -62,12 +62,3 @@ def assert_y_within(y_bits, dt, y_ref, tol, what=""):
     return float(np.max(err / tol))
 
 
-def sub_layer(layer, rows):
-    """The same layer restricted to the given output rows (rows are independent)."""
-    out = {"spec": type(layer["spec"])(len(rows), layer["spec"].K, layer["spec"].fmt, layer["spec"].scale_group)}
-    for k, v in layer.items():
-        if k in ("lo", "hi4", "s2", "idx16", "scales"):
-            out[k] = np.ascontiguousarray(v[rows])
-        elif k in ("cb1", "cb2"):
-            out[k] = v
-    return out

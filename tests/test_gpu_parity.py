@@ -12,7 +12,7 @@ import torch
 import compressed_index_matmul_b200 as vq
 from synth import (DT_BF16, DT_F16, FMT_RVQ12, FMT_RVQ12_4, FMT_VQ16, CONFIGS, LayerSpec, make_layer, make_signs,
                    make_x)
-from tests.gpu_util import assert_y_within, dev, host_bits, layer_on_gpu, require_gpu, run_forward, sub_layer, widen
+from tests.gpu_util import assert_y_within, dev, host_bits, layer_on_gpu, require_gpu, run_forward, widen
 
 pytestmark = pytest.mark.gpu
 
@@ -232,9 +232,8 @@ def _sampled_forward_check(oracle, layer, act, M, path, nrows=192, seed=0):
     x = make_x(M, spec.K, act, cfg_id=70 + M, seed=seed)
     y = run_forward(L, x, act, path)
     rows = np.sort(np.random.default_rng(seed).choice(spec.N, size=min(nrows, spec.N), replace=False))
-    sub = sub_layer(layer, rows)
-    y_ref = oracle.forward(sub, x, act)
-    w, _ = oracle.dequant(sub)
+    y_ref = oracle.forward(layer, x, act, rows=rows)
+    w, _ = oracle.dequant(layer, rows=rows)
     # max|w| over the whole layer bounds the sampled rows' tolerance from below; use the sample's
     tol = oracle.tolerance(x, act, w, TOL)
     return assert_y_within(y[:, rows], act, y_ref, tol, what=f"{spec} M={M}")
@@ -269,9 +268,8 @@ def test_vq16_rotated_end_to_end(oracle, M):
     torch.cuda.synchronize()
     x_rot = oracle.round_to(oracle.rht(x, DT_F16, signs), DT_F16)
     rows = np.sort(np.random.default_rng(M).choice(spec.N, size=512, replace=False))
-    sub = sub_layer(layer, rows)
-    y_ref = oracle.forward(sub, x_rot, DT_F16)
-    w, _ = oracle.dequant(sub)
+    y_ref = oracle.forward(layer, x_rot, DT_F16, rows=rows)
+    w, _ = oracle.dequant(layer, rows=rows)
     assert_y_within(y[:, rows], DT_F16, y_ref, oracle.tolerance(x_rot, DT_F16, w, TOL), what="cfg3")
 
 

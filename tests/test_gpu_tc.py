@@ -5,7 +5,7 @@ import pytest
 
 import compressed_index_matmul_b200 as vq
 from synth import DT_BF16, DT_F16, FMT_RVQ12, FMT_RVQ12_4, FMT_VQ16, CONFIGS, LayerSpec, make_layer, make_x
-from tests.gpu_util import assert_y_within, layer_on_gpu, require_gpu, run_forward, sub_layer
+from tests.gpu_util import assert_y_within, layer_on_gpu, require_gpu, run_forward
 
 pytestmark = pytest.mark.gpu
 TOL = 2e-3
@@ -56,7 +56,6 @@ def test_prefill_8192_sampled(oracle, M):
     y = run_forward(L, x, DT_BF16, vq.VQ_PATH_AUTO)
     vq.vq_linear_check(L.handle)
     rows = np.sort(np.random.default_rng(M).choice(spec.N, size=96, replace=False))
-    sub = sub_layer(layer, rows)
-    y_ref = oracle.forward(sub, x, DT_BF16)
-    w, _ = oracle.dequant(sub)
+    y_ref = oracle.forward(layer, x, DT_BF16, rows=rows)
+    w, _ = oracle.dequant(layer, rows=rows)
     assert_y_within(y[:, rows], DT_BF16, y_ref, oracle.tolerance(x, DT_BF16, w, TOL), what=f"prefill M={M}")
