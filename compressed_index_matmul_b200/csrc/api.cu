@@ -28,6 +28,7 @@ struct vq_linear_s {
   size_t scratch_bytes;
   uint32_t* tickets;  // completion counters, zeroed at create, left zero by every forward
   int num_tickets;
+  uint32_t* gbar;     // grid-barrier words: arrivals (left zero) and a generation counter
   uint32_t* err;      // device word, set by bounded waits that gave up
 };
 
@@ -205,13 +206,14 @@ VQ_API vq_status vq_linear_create(const vq_linear_desc* desc, vq_linear_t* out) 
     }
   }
   h->num_tickets = tickets;
-  const size_t small = sizeof(uint32_t) * (size_t)(1 + tickets);
+  const size_t small = sizeof(uint32_t) * (size_t)(3 + tickets);
   uint32_t* words = nullptr;
   e = cudaMalloc(&words, small);
   if (e == cudaSuccess) e = cudaMemset(words, 0, small);
   if (e == cudaSuccess) e = cudaDeviceSynchronize();  // the zeroing is complete before any forward
   h->err = words;
-  h->tickets = tickets ? words + 1 : nullptr;
+  h->gbar = words + 1;
+  h->tickets = tickets ? words + 3 : nullptr;
   if (e != cudaSuccess) {
     cudaFree(h->scratch);
     cudaFree(words);
@@ -227,7 +229,7 @@ VQ_API vq_status vq_linear_destroy(vq_linear_t h) {
   if (h == nullptr) return VQ_OK;
   cudaError_t e1 = cudaSuccess, e2 = cudaSuccess;
   if (h->scratch) e1 = cudaFree(h->scratch);
-  if (h->err) e2 = cudaFree(h->err);  // also frees the tickets (one allocation)
+  if (h->err) e2 = cudaFree(h->err);  // also frees the barrier words and tickets (one allocation)
   delete h;
   if (e1 != cudaSuccess) return cuda_fail(e1, "cudaFree(scratch)");
   if (e2 != cudaSuccess) return cuda_fail(e2, "cudaFree(err)");
@@ -277,7 +279,7 @@ VQ_API vq_status vq_linear_forward(vq_linear_t h, const void* x, const vq_planes
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e;
   switch (p.path) {
-    case VQ_PATH_LUT: e = vq::launch_lut(a, p, h->scratch, h->tickets, s); break;
+    case VQ_PATH_LUT: e = vq::launch_lut(a, p, h->scratch, h->gbar, h->err, s); break;
     case VQ_PATH_TC: e = vq::launch_tc(a, p, h->scratch, h->tickets, h->err, s); break;
     default: e = vq::launch_gemv(a, p, h->scratch, h->tickets, s); break;
   }

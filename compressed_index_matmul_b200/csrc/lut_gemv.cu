@@ -1,4 +1,5 @@
-// Batch-1 GEMV by per-group lookup tables (M == 1, 12-bit formats, K % 128 == 0).
+// Batch-1 GEMV by per-group lookup tables (M == 1, 12-bit formats, K % 128 == 0,
+// N % 4 == 0).
 //
 // For one token x and one group g of 8 inputs, every weight group of row n
 // contributes s * (x_g . cb1[i1] + x_g . cb2[i2]) (orka README, "How it works":
@@ -13,37 +14,46 @@
 // those MMAs does not depend on x, so each warp loads its share of it into
 // registers once and every rebuild is only MMAs and stores.
 //
-// Work distribution: units are (K-slice s, 256-row chunk c) in slice-major order;
-// a persistent grid of one CTA per SM takes a contiguous run of units.  Thread t
-// handles row t of every unit; its rows' index bytes stream through a private
-// ring of cp.async stages in shared memory, several units ahead, so the loop
-// never waits on DRAM latency.  Each unit writes an fp32 partial sum per row.
-// When a CTA has finished all its units it takes one ticket per unit; the CTA
-// that completes a chunk's last slice sums that chunk's partials in increasing
-// slice order (GLQ README, "Inference kernels": fixed-order split-K reduction, no
-// floating-point atomics) and writes y.  One launch per forward.
+// Work distribution: units are (K-slice s, 512-row chunk) in slice-major order;
+// a persistent grid of at most one CTA per SM takes a contiguous run of units.
+// In the K-slice-major storage a unit's index bytes are one contiguous run per
+// plane, so one thread streams them into a ring of shared-memory stages with
+// bulk copies (TMA), several units ahead.  Thread t handles rows t and t+256 of
+// a unit and writes one fp32 partial sum per row and slice.
 //
-// Activations are scaled by a power of two per slice so that every value fits the
-// fp16 MMA whatever the activation type; the partial sum is scaled back exactly.
+// Split-K reduction: after the last unit every CTA meets at a grid-wide barrier
+// (all CTAs are resident: the grid never exceeds the SM count and a CTA takes a
+// whole SM's shared memory); then each CTA sums the partials of its own share
+// of the rows with a fixed tree (GLQ README, "Inference kernels": fixed-order
+// split-K reduction, no floating-point atomics), so y does not depend on
+// scheduling.  One launch per forward.
+//
+// Activations are scaled by a power of two per group of 8 so that every value
+// fits the fp16 MMA whatever the activation type; the table entries are scaled
+// back exactly before they are stored.
 #include "common.cuh"
 #include "internal.h"
+#include "tc_ptx.cuh"
 
 namespace vq {
 
 constexpr int kLutGroups = 16;                 // groups per K-slice (128 inputs)
-constexpr int kLutThreads = 256;               // one row per thread per unit
+constexpr int kLutThreads = 256;
+constexpr int kLutUnitRows = 512;              // rows per unit (two per thread)
 constexpr int kLutTableBytes = 4096 * 2 + 64;  // one group's T1 (bf16) + pad (bank spread)
-constexpr int kLutStages = 6;                  // cp.async ring depth (units in flight)
-constexpr int kLutRecord = 48;                 // bytes per thread per stage: lo16 hi8 s2 8 scales4 pad
+constexpr int kLutStages = 4;                  // bulk-copy ring depth (units in flight)
 constexpr int kLutMaxX = 4;                    // x slices preloaded per CTA
+// one ring stage: lo 16 B, hi4 8 B, s2 8 B, scales 4 B per row
+constexpr int kLutOffHi = kLutUnitRows * 16;
+constexpr int kLutOffS2 = kLutOffHi + kLutUnitRows * 8;
+constexpr int kLutOffSc = kLutOffS2 + kLutUnitRows * 8;
+constexpr int kLutStageBytes = kLutOffSc + kLutUnitRows * 4;
 constexpr int kLutOffT2 = kLutGroups * kLutTableBytes;
 constexpr int kLutOffXh = kLutOffT2 + kLutGroups * 16 * 4;
 constexpr int kLutOffXf = kLutOffXh + kLutGroups * 8 * 2;
-constexpr int kLutOffRed = kLutOffXf + kLutGroups * 8 * 4;
-constexpr int kLutOffList = kLutOffRed + 64;
-constexpr int kLutMaxList = 256;
-constexpr int kLutOffRing = kLutOffList + 4 * kLutMaxList + 16;
-constexpr int kLutSmem = kLutOffRing + kLutStages * kLutThreads * kLutRecord;
+constexpr int kLutOffMisc = kLutOffXf + kLutGroups * 8 * 4;  // per-group scales, barriers
+constexpr int kLutOffRing = kLutOffMisc + 256;
+constexpr int kLutSmem = kLutOffRing + kLutStages * kLutStageBytes;
 
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   uint32_t r;
@@ -69,34 +79,52 @@ __device__ __forceinline__ float lds_f32(uint32_t addr) {
   return v;
 }
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async8(uint32_t dst, const void* src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+// Sum of the 16 lookups of one row's slice record (lo 16 B, hi4 8 B, s2 8 B),
+// split by 64-input block.
+template <bool kTwo>
+__device__ __forceinline__ void lookup_row(const uint4& lo4, const uint2& h, const uint2& q, uint32_t t1_base,
+                                           uint32_t t2_base, float blk[2]) {
+  const uint32_t low[4] = {lo4.x, lo4.y, lo4.z, lo4.w};
+  const uint32_t hiw[2] = {h.x, h.y};
+  const uint32_t s2w[2] = {q.x, q.y};
+  blk[0] = blk[1] = 0.f;
+#pragma unroll
+  for (int w = 0; w < 2; ++w) {
+    const uint32_t hE = hiw[w] & 0x0F0F0F0Fu, hO = (hiw[w] >> 4) & 0x0F0F0F0Fu;
+    const uint32_t sE = (s2w[w] & 0x0F0F0F0Fu) << 2, sO = ((s2w[w] >> 4) & 0x0F0F0F0Fu) << 2;
+#pragma unroll
+    for (int qq = 0; qq < 8; ++qq) {
+      const int t = 8 * w + qq;  // group within the slice
+      const uint32_t hsel = 4 + (qq >> 1);
+      // bytes: lo byte t, hi nibble t, then two zero bytes (sign copies of a nibble byte)
+      const uint32_t sel = (uint32_t)(t & 3) | (hsel << 4) | ((8u | hsel) << 8) | ((8u | hsel) << 12);
+      const uint32_t i1 = prmt(low[t >> 2], (qq & 1) ? hO : hE, sel);
+      float v = lds_bf16(t1_base + t * kLutTableBytes + i1 * 2);
+      if (kTwo) {
+        const uint32_t b = qq >> 1;
+        const uint32_t bsel = b | ((8u | b) << 4) | ((8u | b) << 8) | ((8u | b) << 12);
+        v += lds_f32(t2_base + t * 64 + prmt((qq & 1) ? sO : sE, 0, bsel));
+      }
+      blk[w] += v;
+    }
+  }
 }
 
 template <int FMT, typename T>
 __global__ void __launch_bounds__(kLutThreads, 1)
-    lut_gemv_kernel(LayerArgs a, float* __restrict__ partial, uint32_t* __restrict__ tickets, int S, int C) {
+    lut_gemv_kernel(LayerArgs a, float* __restrict__ partial, uint32_t* __restrict__ gbar, uint32_t* __restrict__ err,
+                    int S, int C) {
   extern __shared__ __align__(128) unsigned char smem[];
   constexpr bool kTwo = (FMT == kFmtRvq12_4);
   unsigned char* t1 = smem;
   float* t2 = reinterpret_cast<float*>(smem + kLutOffT2);
   uint32_t* xh = reinterpret_cast<uint32_t*>(smem + kLutOffXh);
   float* xf = reinterpret_cast<float*>(smem + kLutOffXf);
-  float* red = reinterpret_cast<float*>(smem + kLutOffRed);
-  int* list = reinterpret_cast<int*>(smem + kLutOffList);
-  int* nlist = reinterpret_cast<int*>(smem + kLutOffRed + 48);
-  const uint32_t t1_base = smem_u32(t1), t2_base = smem_u32(t2), ring = smem_u32(smem + kLutOffRing);
+  float* gsc = reinterpret_cast<float*>(smem + kLutOffMisc);        // [16] per-group 2^-e
+  const uint32_t bars = smem_u32(smem + kLutOffMisc + 64);          // [kLutStages] mbarriers
+  volatile int* flag = reinterpret_cast<volatile int*>(smem + kLutOffMisc + 128);
+  unsigned char* ring = smem + kLutOffRing;
+  const uint32_t t1_base = smem_u32(t1), t2_base = smem_u32(t2), ring_base = smem_u32(ring);
 
   const int N = a.N;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -105,23 +133,24 @@ __global__ void __launch_bounds__(kLutThreads, 1)
   const int64_t u0 = U * blockIdx.x / gridDim.x, u1 = U * (blockIdx.x + 1) / gridDim.x;
   const uint16_t* xg = static_cast<const uint16_t*>(a.x);
 
-  // Row records for unit u go to stage (u - u0) % kLutStages of this thread's ring.
+  // Unit u's bytes: one bulk copy per plane into stage (u - u0) % kLutStages.
   auto issue = [&](int64_t u) {
-    const int s = (int)(u / C), r = (int)(u % C) * kLutThreads + tid;
-    if (r < N) {
-      // K-slice-major planes: this row's 16 groups of slice s are adjacent to the
-      // next row's, so the warp's copies are contiguous.
-      const uint32_t dst = ring + (((int)((u - u0) % kLutStages)) * kLutThreads + tid) * kLutRecord;
-      const int64_t e = (int64_t)16 * s * N + (int64_t)16 * r;
-      cp_async16(dst, a.lo + e);
-      cp_async8(dst + 16, a.hi4 + e / 2);
-      if (kTwo) cp_async8(dst + 24, a.s2 + e / 2);
-      if (block_scales) cp_async4(dst + 32, a.scales + e / 8);  // 2 scales per row per slice
-    }
+    const int s = (int)(u / C), ch = (int)(u % C);
+    const int r0 = ch * kLutUnitRows, rows = min(kLutUnitRows, N - r0);
+    const int st = (int)((u - u0) % kLutStages);
+    const uint32_t dst = ring_base + st * kLutStageBytes, bar = bars + 8 * st;
+    const int64_t e = (int64_t)16 * s * N + (int64_t)16 * r0;  // lo entry of (slice s, row r0)
+    ptx::mbar_arrive_expect_tx(bar, rows * (16 + 8 + (kTwo ? 8 : 0) + (block_scales ? 4 : 0)));
+    ptx::bulk_load(dst, a.lo + e, rows * 16, bar);
+    ptx::bulk_load(dst + kLutOffHi, a.hi4 + e / 2, rows * 8, bar);
+    if (kTwo) ptx::bulk_load(dst + kLutOffS2, a.s2 + e / 2, rows * 8, bar);
+    if (block_scales) ptx::bulk_load(dst + kLutOffSc, a.scales + e / 8, rows * 4, bar);  // 2 per row per slice
   };
-  for (int i = 0; i < kLutStages - 1; ++i) {
-    if (u0 + i < u1) issue(u0 + i);
-    cp_async_commit();
+  if (tid == 0) {
+    for (int i = 0; i < kLutStages; ++i) ptx::mbar_init(bars + 8 * i, 1);
+    ptx::fence_barrier_init();
+    for (int i = 0; i < kLutStages; ++i)
+      if (u0 + i < u1) issue(u0 + i);
   }
 
   // Codebook operand of the table MMAs, held for the whole kernel: warp w covers
@@ -147,10 +176,10 @@ __global__ void __launch_bounds__(kLutThreads, 1)
       c2v[2 * p + 1] = v.y;
     }
   }
-  // Everything above reads only the layer's constant inputs; x, y and the scratch
-  // are touched only after the previous kernel in the stream has completed.
+  // Everything above reads only the layer's constant inputs; x, y, the scratch
+  // and the barrier words are touched only after the previous kernel completed.
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  // x of the first kLutMaxX slices this CTA touches.
+  const uint32_t gen0 = *reinterpret_cast<volatile uint32_t*>(gbar + 1);  // barrier generation of this launch
   const int s_first = (int)(u0 / C);
   float xpre[kLutMaxX];
 #pragma unroll
@@ -158,13 +187,13 @@ __global__ void __launch_bounds__(kLutThreads, 1)
     const int s = s_first + i;
     xpre[i] = (tid < 128 && s < S) ? Elt<T>::to_f32(xg[(int64_t)s * 128 + tid]) : 0.f;
   }
+  __syncthreads();  // barrier init is visible to every waiting thread
 
   int cur = -1;
-  float inv_xscale = 1.f;
+  bool ok = true;
   for (int64_t u = u0; u < u1; ++u) {
     const int s = (int)(u / C), ch = (int)(u % C);
-    if (u + kLutStages - 1 < u1) issue(u + kLutStages - 1);
-    cp_async_commit();
+    const int st = (int)((u - u0) % kLutStages);
     if (s != cur) {
       // ------------------------------------------------------------ build
       __syncthreads();  // everyone is done with the previous tables
@@ -179,23 +208,20 @@ __global__ void __launch_bounds__(kLutThreads, 1)
           xv = Elt<T>::to_f32(xg[(int64_t)s * 128 + tid]);
         }
       }
+      // Per group of 8 inputs, a power-of-two scale 2^e puts the group's largest |x|
+      // in [2^14, 2^15), so the fp16 MMA operand is exact for any activation type;
+      // the table entries are multiplied by 2^-e before they are stored (exact).
       float m = fabsf(xv);
-      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-      if (lane == 0) red[warp] = m;
-      __syncthreads();
-      m = red[0];
-#pragma unroll
-      for (int w = 1; w < kLutThreads / 32; ++w) m = fmaxf(m, red[w]);
+      for (int o = 4; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
       int e = 0;
       if (m > 0.f && isfinite(m)) {
-        frexpf(m, &e);  // m in [2^(e-1), 2^e): scale the slice's max into [2^14, 2^15)
+        frexpf(m, &e);  // m in [2^(e-1), 2^e)
         e = min(100, max(-100, 15 - e));
       }
-      const float xs = ldexpf(1.f, e);
-      inv_xscale = ldexpf(1.f, -e);
       if (tid < 128) {
-        xf[tid] = xv * xs;
-        reinterpret_cast<__half*>(xh)[tid] = __float2half_rn(xv * xs);
+        xf[tid] = xv;
+        reinterpret_cast<__half*>(xh)[tid] = __float2half_rn(xv * ldexpf(1.f, e));
+        if ((tid & 7) == 0) gsc[tid >> 3] = ldexpf(1.f, -e);
       }
       __syncthreads();
       if (kTwo) {
@@ -203,13 +229,14 @@ __global__ void __launch_bounds__(kLutThreads, 1)
         float acc = 0.f;
 #pragma unroll
         for (int d = 0; d < 8; ++d) acc = fmaf(xf[8 * gg + d], c2v[d], acc);
-        t2[tid] = acc;  // T2[gg][tid & 15]
+        t2[tid] = acc;  // T2[gg][tid & 15], from the unscaled x
       }
       {
         // A = x slice (16 groups x 8 dims, fp16).  Column n of MMA j in block `it`
         // is codeword base + 8*(n/2) + 2j + (n%2), so lane (g, c) ends with
         // codewords base+8c .. base+8c+7 of groups g and g+8: one 16-byte store each.
         const uint32_t a0 = xh[g * 4 + c], a1 = xh[(g + 8) * 4 + c];
+        const float ua = gsc[g], ub = gsc[g + 8];  // undo the groups' power-of-two scales
 #pragma unroll
         for (int it = 0; it < 16; ++it) {
           const int base = warp * 512 + it * 32;
@@ -220,10 +247,10 @@ __global__ void __launch_bounds__(kLutThreads, 1)
             mma_16808_f16(d[j], a0, a1, bfrag[it][j]);
           }
           typedef Elt<__nv_bfloat16> B16;
-          const uint4 lo = make_uint4(B16::pack(d[0][0], d[0][1]), B16::pack(d[1][0], d[1][1]),
-                                      B16::pack(d[2][0], d[2][1]), B16::pack(d[3][0], d[3][1]));
-          const uint4 hi = make_uint4(B16::pack(d[0][2], d[0][3]), B16::pack(d[1][2], d[1][3]),
-                                      B16::pack(d[2][2], d[2][3]), B16::pack(d[3][2], d[3][3]));
+          const uint4 lo = make_uint4(B16::pack(d[0][0] * ua, d[0][1] * ua), B16::pack(d[1][0] * ua, d[1][1] * ua),
+                                      B16::pack(d[2][0] * ua, d[2][1] * ua), B16::pack(d[3][0] * ua, d[3][1] * ua));
+          const uint4 hi = make_uint4(B16::pack(d[0][2] * ub, d[0][3] * ub), B16::pack(d[1][2] * ub, d[1][3] * ub),
+                                      B16::pack(d[2][2] * ub, d[2][3] * ub), B16::pack(d[3][2] * ub, d[3][3] * ub));
           *reinterpret_cast<uint4*>(t1 + g * kLutTableBytes + (base + 8 * c) * 2) = lo;
           *reinterpret_cast<uint4*>(t1 + (g + 8) * kLutTableBytes + (base + 8 * c) * 2) = hi;
         }
@@ -233,43 +260,24 @@ __global__ void __launch_bounds__(kLutThreads, 1)
     }
 
     // -------------------------------------------------------------- lookups
-    cp_async_wait<kLutStages - 1>();  // this thread's records for unit u have landed
-    const int r = ch * kLutThreads + tid;
-    if (r < N) {
-      const uint32_t rec = ring + (((int)((u - u0) % kLutStages)) * kLutThreads + tid) * kLutRecord;
-      uint4 lo4, hs;
+    if (!ptx::mbar_wait(bars + 8 * st, (uint32_t)(((u - u0) / kLutStages) & 1), err)) ok = false;
+    const int r0 = ch * kLutUnitRows;
+    const uint32_t sb = ring_base + st * kLutStageBytes;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int lr = tid + 256 * h, r = r0 + lr;
+      if (r >= N) continue;
+      uint4 lo4;
+      uint2 hh, qq = make_uint2(0, 0);
       uint32_t scw = 0;
       asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
                    : "=r"(lo4.x), "=r"(lo4.y), "=r"(lo4.z), "=r"(lo4.w)
-                   : "r"(rec));
-      asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
-                   : "=r"(hs.x), "=r"(hs.y), "=r"(hs.z), "=r"(hs.w)
-                   : "r"(rec + 16));
-      if (block_scales) asm volatile("ld.shared.u32 %0, [%1];" : "=r"(scw) : "r"(rec + 32));
-      const uint32_t low[4] = {lo4.x, lo4.y, lo4.z, lo4.w};
-      const uint32_t hiw[2] = {hs.x, hs.y};
-      const uint32_t s2w[2] = {hs.z, hs.w};
-      float blk[2] = {0.f, 0.f};
-#pragma unroll
-      for (int w = 0; w < 2; ++w) {
-        const uint32_t hE = hiw[w] & 0x0F0F0F0Fu, hO = (hiw[w] >> 4) & 0x0F0F0F0Fu;
-        const uint32_t sE = (s2w[w] & 0x0F0F0F0Fu) << 2, sO = ((s2w[w] >> 4) & 0x0F0F0F0Fu) << 2;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const int t = 8 * w + q;  // group within the slice
-          const uint32_t hsel = 4 + (q >> 1);
-          // bytes: lo byte t, hi nibble t, then two zero bytes (sign copies of a nibble byte)
-          const uint32_t sel = (uint32_t)(t & 3) | (hsel << 4) | ((8u | hsel) << 8) | ((8u | hsel) << 12);
-          const uint32_t i1 = prmt(low[t >> 2], (q & 1) ? hO : hE, sel);
-          float v = lds_bf16(t1_base + t * kLutTableBytes + i1 * 2);
-          if (kTwo) {
-            const uint32_t b = q >> 1;
-            const uint32_t bsel = b | ((8u | b) << 4) | ((8u | b) << 8) | ((8u | b) << 12);
-            v += lds_f32(t2_base + t * 64 + prmt((q & 1) ? sO : sE, 0, bsel));
-          }
-          blk[w] += v;
-        }
-      }
+                   : "r"(sb + 16 * lr));
+      asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(hh.x), "=r"(hh.y) : "r"(sb + kLutOffHi + 8 * lr));
+      if (kTwo) asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(qq.x), "=r"(qq.y) : "r"(sb + kLutOffS2 + 8 * lr));
+      if (block_scales) asm volatile("ld.shared.u32 %0, [%1];" : "=r"(scw) : "r"(sb + kLutOffSc + 4 * lr));
+      float blk[2];
+      lookup_row<kTwo>(lo4, hh, qq, t1_base, t2_base, blk);
       float acc;
       if (block_scales) {
         const float2 sc = f16x2_to_f32x2(scw);
@@ -277,7 +285,6 @@ __global__ void __launch_bounds__(kLutThreads, 1)
       } else {
         acc = blk[0] + blk[1];  // the per-row scale is applied once, at the reduction
       }
-      acc *= inv_xscale;
       if (S == 1) {
         if (!block_scales) acc *= f16_bits_to_f32(a.scales[r]);
         static_cast<uint16_t*>(a.y)[r] = Elt<T>::from_f32(acc);
@@ -285,45 +292,71 @@ __global__ void __launch_bounds__(kLutThreads, 1)
         partial[(int64_t)s * N + r] = acc;
       }
     }
+    __syncthreads();  // stage `st` is free again
+    if (tid == 0 && u + kLutStages < u1) issue(u + kLutStages);
   }
-  cp_async_wait<0>();
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  if (S == 1) return;
+  if (S == 1) {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    return;
+  }
 
-  // ------------------------------------------------------ fixed-order reduce
-  // One ticket per unit, all taken at once (thread i takes unit u0 + i).
+  // --------------------------------------------------- grid barrier + reduce
   __threadfence();
-  if (tid == 0) *nlist = 0;
   __syncthreads();
-  if (tid < u1 - u0) {
-    const int ch = (int)((u0 + tid) % C);
-    if (atomicAdd(&tickets[ch], 1u) == (uint32_t)(S - 1)) list[atomicAdd(nlist, 1)] = ch;
-  }
-  __syncthreads();
-  const int n = *nlist;
-  if (n == 0) return;
-  __threadfence();
-  // Rows of the completed chunks; every split's partial of a row is loaded before
-  // the sum, which then runs in increasing split order.
-  constexpr int kBatch = 16;
-  for (int i = tid; i < n * kLutThreads; i += kLutThreads) {
-    const int ch = list[i / kLutThreads];
-    const int r = ch * kLutThreads + i % kLutThreads;
-    if (r >= N) continue;
-    float sum = 0.f;
-    for (int k0 = 0; k0 < S; k0 += kBatch) {
-      float v[kBatch];
-#pragma unroll
-      for (int j = 0; j < kBatch; ++j) v[j] = (k0 + j < S) ? __ldcg(partial + (int64_t)(k0 + j) * N + r) : 0.f;
-#pragma unroll
-      for (int j = 0; j < kBatch; ++j)
-        if (k0 + j < S) sum += v[j];
+  if (tid == 0) {
+    const uint32_t arrived = atomicAdd(gbar, 1u);
+    if (arrived == gridDim.x - 1) {
+      *reinterpret_cast<volatile uint32_t*>(gbar) = 0u;  // ready for the next forward
+      __threadfence();
+      atomicAdd(gbar + 1, 1u);                           // release this generation
+    } else {
+      const uint64_t t0 = ptx::globaltimer_ns();
+      bool released = false;
+      for (uint32_t i = 0; i < kWaitSpinLimit; ++i) {
+        if (*reinterpret_cast<volatile uint32_t*>(gbar + 1) != gen0) {
+          released = true;
+          break;
+        }
+        if ((i & 255u) == 255u && ptx::globaltimer_ns() - t0 > 1000000000ull) break;
+        __nanosleep(64);
+      }
+      if (!released) atomicOr(err, kErrTimeout);
     }
-    if (!block_scales) sum *= f16_bits_to_f32(a.scales[r]);
-    static_cast<uint16_t*>(a.y)[r] = Elt<T>::from_f32(sum);
+    *flag = ok;
   }
   __syncthreads();
-  if (tid < n) tickets[list[tid]] = 0u;  // ready for the next forward
+  __threadfence();
+  // This CTA's rows; tpr threads per row split the slices, then a fixed xor tree.
+  const int rbeg = (int)((int64_t)N * blockIdx.x / gridDim.x), rend = (int)((int64_t)N * (blockIdx.x + 1) / gridDim.x);
+  const int nr = rend - rbeg;
+  int tpr = 1;
+  while (tpr < 32 && tpr * 2 * nr <= kLutThreads) tpr *= 2;
+  const int per = (S + tpr - 1) / tpr;
+  for (int base = 0; base < nr * tpr; base += kLutThreads) {
+    const int idx = base + tid;
+    const int row = idx / tpr, part = idx % tpr;
+    float sum = 0.f;
+    if (row < nr) {
+      const int r = rbeg + row;
+      const int k0 = part * per, k1 = min(S, k0 + per);
+      constexpr int kBatch = 16;
+      for (int kb = k0; kb < k1; kb += kBatch) {
+        float v[kBatch];
+#pragma unroll
+        for (int j = 0; j < kBatch; ++j) v[j] = (kb + j < k1) ? __ldcg(partial + (int64_t)(kb + j) * N + r) : 0.f;
+#pragma unroll
+        for (int j = 0; j < kBatch; ++j)
+          if (kb + j < k1) sum += v[j];
+      }
+    }
+    for (int o = 1; o < tpr; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    if (row < nr && part == 0) {
+      const int r = rbeg + row;
+      if (!block_scales) sum *= f16_bits_to_f32(a.scales[r]);
+      static_cast<uint16_t*>(a.y)[r] = Elt<T>::from_f32(sum);
+    }
+  }
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 struct LutGeom {
@@ -333,28 +366,27 @@ struct LutGeom {
 static LutGeom lut_geom(int N, int K, int num_sms) {
   LutGeom g;
   g.S = K / (8 * kLutGroups);
-  g.C = (N + kLutThreads - 1) / kLutThreads;
+  g.C = (N + kLutUnitRows - 1) / kLutUnitRows;
   const int64_t U = (int64_t)g.S * g.C;
   g.grid = (int)(U < num_sms ? U : num_sms);
   return g;
 }
 
 bool plan_lut(const vq_linear_desc& d, const DeviceInfo& dev, int M, Plan* p) {
-  if (M != 1 || d.fmt == VQ_FMT_VQ16 || d.K % (8 * kLutGroups) != 0 || dev.smem_optin < kLutSmem) return false;
+  if (M != 1 || d.fmt == VQ_FMT_VQ16 || d.K % (8 * kLutGroups) != 0 || d.N % 4 != 0 || dev.smem_optin < kLutSmem)
+    return false;
   const LutGeom g = lut_geom(d.N, d.K, dev.num_sms);
-  // Every CTA's units fit its completion list (units per CTA <= kLutMaxList).
-  if (((int64_t)g.S * g.C + g.grid - 1) / g.grid > kLutMaxList) return false;
   p->path = VQ_PATH_LUT;
   p->splits = g.S;
   p->k_per_split = kLutGroups * 8;
   p->launches = 1;
   p->scratch_bytes = g.S > 1 ? (size_t)g.S * d.N * sizeof(float) : 0;
-  p->tickets = g.S > 1 ? g.C : 0;
+  p->tickets = 0;  // uses the handle's grid-barrier words instead
   return true;
 }
 
 template <int FMT, typename T>
-static cudaError_t launch_lut_t(const LayerArgs& a, float* scratch, uint32_t* tickets, cudaStream_t s) {
+static cudaError_t launch_lut_t(const LayerArgs& a, float* scratch, uint32_t* tickets, uint32_t* err, cudaStream_t s) {
   int dev = 0, sms = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -372,15 +404,16 @@ static cudaError_t launch_lut_t(const LayerArgs& a, float* scratch, uint32_t* ti
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, a, g.S > 1 ? scratch : nullptr, g.S > 1 ? tickets : nullptr, g.S, g.C);
+  return cudaLaunchKernelEx(&cfg, kern, a, g.S > 1 ? scratch : nullptr, tickets, err, g.S, g.C);
 }
 
-cudaError_t launch_lut(const LayerArgs& a, const Plan&, float* scratch, uint32_t* tickets, cudaStream_t s) {
+cudaError_t launch_lut(const LayerArgs& a, const Plan&, float* scratch, uint32_t* gbar, uint32_t* err,
+                       cudaStream_t s) {
   if (a.fmt == kFmtRvq12_4)
-    return a.act == VQ_BF16 ? launch_lut_t<kFmtRvq12_4, __nv_bfloat16>(a, scratch, tickets, s)
-                            : launch_lut_t<kFmtRvq12_4, __half>(a, scratch, tickets, s);
-  return a.act == VQ_BF16 ? launch_lut_t<kFmtRvq12, __nv_bfloat16>(a, scratch, tickets, s)
-                          : launch_lut_t<kFmtRvq12, __half>(a, scratch, tickets, s);
+    return a.act == VQ_BF16 ? launch_lut_t<kFmtRvq12_4, __nv_bfloat16>(a, scratch, gbar, err, s)
+                            : launch_lut_t<kFmtRvq12_4, __half>(a, scratch, gbar, err, s);
+  return a.act == VQ_BF16 ? launch_lut_t<kFmtRvq12, __nv_bfloat16>(a, scratch, gbar, err, s)
+                          : launch_lut_t<kFmtRvq12, __half>(a, scratch, gbar, err, s);
 }
 
 }  // namespace vq

@@ -58,4 +58,5 @@ def test_prefill_8192_sampled(oracle, M):
     rows = np.sort(np.random.default_rng(M).choice(spec.N, size=96, replace=False))
     y_ref = oracle.forward(layer, x, DT_BF16, rows=rows)
     w, _ = oracle.dequant(layer, rows=rows)
-    assert_y_within(y[:, rows], DT_BF16, y_ref, oracle.tolerance(x, DT_BF16, w, TOL), what=f"prefill M={M}")
+    assert_y_within(y[:, rows], DT_BF16, y_ref, oracle.tolerance(x, DT_BF16, w, TOL), what=f"prefill M={M}",
+                    strict=True)
