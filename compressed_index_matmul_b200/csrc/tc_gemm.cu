@@ -1,26 +1,33 @@
 // Tensor-core path: y = x . W^T for any M (meant for M >= 17, e.g. prefill),
-// with W decoded tile by tile into shared memory and multiplied on the 5th-gen
-// tensor cores (tcgen05.mma, fp32 accumulator in TMEM).  The dense W never
-// reaches device memory (GLQ README, "Inference kernels"; decode per the orka
-// README, "How it works": scale x sum over stages of codebook[index]).
+// with W decoded tile by tile into tensor memory and multiplied on the 5th-gen
+// tensor cores (tcgen05.mma, A from TMEM, B from shared memory, fp32 accumulator
+// in TMEM).  The dense W never reaches device memory (GLQ README, "Inference
+// kernels"; decode per the orka README, "How it works": scale x sum over stages
+// of codebook[index]).
 //
 // One CTA computes a 128-row x T-token tile of y over one K-split:
-//   warp 0    TMA producer: x tiles (T tokens x 64 k, 128-byte swizzle) into a
-//             3-stage ring; it also bulk-copies the 12-bit codebooks into shared
-//             memory once.
-//   warp 1    allocates TMEM; lane 0 issues tcgen05.mma (M=128, N=T, K=16, four
-//             per 64-wide k block) and commits each stage back to the producers.
-//   warps 2-9 decode: two warps per TMEM lane quarter; thread = one row of the
-//             tile (= its TMEM lane) and one half (4 groups) of each 64-wide k
-//             block.  It unpacks, gathers the codewords, scales, rounds to the
-//             activation type and stores 16-byte chunks into the stage's A tile in
-//             the same 128-byte-swizzled K-major layout the TMA uses for x.  Its
-//             index bytes are loaded four blocks ahead into registers.  After the
-//             last block the same threads read the accumulator from TMEM and write
-//             y (or fp32 split-K partials; the last CTA of a tile, by an atomic
-//             ticket, sums the partials in split order).
+//   warp 0     producer: bulk-copies the 12-bit codebook into shared memory once;
+//              per 128-input slice, bulk-copies the tile's index bytes (the
+//              K-slice-major planes make them one contiguous run per plane) into
+//              a 4-slot ring; per 64-wide k block, TMA-loads the x tile (T tokens
+//              x 64, 128-byte swizzle) into a 4-stage ring.
+//   warp 1     allocates TMEM; lane 0 issues tcgen05.mma (M=128, N=T, K=16, four
+//              per k block, A read from TMEM) and commits each stage back.
+//   warps 2-17 decode: four warps per TMEM lane quarter; thread = one row of the
+//              tile (its TMEM lane) and two of the 8 groups of each k block.  Once
+//              per slice it reads its row's index bytes from the staged slice;
+//              per k block it gathers the stage-1 codeword from shared memory and
+//              the stage-2 codeword from the warp's registers (shuffle), decodes
+//              with the materialised-weight rounding and stores the 16 weights
+//              into its own TMEM lane of the stage's A columns (tcgen05.st).
+//              After the last block the same threads read the accumulator from
+//              TMEM and write y (or fp32 split-K partials; the last CTA of a tile,
+//              by an atomic ticket, sums the partials in split order).
 // Every mbarrier wait is bounded; a timeout sets the handle's error word and the
 // CTA winds down (waits for its own copies, frees TMEM) instead of hanging.
+// When N % 8 != 0 the per-slice index runs are not all 16-byte multiples, so
+// bulk copies cannot stage them: the decode threads read their index bytes from
+// global memory instead.
 #include <cuda.h>
 
 #include <type_traits>
@@ -32,65 +39,125 @@
 namespace vq {
 
 constexpr int kTcRows = 128;
-constexpr int kTcStages = 3;
-constexpr int kTcThreads = 320;
-constexpr int kTcDecodeWarps = 8;
-constexpr int kTcAhead = 4;  // k blocks of index bytes in flight per decode thread
+constexpr int kTcStages = 4;        // x tiles in shared memory and A tiles in TMEM
+constexpr int kTcDecodeWarps = 16;
+constexpr int kTcThreads = 64 + 32 * kTcDecodeWarps;
 constexpr int kTcMaxT = 256;
-constexpr uint32_t kTcATileBytes = kTcRows * 128;  // 128 rows x 64 bf16
-constexpr uint32_t kTcTilesOffset = 66560;         // after codebooks + barriers, 1024-aligned
-constexpr uint32_t kTcSmemMax = kTcTilesOffset + kTcStages * (kTcATileBytes + kTcMaxT * 128) + 1024;
+constexpr uint32_t kTcACols = 32;   // TMEM columns of one A stage (64 k of 16-bit pairs)
+// index-slice ring slot: lo 16 B, hi4 8 B, s2 8 B, scales 4 B per row (idx16: 32 B per row)
+constexpr uint32_t kTcIdxLo = 0, kTcIdxHi = 2048, kTcIdxS2 = 3072, kTcIdxSc = 4096;
+constexpr uint32_t kTcIdxSlot = 4608;
+constexpr int kTcIdxSlots = 4;
+constexpr uint32_t kTcOffBars = 65536;   // after the 64 KiB codebook
+constexpr uint32_t kTcOffIdx = 65792;    // index ring
+constexpr uint32_t kTcTilesOffset = 84992;  // 1024-aligned, after the index ring
+static_assert(kTcOffIdx + kTcIdxSlots * kTcIdxSlot <= kTcTilesOffset, "index ring overlaps the tiles");
+constexpr uint32_t kTcSmemMax = kTcTilesOffset + kTcStages * (kTcMaxT * 128) + 1024;
 
 struct TcArgs {
   LayerArgs a;
   int T;            // tokens per tile (MMA N): multiple of 16, <= 256
-  int k_per_split;  // multiple of 64
+  int k_per_split;  // multiple of 128 when splits > 1
   int splits;
   float* partial;   // [splits][M][N] when splits > 1
   uint32_t* tickets;
   uint32_t* err;
 };
 
-template <int FMT, typename T>
+__device__ __forceinline__ uint64_t f32x2_mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f32x2(float lo, float hi) {
+  return (uint64_t)__float_as_uint(lo) | ((uint64_t)__float_as_uint(hi) << 32);
+}
+
+// One-stage group: w_j = RN_T(fl32(s * c1_j)).  The mixed-precision FMA takes the
+// fp16 codeword half and the fp16 scale as they are and rounds the exact product
+// once to fp32 (adding -0 keeps the sign of a zero product).
+template <typename T>
+__device__ __forceinline__ void decode_one_stage(const uint4& c1, unsigned short s, uint32_t* out) {
+  const uint32_t w1[4] = {c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    float lo, hi;
+    asm("{ .reg .f16 l, h; mov.b32 {l, h}, %2; fma.rn.f32.f16 %0, l, %3, %4; fma.rn.f32.f16 %1, h, %3, %4; }"
+        : "=f"(lo), "=f"(hi)
+        : "r"(w1[q]), "h"(s), "f"(-0.0f));
+    out[q] = Elt<T>::pack(lo, hi);
+  }
+}
+
+// Two-stage group: w_j = RN_T(fl32(s * fl32(c1_j + c2_j))).  The mixed-precision
+// add widens the fp16 c1 half exactly and rounds the sum once.
+template <typename T>
+__device__ __forceinline__ void decode_two_stage(const uint4& c1, const uint32_t (&c2)[4], float s, uint32_t* out) {
+  const uint32_t w1[4] = {c1.x, c1.y, c1.z, c1.w};
+  const uint64_t sv = f32x2(s, s);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const float2 b = f16x2_to_f32x2(c2[q]);
+    float lo, hi;
+    asm("{ .reg .f16 l, h; mov.b32 {l, h}, %2; add.rn.f32.f16 %0, l, %3; add.rn.f32.f16 %1, h, %4; }"
+        : "=f"(lo), "=f"(hi)
+        : "r"(w1[q]), "f"(b.x), "f"(b.y));
+    const uint64_t m = f32x2_mul(f32x2(lo, hi), sv);
+    out[q] = Elt<T>::pack(__uint_as_float((uint32_t)m), __uint_as_float((uint32_t)(m >> 32)));
+  }
+}
+
+template <int FMT, typename T, bool kStaged>
 __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_constant__ CUtensorMap xmap, TcArgs p) {
   extern __shared__ unsigned char smem_raw[];
   constexpr bool kSmemCb = (FMT != kFmtVq16);
   constexpr bool kTwo = (FMT == kFmtRvq12_4);
   const LayerArgs& a = p.a;
-  // 1024-byte aligned base (the swizzle pattern is taken from address bits).
+  // 1024-byte aligned base (the swizzle pattern of the x tiles is taken from address bits).
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   unsigned char* sm = smem_raw + (base - raw);
-  uint4* cb1s = reinterpret_cast<uint4*>(sm);
-  uint4* cb2s = reinterpret_cast<uint4*>(sm + 65536);
-  const uint32_t bar0 = base + 65792;
+  const uint4* cb1s = reinterpret_cast<const uint4*>(sm);
+  const uint32_t bar0 = base + kTcOffBars;
   auto full_a = [&](int s) { return bar0 + 8u * s; };
   auto full_b = [&](int s) { return bar0 + 8u * (kTcStages + s); };
   auto empty = [&](int s) { return bar0 + 8u * (2 * kTcStages + s); };
   const uint32_t accum_bar = bar0 + 8u * (3 * kTcStages);
   const uint32_t cb_bar = accum_bar + 8u;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + 65880);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + 65884);
-  volatile int* last_flag = reinterpret_cast<volatile int*>(sm + 65888);
+  auto idx_full = [&](int s) { return cb_bar + 8u + 8u * s; };
+  auto idx_empty = [&](int s) { return cb_bar + 8u + 8u * kTcIdxSlots + 8u * s; };
+  static_assert(8 * (3 * kTcStages + 2 + 2 * kTcIdxSlots) <= 192, "barriers overlap the flags");
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kTcOffBars + 192);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + kTcOffBars + 196);
+  volatile int* last_flag = reinterpret_cast<volatile int*>(sm + kTcOffBars + 200);
   const uint32_t b_bytes = (uint32_t)p.T * 128u;
-  const uint32_t stage_bytes = kTcATileBytes + b_bytes;
-  auto a_tile = [&](int s) { return base + kTcTilesOffset + stage_bytes * s; };
-  auto b_tile = [&](int s) { return base + kTcTilesOffset + stage_bytes * s + kTcATileBytes; };
+  auto b_tile = [&](int s) { return base + kTcTilesOffset + b_bytes * s; };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int K = a.K, G = K / 8, N = a.N, M = a.M;
   const int row0 = blockIdx.x * kTcRows;
+  const int rows_here = min(kTcRows, N - row0);
   const int tok0 = blockIdx.y * p.T;
   const int split = blockIdx.z;
   const int kbeg = split * p.k_per_split;
   const int nkb = (min(K, kbeg + p.k_per_split) - kbeg) / 64;
-  const uint32_t tcols = p.T <= 32 ? 32u : (p.T <= 64 ? 64u : (p.T <= 128 ? 128u : 256u));
+  const int nsl = (nkb + 1) / 2;  // 128-input slices of this split (the last may be 64 wide)
+  const int s_first = kbeg / 128;
+  const bool block_scales = (a.scale_group == 64);
+  // TMEM: the accumulator in columns [0, T), then kTcStages A stages of 32 columns.
+  const uint32_t acol0 = ((uint32_t)p.T + 31u) & ~31u;
+  const uint32_t tneed = acol0 + kTcStages * kTcACols;
+  const uint32_t tcols = tneed <= 32 ? 32u : (tneed <= 64 ? 64u : (tneed <= 128 ? 128u : (tneed <= 256 ? 256u : 512u)));
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kTcStages; ++s) {
       ptx::mbar_init(full_a(s), kTcDecodeWarps);  // one arrival per decode warp
-      ptx::mbar_init(full_b(s), 1);  // the producer's expect_tx arrival (+ bytes)
-      ptx::mbar_init(empty(s), 1);   // one tcgen05.commit
+      ptx::mbar_init(full_b(s), 1);               // the producer's expect_tx arrival (+ bytes)
+      ptx::mbar_init(empty(s), 1);                // one tcgen05.commit
+    }
+    for (int s = 0; s < kTcIdxSlots; ++s) {
+      ptx::mbar_init(idx_full(s), 1);
+      ptx::mbar_init(idx_empty(s), kTcDecodeWarps);
     }
     ptx::mbar_init(accum_bar, 1);
     ptx::mbar_init(cb_bar, 1);
@@ -111,11 +178,29 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
     if (lane == 0) {
       ptx::prefetch_tensormap(&xmap);
       if (kSmemCb) {
-        ptx::mbar_arrive_expect_tx(cb_bar, 65536u + (kTwo ? 256u : 0u));
+        ptx::mbar_arrive_expect_tx(cb_bar, 65536u);
         ptx::bulk_load(base, a.cb1, 65536u, cb_bar);
-        if (kTwo) ptx::bulk_load(base + 65536, a.cb2, 256u, cb_bar);
       }
-      int issued = 0;
+      // Index bytes of slice j (of this split) for rows row0 .. row0+rows_here-1.
+      auto issue_idx = [&](int j) {
+        const int s = s_first + j, w = slice_width(s, G);
+        const uint32_t dst = base + kTcOffIdx + kTcIdxSlot * (j % kTcIdxSlots), bar = idx_full(j % kTcIdxSlots);
+        const int64_t e = (int64_t)16 * s * N + (int64_t)row0 * w;  // entry of (slice s, row row0)
+        const uint32_t sc = block_scales ? rows_here * (w / 8) * 2 : 0;
+        if (FMT == kFmtVq16) {
+          ptx::mbar_arrive_expect_tx(bar, rows_here * w * 2 + sc);
+          ptx::bulk_load(dst, a.idx16 + e, rows_here * w * 2, bar);
+        } else {
+          ptx::mbar_arrive_expect_tx(bar, rows_here * w + rows_here * w / 2 * (kTwo ? 2 : 1) + sc);
+          ptx::bulk_load(dst + kTcIdxLo, a.lo + e, rows_here * w, bar);
+          ptx::bulk_load(dst + kTcIdxHi, a.hi4 + e / 2, rows_here * w / 2, bar);
+          if (kTwo) ptx::bulk_load(dst + kTcIdxS2, a.s2 + e / 2, rows_here * w / 2, bar);
+        }
+        if (block_scales) ptx::bulk_load(dst + kTcIdxSc, a.scales + e / 8, sc, bar);
+      };
+      int issued = 0, issued_idx = 0;
+      if (kStaged)
+        for (; issued_idx < kTcIdxSlots && issued_idx < nsl; ++issued_idx) issue_idx(issued_idx);
       for (int kb = 0; kb < nkb && !*abort_flag; ++kb) {
         const int s = kb % kTcStages;
         if (kb >= kTcStages && !ptx::mbar_wait(empty(s), ((kb / kTcStages) - 1) & 1, p.err)) {
@@ -125,10 +210,26 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         ptx::mbar_arrive_expect_tx(full_b(s), b_bytes);
         ptx::tma_load_2d(b_tile(s), &xmap, kbeg + kb * 64, tok0, full_b(s));
         issued = kb + 1;
+        // After x of block kb (even, >= 4) is issued, refill with slice kb/2 + 2.
+        // Its slot held slice kb/2 - 2, which the decoders released before they
+        // finished block kb - 4; the stage-empty wait above already saw MMA kb - 4
+        // complete, so this wait never holds back the x loads.
+        if (kStaged && (kb & 1) == 0 && kb >= 4 && kb / 2 + 2 == issued_idx && issued_idx < nsl) {
+          const int j = issued_idx;
+          if (!ptx::mbar_wait(idx_empty(j % kTcIdxSlots), ((j / kTcIdxSlots) - 1) & 1, p.err)) {
+            *abort_flag = 1;
+            break;
+          }
+          issue_idx(j);
+          ++issued_idx;
+        }
       }
       // Do not leave while a copy into this CTA's shared memory may be in flight.
       for (int kb = (issued > kTcStages ? issued - kTcStages : 0); kb < issued; ++kb)
         ptx::mbar_wait(full_b(kb % kTcStages), (kb / kTcStages) & 1, p.err);
+      if (kStaged)
+        for (int j = (issued_idx > kTcIdxSlots ? issued_idx - kTcIdxSlots : 0); j < issued_idx; ++j)
+          ptx::mbar_wait(idx_full(j % kTcIdxSlots), (j / kTcIdxSlots) & 1, p.err);
       if (kSmemCb) ptx::mbar_wait(cb_bar, 0, p.err);
     }
   } else if (warp == 1) {
@@ -147,11 +248,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
           break;
         }
         ptx::tc_fence_after();
-        const uint64_t ad = ptx::smem_desc_sw128(a_tile(s));
+        const uint32_t at = tmem + acol0 + kTcACols * s;
         const uint64_t bd = ptx::smem_desc_sw128(b_tile(s));
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)  // +32 bytes along K inside the swizzle atom
-          ptx::umma_f16(tmem, ad + 2u * kk, bd + 2u * kk, idesc, (kb | kk) != 0);
+        for (int kk = 0; kk < 4; ++kk)  // A: +8 TMEM columns; B: +32 bytes along K inside the swizzle atom
+          ptx::umma_f16_ts(tmem, at + 8u * kk, bd + 2u * kk, idesc, (kb | kk) != 0);
         ptx::umma_commit(empty(s));
         issued = kb + 1;
       }
@@ -162,92 +263,146 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
     }
   } else {
     // ------------------------------------------------------------ decode + epilogue
-    const int q = warp & 3;            // TMEM lane quarter of this warp
-    const int half = (warp - 2) >> 2;  // which 4 groups of each k block
-    const int dr = 32 * q + lane;      // row within the tile == TMEM lane
+    const int q = warp & 3;           // TMEM lane quarter of this warp
+    const int part = (warp - 2) >> 2; // groups 2*part, 2*part+1 of each k block
+    const int dr = 32 * q + lane;     // row within the tile == TMEM lane
     const int r = row0 + dr;
     const bool valid = r < N;
     const uint4* cbg = reinterpret_cast<const uint4*>(a.cb1);
-    struct Rec {
-      uint32_t w[4];  // lo (2 words) + hi4 + s2, or idx16 (4 words) of this thread's 4 groups
-      uint32_t sc;
-    };
-    auto load_rec = [&](int kb, Rec& rc) {
-      rc.w[0] = rc.w[1] = rc.w[2] = rc.w[3] = 0;
-      rc.sc = 0;
-      if (!valid || kb >= nkb) return;
-      const int g0 = (kbeg / 8) + kb * 8 + 4 * half;  // first of this thread's 4 groups
-      const int s = g0 >> 4;
-      const int64_t e = (int64_t)16 * s * N + (int64_t)r * slice_width(s, G) + (g0 & 15);
-      if (FMT == kFmtVq16) {
-        const uint2 v = *reinterpret_cast<const uint2*>(a.idx16 + e);
-        rc.w[0] = v.x;
-        rc.w[1] = v.y;
-      } else {
-        rc.w[0] = *reinterpret_cast<const uint32_t*>(a.lo + e);
-        rc.w[1] = *reinterpret_cast<const uint16_t*>(a.hi4 + e / 2);
-        if (kTwo) rc.w[2] = *reinterpret_cast<const uint16_t*>(a.s2 + e / 2);
-      }
-      rc.sc = a.scales[scale_index(r, 8 * g0, N, K, a.scale_group)];
-    };
+    // Stage-2 codebook in registers: lane L holds entry L % 16.
+    uint32_t cb2r[4] = {0, 0, 0, 0};
+    if (kTwo) {
+      const uint4 v = reinterpret_cast<const uint4*>(a.cb2)[lane & 15];
+      cb2r[0] = v.x; cb2r[1] = v.y; cb2r[2] = v.z; cb2r[3] = v.w;
+    }
+    const unsigned short row_scale = (!block_scales && valid) ? a.scales[r] : (unsigned short)0;
+    const uint32_t tlane = tmem + ((uint32_t)(32 * q) << 16) + acol0 + 8u * part;
+    // This row's index bytes of the current slice (staged path).
+    uint4 rlo = make_uint4(0, 0, 0, 0), r16b = make_uint4(0, 0, 0, 0);
+    uint2 rhi = make_uint2(0, 0), rs2 = make_uint2(0, 0);
+    uint32_t rsc = 0;
     bool ok = true;
-    Rec rec[kTcAhead];
-#pragma unroll
-    for (int i = 0; i < kTcAhead; ++i) load_rec(i, rec[i]);
     if (kSmemCb && !ptx::mbar_wait(cb_bar, 0, p.err)) {
       *abort_flag = 1;
       ok = false;
     }
-    for (int kb0 = 0; ok && kb0 < nkb; kb0 += kTcAhead) {
-#pragma unroll
-      for (int i = 0; i < kTcAhead; ++i) {
-        const int kb = kb0 + i;
-        if (kb >= nkb || !ok) break;
-        const Rec cr = rec[i];
-        load_rec(kb + kTcAhead, rec[i]);
-        const int s = kb % kTcStages;
-        if (*abort_flag || (kb >= kTcStages && !ptx::mbar_wait(empty(s), ((kb / kTcStages) - 1) & 1, p.err))) {
-          *abort_flag = 1;
-          ok = false;
-          break;
-        }
-        const float sc = f16_bits_to_f32(cr.sc);
-        unsigned char* at = sm + (a_tile(s) - base) + dr * 128;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          uint32_t i1, i2 = 0;
-          if (FMT == kFmtVq16) {
-            i1 = (cr.w[j >> 1] >> (16 * (j & 1))) & 0xFFFFu;
-          } else {
-            i1 = ((cr.w[0] >> (8 * j)) & 0xFFu) | (((cr.w[1] >> (4 * j)) & 15u) << 8);
-            if (kTwo) i2 = (cr.w[2] >> (4 * j)) & 15u;
-          }
-          const uint4 c1 = kSmemCb ? cb1s[i1] : __ldg(cbg + i1);
-          const uint4 c2 = kTwo ? cb2s[i2] : c1;
-          uint32_t w[4];
-          decode_group_packed<T, kTwo>(c1, c2, valid ? sc : 0.f, w);
-          const int chunk = 4 * half + j;
-          *reinterpret_cast<uint4*>(at + ((chunk ^ (dr & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
-        }
-        ptx::fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(full_a(s));
+    for (int kb = 0; ok && kb < nkb; ++kb) {
+      const int s = kb % kTcStages;
+      const int j = kb >> 1, h = kb & 1;  // slice of this split, half of the slice
+      const int sl = s_first + j, w = slice_width(sl, G);
+      if (*abort_flag || (kb >= kTcStages && !ptx::mbar_wait(empty(s), ((kb / kTcStages) - 1) & 1, p.err)) ||
+          (kStaged && h == 0 && !ptx::mbar_wait(idx_full(j % kTcIdxSlots), (j / kTcIdxSlots) & 1, p.err))) {
+        *abort_flag = 1;
+        ok = false;
+        break;
       }
+      if (kStaged && h == 0) {
+        // Read the whole row of the slice once (vector loads), then free the slot.
+        if (valid) {
+          const unsigned char* slot = sm + kTcOffIdx + kTcIdxSlot * (j % kTcIdxSlots);
+          if (FMT == kFmtVq16) {
+            const uint4* src = reinterpret_cast<const uint4*>(slot + dr * w * 2);
+            rlo = src[0];
+            if (w == 16) r16b = src[1];
+          } else {
+            if (w == 16) {
+              rlo = *reinterpret_cast<const uint4*>(slot + kTcIdxLo + dr * 16);
+              rhi = *reinterpret_cast<const uint2*>(slot + kTcIdxHi + dr * 8);
+              if (kTwo) rs2 = *reinterpret_cast<const uint2*>(slot + kTcIdxS2 + dr * 8);
+            } else {
+              const uint2 l = *reinterpret_cast<const uint2*>(slot + kTcIdxLo + dr * 8);
+              rlo = make_uint4(l.x, l.y, 0, 0);
+              rhi = make_uint2(*reinterpret_cast<const uint32_t*>(slot + kTcIdxHi + dr * 4), 0);
+              if (kTwo) rs2 = make_uint2(*reinterpret_cast<const uint32_t*>(slot + kTcIdxS2 + dr * 4), 0);
+            }
+          }
+          if (block_scales)
+            rsc = (w == 16) ? *reinterpret_cast<const uint32_t*>(slot + kTcIdxSc + dr * 4)
+                            : (uint32_t)*reinterpret_cast<const uint16_t*>(slot + kTcIdxSc + dr * 2);
+        }
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(idx_empty(j % kTcIdxSlots));
+      }
+      // indices and scale of groups 8h + 2part and 8h + 2part + 1 of slice sl, this row
+      uint32_t i1[2] = {0, 0}, i2[2] = {0, 0};
+      unsigned short sc = row_scale;
+      if (valid) {
+        if (kStaged) {
+          if (FMT == kFmtVq16) {
+            const uint4 v = h ? r16b : rlo;
+            const uint32_t wd = part == 0 ? v.x : (part == 1 ? v.y : (part == 2 ? v.z : v.w));
+            i1[0] = wd & 0xFFFFu;
+            i1[1] = wd >> 16;
+          } else {
+            const uint32_t lw = h ? ((part & 2) ? rlo.w : rlo.z) : ((part & 2) ? rlo.y : rlo.x);
+            const uint32_t lo = (lw >> ((part & 1) * 16)) & 0xFFFFu;
+            const uint32_t hb = ((h ? rhi.y : rhi.x) >> (8 * part)) & 0xFFu;
+            i1[0] = (lo & 0xFFu) | ((hb & 15u) << 8);
+            i1[1] = (lo >> 8) | ((hb >> 4) << 8);
+            if (kTwo) {
+              const uint32_t qb = ((h ? rs2.y : rs2.x) >> (8 * part)) & 0xFFu;
+              i2[0] = qb & 15u;
+              i2[1] = qb >> 4;
+            }
+          }
+          if (block_scales) sc = (unsigned short)(h ? (rsc >> 16) : (rsc & 0xFFFFu));
+        } else {
+          const int gs = 8 * h + 2 * part;  // group within the slice
+          const int64_t e = (int64_t)16 * sl * N + (int64_t)r * w + gs;
+          if (FMT == kFmtVq16) {
+            const uint32_t v = *reinterpret_cast<const uint32_t*>(a.idx16 + e);
+            i1[0] = v & 0xFFFFu;
+            i1[1] = v >> 16;
+          } else {
+            const uint32_t lo = *reinterpret_cast<const uint16_t*>(a.lo + e);
+            const uint32_t hb = a.hi4[e / 2];
+            i1[0] = (lo & 0xFFu) | ((hb & 15u) << 8);
+            i1[1] = (lo >> 8) | ((hb >> 4) << 8);
+            if (kTwo) {
+              const uint32_t qb = a.s2[e / 2];
+              i2[0] = qb & 15u;
+              i2[1] = qb >> 4;
+            }
+          }
+          if (block_scales) sc = a.scales[scale_index(r, 128 * sl + 64 * h, N, K, a.scale_group)];
+        }
+      }
+      uint32_t out[8];
+      const float scf = kTwo ? __half2float(__ushort_as_half(sc)) : 0.f;
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        const uint4 c1 = kSmemCb ? cb1s[i1[t]] : __ldg(cbg + i1[t]);
+        if (kTwo) {
+          uint32_t c2[4];
+#pragma unroll
+          for (int w4 = 0; w4 < 4; ++w4) c2[w4] = __shfl_sync(0xffffffffu, cb2r[w4], (int)i2[t]);
+          decode_two_stage<T>(c1, c2, scf, out + 4 * t);
+        } else {
+          decode_one_stage<T>(c1, sc, out + 4 * t);
+        }
+      }
+      // Columns 8part .. 8part+7 of A stage s (k = 16part .. 16part+15 of the block), own lane.
+      ptx::tc_fence_after();
+      ptx::tmem_st8(tlane + kTcACols * s, out);
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(full_a(s));
     }
     // -------------------------------------------------------------- epilogue
     if (ok && !ptx::mbar_wait(accum_bar, 0, p.err)) *abort_flag = 1;
     // One decision for all epilogue threads, so the named barriers below are
     // reached by every one of them or by none.
-    asm volatile("bar.sync 1, 256;" ::: "memory");
+    asm volatile("bar.sync 1, %0;" ::"n"(32 * kTcDecodeWarps) : "memory");
     if (threadIdx.x == 64) *last_flag = *abort_flag ? 0 : 2;
-    asm volatile("bar.sync 1, 256;" ::: "memory");
+    asm volatile("bar.sync 1, %0;" ::"n"(32 * kTcDecodeWarps) : "memory");
     ok = (*last_flag == 2);
-    asm volatile("bar.sync 1, 256;" ::: "memory");
+    asm volatile("bar.sync 1, %0;" ::"n"(32 * kTcDecodeWarps) : "memory");
     if (ok) {
       ptx::tc_fence_after();
       const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16);
       uint16_t* y = static_cast<uint16_t*>(a.y);
-      for (int c0 = 16 * half; c0 < p.T; c0 += 32) {  // the two warps of a quarter alternate 16-column chunks
+      for (int c0 = 16 * part; c0 < p.T; c0 += 64) {  // the four warps of a quarter take turns by 16 columns
         uint32_t v[16];
         ptx::tmem_ld16(taddr + c0, v);
         ptx::tmem_wait_ld();
@@ -264,19 +419,37 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
       ptx::tc_fence_before();
       if (p.splits > 1) {
         __threadfence();
-        asm volatile("bar.sync 1, 256;" ::: "memory");
+        asm volatile("bar.sync 1, %0;" ::"n"(32 * kTcDecodeWarps) : "memory");
         const int tile = blockIdx.y * gridDim.x + blockIdx.x;
         if (threadIdx.x == 64) *last_flag = (atomicAdd(&p.tickets[tile], 1u) == (uint32_t)(p.splits - 1));
-        asm volatile("bar.sync 1, 256;" ::: "memory");
+        asm volatile("bar.sync 1, %0;" ::"n"(32 * kTcDecodeWarps) : "memory");
         if (*last_flag) {
           __threadfence();
-          const int tend = min(M, tok0 + p.T);
-          if (valid)
-            for (int tok = tok0 + half; tok < tend; tok += 2) {
-              float sum = 0.f;
-              for (int k = 0; k < p.splits; ++k) sum += __ldcg(p.partial + ((int64_t)k * M + tok) * N + r);
-              y[(int64_t)tok * N + r] = Elt<T>::from_f32(sum);
+          ptx::tc_fence_after();
+          // y = sum of the splits' partials in split order; this CTA's own split
+          // comes from its accumulator (the same fp32 values it stored).  Sixteen
+          // tokens per step, so each split's loads are all in flight at once.
+          for (int c0 = 16 * part; c0 < p.T; c0 += 64) {
+            float acc[16];
+            for (int k = 0; k < p.splits; ++k) {
+              uint32_t t[16];
+              if (k == split) {
+                ptx::tmem_ld16(taddr + c0, t);
+                ptx::tmem_wait_ld();
+              } else {
+                const float* src = p.partial + ((int64_t)k * M + tok0 + c0) * N + r;
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                  t[i] = (valid && tok0 + c0 + i < M) ? __float_as_uint(__ldcg(src + (int64_t)i * N)) : 0u;
+              }
+#pragma unroll
+              for (int i = 0; i < 16; ++i) acc[i] = k == 0 ? __uint_as_float(t[i]) : acc[i] + __uint_as_float(t[i]);
             }
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              if (valid && tok0 + c0 + i < M) y[(int64_t)(tok0 + c0 + i) * N + r] = Elt<T>::from_f32(acc[i]);
+          }
+          ptx::tc_fence_before();
           if (threadIdx.x == 64) p.tickets[tile] = 0u;
         }
       }
@@ -318,14 +491,14 @@ static TcGeom tc_geom(int M, int N, int K, int num_sms) {
   g.TT = (M + g.T - 1) / g.T;
   g.RT = (N + kTcRows - 1) / kTcRows;
   const int tiles = g.RT * g.TT;
-  const int nb = K / 64;
+  const int nsl = (K + 127) / 128;  // splits start on 128-input slice boundaries
   int S = num_sms / tiles;
   if (S < 1) S = 1;
   if (S > 8) S = 8;
-  if (S > nb) S = nb;
-  const int bps = (nb + S - 1) / S;
-  g.S = (nb + bps - 1) / bps;
-  g.kps = bps * 64;
+  if (S > nsl) S = nsl;
+  const int sps = (nsl + S - 1) / S;
+  g.S = (nsl + sps - 1) / sps;
+  g.kps = sps * 128;
   return g;
 }
 
@@ -341,7 +514,7 @@ bool plan_tc(const vq_linear_desc& d, const DeviceInfo& dev, int M, Plan* p) {
   return true;
 }
 
-template <int FMT, typename T>
+template <int FMT, typename T, bool kStaged>
 static cudaError_t launch_tc_t(const LayerArgs& a, const TcGeom& g, float* scratch, uint32_t* tickets,
                                uint32_t* err, cudaStream_t s) {
   EncodeTiledFn enc = encode_fn();
@@ -356,13 +529,22 @@ static cudaError_t launch_tc_t(const LayerArgs& a, const TcGeom& g, float* scrat
                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
-  const uint32_t smem = kTcTilesOffset + kTcStages * (kTcATileBytes + (uint32_t)g.T * 128u) + 1024u;
-  cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<FMT, T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const uint32_t smem = kTcTilesOffset + kTcStages * ((uint32_t)g.T * 128u) + 1024u;
+  auto kern = tc_gemm_kernel<FMT, T, kStaged>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   TcArgs p{a, g.T, g.kps, g.S, g.S > 1 ? scratch : nullptr, g.S > 1 ? tickets : nullptr, err};
   dim3 grid(g.RT, g.TT, g.S);
-  tc_gemm_kernel<FMT, T><<<grid, kTcThreads, smem, s>>>(map, p);
+  kern<<<grid, kTcThreads, smem, s>>>(map, p);
   return cudaGetLastError();
+}
+
+template <int FMT, typename T>
+static cudaError_t launch_tc_s(const LayerArgs& a, const TcGeom& g, float* scratch, uint32_t* tickets,
+                               uint32_t* err, cudaStream_t s) {
+  // Bulk copies need 16-byte sizes: N % 8 == 0 makes every per-slice run one.
+  return (a.N % 8 == 0) ? launch_tc_t<FMT, T, true>(a, g, scratch, tickets, err, s)
+                        : launch_tc_t<FMT, T, false>(a, g, scratch, tickets, err, s);
 }
 
 cudaError_t launch_tc(const LayerArgs& a, const Plan& pl, float* scratch, uint32_t* tickets, uint32_t* err,
@@ -375,14 +557,14 @@ cudaError_t launch_tc(const LayerArgs& a, const Plan& pl, float* scratch, uint32
   const bool bf = a.act == VQ_BF16;
   switch (a.fmt) {
     case kFmtRvq12:
-      return bf ? launch_tc_t<kFmtRvq12, __nv_bfloat16>(a, g, scratch, tickets, err, s)
-                : launch_tc_t<kFmtRvq12, __half>(a, g, scratch, tickets, err, s);
+      return bf ? launch_tc_s<kFmtRvq12, __nv_bfloat16>(a, g, scratch, tickets, err, s)
+                : launch_tc_s<kFmtRvq12, __half>(a, g, scratch, tickets, err, s);
     case kFmtRvq12_4:
-      return bf ? launch_tc_t<kFmtRvq12_4, __nv_bfloat16>(a, g, scratch, tickets, err, s)
-                : launch_tc_t<kFmtRvq12_4, __half>(a, g, scratch, tickets, err, s);
+      return bf ? launch_tc_s<kFmtRvq12_4, __nv_bfloat16>(a, g, scratch, tickets, err, s)
+                : launch_tc_s<kFmtRvq12_4, __half>(a, g, scratch, tickets, err, s);
     default:
-      return bf ? launch_tc_t<kFmtVq16, __nv_bfloat16>(a, g, scratch, tickets, err, s)
-                : launch_tc_t<kFmtVq16, __half>(a, g, scratch, tickets, err, s);
+      return bf ? launch_tc_s<kFmtVq16, __nv_bfloat16>(a, g, scratch, tickets, err, s)
+                : launch_tc_s<kFmtVq16, __half>(a, g, scratch, tickets, err, s);
   }
 }
 
