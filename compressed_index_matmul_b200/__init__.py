@@ -30,6 +30,7 @@ from ._binding import (  # noqa: F401
     vq_linear_create,
     vq_linear_destroy,
     vq_linear_forward,
+    vq_linear_forward_noalloc,
     vq_linear_launches,
     vq_linear_set_path,
     vq_rht_apply,

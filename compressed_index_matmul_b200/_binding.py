@@ -26,8 +26,8 @@ STATUS_NAMES = {0: "VQ_OK", 1: "VQ_ERR_INVALID_ARG", 2: "VQ_ERR_UNSUPPORTED", 3:
 
 # Every entry point the header declares (checked by the tests against the .so).
 EXPORTS = ("vq_abi_version", "vq_linear_create", "vq_linear_destroy", "vq_linear_set_path", "vq_linear_forward",
-           "vq_linear_launches", "vq_rht_apply", "vq_linear_check", "vq_last_error", "vq_debug_unpack",
-           "vq_debug_dequant")
+           "vq_linear_forward_noalloc", "vq_linear_launches", "vq_rht_apply", "vq_linear_check", "vq_last_error",
+           "vq_debug_unpack", "vq_debug_dequant")
 
 
 class VQError(RuntimeError):
@@ -80,6 +80,9 @@ def load(path: str | None = None):
         lib.vq_linear_forward.restype = st
         lib.vq_linear_forward.argtypes = [P, P, ctypes.POINTER(vq_planes), ctypes.POINTER(vq_codebooks), P, P,
                                           I32, I32, I32, P]
+        lib.vq_linear_forward_noalloc.restype = st
+        lib.vq_linear_forward_noalloc.argtypes = [ctypes.POINTER(vq_linear_desc), P, ctypes.POINTER(vq_planes),
+                                                  ctypes.POINTER(vq_codebooks), P, P, I32, P]
         lib.vq_linear_launches.restype = I32
         lib.vq_linear_launches.argtypes = [P, I32]
         lib.vq_rht_apply.restype = st
@@ -152,6 +155,14 @@ def vq_linear_launches(h, M: int) -> int:
 def vq_linear_forward(h, x, planes: vq_planes, codebooks: vq_codebooks, scales, y, M, N, K, stream=None) -> None:
     _check(load().vq_linear_forward(h, _ptr(x), ctypes.byref(planes), ctypes.byref(codebooks), _ptr(scales),
                                     _ptr(y), M, N, K, _stream(stream)))
+
+
+def vq_linear_forward_noalloc(N, K, fmt, scale_group, act_dtype, x, planes: vq_planes, codebooks: vq_codebooks,
+                              scales, y, M, stream=None, rht=0) -> None:
+    """Handle-free forward of 0 <= M <= 16 tokens that allocates nothing (fixed in-library scratch)."""
+    d = vq_linear_desc(N, K, fmt, scale_group, act_dtype, max(M, 1), rht)
+    _check(load().vq_linear_forward_noalloc(ctypes.byref(d), _ptr(x), ctypes.byref(planes), ctypes.byref(codebooks),
+                                            _ptr(scales), _ptr(y), M, _stream(stream)))
 
 
 def vq_rht_apply(x, x_out, signs, M, K, dtype, stream=None) -> None:

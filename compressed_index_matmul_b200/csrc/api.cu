@@ -7,6 +7,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <string>
 
 #include "internal.h"
@@ -344,5 +345,102 @@ VQ_API vq_status vq_debug_dequant(vq_linear_t h, const vq_planes* planes, const 
   vq::LayerArgs a = make_args(h->d, planes, codebooks, scales);
   cudaError_t e = vq::launch_debug_dequant(a, w_out, wdt, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "vq_debug_dequant launch");
+  return VQ_OK;
+}
+
+// ---------------------------------------------------------------- no-allocation forward
+//
+// vq_linear_forward_noalloc runs the same warp-MMA GEMV kernel as
+// vq_linear_forward (path VQ_PATH_GEMV) but takes its split-K scratch from a
+// fixed buffer compiled into this library instead of from a handle, so a call
+// never allocates device or host memory.
+namespace {
+
+constexpr size_t kNoAllocPartialBytes = size_t(4) << 20;  // split-K partial sums (fp32)
+constexpr int kNoAllocTickets = 4096;                     // per-row-tile completion counters
+constexpr int kNoAllocMaxDevices = 64;
+
+// One copy per device (the module is loaded into each device's context).
+// Partial sums first, then the tickets, which must be zero whenever no call is
+// running: set-up clears them and every call leaves them zero.
+static __device__ __align__(256) unsigned char
+    g_noalloc_scratch[kNoAllocPartialBytes + kNoAllocTickets * sizeof(uint32_t)];
+
+struct NoAllocDevice {
+  bool ready;
+  unsigned char* scratch;  // device address of g_noalloc_scratch on this device
+  vq::DeviceInfo dev;
+};
+std::mutex g_noalloc_mu;
+NoAllocDevice g_noalloc[kNoAllocMaxDevices];
+
+// First use on a device (which must be current): look up the buffer's address,
+// zero the tickets and wait for that to finish.  Later calls only read the cache.
+vq_status noalloc_device(const NoAllocDevice** out) {
+  int cur = -1;
+  cudaError_t e = cudaGetDevice(&cur);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (cur < 0 || cur >= kNoAllocMaxDevices)
+    return fail(VQ_ERR_UNSUPPORTED, "device %d: the no-allocation path supports devices 0..%d", cur,
+                kNoAllocMaxDevices - 1);
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  NoAllocDevice& d = g_noalloc[cur];
+  if (!d.ready) {
+    int major = 0, minor = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, cur);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, cur);
+    if (major != 10 || minor != 0)
+      return fail(VQ_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a only", cur, major,
+                  minor);
+    vq::DeviceInfo info{};
+    info.device = cur;
+    cudaDeviceGetAttribute(&info.num_sms, cudaDevAttrMultiProcessorCount, cur);
+    cudaDeviceGetAttribute(&info.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, cur);
+    unsigned char* ptr = nullptr;
+    e = cudaGetSymbolAddress((void**)&ptr, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(no-allocation scratch)");
+    e = cudaMemset(ptr + kNoAllocPartialBytes, 0, kNoAllocTickets * sizeof(uint32_t));
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the no-allocation tickets");
+    d.scratch = ptr;
+    d.dev = info;
+    d.ready = true;
+  }
+  *out = &d;
+  return VQ_OK;
+}
+
+}  // namespace
+
+VQ_API vq_status vq_linear_forward_noalloc(const vq_linear_desc* desc, const void* x, const vq_planes* planes,
+                                           const vq_codebooks* codebooks, const void* scales, void* y, int32_t M,
+                                           void* stream) {
+  vq_status st = validate_desc(desc);
+  if (st) return st;
+  const vq_linear_desc& d = *desc;
+  if (M < 0 || M > 16) return fail(VQ_ERR_INVALID_ARG, "M=%d outside [0, 16] (the no-allocation path)", M);
+  if ((st = check_ptr(x, "x")) || (st = check_ptr(y, "y")) || (st = validate_planes(d, planes)) ||
+      (st = validate_codebooks(d, codebooks, scales)))
+    return st;
+  if (x == y) return fail(VQ_ERR_INVALID_ARG, "y must not alias x");
+  if (M == 0) return VQ_OK;
+  const NoAllocDevice* nd = nullptr;
+  if ((st = noalloc_device(&nd))) return st;
+  vq::Plan p{};
+  if (!vq::plan_forward(d, nd->dev, M, VQ_PATH_GEMV, &p))
+    return fail(VQ_ERR_UNSUPPORTED, "the GEMV path cannot run M=%d", M);
+  if (p.scratch_bytes > kNoAllocPartialBytes || p.tickets > kNoAllocTickets)
+    return fail(VQ_ERR_UNSUPPORTED,
+                "N=%d, K=%d, M=%d needs %zu bytes of split-K scratch and %d tickets; the no-allocation buffer "
+                "holds %zu bytes and %d tickets (use vq_linear_forward with a handle)",
+                d.N, d.K, M, p.scratch_bytes, p.tickets, kNoAllocPartialBytes, kNoAllocTickets);
+  vq::LayerArgs a = make_args(d, planes, codebooks, scales);
+  a.x = x;
+  a.y = y;
+  a.M = M;
+  cudaError_t e = vq::launch_gemv(a, p, reinterpret_cast<float*>(nd->scratch),
+                                  reinterpret_cast<uint32_t*>(nd->scratch + kNoAllocPartialBytes),
+                                  static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "vq_linear_forward_noalloc launch");
   return VQ_OK;
 }

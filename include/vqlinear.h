@@ -151,6 +151,38 @@ vq_status vq_linear_forward(vq_linear_t h, const void* x, const vq_planes* plane
                             const vq_codebooks* codebooks, const void* scales, void* y,
                             int32_t M, int32_t N, int32_t K, void* stream);
 
+/* y = x . W^T for 0 <= M <= 16 without a handle and without allocating anything.
+ *
+ * The method's source pages have no counterpart to this call; it exists for
+ * callers that cannot allocate device memory at the point where they run the
+ * layer, e.g. code running inside another library's allocator or memory-pool
+ * callback (a nested cudaMalloc would re-enter it), or a process whose device
+ * memory is entirely reserved up front by a serving engine's pool, so that any
+ * later cudaMalloc fails or forces a device-wide synchronisation.
+ *
+ * It runs the same warp-MMA kernel as vq_linear_forward with VQ_PATH_GEMV and
+ * gives the same result for the same inputs.  Arguments are those of
+ * vq_linear_forward, with the layer shape taken from `desc` (validated as by
+ * vq_linear_create; desc->max_M is not used).  Split-K partial sums and
+ * completion counters live in one fixed buffer compiled into this library, one
+ * copy per device: 4 MiB of partials and 4096 counters.  A shape whose plan
+ * needs more (roughly splits x M x N x 4 bytes, or more than 4096 tiles of 16
+ * output rows) returns VQ_ERR_UNSUPPORTED with the sizes in vq_last_error();
+ * use a handle for those.  No call allocates memory: neither this library nor
+ * any library it calls does.
+ *
+ * Set-up: the first call on a device (the current one) looks up the buffer's
+ * address, clears the counters and synchronises the device.  Make that first
+ * call before any stream capture begins; later calls only enqueue the kernel.
+ * The counters must be zero when a call starts; every call leaves them zero.
+ *
+ * Concurrency: all calls on a device share the one buffer.  Two calls whose
+ * kernels overlap on the GPU (different streams, or different host threads)
+ * race on it and give wrong results; order them on one stream or with events. */
+vq_status vq_linear_forward_noalloc(const vq_linear_desc* desc, const void* x, const vq_planes* planes,
+                                    const vq_codebooks* codebooks, const void* scales, void* y, int32_t M,
+                                    void* stream);
+
 /* Number of kernels vq_linear_forward enqueues for this M (0 for M == 0), or -1
  * if M is out of range. */
 int32_t vq_linear_launches(vq_linear_t h, int32_t M);
