@@ -54,8 +54,14 @@ constexpr uint32_t kTcTilesOffset = 84992;  // 1024-aligned, after the index rin
 static_assert(kTcOffIdx + kTcIdxSlots * kTcIdxSlot <= kTcTilesOffset, "index ring overlaps the tiles");
 constexpr uint32_t kTcSmemMax = kTcTilesOffset + kTcStages * (kTcMaxT * 128) + 1024;
 
+// Epilogue kinds: y (or fp32 partials) written per element; y staged in shared
+// memory and written by TMA stores (one split); a K-split pair in a 2-CTA cluster
+// that adds the two halves over distributed shared memory, then TMA stores.
+constexpr int kEpiGlobal = 0, kEpiStore = 1, kEpiPair = 2;
+
 struct TcArgs {
   LayerArgs a;
+  int epi;          // kEpi*
   int T;            // tokens per tile (MMA N): multiple of 16, <= 256
   int k_per_split;  // multiple of 128 when splits > 1
   int splits;
@@ -108,7 +114,8 @@ __device__ __forceinline__ void decode_two_stage(const uint4& c1, const uint32_t
 }
 
 template <int FMT, typename T, bool kStaged>
-__global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_constant__ CUtensorMap xmap, TcArgs p) {
+__global__ void __launch_bounds__(kTcThreads, 1)
+    tc_gemm_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap ymap, TcArgs p) {
   extern __shared__ unsigned char smem_raw[];
   constexpr bool kSmemCb = (FMT != kFmtVq16);
   constexpr bool kTwo = (FMT == kFmtRvq12_4);
@@ -389,20 +396,83 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(full_a(s));
     }
-    // -------------------------------------------------------------- epilogue
     if (ok && !ptx::mbar_wait(accum_bar, 0, p.err)) *abort_flag = 1;
-    // One decision for all epilogue threads, so the named barriers below are
-    // reached by every one of them or by none.
-    asm volatile("bar.sync 1, %0;" ::"n"(32 * kTcDecodeWarps) : "memory");
-    if (threadIdx.x == 64) *last_flag = *abort_flag ? 0 : 2;
-    asm volatile("bar.sync 1, %0;" ::"n"(32 * kTcDecodeWarps) : "memory");
-    ok = (*last_flag == 2);
-    asm volatile("bar.sync 1, %0;" ::"n"(32 * kTcDecodeWarps) : "memory");
-    if (ok) {
+  }
+
+  // ---------------------------------------------------------------- epilogue
+  // Every thread of the CTA gets here (all waits above are bounded), so the
+  // barriers below, the cluster-wide ones included, are reached by all of them.
+  __syncthreads();
+  const bool fine = (*abort_flag == 0);
+  const bool dec = warp >= 2;
+  const int q = warp & 3, part = (warp - 2) >> 2;
+  const int dr = 32 * q + lane, r = row0 + dr;
+  const bool valid = r < N;
+  const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16);
+  const int nch = p.T / 16;  // 16-token chunks; thread (row dr, part) handles chunks part, part+4, ...
+  if (p.epi != kEpiGlobal) {
+    // y through a shared-memory staging tile ([chunk][16 tokens][128 rows] in the
+    // codebook area, free now) and TMA tensor stores, which also clip the ragged
+    // edges.  With a K-split pair (a 2-CTA cluster, rank = split) each CTA owns the
+    // chunks of its parity and sends the others' fp32 sums into its partner's
+    // receive area (the x stages, free now) over distributed shared memory.
+    const bool pair = (p.epi == kEpiPair);
+    const uint32_t rank = (uint32_t)split;
+    auto recv_addr = [&](int ci, int i) { return base + kTcTilesOffset + (uint32_t)(ci >> 1) * 8192u + (uint32_t)(i * 128 + dr) * 4u; };
+    auto stage_addr = [&](int ci, int i) { return base + (uint32_t)(ci * 16 + i) * 256u + (uint32_t)dr * 2u; };
+    if (pair) {
+      ptx::cluster_sync();  // both CTAs are done with their x stages
+      if (dec && fine) {
+        ptx::tc_fence_after();
+        for (int ci = part; ci < nch; ci += 4) {
+          if ((uint32_t)(ci & 1) == rank || tok0 + 16 * ci >= M) continue;
+          uint32_t v[16];
+          ptx::tmem_ld16(taddr + 16 * ci, v);
+          ptx::tmem_wait_ld();
+          const uint32_t dst = ptx::map_shared_rank(recv_addr(ci, 0), rank ^ 1u);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) ptx::st_cluster_f32(dst + (uint32_t)i * 512u, __uint_as_float(v[i]));
+        }
+      }
+      ptx::cluster_sync();  // the partner's sums have arrived
+    }
+    if (dec && fine) {
       ptx::tc_fence_after();
-      const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16);
-      uint16_t* y = static_cast<uint16_t*>(a.y);
-      for (int c0 = 16 * part; c0 < p.T; c0 += 64) {  // the four warps of a quarter take turns by 16 columns
+      for (int ci = part; ci < nch; ci += 4) {
+        if ((pair && (uint32_t)(ci & 1) != rank) || tok0 + 16 * ci >= M) continue;
+        uint32_t v[16];
+        ptx::tmem_ld16(taddr + 16 * ci, v);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          float f = __uint_as_float(v[i]);
+          if (pair) {  // two splits: the sum does not depend on the order
+            float o;
+            asm volatile("ld.shared.f32 %0, [%1];" : "=f"(o) : "r"(recv_addr(ci, i)));
+            f += o;
+          }
+          const uint16_t h = Elt<T>::from_f32(f);
+          asm volatile("st.shared.u16 [%0], %1;" ::"r"(stage_addr(ci, i)), "h"(h) : "memory");
+        }
+      }
+      ptx::fence_proxy_async_smem();
+    }
+    __syncthreads();
+    if (threadIdx.x == 64 && fine) {
+      for (int ci = 0; ci < nch; ++ci) {
+        if ((pair && (uint32_t)(ci & 1) != rank) || tok0 + 16 * ci >= M) continue;
+        ptx::tma_store_2d(&ymap, base + (uint32_t)ci * 4096u, row0, tok0 + 16 * ci);
+      }
+      ptx::bulk_commit();
+      ptx::bulk_wait_all();
+    }
+  } else if (dec) {
+    // y (one split) or fp32 partials written per element; the last CTA of a split
+    // tile, picked by an atomic ticket, sums the partials in split order.
+    uint16_t* y = static_cast<uint16_t*>(a.y);
+    if (fine) {
+      ptx::tc_fence_after();
+      for (int c0 = 16 * part; c0 < p.T; c0 += 64) {
         uint32_t v[16];
         ptx::tmem_ld16(taddr + c0, v);
         ptx::tmem_wait_ld();
@@ -417,44 +487,44 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         }
       }
       ptx::tc_fence_before();
-      if (p.splits > 1) {
+    }
+    if (fine && p.splits > 1) {
+      __threadfence();
+      asm volatile("bar.sync 1, %0;" ::"n"(32 * kTcDecodeWarps) : "memory");
+      const int tile = blockIdx.y * gridDim.x + blockIdx.x;
+      if (threadIdx.x == 64) *last_flag = (atomicAdd(&p.tickets[tile], 1u) == (uint32_t)(p.splits - 1));
+      asm volatile("bar.sync 1, %0;" ::"n"(32 * kTcDecodeWarps) : "memory");
+      if (*last_flag) {
         __threadfence();
-        asm volatile("bar.sync 1, %0;" ::"n"(32 * kTcDecodeWarps) : "memory");
-        const int tile = blockIdx.y * gridDim.x + blockIdx.x;
-        if (threadIdx.x == 64) *last_flag = (atomicAdd(&p.tickets[tile], 1u) == (uint32_t)(p.splits - 1));
-        asm volatile("bar.sync 1, %0;" ::"n"(32 * kTcDecodeWarps) : "memory");
-        if (*last_flag) {
-          __threadfence();
-          ptx::tc_fence_after();
-          // y = sum of the splits' partials in split order; this CTA's own split
-          // comes from its accumulator (the same fp32 values it stored).  Sixteen
-          // tokens per step, so each split's loads are all in flight at once.
-          for (int c0 = 16 * part; c0 < p.T; c0 += 64) {
-            float acc[16];
-            for (int k = 0; k < p.splits; ++k) {
-              uint32_t t[16];
-              if (k == split) {
-                ptx::tmem_ld16(taddr + c0, t);
-                ptx::tmem_wait_ld();
-              } else {
-                const float* src = p.partial + ((int64_t)k * M + tok0 + c0) * N + r;
+        ptx::tc_fence_after();
+        // Sixteen tokens per step, so each split's loads are all in flight at
+        // once; this CTA's own split comes from its accumulator.
+        for (int c0 = 16 * part; c0 < p.T; c0 += 64) {
+          float acc[16];
+          for (int k = 0; k < p.splits; ++k) {
+            uint32_t t[16];
+            if (k == split) {
+              ptx::tmem_ld16(taddr + c0, t);
+              ptx::tmem_wait_ld();
+            } else {
+              const float* src = p.partial + ((int64_t)k * M + tok0 + c0) * N + r;
 #pragma unroll
-                for (int i = 0; i < 16; ++i)
-                  t[i] = (valid && tok0 + c0 + i < M) ? __float_as_uint(__ldcg(src + (int64_t)i * N)) : 0u;
-              }
-#pragma unroll
-              for (int i = 0; i < 16; ++i) acc[i] = k == 0 ? __uint_as_float(t[i]) : acc[i] + __uint_as_float(t[i]);
+              for (int i = 0; i < 16; ++i)
+                t[i] = (valid && tok0 + c0 + i < M) ? __float_as_uint(__ldcg(src + (int64_t)i * N)) : 0u;
             }
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-              if (valid && tok0 + c0 + i < M) y[(int64_t)(tok0 + c0 + i) * N + r] = Elt<T>::from_f32(acc[i]);
+            for (int i = 0; i < 16; ++i) acc[i] = k == 0 ? __uint_as_float(t[i]) : acc[i] + __uint_as_float(t[i]);
           }
-          ptx::tc_fence_before();
-          if (threadIdx.x == 64) p.tickets[tile] = 0u;
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            if (valid && tok0 + c0 + i < M) y[(int64_t)(tok0 + c0 + i) * N + r] = Elt<T>::from_f32(acc[i]);
         }
+        ptx::tc_fence_before();
+        if (threadIdx.x == 64) p.tickets[tile] = 0u;
       }
     }
   }
+  ptx::tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     ptx::tc_fence_after();
@@ -481,7 +551,7 @@ static EncodeTiledFn encode_fn() {
 }
 
 struct TcGeom {
-  int T, TT, RT, S, kps;
+  int T, TT, RT, S, kps, epi;
 };
 
 static TcGeom tc_geom(int M, int N, int K, int num_sms) {
@@ -499,6 +569,8 @@ static TcGeom tc_geom(int M, int N, int K, int num_sms) {
   const int sps = (nsl + S - 1) / S;
   g.S = (nsl + sps - 1) / sps;
   g.kps = sps * 128;
+  // TMA stores of y need 16-byte row pitches (N % 8 == 0).
+  g.epi = (N % 8 != 0 || g.S > 2) ? kEpiGlobal : (g.S == 2 ? kEpiPair : kEpiStore);
   return g;
 }
 
@@ -509,8 +581,9 @@ bool plan_tc(const vq_linear_desc& d, const DeviceInfo& dev, int M, Plan* p) {
   p->splits = g.S;
   p->k_per_split = g.kps;
   p->launches = 1;
-  p->scratch_bytes = g.S > 1 ? (size_t)g.S * M * d.N * sizeof(float) : 0;
-  p->tickets = g.S > 1 ? g.RT * g.TT : 0;
+  const bool partials = g.S > 1 && g.epi == kEpiGlobal;
+  p->scratch_bytes = partials ? (size_t)g.S * M * d.N * sizeof(float) : 0;
+  p->tickets = partials ? g.RT * g.TT : 0;
   return true;
 }
 
@@ -519,23 +592,48 @@ static cudaError_t launch_tc_t(const LayerArgs& a, const TcGeom& g, float* scrat
                                uint32_t* err, cudaStream_t s) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return cudaErrorNotSupported;
-  CUtensorMap map;
+  CUtensorMap map, ymap;
+  const CUtensorMapDataType dt =
+      a.act == VQ_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   const cuuint64_t dims[2] = {(cuuint64_t)a.K, (cuuint64_t)a.M};
   const cuuint64_t strides[1] = {(cuuint64_t)a.K * 2};
   const cuuint32_t box[2] = {64, (cuuint32_t)g.T};
   const cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(&map, a.act == VQ_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
-                   const_cast<void*>(a.x), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+  CUresult r = enc(&map, dt, 2, const_cast<void*>(a.x), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  ymap = map;  // unused unless the epilogue stores y by TMA
+  if (g.epi != kEpiGlobal) {
+    const cuuint64_t ydims[2] = {(cuuint64_t)a.N, (cuuint64_t)a.M};
+    const cuuint64_t ystrides[1] = {(cuuint64_t)a.N * 2};
+    const cuuint32_t ybox[2] = {(cuuint32_t)kTcRows, 16};
+    r = enc(&ymap, dt, 2, a.y, ydims, ystrides, ybox, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  }
   const uint32_t smem = kTcTilesOffset + kTcStages * ((uint32_t)g.T * 128u) + 1024u;
   auto kern = tc_gemm_kernel<FMT, T, kStaged>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  TcArgs p{a, g.T, g.kps, g.S, g.S > 1 ? scratch : nullptr, g.S > 1 ? tickets : nullptr, err};
-  dim3 grid(g.RT, g.TT, g.S);
-  kern<<<grid, kTcThreads, smem, s>>>(map, p);
+  const bool partials = g.S > 1 && g.epi == kEpiGlobal;
+  TcArgs p{a, g.epi, g.T, g.kps, g.S, partials ? scratch : nullptr, partials ? tickets : nullptr, err};
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(g.RT, g.TT, g.S);
+  cfg.blockDim = dim3(kTcThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  if (g.epi == kEpiPair) {  // the two K-splits of a tile form one cluster
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 2;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  e = cudaLaunchKernelEx(&cfg, kern, map, ymap, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

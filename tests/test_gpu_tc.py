@@ -41,6 +41,8 @@ TC_CASES = [
     (256, 640, FMT_RVQ12, 640, DT_F16, 33),       # one scale per row, 64-wide last slice, staged
     (132, 576, FMT_RVQ12_4, 64, DT_F16, 20),      # N % 8 != 0: indices read from global memory
     (256, 8192, FMT_RVQ12_4, 64, DT_BF16, 32),    # 8 slices per split: the index ring refills
+    (2040, 512, FMT_RVQ12_4, 64, DT_BF16, 900),   # 64 tiles: K-split pair (2-CTA cluster), ragged rows/tokens
+    (2040, 256, FMT_RVQ12, 64, DT_F16, 1200),     # 80 tiles: one split, y by TMA stores, ragged edges
 ]
 
 
@@ -87,6 +89,8 @@ ONE_HOT_CASES = [
     (132, 576, FMT_RVQ12, 64, DT_BF16),     # N % 8 != 0: indices from global memory
     (136, 1024, FMT_VQ16, 1024, DT_F16),    # 16-bit indices, one scale per row
     (136, 1024, FMT_VQ16, 64, DT_BF16),
+    (8192, 256, FMT_RVQ12_4, 64, DT_BF16),  # 64 row tiles: K-split pair over a 2-CTA cluster
+    (9600, 256, FMT_RVQ12, 256, DT_F16),    # 75 row tiles: one split, TMA-stored y
 ]
 
 
