@@ -14,12 +14,13 @@
 //   warp 1     allocates TMEM; lane 0 issues tcgen05.mma (M=128, N=T, K=16, four
 //              per k block, A read from TMEM) and commits each stage back.
 //   warps 2-17 decode: four warps per TMEM lane quarter; thread = one row of the
-//              tile (its TMEM lane) and two of the 8 groups of each k block.  Once
-//              per slice it reads its row's index bytes from the staged slice;
-//              per k block it gathers the stage-1 codeword from shared memory and
-//              the stage-2 codeword from the warp's registers (shuffle), decodes
-//              with the materialised-weight rounding and stores the 16 weights
-//              into its own TMEM lane of the stage's A columns (tcgen05.st).
+//              tile (its TMEM lane) and 4 consecutive groups of each slice, which
+//              lie in one of the slice's two k blocks (so each A stage is written
+//              by 8 warps).  Per slice it reads its index bytes from the staged
+//              slice, gathers the stage-1 codewords from shared memory and the
+//              stage-2 codewords from the warp's registers (shuffle), decodes with
+//              the materialised-weight rounding and stores the 32 weights into
+//              its own TMEM lane of the stage's A columns (tcgen05.st).
 //              After the last block the same threads read the accumulator from
 //              TMEM and write y (or fp32 split-K partials; the last CTA of a tile,
 //              by an atomic ticket, sums the partials in split order).
@@ -158,7 +159,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kTcStages; ++s) {
-      ptx::mbar_init(full_a(s), kTcDecodeWarps);  // one arrival per decode warp
+      ptx::mbar_init(full_a(s), kTcDecodeWarps / 2);  // the 8 decode warps of this block's parity
       ptx::mbar_init(full_b(s), 1);               // the producer's expect_tx arrival (+ bytes)
       ptx::mbar_init(empty(s), 1);                // one tcgen05.commit
     }
@@ -217,11 +218,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         ptx::mbar_arrive_expect_tx(full_b(s), b_bytes);
         ptx::tma_load_2d(b_tile(s), &xmap, kbeg + kb * 64, tok0, full_b(s));
         issued = kb + 1;
-        // After x of block kb (even, >= 4) is issued, refill with slice kb/2 + 2.
-        // Its slot held slice kb/2 - 2, which the decoders released before they
-        // finished block kb - 4; the stage-empty wait above already saw MMA kb - 4
-        // complete, so this wait never holds back the x loads.
-        if (kStaged && (kb & 1) == 0 && kb >= 4 && kb / 2 + 2 == issued_idx && issued_idx < nsl) {
+        // After x of block kb (odd, >= 5) is issued, refill with slice (kb+3)/2.
+        // Its slot held slice (kb-5)/2, which every decode warp released before it
+        // decoded block kb - 4 or earlier; the stage-empty wait above already saw
+        // MMA kb - 4 (and so every earlier block) complete, so this wait never
+        // holds back the x loads.
+        if (kStaged && (kb & 1) == 1 && kb >= 5 && (kb + 3) / 2 == issued_idx && issued_idx < nsl) {
           const int j = issued_idx;
           if (!ptx::mbar_wait(idx_empty(j % kTcIdxSlots), ((j / kTcIdxSlots) - 1) & 1, p.err)) {
             *abort_flag = 1;
@@ -269,10 +271,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (!ok && issued) ptx::mbar_wait(accum_bar, 0, p.err);
     }
   } else {
-    // ------------------------------------------------------------ decode + epilogue
-    const int q = warp & 3;           // TMEM lane quarter of this warp
-    const int part = (warp - 2) >> 2; // groups 2*part, 2*part+1 of each k block
-    const int dr = 32 * q + lane;     // row within the tile == TMEM lane
+    // ------------------------------------------------------------ decode
+    // Thread (row dr, part) decodes groups 4part .. 4part+3 of every slice: inputs
+    // 32part .. 32part+31 of the slice, i.e. half of k block 2j + part/2, which is
+    // 16 TMEM columns of that block's A stage.
+    const int q = warp & 3;            // TMEM lane quarter of this warp
+    const int part = (warp - 2) >> 2;  // 0..3
+    const int hsel = part >> 1;        // which k block of each slice
+    const int dr = 32 * q + lane;      // row within the tile == TMEM lane
     const int r = row0 + dr;
     const bool valid = r < N;
     const uint4* cbg = reinterpret_cast<const uint4*>(a.cb1);
@@ -283,114 +289,81 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       cb2r[0] = v.x; cb2r[1] = v.y; cb2r[2] = v.z; cb2r[3] = v.w;
     }
     const unsigned short row_scale = (!block_scales && valid) ? a.scales[r] : (unsigned short)0;
-    const uint32_t tlane = tmem + ((uint32_t)(32 * q) << 16) + acol0 + 8u * part;
-    // This row's index bytes of the current slice (staged path).
-    uint4 rlo = make_uint4(0, 0, 0, 0), r16b = make_uint4(0, 0, 0, 0);
-    uint2 rhi = make_uint2(0, 0), rs2 = make_uint2(0, 0);
-    uint32_t rsc = 0;
+    const uint32_t tlane = tmem + ((uint32_t)(32 * q) << 16) + acol0 + 16u * (uint32_t)(part & 1);
     bool ok = true;
     if (kSmemCb && !ptx::mbar_wait(cb_bar, 0, p.err)) {
       *abort_flag = 1;
       ok = false;
     }
-    for (int kb = 0; ok && kb < nkb; ++kb) {
+    for (int j = 0; ok && j < nsl; ++j) {
+      const int kb = 2 * j + hsel;
+      if (kb >= nkb) {
+        // A 64-wide last slice has no odd block: this warp has nothing to decode
+        // there, but it still releases the slice's index slot.
+        if (kStaged && lane == 0) ptx::mbar_arrive(idx_empty(j % kTcIdxSlots));
+        break;
+      }
       const int s = kb % kTcStages;
-      const int j = kb >> 1, h = kb & 1;  // slice of this split, half of the slice
       const int sl = s_first + j, w = slice_width(sl, G);
       if (*abort_flag || (kb >= kTcStages && !ptx::mbar_wait(empty(s), ((kb / kTcStages) - 1) & 1, p.err)) ||
-          (kStaged && h == 0 && !ptx::mbar_wait(idx_full(j % kTcIdxSlots), (j / kTcIdxSlots) & 1, p.err))) {
+          (kStaged && !ptx::mbar_wait(idx_full(j % kTcIdxSlots), (j / kTcIdxSlots) & 1, p.err))) {
         *abort_flag = 1;
         ok = false;
         break;
       }
-      if (kStaged && h == 0) {
-        // Read the whole row of the slice once (vector loads), then free the slot.
-        if (valid) {
-          const unsigned char* slot = sm + kTcOffIdx + kTcIdxSlot * (j % kTcIdxSlots);
-          if (FMT == kFmtVq16) {
-            const uint4* src = reinterpret_cast<const uint4*>(slot + dr * w * 2);
-            rlo = src[0];
-            if (w == 16) r16b = src[1];
-          } else {
-            if (w == 16) {
-              rlo = *reinterpret_cast<const uint4*>(slot + kTcIdxLo + dr * 16);
-              rhi = *reinterpret_cast<const uint2*>(slot + kTcIdxHi + dr * 8);
-              if (kTwo) rs2 = *reinterpret_cast<const uint2*>(slot + kTcIdxS2 + dr * 8);
-            } else {
-              const uint2 l = *reinterpret_cast<const uint2*>(slot + kTcIdxLo + dr * 8);
-              rlo = make_uint4(l.x, l.y, 0, 0);
-              rhi = make_uint2(*reinterpret_cast<const uint32_t*>(slot + kTcIdxHi + dr * 4), 0);
-              if (kTwo) rs2 = make_uint2(*reinterpret_cast<const uint32_t*>(slot + kTcIdxS2 + dr * 4), 0);
-            }
-          }
-          if (block_scales)
-            rsc = (w == 16) ? *reinterpret_cast<const uint32_t*>(slot + kTcIdxSc + dr * 4)
-                            : (uint32_t)*reinterpret_cast<const uint16_t*>(slot + kTcIdxSc + dr * 2);
-        }
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(idx_empty(j % kTcIdxSlots));
-      }
-      // indices and scale of groups 8h + 2part and 8h + 2part + 1 of slice sl, this row
-      uint32_t i1[2] = {0, 0}, i2[2] = {0, 0};
+      // Index bytes of groups 4part .. 4part+3 of slice sl, this row.
+      uint32_t lo4 = 0, hi2 = 0, s22 = 0;  // 4 lo bytes; 4 packed hi / s2 nibbles
+      uint2 v16 = make_uint2(0, 0);         // 4 idx16 entries
       unsigned short sc = row_scale;
       if (valid) {
         if (kStaged) {
+          const unsigned char* slot = sm + kTcOffIdx + kTcIdxSlot * (j % kTcIdxSlots);
           if (FMT == kFmtVq16) {
-            const uint4 v = h ? r16b : rlo;
-            const uint32_t wd = part == 0 ? v.x : (part == 1 ? v.y : (part == 2 ? v.z : v.w));
-            i1[0] = wd & 0xFFFFu;
-            i1[1] = wd >> 16;
+            v16 = *reinterpret_cast<const uint2*>(slot + (dr * w + 4 * part) * 2);
           } else {
-            const uint32_t lw = h ? ((part & 2) ? rlo.w : rlo.z) : ((part & 2) ? rlo.y : rlo.x);
-            const uint32_t lo = (lw >> ((part & 1) * 16)) & 0xFFFFu;
-            const uint32_t hb = ((h ? rhi.y : rhi.x) >> (8 * part)) & 0xFFu;
-            i1[0] = (lo & 0xFFu) | ((hb & 15u) << 8);
-            i1[1] = (lo >> 8) | ((hb >> 4) << 8);
-            if (kTwo) {
-              const uint32_t qb = ((h ? rs2.y : rs2.x) >> (8 * part)) & 0xFFu;
-              i2[0] = qb & 15u;
-              i2[1] = qb >> 4;
-            }
+            lo4 = *reinterpret_cast<const uint32_t*>(slot + kTcIdxLo + dr * w + 4 * part);
+            hi2 = *reinterpret_cast<const uint16_t*>(slot + kTcIdxHi + dr * (w / 2) + 2 * part);
+            if (kTwo) s22 = *reinterpret_cast<const uint16_t*>(slot + kTcIdxS2 + dr * (w / 2) + 2 * part);
           }
-          if (block_scales) sc = (unsigned short)(h ? (rsc >> 16) : (rsc & 0xFFFFu));
+          if (block_scales) sc = *reinterpret_cast<const uint16_t*>(slot + kTcIdxSc + (dr * (w / 8) + hsel) * 2);
         } else {
-          const int gs = 8 * h + 2 * part;  // group within the slice
-          const int64_t e = (int64_t)16 * sl * N + (int64_t)r * w + gs;
+          const int64_t e = (int64_t)16 * sl * N + (int64_t)r * w + 4 * part;
           if (FMT == kFmtVq16) {
-            const uint32_t v = *reinterpret_cast<const uint32_t*>(a.idx16 + e);
-            i1[0] = v & 0xFFFFu;
-            i1[1] = v >> 16;
+            v16 = *reinterpret_cast<const uint2*>(a.idx16 + e);
           } else {
-            const uint32_t lo = *reinterpret_cast<const uint16_t*>(a.lo + e);
-            const uint32_t hb = a.hi4[e / 2];
-            i1[0] = (lo & 0xFFu) | ((hb & 15u) << 8);
-            i1[1] = (lo >> 8) | ((hb >> 4) << 8);
-            if (kTwo) {
-              const uint32_t qb = a.s2[e / 2];
-              i2[0] = qb & 15u;
-              i2[1] = qb >> 4;
-            }
+            lo4 = *reinterpret_cast<const uint32_t*>(a.lo + e);
+            hi2 = *reinterpret_cast<const uint16_t*>(a.hi4 + e / 2);
+            if (kTwo) s22 = *reinterpret_cast<const uint16_t*>(a.s2 + e / 2);
           }
-          if (block_scales) sc = a.scales[scale_index(r, 128 * sl + 64 * h, N, K, a.scale_group)];
+          if (block_scales) sc = a.scales[scale_index(r, 128 * sl + 64 * hsel, N, K, a.scale_group)];
         }
       }
-      uint32_t out[8];
+      if (kStaged) {
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(idx_empty(j % kTcIdxSlots));
+      }
+      uint32_t out[16];
       const float scf = kTwo ? __half2float(__ushort_as_half(sc)) : 0.f;
 #pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        const uint4 c1 = kSmemCb ? cb1s[i1[t]] : __ldg(cbg + i1[t]);
+      for (int t = 0; t < 4; ++t) {
+        uint32_t i1;
+        if (FMT == kFmtVq16)
+          i1 = ((t < 2 ? v16.x : v16.y) >> (16 * (t & 1))) & 0xFFFFu;
+        else
+          i1 = ((lo4 >> (8 * t)) & 0xFFu) | (((hi2 >> (4 * t)) & 15u) << 8);
+        const uint4 c1 = kSmemCb ? cb1s[i1] : __ldg(cbg + i1);
         if (kTwo) {
+          const int i2 = (int)((s22 >> (4 * t)) & 15u);
           uint32_t c2[4];
 #pragma unroll
-          for (int w4 = 0; w4 < 4; ++w4) c2[w4] = __shfl_sync(0xffffffffu, cb2r[w4], (int)i2[t]);
+          for (int w4 = 0; w4 < 4; ++w4) c2[w4] = __shfl_sync(0xffffffffu, cb2r[w4], i2);
           decode_two_stage<T>(c1, c2, scf, out + 4 * t);
         } else {
           decode_one_stage<T>(c1, sc, out + 4 * t);
         }
       }
-      // Columns 8part .. 8part+7 of A stage s (k = 16part .. 16part+15 of the block), own lane.
       ptx::tc_fence_after();
-      ptx::tmem_st8(tlane + kTcACols * s, out);
+      ptx::tmem_st16(tlane + kTcACols * s, out);
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
       __syncwarp();
