@@ -379,11 +379,22 @@ def gpu_arm(args):
     dominant = "lut_gemv_kernel" if (M == 1 and wl.layers[0][1].fmt != FMT_VQ16) else (
         "gemv_kernel" if M <= 16 else "tc_gemm_kernel")
     traffic = lookup_traffic(dominant, args.workload, M)
-    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,
-                "kernel": dominant, "peak_source": f"{peak_src} hbm_gbs",
-                "avg_launch_us": round(1e3 * float(np.mean(per_fwd)) / max(1, np.mean(launches_per_fwd)), 3),
-                "algorithmic_bytes_per_launch": int(np.mean(bytes_per_fwd))}
+    avg_launch_us = round(1e3 * float(np.mean(per_fwd)) / max(1, np.mean(launches_per_fwd)), 3)
+    if dominant == "tc_gemm_kernel":
+        # a dense contraction: 2*M*N*K flops per forward against the bf16 tensor peak
+        flops_per_fwd = [2.0 * M * spec.N * spec.K for _, spec, _ in wl.layers]
+        tflops = sum(flops_per_fwd) / (sum(per_fwd) * 1e-3) / 1e12
+        roofline = {"bound": "tensor", "achieved": round(tflops, 1), "peak": peaks["bf16_tflops"],
+                    "unit": "TFLOP/s", "frac": round(tflops / peaks["bf16_tflops"], 4), "traffic": traffic,
+                    "kernel": dominant, "peak_source": f"{peak_src} bf16_tflops (burst)",
+                    "frac_of_sustained": round(tflops / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]), 4),
+                    "avg_launch_us": avg_launch_us, "algorithmic_flops_per_launch": int(np.mean(flops_per_fwd))}
+    else:
+        roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,
+                    "kernel": dominant, "peak_source": f"{peak_src} hbm_gbs",
+                    "avg_launch_us": avg_launch_us,
+                    "algorithmic_bytes_per_launch": int(np.mean(bytes_per_fwd))}
 
     # ------------------------------------------------ end to end through the public API
     e2e_ms, h2d, d2h = time_e2e(wl, M, min(args.steps, 200), 3, flush)

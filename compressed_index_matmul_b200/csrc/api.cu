@@ -29,7 +29,7 @@ struct vq_linear_s {
   size_t scratch_bytes;
   uint32_t* tickets;  // completion counters, zeroed at create, left zero by every forward
   int num_tickets;
-  uint32_t* gbar;     // grid-barrier words: arrivals (left zero) and a generation counter
+  uint32_t* gbar;     // grid-barrier arrival counter (64-bit, 8-byte aligned; only ever grows)
   uint32_t* err;      // device word, set by bounded waits that gave up
 };
 
@@ -207,14 +207,14 @@ VQ_API vq_status vq_linear_create(const vq_linear_desc* desc, vq_linear_t* out) 
     }
   }
   h->num_tickets = tickets;
-  const size_t small = sizeof(uint32_t) * (size_t)(3 + tickets);
+  const size_t small = sizeof(uint32_t) * (size_t)(4 + tickets);
   uint32_t* words = nullptr;
   e = cudaMalloc(&words, small);
   if (e == cudaSuccess) e = cudaMemset(words, 0, small);
   if (e == cudaSuccess) e = cudaDeviceSynchronize();  // the zeroing is complete before any forward
   h->err = words;
-  h->gbar = words + 1;
-  h->tickets = tickets ? words + 3 : nullptr;
+  h->gbar = words + 2;
+  h->tickets = tickets ? words + 4 : nullptr;
   if (e != cudaSuccess) {
     cudaFree(h->scratch);
     cudaFree(words);

@@ -50,7 +50,8 @@ bool plan_forward(const vq_linear_desc& d, const DeviceInfo& dev, int M, int for
 // `tickets` are per-launch completion counters: zero before every forward, and
 // every forward leaves them zero again.
 cudaError_t launch_gemv(const LayerArgs& a, const Plan& p, float* scratch, uint32_t* tickets, cudaStream_t s);
-// `gbar` is the handle's two grid-barrier words (arrivals, generation).
+// `gbar` is the handle's grid-barrier arrival counter: 64 bits, 8-byte aligned,
+// zero at create and only ever incremented (each launch adds its grid size).
 cudaError_t launch_lut(const LayerArgs& a, const Plan& p, float* scratch, uint32_t* gbar, uint32_t* err,
                        cudaStream_t s);
 cudaError_t launch_tc(const LayerArgs& a, const Plan& p, float* scratch, uint32_t* tickets, uint32_t* err_flag,

@@ -14,14 +14,18 @@
 // those MMAs does not depend on x, so each warp loads its share of it into
 // registers once and every rebuild is only MMAs and stores.
 //
-// Work distribution: units are (K-slice s, 512-row chunk) in slice-major order;
-// a persistent grid of at most one CTA per SM takes a contiguous run of units.
-// In the K-slice-major storage a unit's index bytes are one contiguous run per
-// plane, so one thread streams them into a ring of shared-memory stages with
-// bulk copies (TMA), several units ahead.  Thread t handles rows t and t+256 of
-// a unit and writes one fp32 partial sum per row and slice.
+// Work distribution: the (K-slice, row) pairs in slice-major order are cut into
+// one contiguous, equal range per CTA of a persistent grid (at most one CTA per
+// SM), so every CTA sweeps the same number of rows and rebuilds its tables at
+// most once more than the others.  A range is walked in chunks of up to 512 rows
+// that never cross a slice; in the K-slice-major storage a chunk's index bytes
+// are one contiguous run per plane.  A producer warp streams the chunks into a
+// ring of shared-memory stages with bulk copies (TMA), several chunks ahead, and
+// 8 lookup warps consume them (full / empty mbarriers per stage, no CTA-wide
+// barrier per chunk).  Lookup thread t handles rows t and t+256 of a chunk and
+// writes one fp32 partial sum per row and slice.
 //
-// Split-K reduction: after the last unit every CTA meets at a grid-wide barrier
+// Split-K reduction: after the last chunk every CTA meets at a grid-wide barrier
 // (all CTAs are resident: the grid never exceeds the SM count and a CTA takes a
 // whole SM's shared memory); then each CTA sums the partials of its own share
 // of the rows with a fixed tree (GLQ README, "Inference kernels": fixed-order
@@ -38,22 +42,64 @@
 namespace vq {
 
 constexpr int kLutGroups = 16;                 // groups per K-slice (128 inputs)
-constexpr int kLutThreads = 256;
-constexpr int kLutUnitRows = 512;              // rows per unit (two per thread)
+constexpr int kLutConsumers = 256;             // lookup threads (8 warps)
+constexpr int kLutThreads = kLutConsumers + 32;  // + one producer warp
+constexpr int kLutChunkRows = 512;             // rows per chunk (two per lookup thread)
 constexpr int kLutTableBytes = 4096 * 2 + 64;  // one group's T1 (bf16) + pad (bank spread)
-constexpr int kLutStages = 4;                  // bulk-copy ring depth (units in flight)
+constexpr int kLutStages = 4;                  // bulk-copy ring depth (chunks in flight)
 constexpr int kLutMaxX = 4;                    // x slices preloaded per CTA
 // one ring stage: lo 16 B, hi4 8 B, s2 8 B, scales 4 B per row
-constexpr int kLutOffHi = kLutUnitRows * 16;
-constexpr int kLutOffS2 = kLutOffHi + kLutUnitRows * 8;
-constexpr int kLutOffSc = kLutOffS2 + kLutUnitRows * 8;
-constexpr int kLutStageBytes = kLutOffSc + kLutUnitRows * 4;
+constexpr int kLutOffHi = kLutChunkRows * 16;
+constexpr int kLutOffS2 = kLutOffHi + kLutChunkRows * 8;
+constexpr int kLutOffSc = kLutOffS2 + kLutChunkRows * 8;
+constexpr int kLutStageBytes = kLutOffSc + kLutChunkRows * 4;
 constexpr int kLutOffT2 = kLutGroups * kLutTableBytes;
 constexpr int kLutOffXh = kLutOffT2 + kLutGroups * 16 * 4;
 constexpr int kLutOffXf = kLutOffXh + kLutGroups * 8 * 2;
-constexpr int kLutOffMisc = kLutOffXf + kLutGroups * 8 * 4;  // per-group scales, barriers
+constexpr int kLutOffMisc = kLutOffXf + kLutGroups * 8 * 4;  // group scales, barriers, chunk records
 constexpr int kLutOffRing = kLutOffMisc + 256;
 constexpr int kLutSmem = kLutOffRing + kLutStages * kLutStageBytes;
+
+// Table builds per slice, counted in rows of lookups (a build costs about as
+// much as one chunk of lookups) when the (slice, row) sequence is split.
+constexpr int kLutBuildRows = 512;
+
+// Walks one CTA's range of (slice, row) positions in chunks that stay inside a
+// slice and hold at most kLutChunkRows rows (a multiple of 4, as N is).  The
+// ranges are equal in "virtual" rows: each slice is preceded by kLutBuildRows
+// virtual rows standing for its table build, so a CTA whose range spans a slice
+// start gets correspondingly fewer real rows.
+struct LutChunks {
+  int s, r;  // next chunk's slice and first row
+  int64_t pos, end;
+  static __device__ int64_t real_pos(int64_t v, int N) {
+    const int64_t span = (int64_t)N + kLutBuildRows;
+    const int64_t sl = v / span, off = v - sl * span;
+    return sl * N + (off > kLutBuildRows ? off - kLutBuildRows : 0);
+  }
+  __device__ void init(int N, int S, int cta, int grid) {
+    const int64_t total = (int64_t)S * N, vtotal = (int64_t)S * ((int64_t)N + kLutBuildRows);
+    pos = real_pos(vtotal * cta / grid, N) & ~int64_t(3);
+    end = cta == grid - 1 ? total : (real_pos(vtotal * (cta + 1) / grid, N) & ~int64_t(3));
+    s = (int)(pos / N);
+    r = (int)(pos - (int64_t)s * N);
+  }
+  __device__ bool next(int N, int& cs, int& cr, int& rows) {
+    if (pos >= end) return false;
+    const int64_t left = end - pos;
+    rows = min(kLutChunkRows, N - r);
+    if (left < rows) rows = (int)left;
+    cs = s;
+    cr = r;
+    pos += rows;
+    r += rows;
+    if (r == N) {
+      r = 0;
+      ++s;
+    }
+    return true;
+  }
+};
 
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   uint32_t r;
@@ -113,7 +159,7 @@ __device__ __forceinline__ void lookup_row(const uint4& lo4, const uint2& h, con
 template <int FMT, typename T>
 __global__ void __launch_bounds__(kLutThreads, 1)
     lut_gemv_kernel(LayerArgs a, float* __restrict__ partial, uint32_t* __restrict__ gbar, uint32_t* __restrict__ err,
-                    int S, int C) {
+                    int S) {
   extern __shared__ __align__(128) unsigned char smem[];
   constexpr bool kTwo = (FMT == kFmtRvq12_4);
   unsigned char* t1 = smem;
@@ -121,207 +167,237 @@ __global__ void __launch_bounds__(kLutThreads, 1)
   uint32_t* xh = reinterpret_cast<uint32_t*>(smem + kLutOffXh);
   float* xf = reinterpret_cast<float*>(smem + kLutOffXf);
   float* gsc = reinterpret_cast<float*>(smem + kLutOffMisc);        // [16] per-group 2^-e
-  const uint32_t bars = smem_u32(smem + kLutOffMisc + 64);          // [kLutStages] mbarriers
-  volatile int* flag = reinterpret_cast<volatile int*>(smem + kLutOffMisc + 128);
-  unsigned char* ring = smem + kLutOffRing;
-  const uint32_t t1_base = smem_u32(t1), t2_base = smem_u32(t2), ring_base = smem_u32(ring);
+  const uint32_t full0 = smem_u32(smem + kLutOffMisc + 64);         // [kLutStages] mbarriers: chunk landed
+  const uint32_t empty0 = smem_u32(smem + kLutOffMisc + 96);        // [kLutStages] mbarriers: chunk consumed
+  volatile int* abortf = reinterpret_cast<volatile int*>(smem + kLutOffMisc + 128);  // a bounded wait gave up
+  volatile int* flag = reinterpret_cast<volatile int*>(smem + kLutOffMisc + 192);
+  const uint32_t t1_base = smem_u32(t1), t2_base = smem_u32(t2), ring_base = smem_u32(smem + kLutOffRing);
 
   const int N = a.N;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const bool block_scales = (a.scale_group == 64);
-  const int64_t U = (int64_t)S * C;
-  const int64_t u0 = U * blockIdx.x / gridDim.x, u1 = U * (blockIdx.x + 1) / gridDim.x;
   const uint16_t* xg = static_cast<const uint16_t*>(a.x);
+  LutChunks chunks;
+  chunks.init(N, S, blockIdx.x, gridDim.x);
+  const int s_first = chunks.s;
 
-  // Unit u's bytes: one bulk copy per plane into stage (u - u0) % kLutStages.
-  auto issue = [&](int64_t u) {
-    const int s = (int)(u / C), ch = (int)(u % C);
-    const int r0 = ch * kLutUnitRows, rows = min(kLutUnitRows, N - r0);
-    const int st = (int)((u - u0) % kLutStages);
-    const uint32_t dst = ring_base + st * kLutStageBytes, bar = bars + 8 * st;
-    const int64_t e = (int64_t)16 * s * N + (int64_t)16 * r0;  // lo entry of (slice s, row r0)
-    ptx::mbar_arrive_expect_tx(bar, rows * (16 + 8 + (kTwo ? 8 : 0) + (block_scales ? 4 : 0)));
-    ptx::bulk_load(dst, a.lo + e, rows * 16, bar);
-    ptx::bulk_load(dst + kLutOffHi, a.hi4 + e / 2, rows * 8, bar);
-    if (kTwo) ptx::bulk_load(dst + kLutOffS2, a.s2 + e / 2, rows * 8, bar);
-    if (block_scales) ptx::bulk_load(dst + kLutOffSc, a.scales + e / 8, rows * 4, bar);  // 2 per row per slice
-  };
   if (tid == 0) {
-    for (int i = 0; i < kLutStages; ++i) ptx::mbar_init(bars + 8 * i, 1);
+    for (int i = 0; i < kLutStages; ++i) {
+      ptx::mbar_init(full0 + 8 * i, 1);
+      ptx::mbar_init(empty0 + 8 * i, kLutConsumers / 32);
+    }
+    *abortf = 0;
     ptx::fence_barrier_init();
-    for (int i = 0; i < kLutStages; ++i)
-      if (u0 + i < u1) issue(u0 + i);
   }
-
-  // Codebook operand of the table MMAs, held for the whole kernel: warp w covers
-  // codewords 512w .. 512w+511 in 16 blocks of 32; see the build below.
-  const int g = lane >> 2, c = lane & 3;
-  uint32_t bfrag[16][4];
-  {
-    const uint32_t* cbw = reinterpret_cast<const uint32_t*>(a.cb1);
-#pragma unroll
-    for (int it = 0; it < 16; ++it)
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-        bfrag[it][j] = __ldg(cbw + (size_t)(warp * 512 + it * 32 + 8 * (g >> 1) + 2 * j + (g & 1)) * 4 + c);
-  }
-  float c2v[8];
-  if (kTwo) {
-    const uint4 q = reinterpret_cast<const uint4*>(a.cb2)[tid & 15];
-    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-    for (int p = 0; p < 4; ++p) {
-      const float2 v = f16x2_to_f32x2(w[p]);
-      c2v[2 * p] = v.x;
-      c2v[2 * p + 1] = v.y;
-    }
-  }
-  // Everything above reads only the layer's constant inputs; x, y, the scratch
-  // and the barrier words are touched only after the previous kernel completed.
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  const uint32_t gen0 = *reinterpret_cast<volatile uint32_t*>(gbar + 1);  // barrier generation of this launch
-  const int s_first = (int)(u0 / C);
-  float xpre[kLutMaxX];
-#pragma unroll
-  for (int i = 0; i < kLutMaxX; ++i) {
-    const int s = s_first + i;
-    xpre[i] = (tid < 128 && s < S) ? Elt<T>::to_f32(xg[(int64_t)s * 128 + tid]) : 0.f;
-  }
-  __syncthreads();  // barrier init is visible to every waiting thread
-
-  int cur = -1;
+  __syncthreads();
   bool ok = true;
-  for (int64_t u = u0; u < u1; ++u) {
-    const int s = (int)(u / C), ch = (int)(u % C);
-    const int st = (int)((u - u0) % kLutStages);
-    if (s != cur) {
-      // ------------------------------------------------------------ build
-      __syncthreads();  // everyone is done with the previous tables
-      float xv = 0.f;
-      if (tid < 128) {
-        const int i = s - s_first;
-        if (i < kLutMaxX) {
-#pragma unroll
-          for (int k = 0; k < kLutMaxX; ++k)
-            if (k == i) xv = xpre[k];
-        } else {
-          xv = Elt<T>::to_f32(xg[(int64_t)s * 128 + tid]);
+
+  if (warp == kLutConsumers / 32) {
+    // ------------------------------------------------------------ producer
+    // Reads only the layer's constant index planes and scales, so it may run
+    // while the previous kernel in the stream is still finishing.
+    if (lane == 0) {
+      int k = 0, cs, cr, rows;
+      while (chunks.next(N, cs, cr, rows)) {
+        const int st = k % kLutStages;
+        if (*abortf || (k >= kLutStages && !ptx::mbar_wait(empty0 + 8 * st, ((k / kLutStages) - 1) & 1, err))) {
+          *abortf = 1;
+          break;
         }
+        const uint32_t dst = ring_base + st * kLutStageBytes, bar = full0 + 8 * st;
+        const int64_t e = (int64_t)16 * cs * N + (int64_t)16 * cr;  // lo entry of (slice cs, row cr)
+        ptx::mbar_arrive_expect_tx(bar, rows * (16 + 8 + (kTwo ? 8 : 0) + (block_scales ? 4 : 0)));
+        ptx::bulk_load(dst, a.lo + e, rows * 16, bar);
+        ptx::bulk_load(dst + kLutOffHi, a.hi4 + e / 2, rows * 8, bar);
+        if (kTwo) ptx::bulk_load(dst + kLutOffS2, a.s2 + e / 2, rows * 8, bar);
+        if (block_scales) ptx::bulk_load(dst + kLutOffSc, a.scales + e / 8, rows * 4, bar);  // 2 per row per slice
+        ++k;
       }
-      // Per group of 8 inputs, a power-of-two scale 2^e puts the group's largest |x|
-      // in [2^14, 2^15), so the fp16 MMA operand is exact for any activation type;
-      // the table entries are multiplied by 2^-e before they are stored (exact).
-      float m = fabsf(xv);
-      for (int o = 4; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-      int e = 0;
-      if (m > 0.f && isfinite(m)) {
-        frexpf(m, &e);  // m in [2^(e-1), 2^e)
-        e = min(100, max(-100, 15 - e));
-      }
-      if (tid < 128) {
-        xf[tid] = xv;
-        reinterpret_cast<__half*>(xh)[tid] = __float2half_rn(xv * ldexpf(1.f, e));
-        if ((tid & 7) == 0) gsc[tid >> 3] = ldexpf(1.f, -e);
-      }
-      __syncthreads();
-      if (kTwo) {
-        const int gg = tid >> 4;
-        float acc = 0.f;
+      // Do not leave copies into this CTA's shared memory in flight.
+      for (int i = (k > kLutStages ? k - kLutStages : 0); i < k; ++i)
+        ptx::mbar_wait(full0 + 8 * (i % kLutStages), (i / kLutStages) & 1, err);
+    }
+  } else {
+    // ------------------------------------------------------------ lookups
+    // Codebook operand of the table MMAs, held for the whole kernel: warp w covers
+    // codewords 512w .. 512w+511 in 16 blocks of 32; see the build below.
+    const int g = lane >> 2, c = lane & 3;
+    uint32_t bfrag[16][4];
+    {
+      const uint32_t* cbw = reinterpret_cast<const uint32_t*>(a.cb1);
 #pragma unroll
-        for (int d = 0; d < 8; ++d) acc = fmaf(xf[8 * gg + d], c2v[d], acc);
-        t2[tid] = acc;  // T2[gg][tid & 15], from the unscaled x
-      }
-      {
-        // A = x slice (16 groups x 8 dims, fp16).  Column n of MMA j in block `it`
-        // is codeword base + 8*(n/2) + 2j + (n%2), so lane (g, c) ends with
-        // codewords base+8c .. base+8c+7 of groups g and g+8: one 16-byte store each.
-        const uint32_t a0 = xh[g * 4 + c], a1 = xh[(g + 8) * 4 + c];
-        const float ua = gsc[g], ub = gsc[g + 8];  // undo the groups' power-of-two scales
+      for (int it = 0; it < 16; ++it)
 #pragma unroll
-        for (int it = 0; it < 16; ++it) {
-          const int base = warp * 512 + it * 32;
-          float d[4][4];
+        for (int j = 0; j < 4; ++j)
+          bfrag[it][j] = __ldg(cbw + (size_t)(warp * 512 + it * 32 + 8 * (g >> 1) + 2 * j + (g & 1)) * 4 + c);
+    }
+    float c2v[8];
+    if (kTwo) {
+      const uint4 q = reinterpret_cast<const uint4*>(a.cb2)[tid & 15];
+      const uint32_t w[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            d[j][0] = d[j][1] = d[j][2] = d[j][3] = 0.f;
-            mma_16808_f16(d[j], a0, a1, bfrag[it][j]);
-          }
-          typedef Elt<__nv_bfloat16> B16;
-          const uint4 lo = make_uint4(B16::pack(d[0][0] * ua, d[0][1] * ua), B16::pack(d[1][0] * ua, d[1][1] * ua),
-                                      B16::pack(d[2][0] * ua, d[2][1] * ua), B16::pack(d[3][0] * ua, d[3][1] * ua));
-          const uint4 hi = make_uint4(B16::pack(d[0][2] * ub, d[0][3] * ub), B16::pack(d[1][2] * ub, d[1][3] * ub),
-                                      B16::pack(d[2][2] * ub, d[2][3] * ub), B16::pack(d[3][2] * ub, d[3][3] * ub));
-          *reinterpret_cast<uint4*>(t1 + g * kLutTableBytes + (base + 8 * c) * 2) = lo;
-          *reinterpret_cast<uint4*>(t1 + (g + 8) * kLutTableBytes + (base + 8 * c) * 2) = hi;
-        }
+      for (int p = 0; p < 4; ++p) {
+        const float2 v = f16x2_to_f32x2(w[p]);
+        c2v[2 * p] = v.x;
+        c2v[2 * p + 1] = v.y;
       }
-      __syncthreads();
-      cur = s;
+    }
+    // Everything above reads only the layer's constant inputs; x, y and the
+    // scratch are touched only after the previous kernel completed.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    float xpre[kLutMaxX];
+#pragma unroll
+    for (int i = 0; i < kLutMaxX; ++i) {
+      const int s = s_first + i;
+      xpre[i] = (tid < 128 && s < S) ? Elt<T>::to_f32(xg[(int64_t)s * 128 + tid]) : 0.f;
     }
 
-    // -------------------------------------------------------------- lookups
-    if (!ptx::mbar_wait(bars + 8 * st, (uint32_t)(((u - u0) / kLutStages) & 1), err)) ok = false;
-    const int r0 = ch * kLutUnitRows;
-    const uint32_t sb = ring_base + st * kLutStageBytes;
+    // Every lookup thread walks the same chunk sequence as the producer, so all
+    // of them rebuild the tables at the same chunks (the named barriers below are
+    // reached by all 256 or by none).  After a wait gives up the rest of the walk
+    // skips the waits (the result is then wrong and the error word is set).
+    int cur = -1, s, r0, rows;
+    for (int k = 0; chunks.next(N, s, r0, rows); ++k) {
+      const int st = k % kLutStages;
+      if (*abortf || !ptx::mbar_wait(full0 + 8 * st, (uint32_t)((k / kLutStages) & 1), err)) {
+        ok = false;
+        *abortf = 1;
+      }
+      if (s != cur) {
+        // ------------------------------------------------------------ build
+        asm volatile("bar.sync 1, %0;" ::"n"(kLutConsumers) : "memory");  // everyone is done with the old tables
+        float xv = 0.f;
+        if (tid < 128) {
+          const int i = s - s_first;
+          if (i < kLutMaxX) {
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int lr = tid + 256 * h, r = r0 + lr;
-      if (r >= N) continue;
-      uint4 lo4;
-      uint2 hh, qq = make_uint2(0, 0);
-      uint32_t scw = 0;
-      asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
-                   : "=r"(lo4.x), "=r"(lo4.y), "=r"(lo4.z), "=r"(lo4.w)
-                   : "r"(sb + 16 * lr));
-      asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(hh.x), "=r"(hh.y) : "r"(sb + kLutOffHi + 8 * lr));
-      if (kTwo) asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(qq.x), "=r"(qq.y) : "r"(sb + kLutOffS2 + 8 * lr));
-      if (block_scales) asm volatile("ld.shared.u32 %0, [%1];" : "=r"(scw) : "r"(sb + kLutOffSc + 4 * lr));
-      float blk[2];
-      lookup_row<kTwo>(lo4, hh, qq, t1_base, t2_base, blk);
-      float acc;
-      if (block_scales) {
-        const float2 sc = f16x2_to_f32x2(scw);
-        acc = fmaf(blk[1], sc.y, blk[0] * sc.x);
-      } else {
-        acc = blk[0] + blk[1];  // the per-row scale is applied once, at the reduction
+            for (int kk = 0; kk < kLutMaxX; ++kk)
+              if (kk == i) xv = xpre[kk];
+          } else {
+            xv = Elt<T>::to_f32(xg[(int64_t)s * 128 + tid]);
+          }
+        }
+        // Per group of 8 inputs, a power-of-two scale 2^e puts the group's largest |x|
+        // in [2^14, 2^15), so the fp16 MMA operand is exact for any activation type;
+        // the table entries are multiplied by 2^-e before they are stored (exact).
+        float m = fabsf(xv);
+        for (int o = 4; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        // e = 15 - (exponent of m as frexpf gives it), taken from the bits for
+        // normal m (zero, inf and NaN get no scaling); clamped so 2^e and 2^-e are
+        // normal floats.
+        const int be = (int)(__float_as_uint(m) >> 23);  // biased exponent (sign bit is 0)
+        int e = 0;
+        if (be > 0 && be < 255) {
+          e = min(100, max(-100, 15 - (be - 126)));
+        } else if (be == 0 && m > 0.f) {  // subnormal: rare, take the library route
+          frexpf(m, &e);
+          e = min(100, max(-100, 15 - e));
+        }
+        if (tid < 128) {
+          xf[tid] = xv;
+          reinterpret_cast<__half*>(xh)[tid] = __float2half_rn(xv * __uint_as_float((uint32_t)(127 + e) << 23));
+          if ((tid & 7) == 0) gsc[tid >> 3] = __uint_as_float((uint32_t)(127 - e) << 23);
+        }
+        asm volatile("bar.sync 1, %0;" ::"n"(kLutConsumers) : "memory");
+        if (kTwo) {
+          const int gg = tid >> 4;
+          float acc = 0.f;
+#pragma unroll
+          for (int d = 0; d < 8; ++d) acc = fmaf(xf[8 * gg + d], c2v[d], acc);
+          t2[tid] = acc;  // T2[gg][tid & 15], from the unscaled x
+        }
+        {
+          // A = x slice (16 groups x 8 dims, fp16).  Column n of MMA j in block `it`
+          // is codeword base + 8*(n/2) + 2j + (n%2), so lane (g, c) ends with
+          // codewords base+8c .. base+8c+7 of groups g and g+8: one 16-byte store each.
+          const uint32_t a0 = xh[g * 4 + c], a1 = xh[(g + 8) * 4 + c];
+          const float ua = gsc[g], ub = gsc[g + 8];  // undo the groups' power-of-two scales
+#pragma unroll
+          for (int it = 0; it < 16; ++it) {
+            const int base = warp * 512 + it * 32;
+            float d[4][4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              d[j][0] = d[j][1] = d[j][2] = d[j][3] = 0.f;
+              mma_16808_f16(d[j], a0, a1, bfrag[it][j]);
+            }
+            typedef Elt<__nv_bfloat16> B16;
+            const uint4 lo = make_uint4(B16::pack(d[0][0] * ua, d[0][1] * ua), B16::pack(d[1][0] * ua, d[1][1] * ua),
+                                        B16::pack(d[2][0] * ua, d[2][1] * ua), B16::pack(d[3][0] * ua, d[3][1] * ua));
+            const uint4 hi = make_uint4(B16::pack(d[0][2] * ub, d[0][3] * ub), B16::pack(d[1][2] * ub, d[1][3] * ub),
+                                        B16::pack(d[2][2] * ub, d[2][3] * ub), B16::pack(d[3][2] * ub, d[3][3] * ub));
+            *reinterpret_cast<uint4*>(t1 + g * kLutTableBytes + (base + 8 * c) * 2) = lo;
+            *reinterpret_cast<uint4*>(t1 + (g + 8) * kLutTableBytes + (base + 8 * c) * 2) = hi;
+          }
+        }
+        asm volatile("bar.sync 1, %0;" ::"n"(kLutConsumers) : "memory");
+        cur = s;
       }
-      if (S == 1) {
-        if (!block_scales) acc *= f16_bits_to_f32(a.scales[r]);
-        static_cast<uint16_t*>(a.y)[r] = Elt<T>::from_f32(acc);
-      } else {
-        partial[(int64_t)s * N + r] = acc;
+
+      // -------------------------------------------------------------- lookups
+      const uint32_t sb = ring_base + st * kLutStageBytes;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int lr = tid + 256 * h, r = r0 + lr;
+        if (lr >= rows) continue;
+        uint4 lo4;
+        uint2 hh, qq = make_uint2(0, 0);
+        uint32_t scw = 0;
+        asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                     : "=r"(lo4.x), "=r"(lo4.y), "=r"(lo4.z), "=r"(lo4.w)
+                     : "r"(sb + 16 * lr));
+        asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(hh.x), "=r"(hh.y) : "r"(sb + kLutOffHi + 8 * lr));
+        if (kTwo)
+          asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(qq.x), "=r"(qq.y) : "r"(sb + kLutOffS2 + 8 * lr));
+        if (block_scales) asm volatile("ld.shared.u32 %0, [%1];" : "=r"(scw) : "r"(sb + kLutOffSc + 4 * lr));
+        float blk[2];
+        lookup_row<kTwo>(lo4, hh, qq, t1_base, t2_base, blk);
+        float acc;
+        if (block_scales) {
+          const float2 sc = f16x2_to_f32x2(scw);
+          acc = fmaf(blk[1], sc.y, blk[0] * sc.x);
+        } else {
+          acc = blk[0] + blk[1];  // the per-row scale is applied once, at the reduction
+        }
+        if (S == 1) {
+          if (!block_scales) acc *= f16_bits_to_f32(a.scales[r]);
+          static_cast<uint16_t*>(a.y)[r] = Elt<T>::from_f32(acc);
+        } else {
+          partial[(int64_t)s * N + r] = acc;
+        }
       }
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(empty0 + 8 * st);  // this warp is done with stage st
     }
-    __syncthreads();  // stage `st` is free again
-    if (tid == 0 && u + kLutStages < u1) issue(u + kLutStages);
   }
   if (S == 1) {
+    __syncthreads();
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     return;
   }
 
   // --------------------------------------------------- grid barrier + reduce
+  // The counter only grows: this launch's CTAs take it from a multiple of the
+  // grid size to the next one, so each CTA's target follows from its own ticket.
   __threadfence();
   __syncthreads();
   if (tid == 0) {
-    const uint32_t arrived = atomicAdd(gbar, 1u);
-    if (arrived == gridDim.x - 1) {
-      *reinterpret_cast<volatile uint32_t*>(gbar) = 0u;  // ready for the next forward
-      __threadfence();
-      atomicAdd(gbar + 1, 1u);                           // release this generation
-    } else {
-      const uint64_t t0 = ptx::globaltimer_ns();
-      bool released = false;
-      for (uint32_t i = 0; i < kWaitSpinLimit; ++i) {
-        if (*reinterpret_cast<volatile uint32_t*>(gbar + 1) != gen0) {
-          released = true;
-          break;
-        }
-        if ((i & 255u) == 255u && ptx::globaltimer_ns() - t0 > 1000000000ull) break;
-        __nanosleep(64);
+    unsigned long long* cnt = reinterpret_cast<unsigned long long*>(gbar);
+    unsigned long long old;
+    asm volatile("atom.add.release.gpu.u64 %0, [%1], 1;" : "=l"(old) : "l"(cnt) : "memory");
+    const unsigned long long target = (old / gridDim.x + 1) * gridDim.x;
+    const uint64_t t0 = ptx::globaltimer_ns();
+    bool released = false;
+    for (uint32_t i = 0; i < kWaitSpinLimit; ++i) {
+      unsigned long long v;
+      asm volatile("ld.acquire.gpu.u64 %0, [%1];" : "=l"(v) : "l"(cnt) : "memory");
+      if (v >= target) {
+        released = true;
+        break;
       }
-      if (!released) atomicOr(err, kErrTimeout);
+      if ((i & 63u) == 63u && ptx::globaltimer_ns() - t0 > 1000000000ull) break;
     }
+    if (!released) atomicOr(err, kErrTimeout);
     *flag = ok;
   }
   __syncthreads();
@@ -360,15 +436,16 @@ __global__ void __launch_bounds__(kLutThreads, 1)
 }
 
 struct LutGeom {
-  int S, C, grid;
+  int S, grid;
 };
 
 static LutGeom lut_geom(int N, int K, int num_sms) {
   LutGeom g;
   g.S = K / (8 * kLutGroups);
-  g.C = (N + kLutUnitRows - 1) / kLutUnitRows;
-  const int64_t U = (int64_t)g.S * g.C;
-  g.grid = (int)(U < num_sms ? U : num_sms);
+  // Enough (slice, row) work for every CTA to sweep a few hundred rows.
+  const int64_t rows = (int64_t)g.S * N;
+  const int64_t want = (rows + 255) / 256;
+  g.grid = (int)(want < num_sms ? (want < 1 ? 1 : want) : num_sms);
   return g;
 }
 
@@ -404,7 +481,7 @@ static cudaError_t launch_lut_t(const LayerArgs& a, float* scratch, uint32_t* ti
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, a, g.S > 1 ? scratch : nullptr, tickets, err, g.S, g.C);
+  return cudaLaunchKernelEx(&cfg, kern, a, g.S > 1 ? scratch : nullptr, tickets, err, g.S);
 }
 
 cudaError_t launch_lut(const LayerArgs& a, const Plan&, float* scratch, uint32_t* gbar, uint32_t* err,
