@@ -133,7 +133,12 @@ namespace vq {
 
 bool plan_forward(const vq_linear_desc& d, const DeviceInfo& dev, int M, int forced_path, Plan* out) {
   int path = forced_path;
-  if (path == VQ_PATH_AUTO) path = (M == 1) ? VQ_PATH_LUT : (M <= 16 ? VQ_PATH_GEMV : VQ_PATH_TC);
+  if (path == VQ_PATH_AUTO) {
+    // Measured on B200: from M = 2 the tensor-core path decodes large layers
+    // faster than the warp-MMA GEMV; on small layers both are launch-bound.
+    const bool large = (int64_t)d.N * d.K >= (int64_t(1) << 22);
+    path = (M == 1) ? VQ_PATH_LUT : ((M <= 16 && !large) ? VQ_PATH_GEMV : VQ_PATH_TC);
+  }
   switch (path) {
     case VQ_PATH_LUT:
       if (plan_lut(d, dev, M, out)) return true;

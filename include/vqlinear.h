@@ -85,12 +85,15 @@ enum {
 /* Element types of x / y / materialised weights. */
 enum { VQ_F16 = 0, VQ_BF16 = 1 };
 
-/* Kernel choice for vq_linear_set_path (VQ_PATH_AUTO picks by M). */
+/* Kernel choice for vq_linear_set_path.  VQ_PATH_AUTO picks by M and layer size:
+ * M == 1 -> VQ_PATH_LUT where it applies (12-bit formats, K % 128 == 0, N % 4 == 0),
+ * else VQ_PATH_GEMV; 2 <= M <= 16 -> VQ_PATH_TC for layers of at least 2^22 weights,
+ * else VQ_PATH_GEMV; M >= 17 -> VQ_PATH_TC. */
 enum {
   VQ_PATH_AUTO = 0,
   VQ_PATH_LUT = 1,    /* M == 1 only: per-group x.codebook tables in shared memory */
   VQ_PATH_GEMV = 2,   /* 1 <= M <= 16: decode to registers, warp MMA, split-K */
-  VQ_PATH_TC = 3      /* any M: decode to shared memory, tcgen05 MMA into TMEM */
+  VQ_PATH_TC = 3      /* any M: decode into tensor memory, tcgen05 MMA (fp32 in TMEM) */
 };
 
 typedef struct {

@@ -240,7 +240,7 @@ def _sampled_forward_check(oracle, layer, act, M, path, nrows=192, seed=0):
     return assert_y_within(y[:, rows], act, y_ref, tol, what=f"{spec} M={M}", strict=True)
 
 
-@pytest.mark.parametrize("M", [1, 4, 16])
+@pytest.mark.parametrize("M", [1, 2, 4, 16])
 def test_llama3_8b_mlp_sampled(oracle, M):
     for label, spec in CONFIGS[4]["tensors"]:
         layer = make_layer(spec, cfg_id=4, tensor_id={"gate": 0, "up": 1, "down": 2}[label])
