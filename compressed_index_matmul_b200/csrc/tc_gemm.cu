@@ -14,13 +14,14 @@
 //   warp 1     allocates TMEM; lane 0 issues tcgen05.mma (M=128, N=T, K=16, four
 //              per k block, A read from TMEM) and commits each stage back.
 //   warps 2-17 decode: four warps per TMEM lane quarter; thread = one row of the
-//              tile (its TMEM lane) and 4 consecutive groups of each slice, which
-//              lie in one of the slice's two k blocks (so each A stage is written
-//              by 8 warps).  Per slice it reads its index bytes from the staged
-//              slice, gathers the stage-1 codewords from shared memory and the
-//              stage-2 codewords from the warp's registers (shuffle), decodes with
-//              the materialised-weight rounding and stores the 32 weights into
-//              its own TMEM lane of the stage's A columns (tcgen05.st).
+//              tile (its TMEM lane); warp `part` of a quarter decodes every 4th k
+//              block (kb % 4 == part), all 8 groups of it, so A stage `part` is
+//              always written by the same 4 warps.  Per block a thread reads its 8
+//              index bytes (plus nibbles and scale) from the staged slice, gathers
+//              the stage-1 codewords from shared memory and the stage-2 codewords
+//              from the warp's registers (shuffle), decodes with the
+//              materialised-weight rounding and stores the 64 weights into its
+//              own TMEM lane of the stage's A columns (tcgen05.st).
 //              After the last block the same threads read the accumulator from
 //              TMEM and write y (or fp32 split-K partials; the last CTA of a tile,
 //              by an atomic ticket, sums the partials in split order).
@@ -159,13 +160,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kTcStages; ++s) {
-      ptx::mbar_init(full_a(s), kTcDecodeWarps / 2);  // the 8 decode warps of this block's parity
+      ptx::mbar_init(full_a(s), 4);  // one decode warp per TMEM lane quarter
       ptx::mbar_init(full_b(s), 1);               // the producer's expect_tx arrival (+ bytes)
       ptx::mbar_init(empty(s), 1);                // one tcgen05.commit
     }
     for (int s = 0; s < kTcIdxSlots; ++s) {
       ptx::mbar_init(idx_full(s), 1);
-      ptx::mbar_init(idx_empty(s), kTcDecodeWarps);
+      ptx::mbar_init(idx_empty(s), kTcDecodeWarps / 2);  // the 8 warps that decode the slice's two blocks
     }
     ptx::mbar_init(accum_bar, 1);
     ptx::mbar_init(cb_bar, 1);
@@ -219,9 +220,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         ptx::tma_load_2d(b_tile(s), &xmap, kbeg + kb * 64, tok0, full_b(s));
         issued = kb + 1;
         // After x of block kb (odd, >= 5) is issued, refill with slice (kb+3)/2.
-        // Its slot held slice (kb-5)/2, which every decode warp released before it
-        // decoded block kb - 4 or earlier; the stage-empty wait above already saw
-        // MMA kb - 4 (and so every earlier block) complete, so this wait never
+        // Its slot held slice (kb-5)/2, which the warps decoding blocks kb - 5 and
+        // kb - 4 released before decoding them; the stage-empty wait above already
+        // saw MMA kb - 4 (and so every earlier block) complete, so this wait never
         // holds back the x loads.
         if (kStaged && (kb & 1) == 1 && kb >= 5 && (kb + 3) / 2 == issued_idx && issued_idx < nsl) {
           const int j = issued_idx;
@@ -272,102 +273,99 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ decode
-    // Thread (row dr, part) decodes groups 4part .. 4part+3 of every slice: inputs
-    // 32part .. 32part+31 of the slice, i.e. half of k block 2j + part/2, which is
-    // 16 TMEM columns of that block's A stage.
+    // Warp (quarter q, part) decodes every 4th k block, kb = part, part+4, ...: all
+    // 8 groups of the block for its 32 rows, i.e. the whole A stage kb % 4 == part
+    // for its TMEM lane quarter.
     const int q = warp & 3;            // TMEM lane quarter of this warp
-    const int part = (warp - 2) >> 2;  // 0..3
-    const int hsel = part >> 1;        // which k block of each slice
+    const int part = (warp - 2) >> 2;  // 0..3 == the A stage this warp writes
     const int dr = 32 * q + lane;      // row within the tile == TMEM lane
     const int r = row0 + dr;
     const bool valid = r < N;
     const uint4* cbg = reinterpret_cast<const uint4*>(a.cb1);
-    // Stage-2 codebook in registers: lane L holds entry L % 16.
     uint32_t cb2r[4] = {0, 0, 0, 0};
     if (kTwo) {
       const uint4 v = reinterpret_cast<const uint4*>(a.cb2)[lane & 15];
       cb2r[0] = v.x; cb2r[1] = v.y; cb2r[2] = v.z; cb2r[3] = v.w;
     }
     const unsigned short row_scale = (!block_scales && valid) ? a.scales[r] : (unsigned short)0;
-    const uint32_t tlane = tmem + ((uint32_t)(32 * q) << 16) + acol0 + 16u * (uint32_t)(part & 1);
+    const uint32_t tlane = tmem + ((uint32_t)(32 * q) << 16) + acol0 + kTcACols * (uint32_t)part;
     bool ok = true;
     if (kSmemCb && !ptx::mbar_wait(cb_bar, 0, p.err)) {
       *abort_flag = 1;
       ok = false;
     }
-    for (int j = 0; ok && j < nsl; ++j) {
-      const int kb = 2 * j + hsel;
-      if (kb >= nkb) {
-        // A 64-wide last slice has no odd block: this warp has nothing to decode
-        // there, but it still releases the slice's index slot.
-        if (kStaged && lane == 0) ptx::mbar_arrive(idx_empty(j % kTcIdxSlots));
-        break;
-      }
-      const int s = kb % kTcStages;
+    for (int kb = part; ok && kb < nkb; kb += 4) {
+      const int j = kb >> 1, h = kb & 1;
       const int sl = s_first + j, w = slice_width(sl, G);
-      if (*abort_flag || (kb >= kTcStages && !ptx::mbar_wait(empty(s), ((kb / kTcStages) - 1) & 1, p.err)) ||
+      if (*abort_flag || (kb >= kTcStages && !ptx::mbar_wait(empty(part), ((kb / kTcStages) - 1) & 1, p.err)) ||
           (kStaged && !ptx::mbar_wait(idx_full(j % kTcIdxSlots), (j / kTcIdxSlots) & 1, p.err))) {
         *abort_flag = 1;
         ok = false;
         break;
       }
-      // Index bytes of groups 4part .. 4part+3 of slice sl, this row.
-      uint32_t lo4 = 0, hi2 = 0, s22 = 0;  // 4 lo bytes; 4 packed hi / s2 nibbles
-      uint2 v16 = make_uint2(0, 0);         // 4 idx16 entries
+      uint2 lo8 = make_uint2(0, 0);
+      uint32_t hi4w = 0, s24w = 0;
+      uint4 v16 = make_uint4(0, 0, 0, 0);
       unsigned short sc = row_scale;
       if (valid) {
         if (kStaged) {
           const unsigned char* slot = sm + kTcOffIdx + kTcIdxSlot * (j % kTcIdxSlots);
           if (FMT == kFmtVq16) {
-            v16 = *reinterpret_cast<const uint2*>(slot + (dr * w + 4 * part) * 2);
+            v16 = *reinterpret_cast<const uint4*>(slot + (dr * w + 8 * h) * 2);
           } else {
-            lo4 = *reinterpret_cast<const uint32_t*>(slot + kTcIdxLo + dr * w + 4 * part);
-            hi2 = *reinterpret_cast<const uint16_t*>(slot + kTcIdxHi + dr * (w / 2) + 2 * part);
-            if (kTwo) s22 = *reinterpret_cast<const uint16_t*>(slot + kTcIdxS2 + dr * (w / 2) + 2 * part);
+            lo8 = *reinterpret_cast<const uint2*>(slot + kTcIdxLo + dr * w + 8 * h);
+            hi4w = *reinterpret_cast<const uint32_t*>(slot + kTcIdxHi + dr * (w / 2) + 4 * h);
+            if (kTwo) s24w = *reinterpret_cast<const uint32_t*>(slot + kTcIdxS2 + dr * (w / 2) + 4 * h);
           }
-          if (block_scales) sc = *reinterpret_cast<const uint16_t*>(slot + kTcIdxSc + (dr * (w / 8) + hsel) * 2);
+          if (block_scales) sc = *reinterpret_cast<const uint16_t*>(slot + kTcIdxSc + (dr * (w / 8) + h) * 2);
         } else {
-          const int64_t e = (int64_t)16 * sl * N + (int64_t)r * w + 4 * part;
+          const int64_t e = (int64_t)16 * sl * N + (int64_t)r * w + 8 * h;
           if (FMT == kFmtVq16) {
-            v16 = *reinterpret_cast<const uint2*>(a.idx16 + e);
+            v16 = *reinterpret_cast<const uint4*>(a.idx16 + e);
           } else {
-            lo4 = *reinterpret_cast<const uint32_t*>(a.lo + e);
-            hi2 = *reinterpret_cast<const uint16_t*>(a.hi4 + e / 2);
-            if (kTwo) s22 = *reinterpret_cast<const uint16_t*>(a.s2 + e / 2);
+            lo8 = *reinterpret_cast<const uint2*>(a.lo + e);
+            hi4w = *reinterpret_cast<const uint32_t*>(a.hi4 + e / 2);
+            if (kTwo) s24w = *reinterpret_cast<const uint32_t*>(a.s2 + e / 2);
           }
-          if (block_scales) sc = a.scales[scale_index(r, 128 * sl + 64 * hsel, N, K, a.scale_group)];
+          if (block_scales) sc = a.scales[scale_index(r, 128 * sl + 64 * h, N, K, a.scale_group)];
         }
       }
       if (kStaged) {
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(idx_empty(j % kTcIdxSlots));
       }
-      uint32_t out[16];
       const float scf = kTwo ? __half2float(__ushort_as_half(sc)) : 0.f;
-#pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        uint32_t i1;
-        if (FMT == kFmtVq16)
-          i1 = ((t < 2 ? v16.x : v16.y) >> (16 * (t & 1))) & 0xFFFFu;
-        else
-          i1 = ((lo4 >> (8 * t)) & 0xFFu) | (((hi2 >> (4 * t)) & 15u) << 8);
-        const uint4 c1 = kSmemCb ? cb1s[i1] : __ldg(cbg + i1);
-        if (kTwo) {
-          const int i2 = (int)((s22 >> (4 * t)) & 15u);
-          uint32_t c2[4];
-#pragma unroll
-          for (int w4 = 0; w4 < 4; ++w4) c2[w4] = __shfl_sync(0xffffffffu, cb2r[w4], i2);
-          decode_two_stage<T>(c1, c2, scf, out + 4 * t);
-        } else {
-          decode_one_stage<T>(c1, sc, out + 4 * t);
-        }
-      }
       ptx::tc_fence_after();
-      ptx::tmem_st16(tlane + kTcACols * s, out);
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {  // 4 groups (16 TMEM columns) at a time
+        uint32_t out[16];
+        const uint32_t low = c ? lo8.y : lo8.x;
+        const uint32_t v0 = FMT == kFmtVq16 ? (c ? v16.z : v16.x) : 0u, v1 = FMT == kFmtVq16 ? (c ? v16.w : v16.y) : 0u;
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const int g = 4 * c + t;
+          uint32_t i1;
+          if (FMT == kFmtVq16)
+            i1 = ((t < 2 ? v0 : v1) >> (16 * (t & 1))) & 0xFFFFu;
+          else
+            i1 = ((low >> (8 * t)) & 0xFFu) | (((hi4w >> (4 * g)) & 15u) << 8);
+          const uint4 c1 = kSmemCb ? cb1s[i1] : __ldg(cbg + i1);
+          if (kTwo) {
+            const int i2 = (int)((s24w >> (4 * g)) & 15u);
+            uint32_t c2[4];
+#pragma unroll
+            for (int w4 = 0; w4 < 4; ++w4) c2[w4] = __shfl_sync(0xffffffffu, cb2r[w4], i2);
+            decode_two_stage<T>(c1, c2, scf, out + 4 * t);
+          } else {
+            decode_one_stage<T>(c1, sc, out + 4 * t);
+          }
+        }
+        ptx::tmem_st16(tlane + 16u * c, out);
+      }
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(full_a(s));
+      if (lane == 0) ptx::mbar_arrive(full_a(part));
     }
     if (ok && !ptx::mbar_wait(accum_bar, 0, p.err)) *abort_flag = 1;
   }
