@@ -13,12 +13,15 @@ and reported under "detail" (the SmolLM-135M-shaped 30-layer stack at M=1 and
 16, the rotated 16-bit-index layer, batch 16 of the MLP, and M=256 of the
 8192 x 8192 prefill tile on the tensor-core path).
 
-Timing: W untimed warm-up steps; then exactly K steps, each a replay of a CUDA
-graph of the step's forwards, bracketed by CUDA events on the launching stream;
-the L2 cache is flushed between timed steps, outside the events, by writing a
-512 MiB buffer and then reading it back (so L2 is left holding clean lines and
-the timed kernels pay no write-back of the flush).  Barrier + synchronize before and after; the max over ranks
-is reported.  With --gpus N (torchrun) every rank runs an independent replica
+Timing: W untimed warm-up steps; then exactly K steps bracketed by one pair of
+CUDA events on the launching stream.  The steps are replays of CUDA graphs: one
+graph holds a step on each weight copy in turn (whole cycles), single-step
+graphs make up the rest, so K is exact.
+The inputs are larger than L2: the step's weights exist in R device copies
+(R x the step's weight bytes >= 4 x the L2 size) and step k runs on copy k mod R,
+so every timed step reads weights that are not in L2, as the layers of a deep
+model do, while the kernels' own code stays cached.  Barrier + synchronize
+before and after; the max over ranks is reported.  With --gpus N (torchrun) every rank runs an independent replica
 (the layer does not shard here) and ``value`` aggregates all ranks' layers.
 
 ``--impl reference`` times the CPU oracle (oracle/, plain C in fp64) on a bounded
@@ -137,7 +140,7 @@ class ClockSampler:
 class Workload:
     """A workload's layers resident on the GPU plus chained activation buffers."""
 
-    def __init__(self, name, max_M, seed=0):
+    def __init__(self, name, max_M, seed=0, replicas=None):
         import torch
 
         import compressed_index_matmul_b200 as vq
@@ -154,6 +157,15 @@ class Workload:
                 arr = make_layer(spec, cfg_id=w["cfg"], layer=li, tensor_id=ti, seed=seed)
                 L = vq.VQLinear(spec.N, spec.K, spec.fmt, spec.scale_group, self.act, max_M, arr)
                 self.layers.append((f"{li}.{label}", spec, L))
+        # Copies of every layer's device arrays, cycled step by step so that the
+        # weights a step reads are never in L2 (their total is >= 4x the L2 size);
+        # the copies share the handle (forwards run one after another).
+        if replicas is None:
+            l2 = torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size
+            replicas = max(1, -(-4 * l2 // max(1, self.weight_bytes())))
+        self.replicas = [self.layers]
+        for _ in range(1, replicas):
+            self.replicas.append([(name, spec, _clone_layer(L)) for name, spec, L in self.layers])
         self.rht = self.cfg["rht"]
         K0 = self.layers[0][1].K
         self.x0 = torch.from_numpy(make_x(max_M, K0, self.act, cfg_id=w["cfg"], seed=seed).view(np.int16)).cuda() \
@@ -163,14 +175,18 @@ class Workload:
             self.xr = torch.empty_like(self.x0)
         self.outs = {}
 
-    def plan(self, M):
+    def weight_bytes(self):
+        """Bytes of one copy of the step's layer inputs that do not depend on M."""
+        return sum(layer_bytes(spec, 0) for _, spec, _ in self.layers)
+
+    def plan(self, M, replica=0):
         """Forward calls of one step: (layer, input tensor, output tensor) with the stack's chaining."""
         import torch
 
         calls = []
         x = self.xr[:M] if self.rht else self.x0[:M]
         prev_by_width = {}
-        for name, spec, L in self.layers:
+        for name, spec, L in self.replicas[replica]:
             label = name.split(".")[1]
             key = (name, M)
             if key not in self.outs:
@@ -211,65 +227,109 @@ class Workload:
         return sum(2.0 * M * spec.N * spec.K for _, spec, _ in self.layers)
 
 
-class _Flush:
-    """Evicts L2: write a 512 MiB buffer, then read it (leaving clean lines in L2)."""
+def _clone_layer(L):
+    """A VQLinear sharing L's handle but reading its own copy of the device arrays."""
+    import copy
 
-    def __init__(self):
-        import torch
+    from compressed_index_matmul_b200 import _binding as B
 
-        self.buf = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
-
-    def zero_(self):
-        self.buf.zero_()
-        self.buf.sum()
-
-
-def _flush_buffer():
-    return _Flush()
+    c = copy.copy(L)
+    c.t = {k: v.clone() for k, v in L.t.items()}
+    c.planes = B.make_planes(c.t.get("lo"), c.t.get("hi4"), c.t.get("s2"), c.t.get("idx16"))
+    c.codebooks = B.make_codebooks(c.t["cb1"], c.t.get("cb2"))
+    c.close = lambda: None  # the handle belongs to L
+    return c
 
 
-def time_graph(wl, M, steps, warmup, flush, per_kernel=False):
-    """Replay a CUDA graph of one step `steps` times; return per-step ms (and per-forward ms)."""
+L2_NOTE = "inputs larger than L2: the step's weights are cycled over {r} copies ({mb:.0f} MB, >= 4x L2)"
+
+
+def capture_steps(wl, M, stream, evs=None):
+    """One CUDA graph per weight copy, each holding one step's forwards."""
+    import torch
+
+    graphs = []
+    for r in range(len(wl.replicas)):
+        calls = wl.plan(M, r)
+        with torch.cuda.stream(stream):
+            wl.enqueue(calls, M)  # plain run: every call validated outside capture
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream, capture_error_mode="relaxed"):
+            wl.enqueue(calls, M, evs)
+        graphs.append(g)
+    return graphs
+
+
+def capture_cycle(wl, M, stream):
+    """One CUDA graph holding one step on each weight copy in turn (R steps back to back)."""
+    import torch
+
+    g = torch.cuda.CUDAGraph()
+    plans = [wl.plan(M, r) for r in range(len(wl.replicas))]
+    with torch.cuda.graph(g, stream=stream, capture_error_mode="relaxed"):
+        for calls in plans:
+            wl.enqueue(calls, M)
+    return g
+
+
+def run_steps(graphs, cycle, first, steps, stream):
+    """Enqueue exactly `steps` steps starting at step index `first`: whole cycles by the
+    cycle graph where they line up, single-step graphs for the rest."""
+    R = len(graphs)
+    k = first
+    end = first + steps
+    while k < end:
+        if k % R == 0 and end - k >= R:
+            cycle.replay()
+            k += R
+        else:
+            graphs[k % R].replay()
+            k += 1
+
+
+def time_graph(wl, M, steps, warmup, per_kernel=False):
+    """Replay the step graphs `steps` times (cycling the weight copies); per-step ms (and per-forward ms)."""
     import torch
 
     stream = torch.cuda.Stream()
-    calls = wl.plan(M)
-    n = len(calls)
+    n = len(wl.plan(M))
     evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n + 1)] if per_kernel else None
-    with torch.cuda.stream(stream):
-        wl.enqueue(calls, M)  # plain run: every call validated outside capture
-    stream.synchronize()
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g, stream=stream, capture_error_mode="relaxed"):
-        wl.enqueue(calls, M, evs)
-    start = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
-    end = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    graphs = capture_steps(wl, M, stream, evs)
+    R = len(graphs)
     per_fwd = np.zeros(n) if per_kernel else None
-    with torch.cuda.stream(stream):
-        for _ in range(warmup):
-            flush.zero_()
-            g.replay()
-        stream.synchronize()
-        for k in range(steps):
-            flush.zero_()
-            start[k].record(stream)
-            g.replay()
-            end[k].record(stream)
-            if per_kernel:
+    if per_kernel:  # one step at a time, events between the forwards
+        with torch.cuda.stream(stream):
+            for k in range(warmup):
+                graphs[k % R].replay()
+            stream.synchronize()
+            for k in range(steps):
+                graphs[(warmup + k) % R].replay()
                 stream.synchronize()
                 per_fwd += np.array([evs[i].elapsed_time(evs[i + 1]) for i in range(n)])
+        del graphs
+        return None, per_fwd / steps
+    cycle = capture_cycle(wl, M, stream)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        run_steps(graphs, cycle, 0, warmup, stream)
+        stream.synchronize()
+        t0.record(stream)
+        run_steps(graphs, cycle, warmup, steps, stream)
+        t1.record(stream)
     stream.synchronize()
-    ms = [start[k].elapsed_time(end[k]) for k in range(steps)]
-    del g
-    return ms, (per_fwd / steps if per_kernel else None)
+    total = t0.elapsed_time(t1)
+    del graphs, cycle
+    return [total / steps] * steps, None
 
 
-def time_e2e(wl, M, steps, warmup, flush):
+def time_e2e(wl, M, steps, warmup):
     """Public API end to end: pinned-host x -> device, eager vq_linear_forward calls, y -> pinned host."""
     import torch
 
     stream = torch.cuda.Stream()
-    calls = wl.plan(M)
+    plans = [wl.plan(M, r) for r in range(len(wl.replicas))]
+    calls = plans[0]
     src = wl.x0[:M]
     host_x = torch.empty(src.shape, dtype=src.dtype, pin_memory=True)
     host_x.copy_(src.cpu())
@@ -279,7 +339,7 @@ def time_e2e(wl, M, steps, warmup, flush):
     ms = []
     with torch.cuda.stream(stream):
         for k in range(warmup + steps):
-            flush.zero_()
+            calls = plans[k % len(plans)]
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
             e0.record(stream)
@@ -293,8 +353,8 @@ def time_e2e(wl, M, steps, warmup, flush):
     return ms, host_x.numel() * host_x.element_size(), host_y.numel() * host_y.element_size()
 
 
-def measure(wl, M, steps, warmup, flush, peaks, with_kernels=True):
-    ms, per_fwd = time_graph(wl, M, steps, warmup, flush, per_kernel=False)
+def measure(wl, M, steps, warmup, peaks, with_kernels=True):
+    ms, per_fwd = time_graph(wl, M, steps, warmup, per_kernel=False)
     res = {"M": M, "ms_per_step": statistics.fmean(ms), "layers_per_step": len(wl.layers)}
     res["us_per_layer"] = 1e3 * res["ms_per_step"] / len(wl.layers)
     b = wl.bytes_per_step(M)
@@ -303,7 +363,7 @@ def measure(wl, M, steps, warmup, flush, peaks, with_kernels=True):
     res["hbm_frac"] = res["hbm_gbs"] / peaks["hbm_gbs"]
     res["tflops"] = wl.flops_per_step(M) / (res["ms_per_step"] * 1e-3) / 1e12
     if with_kernels:
-        _, per_fwd = time_graph(wl, M, max(5, min(steps, 50)), 2, flush, per_kernel=True)
+        _, per_fwd = time_graph(wl, M, max(5, min(steps, 50)), 2, per_kernel=True)
         res["per_forward_us"] = [float(1e3 * v) for v in per_fwd]
     return res
 
@@ -329,25 +389,17 @@ def gpu_arm(args):
         dist.barrier()
     vq.load()
     peaks, peak_src = load_peaks()
-    flush = _flush_buffer()
     M = args.batch
     wl = Workload(args.workload, max_M=max(M, 16))
-    calls = wl.plan(M)
+    R = len(wl.replicas)
 
     # ------------------------------------------------ timed region (exactly K steps)
     stream = torch.cuda.Stream()
+    graphs = capture_steps(wl, M, stream)
+    cycle = capture_cycle(wl, M, stream)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
-        wl.enqueue(calls, M)
-    stream.synchronize()
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g, stream=stream, capture_error_mode="relaxed"):
-        wl.enqueue(calls, M)
-    start = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    end = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    with torch.cuda.stream(stream):
-        for _ in range(args.warmup):
-            flush.zero_()
-            g.replay()
+        run_steps(graphs, cycle, 0, args.warmup, stream)
     stream.synchronize()
     if world > 1:
         dist.barrier()
@@ -357,47 +409,56 @@ def gpu_arm(args):
     smi_index = int(ids[local]) if local < len(ids) and ids[local].strip().isdigit() else local
     with ClockSampler(smi_index) as clk:
         with torch.cuda.stream(stream):
-            for k in range(args.steps):
-                flush.zero_()
-                start[k].record(stream)
-                g.replay()
-                end[k].record(stream)
+            t0.record(stream)
+            run_steps(graphs, cycle, args.warmup, args.steps, stream)
+            t1.record(stream)
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    del g
-    step_ms = [start[k].elapsed_time(end[k]) for k in range(args.steps)]
+    del graphs, cycle
+    step_ms = [t0.elapsed_time(t1) / args.steps] * args.steps
     layers = len(wl.layers)
     ms_per_step, us_per_layer = aggregate_over_ranks(float(sum(step_ms)), args.steps, layers, world)
 
     # ------------------------------------------------ per-kernel roofline (same stream, graph nodes)
-    _, per_fwd = time_graph(wl, M, min(args.steps, 200), 3, flush, per_kernel=True)
+    _, per_fwd = time_graph(wl, M, min(args.steps, 200), 3, per_kernel=True)
     launches_per_fwd = [L.launches(M) for _, _, L in wl.layers]
     bytes_per_fwd = [layer_bytes(spec, M) for _, spec, _ in wl.layers]
-    achieved = sum(bytes_per_fwd) / (sum(per_fwd) * 1e-3) / 1e9
+    # When every launch of the timed region is one forward of the dominant kernel,
+    # the region's time per launch is that kernel's average launch duration; else
+    # use the event nodes captured between the forwards (which include the gaps).
+    uniform = (not wl.rht) and all(n == 1 for n in launches_per_fwd)
+    fwd_ms = ms_per_step / len(wl.layers) if uniform else float(np.mean(per_fwd))
+    per_fwd_eff = [fwd_ms] * len(wl.layers) if uniform else list(per_fwd)
+    achieved = sum(bytes_per_fwd) / (sum(per_fwd_eff) * 1e-3) / 1e9
     dominant = "lut_gemv_kernel" if (M == 1 and wl.layers[0][1].fmt != FMT_VQ16) else (
         "gemv_kernel" if M <= 16 else "tc_gemm_kernel")
     traffic = lookup_traffic(dominant, args.workload, M)
-    avg_launch_us = round(1e3 * float(np.mean(per_fwd)) / max(1, np.mean(launches_per_fwd)), 3)
+    avg_launch_us = round(1e3 * float(np.mean(per_fwd_eff)) / max(1, np.mean(launches_per_fwd)), 3)
+    launch_source = ("timed region / launches (every launch is this kernel)" if uniform
+                     else "CUDA event nodes between the forwards")
     if dominant == "tc_gemm_kernel":
         # a dense contraction: 2*M*N*K flops per forward against the bf16 tensor peak
         flops_per_fwd = [2.0 * M * spec.N * spec.K for _, spec, _ in wl.layers]
-        tflops = sum(flops_per_fwd) / (sum(per_fwd) * 1e-3) / 1e12
+        tflops = sum(flops_per_fwd) / (sum(per_fwd_eff) * 1e-3) / 1e12
         roofline = {"bound": "tensor", "achieved": round(tflops, 1), "peak": peaks["bf16_tflops"],
                     "unit": "TFLOP/s", "frac": round(tflops / peaks["bf16_tflops"], 4), "traffic": traffic,
                     "kernel": dominant, "peak_source": f"{peak_src} bf16_tflops (burst)",
                     "frac_of_sustained": round(tflops / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]), 4),
-                    "avg_launch_us": avg_launch_us, "algorithmic_flops_per_launch": int(np.mean(flops_per_fwd))}
+                    "avg_launch_us": avg_launch_us, "launch_time_from": launch_source,
+                    "event_node_us": round(1e3 * float(np.mean(per_fwd)), 3),
+                    "algorithmic_flops_per_launch": int(np.mean(flops_per_fwd))}
     else:
         roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                     "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,
                     "kernel": dominant, "peak_source": f"{peak_src} hbm_gbs",
-                    "avg_launch_us": avg_launch_us,
+                    "avg_launch_us": avg_launch_us, "launch_time_from": launch_source,
+                    "event_node_us": round(1e3 * float(np.mean(per_fwd)), 3),
                     "algorithmic_bytes_per_launch": int(np.mean(bytes_per_fwd))}
 
     # ------------------------------------------------ end to end through the public API
-    e2e_ms, h2d, d2h = time_e2e(wl, M, min(args.steps, 200), 3, flush)
+    e2e_ms, h2d, d2h = time_e2e(wl, M, min(args.steps, 200), 3)
     e2e = {"value": round(1e3 * statistics.fmean(e2e_ms) / layers, 3), "unit": "us/layer",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
@@ -410,7 +471,7 @@ def gpu_arm(args):
                    "shapes": [[spec.N, spec.K] for _, spec, _ in wl.layers[:7]],
                    "format": "rvq12_4 block-64" if args.workload != "vq16-4096-rht" else "vq16 per-row",
                    "parallelism": f"replicas x{world}",
-                   "l2": "flushed between timed steps (512 MiB write then read)",
+                   "l2": L2_NOTE.format(r=R, mb=R * wl.weight_bytes() / 1e6),
                    "layer": "one vq_linear_forward (one weight matrix)",
                    "hbm_gbs": round(sum(bytes_per_fwd) / (ms_per_step * 1e-3) / 1e9, 1)},
         "roofline": roofline,
@@ -421,7 +482,7 @@ def gpu_arm(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(args.workload, M, budget_s=args.cpu_seconds)
     if rank == 0 and not args.no_detail:
-        out["detail"] = detail(args, peaks, flush, wl)
+        out["detail"] = detail(args, peaks, wl)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -472,18 +533,18 @@ def lookup_traffic(kernel, workload, M):
     return e.get("dram_bytes_per_launch")
 
 
-def detail(args, peaks, flush, main_wl):
+def detail(args, peaks, main_wl):
     """The rest of the metric: batch 16 of the headline workload and the other workloads."""
     steps = max(10, min(args.steps, 300))
     res = {}
-    r = measure(main_wl, 16, steps, 3, flush, peaks)
+    r = measure(main_wl, 16, steps, 3, peaks)
     res[f"{args.workload} M=16"] = r
     for name, Ms in (("smollm-135m-stack", (1, 16)), ("vq16-4096-rht", (1, 8))):
         if name == args.workload:
             continue
         wl = Workload(name, max_M=16)
         for M in Ms:
-            r = measure(wl, M, steps, 3, flush, peaks, with_kernels=(name != "smollm-135m-stack"))
+            r = measure(wl, M, steps, 3, peaks, with_kernels=(name != "smollm-135m-stack"))
             if name == "smollm-135m-stack":
                 r["us_per_transformer_layer"] = 1e3 * r["ms_per_step"] / 30
             res[f"{name} M={M}"] = r
@@ -491,7 +552,7 @@ def detail(args, peaks, flush, main_wl):
     try:
         wl = Workload("prefill-8192", max_M=256)
         wl.plan(256)
-        r = measure(wl, 256, max(5, steps // 10), 2, flush, peaks, with_kernels=False)
+        r = measure(wl, 256, max(5, steps // 10), 2, peaks, with_kernels=False)
         r["tensor_frac"] = r["tflops"] / peaks["bf16_tflops"]
         r["tensor_frac_sustained"] = r["tflops"] / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
         res["prefill-8192 M=256"] = r
