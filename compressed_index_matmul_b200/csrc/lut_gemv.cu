@@ -11,8 +11,9 @@
 // gathering and decoding 8-wide codewords.  T1 is a small matrix product
 // (16 groups x 8 dims times 8 dims x 4096 codewords) built on the tensor cores
 // with mma.sync m16n8k8 (fp16 in, fp32 accumulate).  The codebook operand of
-// those MMAs does not depend on x, so each warp loads its share of it into
-// registers once and every rebuild is only MMAs and stores.
+// those MMAs does not depend on x: the codebook is bulk-copied once into the table
+// area (free until the first build), each warp takes its share into registers with
+// ldmatrix, and every rebuild is only MMAs and stores.
 //
 // Work distribution: the (K-slice, row) pairs in slice-major order are cut into
 // one contiguous, equal range per CTA of a persistent grid (at most one CTA per
@@ -170,6 +171,7 @@ __global__ void __launch_bounds__(kLutThreads, 1)
   const uint32_t full0 = smem_u32(smem + kLutOffMisc + 64);         // [kLutStages] mbarriers: chunk landed
   const uint32_t empty0 = smem_u32(smem + kLutOffMisc + 96);        // [kLutStages] mbarriers: chunk consumed
   volatile int* abortf = reinterpret_cast<volatile int*>(smem + kLutOffMisc + 128);  // a bounded wait gave up
+  const uint32_t cb_bar = smem_u32(smem + kLutOffMisc + 136);       // codebook copy landed
   volatile int* flag = reinterpret_cast<volatile int*>(smem + kLutOffMisc + 192);
   const uint32_t t1_base = smem_u32(t1), t2_base = smem_u32(t2), ring_base = smem_u32(smem + kLutOffRing);
 
@@ -186,6 +188,7 @@ __global__ void __launch_bounds__(kLutThreads, 1)
       ptx::mbar_init(full0 + 8 * i, 1);
       ptx::mbar_init(empty0 + 8 * i, kLutConsumers / 32);
     }
+    ptx::mbar_init(cb_bar, 1);
     *abortf = 0;
     ptx::fence_barrier_init();
   }
@@ -197,6 +200,10 @@ __global__ void __launch_bounds__(kLutThreads, 1)
     // Reads only the layer's constant index planes and scales, so it may run
     // while the previous kernel in the stream is still finishing.
     if (lane == 0) {
+      // The stage-1 codebook into the table area (free until the first build),
+      // where the lookup warps read their MMA operands from it.
+      ptx::mbar_arrive_expect_tx(cb_bar, 65536u);
+      ptx::bulk_load(t1_base, a.cb1, 65536u, cb_bar);
       int k = 0, cs, cr, rows;
       while (chunks.next(N, cs, cr, rows)) {
         const int st = k % kLutStages;
@@ -216,6 +223,7 @@ __global__ void __launch_bounds__(kLutThreads, 1)
       // Do not leave copies into this CTA's shared memory in flight.
       for (int i = (k > kLutStages ? k - kLutStages : 0); i < k; ++i)
         ptx::mbar_wait(full0 + 8 * (i % kLutStages), (i / kLutStages) & 1, err);
+      ptx::mbar_wait(cb_bar, 0, err);
     }
   } else {
     // ------------------------------------------------------------ lookups
@@ -224,12 +232,20 @@ __global__ void __launch_bounds__(kLutThreads, 1)
     const int g = lane >> 2, c = lane & 3;
     uint32_t bfrag[16][4];
     {
-      const uint32_t* cbw = reinterpret_cast<const uint32_t*>(a.cb1);
+      // ldmatrix: lanes 8j..8j+7 give the rows (codewords) of matrix j; lane (g, c)
+      // receives word c of row g of each matrix, the MMA B fragment.
+      if (!ptx::mbar_wait(cb_bar, 0, err)) {
+        ok = false;
+        *abortf = 1;
+      }
+      const int n = lane & 7, jm = lane >> 3;
 #pragma unroll
-      for (int it = 0; it < 16; ++it)
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          bfrag[it][j] = __ldg(cbw + (size_t)(warp * 512 + it * 32 + 8 * (g >> 1) + 2 * j + (g & 1)) * 4 + c);
+      for (int it = 0; it < 16; ++it) {
+        const uint32_t addr = t1_base + (uint32_t)(warp * 512 + it * 32 + 8 * (n >> 1) + 2 * jm + (n & 1)) * 16u;
+        asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                     : "=r"(bfrag[it][0]), "=r"(bfrag[it][1]), "=r"(bfrag[it][2]), "=r"(bfrag[it][3])
+                     : "r"(addr));
+      }
     }
     float c2v[8];
     if (kTwo) {
