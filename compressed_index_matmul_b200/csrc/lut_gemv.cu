@@ -230,6 +230,28 @@ __global__ void __launch_bounds__(kLutThreads, 1)
     // Codebook operand of the table MMAs, held for the whole kernel: warp w covers
     // codewords 512w .. 512w+511 in 16 blocks of 32; see the build below.
     const int g = lane >> 2, c = lane & 3;
+    float c2v[8];
+    if (kTwo) {
+      const uint4 q = reinterpret_cast<const uint4*>(a.cb2)[tid & 15];
+      const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        const float2 v = f16x2_to_f32x2(w[p]);
+        c2v[2 * p] = v.x;
+        c2v[2 * p + 1] = v.y;
+      }
+    }
+    // Everything above reads only the layer's constant inputs; x, y and the
+    // scratch are touched only after the previous kernel completed.  The x loads
+    // go out before the wait for the codebook copy, so the two latencies overlap.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    float xpre[kLutMaxX];
+#pragma unroll
+    for (int i = 0; i < kLutMaxX; ++i) {
+      const int s = s_first + i;
+      xpre[i] = (tid < 128 && s < S) ? Elt<T>::to_f32(xg[(int64_t)s * 128 + tid]) : 0.f;
+    }
+
     uint32_t bfrag[16][4];
     {
       // ldmatrix: lanes 8j..8j+7 give the rows (codewords) of matrix j; lane (g, c)
@@ -246,26 +268,6 @@ __global__ void __launch_bounds__(kLutThreads, 1)
                      : "=r"(bfrag[it][0]), "=r"(bfrag[it][1]), "=r"(bfrag[it][2]), "=r"(bfrag[it][3])
                      : "r"(addr));
       }
-    }
-    float c2v[8];
-    if (kTwo) {
-      const uint4 q = reinterpret_cast<const uint4*>(a.cb2)[tid & 15];
-      const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-      for (int p = 0; p < 4; ++p) {
-        const float2 v = f16x2_to_f32x2(w[p]);
-        c2v[2 * p] = v.x;
-        c2v[2 * p + 1] = v.y;
-      }
-    }
-    // Everything above reads only the layer's constant inputs; x, y and the
-    // scratch are touched only after the previous kernel completed.
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    float xpre[kLutMaxX];
-#pragma unroll
-    for (int i = 0; i < kLutMaxX; ++i) {
-      const int s = s_first + i;
-      xpre[i] = (tid < 128 && s < S) ? Elt<T>::to_f32(xg[(int64_t)s * 128 + tid]) : 0.f;
     }
 
     // Every lookup thread walks the same chunk sequence as the producer, so all
