@@ -27,7 +27,7 @@ STATUS_NAMES = {0: "VQ_OK", 1: "VQ_ERR_INVALID_ARG", 2: "VQ_ERR_UNSUPPORTED", 3:
 # Every entry point the header declares (checked by the tests against the .so).
 EXPORTS = ("vq_abi_version", "vq_linear_create", "vq_linear_destroy", "vq_linear_set_path", "vq_linear_forward",
            "vq_linear_forward_noalloc", "vq_linear_launches", "vq_rht_apply", "vq_linear_check", "vq_last_error",
-           "vq_debug_unpack", "vq_debug_dequant")
+           "vq_debug_unpack", "vq_debug_dequant", "vq_debug_wait_timeout")
 
 
 class VQError(RuntimeError):
@@ -83,6 +83,8 @@ def load(path: str | None = None):
         lib.vq_linear_forward_noalloc.restype = st
         lib.vq_linear_forward_noalloc.argtypes = [ctypes.POINTER(vq_linear_desc), P, ctypes.POINTER(vq_planes),
                                                   ctypes.POINTER(vq_codebooks), P, P, I32, P]
+        lib.vq_debug_wait_timeout.restype = st
+        lib.vq_debug_wait_timeout.argtypes = [P, P]
         lib.vq_linear_launches.restype = I32
         lib.vq_linear_launches.argtypes = [P, I32]
         lib.vq_rht_apply.restype = st
@@ -180,3 +182,7 @@ def vq_debug_unpack(h, planes: vq_planes, i1_out, i2_out=None, stream=None) -> N
 def vq_debug_dequant(h, planes: vq_planes, codebooks: vq_codebooks, scales, w_out, wdt, stream=None) -> None:
     _check(load().vq_debug_dequant(h, ctypes.byref(planes), ctypes.byref(codebooks), _ptr(scales), _ptr(w_out),
                                    wdt, _stream(stream)))
+
+
+def vq_debug_wait_timeout(h, stream=None) -> None:
+    _check(load().vq_debug_wait_timeout(h, _stream(stream)))

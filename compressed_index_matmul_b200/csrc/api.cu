@@ -6,6 +6,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <string>
@@ -197,6 +198,11 @@ VQ_API vq_status vq_linear_create(const vq_linear_desc* desc, vq_linear_t* out) 
       if (p.tickets > tickets) tickets = p.tickets;
     }
   }
+  // Test hook: VQ_TEST_FAIL_ALLOC=1 makes the device allocations fail, so callers'
+  // handling of VQ_ERR_NOMEM can be tested without exhausting a shared GPU.
+  const char* fail_alloc = getenv("VQ_TEST_FAIL_ALLOC");
+  if (fail_alloc && fail_alloc[0] == '1')
+    return fail(VQ_ERR_NOMEM, "device allocation refused (VQ_TEST_FAIL_ALLOC=1)");
   vq_linear_s* h = new (std::nothrow) vq_linear_s{};
   if (!h) return fail(VQ_ERR_NOMEM, "host allocation of the handle failed");
   h->d = *desc;
@@ -335,6 +341,15 @@ VQ_API vq_status vq_debug_unpack(vq_linear_t h, const vq_planes* planes, uint16_
   vq::LayerArgs a = make_args(h->d, planes, nullptr, nullptr);
   cudaError_t e = vq::launch_debug_unpack(a, i1_out, i2_out, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "vq_debug_unpack launch");
+  return VQ_OK;
+}
+
+VQ_API vq_status vq_debug_wait_timeout(vq_linear_t h, void* stream) {
+  if (h == nullptr) return fail(VQ_ERR_INVALID_ARG, "handle is NULL");
+  vq_status st;
+  if ((st = check_device(h))) return st;
+  cudaError_t e = vq::launch_debug_wait_timeout(h->err, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "vq_debug_wait_timeout launch");
   return VQ_OK;
 }
 

@@ -3,6 +3,7 @@
 // that materialise unpacked indices / decoded weights into caller buffers.
 #include "common.cuh"
 #include "internal.h"
+#include "tc_ptx.cuh"
 
 namespace vq {
 
@@ -141,6 +142,24 @@ __global__ void debug_dequant_kernel(LayerArgs a, uint16_t* __restrict__ w) {
     }
     reinterpret_cast<uint4*>(w)[t] = make_uint4(out[0], out[1], out[2], out[3]);
   }
+}
+
+// Test of the bounded waits: one thread waits on an mbarrier that nothing
+// arrives on, with the same bounded wait the pipelines use.  It gives up after
+// about a second, records kErrTimeout in *err and the kernel ends normally.
+__global__ void debug_wait_timeout_kernel(uint32_t* err) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    const uint32_t b = smem_u32(&bar);
+    ptx::mbar_init(b, 1);
+    ptx::fence_barrier_init();
+    ptx::mbar_wait(b, 0, err);
+  }
+}
+
+cudaError_t launch_debug_wait_timeout(uint32_t* err, cudaStream_t s) {
+  debug_wait_timeout_kernel<<<1, 32, 0, s>>>(err);
+  return cudaGetLastError();
 }
 
 static int grid_for(int64_t total, int threads) {

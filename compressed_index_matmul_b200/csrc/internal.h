@@ -61,5 +61,6 @@ cudaError_t launch_rht(const void* x, void* x_out, const int8_t* signs, int M, i
                        cudaStream_t s);
 cudaError_t launch_debug_unpack(const LayerArgs& a, uint16_t* i1, uint8_t* i2, cudaStream_t s);
 cudaError_t launch_debug_dequant(const LayerArgs& a, void* w, int wdt, cudaStream_t s);
+cudaError_t launch_debug_wait_timeout(uint32_t* err, cudaStream_t s);
 
 }  // namespace vq

@@ -226,6 +226,15 @@ vq_status vq_debug_unpack(vq_linear_t h, const vq_planes* planes, uint16_t* i1_o
 vq_status vq_debug_dequant(vq_linear_t h, const vq_planes* planes, const vq_codebooks* codebooks,
                            const void* scales, void* w_out, int32_t wdt, void* stream);
 
+/* Test of the failure path of the bounded device-side waits: enqueues one small
+ * kernel that waits on a barrier nothing ever completes, with the same bounded
+ * wait every pipeline kernel uses.  After about a second it gives up, sets the
+ * handle's error flag and ends normally (nothing faults, the context stays
+ * usable); vq_linear_check then returns VQ_ERR_TIMEOUT and clears the flag.
+ * The test hook for allocation failures is the environment variable
+ * VQ_TEST_FAIL_ALLOC=1, which makes vq_linear_create return VQ_ERR_NOMEM. */
+vq_status vq_debug_wait_timeout(vq_linear_t h, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
