@@ -115,22 +115,12 @@ __device__ __forceinline__ void mma_16808_f16(float d[4], uint32_t a0, uint32_t 
       : "r"(a0), "r"(a1), "r"(b0));
 }
 
-__device__ __forceinline__ float lds_bf16(uint32_t addr) {
-  uint16_t v;
-  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
-  return __uint_as_float(uint32_t(v) << 16);
-}
-__device__ __forceinline__ float lds_f32(uint32_t addr) {
-  float v;
-  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
-  return v;
-}
-
 // Sum of the 16 lookups of one row's slice record (lo 16 B, hi4 8 B, s2 8 B),
 // split by 64-input block.
 template <bool kTwo>
-__device__ __forceinline__ void lookup_row(const uint4& lo4, const uint2& h, const uint2& q, uint32_t t1_base,
-                                           uint32_t t2_base, float blk[2]) {
+__device__ __forceinline__ void lookup_row(const uint4& lo4, const uint2& h, const uint2& q,
+                                           const unsigned char* __restrict__ t1, const float* __restrict__ t2,
+                                           float blk[2]) {
   const uint32_t low[4] = {lo4.x, lo4.y, lo4.z, lo4.w};
   const uint32_t hiw[2] = {h.x, h.y};
   const uint32_t s2w[2] = {q.x, q.y};
@@ -146,11 +136,14 @@ __device__ __forceinline__ void lookup_row(const uint4& lo4, const uint2& h, con
       // bytes: lo byte t, hi nibble t, then two zero bytes (sign copies of a nibble byte)
       const uint32_t sel = (uint32_t)(t & 3) | (hsel << 4) | ((8u | hsel) << 8) | ((8u | hsel) << 12);
       const uint32_t i1 = prmt(low[t >> 2], (qq & 1) ? hO : hE, sel);
-      float v = lds_bf16(t1_base + t * kLutTableBytes + i1 * 2);
+      // plain shared-memory loads: the compiler may issue all of a row's lookups
+      // before the additions that consume them
+      float v = __uint_as_float((uint32_t)*reinterpret_cast<const uint16_t*>(t1 + t * kLutTableBytes + i1 * 2) << 16);
       if (kTwo) {
         const uint32_t b = qq >> 1;
         const uint32_t bsel = b | ((8u | b) << 4) | ((8u | b) << 8) | ((8u | b) << 12);
-        v += lds_f32(t2_base + t * 64 + prmt((qq & 1) ? sO : sE, 0, bsel));
+        v += *reinterpret_cast<const float*>(reinterpret_cast<const unsigned char*>(t2) + t * 64 +
+                                             prmt((qq & 1) ? sO : sE, 0, bsel));
       }
       blk[w] += v;
     }
@@ -173,7 +166,7 @@ __global__ void __launch_bounds__(kLutThreads, 1)
   volatile int* abortf = reinterpret_cast<volatile int*>(smem + kLutOffMisc + 128);  // a bounded wait gave up
   const uint32_t cb_bar = smem_u32(smem + kLutOffMisc + 136);       // codebook copy landed
   volatile int* flag = reinterpret_cast<volatile int*>(smem + kLutOffMisc + 192);
-  const uint32_t t1_base = smem_u32(t1), t2_base = smem_u32(t2), ring_base = smem_u32(smem + kLutOffRing);
+  const uint32_t t1_base = smem_u32(t1), ring_base = smem_u32(smem + kLutOffRing);
 
   const int N = a.N;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -353,23 +346,17 @@ __global__ void __launch_bounds__(kLutThreads, 1)
       }
 
       // -------------------------------------------------------------- lookups
-      const uint32_t sb = ring_base + st * kLutStageBytes;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const int lr = tid + 256 * h, r = r0 + lr;
         if (lr >= rows) continue;
-        uint4 lo4;
-        uint2 hh, qq = make_uint2(0, 0);
-        uint32_t scw = 0;
-        asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
-                     : "=r"(lo4.x), "=r"(lo4.y), "=r"(lo4.z), "=r"(lo4.w)
-                     : "r"(sb + 16 * lr));
-        asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(hh.x), "=r"(hh.y) : "r"(sb + kLutOffHi + 8 * lr));
-        if (kTwo)
-          asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(qq.x), "=r"(qq.y) : "r"(sb + kLutOffS2 + 8 * lr));
-        if (block_scales) asm volatile("ld.shared.u32 %0, [%1];" : "=r"(scw) : "r"(sb + kLutOffSc + 4 * lr));
+        const unsigned char* sp = smem + kLutOffRing + st * kLutStageBytes;
+        const uint4 lo4 = *reinterpret_cast<const uint4*>(sp + 16 * lr);
+        const uint2 hh = *reinterpret_cast<const uint2*>(sp + kLutOffHi + 8 * lr);
+        const uint2 qq = kTwo ? *reinterpret_cast<const uint2*>(sp + kLutOffS2 + 8 * lr) : make_uint2(0, 0);
+        const uint32_t scw = block_scales ? *reinterpret_cast<const uint32_t*>(sp + kLutOffSc + 4 * lr) : 0u;
         float blk[2];
-        lookup_row<kTwo>(lo4, hh, qq, t1_base, t2_base, blk);
+        lookup_row<kTwo>(lo4, hh, qq, t1, t2, blk);
         float acc;
         if (block_scales) {
           const float2 sc = f16x2_to_f32x2(scw);
