@@ -25,7 +25,8 @@ STATUS_NAMES = {0: "VQ_OK", 1: "VQ_ERR_INVALID_ARG", 2: "VQ_ERR_UNSUPPORTED", 3:
                 4: "VQ_ERR_NOMEM", 5: "VQ_ERR_TIMEOUT"}
 
 # Every entry point the header declares (checked by the tests against the .so).
-EXPORTS = ("vq_abi_version", "vq_linear_create", "vq_linear_destroy", "vq_linear_set_path", "vq_linear_forward",
+EXPORTS = ("vq_abi_version", "vq_linear_create", "vq_linear_destroy", "vq_linear_set_path", "vq_linear_set_sm_budget",
+           "vq_linear_forward",
            "vq_linear_forward_noalloc", "vq_linear_launches", "vq_rht_apply", "vq_linear_check", "vq_last_error",
            "vq_debug_unpack", "vq_debug_dequant", "vq_debug_wait_timeout")
 
@@ -77,6 +78,8 @@ def load(path: str | None = None):
         lib.vq_linear_destroy.argtypes = [P]
         lib.vq_linear_set_path.restype = st
         lib.vq_linear_set_path.argtypes = [P, I32]
+        lib.vq_linear_set_sm_budget.restype = st
+        lib.vq_linear_set_sm_budget.argtypes = [P, I32]
         lib.vq_linear_forward.restype = st
         lib.vq_linear_forward.argtypes = [P, P, ctypes.POINTER(vq_planes), ctypes.POINTER(vq_codebooks), P, P,
                                           I32, I32, I32, P]
@@ -148,6 +151,10 @@ def vq_linear_destroy(h) -> None:
 
 def vq_linear_set_path(h, path: int) -> None:
     _check(load().vq_linear_set_path(h, path))
+
+
+def vq_linear_set_sm_budget(h, sms: int) -> None:
+    _check(load().vq_linear_set_sm_budget(h, sms))
 
 
 def vq_linear_launches(h, M: int) -> int:

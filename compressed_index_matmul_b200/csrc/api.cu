@@ -30,8 +30,10 @@ struct vq_linear_s {
   size_t scratch_bytes;
   uint32_t* tickets;  // completion counters, zeroed at create, left zero by every forward
   int num_tickets;
-  uint32_t* gbar;     // grid-barrier arrival counter (64-bit, 8-byte aligned; only ever grows)
+  uint32_t* gbar;     // grid-barrier arrival counters, one 64-bit word per grid size 0..num_sms
+                      // (8-byte aligned; each only ever grows by whole grids)
   uint32_t* err;      // device word, set by bounded waits that gave up
+  int sm_budget;      // CTAs of the table kernel (0: every SM)
 };
 
 namespace {
@@ -218,14 +220,16 @@ VQ_API vq_status vq_linear_create(const vq_linear_desc* desc, vq_linear_t* out) 
     }
   }
   h->num_tickets = tickets;
-  const size_t small = sizeof(uint32_t) * (size_t)(4 + tickets);
+  // words: [0] error flag, [1] pad, then (num_sms + 1) 64-bit barrier counters, then tickets
+  const size_t bar_words = 2 * ((size_t)dev.num_sms + 1);
+  const size_t small = sizeof(uint32_t) * (2 + bar_words + (size_t)tickets);
   uint32_t* words = nullptr;
   e = cudaMalloc(&words, small);
   if (e == cudaSuccess) e = cudaMemset(words, 0, small);
   if (e == cudaSuccess) e = cudaDeviceSynchronize();  // the zeroing is complete before any forward
   h->err = words;
-  h->gbar = words + 2;
-  h->tickets = tickets ? words + 4 : nullptr;
+  h->gbar = words ? words + 2 : nullptr;
+  h->tickets = (words && tickets) ? words + 2 + bar_words : nullptr;
   if (e != cudaSuccess) {
     cudaFree(h->scratch);
     cudaFree(words);
@@ -255,6 +259,14 @@ VQ_API vq_status vq_linear_set_path(vq_linear_t h, int32_t path) {
   return VQ_OK;
 }
 
+VQ_API vq_status vq_linear_set_sm_budget(vq_linear_t h, int32_t sms) {
+  if (h == nullptr) return fail(VQ_ERR_INVALID_ARG, "handle is NULL");
+  if (sms < 0 || sms > h->dev.num_sms)
+    return fail(VQ_ERR_INVALID_ARG, "sms=%d outside [0, %d] (0 = every SM)", sms, h->dev.num_sms);
+  h->sm_budget = sms;
+  return VQ_OK;
+}
+
 VQ_API int32_t vq_linear_launches(vq_linear_t h, int32_t M) {
   if (h == nullptr || M < 0 || M > h->d.max_M) return -1;
   if (M == 0) return 0;
@@ -281,6 +293,7 @@ VQ_API vq_status vq_linear_forward(vq_linear_t h, const void* x, const vq_planes
   vq::Plan p{};
   if (!vq::plan_forward(d, h->dev, M, h->path, &p))
     return fail(VQ_ERR_UNSUPPORTED, "path %d cannot run M=%d", h->path, M);
+  if (p.path == VQ_PATH_LUT && h->sm_budget > 0 && p.grid > h->sm_budget) p.grid = h->sm_budget;
   if (p.scratch_bytes > h->scratch_bytes || p.tickets > h->num_tickets)
     return fail(VQ_ERR_UNSUPPORTED, "plan needs %zu scratch bytes / %d tickets, handle has %zu / %d",
                 p.scratch_bytes, p.tickets, h->scratch_bytes, h->num_tickets);
@@ -291,7 +304,7 @@ VQ_API vq_status vq_linear_forward(vq_linear_t h, const void* x, const vq_planes
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e;
   switch (p.path) {
-    case VQ_PATH_LUT: e = vq::launch_lut(a, p, h->scratch, h->gbar, h->err, s); break;
+    case VQ_PATH_LUT: e = vq::launch_lut(a, p, h->scratch, h->gbar, h->err, s); break;  // p.grid CTAs
     case VQ_PATH_TC: e = vq::launch_tc(a, p, h->scratch, h->tickets, h->err, s); break;
     default: e = vq::launch_gemv(a, p, h->scratch, h->tickets, s); break;
   }

@@ -35,6 +35,7 @@ struct Plan {
   int launches;      // kernels enqueued
   size_t scratch_bytes;
   int tickets;       // completion counters needed (zero between forwards)
+  int grid;          // CTAs of the persistent table kernel (VQ_PATH_LUT), else 0
 };
 
 struct DeviceInfo {
@@ -50,8 +51,11 @@ bool plan_forward(const vq_linear_desc& d, const DeviceInfo& dev, int M, int for
 // `tickets` are per-launch completion counters: zero before every forward, and
 // every forward leaves them zero again.
 cudaError_t launch_gemv(const LayerArgs& a, const Plan& p, float* scratch, uint32_t* tickets, cudaStream_t s);
-// `gbar` is the handle's grid-barrier arrival counter: 64 bits, 8-byte aligned,
-// zero at create and only ever incremented (each launch adds its grid size).
+// `gbar` is the handle's array of grid-barrier arrival counters, one 64-bit word
+// per grid size (index = the launch's grid, up to the SM count): zero at create
+// and only ever incremented (each launch adds its grid size to its own word, so
+// every word stays a multiple of its grid size between launches, whatever grid
+// sizes other launches of the handle used).
 cudaError_t launch_lut(const LayerArgs& a, const Plan& p, float* scratch, uint32_t* gbar, uint32_t* err,
                        cudaStream_t s);
 cudaError_t launch_tc(const LayerArgs& a, const Plan& p, float* scratch, uint32_t* tickets, uint32_t* err_flag,

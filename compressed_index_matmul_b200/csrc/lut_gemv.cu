@@ -36,6 +36,8 @@
 // Activations are scaled by a power of two per group of 8 so that every value
 // fits the fp16 MMA whatever the activation type; the table entries are scaled
 // back exactly before they are stored.
+#include <atomic>
+
 #include "common.cuh"
 #include "internal.h"
 #include "tc_ptx.cuh"
@@ -382,12 +384,13 @@ __global__ void __launch_bounds__(kLutThreads, 1)
   }
 
   // --------------------------------------------------- grid barrier + reduce
-  // The counter only grows: this launch's CTAs take it from a multiple of the
-  // grid size to the next one, so each CTA's target follows from its own ticket.
+  // Each grid size has its own counter, which only grows: this launch's CTAs take
+  // it from a multiple of the grid size to the next one, so each CTA's target
+  // follows from its own ticket (also when a CUDA graph replays the launch).
   __threadfence();
   __syncthreads();
   if (tid == 0) {
-    unsigned long long* cnt = reinterpret_cast<unsigned long long*>(gbar);
+    unsigned long long* cnt = reinterpret_cast<unsigned long long*>(gbar) + gridDim.x;
     unsigned long long old;
     asm volatile("atom.add.release.gpu.u64 %0, [%1], 1;" : "=l"(old) : "l"(cnt) : "memory");
     const unsigned long long target = (old / gridDim.x + 1) * gridDim.x;
@@ -407,6 +410,10 @@ __global__ void __launch_bounds__(kLutThreads, 1)
   }
   __syncthreads();
   __threadfence();
+  // Every CTA of this grid has passed the barrier, so all of them are resident:
+  // the next kernel in the stream may launch now and take each SM as its CTA here
+  // exits (it reads x, y and the scratch only after this grid completes).
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   // This CTA's rows; tpr threads per row split the slices, then a fixed xor tree.
   const int rbeg = (int)((int64_t)N * blockIdx.x / gridDim.x), rend = (int)((int64_t)N * (blockIdx.x + 1) / gridDim.x);
   const int nr = rend - rbeg;
@@ -437,7 +444,6 @@ __global__ void __launch_bounds__(kLutThreads, 1)
       static_cast<uint16_t*>(a.y)[r] = Elt<T>::from_f32(sum);
     }
   }
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 struct LutGeom {
@@ -464,20 +470,29 @@ bool plan_lut(const vq_linear_desc& d, const DeviceInfo& dev, int M, Plan* p) {
   p->launches = 1;
   p->scratch_bytes = g.S > 1 ? (size_t)g.S * d.N * sizeof(float) : 0;
   p->tickets = 0;  // uses the handle's grid-barrier words instead
+  p->grid = g.grid;
   return true;
 }
 
 template <int FMT, typename T>
-static cudaError_t launch_lut_t(const LayerArgs& a, float* scratch, uint32_t* tickets, uint32_t* err, cudaStream_t s) {
-  int dev = 0, sms = 0;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const LutGeom g = lut_geom(a.N, a.K, sms);
+static cudaError_t launch_lut_t(const LayerArgs& a, int grid, float* scratch, uint32_t* tickets, uint32_t* err,
+                                cudaStream_t s) {
+  const int S = a.K / (8 * kLutGroups);
   auto kern = lut_gemv_kernel<FMT, T>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kLutSmem);
+  // The shared-memory opt-in is a per-device property of the function: set it
+  // once per device (repeating it from two threads is harmless).
+  static std::atomic<uint64_t> opted{0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
+  const uint64_t bit = dev < 64 ? (uint64_t(1) << dev) : 0;
+  if (!(opted.load(std::memory_order_acquire) & bit)) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kLutSmem);
+    if (e != cudaSuccess) return e;
+    opted.fetch_or(bit, std::memory_order_acq_rel);
+  }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(g.grid);
+  cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kLutThreads);
   cfg.dynamicSmemBytes = kLutSmem;
   cfg.stream = s;
@@ -486,16 +501,16 @@ static cudaError_t launch_lut_t(const LayerArgs& a, float* scratch, uint32_t* ti
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, a, g.S > 1 ? scratch : nullptr, tickets, err, g.S);
+  return cudaLaunchKernelEx(&cfg, kern, a, S > 1 ? scratch : nullptr, tickets, err, S);
 }
 
-cudaError_t launch_lut(const LayerArgs& a, const Plan&, float* scratch, uint32_t* gbar, uint32_t* err,
+cudaError_t launch_lut(const LayerArgs& a, const Plan& p, float* scratch, uint32_t* gbar, uint32_t* err,
                        cudaStream_t s) {
   if (a.fmt == kFmtRvq12_4)
-    return a.act == VQ_BF16 ? launch_lut_t<kFmtRvq12_4, __nv_bfloat16>(a, scratch, gbar, err, s)
-                            : launch_lut_t<kFmtRvq12_4, __half>(a, scratch, gbar, err, s);
-  return a.act == VQ_BF16 ? launch_lut_t<kFmtRvq12, __nv_bfloat16>(a, scratch, gbar, err, s)
-                          : launch_lut_t<kFmtRvq12, __half>(a, scratch, gbar, err, s);
+    return a.act == VQ_BF16 ? launch_lut_t<kFmtRvq12_4, __nv_bfloat16>(a, p.grid, scratch, gbar, err, s)
+                            : launch_lut_t<kFmtRvq12_4, __half>(a, p.grid, scratch, gbar, err, s);
+  return a.act == VQ_BF16 ? launch_lut_t<kFmtRvq12, __nv_bfloat16>(a, p.grid, scratch, gbar, err, s)
+                          : launch_lut_t<kFmtRvq12, __half>(a, p.grid, scratch, gbar, err, s);
 }
 
 }  // namespace vq

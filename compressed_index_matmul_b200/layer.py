@@ -57,6 +57,10 @@ class VQLinear:
     def set_path(self, path: int):
         B.vq_linear_set_path(self.handle, path)
 
+    def set_sm_budget(self, sms: int):
+        """Run the batch-1 table kernel on at most `sms` SMs (0: all of them)."""
+        B.vq_linear_set_sm_budget(self.handle, sms)
+
     def launches(self, M: int) -> int:
         return B.vq_linear_launches(self.handle, M)
 

@@ -138,6 +138,18 @@ vq_status vq_linear_destroy(vq_linear_t h);
  * returns VQ_ERR_UNSUPPORTED. */
 vq_status vq_linear_set_path(vq_linear_t h, int32_t path);
 
+/* Limit the batch-1 table kernel (VQ_PATH_LUT) of this handle to `sms` CTAs, one
+ * per SM; 0 restores the default (every SM).  That kernel keeps all of its CTAs
+ * resident and meets them at a grid barrier, so it can share the GPU with another
+ * forward only on disjoint SMs: two independent forwards (say the gate and up
+ * projections of an MLP, both reading the same x) may run concurrently on two
+ * streams when the sum of their budgets does not exceed the SM count.  With a
+ * larger sum the barrier's bounded wait can give up (VQ_ERR_TIMEOUT from
+ * vq_linear_check; y is then not valid).  The other kernels are not persistent
+ * and ignore the budget.  Returns VQ_ERR_INVALID_ARG when `sms` is negative or
+ * above the device's SM count. */
+vq_status vq_linear_set_sm_budget(vq_linear_t h, int32_t sms);
+
 /* y = x . W^T with W decoded on the fly from planes / codebooks / scales
  * (GLQ README, "Inference kernels"; orka README, "How it works" for the decode).
  *   x [M][K] and y [M][N] have the handle's act_dtype; y is overwritten (no bias,

@@ -74,6 +74,7 @@ def test_null_arguments_are_rejected(lib):
     assert lib.vq_linear_create(None, None) == B.VQ_ERR_INVALID_ARG
     assert lib.vq_linear_forward(None, None, None, None, None, None, 1, 1, 1, None) == B.VQ_ERR_INVALID_ARG
     assert lib.vq_linear_set_path(None, 0) == B.VQ_ERR_INVALID_ARG
+    assert lib.vq_linear_set_sm_budget(None, 0) == B.VQ_ERR_INVALID_ARG
     assert lib.vq_linear_launches(None, 1) == -1
     assert lib.vq_linear_destroy(None) == B.VQ_OK
     assert lib.vq_linear_check(None, None) == B.VQ_ERR_INVALID_ARG
