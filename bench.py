@@ -425,19 +425,27 @@ def gpu_arm(args):
     _, per_fwd = time_graph(wl, M, min(args.steps, 200), 3, per_kernel=True)
     launches_per_fwd = [L.launches(M) for _, _, L in wl.layers]
     bytes_per_fwd = [layer_bytes(spec, M) for _, spec, _ in wl.layers]
-    # When every launch of the timed region is one forward of the dominant kernel,
-    # the region's time per launch is that kernel's average launch duration; else
+    # When every forward of the timed region runs the same kernels (no rotation
+    # launch), the region's time per forward is a forward's average duration; else
     # use the event nodes captured between the forwards (which include the gaps).
-    uniform = (not wl.rht) and all(n == 1 for n in launches_per_fwd)
+    # The batch-1 table path is two kernels per forward (lookups, then the split-K
+    # reduction) that overlap by programmatic dependent launch, so the forward,
+    # not either kernel alone, is the unit its bytes are divided by.
+    uniform = (not wl.rht) and len(set(launches_per_fwd)) == 1
     fwd_ms = ms_per_step / len(wl.layers) if uniform else float(np.mean(per_fwd))
     per_fwd_eff = [fwd_ms] * len(wl.layers) if uniform else list(per_fwd)
     achieved = sum(bytes_per_fwd) / (sum(per_fwd_eff) * 1e-3) / 1e9
-    dominant = "lut_gemv_kernel" if (M == 1 and wl.layers[0][1].fmt != FMT_VQ16) else (
-        "gemv_kernel" if M <= 16 else "tc_gemm_kernel")
+    lut = M == 1 and wl.layers[0][1].fmt != FMT_VQ16
+    dominant = "lut_gemv_kernel" if lut else ("gemv_kernel" if M <= 16 else "tc_gemm_kernel")
     traffic = lookup_traffic(dominant, args.workload, M)
-    avg_launch_us = round(1e3 * float(np.mean(per_fwd_eff)) / max(1, np.mean(launches_per_fwd)), 3)
-    launch_source = ("timed region / launches (every launch is this kernel)" if uniform
-                     else "CUDA event nodes between the forwards")
+    avg_launch_us = round(1e3 * float(np.mean(per_fwd_eff)), 3)
+    if not uniform:
+        launch_source = "CUDA event nodes between the forwards"
+    elif launches_per_fwd[0] == 1:
+        launch_source = "timed region / launches (every launch is this kernel)"
+    else:
+        launch_source = ("timed region / forwards (one forward = lut_gemv_kernel + lut_reduce_kernel, "
+                         "overlapped by programmatic dependent launch)")
     if dominant == "tc_gemm_kernel":
         # a dense contraction: 2*M*N*K flops per forward against the bf16 tensor peak
         flops_per_fwd = [2.0 * M * spec.N * spec.K for _, spec, _ in wl.layers]
@@ -454,6 +462,7 @@ def gpu_arm(args):
                     "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,
                     "kernel": dominant, "peak_source": f"{peak_src} hbm_gbs",
                     "avg_launch_us": avg_launch_us, "launch_time_from": launch_source,
+                    "launches_per_forward": launches_per_fwd[0],
                     "event_node_us": round(1e3 * float(np.mean(per_fwd)), 3),
                     "algorithmic_bytes_per_launch": int(np.mean(bytes_per_fwd))}
 

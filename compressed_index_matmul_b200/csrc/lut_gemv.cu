@@ -33,9 +33,10 @@
 // split-K reduction, no floating-point atomics), so y does not depend on
 // scheduling.  One launch per forward.
 //
-// Activations are scaled by a power of two per group of 8 so that every value
-// fits the fp16 MMA whatever the activation type; the table entries are scaled
-// back exactly before they are stored.
+// Activations are scaled by one power of two per K-slice (the slice's largest
+// |x| lands in [2^14, 2^15)), so the fp16 MMA operand is exact for either
+// activation type except for values more than 2^31 below that maximum; the
+// factor is undone once per (slice, row) partial, exactly.
 #include <atomic>
 
 #include "common.cuh"
@@ -57,15 +58,13 @@ constexpr int kLutOffS2 = kLutOffHi + kLutChunkRows * 8;
 constexpr int kLutOffSc = kLutOffS2 + kLutChunkRows * 8;
 constexpr int kLutStageBytes = kLutOffSc + kLutChunkRows * 4;
 constexpr int kLutOffT2 = kLutGroups * kLutTableBytes;
-constexpr int kLutOffXh = kLutOffT2 + kLutGroups * 16 * 4;
-constexpr int kLutOffXf = kLutOffXh + kLutGroups * 8 * 2;
-constexpr int kLutOffMisc = kLutOffXf + kLutGroups * 8 * 4;  // group scales, barriers, chunk records
+constexpr int kLutOffMisc = kLutOffT2 + kLutGroups * 16 * 4;  // barriers, flags
 constexpr int kLutOffRing = kLutOffMisc + 256;
 constexpr int kLutSmem = kLutOffRing + kLutStages * kLutStageBytes;
 
-// Table builds per slice, counted in rows of lookups (a build costs about as
-// much as one chunk of lookups) when the (slice, row) sequence is split.
-constexpr int kLutBuildRows = 512;
+// A table build, counted in rows of lookups of equal cost, when the (slice, row)
+// sequence is split over the CTAs.
+constexpr int kLutBuildRows = 640;
 
 // Walks one CTA's range of (slice, row) positions in chunks that stay inside a
 // slice and hold at most kLutChunkRows rows (a multiple of 4, as N is).  The
@@ -110,11 +109,12 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   return r;
 }
 
+// D = A.B with a zero accumulator (fp16 in, fp32 out).
 __device__ __forceinline__ void mma_16808_f16(float d[4], uint32_t a0, uint32_t a1, uint32_t b0) {
   asm volatile(
-      "mma.sync.aligned.m16n8k8.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5}, {%6}, {%0,%1,%2,%3};\n"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(a1), "r"(b0));
+      "mma.sync.aligned.m16n8k8.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5}, {%6}, {%7,%7,%7,%7};\n"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a0), "r"(a1), "r"(b0), "f"(0.f));
 }
 
 // Sum of the 16 lookups of one row's slice record (lo 16 B, hi4 8 B, s2 8 B),
@@ -160,14 +160,11 @@ __global__ void __launch_bounds__(kLutThreads, 1)
   constexpr bool kTwo = (FMT == kFmtRvq12_4);
   unsigned char* t1 = smem;
   float* t2 = reinterpret_cast<float*>(smem + kLutOffT2);
-  uint32_t* xh = reinterpret_cast<uint32_t*>(smem + kLutOffXh);
-  float* xf = reinterpret_cast<float*>(smem + kLutOffXf);
-  float* gsc = reinterpret_cast<float*>(smem + kLutOffMisc);        // [16] per-group 2^-e
   const uint32_t full0 = smem_u32(smem + kLutOffMisc + 64);         // [kLutStages] mbarriers: chunk landed
   const uint32_t empty0 = smem_u32(smem + kLutOffMisc + 96);        // [kLutStages] mbarriers: chunk consumed
   volatile int* abortf = reinterpret_cast<volatile int*>(smem + kLutOffMisc + 128);  // a bounded wait gave up
   const uint32_t cb_bar = smem_u32(smem + kLutOffMisc + 136);       // codebook copy landed
-  volatile int* flag = reinterpret_cast<volatile int*>(smem + kLutOffMisc + 192);
+  volatile unsigned long long* bar_base = reinterpret_cast<volatile unsigned long long*>(smem + kLutOffMisc + 144);
   const uint32_t t1_base = smem_u32(t1), ring_base = smem_u32(smem + kLutOffRing);
 
   const int N = a.N;
@@ -188,8 +185,6 @@ __global__ void __launch_bounds__(kLutThreads, 1)
     ptx::fence_barrier_init();
   }
   __syncthreads();
-  bool ok = true;
-
   if (warp == kLutConsumers / 32) {
     // ------------------------------------------------------------ producer
     // Reads only the layer's constant index planes and scales, so it may run
@@ -236,25 +231,33 @@ __global__ void __launch_bounds__(kLutThreads, 1)
         c2v[2 * p + 1] = v.y;
       }
     }
-    // Everything above reads only the layer's constant inputs; x, y and the
-    // scratch are touched only after the previous kernel completed.  The x loads
-    // go out before the wait for the codebook copy, so the two latencies overlap.
+    // Everything above reads only the layer's constant inputs; x and the scratch
+    // are touched only after the previous kernel completed.  The x loads go out
+    // before the wait for the codebook copy, so the two latencies overlap.  Every
+    // warp holds a whole x slice: lane l has inputs 4l .. 4l+3 of it.
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    float xpre[kLutMaxX];
+    if (tid == 0 && S > 1) {
+      // The grid-barrier counter of this grid size before any CTA of this launch
+      // arrives: the previous launch of this handle has completed.
+      unsigned long long v;
+      asm volatile("ld.relaxed.gpu.u64 %0, [%1];"
+                   : "=l"(v)
+                   : "l"(reinterpret_cast<unsigned long long*>(gbar) + gridDim.x)
+                   : "memory");
+      *bar_base = v;
+    }
+    uint2 xpre[kLutMaxX];
 #pragma unroll
     for (int i = 0; i < kLutMaxX; ++i) {
       const int s = s_first + i;
-      xpre[i] = (tid < 128 && s < S) ? Elt<T>::to_f32(xg[(int64_t)s * 128 + tid]) : 0.f;
+      xpre[i] = s < S ? *reinterpret_cast<const uint2*>(xg + (int64_t)s * 128 + 4 * lane) : make_uint2(0, 0);
     }
 
     uint32_t bfrag[16][4];
     {
       // ldmatrix: lanes 8j..8j+7 give the rows (codewords) of matrix j; lane (g, c)
       // receives word c of row g of each matrix, the MMA B fragment.
-      if (!ptx::mbar_wait(cb_bar, 0, err)) {
-        ok = false;
-        *abortf = 1;
-      }
+      if (!ptx::mbar_wait(cb_bar, 0, err)) *abortf = 1;
       const int n = lane & 7, jm = lane >> 3;
 #pragma unroll
       for (int it = 0; it < 16; ++it) {
@@ -270,31 +273,33 @@ __global__ void __launch_bounds__(kLutThreads, 1)
     // reached by all 256 or by none).  After a wait gives up the rest of the walk
     // skips the waits (the result is then wrong and the error word is set).
     int cur = -1, s, r0, rows;
+    float unscale = 1.f;  // 2^-e of the current slice
     for (int k = 0; chunks.next(N, s, r0, rows); ++k) {
       const int st = k % kLutStages;
-      if (*abortf || !ptx::mbar_wait(full0 + 8 * st, (uint32_t)((k / kLutStages) & 1), err)) {
-        ok = false;
-        *abortf = 1;
-      }
+      // A new slice's tables need only x and the codebook, so they are built
+      // before the wait for the chunk's index bytes.
       if (s != cur) {
         // ------------------------------------------------------------ build
         asm volatile("bar.sync 1, %0;" ::"n"(kLutConsumers) : "memory");  // everyone is done with the old tables
-        float xv = 0.f;
-        if (tid < 128) {
+        uint2 xw;
+        {
           const int i = s - s_first;
           if (i < kLutMaxX) {
+            xw = xpre[0];
 #pragma unroll
-            for (int kk = 0; kk < kLutMaxX; ++kk)
-              if (kk == i) xv = xpre[kk];
+            for (int kk = 1; kk < kLutMaxX; ++kk)
+              if (kk == i) xw = xpre[kk];
           } else {
-            xv = Elt<T>::to_f32(xg[(int64_t)s * 128 + tid]);
+            xw = *reinterpret_cast<const uint2*>(xg + (int64_t)s * 128 + 4 * lane);
           }
         }
-        // Per group of 8 inputs, a power-of-two scale 2^e puts the group's largest |x|
-        // in [2^14, 2^15), so the fp16 MMA operand is exact for any activation type;
-        // the table entries are multiplied by 2^-e before they are stored (exact).
-        float m = fabsf(xv);
-        for (int o = 4; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        // One power of two 2^e per slice puts the slice's largest |x| in [2^14, 2^15),
+        // so the fp16 MMA operand is exact (bar values 2^31 below it) for either
+        // activation type; T1 and T2 are built from 2^e x and every partial is
+        // multiplied by 2^-e (exact).
+        float m = fmaxf(fmaxf(fabsf(Elt<T>::to_f32((uint16_t)xw.x)), fabsf(Elt<T>::to_f32((uint16_t)(xw.x >> 16)))),
+                        fmaxf(fabsf(Elt<T>::to_f32((uint16_t)xw.y)), fabsf(Elt<T>::to_f32((uint16_t)(xw.y >> 16)))));
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
         // e = 15 - (exponent of m as frexpf gives it), taken from the bits for
         // normal m (zero, inf and NaN get no scaling); clamped so 2^e and 2^-e are
         // normal floats.
@@ -306,39 +311,48 @@ __global__ void __launch_bounds__(kLutThreads, 1)
           frexpf(m, &e);
           e = min(100, max(-100, 15 - e));
         }
-        if (tid < 128) {
-          xf[tid] = xv;
-          reinterpret_cast<__half*>(xh)[tid] = __float2half_rn(xv * __uint_as_float((uint32_t)(127 + e) << 23));
-          if ((tid & 7) == 0) gsc[tid >> 3] = __uint_as_float((uint32_t)(127 - e) << 23);
+        const float up = __uint_as_float((uint32_t)(127 + e) << 23);
+        unscale = __uint_as_float((uint32_t)(127 - e) << 23);
+        // A operand (x slice, 16 groups x 8 dims, fp16): lane (g, c) needs inputs
+        // 8g+2c, 8g+2c+1 (held by lane 2g + c/2) and the same of group g+8.
+        uint32_t a0, a1;
+        {
+          const int src0 = 2 * g + (c >> 1), src1 = src0 + 16;
+          const uint32_t u0 = __shfl_sync(0xffffffffu, xw.x, src0), v0 = __shfl_sync(0xffffffffu, xw.y, src0);
+          const uint32_t u1 = __shfl_sync(0xffffffffu, xw.x, src1), v1 = __shfl_sync(0xffffffffu, xw.y, src1);
+          const uint32_t p0 = (c & 1) ? v0 : u0, p1 = (c & 1) ? v1 : u1;
+          a0 = Elt<__half>::pack(Elt<T>::to_f32((uint16_t)p0) * up, Elt<T>::to_f32((uint16_t)(p0 >> 16)) * up);
+          a1 = Elt<__half>::pack(Elt<T>::to_f32((uint16_t)p1) * up, Elt<T>::to_f32((uint16_t)(p1 >> 16)) * up);
         }
-        asm volatile("bar.sync 1, %0;" ::"n"(kLutConsumers) : "memory");
         if (kTwo) {
-          const int gg = tid >> 4;
+          // T2[gg][ee] = 2^e x_gg . cb2[ee] for thread gg*16 + ee; group gg's inputs
+          // are held by lanes 2gg and 2gg+1.
+          const int src = 2 * (tid >> 4);  // lane 2gg (every warp holds the whole slice)
+          const uint32_t q[4] = {__shfl_sync(0xffffffffu, xw.x, src), __shfl_sync(0xffffffffu, xw.y, src),
+                                 __shfl_sync(0xffffffffu, xw.x, src + 1), __shfl_sync(0xffffffffu, xw.y, src + 1)};
           float acc = 0.f;
 #pragma unroll
-          for (int d = 0; d < 8; ++d) acc = fmaf(xf[8 * gg + d], c2v[d], acc);
-          t2[tid] = acc;  // T2[gg][tid & 15], from the unscaled x
+          for (int d = 0; d < 4; ++d) {
+            acc = fmaf(Elt<T>::to_f32((uint16_t)q[d]), c2v[2 * d], acc);
+            acc = fmaf(Elt<T>::to_f32((uint16_t)(q[d] >> 16)), c2v[2 * d + 1], acc);
+          }
+          t2[tid] = acc * up;
         }
         {
-          // A = x slice (16 groups x 8 dims, fp16).  Column n of MMA j in block `it`
-          // is codeword base + 8*(n/2) + 2j + (n%2), so lane (g, c) ends with
-          // codewords base+8c .. base+8c+7 of groups g and g+8: one 16-byte store each.
-          const uint32_t a0 = xh[g * 4 + c], a1 = xh[(g + 8) * 4 + c];
-          const float ua = gsc[g], ub = gsc[g + 8];  // undo the groups' power-of-two scales
+          // Column n of MMA j in block `it` is codeword base + 8*(n/2) + 2j + (n%2), so
+          // lane (g, c) ends with codewords base+8c .. base+8c+7 of groups g and g+8:
+          // one 16-byte store each.
 #pragma unroll
           for (int it = 0; it < 16; ++it) {
             const int base = warp * 512 + it * 32;
             float d[4][4];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              d[j][0] = d[j][1] = d[j][2] = d[j][3] = 0.f;
-              mma_16808_f16(d[j], a0, a1, bfrag[it][j]);
-            }
+            for (int j = 0; j < 4; ++j) mma_16808_f16(d[j], a0, a1, bfrag[it][j]);
             typedef Elt<__nv_bfloat16> B16;
-            const uint4 lo = make_uint4(B16::pack(d[0][0] * ua, d[0][1] * ua), B16::pack(d[1][0] * ua, d[1][1] * ua),
-                                        B16::pack(d[2][0] * ua, d[2][1] * ua), B16::pack(d[3][0] * ua, d[3][1] * ua));
-            const uint4 hi = make_uint4(B16::pack(d[0][2] * ub, d[0][3] * ub), B16::pack(d[1][2] * ub, d[1][3] * ub),
-                                        B16::pack(d[2][2] * ub, d[2][3] * ub), B16::pack(d[3][2] * ub, d[3][3] * ub));
+            const uint4 lo = make_uint4(B16::pack(d[0][0], d[0][1]), B16::pack(d[1][0], d[1][1]),
+                                        B16::pack(d[2][0], d[2][1]), B16::pack(d[3][0], d[3][1]));
+            const uint4 hi = make_uint4(B16::pack(d[0][2], d[0][3]), B16::pack(d[1][2], d[1][3]),
+                                        B16::pack(d[2][2], d[2][3]), B16::pack(d[3][2], d[3][3]));
             *reinterpret_cast<uint4*>(t1 + g * kLutTableBytes + (base + 8 * c) * 2) = lo;
             *reinterpret_cast<uint4*>(t1 + (g + 8) * kLutTableBytes + (base + 8 * c) * 2) = hi;
           }
@@ -346,6 +360,7 @@ __global__ void __launch_bounds__(kLutThreads, 1)
         asm volatile("bar.sync 1, %0;" ::"n"(kLutConsumers) : "memory");
         cur = s;
       }
+      if (*abortf || !ptx::mbar_wait(full0 + 8 * st, (uint32_t)((k / kLutStages) & 1), err)) *abortf = 1;
 
       // -------------------------------------------------------------- lookups
 #pragma unroll
@@ -362,9 +377,9 @@ __global__ void __launch_bounds__(kLutThreads, 1)
         float acc;
         if (block_scales) {
           const float2 sc = f16x2_to_f32x2(scw);
-          acc = fmaf(blk[1], sc.y, blk[0] * sc.x);
+          acc = fmaf(blk[1], sc.y, blk[0] * sc.x) * unscale;
         } else {
-          acc = blk[0] + blk[1];  // the per-row scale is applied once, at the reduction
+          acc = (blk[0] + blk[1]) * unscale;  // the per-row scale is applied once, at the reduction
         }
         if (S == 1) {
           if (!block_scales) acc *= f16_bits_to_f32(a.scales[r]);
@@ -384,16 +399,16 @@ __global__ void __launch_bounds__(kLutThreads, 1)
   }
 
   // --------------------------------------------------- grid barrier + reduce
-  // Each grid size has its own counter, which only grows: this launch's CTAs take
-  // it from a multiple of the grid size to the next one, so each CTA's target
-  // follows from its own ticket (also when a CUDA graph replays the launch).
-  __threadfence();
+  // Each grid size has its own arrival counter, which only grows by whole grids:
+  // this launch's CTAs take it from `base` (read after the previous kernel
+  // completed) to base + grid.  The CTA barrier orders every thread's partial
+  // stores before thread 0's release add; thread 0's acquire load and the second
+  // CTA barrier order them before every thread's reads below.
   __syncthreads();
   if (tid == 0) {
     unsigned long long* cnt = reinterpret_cast<unsigned long long*>(gbar) + gridDim.x;
-    unsigned long long old;
-    asm volatile("atom.add.release.gpu.u64 %0, [%1], 1;" : "=l"(old) : "l"(cnt) : "memory");
-    const unsigned long long target = (old / gridDim.x + 1) * gridDim.x;
+    const unsigned long long target = *bar_base + gridDim.x;
+    asm volatile("red.release.gpu.global.add.u64 [%0], 1;" ::"l"(cnt) : "memory");
     const uint64_t t0 = ptx::globaltimer_ns();
     bool released = false;
     for (uint32_t i = 0; i < kWaitSpinLimit; ++i) {
@@ -406,42 +421,62 @@ __global__ void __launch_bounds__(kLutThreads, 1)
       if ((i & 63u) == 63u && ptx::globaltimer_ns() - t0 > 1000000000ull) break;
     }
     if (!released) atomicOr(err, kErrTimeout);
-    *flag = ok;
   }
   __syncthreads();
-  __threadfence();
   // Every CTA of this grid has passed the barrier, so all of them are resident:
   // the next kernel in the stream may launch now and take each SM as its CTA here
   // exits (it reads x, y and the scratch only after this grid completes).
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  // This CTA's rows; tpr threads per row split the slices, then a fixed xor tree.
-  const int rbeg = (int)((int64_t)N * blockIdx.x / gridDim.x), rend = (int)((int64_t)N * (blockIdx.x + 1) / gridDim.x);
-  const int nr = rend - rbeg;
+  // This CTA's rows, in quads (N % 4 == 0): tpr threads per quad split the slices
+  // (at most 8 each, one batch of independent 16-byte loads, when the CTA has the
+  // threads for it), then a fixed xor tree combines the parts.
+  const int Q = N / 4;
+  const int qbeg = (int)((int64_t)Q * blockIdx.x / gridDim.x), qend = (int)((int64_t)Q * (blockIdx.x + 1) / gridDim.x);
+  const int nq = qend - qbeg;
   int tpr = 1;
-  while (tpr < 32 && tpr * 2 * nr <= kLutThreads) tpr *= 2;
+  while (tpr < 32 && (S + tpr - 1) / tpr > 8 && 2 * tpr * nq <= kLutThreads) tpr *= 2;
   const int per = (S + tpr - 1) / tpr;
-  for (int base = 0; base < nr * tpr; base += kLutThreads) {
+  for (int base = 0; base < nq * tpr; base += kLutThreads) {
     const int idx = base + tid;
-    const int row = idx / tpr, part = idx % tpr;
-    float sum = 0.f;
-    if (row < nr) {
-      const int r = rbeg + row;
+    const int q = idx / tpr, part = idx % tpr;
+    float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (q < nq) {
+      const int r = 4 * (qbeg + q);
       const int k0 = part * per, k1 = min(S, k0 + per);
-      constexpr int kBatch = 16;
+      constexpr int kBatch = 8;
       for (int kb = k0; kb < k1; kb += kBatch) {
-        float v[kBatch];
-#pragma unroll
-        for (int j = 0; j < kBatch; ++j) v[j] = (kb + j < k1) ? __ldcg(partial + (int64_t)(kb + j) * N + r) : 0.f;
+        float4 v[kBatch];
 #pragma unroll
         for (int j = 0; j < kBatch; ++j)
-          if (kb + j < k1) sum += v[j];
+          v[j] = (kb + j < k1) ? __ldcg(reinterpret_cast<const float4*>(partial + (int64_t)(kb + j) * N + r))
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int j = 0; j < kBatch; ++j)
+          if (kb + j < k1) {
+            sum.x += v[j].x;
+            sum.y += v[j].y;
+            sum.z += v[j].z;
+            sum.w += v[j].w;
+          }
       }
     }
-    for (int o = 1; o < tpr; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-    if (row < nr && part == 0) {
-      const int r = rbeg + row;
-      if (!block_scales) sum *= f16_bits_to_f32(a.scales[r]);
-      static_cast<uint16_t*>(a.y)[r] = Elt<T>::from_f32(sum);
+    for (int o = 1; o < tpr; o <<= 1) {
+      sum.x += __shfl_xor_sync(0xffffffffu, sum.x, o);
+      sum.y += __shfl_xor_sync(0xffffffffu, sum.y, o);
+      sum.z += __shfl_xor_sync(0xffffffffu, sum.z, o);
+      sum.w += __shfl_xor_sync(0xffffffffu, sum.w, o);
+    }
+    if (q < nq && part == 0) {
+      const int r = 4 * (qbeg + q);
+      float o4[4] = {sum.x, sum.y, sum.z, sum.w};
+      if (!block_scales) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) o4[i] *= f16_bits_to_f32(a.scales[r + i]);
+      }
+      uint16_t* yr = static_cast<uint16_t*>(a.y) + r;
+      *reinterpret_cast<uint2*>(yr) =
+          make_uint2((uint32_t)Elt<T>::from_f32(o4[0]) | ((uint32_t)Elt<T>::from_f32(o4[1]) << 16),
+                     (uint32_t)Elt<T>::from_f32(o4[2]) | ((uint32_t)Elt<T>::from_f32(o4[3]) << 16));
     }
   }
 }
