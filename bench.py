@@ -155,7 +155,8 @@ class Workload:
         for li in range(w["layers"]):
             for ti, (label, spec) in enumerate(self.cfg["tensors"]):
                 arr = make_layer(spec, cfg_id=w["cfg"], layer=li, tensor_id=ti, seed=seed)
-                L = vq.VQLinear(spec.N, spec.K, spec.fmt, spec.scale_group, self.act, max_M, arr)
+                L = vq.VQLinear(spec.N, spec.K, spec.fmt, spec.scale_group, self.act, max_M, arr,
+                                rht=int(self.cfg["rht"]))
                 self.layers.append((f"{li}.{label}", spec, L))
         # Copies of every layer's device arrays, cycled step by step so that the
         # weights a step reads are never in L2 (their total is >= 4x the L2 size);
@@ -172,7 +173,6 @@ class Workload:
             .view(self.tdtype)
         if self.rht:
             self.signs = torch.from_numpy(make_signs(K0, cfg_id=w["cfg"], seed=seed)).cuda()
-            self.xr = torch.empty_like(self.x0)
         self.outs = {}
 
     def weight_bytes(self):
@@ -184,7 +184,7 @@ class Workload:
         import torch
 
         calls = []
-        x = self.xr[:M] if self.rht else self.x0[:M]
+        x = self.x0[:M]
         prev_by_width = {}
         for name, spec, L in self.replicas[replica]:
             label = name.split(".")[1]
@@ -207,21 +207,30 @@ class Workload:
     def enqueue(self, calls, M, events=None):
         import compressed_index_matmul_b200 as vq
 
-        if self.rht:
-            vq.vq_rht_apply(self.x0, self.xr, self.signs, M, self.x0.shape[1], self.act)
         for i, (L, inp, y) in enumerate(calls):
             if events is not None:
                 events[i].record()
-            L.forward(inp, y)
+            if self.rht:  # the layer rotates its input (vq_linear_forward_rotated)
+                L.forward_rotated(inp, self.signs, y)
+            else:
+                L.forward(inp, y)
         if events is not None:
             events[len(calls)].record()
 
+    def rotation_fused(self, spec, M):
+        """True where vq_linear_forward_rotated is one kernel (the batch-1 gather kernel)."""
+        return M == 1 and spec.fmt == FMT_VQ16 and spec.K % 128 == 0 and spec.K <= 16384 and spec.N % 4 == 0
+
     def launches_per_step(self, M):
-        n = sum(L.launches(M) for _, _, L in self.layers)
-        return n + (1 if self.rht else 0)
+        n = 0
+        for _, spec, L in self.layers:
+            n += L.launches(M) + (1 if self.rht and not self.rotation_fused(spec, M) else 0)
+        return n
 
     def bytes_per_step(self, M):
-        return sum(layer_bytes(spec, M) for _, spec, _ in self.layers) + (4 * M * self.x0.shape[1] if self.rht else 0)
+        # an unfused rotation reads and writes x once more (2 + 2 bytes per element)
+        extra = sum(4 * M * spec.K for _, spec, _ in self.layers if self.rht and not self.rotation_fused(spec, M))
+        return sum(layer_bytes(spec, M) for _, spec, _ in self.layers) + extra
 
     def flops_per_step(self, M):
         return sum(2.0 * M * spec.N * spec.K for _, spec, _ in self.layers)
@@ -234,7 +243,11 @@ def _clone_layer(L):
     from compressed_index_matmul_b200 import _binding as B
 
     c = copy.copy(L)
-    c.t = {k: v.clone() for k, v in L.t.items()}
+    # The 65,536-entry codebook of the 16-bit format is one table shared by every
+    # copy: GLQ's lattice codebook is shared by all layers and served from L2.  The
+    # index planes, scales and 4096-entry codebooks are copied.
+    shared = ("cb1",) if L.fmt == FMT_VQ16 else ()
+    c.t = {k: (v if k in shared else v.clone()) for k, v in L.t.items()}
     c.planes = B.make_planes(c.t.get("lo"), c.t.get("hi4"), c.t.get("s2"), c.t.get("idx16"))
     c.codebooks = B.make_codebooks(c.t["cb1"], c.t.get("cb2"))
     c.close = lambda: None  # the handle belongs to L
@@ -431,12 +444,14 @@ def gpu_arm(args):
     # The batch-1 table path is two kernels per forward (lookups, then the split-K
     # reduction) that overlap by programmatic dependent launch, so the forward,
     # not either kernel alone, is the unit its bytes are divided by.
-    uniform = (not wl.rht) and len(set(launches_per_fwd)) == 1
+    fused = all(wl.rotation_fused(spec, M) for _, spec, _ in wl.layers)
+    uniform = (not wl.rht or fused) and len(set(launches_per_fwd)) == 1
     fwd_ms = ms_per_step / len(wl.layers) if uniform else float(np.mean(per_fwd))
     per_fwd_eff = [fwd_ms] * len(wl.layers) if uniform else list(per_fwd)
     achieved = sum(bytes_per_fwd) / (sum(per_fwd_eff) * 1e-3) / 1e9
-    lut = M == 1 and wl.layers[0][1].fmt != FMT_VQ16
-    dominant = "lut_gemv_kernel" if lut else ("gemv_kernel" if M <= 16 else "tc_gemm_kernel")
+    fmt0 = wl.layers[0][1].fmt
+    dominant = ("lut_gemv_kernel" if M == 1 and fmt0 != FMT_VQ16 else
+                "vq16_gemv_kernel" if M == 1 else "gemv_kernel" if M <= 16 else "tc_gemm_kernel")
     traffic = lookup_traffic(dominant, args.workload, M)
     avg_launch_us = round(1e3 * float(np.mean(per_fwd_eff)), 3)
     if not uniform:
@@ -480,7 +495,9 @@ def gpu_arm(args):
                    "shapes": [[spec.N, spec.K] for _, spec, _ in wl.layers[:7]],
                    "format": "rvq12_4 block-64" if args.workload != "vq16-4096-rht" else "vq16 per-row",
                    "parallelism": f"replicas x{world}",
-                   "l2": L2_NOTE.format(r=R, mb=R * wl.weight_bytes() / 1e6),
+                   "l2": L2_NOTE.format(r=R, mb=R * wl.weight_bytes() / 1e6) + (
+                       "; the 65,536-entry codebook is one table shared by the copies (L2-resident)"
+                       if fmt0 == FMT_VQ16 else ""),
                    "layer": "one vq_linear_forward (one weight matrix)",
                    "hbm_gbs": round(sum(bytes_per_fwd) / (ms_per_step * 1e-3) / 1e9, 1)},
         "roofline": roofline,

@@ -16,6 +16,7 @@ from ._binding import (  # noqa: F401
     VQ_FMT_RVQ12_4,
     VQ_FMT_VQ16,
     VQ_PATH_AUTO,
+    VQ_PATH_GATHER,
     VQ_PATH_GEMV,
     VQ_PATH_LUT,
     VQ_PATH_TC,
@@ -32,6 +33,7 @@ from ._binding import (  # noqa: F401
     vq_linear_destroy,
     vq_linear_forward,
     vq_linear_forward_noalloc,
+    vq_linear_forward_rotated,
     vq_linear_launches,
     vq_linear_set_path,
     vq_linear_set_sm_budget,

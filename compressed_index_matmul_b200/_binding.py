@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(PKG, "libvqlinear.so")
 VQ_OK, VQ_ERR_INVALID_ARG, VQ_ERR_UNSUPPORTED, VQ_ERR_CUDA, VQ_ERR_NOMEM, VQ_ERR_TIMEOUT = range(6)
 VQ_FMT_RVQ12, VQ_FMT_RVQ12_4, VQ_FMT_VQ16 = 1, 2, 3
 VQ_F16, VQ_BF16 = 0, 1
-VQ_PATH_AUTO, VQ_PATH_LUT, VQ_PATH_GEMV, VQ_PATH_TC = 0, 1, 2, 3
+VQ_PATH_AUTO, VQ_PATH_LUT, VQ_PATH_GEMV, VQ_PATH_TC, VQ_PATH_GATHER = 0, 1, 2, 3, 4
 
 STATUS_NAMES = {0: "VQ_OK", 1: "VQ_ERR_INVALID_ARG", 2: "VQ_ERR_UNSUPPORTED", 3: "VQ_ERR_CUDA",
                 4: "VQ_ERR_NOMEM", 5: "VQ_ERR_TIMEOUT"}
@@ -27,7 +27,7 @@ STATUS_NAMES = {0: "VQ_OK", 1: "VQ_ERR_INVALID_ARG", 2: "VQ_ERR_UNSUPPORTED", 3:
 # Every entry point the header declares (checked by the tests against the .so).
 EXPORTS = ("vq_abi_version", "vq_linear_create", "vq_linear_destroy", "vq_linear_set_path", "vq_linear_set_sm_budget",
            "vq_linear_forward",
-           "vq_linear_forward_noalloc", "vq_linear_launches", "vq_rht_apply", "vq_linear_check", "vq_last_error",
+           "vq_linear_forward_noalloc", "vq_linear_forward_rotated", "vq_linear_launches", "vq_rht_apply", "vq_linear_check", "vq_last_error",
            "vq_debug_unpack", "vq_debug_dequant", "vq_debug_wait_timeout")
 
 
@@ -90,6 +90,9 @@ def load(path: str | None = None):
         lib.vq_debug_wait_timeout.argtypes = [P, P]
         lib.vq_linear_launches.restype = I32
         lib.vq_linear_launches.argtypes = [P, I32]
+        lib.vq_linear_forward_rotated.restype = st
+        lib.vq_linear_forward_rotated.argtypes = [P, P, P, ctypes.POINTER(vq_planes), ctypes.POINTER(vq_codebooks), P,
+                                                  P, I32, I32, I32, P]
         lib.vq_rht_apply.restype = st
         lib.vq_rht_apply.argtypes = [P, P, P, I32, I32, I32, P]
         lib.vq_linear_check.restype = st
@@ -164,6 +167,13 @@ def vq_linear_launches(h, M: int) -> int:
 def vq_linear_forward(h, x, planes: vq_planes, codebooks: vq_codebooks, scales, y, M, N, K, stream=None) -> None:
     _check(load().vq_linear_forward(h, _ptr(x), ctypes.byref(planes), ctypes.byref(codebooks), _ptr(scales),
                                     _ptr(y), M, N, K, _stream(stream)))
+
+
+def vq_linear_forward_rotated(h, x, signs, planes: vq_planes, codebooks: vq_codebooks, scales, y, M, N, K,
+                              stream=None) -> None:
+    """y = rotate(x) . W^T with the rotation's +-1 `signs` (int8 device tensor [K])."""
+    _check(load().vq_linear_forward_rotated(h, _ptr(x), _ptr(signs), ctypes.byref(planes), ctypes.byref(codebooks),
+                                            _ptr(scales), _ptr(y), M, N, K, _stream(stream)))
 
 
 def vq_linear_forward_noalloc(N, K, fmt, scale_group, act_dtype, x, planes: vq_planes, codebooks: vq_codebooks,

@@ -20,6 +20,7 @@ namespace vq {
 void plan_gemv(const vq_linear_desc& d, const DeviceInfo& dev, int M, Plan* p);
 bool plan_lut(const vq_linear_desc& d, const DeviceInfo& dev, int M, Plan* p);
 bool plan_tc(const vq_linear_desc& d, const DeviceInfo& dev, int M, Plan* p);
+bool plan_vq16(const vq_linear_desc& d, const DeviceInfo& dev, int M, Plan* p);
 }  // namespace vq
 
 struct vq_linear_s {
@@ -34,6 +35,7 @@ struct vq_linear_s {
                       // (8-byte aligned; each only ever grows by whole grids)
   uint32_t* err;      // device word, set by bounded waits that gave up
   int sm_budget;      // CTAs of the table kernel (0: every SM)
+  void* xrot;         // rotated-x buffer [max_M][K] (desc.rht == 1), for the unfused rotated forward
 };
 
 namespace {
@@ -140,9 +142,15 @@ bool plan_forward(const vq_linear_desc& d, const DeviceInfo& dev, int M, int for
     // Measured on B200: from M = 2 the tensor-core path decodes large layers
     // faster than the warp-MMA GEMV; on small layers both are launch-bound.
     const bool large = (int64_t)d.N * d.K >= (int64_t(1) << 22);
-    path = (M == 1) ? VQ_PATH_LUT : ((M <= 16 && !large) ? VQ_PATH_GEMV : VQ_PATH_TC);
+    path = (M == 1) ? (d.fmt == VQ_FMT_VQ16 ? VQ_PATH_GATHER : VQ_PATH_LUT)
+                    : ((M <= 16 && !large) ? VQ_PATH_GEMV : VQ_PATH_TC);
   }
   switch (path) {
+    case VQ_PATH_GATHER:
+      if (plan_vq16(d, dev, M, out)) return true;
+      if (forced_path != VQ_PATH_AUTO) return false;
+      plan_gemv(d, dev, M, out);
+      return true;
     case VQ_PATH_LUT:
       if (plan_lut(d, dev, M, out)) return true;
       if (forced_path != VQ_PATH_AUTO) return false;
@@ -192,7 +200,7 @@ VQ_API vq_status vq_linear_create(const vq_linear_desc* desc, vq_linear_t* out) 
   size_t need = 0;
   int tickets = 0;
   for (int M = 1; M <= desc->max_M; ++M) {
-    const int paths[3] = {VQ_PATH_LUT, VQ_PATH_GEMV, VQ_PATH_TC};
+    const int paths[4] = {VQ_PATH_LUT, VQ_PATH_GEMV, VQ_PATH_TC, VQ_PATH_GATHER};
     for (int pth : paths) {
       vq::Plan p{};
       if (!vq::plan_forward(*desc, dev, M, pth, &p)) continue;
@@ -219,6 +227,16 @@ VQ_API vq_status vq_linear_create(const vq_linear_desc* desc, vq_linear_t* out) 
       return fail(VQ_ERR_NOMEM, "cudaMalloc of %zu scratch bytes failed: %s", need, cudaGetErrorString(e));
     }
   }
+  if (desc->rht) {
+    e = cudaMalloc(&h->xrot, (size_t)desc->max_M * desc->K * 2);
+    if (e != cudaSuccess) {
+      cudaFree(h->scratch);
+      delete h;
+      cudaGetLastError();
+      return fail(VQ_ERR_NOMEM, "cudaMalloc of the %d x %d rotation buffer failed: %s", desc->max_M, desc->K,
+                  cudaGetErrorString(e));
+    }
+  }
   h->num_tickets = tickets;
   // words: [0] error flag, [1] pad, then (num_sms + 1) 64-bit barrier counters, then tickets
   const size_t bar_words = 2 * ((size_t)dev.num_sms + 1);
@@ -232,6 +250,7 @@ VQ_API vq_status vq_linear_create(const vq_linear_desc* desc, vq_linear_t* out) 
   h->tickets = (words && tickets) ? words + 2 + bar_words : nullptr;
   if (e != cudaSuccess) {
     cudaFree(h->scratch);
+    cudaFree(h->xrot);
     cudaFree(words);
     delete h;
     cudaGetLastError();
@@ -245,6 +264,7 @@ VQ_API vq_status vq_linear_destroy(vq_linear_t h) {
   if (h == nullptr) return VQ_OK;
   cudaError_t e1 = cudaSuccess, e2 = cudaSuccess;
   if (h->scratch) e1 = cudaFree(h->scratch);
+  if (h->xrot && e1 == cudaSuccess) e1 = cudaFree(h->xrot);
   if (h->err) e2 = cudaFree(h->err);  // also frees the barrier words and tickets (one allocation)
   delete h;
   if (e1 != cudaSuccess) return cuda_fail(e1, "cudaFree(scratch)");
@@ -254,7 +274,7 @@ VQ_API vq_status vq_linear_destroy(vq_linear_t h) {
 
 VQ_API vq_status vq_linear_set_path(vq_linear_t h, int32_t path) {
   if (h == nullptr) return fail(VQ_ERR_INVALID_ARG, "handle is NULL");
-  if (path < VQ_PATH_AUTO || path > VQ_PATH_TC) return fail(VQ_ERR_INVALID_ARG, "path=%d is not a VQ_PATH_*", path);
+  if (path < VQ_PATH_AUTO || path > VQ_PATH_GATHER) return fail(VQ_ERR_INVALID_ARG, "path=%d is not a VQ_PATH_*", path);
   h->path = path;
   return VQ_OK;
 }
@@ -293,7 +313,8 @@ VQ_API vq_status vq_linear_forward(vq_linear_t h, const void* x, const vq_planes
   vq::Plan p{};
   if (!vq::plan_forward(d, h->dev, M, h->path, &p))
     return fail(VQ_ERR_UNSUPPORTED, "path %d cannot run M=%d", h->path, M);
-  if (p.path == VQ_PATH_LUT && h->sm_budget > 0 && p.grid > h->sm_budget) p.grid = h->sm_budget;
+  if ((p.path == VQ_PATH_LUT || p.path == VQ_PATH_GATHER) && h->sm_budget > 0 && p.grid > h->sm_budget)
+    p.grid = h->sm_budget;
   if (p.scratch_bytes > h->scratch_bytes || p.tickets > h->num_tickets)
     return fail(VQ_ERR_UNSUPPORTED, "plan needs %zu scratch bytes / %d tickets, handle has %zu / %d",
                 p.scratch_bytes, p.tickets, h->scratch_bytes, h->num_tickets);
@@ -305,11 +326,54 @@ VQ_API vq_status vq_linear_forward(vq_linear_t h, const void* x, const vq_planes
   cudaError_t e;
   switch (p.path) {
     case VQ_PATH_LUT: e = vq::launch_lut(a, p, h->scratch, h->gbar, h->err, s); break;  // p.grid CTAs
+    case VQ_PATH_GATHER: e = vq::launch_vq16(a, p, nullptr, s); break;
     case VQ_PATH_TC: e = vq::launch_tc(a, p, h->scratch, h->tickets, h->err, s); break;
     default: e = vq::launch_gemv(a, p, h->scratch, h->tickets, s); break;
   }
   if (e != cudaSuccess) return cuda_fail(e, "vq_linear_forward launch");
   return VQ_OK;
+}
+
+VQ_API vq_status vq_linear_forward_rotated(vq_linear_t h, const void* x, const int8_t* signs, const vq_planes* planes,
+                                           const vq_codebooks* codebooks, const void* scales, void* y, int32_t M,
+                                           int32_t N, int32_t K, void* stream) {
+  if (h == nullptr) return fail(VQ_ERR_INVALID_ARG, "handle is NULL");
+  const vq_linear_desc& d = h->d;
+  if (N != d.N || K != d.K)
+    return fail(VQ_ERR_INVALID_ARG, "N=%d, K=%d do not match the handle's N=%d, K=%d", N, K, d.N, d.K);
+  if (K < 64 || K > 32768 || (K & (K - 1)) != 0)
+    return fail(VQ_ERR_INVALID_ARG, "K=%d: the rotation needs a power of two in [64, 32768]", K);
+  if (M < 0 || M > d.max_M) return fail(VQ_ERR_INVALID_ARG, "M=%d outside [0, max_M=%d]", M, d.max_M);
+  vq_status st;
+  if ((st = check_ptr(signs, "signs")) || (st = check_ptr(x, "x")) || (st = check_ptr(y, "y")) || (st = validate_planes(d, planes)) ||
+      (st = validate_codebooks(d, codebooks, scales)))
+    return st;
+  if (x == y) return fail(VQ_ERR_INVALID_ARG, "y must not alias x");
+  if (M == 0) return VQ_OK;
+  if ((st = check_device(h))) return st;
+  vq::Plan p{};
+  if (!vq::plan_forward(d, h->dev, M, h->path, &p))
+    return fail(VQ_ERR_UNSUPPORTED, "path %d cannot run M=%d", h->path, M);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (p.path == VQ_PATH_GATHER) {
+    if (h->sm_budget > 0 && p.grid > h->sm_budget) p.grid = h->sm_budget;
+    if (p.scratch_bytes > h->scratch_bytes)
+      return fail(VQ_ERR_UNSUPPORTED, "plan needs %zu scratch bytes, handle has %zu", p.scratch_bytes,
+                  h->scratch_bytes);
+    vq::LayerArgs a = make_args(d, planes, codebooks, scales);
+    a.x = x;
+    a.y = y;
+    a.M = M;
+    cudaError_t e = vq::launch_vq16(a, p, signs, s);
+    if (e != cudaSuccess) return cuda_fail(e, "vq_linear_forward_rotated launch");
+    return VQ_OK;
+  }
+  if (h->xrot == nullptr)
+    return fail(VQ_ERR_INVALID_ARG,
+                "this shape's rotation is not fused and the handle has no rotation buffer (create it with rht = 1)");
+  cudaError_t e = vq::launch_rht(x, h->xrot, signs, M, K, d.act_dtype, s);
+  if (e != cudaSuccess) return cuda_fail(e, "vq_linear_forward_rotated rotation launch");
+  return vq_linear_forward(h, h->xrot, planes, codebooks, scales, y, M, N, K, stream);
 }
 
 VQ_API vq_status vq_rht_apply(const void* x, void* x_out, const int8_t* signs, int32_t M, int32_t K, int32_t dtype,

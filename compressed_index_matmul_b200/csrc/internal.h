@@ -29,13 +29,13 @@ struct LayerArgs {
 
 // Work split chosen for one forward.
 struct Plan {
-  int path;          // VQ_PATH_LUT / GEMV / TC
+  int path;          // VQ_PATH_LUT / GEMV / TC / GATHER
   int splits;        // K splits (1 = the kernel writes y directly)
   int k_per_split;   // multiple of 64
   int launches;      // kernels enqueued
   size_t scratch_bytes;
   int tickets;       // completion counters needed (zero between forwards)
-  int grid;          // CTAs of the persistent table kernel (VQ_PATH_LUT), else 0
+  int grid;          // CTAs of the persistent batch-1 kernels (VQ_PATH_LUT / GATHER), else 0
 };
 
 struct DeviceInfo {
@@ -58,6 +58,10 @@ cudaError_t launch_gemv(const LayerArgs& a, const Plan& p, float* scratch, uint3
 // sizes other launches of the handle used).
 cudaError_t launch_lut(const LayerArgs& a, const Plan& p, float* scratch, uint32_t* gbar, uint32_t* err,
                        cudaStream_t s);
+// The batch-1 kernel of the 16-bit format (VQ_PATH_GATHER, clusters of 8 CTAs,
+// no scratch); `signs` (may be NULL) makes it rotate x itself
+// (vq_linear_forward_rotated).
+cudaError_t launch_vq16(const LayerArgs& a, const Plan& p, const int8_t* signs, cudaStream_t s);
 cudaError_t launch_tc(const LayerArgs& a, const Plan& p, float* scratch, uint32_t* tickets, uint32_t* err_flag,
                       cudaStream_t s);
 cudaError_t launch_split_reduce(const float* partial, void* y, int splits, int M, int N, int act, cudaStream_t s);

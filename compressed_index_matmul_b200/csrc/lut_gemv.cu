@@ -111,7 +111,7 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
 
 // D = A.B with a zero accumulator (fp16 in, fp32 out).
 __device__ __forceinline__ void mma_16808_f16(float d[4], uint32_t a0, uint32_t a1, uint32_t b0) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k8.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5}, {%6}, {%7,%7,%7,%7};\n"
       : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
       : "r"(a0), "r"(a1), "r"(b0), "f"(0.f));
@@ -446,10 +446,15 @@ __global__ void __launch_bounds__(kLutThreads, 1)
       constexpr int kBatch = 8;
       for (int kb = k0; kb < k1; kb += kBatch) {
         float4 v[kBatch];
+        const float4* src = reinterpret_cast<const float4*>(partial + (int64_t)kb * N + r);
+        if (k1 - kb >= kBatch) {  // a full batch: unpredicated loads, all in flight at once
 #pragma unroll
-        for (int j = 0; j < kBatch; ++j)
-          v[j] = (kb + j < k1) ? __ldcg(reinterpret_cast<const float4*>(partial + (int64_t)(kb + j) * N + r))
-                               : make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int j = 0; j < kBatch; ++j) v[j] = __ldcg(src + (int64_t)j * (N / 4));
+        } else {
+#pragma unroll
+          for (int j = 0; j < kBatch; ++j)
+            v[j] = (kb + j < k1) ? __ldcg(src + (int64_t)j * (N / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
 #pragma unroll
         for (int j = 0; j < kBatch; ++j)
           if (kb + j < k1) {

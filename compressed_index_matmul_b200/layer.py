@@ -54,6 +54,17 @@ class VQLinear:
 
     __call__ = forward
 
+    def forward_rotated(self, x, signs, y=None, stream=None):
+        """y = rotate(x) . W^T (vq_linear_forward_rotated); `signs` is an int8 tensor of +-1 [K]."""
+        import torch
+
+        M = x.shape[0]
+        if y is None:
+            y = torch.empty((M, self.N), dtype=self.torch_dtype, device=self.device)
+        B.vq_linear_forward_rotated(self.handle, x, signs, self.planes, self.codebooks, self.t["scales"], y, M, self.N,
+                                    self.K, stream)
+        return y
+
     def set_path(self, path: int):
         B.vq_linear_set_path(self.handle, path)
 

@@ -87,13 +87,16 @@ enum { VQ_F16 = 0, VQ_BF16 = 1 };
 
 /* Kernel choice for vq_linear_set_path.  VQ_PATH_AUTO picks by M and layer size:
  * M == 1 -> VQ_PATH_LUT where it applies (12-bit formats, K % 128 == 0, N % 4 == 0),
- * else VQ_PATH_GEMV; 2 <= M <= 16 -> VQ_PATH_TC for layers of at least 2^22 weights,
- * else VQ_PATH_GEMV; M >= 17 -> VQ_PATH_TC. */
+ * VQ_PATH_GATHER where it applies (VQ_FMT_VQ16, K % 128 == 0, K <= 16384,
+ * N % 4 == 0), else VQ_PATH_GEMV; 2 <= M <= 16 -> VQ_PATH_TC for layers of at
+ * least 2^22 weights, else VQ_PATH_GEMV; M >= 17 -> VQ_PATH_TC. */
 enum {
   VQ_PATH_AUTO = 0,
   VQ_PATH_LUT = 1,    /* M == 1 only: per-group x.codebook tables in shared memory */
   VQ_PATH_GEMV = 2,   /* 1 <= M <= 16: decode to registers, warp MMA, split-K */
-  VQ_PATH_TC = 3      /* any M: decode into tensor memory, tcgen05 MMA (fp32 in TMEM) */
+  VQ_PATH_TC = 3,     /* any M: decode into tensor memory, tcgen05 MMA (fp32 in TMEM) */
+  VQ_PATH_GATHER = 4  /* M == 1, VQ_FMT_VQ16 only: codewords gathered from L2 into
+                         fp32 dot products; can apply the input rotation itself */
 };
 
 typedef struct {
@@ -103,8 +106,11 @@ typedef struct {
   int32_t scale_group; /* 64 (block scales along K) or K (one scale per row) */
   int32_t act_dtype;   /* VQ_F16 or VQ_BF16: dtype of x and y */
   int32_t max_M;       /* largest token count a forward will be given, >= 1 */
-  int32_t rht;         /* informational: 1 if the planes encode W . R^T for a
-                          rotated input (the caller applies vq_rht_apply to x) */
+  int32_t rht;         /* 1 if the planes encode W . R^T for a rotated input: the
+                          caller either applies vq_rht_apply to x and calls
+                          vq_linear_forward, or calls vq_linear_forward_rotated
+                          (create then also allocates a max_M x K rotation buffer
+                          for the shapes whose rotation is not fused) */
 } vq_linear_desc;
 
 typedef struct {
@@ -197,6 +203,26 @@ vq_status vq_linear_forward(vq_linear_t h, const void* x, const vq_planes* plane
 vq_status vq_linear_forward_noalloc(const vq_linear_desc* desc, const void* x, const vq_planes* planes,
                                     const vq_codebooks* codebooks, const void* scales, void* y, int32_t M,
                                     void* stream);
+
+/* y = R(x) . W^T, where R is the input rotation of vq_rht_apply with these
+ * `signs` (GLQ README, "How it works": Randomized Hadamard Transform; "Inference
+ * kernels" / "Bit widths": the rotation is applied to the activations inside the
+ * fused kernels).  x is the unrotated input; the planes encode W . R^T, so y
+ * approximates x . W^T.  Arguments are those of vq_linear_forward plus `signs`,
+ * a device int8 array of +1/-1 [K] (16-byte aligned, like every pointer); K must
+ * be a power of two, 64 <= K <= 32768.
+ *   - Where VQ_PATH_GATHER runs (M == 1, VQ_FMT_VQ16, K <= 16384) this is one
+ *     kernel: every CTA rotates x in fp32 in shared memory and uses it unrounded;
+ *     nothing else is written.
+ *   - Otherwise it enqueues vq_rht_apply into a buffer of the handle (allocated
+ *     by vq_linear_create when desc->rht == 1: max_M x K elements) followed by
+ *     vq_linear_forward on it, so the rotated x is rounded to the activation type
+ *     as with the two separate calls.  Without that buffer (desc->rht == 0) such
+ *     a call returns VQ_ERR_INVALID_ARG.
+ * Same synchronisation, ownership and error behaviour as vq_linear_forward. */
+vq_status vq_linear_forward_rotated(vq_linear_t h, const void* x, const int8_t* signs, const vq_planes* planes,
+                                    const vq_codebooks* codebooks, const void* scales, void* y, int32_t M,
+                                    int32_t N, int32_t K, void* stream);
 
 /* Number of kernels vq_linear_forward enqueues for this M (0 for M == 0), or -1
  * if M is out of range. */

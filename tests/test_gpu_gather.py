@@ -1,0 +1,162 @@
+"""GPU parity of the batch-1 gather kernel for the 16-bit format (VQ_PATH_GATHER) and of
+vq_linear_forward_rotated, the forward that applies the input rotation itself.
+
+y must satisfy max|y_gpu - y_oracle| <= 2e-3 * ||x_m||_2 * max|w| per element and be
+bit-identical from run to run.  For the fused rotation the kernel keeps the rotated x
+in fp32, so its reference is the oracle's fp64 rotation, unrounded, times the oracle's
+exact weights; the unfused fallback rounds the rotated x to the activation type, as
+vq_rht_apply does, and is compared with the oracle forward of that rounded x."""
+
+import numpy as np
+import pytest
+import torch
+
+import compressed_index_matmul_b200 as vq
+from synth import CONFIGS, DT_BF16, DT_F16, FMT_RVQ12_4, FMT_VQ16, LayerSpec, make_layer, make_signs, make_x
+from tests.gpu_util import assert_y_within, dev, host_bits, layer_on_gpu, require_gpu, run_forward
+
+pytestmark = pytest.mark.gpu
+
+TOL = 2e-3
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    require_gpu()
+
+
+def _tdt(act):
+    return torch.bfloat16 if act == DT_BF16 else torch.float16
+
+
+SHAPES = [
+    # (N, K, scale_group, act)
+    (256, 256, 256, DT_F16),      # per-row scales, two slices
+    (1000, 2048, 64, DT_BF16),    # block scales, ragged row chunks
+    (4, 128, 128, DT_F16),        # one slice: no split-K, y written directly
+    (132, 16384, 64, DT_F16),     # the largest K this kernel takes
+    (2052, 1024, 1024, DT_BF16),  # rows not a multiple of the 512-row chunk
+]
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: f"{s[0]}x{s[1]}sg{s[2]}a{s[3]}")
+@pytest.mark.parametrize("path", [vq.VQ_PATH_GATHER, vq.VQ_PATH_AUTO], ids=["forced", "auto"])
+def test_gather_matches_oracle(oracle, shape, path):
+    N, K, sg, act = shape
+    layer = make_layer(LayerSpec(N, K, FMT_VQ16, sg), cfg_id=70, tensor_id=N)
+    L = layer_on_gpu(layer, act, 1)
+    x = make_x(1, K, act, cfg_id=70)
+    y1 = run_forward(L, x, act, path)
+    y2 = run_forward(L, x, act, path)
+    vq.vq_linear_check(L.handle)
+    y_ref = oracle.forward(layer, x, act)
+    w, _ = oracle.dequant(layer)
+    assert_y_within(y1, act, y_ref, oracle.tolerance(x, act, w, TOL), what=f"gather {shape}")
+    assert np.array_equal(y1, y2), "not bit-identical run to run"
+
+
+def test_gather_config3_sampled(oracle):
+    spec = CONFIGS[3]["tensors"][0][1]
+    layer = make_layer(spec, cfg_id=3)
+    L = layer_on_gpu(layer, DT_F16, 1)
+    x = make_x(1, spec.K, DT_F16, cfg_id=71)
+    y = run_forward(L, x, DT_F16, vq.VQ_PATH_GATHER)
+    rows = np.sort(np.random.default_rng(3).choice(spec.N, size=512, replace=False))
+    y_ref = oracle.forward(layer, x, DT_F16, rows=rows)
+    w, _ = oracle.dequant(layer, rows=rows)
+    assert_y_within(y[:, rows], DT_F16, y_ref, oracle.tolerance(x, DT_F16, w, TOL), what="cfg3 gather", strict=True)
+
+
+def test_gather_with_sm_budget(oracle):
+    layer = make_layer(LayerSpec(1000, 2048, FMT_VQ16, 64), cfg_id=72)
+    L = layer_on_gpu(layer, DT_F16, 1)
+    x = make_x(1, 2048, DT_F16, cfg_id=72)
+    y_ref = oracle.forward(layer, x, DT_F16)
+    w, _ = oracle.dequant(layer)
+    for budget in (1, 5, 0):
+        L.set_sm_budget(budget)
+        y = run_forward(L, x, DT_F16, vq.VQ_PATH_GATHER)
+        assert_y_within(y, DT_F16, y_ref, oracle.tolerance(x, DT_F16, w, TOL), what=f"budget {budget}")
+
+
+@pytest.mark.parametrize("N, K, fmt, M", [(256, 16512, FMT_VQ16, 1), (258, 256, FMT_VQ16, 1),
+                                          (256, 256, FMT_VQ16, 2), (256, 256, FMT_RVQ12_4, 1)])
+def test_gather_rejects_what_it_does_not_take(N, K, fmt, M):
+    layer = make_layer(LayerSpec(N, K, fmt, 64), cfg_id=73)
+    L = layer_on_gpu(layer, DT_F16, 2)
+    L.set_path(vq.VQ_PATH_GATHER)
+    x = torch.zeros((M, K), dtype=torch.float16, device="cuda")
+    with pytest.raises(vq.VQError) as ei:
+        L.forward(x)
+    assert ei.value.status == vq._binding.VQ_ERR_UNSUPPORTED
+
+
+def _rotated_reference(oracle, layer, x, act, signs, rows):
+    """Unrounded fp64 rotation of x times the exact weights of `rows`, with its bound."""
+    xr = oracle.rht(x, act, signs)
+    w, _ = oracle.dequant(layer, rows=rows)
+    y_ref = xr @ w.T
+    tol = TOL * np.sqrt((xr * xr).sum(axis=1, keepdims=True)) * np.abs(w).max()
+    return y_ref, tol
+
+
+@pytest.mark.parametrize("shape", [(256, 256, 256, DT_F16), (520, 2048, 64, DT_BF16), (64, 128, 128, DT_F16),
+                                   (256, 512, 512, DT_BF16), (128, 1024, 64, DT_F16), (132, 16384, 64, DT_F16)],
+                         ids=lambda s: f"{s[0]}x{s[1]}sg{s[2]}a{s[3]}")
+def test_rotated_fused_matches_oracle(oracle, shape):
+    N, K, sg, act = shape
+    layer = make_layer(LayerSpec(N, K, FMT_VQ16, sg), cfg_id=74, tensor_id=N)
+    L = layer_on_gpu(layer, act, 1)
+    assert L.launches(1) == 1
+    x = make_x(1, K, act, cfg_id=74)
+    signs = make_signs(K, cfg_id=74)
+    xt, st = dev(x).view(_tdt(act)), dev(signs)
+    y1 = host_bits(L.forward_rotated(xt, st))
+    y2 = host_bits(L.forward_rotated(xt, st))
+    torch.cuda.synchronize()
+    vq.vq_linear_check(L.handle)
+    y_ref, tol = _rotated_reference(oracle, layer, x, act, signs, None)
+    assert_y_within(y1, act, y_ref, tol, what=f"fused rotation {shape}")
+    assert np.array_equal(y1, y2), "not bit-identical run to run"
+
+
+@pytest.mark.parametrize("M", [1, 8])
+def test_rotated_config3(oracle, M):
+    """Config 3: M = 1 runs the fused kernel, M = 8 the rotation into the handle's
+    buffer followed by the forward (the handle is created with rht = 1)."""
+    spec = CONFIGS[3]["tensors"][0][1]
+    layer = make_layer(spec, cfg_id=3)
+    L = vq.VQLinear(spec.N, spec.K, spec.fmt, spec.scale_group, DT_F16, 8, layer, rht=1)
+    x = make_x(M, spec.K, DT_F16, cfg_id=3)
+    signs = make_signs(spec.K, cfg_id=3)
+    y = host_bits(L.forward_rotated(dev(x).view(torch.float16), dev(signs)))
+    torch.cuda.synchronize()
+    vq.vq_linear_check(L.handle)
+    rows = np.sort(np.random.default_rng(M).choice(spec.N, size=512, replace=False))
+    if M == 1:
+        y_ref, tol = _rotated_reference(oracle, layer, x, DT_F16, signs, rows)
+    else:
+        x_rot = oracle.round_to(oracle.rht(x, DT_F16, signs), DT_F16)
+        y_ref = oracle.forward(layer, x_rot, DT_F16, rows=rows)
+        w, _ = oracle.dequant(layer, rows=rows)
+        tol = oracle.tolerance(x_rot, DT_F16, w, TOL)
+    assert_y_within(y[:, rows], DT_F16, y_ref, tol, what=f"cfg3 rotated M={M}", strict=True)
+
+
+def test_rotated_argument_errors():
+    layer = make_layer(LayerSpec(256, 256, FMT_VQ16, 256), cfg_id=75)
+    L = layer_on_gpu(layer, DT_F16, 8)  # rht = 0: no rotation buffer
+    signs = dev(make_signs(256, cfg_id=75))
+    x8 = torch.zeros((8, 256), dtype=torch.float16, device="cuda")
+    with pytest.raises(vq.VQError) as ei:  # M = 8 is not fused and the handle has no buffer
+        L.forward_rotated(x8, signs)
+    assert ei.value.status == vq._binding.VQ_ERR_INVALID_ARG
+    y = torch.empty((1, 256), dtype=torch.float16, device="cuda")
+    with pytest.raises(vq.VQError) as ei:
+        vq.vq_linear_forward_rotated(L.handle, x8[:1], None, L.planes, L.codebooks, L.t["scales"], y, 1, 256, 256)
+    assert ei.value.status == vq._binding.VQ_ERR_INVALID_ARG
+    layer2 = make_layer(LayerSpec(256, 384, FMT_VQ16, 384), cfg_id=75)
+    L2 = layer_on_gpu(layer2, DT_F16, 1)
+    with pytest.raises(vq.VQError) as ei:  # K not a power of two
+        L2.forward_rotated(torch.zeros((1, 384), dtype=torch.float16, device="cuda"), dev(make_signs(384, cfg_id=75)))
+    assert ei.value.status == vq._binding.VQ_ERR_INVALID_ARG
