@@ -50,7 +50,7 @@ METRIC = "vq_linear µs/layer & achieved HBM GB/s (% of roofline) at batch 1/16;
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 WORKLOADS = {
-    "llama3-8b-mlp": dict(cfg=4, layers=1),
+    "llama3-8b-mlp": dict(cfg=4, layers=1, gate_up_concurrent=True),
     "smollm-135m-stack": dict(cfg=2, layers=30),
     "vq16-4096-rht": dict(cfg=3, layers=1),
     "prefill-8192": dict(cfg=5, layers=1),
@@ -167,6 +167,14 @@ class Workload:
         self.replicas = [self.layers]
         for _ in range(1, replicas):
             self.replicas.append([(name, spec, _clone_layer(L)) for name, spec, L in self.layers])
+        # An MLP's gate and up projections read the same x and are independent: a step
+        # issues them concurrently on two streams, each limited to half of the SMs
+        # (vq_linear_set_sm_budget), then the down projection.
+        self.role = {id(L): name.split(".")[1] for rep in self.replicas for name, _, L in rep}
+        self.concurrent_gate_up = any(self.role[id(L)] == "gate" for _, _, L in self.layers) and \
+            w.get("gate_up_concurrent", False)
+        self.side = torch.cuda.Stream()
+        self.sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
         self.rht = self.cfg["rht"]
         K0 = self.layers[0][1].K
         self.x0 = torch.from_numpy(make_x(max_M, K0, self.act, cfg_id=w["cfg"], seed=seed).view(np.int16)).cuda() \
@@ -204,16 +212,43 @@ class Workload:
                 x = y
         return calls
 
-    def enqueue(self, calls, M, events=None):
-        import compressed_index_matmul_b200 as vq
+    def _forward(self, L, inp, y):
+        if self.rht:  # the layer rotates its input (vq_linear_forward_rotated)
+            L.forward_rotated(inp, self.signs, y)
+        else:
+            L.forward(inp, y)
 
-        for i, (L, inp, y) in enumerate(calls):
+    def _pair(self, a, b):
+        return (self.concurrent_gate_up and self.role[id(a[0])] == "gate" and self.role[id(b[0])] == "up"
+                and a[1] is b[1])
+
+    def enqueue(self, calls, M, events=None, concurrent=True):
+        """Enqueue one step on the current stream.  With `events` (per-forward timing) or
+        `concurrent` false every forward runs alone on the current stream; otherwise gate
+        and up run concurrently."""
+        import torch
+
+        cur = torch.cuda.current_stream()
+        i = 0
+        while i < len(calls):
+            if concurrent and events is None and i + 1 < len(calls) and self._pair(calls[i], calls[i + 1]):
+                (g, gi, gy), (u, ui, uy) = calls[i], calls[i + 1]
+                half = self.sms // 2
+                g.set_sm_budget(half)
+                u.set_sm_budget(self.sms - half)
+                self.side.wait_stream(cur)
+                with torch.cuda.stream(self.side):
+                    self._forward(u, ui, uy)
+                self._forward(g, gi, gy)
+                cur.wait_stream(self.side)
+                g.set_sm_budget(0)
+                u.set_sm_budget(0)
+                i += 2
+                continue
             if events is not None:
                 events[i].record()
-            if self.rht:  # the layer rotates its input (vq_linear_forward_rotated)
-                L.forward_rotated(inp, self.signs, y)
-            else:
-                L.forward(inp, y)
+            self._forward(*calls[i])
+            i += 1
         if events is not None:
             events[len(calls)].record()
 
@@ -337,7 +372,8 @@ def time_graph(wl, M, steps, warmup, per_kernel=False):
 
 
 def time_e2e(wl, M, steps, warmup):
-    """Public API end to end: pinned-host x -> device, eager vq_linear_forward calls, y -> pinned host."""
+    """Public API end to end: pinned-host x -> device, eager vq_linear_forward calls one after
+    another on one stream, y -> pinned host."""
     import torch
 
     stream = torch.cuda.Stream()
@@ -357,7 +393,7 @@ def time_e2e(wl, M, steps, warmup):
             e1 = torch.cuda.Event(enable_timing=True)
             e0.record(stream)
             dev_x[:M].copy_(host_x, non_blocking=True)
-            wl.enqueue(calls, M)
+            wl.enqueue(calls, M, concurrent=False)  # eager calls on one stream (no fork / join per step)
             host_y.copy_(last, non_blocking=True)
             e1.record(stream)
             e1.synchronize()
@@ -456,6 +492,9 @@ def gpu_arm(args):
     avg_launch_us = round(1e3 * float(np.mean(per_fwd_eff)), 3)
     if not uniform:
         launch_source = "CUDA event nodes between the forwards"
+    elif launches_per_fwd[0] == 1 and wl.concurrent_gate_up:
+        launch_source = ("timed region / forwards (every launch is this kernel; gate and up overlap on two "
+                         "streams, so this is the step's time per weight matrix)")
     elif launches_per_fwd[0] == 1:
         launch_source = "timed region / launches (every launch is this kernel)"
     else:
@@ -498,7 +537,9 @@ def gpu_arm(args):
                    "l2": L2_NOTE.format(r=R, mb=R * wl.weight_bytes() / 1e6) + (
                        "; the 65,536-entry codebook is one table shared by the copies (L2-resident)"
                        if fmt0 == FMT_VQ16 else ""),
-                   "layer": "one vq_linear_forward (one weight matrix)",
+                   "layer": ("MLP step / 3 weight matrices: gate and up (same x) run concurrently on two "
+                             "streams, half of the SMs each (vq_linear_set_sm_budget), then down"
+                             if wl.concurrent_gate_up else "one vq_linear_forward (one weight matrix)"),
                    "hbm_gbs": round(sum(bytes_per_fwd) / (ms_per_step * 1e-3) / 1e9, 1)},
         "roofline": roofline,
         "e2e": e2e,
