@@ -142,15 +142,14 @@ bool plan_forward(const vq_linear_desc& d, const DeviceInfo& dev, int M, int for
     // Measured on B200: from M = 2 the tensor-core path decodes large layers
     // faster than the warp-MMA GEMV; on small layers both are launch-bound.
     const bool large = (int64_t)d.N * d.K >= (int64_t(1) << 22);
-    path = (M == 1) ? (d.fmt == VQ_FMT_VQ16 ? VQ_PATH_GATHER : VQ_PATH_LUT)
-                    : ((M <= 16 && !large) ? VQ_PATH_GEMV : VQ_PATH_TC);
+    path = (M == 1) ? VQ_PATH_LUT : ((M <= 16 && !large) ? VQ_PATH_GEMV : VQ_PATH_TC);
+    // 16-bit indices, up to 4 tokens: the gather kernel where it applies (measured on
+    // B200, 4096 x 4096: faster than the tensor-core path up to M = 4, slower at 8)
+    if (d.fmt == VQ_FMT_VQ16 && M <= 4 && plan_vq16(d, dev, M, out)) return true;
   }
   switch (path) {
     case VQ_PATH_GATHER:
-      if (plan_vq16(d, dev, M, out)) return true;
-      if (forced_path != VQ_PATH_AUTO) return false;
-      plan_gemv(d, dev, M, out);
-      return true;
+      return plan_vq16(d, dev, M, out);
     case VQ_PATH_LUT:
       if (plan_lut(d, dev, M, out)) return true;
       if (forced_path != VQ_PATH_AUTO) return false;
@@ -355,7 +354,7 @@ VQ_API vq_status vq_linear_forward_rotated(vq_linear_t h, const void* x, const i
   if (!vq::plan_forward(d, h->dev, M, h->path, &p))
     return fail(VQ_ERR_UNSUPPORTED, "path %d cannot run M=%d", h->path, M);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (p.path == VQ_PATH_GATHER) {
+  if (p.path == VQ_PATH_GATHER && M == 1) {  // the kernel rotates x itself
     if (h->sm_budget > 0 && p.grid > h->sm_budget) p.grid = h->sm_budget;
     if (p.scratch_bytes > h->scratch_bytes)
       return fail(VQ_ERR_UNSUPPORTED, "plan needs %zu scratch bytes, handle has %zu", p.scratch_bytes,

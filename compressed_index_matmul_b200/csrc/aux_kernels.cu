@@ -2,6 +2,7 @@
 // rotation (sign flip + fast Walsh-Hadamard transform), and the debug exports
 // that materialise unpacked indices / decoded weights into caller buffers.
 #include "common.cuh"
+#include "rotate.cuh"
 #include "internal.h"
 #include "tc_ptx.cuh"
 
@@ -37,57 +38,36 @@ cudaError_t launch_split_reduce(const float* partial, void* y, int splits, int M
 // ---------------------------------------------------------------------- rotation
 //
 // GLQ README, "How it works": Randomized Hadamard Transform = random sign flips
-// followed by a fast Walsh-Hadamard transform.  One CTA per token row: the row is
-// loaded into shared memory as fp32 with the signs applied, transformed with
-// in-place radix-2 butterflies in natural (Sylvester) order, scaled by 1/sqrt(K)
-// and rounded to the element type.  The five lowest stages (pairs inside 32
-// consecutive elements) run on registers with warp shuffles; the rest in shared
-// memory.  Each CTA reads its whole row before writing it, so x_out may be x.
+// followed by a fast Walsh-Hadamard transform.  One CTA of 512 threads per token
+// row: hadamard_to_smem (rotate.cuh) computes H_K (signs . x) in fp32 in shared
+// memory (butterflies on registers and lane shuffles, one shared-memory pass for
+// the highest stages, natural Sylvester order); the row is then scaled by
+// 1/sqrt(K) and rounded to the element type.  Each CTA reads its whole row before
+// writing it, so x_out may be x.
+constexpr int kRhtThreads = 512;
+
 template <typename T>
-__global__ void __launch_bounds__(1024) rht_kernel(const uint16_t* __restrict__ x, uint16_t* __restrict__ xo,
-                                                   const int8_t* __restrict__ signs, int K, float scale) {
+__global__ void __launch_bounds__(kRhtThreads) rht_kernel(const uint16_t* __restrict__ x, uint16_t* __restrict__ xo,
+                                                          const int8_t* __restrict__ signs, int K, float scale) {
   extern __shared__ float buf[];
   const int64_t row = blockIdx.x;
-  const uint16_t* xr = x + row * K;
-  const int lane = threadIdx.x & 31;
-  // Stages h = 1..16 on registers: element i = 32*w + lane of each 32-chunk.
-  for (int base = (threadIdx.x & ~31); base < K; base += blockDim.x) {
-    const int i = base + lane;
-    float v = Elt<T>::to_f32(xr[i]) * (float)signs[i];
-#pragma unroll
-    for (int h = 1; h < 32; h <<= 1) {
-      const float o = __shfl_xor_sync(0xffffffffu, v, h);
-      v = (lane & h) ? (o - v) : (v + o);
-    }
-    buf[i] = v;
-  }
-  __syncthreads();
-  for (int h = 32; h < K; h <<= 1) {
-    for (int t = threadIdx.x; t < K / 2; t += blockDim.x) {
-      const int i = (t / h) * (2 * h) + (t % h);
-      const float a = buf[i], b = buf[i + h];
-      buf[i] = a + b;
-      buf[i + h] = a - b;
-    }
-    __syncthreads();
-  }
+  hadamard_to_smem<T, kRhtThreads, 32768>(x + row * K, signs, buf, K, threadIdx.x);
   uint16_t* orow = xo + row * K;
-  for (int i = threadIdx.x; i < K; i += blockDim.x) orow[i] = Elt<T>::from_f32(buf[i] * scale);
+  for (int i = threadIdx.x; i < K; i += kRhtThreads) orow[i] = Elt<T>::from_f32(buf[i] * scale);
 }
 
 cudaError_t launch_rht(const void* x, void* x_out, const int8_t* signs, int M, int K, int dtype, cudaStream_t s) {
-  const int threads = K < 1024 ? K : 1024;
   const size_t smem = (size_t)K * sizeof(float);
   const float scale = (float)(1.0 / __builtin_sqrt((double)K));
   cudaError_t e;
   if (dtype == VQ_BF16) {
     e = cudaFuncSetAttribute(rht_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    rht_kernel<__nv_bfloat16><<<M, threads, smem, s>>>((const uint16_t*)x, (uint16_t*)x_out, signs, K, scale);
+    rht_kernel<__nv_bfloat16><<<M, kRhtThreads, smem, s>>>((const uint16_t*)x, (uint16_t*)x_out, signs, K, scale);
   } else {
     e = cudaFuncSetAttribute(rht_kernel<__half>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    rht_kernel<__half><<<M, threads, smem, s>>>((const uint16_t*)x, (uint16_t*)x_out, signs, K, scale);
+    rht_kernel<__half><<<M, kRhtThreads, smem, s>>>((const uint16_t*)x, (uint16_t*)x_out, signs, K, scale);
   }
   return cudaGetLastError();
 }

@@ -1,0 +1,114 @@
+// Unnormalised randomized Hadamard rotation of one token, H_K (signs . x), into
+// shared memory (fp32), by NT threads of a CTA (named barrier 1).
+//
+// GLQ README, "How it works": random sign flips followed by a fast Walsh-Hadamard
+// transform.  K = 2^p with 64 <= K <= 64 NT.  Every stage is a butterfly
+// (u + w, u - w) on one index bit; the stages commute, so the result is
+// H_K (signs . x) with H_K[k][j] = (-1)^popcount(k & j) (natural Sylvester
+// order) whatever order they run in.  With E = max(1, K / NT) elements per thread
+// and R = K / (32 E) (both compile-time, so every stage is straight-line code):
+//   pass 1: thread t holds E consecutive elements; the log2(E) lowest stages run
+//           on registers, the next five across the warp's lanes with shuffles;
+//   pass 2: the log2(R) highest stages run on registers over groups of R
+//           elements at stride 32 E.
+// Used by the rotation kernel (vq_rht_apply) and by the batch-1 16-bit kernel,
+// which rotates x itself.
+#pragma once
+
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace vq {
+
+template <typename T, int E, int R, int NT>
+__device__ __forceinline__ void hadamard_pass(const uint16_t* __restrict__ x, const int8_t* __restrict__ signs,
+                                              float* xs, int tid) {
+  constexpr int K = 32 * E * R;
+  constexpr int D = 32 * E;
+  const int lane = tid & 31;
+  if (tid * E < K) {  // whole warps (K is a multiple of 32 E)
+    float v[E];
+    if (E >= 8) {
+      // E consecutive inputs (16-byte loads) and signs (8-byte loads)
+#pragma unroll
+      for (int c = 0; c < E / 8; ++c) {
+        const uint4 xw = *reinterpret_cast<const uint4*>(x + tid * E + 8 * c);
+        const uint2 sw = *reinterpret_cast<const uint2*>(signs + tid * E + 8 * c);
+        const uint32_t xa[4] = {xw.x, xw.y, xw.z, xw.w};
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const int8_t sg = (int8_t)(((q < 4 ? sw.x : sw.y) >> (8 * (q & 3))) & 0xFFu);
+          v[8 * c + q] = Elt<T>::to_f32((uint16_t)(xa[q >> 1] >> (16 * (q & 1)))) * (float)sg;
+        }
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < E; ++e) v[e] = Elt<T>::to_f32(x[tid * E + e]) * (float)signs[tid * E + e];
+    }
+#pragma unroll
+    for (int h = 1; h < E; h <<= 1)  // stages h = 1 .. E/2 on registers
+#pragma unroll
+      for (int e = 0; e < E; ++e)
+        if (!(e & h)) {
+          const float u = v[e], w = v[e + h];
+          v[e] = u + w;
+          v[e + h] = u - w;
+        }
+#pragma unroll
+    for (int m = 1; m < 32; m <<= 1)  // stages h = E .. 16 E across the lanes
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const float o = __shfl_xor_sync(0xffffffffu, v[e], m);
+        v[e] = (lane & m) ? (o - v[e]) : (v[e] + o);
+      }
+#pragma unroll
+    for (int e = 0; e < E; ++e) xs[tid * E + e] = v[e];
+  }
+  asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory");
+  for (int gb = tid; gb < D; gb += NT) {  // stages h = 32 E .. K/2
+    float u[R];
+#pragma unroll
+    for (int j = 0; j < R; ++j) u[j] = xs[gb + j * D];
+#pragma unroll
+    for (int h = 1; h < R; h <<= 1)
+#pragma unroll
+      for (int j = 0; j < R; ++j)
+        if (!(j & h)) {
+          const float p = u[j], q = u[j + h];
+          u[j] = p + q;
+          u[j + h] = p - q;
+        }
+#pragma unroll
+    for (int j = 0; j < R; ++j) xs[gb + j * D] = u[j];
+  }
+  asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory");
+}
+
+// hadamard_pass for a power-of-two K in [64, kMaxK] (NT = 512; kMaxK <= 32768 bounds
+// the registers the instantiations need).
+template <typename T, int NT, int kMaxK>
+__device__ __forceinline__ void hadamard_to_smem(const uint16_t* x, const int8_t* signs, float* xs, int K, int tid) {
+  static_assert(NT == 512 && kMaxK >= 16384 && kMaxK <= 32768, "the stage split below assumes 512 threads");
+  switch (K) {
+    case 64: hadamard_pass<T, 1, 2, NT>(x, signs, xs, tid); break;
+    case 128: hadamard_pass<T, 1, 4, NT>(x, signs, xs, tid); break;
+    case 256: hadamard_pass<T, 1, 8, NT>(x, signs, xs, tid); break;
+    case 512: hadamard_pass<T, 1, 16, NT>(x, signs, xs, tid); break;
+    case 1024: hadamard_pass<T, 2, 16, NT>(x, signs, xs, tid); break;
+    case 2048: hadamard_pass<T, 4, 16, NT>(x, signs, xs, tid); break;
+    case 4096: hadamard_pass<T, 8, 16, NT>(x, signs, xs, tid); break;
+    case 8192: hadamard_pass<T, 16, 16, NT>(x, signs, xs, tid); break;
+    default:
+      if constexpr (kMaxK >= 32768) {
+        if (K == 32768) {
+          hadamard_pass<T, 64, 16, NT>(x, signs, xs, tid);
+          break;
+        }
+      }
+      hadamard_pass<T, 32, 16, NT>(x, signs, xs, tid);  // 16384
+      break;
+  }
+}
+
+}  // namespace vq

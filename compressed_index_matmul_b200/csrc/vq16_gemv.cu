@@ -1,6 +1,6 @@
-// Batch-1 GEMV for the single-stage 16-bit format (M == 1, VQ_FMT_VQ16,
-// K % 128 == 0, K <= 16384, N % 4 == 0), with the input rotation optionally
-// applied inside the kernel.
+// Small-batch GEMV for the single-stage 16-bit format (1 <= M <= 8, VQ_FMT_VQ16,
+// K % 128 == 0, K <= 16384, M K <= 32768, N % 4 == 0), with the input rotation
+// optionally applied inside the kernel at M == 1.
 //
 // GLQ README, "How it works": one 16-bit index per group of 8 weights selects a
 // codeword of a 65,536 x 8 codebook (1 MiB of fp16), too large for shared memory;
@@ -8,20 +8,21 @@
 // L2-resident codebook.  Each group of row n contributes s * (x_g . cb[i]), so a
 // lookup thread gathers its row's 16 codewords of a K-slice at once (16 x 16-byte
 // loads in flight per thread, 8192 per SM) and dots them with the slice's x held
-// in shared memory (one broadcast load per 4 inputs).
+// in shared memory (one broadcast load per 4 inputs and token); every gathered
+// codeword serves all M tokens.
 //
 // Rotated input (GLQ README, "How it works": random sign flips followed by a fast
-// Walsh-Hadamard transform): when `signs` is given, every CTA computes the whole
-// rotated vector x' = H (signs . x) in fp32 in shared memory (the five lowest
-// butterfly stages on registers with warp shuffles, the rest in shared memory,
-// natural Sylvester order); the orthonormal factor 1/sqrt(K) multiplies every
-// partial sum.  The caller's x is the unrotated input, and no rotated copy of it
+// Walsh-Hadamard transform): when `signs` is given (M == 1), every CTA computes the
+// whole rotated vector x' = H (signs . x) in fp32 in shared memory
+// (hadamard_to_smem, rotate.cuh); the orthonormal factor 1/sqrt(K) multiplies
+// every partial sum.  The caller's x is the unrotated input, and no rotated copy of it
 // is ever written to memory.
 //
 // Work split and reduction: no table is built, so the (K-slice, row) grid is cut
 // in two dimensions.  CTAs form clusters of 2 (pairs fill every SM; larger
 // clusters leave SMs of each GPC idle); a cluster owns blocks of up to 512 output
-// rows, and CTA j of the pair takes slices [S j / 2, S (j+1) / 2) of them.  Each thread handles one (slice, row) position of a chunk of 512: it
+// rows, and CTA j of the pair takes slices [S j / 2, S (j+1) / 2) of them.  Each
+// thread handles one (slice, row) position of a chunk of 512: it
 // loads the row's 16 indices (two 16-byte loads, issued one chunk ahead) and its
 // scales, gathers and dots, and stores the position's partial sum in shared
 // memory.  Each CTA then adds its slices per row in slice order, and CTA j reduces
@@ -34,6 +35,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "rotate.cuh"
 #include "tc_ptx.cuh"
 
 namespace vq {
@@ -44,17 +46,21 @@ constexpr int kV16MaxBlk = 512;     // rows per cluster block
 constexpr int kV16MaxK = 16384;
 constexpr int kV16MaxSpc = kV16MaxK / 128 / kV16Cluster;  // slices per CTA
 
-// Shared memory of one CTA: partials [ceil(S / C)][rblk], row sums [rblk], fp32 x [K]
-// (byte offsets, 16-byte aligned; rblk is a multiple of 4).
+constexpr int kV16MaxM = 8;           // tokens
+constexpr int kV16MaxMK = 32768;      // tokens x K (the fp32 x of all tokens is in shared memory)
+constexpr int kV16PartBytes = 65536;  // partial sums of one block
+
+// Shared memory of one CTA: partials [ceil(S / C)][MT][rblk], row sums [MT][rblk],
+// fp32 x [MT][K] (byte offsets, 16-byte aligned; rblk is a multiple of 4).
 struct V16Smem {
   int off_sum, off_x, bytes;
 };
-__host__ __device__ inline V16Smem v16_smem(int S, int rblk, int K) {
+__host__ __device__ inline V16Smem v16_smem(int S, int MT, int rblk, int K) {
   V16Smem m;
   const int spc = (S + kV16Cluster - 1) / kV16Cluster;
-  m.off_sum = spc * rblk * 4;
-  m.off_x = m.off_sum + rblk * 4;
-  m.bytes = m.off_x + 4 * K;
+  m.off_sum = spc * MT * rblk * 4;
+  m.off_x = m.off_sum + MT * rblk * 4;
+  m.bytes = m.off_x + 4 * MT * K;
   return m;
 }
 
@@ -73,94 +79,6 @@ __device__ __forceinline__ float dot8(const uint4& c, const float4& xa, const fl
   return acc;
 }
 
-// Unnormalised rotation H_K (signs . x) of one token into xs (fp32), K = 2^p with
-// 128 <= K <= kV16MaxK, by the kV16Consumers threads (named barrier 1), with
-// E = max(1, K/512) elements per thread and R = K / (32 E) (compile-time, so every
-// stage is straight-line code).  Pass 1: thread t holds E consecutive elements;
-// the log2(E) lowest butterfly stages run on registers, the next five across the
-// warp's lanes with shuffles.  Pass 2: the log2(R) remaining (highest) stages run
-// on registers over groups of R elements at stride 32 E.  Every stage is a
-// butterfly (u + w, u - w) on one index bit, so the result is H_K (signs . x) with
-// H_K[k][j] = (-1)^popcount(k & j) (natural Sylvester order).
-template <typename T, int E, int R>
-__device__ __forceinline__ void rotate_to_smem(const uint16_t* __restrict__ x, const int8_t* __restrict__ signs,
-                                               float* xs, int tid) {
-  constexpr int K = 32 * E * R;
-  constexpr int D = 32 * E;
-  const int lane = tid & 31;
-  if (tid * E < K) {  // whole warps (K is a multiple of 32 E)
-    float v[E];
-    if (E >= 8) {
-      // E consecutive inputs (16-byte loads) and signs (8-byte loads)
-#pragma unroll
-      for (int c = 0; c < E / 8; ++c) {
-        const uint4 xw = *reinterpret_cast<const uint4*>(x + tid * E + 8 * c);
-        const uint2 sw = *reinterpret_cast<const uint2*>(signs + tid * E + 8 * c);
-        const uint32_t xa[4] = {xw.x, xw.y, xw.z, xw.w};
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const int8_t sg = (int8_t)(((q < 4 ? sw.x : sw.y) >> (8 * (q & 3))) & 0xFFu);
-          v[8 * c + q] = Elt<T>::to_f32((uint16_t)(xa[q >> 1] >> (16 * (q & 1)))) * (float)sg;
-        }
-      }
-    } else {
-#pragma unroll
-      for (int e = 0; e < E; ++e) v[e] = Elt<T>::to_f32(x[tid * E + e]) * (float)signs[tid * E + e];
-    }
-#pragma unroll
-    for (int h = 1; h < E; h <<= 1)  // stages h = 1 .. E/2 on registers
-#pragma unroll
-      for (int e = 0; e < E; ++e)
-        if (!(e & h)) {
-          const float u = v[e], w = v[e + h];
-          v[e] = u + w;
-          v[e + h] = u - w;
-        }
-#pragma unroll
-    for (int m = 1; m < 32; m <<= 1)  // stages h = E .. 16 E across the lanes
-#pragma unroll
-      for (int e = 0; e < E; ++e) {
-        const float o = __shfl_xor_sync(0xffffffffu, v[e], m);
-        v[e] = (lane & m) ? (o - v[e]) : (v[e] + o);
-      }
-#pragma unroll
-    for (int e = 0; e < E; ++e) xs[tid * E + e] = v[e];
-  }
-  asm volatile("bar.sync 1, %0;" ::"n"(kV16Consumers) : "memory");
-  for (int gb = tid; gb < D; gb += kV16Consumers) {  // stages h = 32 E .. K/2
-    float u[R];
-#pragma unroll
-    for (int j = 0; j < R; ++j) u[j] = xs[gb + j * D];
-#pragma unroll
-    for (int h = 1; h < R; h <<= 1)
-#pragma unroll
-      for (int j = 0; j < R; ++j)
-        if (!(j & h)) {
-          const float p = u[j], q = u[j + h];
-          u[j] = p + q;
-          u[j + h] = p - q;
-        }
-#pragma unroll
-    for (int j = 0; j < R; ++j) xs[gb + j * D] = u[j];
-  }
-  asm volatile("bar.sync 1, %0;" ::"n"(kV16Consumers) : "memory");
-}
-
-// rotate_to_smem for a power-of-two K in [128, kV16MaxK].
-template <typename T>
-__device__ __forceinline__ void rotate_any(const uint16_t* x, const int8_t* signs, float* xs, int K, int tid) {
-  switch (K) {
-    case 128: rotate_to_smem<T, 1, 4>(x, signs, xs, tid); break;
-    case 256: rotate_to_smem<T, 1, 8>(x, signs, xs, tid); break;
-    case 512: rotate_to_smem<T, 1, 16>(x, signs, xs, tid); break;
-    case 1024: rotate_to_smem<T, 2, 16>(x, signs, xs, tid); break;
-    case 2048: rotate_to_smem<T, 4, 16>(x, signs, xs, tid); break;
-    case 4096: rotate_to_smem<T, 8, 16>(x, signs, xs, tid); break;
-    case 8192: rotate_to_smem<T, 16, 16>(x, signs, xs, tid); break;
-    default: rotate_to_smem<T, 32, 16>(x, signs, xs, tid); break;  // 16384
-  }
-}
-
 __device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
   float v;
   asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
@@ -173,16 +91,17 @@ struct V16Pos {
   uint32_t sc;
 };
 
-template <typename T>
+// MT: tokens rounded up to 1, 2, 4 or 8 (the x of tokens M .. MT-1 is zero).
+template <typename T, int MT>
 __global__ void __launch_bounds__(kV16Consumers, 1)
     vq16_gemv_kernel(LayerArgs a, const int8_t* __restrict__ signs, float xscale, int S, int blocks_per_cluster,
                      int rblk) {
   extern __shared__ __align__(128) unsigned char smem[];
-  const int N = a.N, K = a.K;
-  const V16Smem lay = v16_smem(S, rblk, K);
-  float* part = reinterpret_cast<float*>(smem);                 // [ceil(S / C)][rblk]
-  float* csum = reinterpret_cast<float*>(smem + lay.off_sum);  // [rblk]
-  float* xs = reinterpret_cast<float*>(smem + lay.off_x);      // [K]
+  const int N = a.N, K = a.K, M = a.M;
+  const V16Smem lay = v16_smem(S, MT, rblk, K);
+  float* part = reinterpret_cast<float*>(smem);                 // [ceil(S / C)][MT][rblk]
+  float* csum = reinterpret_cast<float*>(smem + lay.off_sum);  // [MT][rblk]
+  float* xs = reinterpret_cast<float*>(smem + lay.off_x);      // [MT][K]
   const int tid = threadIdx.x;
   const bool block_scales = (a.scale_group == 64);
   uint32_t rank;
@@ -210,11 +129,11 @@ __global__ void __launch_bounds__(kV16Consumers, 1)
   if (tid < ns * nrows) load_pos(tid, r0, nrows, cur);
 
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  if (signs) {
-    rotate_any<T>(static_cast<const uint16_t*>(a.x), signs, xs, K, tid);
+  if (MT == 1 && signs) {
+    hadamard_to_smem<T, kV16Consumers, kV16MaxK>(static_cast<const uint16_t*>(a.x), signs, xs, K, tid);
   } else {
     const uint16_t* xg = static_cast<const uint16_t*>(a.x);
-    for (int i = tid; i < K; i += kV16Consumers) xs[i] = Elt<T>::to_f32(xg[i]);
+    for (int i = tid; i < MT * K; i += kV16Consumers) xs[i] = i < M * K ? Elt<T>::to_f32(xg[i]) : 0.f;
     __syncthreads();
   }
 
@@ -237,39 +156,57 @@ __global__ void __launch_bounds__(kV16Consumers, 1)
         uint4 c[16];
 #pragma unroll
         for (int g = 0; g < 16; ++g) c[g] = __ldg(cb + ((iw[g >> 1] >> (16 * (g & 1))) & 0xFFFFu));
-        const float4* xv = reinterpret_cast<const float4*>(xs + (int64_t)(sa + p / nrows) * 128);
-        float blk[2] = {0.f, 0.f};
+        const float* xsl = xs + (sa + p / nrows) * 128;
+        float blk[MT][2];
 #pragma unroll
-        for (int g = 0; g < 16; ++g) blk[g >> 3] = dot8(c[g], xv[2 * g], xv[2 * g + 1], blk[g >> 3]);
-        float acc;
-        if (block_scales) {
-          const float2 sc = f16x2_to_f32x2(cur.sc);
-          acc = fmaf(blk[1], sc.y, blk[0] * sc.x);
-        } else {
-          acc = blk[0] + blk[1];
+        for (int m = 0; m < MT; ++m) blk[m][0] = blk[m][1] = 0.f;
+#pragma unroll
+        for (int g = 0; g < 16; ++g) {
+#pragma unroll
+          for (int m = 0; m < MT; ++m) {
+            const float4* xv = reinterpret_cast<const float4*>(xsl + m * K + 8 * g);
+            blk[m][g >> 3] = dot8(c[g], xv[0], xv[1], blk[m][g >> 3]);
+          }
         }
-        part[(p / nrows) * rblk + p % nrows] = acc;
+        const float2 sc = block_scales ? f16x2_to_f32x2(cur.sc) : make_float2(1.f, 1.f);
+#pragma unroll
+        for (int m = 0; m < MT; ++m)  // the per-row scale is applied once, at the reduction
+          part[((p / nrows) * MT + m) * rblk + p % nrows] =
+              block_scales ? fmaf(blk[m][1], sc.y, blk[m][0] * sc.x) : blk[m][0] + blk[m][1];
       }
       cur = nxt;
     }
     __syncthreads();
     // this CTA's slices, in order, per row of the block
-    for (int r = tid; r < nrows; r += kV16Consumers) {
+    for (int i = tid; i < MT * nrows; i += kV16Consumers) {
+      const int m = i / nrows, r = i - m * nrows;
       float v = 0.f;
-      for (int k = 0; k < ns; ++k) v += part[k * rblk + r];
-      csum[r] = v;
+      for (int k = 0; k < ns; ++k) v += part[(k * MT + m) * rblk + r];
+      csum[m * rblk + r] = v;
     }
-    // rows [nrows j / C, nrows (j+1) / C) of the block: the C CTAs' sums in rank order
+    // rows [nrows j / C, nrows (j+1) / C) of the block, every token: the C CTAs' sums
+    // in rank order (at most MT x kV16MaxBlk / kV16Cluster outputs per CTA)
     const int ra = (int)((int64_t)nrows * rank / kV16Cluster), rb = (int)((int64_t)nrows * (rank + 1) / kV16Cluster);
-    const int r = ra + tid;  // a block has at most kV16MaxBlk / kV16Cluster <= kV16Consumers rows per CTA
-    const float row_scale = (r < rb && !block_scales) ? f16_bits_to_f32(a.scales[r0 + r]) : 1.f;
-    ptx::cluster_sync();  // every CTA's csum is complete and visible to the cluster
-    if (r < rb) {
-      const uint32_t local = smem_u32(csum + r);
-      float v = 0.f;
+    const int nr = rb - ra;
+    constexpr int kOut = (MT * kV16MaxBlk / kV16Cluster + kV16Consumers - 1) / kV16Consumers;
+    float row_scale[kOut];
 #pragma unroll
-      for (int q = 0; q < kV16Cluster; ++q) v += ld_cluster_f32(ptx::map_shared_rank(local, q));
-      static_cast<uint16_t*>(a.y)[r0 + r] = Elt<T>::from_f32(v * xscale * row_scale);
+    for (int o = 0; o < kOut; ++o) {
+      const int i = tid + o * kV16Consumers;
+      row_scale[o] = (i < M * nr && !block_scales) ? f16_bits_to_f32(a.scales[r0 + ra + i % nr]) : 1.f;
+    }
+    ptx::cluster_sync();  // every CTA's csum is complete and visible to the cluster
+#pragma unroll
+    for (int o = 0; o < kOut; ++o) {
+      const int i = tid + o * kV16Consumers;
+      if (i < M * nr) {
+        const int m = i / nr, r = ra + i - m * nr;
+        const uint32_t local = smem_u32(csum + m * rblk + r);
+        float v = 0.f;
+#pragma unroll
+        for (int q = 0; q < kV16Cluster; ++q) v += ld_cluster_f32(ptx::map_shared_rank(local, q));
+        static_cast<uint16_t*>(a.y)[(int64_t)m * N + r0 + r] = Elt<T>::from_f32(v * xscale * row_scale[o]);
+      }
     }
     ptx::cluster_sync();  // no CTA reuses or releases its csum while another reads it
     if (bi + 1 < blocks_per_cluster) {
@@ -282,31 +219,43 @@ __global__ void __launch_bounds__(kV16Consumers, 1)
 
 // Clusters of kV16Cluster CTAs that can be resident at once (the grid may exceed
 // it; clusters are independent).  Queried once per device.
-static int v16_max_clusters(int smem, int num_sms);
+static int v16_max_clusters(int num_sms);
 
 struct V16Geom {
   int ncl, blocks_per_cluster, rblk;
 };
 
-static V16Geom v16_geom(int N, int clusters) {
+// Tokens the kernel is compiled for: M rounded up to 1, 2, 4 or 8.
+static int v16_mt(int M) { return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : 8; }
+
+static V16Geom v16_geom(int N, int clusters, int S, int MT) {
   V16Geom g;
   g.ncl = clusters < 1 ? 1 : clusters;
   const int quads = (N + 3) / 4;
-  g.blocks_per_cluster = (N + g.ncl * kV16MaxBlk - 1) / (g.ncl * kV16MaxBlk);
+  // rows per block: at most 512, and the block's partial sums fit kV16PartBytes
+  const int spc = (S + kV16Cluster - 1) / kV16Cluster;
+  int cap = kV16PartBytes / (spc * MT * 4) / 4 * 4;
+  if (cap > kV16MaxBlk) cap = kV16MaxBlk;
+  if (cap < 4) cap = 4;
+  g.blocks_per_cluster = (N + g.ncl * cap - 1) / (g.ncl * cap);
   const int blocks = g.ncl * g.blocks_per_cluster;
   g.rblk = 4 * ((quads + blocks - 1) / blocks);
-  if (g.rblk > kV16MaxBlk) g.rblk = kV16MaxBlk;
+  if (g.rblk > cap) g.rblk = cap;
   g.ncl = (N + g.rblk * g.blocks_per_cluster - 1) / (g.rblk * g.blocks_per_cluster);  // drop idle clusters
   return g;
 }
 
-static int v16_max_clusters(int smem, int num_sms) {
-  // (the largest shared-memory size any launch asks for, so the count holds for all)
+// Largest shared-memory size of any launch: capped partials, row sums of 8 tokens x
+// 512 rows, fp32 x of M K <= kV16MaxMK inputs.
+static int v16_max_smem() { return kV16PartBytes + kV16MaxM * kV16MaxBlk * 4 + 4 * kV16MaxMK; }
+
+static int v16_max_clusters(int num_sms) {
   static std::atomic<int> cached[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return num_sms / kV16Cluster;
   int c = cached[dev].load(std::memory_order_acquire);
   if (c > 0) return c;
+  const int smem = v16_max_smem();
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(kV16Cluster * (num_sms / kV16Cluster));
   cfg.blockDim = dim3(kV16Consumers);
@@ -319,9 +268,9 @@ static int v16_max_clusters(int smem, int num_sms) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaFuncSetAttribute(vq16_gemv_kernel<__half>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+  if (cudaFuncSetAttribute(vq16_gemv_kernel<__half, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
           cudaSuccess ||
-      cudaOccupancyMaxActiveClusters(&n, vq16_gemv_kernel<__half>, &cfg) != cudaSuccess || n < 1) {
+      cudaOccupancyMaxActiveClusters(&n, vq16_gemv_kernel<__half, 8>, &cfg) != cudaSuccess || n < 1) {
     cudaGetLastError();
     n = num_sms / kV16Cluster;
   }
@@ -330,11 +279,10 @@ static int v16_max_clusters(int smem, int num_sms) {
 }
 
 bool plan_vq16(const vq_linear_desc& d, const DeviceInfo& dev, int M, Plan* p) {
-  if (M != 1 || d.fmt != VQ_FMT_VQ16 || d.K % 128 != 0 || d.K > kV16MaxK || d.N % 4 != 0 ||
-      dev.smem_optin < v16_smem(kV16MaxK / 128, kV16MaxBlk, kV16MaxK).bytes)
+  if (M < 1 || M > kV16MaxM || d.fmt != VQ_FMT_VQ16 || d.K % 128 != 0 || d.K > kV16MaxK ||
+      v16_mt(M) * d.K > kV16MaxMK || d.N % 4 != 0 || dev.smem_optin < v16_max_smem())
     return false;
-  const V16Geom g =
-      v16_geom(d.N, v16_max_clusters(v16_smem(kV16MaxK / 128, kV16MaxBlk, kV16MaxK).bytes, dev.num_sms));
+  const V16Geom g = v16_geom(d.N, v16_max_clusters(dev.num_sms), d.K / 128, v16_mt(M));
   p->path = VQ_PATH_GATHER;
   p->splits = d.K / 128;
   p->k_per_split = 128;
@@ -345,18 +293,17 @@ bool plan_vq16(const vq_linear_desc& d, const DeviceInfo& dev, int M, Plan* p) {
   return true;
 }
 
-template <typename T>
+template <typename T, int MT>
 static cudaError_t launch_vq16_t(const LayerArgs& a, int grid, const int8_t* signs, cudaStream_t s) {
   const int S = a.K / 128;
-  auto kern = vq16_gemv_kernel<T>;
+  auto kern = vq16_gemv_kernel<T, MT>;
   static std::atomic<uint64_t> opted{0};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   const uint64_t bit = dev < 64 ? (uint64_t(1) << dev) : 0;
   if (!(opted.load(std::memory_order_acquire) & bit)) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             v16_smem(kV16MaxK / 128, kV16MaxBlk, kV16MaxK).bytes);
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, v16_max_smem());
     // Prefer L1 over shared memory beyond what a launch asks for: the L1 caches
     // part of the 1 MiB codebook for the gathers.
     if (e == cudaSuccess)
@@ -366,8 +313,8 @@ static cudaError_t launch_vq16_t(const LayerArgs& a, int grid, const int8_t* sig
   }
   int ncl = grid / kV16Cluster;
   if (ncl < 1) ncl = 1;
-  const V16Geom g = v16_geom(a.N, ncl);
-  const int smem = v16_smem(S, g.rblk, a.K).bytes;
+  const V16Geom g = v16_geom(a.N, ncl, S, MT);
+  const int smem = v16_smem(S, MT, g.rblk, a.K).bytes;
   // Orthonormal factor of the rotation, rounded once from double precision.
   const float xscale = signs ? (float)(1.0 / std::sqrt((double)a.K)) : 1.f;
   cudaLaunchConfig_t cfg = {};
@@ -387,9 +334,19 @@ static cudaError_t launch_vq16_t(const LayerArgs& a, int grid, const int8_t* sig
   return cudaLaunchKernelEx(&cfg, kern, a, signs, xscale, S, g.blocks_per_cluster, g.rblk);
 }
 
+template <typename T>
+static cudaError_t launch_vq16_m(const LayerArgs& a, int grid, const int8_t* signs, cudaStream_t s) {
+  switch (v16_mt(a.M)) {
+    case 1: return launch_vq16_t<T, 1>(a, grid, signs, s);
+    case 2: return launch_vq16_t<T, 2>(a, grid, nullptr, s);
+    case 4: return launch_vq16_t<T, 4>(a, grid, nullptr, s);
+    default: return launch_vq16_t<T, 8>(a, grid, nullptr, s);
+  }
+}
+
 cudaError_t launch_vq16(const LayerArgs& a, const Plan& p, const int8_t* signs, cudaStream_t s) {
-  return a.act == VQ_BF16 ? launch_vq16_t<__nv_bfloat16>(a, p.grid, signs, s)
-                          : launch_vq16_t<__half>(a, p.grid, signs, s);
+  return a.act == VQ_BF16 ? launch_vq16_m<__nv_bfloat16>(a, p.grid, signs, s)
+                          : launch_vq16_m<__half>(a, p.grid, signs, s);
 }
 
 }  // namespace vq

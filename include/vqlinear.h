@@ -85,18 +85,20 @@ enum {
 /* Element types of x / y / materialised weights. */
 enum { VQ_F16 = 0, VQ_BF16 = 1 };
 
-/* Kernel choice for vq_linear_set_path.  VQ_PATH_AUTO picks by M and layer size:
- * M == 1 -> VQ_PATH_LUT where it applies (12-bit formats, K % 128 == 0, N % 4 == 0),
- * VQ_PATH_GATHER where it applies (VQ_FMT_VQ16, K % 128 == 0, K <= 16384,
- * N % 4 == 0), else VQ_PATH_GEMV; 2 <= M <= 16 -> VQ_PATH_TC for layers of at
- * least 2^22 weights, else VQ_PATH_GEMV; M >= 17 -> VQ_PATH_TC. */
+/* Kernel choice for vq_linear_set_path.  VQ_PATH_AUTO picks by format, M and layer
+ * size: VQ_FMT_VQ16 with M <= 4 -> VQ_PATH_GATHER where it applies (K % 128 == 0,
+ * K <= 16384, M' K <= 32768 with M' = M rounded up to 1, 2, 4 or 8, N % 4 == 0);
+ * otherwise M == 1 -> VQ_PATH_LUT where it applies (12-bit formats, K % 128 == 0,
+ * N % 4 == 0), else VQ_PATH_GEMV; 2 <= M <= 16 -> VQ_PATH_TC for layers of at least
+ * 2^22 weights, else VQ_PATH_GEMV; M >= 17 -> VQ_PATH_TC. */
 enum {
   VQ_PATH_AUTO = 0,
   VQ_PATH_LUT = 1,    /* M == 1 only: per-group x.codebook tables in shared memory */
   VQ_PATH_GEMV = 2,   /* 1 <= M <= 16: decode to registers, warp MMA, split-K */
   VQ_PATH_TC = 3,     /* any M: decode into tensor memory, tcgen05 MMA (fp32 in TMEM) */
-  VQ_PATH_GATHER = 4  /* M == 1, VQ_FMT_VQ16 only: codewords gathered from L2 into
-                         fp32 dot products; can apply the input rotation itself */
+  VQ_PATH_GATHER = 4  /* 1 <= M <= 8, VQ_FMT_VQ16 only: codewords gathered from L2
+                         into fp32 dot products; at M == 1 it can apply the input
+                         rotation itself */
 };
 
 typedef struct {
@@ -211,7 +213,7 @@ vq_status vq_linear_forward_noalloc(const vq_linear_desc* desc, const void* x, c
  * approximates x . W^T.  Arguments are those of vq_linear_forward plus `signs`,
  * a device int8 array of +1/-1 [K] (16-byte aligned, like every pointer); K must
  * be a power of two, 64 <= K <= 32768.
- *   - Where VQ_PATH_GATHER runs (M == 1, VQ_FMT_VQ16, K <= 16384) this is one
+ *   - Where VQ_PATH_GATHER runs with M == 1 (VQ_FMT_VQ16, K <= 16384) this is one
  *     kernel: every CTA rotates x in fp32 in shared memory and uses it unrounded;
  *     nothing else is written.
  *   - Otherwise it enqueues vq_rht_apply into a buffer of the handle (allocated

@@ -55,6 +55,35 @@ def test_gather_matches_oracle(oracle, shape, path):
     assert np.array_equal(y1, y2), "not bit-identical run to run"
 
 
+MULTI = [
+    # (N, K, scale_group, act, M): several tokens share every gathered codeword
+    (256, 256, 256, DT_F16, 2),
+    (1000, 2048, 64, DT_BF16, 3),
+    (520, 4096, 4096, DT_F16, 8),
+    (132, 8192, 64, DT_F16, 4),
+    (2052, 1024, 64, DT_BF16, 5),
+]
+
+
+@pytest.mark.parametrize("shape", MULTI, ids=lambda s: f"{s[0]}x{s[1]}sg{s[2]}a{s[3]}M{s[4]}")
+def test_gather_several_tokens(oracle, shape):
+    N, K, sg, act, M = shape
+    layer = make_layer(LayerSpec(N, K, FMT_VQ16, sg), cfg_id=76, tensor_id=N)
+    L = layer_on_gpu(layer, act, M)
+    x = make_x(M, K, act, cfg_id=76)
+    y1 = run_forward(L, x, act, vq.VQ_PATH_GATHER)
+    y2 = run_forward(L, x, act, vq.VQ_PATH_AUTO)  # the gather kernel up to M = 4, else another path
+    vq.vq_linear_check(L.handle)
+    y_ref = oracle.forward(layer, x, act)
+    w, _ = oracle.dequant(layer)
+    tol = oracle.tolerance(x, act, w, TOL)
+    assert_y_within(y1, act, y_ref, tol, what=f"gather {shape}")
+    if M <= 4:
+        assert np.array_equal(y1, y2), "forced and automatic paths differ"
+    else:
+        assert_y_within(y2, act, y_ref, tol, what=f"auto {shape}")
+
+
 def test_gather_config3_sampled(oracle):
     spec = CONFIGS[3]["tensors"][0][1]
     layer = make_layer(spec, cfg_id=3)
@@ -80,10 +109,11 @@ def test_gather_with_sm_budget(oracle):
 
 
 @pytest.mark.parametrize("N, K, fmt, M", [(256, 16512, FMT_VQ16, 1), (258, 256, FMT_VQ16, 1),
-                                          (256, 256, FMT_VQ16, 2), (256, 256, FMT_RVQ12_4, 1)])
+                                          (256, 256, FMT_VQ16, 9), (256, 8192, FMT_VQ16, 5),
+                                          (256, 256, FMT_RVQ12_4, 1)])
 def test_gather_rejects_what_it_does_not_take(N, K, fmt, M):
     layer = make_layer(LayerSpec(N, K, fmt, 64), cfg_id=73)
-    L = layer_on_gpu(layer, DT_F16, 2)
+    L = layer_on_gpu(layer, DT_F16, M)
     L.set_path(vq.VQ_PATH_GATHER)
     x = torch.zeros((M, K), dtype=torch.float16, device="cuda")
     with pytest.raises(vq.VQError) as ei:
