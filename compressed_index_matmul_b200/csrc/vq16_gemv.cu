@@ -44,7 +44,6 @@ constexpr int kV16Consumers = 512;  // threads: one (slice, row) position each p
 constexpr int kV16Cluster = 2;      // CTAs per cluster (the K-slices are split over them)
 constexpr int kV16MaxBlk = 512;     // rows per cluster block
 constexpr int kV16MaxK = 16384;
-constexpr int kV16MaxSpc = kV16MaxK / 128 / kV16Cluster;  // slices per CTA
 
 constexpr int kV16MaxM = 8;           // tokens
 constexpr int kV16MaxMK = 32768;      // tokens x K (the fp32 x of all tokens is in shared memory)
