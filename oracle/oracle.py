@@ -59,6 +59,8 @@ def _load():
             lib.vqo_decode_array.argtypes = [P, ctypes.c_int64, I, P]
             lib.vqo_rht_f64.restype = I
             lib.vqo_rht_f64.argtypes = [I, I, P, P, P]
+            lib.vqo_rht_out_f64.restype = I
+            lib.vqo_rht_out_f64.argtypes = [I, I, P, P, P]
             lib.vqo_round_array.restype = None
             lib.vqo_round_array.argtypes = [P, ctypes.c_int64, I, P]
             lib.vqo_unpack.restype = I
@@ -196,6 +198,19 @@ def rht_f64(x, signs) -> np.ndarray:
     rc = lib.vqo_rht_f64(M, K, _p(xd), _p(sg), _p(out))
     if rc:
         raise ValueError(f"vqo_rht_f64 failed rc={rc}")
+    return out
+
+
+def rht_out_f64(y, signs) -> np.ndarray:
+    """Output-side rotation of fp64 values [M,N]: signs * (1/sqrt N) H y (transform, then signs)."""
+    lib = _load()
+    yd = _c(y, np.float64)
+    sg = _c(signs, np.int8)
+    M, N = yd.shape
+    out = np.empty((M, N), dtype=np.float64)
+    rc = lib.vqo_rht_out_f64(M, N, _p(yd), _p(sg), _p(out))
+    if rc:
+        raise ValueError(f"vqo_rht_out_f64 failed rc={rc}")
     return out
 
 

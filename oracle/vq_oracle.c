@@ -324,6 +324,25 @@ int vqo_rht_f64(int M, int K, const double* x, const int8_t* signs, double* out)
 }
 
 /* Same rotation with x given as fp16 / bf16 bits (taken exactly). */
+/* Output-side rotation (GLQ README, "Bit widths": the fused linear ends with an
+ * output RHT): the transpose of the input rotation, undoing it on the layer's
+ * output side.  out[m][k] = signs[k] / sqrt(N) * sum_j H[k][j] y[m][j], the
+ * Walsh-Hadamard transform first, then the sign flips, as an explicit O(N^2)
+ * product in fp64. */
+int vqo_rht_out_f64(int M, int N, const double* y, const int8_t* signs, double* out) {
+  if (M < 0 || N <= 0 || (N & (N - 1)) != 0) return 1;
+  const double inv_sqrt_n = 1.0 / sqrt((double)N);
+  for (int m = 0; m < M; ++m) {
+    const double* row = y + (int64_t)m * N;
+    for (int k = 0; k < N; ++k) {
+      double acc = 0.0;
+      for (int j = 0; j < N; ++j) acc += vqo_parity((uint32_t)(k & j)) ? -row[j] : row[j];
+      out[(int64_t)m * N + k] = (double)signs[k] * acc * inv_sqrt_n;
+    }
+  }
+  return 0;
+}
+
 int vqo_rht(int M, int K, const uint16_t* x, int xdt, const int8_t* signs, double* out) {
   if (M < 0 || K <= 0 || (K & (K - 1)) != 0) return 1;
   double* xd = (double*)malloc(sizeof(double) * (size_t)M * K + 1);

@@ -378,3 +378,50 @@ def test_rht_bits_entry_matches_f64(oracle):
     signs = np.where(np.arange(K) % 3 == 0, -1, 1).astype(np.int8)
     xd = (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
     assert np.array_equal(oracle.rht(x, DT_BF16, signs), oracle.rht_f64(xd, signs))
+
+
+# ----------------------------------------------------------------- output rotation
+
+@pytest.mark.parametrize("N", [1, 2, 8, 128])
+def test_rht_out_matches_sylvester_hadamard(oracle, N):
+    """signs * (1/sqrt N) H y: the library's Sylvester matrix, signs applied after it."""
+    rng = np.random.default_rng(100 + N)
+    y = rng.standard_normal((3, N))
+    signs = rng.choice([-1, 1], size=N).astype(np.int8)
+    ref = signs * (scipy.linalg.hadamard(N).astype(np.float64) @ y.T).T / np.sqrt(N)
+    assert np.allclose(oracle.rht_out_f64(y, signs), ref, rtol=1e-13, atol=1e-13)
+
+
+def test_rht_out_small_case_by_hand(oracle):
+    a, b = 5.0, 2.0
+    out = oracle.rht_out_f64(np.array([[a, b]]), np.array([1, -1], np.int8))
+    r = 1 / np.sqrt(2)
+    # H y = (a + b, a - b), then the signs (+1, -1): differs from the input rotation's (a - b, a + b)
+    assert np.allclose(out, [[(a + b) * r, -(a - b) * r]], rtol=1e-15)
+
+
+def test_rht_out_undoes_the_input_rotation(oracle):
+    """R^T R = I: rotating an input, then applying the output rotation with the same signs,
+    returns it (the two differ in where the signs go)."""
+    K = 256
+    rng = np.random.default_rng(7)
+    x = rng.standard_normal((3, K))
+    signs = rng.choice([-1, 1], size=K).astype(np.int8)
+    assert np.allclose(oracle.rht_out_f64(oracle.rht_f64(x, signs), signs), x, atol=1e-12)
+    assert not np.allclose(oracle.rht_f64(oracle.rht_f64(x, signs), signs), x, atol=1e-3)
+
+
+def test_two_sided_rotation_end_to_end(oracle):
+    """A layer stored as W_hat = R_out W R_in^T gives back y = W x through
+    y = R_out^T (W_hat (R_in x)), with R = (1/sqrt n) H diag(signs) built explicitly."""
+    N, K = 16, 32
+    rng = np.random.default_rng(11)
+    W = rng.standard_normal((N, K))
+    x = rng.standard_normal((2, K))
+    s_in = rng.choice([-1, 1], size=K).astype(np.int8)
+    s_out = rng.choice([-1, 1], size=N).astype(np.int8)
+    R_in = scipy.linalg.hadamard(K) * s_in[None, :] / np.sqrt(K)
+    R_out = scipy.linalg.hadamard(N) * s_out[None, :] / np.sqrt(N)
+    W_hat = R_out @ W @ R_in.T
+    y = oracle.rht_out_f64(oracle.rht_f64(x, s_in) @ W_hat.T, s_out)
+    assert np.allclose(y, x @ W.T, atol=1e-12)
