@@ -625,10 +625,44 @@ def detail(args, peaks, main_wl):
         res["prefill-8192 M=256"] = r
     except Exception as exc:  # the tensor-core path reports why it could not run
         res["prefill-8192 M=256"] = {"error": str(exc)[:300]}
+    for M in (1, 8):
+        res[f"rotation 4096 M={M}"] = time_rotations(4096, M, steps)
     for v in res.values():
         for k in list(v):
             if isinstance(v[k], float):
                 v[k] = round(v[k], 4)
+    return res
+
+
+def time_rotations(K, M, steps):
+    """Device time per launch of the standalone input rotation (vq_rht_apply) and the
+    output rotation (vq_rht_apply_output) on M rows of K fp16 values, as CUDA graphs."""
+    import torch
+
+    import compressed_index_matmul_b200 as vq
+
+    x = torch.from_numpy(make_x(M, K, DT_F16, cfg_id=3).view(np.int16)).cuda().view(torch.float16)
+    sg = torch.from_numpy(make_signs(K, cfg_id=3)).cuda()
+    out = torch.empty_like(x)
+    res = {"M": M, "K": K}
+    for name, fn in (("input_us", vq.vq_rht_apply), ("output_us", vq.vq_rht_apply_output)):
+        stream = torch.cuda.Stream()
+        with torch.cuda.stream(stream):
+            fn(x, out, sg, M, K, DT_F16, stream.cuda_stream)
+            stream.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for _ in range(20):
+                    fn(x, out, sg, M, K, DT_F16, stream.cuda_stream)
+            g.replay()
+            stream.synchronize()
+            t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            t0.record(stream)
+            for _ in range(max(1, steps // 20)):
+                g.replay()
+            t1.record(stream)
+        torch.cuda.synchronize()
+        res[name] = 1e3 * t0.elapsed_time(t1) / (20 * max(1, steps // 20))
     return res
 
 

@@ -394,6 +394,25 @@ VQ_API vq_status vq_rht_apply(const void* x, void* x_out, const int8_t* signs, i
   return VQ_OK;
 }
 
+VQ_API vq_status vq_rht_apply_output(const void* y, void* y_out, const int8_t* signs, int32_t M, int32_t N,
+                                     int32_t dtype, void* stream) {
+  if (N < 64 || N > 32768 || (N & (N - 1)) != 0)
+    return fail(VQ_ERR_INVALID_ARG, "N=%d must be a power of two in [64, 32768]", N);
+  if (M < 0) return fail(VQ_ERR_INVALID_ARG, "M=%d is negative", M);
+  if (dtype != VQ_F16 && dtype != VQ_BF16) return fail(VQ_ERR_INVALID_ARG, "dtype=%d", dtype);
+  vq_status st;
+  if ((st = check_ptr(y, "y")) || (st = check_ptr(y_out, "y_out"))) return st;
+  if (signs == nullptr) return fail(VQ_ERR_INVALID_ARG, "signs is NULL");
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(y), b0 = reinterpret_cast<uintptr_t>(y_out);
+  const uintptr_t bytes = (uintptr_t)M * N * 2;
+  if (a0 != b0 && a0 < b0 + bytes && b0 < a0 + bytes)
+    return fail(VQ_ERR_INVALID_ARG, "y_out partially overlaps y");
+  if (M == 0) return VQ_OK;
+  cudaError_t e = vq::launch_rht_output(y, y_out, signs, M, N, dtype, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "vq_rht_apply_output launch");
+  return VQ_OK;
+}
+
 VQ_API vq_status vq_linear_check(vq_linear_t h, void* stream) {
   if (h == nullptr) return fail(VQ_ERR_INVALID_ARG, "handle is NULL");
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));

@@ -46,30 +46,39 @@ cudaError_t launch_split_reduce(const float* partial, void* y, int splits, int M
 // writing it, so x_out may be x.
 constexpr int kRhtThreads = 512;
 
-template <typename T>
+// kOutput: the output-side rotation signs / sqrt(K) * H x (GLQ README, "Bit
+// widths": the fused linear ends with an output RHT), the transpose of the input
+// rotation: the transform first, the signs at the store.
+template <typename T, bool kOutput>
 __global__ void __launch_bounds__(kRhtThreads) rht_kernel(const uint16_t* __restrict__ x, uint16_t* __restrict__ xo,
                                                           const int8_t* __restrict__ signs, int K, float scale) {
   extern __shared__ float buf[];
   const int64_t row = blockIdx.x;
-  hadamard_to_smem<T, kRhtThreads, 32768>(x + row * K, signs, buf, K, threadIdx.x);
+  hadamard_to_smem<T, kRhtThreads, 32768, !kOutput>(x + row * K, signs, buf, K, threadIdx.x);
   uint16_t* orow = xo + row * K;
-  for (int i = threadIdx.x; i < K; i += kRhtThreads) orow[i] = Elt<T>::from_f32(buf[i] * scale);
+  for (int i = threadIdx.x; i < K; i += kRhtThreads)
+    orow[i] = Elt<T>::from_f32(kOutput ? buf[i] * scale * (float)signs[i] : buf[i] * scale);
+}
+
+template <typename T, bool kOutput>
+static cudaError_t launch_rht_t(const void* x, void* x_out, const int8_t* signs, int M, int K, cudaStream_t s) {
+  const size_t smem = (size_t)K * sizeof(float);
+  const float scale = (float)(1.0 / __builtin_sqrt((double)K));
+  cudaError_t e = cudaFuncSetAttribute(rht_kernel<T, kOutput>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  rht_kernel<T, kOutput><<<M, kRhtThreads, smem, s>>>((const uint16_t*)x, (uint16_t*)x_out, signs, K, scale);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_rht(const void* x, void* x_out, const int8_t* signs, int M, int K, int dtype, cudaStream_t s) {
-  const size_t smem = (size_t)K * sizeof(float);
-  const float scale = (float)(1.0 / __builtin_sqrt((double)K));
-  cudaError_t e;
-  if (dtype == VQ_BF16) {
-    e = cudaFuncSetAttribute(rht_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    rht_kernel<__nv_bfloat16><<<M, kRhtThreads, smem, s>>>((const uint16_t*)x, (uint16_t*)x_out, signs, K, scale);
-  } else {
-    e = cudaFuncSetAttribute(rht_kernel<__half>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    rht_kernel<__half><<<M, kRhtThreads, smem, s>>>((const uint16_t*)x, (uint16_t*)x_out, signs, K, scale);
-  }
-  return cudaGetLastError();
+  return dtype == VQ_BF16 ? launch_rht_t<__nv_bfloat16, false>(x, x_out, signs, M, K, s)
+                          : launch_rht_t<__half, false>(x, x_out, signs, M, K, s);
+}
+
+cudaError_t launch_rht_output(const void* y, void* y_out, const int8_t* signs, int M, int N, int dtype,
+                              cudaStream_t s) {
+  return dtype == VQ_BF16 ? launch_rht_t<__nv_bfloat16, true>(y, y_out, signs, M, N, s)
+                          : launch_rht_t<__half, true>(y, y_out, signs, M, N, s);
 }
 
 // ------------------------------------------------------------------ debug exports

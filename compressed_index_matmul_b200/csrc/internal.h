@@ -67,6 +67,8 @@ cudaError_t launch_tc(const LayerArgs& a, const Plan& p, float* scratch, uint32_
 cudaError_t launch_split_reduce(const float* partial, void* y, int splits, int M, int N, int act, cudaStream_t s);
 cudaError_t launch_rht(const void* x, void* x_out, const int8_t* signs, int M, int K, int dtype,
                        cudaStream_t s);
+cudaError_t launch_rht_output(const void* y, void* y_out, const int8_t* signs, int M, int N, int dtype,
+                              cudaStream_t s);
 cudaError_t launch_debug_unpack(const LayerArgs& a, uint16_t* i1, uint8_t* i2, cudaStream_t s);
 cudaError_t launch_debug_dequant(const LayerArgs& a, void* w, int wdt, cudaStream_t s);
 cudaError_t launch_debug_wait_timeout(uint32_t* err, cudaStream_t s);

@@ -11,8 +11,9 @@
 //           on registers, the next five across the warp's lanes with shuffles;
 //   pass 2: the log2(R) highest stages run on registers over groups of R
 //           elements at stride 32 E.
-// Used by the rotation kernel (vq_rht_apply) and by the batch-1 16-bit kernel,
-// which rotates x itself.
+// With kSignsFirst false the signs are not applied (the output-side rotation
+// applies them after the transform).  Used by the rotation kernels (vq_rht_apply,
+// vq_rht_apply_output) and by the batch-1 16-bit kernel, which rotates x itself.
 #pragma once
 
 #include <stdint.h>
@@ -21,7 +22,7 @@
 
 namespace vq {
 
-template <typename T, int E, int R, int NT>
+template <typename T, int E, int R, int NT, bool kSignsFirst>
 __device__ __forceinline__ void hadamard_pass(const uint16_t* __restrict__ x, const int8_t* __restrict__ signs,
                                               float* xs, int tid) {
   constexpr int K = 32 * E * R;
@@ -34,17 +35,19 @@ __device__ __forceinline__ void hadamard_pass(const uint16_t* __restrict__ x, co
 #pragma unroll
       for (int c = 0; c < E / 8; ++c) {
         const uint4 xw = *reinterpret_cast<const uint4*>(x + tid * E + 8 * c);
-        const uint2 sw = *reinterpret_cast<const uint2*>(signs + tid * E + 8 * c);
+        const uint2 sw = kSignsFirst ? *reinterpret_cast<const uint2*>(signs + tid * E + 8 * c) : make_uint2(0, 0);
         const uint32_t xa[4] = {xw.x, xw.y, xw.z, xw.w};
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
           const int8_t sg = (int8_t)(((q < 4 ? sw.x : sw.y) >> (8 * (q & 3))) & 0xFFu);
-          v[8 * c + q] = Elt<T>::to_f32((uint16_t)(xa[q >> 1] >> (16 * (q & 1)))) * (float)sg;
+          const float xv = Elt<T>::to_f32((uint16_t)(xa[q >> 1] >> (16 * (q & 1))));
+          v[8 * c + q] = kSignsFirst ? xv * (float)sg : xv;
         }
       }
     } else {
 #pragma unroll
-      for (int e = 0; e < E; ++e) v[e] = Elt<T>::to_f32(x[tid * E + e]) * (float)signs[tid * E + e];
+      for (int e = 0; e < E; ++e)
+        v[e] = kSignsFirst ? Elt<T>::to_f32(x[tid * E + e]) * (float)signs[tid * E + e] : Elt<T>::to_f32(x[tid * E + e]);
     }
 #pragma unroll
     for (int h = 1; h < E; h <<= 1)  // stages h = 1 .. E/2 on registers
@@ -87,26 +90,26 @@ __device__ __forceinline__ void hadamard_pass(const uint16_t* __restrict__ x, co
 
 // hadamard_pass for a power-of-two K in [64, kMaxK] (NT = 512; kMaxK <= 32768 bounds
 // the registers the instantiations need).
-template <typename T, int NT, int kMaxK>
+template <typename T, int NT, int kMaxK, bool kSignsFirst = true>
 __device__ __forceinline__ void hadamard_to_smem(const uint16_t* x, const int8_t* signs, float* xs, int K, int tid) {
   static_assert(NT == 512 && kMaxK >= 16384 && kMaxK <= 32768, "the stage split below assumes 512 threads");
   switch (K) {
-    case 64: hadamard_pass<T, 1, 2, NT>(x, signs, xs, tid); break;
-    case 128: hadamard_pass<T, 1, 4, NT>(x, signs, xs, tid); break;
-    case 256: hadamard_pass<T, 1, 8, NT>(x, signs, xs, tid); break;
-    case 512: hadamard_pass<T, 1, 16, NT>(x, signs, xs, tid); break;
-    case 1024: hadamard_pass<T, 2, 16, NT>(x, signs, xs, tid); break;
-    case 2048: hadamard_pass<T, 4, 16, NT>(x, signs, xs, tid); break;
-    case 4096: hadamard_pass<T, 8, 16, NT>(x, signs, xs, tid); break;
-    case 8192: hadamard_pass<T, 16, 16, NT>(x, signs, xs, tid); break;
+    case 64: hadamard_pass<T, 1, 2, NT, kSignsFirst>(x, signs, xs, tid); break;
+    case 128: hadamard_pass<T, 1, 4, NT, kSignsFirst>(x, signs, xs, tid); break;
+    case 256: hadamard_pass<T, 1, 8, NT, kSignsFirst>(x, signs, xs, tid); break;
+    case 512: hadamard_pass<T, 1, 16, NT, kSignsFirst>(x, signs, xs, tid); break;
+    case 1024: hadamard_pass<T, 2, 16, NT, kSignsFirst>(x, signs, xs, tid); break;
+    case 2048: hadamard_pass<T, 4, 16, NT, kSignsFirst>(x, signs, xs, tid); break;
+    case 4096: hadamard_pass<T, 8, 16, NT, kSignsFirst>(x, signs, xs, tid); break;
+    case 8192: hadamard_pass<T, 16, 16, NT, kSignsFirst>(x, signs, xs, tid); break;
     default:
       if constexpr (kMaxK >= 32768) {
         if (K == 32768) {
-          hadamard_pass<T, 64, 16, NT>(x, signs, xs, tid);
+          hadamard_pass<T, 64, 16, NT, kSignsFirst>(x, signs, xs, tid);
           break;
         }
       }
-      hadamard_pass<T, 32, 16, NT>(x, signs, xs, tid);  // 16384
+      hadamard_pass<T, 32, 16, NT, kSignsFirst>(x, signs, xs, tid);  // 16384
       break;
   }
 }

@@ -242,6 +242,19 @@ int32_t vq_linear_launches(vq_linear_t h, int32_t M);
 vq_status vq_rht_apply(const void* x, void* x_out, const int8_t* signs, int32_t M, int32_t K,
                        int32_t dtype, void* stream);
 
+/* Output-side rotation (GLQ README, "Bit widths": the fused linear ends with an
+ * output RHT), the transpose of vq_rht_apply's rotation: for every row m,
+ *   y_out[m][k] = signs[k] * (1/sqrt N) * sum_j (-1)^popcount(k & j) * y[m][j],
+ * i.e. the Walsh-Hadamard transform in natural (Sylvester) order first, then the
+ * sign flips.  A layer stored as W_hat = R_out W R_in^T gives y = x . W^T as
+ *   vq_rht_apply_output(vq_linear_forward_rotated(x, signs_in), signs_out).
+ * Computed in fp32, rounded to nearest even into y_out.  N must be a power of
+ * two, 64 <= N <= 32768; dtype is VQ_F16 or VQ_BF16 for both; signs is a device
+ * int8 array of +1/-1 [N]; y_out may be y (in place), partial overlap is invalid.
+ * One kernel launch on `stream`. */
+vq_status vq_rht_apply_output(const void* y, void* y_out, const int8_t* signs, int32_t M, int32_t N,
+                              int32_t dtype, void* stream);
+
 /* Synchronise `stream` and report (then clear) any error flag a bounded
  * device-side wait of this handle's kernels raised: VQ_ERR_TIMEOUT if one gave
  * up, else VQ_OK.  Synchronous. */

@@ -13,7 +13,7 @@ import torch
 
 import compressed_index_matmul_b200 as vq
 from synth import CONFIGS, DT_BF16, DT_F16, FMT_RVQ12_4, FMT_VQ16, LayerSpec, make_layer, make_signs, make_x
-from tests.gpu_util import assert_y_within, dev, host_bits, layer_on_gpu, require_gpu, run_forward
+from tests.gpu_util import assert_y_within, dev, host_bits, layer_on_gpu, require_gpu, run_forward, widen
 
 pytestmark = pytest.mark.gpu
 
@@ -190,3 +190,51 @@ def test_rotated_argument_errors():
     with pytest.raises(vq.VQError) as ei:  # K not a power of two
         L2.forward_rotated(torch.zeros((1, 384), dtype=torch.float16, device="cuda"), dev(make_signs(384, cfg_id=75)))
     assert ei.value.status == vq._binding.VQ_ERR_INVALID_ARG
+
+
+# ------------------------------------------------------------------- output rotation
+
+@pytest.mark.parametrize("N", [64, 1024, 4096, 32768])
+@pytest.mark.parametrize("dt", [DT_F16, DT_BF16])
+def test_rht_output_matches_oracle(oracle, N, dt):
+    """signs * (1/sqrt N) H y against the oracle's explicit product: within one output ulp
+    (double rounding) plus the fp32 transform error, and the same bits in place."""
+    M = 3
+    y = make_x(M, N, dt, cfg_id=77)
+    signs = make_signs(N, cfg_id=77)
+    yt, st = dev(y), dev(signs)
+    out = torch.empty_like(yt)
+    vq.vq_rht_apply_output(yt, out, st, M, N, dt)
+    torch.cuda.synchronize()
+    got = widen(host_bits(out), dt)
+    ref = oracle.rht_out_f64(widen(y, dt), signs)
+    ulp = np.spacing(np.abs(ref).astype(np.float16)).astype(np.float64) if dt == DT_F16 else np.abs(ref) * 2.0 ** -7
+    atol = 2 * np.log2(N) * 2.0 ** -24 * np.linalg.norm(widen(y, dt), axis=1, keepdims=True)
+    err = np.abs(got - ref)
+    assert np.all(err <= ulp + atol), f"max err/(ulp+atol) = {np.max(err / (ulp + atol))}"
+    vq.vq_rht_apply_output(yt, yt, st, M, N, dt)
+    torch.cuda.synchronize()
+    assert np.array_equal(host_bits(yt), host_bits(out))
+
+
+def test_two_sided_rotation(oracle):
+    """A layer stored as W_hat = R_out W R_in^T: forward_rotated with the input signs, then
+    the output rotation, against the oracle's rotations around the exact W_hat product.
+    The output rotation is orthogonal, so the per-row error norm is bounded by sqrt(N)
+    times the per-element bound of the unrotated product, plus the final rounding."""
+    N, K = 1024, 2048
+    layer = make_layer(LayerSpec(N, K, FMT_VQ16, 64), cfg_id=78)
+    L = layer_on_gpu(layer, DT_F16, 1)
+    x = make_x(1, K, DT_F16, cfg_id=78)
+    s_in, s_out = make_signs(K, cfg_id=78), make_signs(N, cfg_id=79)
+    yh = L.forward_rotated(dev(x).view(torch.float16), dev(s_in))
+    y = torch.empty_like(yh)
+    vq.vq_rht_apply_output(yh, y, dev(s_out), 1, N, DT_F16)
+    torch.cuda.synchronize()
+    got = widen(host_bits(y), DT_F16)
+    w, _ = oracle.dequant(layer)
+    xr = oracle.rht(x, DT_F16, s_in)
+    ref = oracle.rht_out_f64(xr @ w.T, s_out)
+    tau = TOL * np.linalg.norm(xr) * np.abs(w).max()
+    bound = np.sqrt(N) * tau + np.linalg.norm(0.5 * np.spacing(np.abs(ref).astype(np.float16)).astype(np.float64))
+    assert np.linalg.norm(got - ref) <= bound, f"{np.linalg.norm(got - ref)} > {bound}"
