@@ -176,7 +176,8 @@ def forward(layer, x_bits, xdt: int, rows=None) -> np.ndarray:
 
 
 def rht(x_bits, xdt: int, signs) -> np.ndarray:
-    """Rotated activations (1/sqrt K) H (signs * x) in fp64, x given as bits [M,K]."""
+    """Rotated activations (1/sqrt K) H (signs * x) in fp64, x given as bits [M,K]
+    (block-diagonal over the binary expansion of K when K is not a power of two)."""
     lib = _load()
     x = _c(x_bits, np.uint16)
     sg = _c(signs, np.int8)
@@ -189,7 +190,11 @@ def rht(x_bits, xdt: int, signs) -> np.ndarray:
 
 
 def rht_f64(x, signs) -> np.ndarray:
-    """Rotation of fp64 activations [M,K]: (1/sqrt K) H (signs * x)."""
+    """Rotation of fp64 activations [M,K]: (1/sqrt K) H (signs * x).
+
+    GLQ README, "Bit widths": a K that is not a power of two is cut into the powers of
+    two of its binary expansion, largest first along K (2688 = 2048 + 512 + 128), and
+    each block b is rotated by its own (1/sqrt b) H_b."""
     lib = _load()
     xd = _c(x, np.float64)
     sg = _c(signs, np.int8)
@@ -202,7 +207,8 @@ def rht_f64(x, signs) -> np.ndarray:
 
 
 def rht_out_f64(y, signs) -> np.ndarray:
-    """Output-side rotation of fp64 values [M,N]: signs * (1/sqrt N) H y (transform, then signs)."""
+    """Output-side rotation of fp64 values [M,N]: signs * (1/sqrt N) H y (transform, then
+    signs); block-diagonal like rht_f64 when N is not a power of two."""
     lib = _load()
     yd = _c(y, np.float64)
     sg = _c(signs, np.int8)

@@ -299,6 +299,12 @@ int vqo_forward(int fmt, int M, int N, int K, const uint16_t* x, int xdt, const 
  * random sign flips followed by a Walsh-Hadamard transform).  Written as the
  * explicit O(K^2) matrix-vector product with the Sylvester matrix, not as a
  * butterfly: out[m][k] = (1/sqrt K) sum_j (-1)^popcount(k & j) sigma_j x[m][j].
+ *
+ * K that is not a power of two (GLQ README, "Bit widths": block-diagonal FHT, 2688
+ * decomposed as 2048 + 512 + 128): K is cut into the powers of two of its binary
+ * expansion, the largest block first along K, and each block b at offset o gets its
+ * own orthonormal transform: out[o + k] = (1/sqrt b) sum_{j<b} H_b[k][j] sigma[o+j]
+ * x[o+j].  For a power of two this is the single block above.
  * ------------------------------------------------------------------------- */
 static int vqo_parity(uint32_t v) {
   int p = 0;
@@ -306,45 +312,61 @@ static int vqo_parity(uint32_t v) {
   return p;
 }
 
+/* The block of the block-diagonal decomposition that holds index k of a K-vector:
+ * its offset and size (binary expansion of K, largest power of two first). */
+static void vqo_block_of(int K, int k, int* off, int* size) {
+  int o = 0;
+  for (int bit = 30; bit >= 0; --bit) {
+    const int b = 1 << bit;
+    if (!(K & b)) continue;
+    if (k < o + b) { *off = o; *size = b; return; }
+    o += b;
+  }
+  *off = 0; *size = 0; /* not reached for 0 <= k < K */
+}
+
 int vqo_rht_f64(int M, int K, const double* x, const int8_t* signs, double* out) {
-  if (M < 0 || K <= 0 || (K & (K - 1)) != 0) return 1;
+  if (M < 0 || K <= 0) return 1;
   double* row = (double*)malloc(sizeof(double) * (size_t)K);
   if (!row) return 3;
-  const double inv_sqrt_k = 1.0 / sqrt((double)K);
   for (int m = 0; m < M; ++m) {
     for (int j = 0; j < K; ++j) row[j] = (double)signs[j] * x[(int64_t)m * K + j];
     for (int k = 0; k < K; ++k) {
+      int o, b;
+      vqo_block_of(K, k, &o, &b);
       double acc = 0.0;
-      for (int j = 0; j < K; ++j) acc += vqo_parity((uint32_t)(k & j)) ? -row[j] : row[j];
-      out[(int64_t)m * K + k] = acc * inv_sqrt_k;
+      for (int j = 0; j < b; ++j) acc += vqo_parity((uint32_t)((k - o) & j)) ? -row[o + j] : row[o + j];
+      out[(int64_t)m * K + k] = acc * (1.0 / sqrt((double)b));
     }
   }
   free(row);
   return 0;
 }
 
-/* Same rotation with x given as fp16 / bf16 bits (taken exactly). */
 /* Output-side rotation (GLQ README, "Bit widths": the fused linear ends with an
  * output RHT): the transpose of the input rotation, undoing it on the layer's
- * output side.  out[m][k] = signs[k] / sqrt(N) * sum_j H[k][j] y[m][j], the
- * Walsh-Hadamard transform first, then the sign flips, as an explicit O(N^2)
- * product in fp64. */
+ * output side.  out[m][k] = signs[k] / sqrt(b) * sum_j H_b[k-o][j] y[m][o+j] over
+ * the block (o, b) that holds k (one block of size N for a power of two): the
+ * Walsh-Hadamard transform first, then the sign flips, as an explicit product in
+ * fp64. */
 int vqo_rht_out_f64(int M, int N, const double* y, const int8_t* signs, double* out) {
-  if (M < 0 || N <= 0 || (N & (N - 1)) != 0) return 1;
-  const double inv_sqrt_n = 1.0 / sqrt((double)N);
+  if (M < 0 || N <= 0) return 1;
   for (int m = 0; m < M; ++m) {
     const double* row = y + (int64_t)m * N;
     for (int k = 0; k < N; ++k) {
+      int o, b;
+      vqo_block_of(N, k, &o, &b);
       double acc = 0.0;
-      for (int j = 0; j < N; ++j) acc += vqo_parity((uint32_t)(k & j)) ? -row[j] : row[j];
-      out[(int64_t)m * N + k] = (double)signs[k] * acc * inv_sqrt_n;
+      for (int j = 0; j < b; ++j) acc += vqo_parity((uint32_t)((k - o) & j)) ? -row[o + j] : row[o + j];
+      out[(int64_t)m * N + k] = (double)signs[k] * acc * (1.0 / sqrt((double)b));
     }
   }
   return 0;
 }
 
+/* Same rotation with x given as fp16 / bf16 bits (taken exactly). */
 int vqo_rht(int M, int K, const uint16_t* x, int xdt, const int8_t* signs, double* out) {
-  if (M < 0 || K <= 0 || (K & (K - 1)) != 0) return 1;
+  if (M < 0 || K <= 0) return 1;
   double* xd = (double*)malloc(sizeof(double) * (size_t)M * K + 1);
   if (!xd) return 3;
   vqo_decode_array(x, (int64_t)M * K, xdt, xd);

@@ -380,6 +380,58 @@ def test_rht_bits_entry_matches_f64(oracle):
     assert np.array_equal(oracle.rht(x, DT_BF16, signs), oracle.rht_f64(xd, signs))
 
 
+# ------------------------------------------------- block-diagonal rotation (K not 2^p)
+
+def _block_diag_hadamard(K):
+    """GLQ README, "Bit widths": 2688 is cut as 2048 + 512 + 128.  The dense orthonormal
+    matrix built from scipy's Sylvester blocks in that order (binary expansion of K,
+    largest block first)."""
+    sizes = [1 << b for b in range(30, -1, -1) if K & (1 << b)]
+    return scipy.linalg.block_diag(*[scipy.linalg.hadamard(b).astype(np.float64) / np.sqrt(b) for b in sizes]), sizes
+
+
+def test_block_sizes_of_the_pages_example():
+    assert _block_diag_hadamard(2688)[1] == [2048, 512, 128]
+
+
+@pytest.mark.parametrize("K", [3, 192, 320, 2688])
+def test_rht_block_diagonal_matches_dense_blocks(oracle, K):
+    rng = np.random.default_rng(200 + K)
+    x = rng.standard_normal((2, K))
+    signs = rng.choice([-1, 1], size=K).astype(np.int8)
+    H, _ = _block_diag_hadamard(K)
+    assert np.allclose(oracle.rht_f64(x, signs), (H @ (signs * x).T).T, rtol=1e-12, atol=1e-12)
+    assert np.allclose(oracle.rht_out_f64(x, signs), signs * (H @ x.T).T, rtol=1e-12, atol=1e-12)
+
+
+def test_rht_block_diagonal_by_hand(oracle):
+    """K = 3 = 2 + 1: a 2-point butterfly on the first two entries, the last one only
+    sign-flipped."""
+    a, b, c = 5.0, 2.0, 7.0
+    out = oracle.rht_f64(np.array([[a, b, c]]), np.array([1, -1, -1], np.int8))
+    r = 1 / np.sqrt(2)
+    assert np.allclose(out, [[(a - b) * r, (a + b) * r, -c]], rtol=1e-15)
+
+
+def test_rht_block_diagonal_invariants(oracle):
+    """Blocks do not mix (a one-hot input in block j stays in block j), norms are kept,
+    and the output rotation undoes the input one."""
+    K = 2688
+    rng = np.random.default_rng(9)
+    x = rng.standard_normal((2, K))
+    signs = rng.choice([-1, 1], size=K).astype(np.int8)
+    y = oracle.rht_f64(x, signs)
+    assert np.allclose(np.linalg.norm(y, axis=1), np.linalg.norm(x, axis=1), rtol=1e-12)
+    assert np.allclose(oracle.rht_out_f64(y, signs), x, atol=1e-12)
+    ones = np.ones(K, np.int8)
+    for off, b in ((0, 2048), (2048, 512), (2560, 128)):
+        e = np.zeros((1, K))
+        e[0, off + 5] = 1.0
+        out = oracle.rht_f64(e, ones)[0]
+        assert np.allclose(np.abs(out[off:off + b]), 1 / np.sqrt(b), rtol=1e-14)
+        assert np.count_nonzero(out) == b
+
+
 # ----------------------------------------------------------------- output rotation
 
 @pytest.mark.parametrize("N", [1, 2, 8, 128])
