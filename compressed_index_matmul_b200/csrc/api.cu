@@ -340,8 +340,8 @@ VQ_API vq_status vq_linear_forward_rotated(vq_linear_t h, const void* x, const i
   const vq_linear_desc& d = h->d;
   if (N != d.N || K != d.K)
     return fail(VQ_ERR_INVALID_ARG, "N=%d, K=%d do not match the handle's N=%d, K=%d", N, K, d.N, d.K);
-  if (K < 64 || K > 32768 || (K & (K - 1)) != 0)
-    return fail(VQ_ERR_INVALID_ARG, "K=%d: the rotation needs a power of two in [64, 32768]", K);
+  if (K < 64 || K > 32768 || K % 64 != 0)
+    return fail(VQ_ERR_INVALID_ARG, "K=%d: the rotation needs a multiple of 64 in [64, 32768]", K);
   if (M < 0 || M > d.max_M) return fail(VQ_ERR_INVALID_ARG, "M=%d outside [0, max_M=%d]", M, d.max_M);
   vq_status st;
   if ((st = check_ptr(signs, "signs")) || (st = check_ptr(x, "x")) || (st = check_ptr(y, "y")) || (st = validate_planes(d, planes)) ||
@@ -377,13 +377,12 @@ VQ_API vq_status vq_linear_forward_rotated(vq_linear_t h, const void* x, const i
 
 VQ_API vq_status vq_rht_apply(const void* x, void* x_out, const int8_t* signs, int32_t M, int32_t K, int32_t dtype,
                               void* stream) {
-  if (K < 64 || K > 32768 || (K & (K - 1)) != 0)
-    return fail(VQ_ERR_INVALID_ARG, "K=%d must be a power of two in [64, 32768]", K);
+  if (K < 64 || K > 32768 || K % 64 != 0)
+    return fail(VQ_ERR_INVALID_ARG, "K=%d must be a multiple of 64 in [64, 32768]", K);
   if (M < 0) return fail(VQ_ERR_INVALID_ARG, "M=%d is negative", M);
   if (dtype != VQ_F16 && dtype != VQ_BF16) return fail(VQ_ERR_INVALID_ARG, "dtype=%d", dtype);
   vq_status st;
-  if ((st = check_ptr(x, "x")) || (st = check_ptr(x_out, "x_out"))) return st;
-  if (signs == nullptr) return fail(VQ_ERR_INVALID_ARG, "signs is NULL");
+  if ((st = check_ptr(x, "x")) || (st = check_ptr(x_out, "x_out")) || (st = check_ptr(signs, "signs"))) return st;
   const uintptr_t a0 = reinterpret_cast<uintptr_t>(x), b0 = reinterpret_cast<uintptr_t>(x_out);
   const uintptr_t bytes = (uintptr_t)M * K * 2;
   if (a0 != b0 && a0 < b0 + bytes && b0 < a0 + bytes)
@@ -396,13 +395,12 @@ VQ_API vq_status vq_rht_apply(const void* x, void* x_out, const int8_t* signs, i
 
 VQ_API vq_status vq_rht_apply_output(const void* y, void* y_out, const int8_t* signs, int32_t M, int32_t N,
                                      int32_t dtype, void* stream) {
-  if (N < 64 || N > 32768 || (N & (N - 1)) != 0)
-    return fail(VQ_ERR_INVALID_ARG, "N=%d must be a power of two in [64, 32768]", N);
+  if (N < 64 || N > 32768 || N % 64 != 0)
+    return fail(VQ_ERR_INVALID_ARG, "N=%d must be a multiple of 64 in [64, 32768]", N);
   if (M < 0) return fail(VQ_ERR_INVALID_ARG, "M=%d is negative", M);
   if (dtype != VQ_F16 && dtype != VQ_BF16) return fail(VQ_ERR_INVALID_ARG, "dtype=%d", dtype);
   vq_status st;
-  if ((st = check_ptr(y, "y")) || (st = check_ptr(y_out, "y_out"))) return st;
-  if (signs == nullptr) return fail(VQ_ERR_INVALID_ARG, "signs is NULL");
+  if ((st = check_ptr(y, "y")) || (st = check_ptr(y_out, "y_out")) || (st = check_ptr(signs, "signs"))) return st;
   const uintptr_t a0 = reinterpret_cast<uintptr_t>(y), b0 = reinterpret_cast<uintptr_t>(y_out);
   const uintptr_t bytes = (uintptr_t)M * N * 2;
   if (a0 != b0 && a0 < b0 + bytes && b0 < a0 + bytes)

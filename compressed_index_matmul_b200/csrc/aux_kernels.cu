@@ -38,35 +38,43 @@ cudaError_t launch_split_reduce(const float* partial, void* y, int splits, int M
 // ---------------------------------------------------------------------- rotation
 //
 // GLQ README, "How it works": Randomized Hadamard Transform = random sign flips
-// followed by a fast Walsh-Hadamard transform.  One CTA of 512 threads per token
-// row: hadamard_to_smem (rotate.cuh) computes H_K (signs . x) in fp32 in shared
-// memory (butterflies on registers and lane shuffles, one shared-memory pass for
-// the highest stages, natural Sylvester order); the row is then scaled by
-// 1/sqrt(K) and rounded to the element type.  Each CTA reads its whole row before
-// writing it, so x_out may be x.
+// followed by a fast Walsh-Hadamard transform; "Bit widths": a K that is not a
+// power of two is cut into power-of-two blocks (binary expansion, largest first),
+// each rotated on its own.  One CTA of 512 threads per token row: for each block b,
+// hadamard_to_smem (rotate.cuh) computes H_b (signs . x) in fp32 in shared memory
+// (butterflies on registers and lane shuffles, one shared-memory pass for the
+// highest stages, natural Sylvester order); the block is then scaled by 1/sqrt(b)
+// and rounded to the element type.  Every block is read before it is written and
+// blocks are disjoint, so x_out may be x.
 constexpr int kRhtThreads = 512;
 
-// kOutput: the output-side rotation signs / sqrt(K) * H x (GLQ README, "Bit
+// kOutput: the output-side rotation signs / sqrt(b) * H_b x (GLQ README, "Bit
 // widths": the fused linear ends with an output RHT), the transpose of the input
 // rotation: the transform first, the signs at the store.
 template <typename T, bool kOutput>
 __global__ void __launch_bounds__(kRhtThreads) rht_kernel(const uint16_t* __restrict__ x, uint16_t* __restrict__ xo,
-                                                          const int8_t* __restrict__ signs, int K, float scale) {
+                                                          const int8_t* __restrict__ signs, int K) {
   extern __shared__ float buf[];
   const int64_t row = blockIdx.x;
-  hadamard_to_smem<T, kRhtThreads, 32768, !kOutput>(x + row * K, signs, buf, K, threadIdx.x);
+  const uint16_t* xrow = x + row * K;
   uint16_t* orow = xo + row * K;
-  for (int i = threadIdx.x; i < K; i += kRhtThreads)
-    orow[i] = Elt<T>::from_f32(kOutput ? buf[i] * scale * (float)signs[i] : buf[i] * scale);
+  for (int o = 0, rest = K; rest > 0;) {
+    const int b = 1 << (31 - __clz(rest));  // the largest power of two left
+    hadamard_to_smem<T, kRhtThreads, 32768, !kOutput>(xrow + o, signs + o, buf + o, b, threadIdx.x);
+    const float scale = block_scale(b);
+    for (int i = threadIdx.x; i < b; i += kRhtThreads)
+      orow[o + i] = Elt<T>::from_f32(kOutput ? buf[o + i] * scale * (float)signs[o + i] : buf[o + i] * scale);
+    o += b;
+    rest -= b;
+  }
 }
 
 template <typename T, bool kOutput>
 static cudaError_t launch_rht_t(const void* x, void* x_out, const int8_t* signs, int M, int K, cudaStream_t s) {
   const size_t smem = (size_t)K * sizeof(float);
-  const float scale = (float)(1.0 / __builtin_sqrt((double)K));
   cudaError_t e = cudaFuncSetAttribute(rht_kernel<T, kOutput>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  rht_kernel<T, kOutput><<<M, kRhtThreads, smem, s>>>((const uint16_t*)x, (uint16_t*)x_out, signs, K, scale);
+  rht_kernel<T, kOutput><<<M, kRhtThreads, smem, s>>>((const uint16_t*)x, (uint16_t*)x_out, signs, K);
   return cudaGetLastError();
 }
 

@@ -114,4 +114,29 @@ __device__ __forceinline__ void hadamard_to_smem(const uint16_t* x, const int8_t
   }
 }
 
+// The rotation for any K that is a multiple of 64 up to kMaxK (GLQ README, "Bit
+// widths": a hidden size that is not a power of two is cut into power-of-two blocks,
+// 2688 = 2048 + 512 + 128, each with its own transform).  The blocks are the binary
+// expansion of K, largest first along K: each is hadamard_to_smem of its slice of x
+// and signs into its slice of xs.  With scale_blocks each block is multiplied in
+// place by its orthonormal factor 1/sqrt(b) (where K is not a power of two no single
+// factor applies to the whole vector); otherwise the caller applies 1/sqrt(K).
+__device__ __forceinline__ float block_scale(int b) { return (float)(1.0 / sqrt((double)b)); }
+
+template <typename T, int NT, int kMaxK, bool kSignsFirst = true>
+__device__ __forceinline__ void hadamard_blocks_to_smem(const uint16_t* x, const int8_t* signs, float* xs, int K,
+                                                        int tid, bool scale_blocks) {
+  for (int o = 0, rest = K; rest > 0;) {
+    const int b = 1 << (31 - __clz(rest));  // the largest power of two left
+    hadamard_to_smem<T, NT, kMaxK, kSignsFirst>(x + o, signs + o, xs + o, b, tid);
+    if (scale_blocks) {
+      const float sc = block_scale(b);
+      for (int i = tid; i < b; i += NT) xs[o + i] *= sc;
+    }
+    o += b;
+    rest -= b;
+  }
+  if (scale_blocks) asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory");
+}
+
 }  // namespace vq

@@ -14,8 +14,10 @@
 // Rotated input (GLQ README, "How it works": random sign flips followed by a fast
 // Walsh-Hadamard transform): when `signs` is given (M == 1), every CTA computes the
 // whole rotated vector x' = H (signs . x) in fp32 in shared memory
-// (hadamard_to_smem, rotate.cuh); the orthonormal factor 1/sqrt(K) multiplies
-// every partial sum.  The caller's x is the unrotated input, and no rotated copy of it
+// (hadamard_blocks_to_smem, rotate.cuh); for a power-of-two K the orthonormal factor
+// 1/sqrt(K) multiplies every partial sum, otherwise ("Bit widths": block-diagonal
+// transform over the binary expansion of K) each block of x' is scaled by its own
+// 1/sqrt(b) in shared memory.  The caller's x is the unrotated input, and no rotated copy of it
 // is ever written to memory.
 //
 // Work split and reduction: no table is built, so the (K-slice, row) grid is cut
@@ -129,7 +131,8 @@ __global__ void __launch_bounds__(kV16Consumers, 1)
 
   asm volatile("griddepcontrol.wait;" ::: "memory");
   if (MT == 1 && signs) {
-    hadamard_to_smem<T, kV16Consumers, kV16MaxK>(static_cast<const uint16_t*>(a.x), signs, xs, K, tid);
+    hadamard_blocks_to_smem<T, kV16Consumers, kV16MaxK>(static_cast<const uint16_t*>(a.x), signs, xs, K, tid,
+                                                        (K & (K - 1)) != 0);
   } else {
     const uint16_t* xg = static_cast<const uint16_t*>(a.x);
     for (int i = tid; i < MT * K; i += kV16Consumers) xs[i] = i < M * K ? Elt<T>::to_f32(xg[i]) : 0.f;
@@ -315,7 +318,10 @@ static cudaError_t launch_vq16_t(const LayerArgs& a, int grid, const int8_t* sig
   const V16Geom g = v16_geom(a.N, ncl, S, MT);
   const int smem = v16_smem(S, MT, g.rblk, a.K).bytes;
   // Orthonormal factor of the rotation, rounded once from double precision.
-  const float xscale = signs ? (float)(1.0 / std::sqrt((double)a.K)) : 1.f;
+  // a power-of-two K takes its orthonormal factor at the store; otherwise each block
+  // was scaled in shared memory
+  const bool pow2 = (a.K & (a.K - 1)) == 0;
+  const float xscale = signs && pow2 ? (float)(1.0 / std::sqrt((double)a.K)) : 1.f;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(g.ncl * kV16Cluster);
   cfg.blockDim = dim3(kV16Consumers);

@@ -212,7 +212,8 @@ vq_status vq_linear_forward_noalloc(const vq_linear_desc* desc, const void* x, c
  * fused kernels).  x is the unrotated input; the planes encode W . R^T, so y
  * approximates x . W^T.  Arguments are those of vq_linear_forward plus `signs`,
  * a device int8 array of +1/-1 [K] (16-byte aligned, like every pointer); K must
- * be a power of two, 64 <= K <= 32768.
+ * be a multiple of 64, 64 <= K <= 32768 (block-diagonal when not a power of two,
+ * as in vq_rht_apply).
  *   - Where VQ_PATH_GATHER runs with M == 1 (VQ_FMT_VQ16, K <= 16384) this is one
  *     kernel: every CTA rotates x in fp32 in shared memory and uses it unrounded;
  *     nothing else is written.
@@ -234,9 +235,14 @@ int32_t vq_linear_launches(vq_linear_t h, int32_t M);
  * Randomized Hadamard Transform): for every row m,
  *   x_out[m][k] = (1/sqrt K) * sum_j (-1)^popcount(k & j) * signs[j] * x[m][j],
  * i.e. sign flips first, then the Walsh-Hadamard transform in natural (Sylvester)
- * order, orthonormal scaling.  Computed in fp32 and rounded to nearest even into
- * x_out.  K must be a power of two, 16 <= K <= 32768; dtype is VQ_F16 or
- * VQ_BF16 for both x and x_out; signs is a device int8 array of +1/-1 [K].
+ * order, orthonormal scaling.  A K that is not a power of two (GLQ README, "Bit
+ * widths": block-diagonal FHT, 2688 = 2048 + 512 + 128) is cut into the powers of
+ * two of its binary expansion, the largest first along K, and the formula applies
+ * to each block (offset o, size b) on its own:
+ *   x_out[m][o+k] = (1/sqrt b) * sum_{j<b} (-1)^popcount(k & j) * signs[o+j] * x[m][o+j].
+ * Computed in fp32 and rounded to nearest even into x_out.  K must be a multiple
+ * of 64, 64 <= K <= 32768; dtype is VQ_F16 or VQ_BF16 for both x and x_out;
+ * signs is a device int8 array of +1/-1 [K], 16-byte aligned.
  * x_out may be the same buffer as x (in place); partial overlap is invalid.
  * One kernel launch on `stream`. */
 vq_status vq_rht_apply(const void* x, void* x_out, const int8_t* signs, int32_t M, int32_t K,
@@ -248,9 +254,11 @@ vq_status vq_rht_apply(const void* x, void* x_out, const int8_t* signs, int32_t 
  * i.e. the Walsh-Hadamard transform in natural (Sylvester) order first, then the
  * sign flips.  A layer stored as W_hat = R_out W R_in^T gives y = x . W^T as
  *   vq_rht_apply_output(vq_linear_forward_rotated(x, signs_in), signs_out).
- * Computed in fp32, rounded to nearest even into y_out.  N must be a power of
- * two, 64 <= N <= 32768; dtype is VQ_F16 or VQ_BF16 for both; signs is a device
- * int8 array of +1/-1 [N]; y_out may be y (in place), partial overlap is invalid.
+ * An N that is not a power of two is cut into blocks as in vq_rht_apply, each
+ * transformed with its own 1/sqrt(b).  Computed in fp32, rounded to nearest even
+ * into y_out.  N must be a multiple of 64, 64 <= N <= 32768; dtype is VQ_F16 or
+ * VQ_BF16 for both; signs is a device int8 array of +1/-1 [N], 16-byte aligned;
+ * y_out may be y (in place), partial overlap is invalid.
  * One kernel launch on `stream`. */
 vq_status vq_rht_apply_output(const void* y, void* y_out, const int8_t* signs, int32_t M, int32_t N,
                               int32_t dtype, void* stream);

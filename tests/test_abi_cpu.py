@@ -81,7 +81,8 @@ def test_null_arguments_are_rejected(lib):
 
 
 @pytest.mark.parametrize("M,K,dt,x,xo,signs", [
-    (1, 100, 0, 16, 16, 16),      # K not a power of two
+    (1, 100, 0, 16, 16, 16),      # K not a multiple of 64
+    (1, 96, 0, 16, 16, 16),       # K not a multiple of 64
     (1, 32, 0, 16, 16, 16),       # K below 64
     (1, 65536, 0, 16, 16, 16),    # K above 32768
     (-1, 64, 0, 16, 16, 16),
@@ -89,12 +90,14 @@ def test_null_arguments_are_rejected(lib):
     (1, 64, 0, 0, 16, 16),        # NULL x
     (1, 64, 0, 24, 16, 16),       # misaligned x
     (1, 64, 0, 16, 16, 0),        # NULL signs
+    (1, 64, 0, 16, 16, 24),       # misaligned signs (read in 8-byte words)
     (2, 64, 0, 1024, 1024 + 64, 16),  # partial overlap
 ])
 def test_rht_rejects_bad_arguments_without_a_gpu(lib, M, K, dt, x, xo, signs):
     assert lib.vq_rht_apply(x or None, xo or None, signs or None, M, K, dt, None) == B.VQ_ERR_INVALID_ARG
+    assert lib.vq_rht_apply_output(x or None, xo or None, signs or None, M, K, dt, None) == B.VQ_ERR_INVALID_ARG
 
 
 def test_python_binding_raises_with_message(lib):
-    with pytest.raises(B.VQError, match="power of two"):
+    with pytest.raises(B.VQError, match="multiple of 64"):
         B.vq_rht_apply(16, 16, 16, 1, 100, 0, stream=0)

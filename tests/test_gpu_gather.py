@@ -131,7 +131,9 @@ def _rotated_reference(oracle, layer, x, act, signs, rows):
 
 
 @pytest.mark.parametrize("shape", [(256, 256, 256, DT_F16), (520, 2048, 64, DT_BF16), (64, 128, 128, DT_F16),
-                                   (256, 512, 512, DT_BF16), (128, 1024, 64, DT_F16), (132, 16384, 64, DT_F16)],
+                                   (256, 512, 512, DT_BF16), (128, 1024, 64, DT_F16), (132, 16384, 64, DT_F16),
+                                   # K not a power of two: block-diagonal rotation (2048 + 512 + 128, ...)
+                                   (256, 2688, 64, DT_BF16), (200, 384, 384, DT_F16), (132, 16256, 64, DT_F16)],
                          ids=lambda s: f"{s[0]}x{s[1]}sg{s[2]}a{s[3]}")
 def test_rotated_fused_matches_oracle(oracle, shape):
     N, K, sg, act = shape
@@ -185,16 +187,37 @@ def test_rotated_argument_errors():
     with pytest.raises(vq.VQError) as ei:
         vq.vq_linear_forward_rotated(L.handle, x8[:1], None, L.planes, L.codebooks, L.t["scales"], y, 1, 256, 256)
     assert ei.value.status == vq._binding.VQ_ERR_INVALID_ARG
-    layer2 = make_layer(LayerSpec(256, 384, FMT_VQ16, 384), cfg_id=75)
+    layer2 = make_layer(LayerSpec(8, 65536, FMT_VQ16, 65536), cfg_id=75)
     L2 = layer_on_gpu(layer2, DT_F16, 1)
-    with pytest.raises(vq.VQError) as ei:  # K not a power of two
-        L2.forward_rotated(torch.zeros((1, 384), dtype=torch.float16, device="cuda"), dev(make_signs(384, cfg_id=75)))
+    with pytest.raises(vq.VQError) as ei:  # K above the rotation's 32768
+        L2.forward_rotated(torch.zeros((1, 65536), dtype=torch.float16, device="cuda"),
+                           dev(make_signs(65536, cfg_id=75)))
     assert ei.value.status == vq._binding.VQ_ERR_INVALID_ARG
+    with pytest.raises(vq.VQError) as ei:  # signs not 16-byte aligned
+        L.forward_rotated(x8[:1], dev(make_signs(264, cfg_id=75))[8:])
+    assert ei.value.status == vq._binding.VQ_ERR_INVALID_ARG
+
+
+def test_rotated_block_diagonal_unfused(oracle):
+    """K = 2688 = 2048 + 512 + 128 at M = 8: the rotation kernel into the handle's buffer,
+    then the forward, against the oracle's block-diagonal rotation rounded the same way."""
+    N, K, M = 384, 2688, 8
+    layer = make_layer(LayerSpec(N, K, FMT_VQ16, 64), cfg_id=76)
+    L = vq.VQLinear(N, K, FMT_VQ16, 64, DT_BF16, M, layer, rht=1)
+    x = make_x(M, K, DT_BF16, cfg_id=76)
+    signs = make_signs(K, cfg_id=76)
+    y = host_bits(L.forward_rotated(dev(x).view(torch.bfloat16), dev(signs)))
+    torch.cuda.synchronize()
+    vq.vq_linear_check(L.handle)
+    x_rot = oracle.round_to(oracle.rht(x, DT_BF16, signs), DT_BF16)
+    y_ref = oracle.forward(layer, x_rot, DT_BF16)
+    w, _ = oracle.dequant(layer)
+    assert_y_within(y, DT_BF16, y_ref, oracle.tolerance(x_rot, DT_BF16, w, TOL), what="K=2688 M=8 rotated")
 
 
 # ------------------------------------------------------------------- output rotation
 
-@pytest.mark.parametrize("N", [64, 1024, 4096, 32768])
+@pytest.mark.parametrize("N", [64, 1024, 4096, 32768, 2688, 32704])
 @pytest.mark.parametrize("dt", [DT_F16, DT_BF16])
 def test_rht_output_matches_oracle(oracle, N, dt):
     """signs * (1/sqrt N) H y against the oracle's explicit product: within one output ulp

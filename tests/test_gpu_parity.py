@@ -218,7 +218,8 @@ def _rht_check(oracle, M, K, dt):
     return got
 
 
-@pytest.mark.parametrize("K", [64, 128, 1024, 4096, 32768])
+@pytest.mark.parametrize("K", [64, 128, 1024, 4096, 32768,
+                               192, 2688, 12288, 32704])  # block-diagonal: 32704 has all nine blocks 16384..64
 @pytest.mark.parametrize("dt", [DT_F16, DT_BF16])
 def test_rht_matches_oracle(oracle, K, dt):
     _rht_check(oracle, 3, K, dt)
