@@ -20,7 +20,11 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 SRC = os.path.join(HERE, "vq_oracle.c")
 LIB = os.path.join(HERE, "liboracle.so")
 
-FMT_RVQ12, FMT_RVQ12_4, FMT_VQ16 = 1, 2, 3
+FMT_RVQ12, FMT_RVQ12_4, FMT_VQ16, FMT_VQ16_RVQ = 1, 2, 3, 4
+
+# GLQ README, "Bit widths" table: bits per weight -> (16-bit stages including the
+# primary, 8-bit residual stages).
+LADDER_STAGES = {2: (1, 0), 3: (1, 1), 4: (2, 0), 5: (2, 1), 6: (3, 0), 7: (3, 1), 8: (4, 0)}
 DT_F16, DT_BF16 = 0, 1
 
 _lock = threading.Lock()
@@ -71,6 +75,10 @@ def _load():
             lib.vqo_forward.argtypes = [I, I, I, I, P, I, P, P, P, P, P, P, P, I, P, I, P]
             lib.vqo_rht.restype = I
             lib.vqo_rht.argtypes = [I, I, P, I, P, P]
+            lib.vqo_ladder_dequant.restype = I
+            lib.vqo_ladder_dequant.argtypes = [I, I, I, I, P, P, P, P, P, P, P, I, P, I, P, P, I]
+            lib.vqo_ladder_forward.restype = I
+            lib.vqo_ladder_forward.argtypes = [I, I, I, I, I, P, I, P, P, P, P, P, P, P, I, P, I, P]
             _lib = lib
     return _lib
 
@@ -123,9 +131,12 @@ def unpack(layer) -> tuple[np.ndarray, np.ndarray]:
     lib = _load()
     spec = layer["spec"]
     lo, hi4, s2, idx16 = _planes(layer)
+    fmt = spec.fmt
+    if fmt == FMT_VQ16_RVQ:  # the primary stage's plane
+        fmt, idx16 = FMT_VQ16, np.ascontiguousarray(idx16[: spec.N * spec.G])
     i1 = np.empty((spec.N, spec.G), dtype=np.uint32)
     i2 = np.empty((spec.N, spec.G), dtype=np.uint8)
-    rc = lib.vqo_unpack(spec.fmt, spec.N, spec.K, _p(lo), _p(hi4), _p(s2), _p(idx16), _p(i1), _p(i2))
+    rc = lib.vqo_unpack(fmt, spec.N, spec.K, _p(lo), _p(hi4), _p(s2), _p(idx16), _p(i1), _p(i2))
     if rc:
         raise ValueError(f"vqo_unpack failed rc={rc}")
     return i1, i2
@@ -138,10 +149,32 @@ def _rows(rows):
     return r, int(r.size)
 
 
+def _ladder(layer):
+    """The residual ladder's arrays (GLQ README, "Bit widths") in the oracle's calling form."""
+    spec = layer["spec"]
+    n16, _ = LADDER_STAGES[spec.bpw]
+    cbr = layer["cbr"] if n16 > 1 else np.zeros((1, 65536, 8), np.uint16)
+    return (_c(layer["idx16"], np.uint16), _c(layer.get("idx8"), np.uint8), _c(layer["cb1"], np.uint16),
+            _c(cbr, np.uint16), _c(layer["cb8"], np.uint16), _c(layer["mult"], np.float32).astype(np.float64),
+            _c(layer["scales"], np.uint16))
+
+
 def dequant(layer, wdt: int = DT_F16, rows=None) -> tuple[np.ndarray, np.ndarray]:
     """Return (W exact fp64 [n,K], W materialised fp16/bf16 bits [n,K]) for `rows` (default: all)."""
     lib = _load()
     spec = layer["spec"]
+    if spec.fmt == FMT_VQ16_RVQ:
+        idx16, idx8, cb1, cbr, cb8, mult, sc = _ladder(layer)
+        r, nr = _rows(rows)
+        n = spec.N if r is None else nr
+        w = np.empty((n, spec.K), dtype=np.float64)
+        wb = np.empty((n, spec.K), dtype=np.uint16)
+        n16, n8 = LADDER_STAGES[spec.bpw]
+        rc = lib.vqo_ladder_dequant(spec.N, spec.K, n16, n8, _p(idx16), _p(idx8), _p(cb1), _p(cbr),
+                                    _p(cb8), _p(mult), _p(sc), spec.scale_group, _p(r), nr, _p(w), _p(wb), wdt)
+        if rc:
+            raise ValueError(f"vqo_ladder_dequant failed rc={rc}")
+        return w, wb
     lo, hi4, s2, idx16 = _planes(layer)
     cb1, cb2, sc = _c(layer["cb1"], np.uint16), _c(layer.get("cb2"), np.uint16), _c(layer["scales"], np.uint16)
     r, nr = _rows(rows)
@@ -163,11 +196,20 @@ def forward(layer, x_bits, xdt: int, rows=None) -> np.ndarray:
     M = x.shape[0]
     if x.shape[1] != spec.K:
         raise ValueError("x has the wrong K")
-    lo, hi4, s2, idx16 = _planes(layer)
-    cb1, cb2, sc = _c(layer["cb1"], np.uint16), _c(layer.get("cb2"), np.uint16), _c(layer["scales"], np.uint16)
     r, nr = _rows(rows)
     n = spec.N if r is None else nr
     y = np.empty((M, n), dtype=np.float64)
+    if spec.fmt == FMT_VQ16_RVQ:
+        idx16, idx8, cb1, cbr, cb8, mult, sc = _ladder(layer)
+        n16, n8 = LADDER_STAGES[spec.bpw]
+        rc = lib.vqo_ladder_forward(M, spec.N, spec.K, n16, n8, _p(x), xdt, _p(idx16), _p(idx8),
+                                    _p(cb1), _p(cbr), _p(cb8), _p(mult), _p(sc), spec.scale_group, _p(r), nr,
+                                    _p(y))
+        if rc:
+            raise ValueError(f"vqo_ladder_forward failed rc={rc}")
+        return y
+    lo, hi4, s2, idx16 = _planes(layer)
+    cb1, cb2, sc = _c(layer["cb1"], np.uint16), _c(layer.get("cb2"), np.uint16), _c(layer["scales"], np.uint16)
     rc = lib.vqo_forward(spec.fmt, M, spec.N, spec.K, _p(x), xdt, _p(lo), _p(hi4), _p(s2), _p(idx16), _p(cb1),
                          _p(cb2), _p(sc), spec.scale_group, _p(r), nr, _p(y))
     if rc:

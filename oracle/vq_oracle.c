@@ -15,6 +15,8 @@
  *     of 8 into a 65,536-entry table; "Randomized Hadamard Transform": random sign
  *     flips followed by a fast Walsh-Hadamard transform.
  *   - GLQ README, "Inference kernels": Y = X . dequant(W)^T without materialising W.
+ *   - GLQ README, "Bit widths": the residual ladder (16-bit primary, 16-bit
+ *     residual stages, one 8-bit stage for odd bit widths), vqo_ladder_*.
  *
  * Readings taken where the pages are silent (all fixed here, by construction):
  *   - groups run along K (the input dimension), G = K/8 groups per row;
@@ -289,6 +291,129 @@ int vqo_forward(int fmt, int M, int N, int K, const uint16_t* x, int xdt, const 
   }
   free(i1);
   free(i2);
+  free(wrow);
+  free(xd);
+  return rc;
+}
+
+/* ---------------------------------------------------------------------------
+ * Residual ladder (GLQ README, "Bit widths": a 16-bit primary stage, then 16-bit
+ * residual stages, and for an odd bit width one final 8-bit stage -- 3 bpw is
+ * 16 + 8, 4 is 16 + 16, ..., 8 is four 16-bit stages; "Direct kernel access":
+ * each residual stage comes with its own codebook and an inverse residual scale).
+ * Weight (n, k) with g = k / 8, j = k % 8:
+ *   W = s(n, k) * ( cb1[i_1][j] + sum_{t=2..n16} mult[t-2] * cbr[t-2][i_t][j]
+ *                   + [n8 = 1] mult[n16-1] * cb8[i_8][j] )
+ * i_t is the entry of 16-bit plane t (planes stage-major, each K-slice-major like
+ * idx16), i_8 that of the 8-bit plane (same layout, one byte per group).
+ * Materialised weight (reading): v = c1, then v = fl32(mult * c + v) for each
+ * residual stage in order (one rounding per stage, a fused multiply-add), then
+ * RN(fl32(s * v)) to fp16 or bf16.
+ * ------------------------------------------------------------------------- */
+
+/* fl32(p + c) with one rounding, for fp64 p and c: TwoSum keeps the exact sum as
+ * t + e; t + e rounds like t unless t is exactly halfway between two binary32
+ * values, where the sign of e decides. */
+static double vqo_fl32_sum(double p, double c) {
+  const double t = p + c;
+  const double pv = t - c;
+  const double e = (p - pv) + (c - (t - pv));
+  const double r = vqo_fl32(t);
+  if (e == 0.0 || r == t) return r;
+  const uint32_t bits = vqo_round_bits(r, 8, 23);
+  const uint32_t sign = bits & 0x80000000u, mag = bits & 0x7FFFFFFFu;
+  double other;
+  if (mag == 0)
+    other = vqo_decode_bits((t < 0 ? 0x80000000u : 0u) | 1u, 8, 23);
+  else
+    other = vqo_decode_bits(sign | (fabs(t) > fabs(r) ? mag + 1u : mag - 1u), 8, 23);
+  if (t != 0.5 * (r + other)) return r;
+  return (e > 0) == (other > r) ? other : r;
+}
+
+static int vqo_ladder_check(int N, int K, int n16, int n8, int scale_group) {
+  if (n16 < 1 || n16 > 4 || n8 < 0 || n8 > 1 || n16 + n8 > 4) return 1;
+  return vqo_check(VQO_FMT_VQ16, N, K, scale_group);
+}
+
+/* Exact stage sum c and materialised stage sum v (fp32 value) of group g of row n. */
+static void vqo_ladder_group(int n, int g, int N, int K, int n16, int n8, const uint16_t* idx16,
+                             const uint8_t* idx8, const uint16_t* cb1, const uint16_t* cbr, const uint16_t* cb8,
+                             const double* mult, double c[8], double v[8]) {
+  const int G = K / 8;
+  const int64_t e = vqo_slice_entry(n, g, N, G), NG = (int64_t)N * G;
+  for (int j = 0; j < 8; ++j) c[j] = v[j] = vqo_f16_to_f64(cb1[(int64_t)idx16[e] * 8 + j]);
+  for (int t = 1; t < n16; ++t) {
+    const uint16_t* cb = cbr + (int64_t)(t - 1) * 65536 * 8;
+    const int64_t i = idx16[(int64_t)t * NG + e];
+    for (int j = 0; j < 8; ++j) {
+      const double cw = vqo_f16_to_f64(cb[i * 8 + j]);
+      c[j] += mult[t - 1] * cw;
+      v[j] = vqo_fl32_sum(mult[t - 1] * cw, v[j]); /* the product is exact in fp64 */
+    }
+  }
+  if (n8) {
+    const int64_t i = idx8[e];
+    for (int j = 0; j < 8; ++j) {
+      const double cw = vqo_f16_to_f64(cb8[i * 8 + j]);
+      c[j] += mult[n16 - 1] * cw;
+      v[j] = vqo_fl32_sum(mult[n16 - 1] * cw, v[j]);
+    }
+  }
+}
+
+/* As vqo_dequant, for the ladder: cbr is [n16-1][65536][8], mult [n16-1+n8]. */
+int vqo_ladder_dequant(int N, int K, int n16, int n8, const uint16_t* idx16, const uint8_t* idx8,
+                       const uint16_t* cb1, const uint16_t* cbr, const uint16_t* cb8, const double* mult,
+                       const uint16_t* scales, int scale_group, const int32_t* rows, int nrows, double* w_exact,
+                       uint16_t* w_bits, int wdt) {
+  int rc = vqo_ladder_check(N, K, n16, n8, scale_group);
+  if (rc) return rc;
+  if (!rows) nrows = N;
+  const int G = K / 8;
+  for (int t = 0; t < nrows; ++t) {
+    const int n = rows ? rows[t] : t;
+    if (n < 0 || n >= N) return 1;
+    for (int g = 0; g < G; ++g) {
+      double c[8], v[8];
+      vqo_ladder_group(n, g, N, K, n16, n8, idx16, idx8, cb1, cbr, cb8, mult, c, v);
+      for (int j = 0; j < 8; ++j) {
+        const int k = 8 * g + j;
+        const double sc = vqo_f16_to_f64(scales[vqo_scale_index(n, k, N, K, scale_group)]);
+        if (w_exact) w_exact[(int64_t)t * K + k] = sc * c[j];
+        if (w_bits) {
+          const double p32 = vqo_fl32(sc * v[j]); /* exact product of two fp32 values, rounded once */
+          w_bits[(int64_t)t * K + k] = wdt == VQO_DT_BF16 ? vqo_f64_to_bf16(p32) : vqo_f64_to_f16(p32);
+        }
+      }
+    }
+  }
+  return 0;
+}
+
+/* As vqo_forward, for the ladder: y[m][t] = sum_k x[m][k] W[rows[t]][k] in fp64. */
+int vqo_ladder_forward(int M, int N, int K, int n16, int n8, const uint16_t* x, int xdt, const uint16_t* idx16,
+                       const uint8_t* idx8, const uint16_t* cb1, const uint16_t* cbr, const uint16_t* cb8,
+                       const double* mult, const uint16_t* scales, int scale_group, const int32_t* rows, int nrows,
+                       double* y) {
+  int rc = vqo_ladder_check(N, K, n16, n8, scale_group);
+  if (rc || M < 0) return rc ? rc : 1;
+  if (!rows) nrows = N;
+  double* wrow = (double*)malloc(sizeof(double) * (size_t)K);
+  double* xd = (double*)malloc(sizeof(double) * (size_t)M * K + 1);
+  if (!wrow || !xd) { free(wrow); free(xd); return 3; }
+  for (int64_t t = 0; t < (int64_t)M * K; ++t) xd[t] = vqo_act_to_f64(x[t], xdt);
+  for (int t = 0; rc == 0 && t < nrows; ++t) {
+    const int n = rows ? rows[t] : t;
+    if (n < 0 || n >= N) { rc = 1; break; }
+    rc = vqo_ladder_dequant(N, K, n16, n8, idx16, idx8, cb1, cbr, cb8, mult, scales, scale_group, &n, 1, wrow,
+                            NULL, 0);
+    for (int m = 0; rc == 0 && m < M; ++m) {
+      double acc = 0.0;
+      for (int k = 0; k < K; ++k) acc += xd[(int64_t)m * K + k] * wrow[k];
+      y[(int64_t)m * nrows + t] = acc;
+    }
+  }
   free(wrow);
   free(xd);
   return rc;

@@ -19,7 +19,11 @@ Storage format (the encoder's output, consumed by both implementations):
   byte within a row's slice entries: group 2t in bits 0..3, group 2t+1 in 4..7
 * ``s2``  uint8  [N*G/2]    4-bit stage-2 index, packed like ``hi4``
 * ``idx16`` uint16 [N*G]    16-bit single-stage index (GLQ README, "How it
-  works", E8 lattice codebooks: one 16-bit index per group of 8)
+  works", E8 lattice codebooks: one 16-bit index per group of 8); for the
+  residual ladder [n16*N*G], one plane per 16-bit stage, stage-major
+* ``idx8`` uint8 [N*G]      the ladder's 8-bit stage index, same layout as ``lo``
+* ``cbr`` fp16 [n16-1, 65536, 8], ``cb8`` fp16 [256, 8], ``mult`` fp32 [n16-1+n8]:
+  the ladder's residual codebooks and stage multipliers (GLQ README, "Bit widths")
 * ``cb1`` fp16 [4096, 8] (or [65536, 8] for 16-bit indices), ``cb2`` fp16 [16, 8]
 * ``scales`` fp16 [N * K // scale_group]: block scales (scale_group dividing 64)
   in K-slice-major order like the planes (a row's scales of one slice are
@@ -33,6 +37,7 @@ from .layers import (  # noqa: F401
     FMT_RVQ12,
     FMT_RVQ12_4,
     FMT_VQ16,
+    FMT_VQ16_RVQ,
     DT_F16,
     DT_BF16,
     LayerSpec,

@@ -5,6 +5,10 @@ Recipe (one ``numpy.random.Generator`` per tensor, seeded from
 
 * stage-1 codebook: 4096 x 8 (12-bit) or 65536 x 8 (16-bit) fp16 values ~ N(0, 1)
 * stage-2 codebook: 16 x 8 fp16 ~ N(0, 1)
+* residual ladder (16-bit primary + residual stages): one 65536 x 8 codebook per
+  16-bit stage and a 256 x 8 codebook for the 8-bit stage, all fp16 ~ N(0, 1);
+  stage multipliers (inverse residual scales) fp32 4^-(s-1) * U(0.25, 0.5) for
+  residual stage s = 1, 2, 3
 * indices: uniform over their range, i.e. the packed planes are uniform random bytes
 * scales: fp16 lognormal(mu=-4, sigma=0.5), per 64-weight block along K or per row
 * activations: fp16 or bf16 ~ N(0, 1); rotation signs: +-1 with probability 1/2
@@ -21,6 +25,7 @@ import numpy as np
 FMT_RVQ12 = 1     # one 12-bit stage (lo byte + packed hi nibble)
 FMT_RVQ12_4 = 2   # 12-bit stage 1 + 4-bit stage 2
 FMT_VQ16 = 3      # one 16-bit index into a 65,536 x 8 codebook
+FMT_VQ16_RVQ = 4  # 16-bit primary + residual stages (16-bit ones, then at most one 8-bit)
 
 DT_F16 = 0
 DT_BF16 = 1
@@ -45,10 +50,21 @@ class LayerSpec:
     K: int
     fmt: int
     scale_group: int  # 64, or K for one scale per row
+    bpw: int = 2      # FMT_VQ16_RVQ: bits per weight, 2..8 (GLQ README, "Bit widths")
 
     @property
     def G(self) -> int:
         return self.K // 8
+
+    @property
+    def n16(self) -> int:
+        """16-bit stages of the ladder (primary included): bpw // 2."""
+        return self.bpw // 2
+
+    @property
+    def n8(self) -> int:
+        """8-bit stages after them: 1 for odd bpw."""
+        return self.bpw % 2
 
 
 def _rng(cfg_id: int, layer: int, tensor_id: int, seed: int, stream: int = 0) -> np.random.Generator:
@@ -67,6 +83,19 @@ def make_layer(spec: LayerSpec, cfg_id: int = 0, layer: int = 0, tensor_id: int 
     if spec.fmt == FMT_VQ16:
         out["cb1"] = f32_to_f16_bits(r.standard_normal((65536, 8), dtype=np.float32))
         out["idx16"] = r.integers(0, 65536, size=N * G, dtype=np.uint16)
+    elif spec.fmt == FMT_VQ16_RVQ:
+        if not 2 <= spec.bpw <= 8:
+            raise ValueError(f"bpw={spec.bpw} outside 2..8")
+        n16, n8 = spec.n16, spec.n8
+        out["cb1"] = f32_to_f16_bits(r.standard_normal((65536, 8), dtype=np.float32))
+        # residual 16-bit codebooks, stage-major [n16 - 1, 65536, 8]
+        out["cbr"] = f32_to_f16_bits(r.standard_normal((n16 - 1, 65536, 8), dtype=np.float32))
+        out["cb8"] = f32_to_f16_bits(r.standard_normal((256, 8), dtype=np.float32))
+        # stage-major planes: 16-bit stage s at entries [s N G, (s + 1) N G)
+        out["idx16"] = r.integers(0, 65536, size=n16 * N * G, dtype=np.uint16)
+        out["idx8"] = r.integers(0, 256, size=N * G, dtype=np.uint8) if n8 else None
+        nres = n16 - 1 + n8
+        out["mult"] = (4.0 ** -np.arange(nres) * r.uniform(0.25, 0.5, size=nres)).astype(np.float32)
     else:
         out["cb1"] = f32_to_f16_bits(r.standard_normal((4096, 8), dtype=np.float32))
         out["lo"] = r.integers(0, 256, size=N * G, dtype=np.uint8)

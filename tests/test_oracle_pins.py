@@ -14,7 +14,8 @@ import pytest
 import scipy.linalg
 import torch
 
-from synth import FMT_RVQ12, FMT_RVQ12_4, FMT_VQ16, DT_BF16, DT_F16, LayerSpec, make_layer, make_x
+from synth import (FMT_RVQ12, FMT_RVQ12_4, FMT_VQ16, FMT_VQ16_RVQ, DT_BF16, DT_F16, LayerSpec, f32_to_bf16_bits,
+                   make_layer, make_x)
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
@@ -378,6 +379,138 @@ def test_rht_bits_entry_matches_f64(oracle):
     signs = np.where(np.arange(K) % 3 == 0, -1, 1).astype(np.int8)
     xd = (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
     assert np.array_equal(oracle.rht(x, DT_BF16, signs), oracle.rht_f64(xd, signs))
+
+
+# ------------------------------------------------------------ residual ladder (F3)
+
+def _f16(a):
+    return np.asarray(a, np.float32).astype(np.float16).view(np.uint16)
+
+
+def _hand_ladder(N, K, bpw, sg, seed=0):
+    """A small ladder layer drawn here (not by synth), for the by-hand pins."""
+    rng = np.random.default_rng(seed)
+    n16, n8 = {2: (1, 0), 3: (1, 1), 4: (2, 0), 5: (2, 1), 6: (3, 0), 7: (3, 1), 8: (4, 0)}[bpw]
+    G = K // 8
+    lay = {"spec": LayerSpec(N, K, FMT_VQ16_RVQ, sg, bpw=bpw),
+           "cb1": _f16(rng.standard_normal((65536, 8))),
+           "cbr": _f16(rng.standard_normal((max(n16 - 1, 1), 65536, 8))),
+           "cb8": _f16(rng.standard_normal((256, 8))),
+           "idx16": rng.integers(0, 65536, size=n16 * N * G).astype(np.uint16),
+           "idx8": rng.integers(0, 256, size=N * G).astype(np.uint8) if n8 else None,
+           "mult": rng.uniform(0.01, 0.5, size=n16 - 1 + n8).astype(np.float32),
+           "scales": _f16(rng.uniform(0.5, 2.0, size=N * K // sg))}
+    return lay, n16, n8
+
+
+@pytest.mark.parametrize("bpw", [3, 4, 5, 6, 7, 8])
+def test_ladder_by_hand_one_slice(oracle, bpw):
+    """GLQ README, "Bit widths": W = s * (cb1[i1] + sum of mult_t * codebook_t[i_t]).  K = 128 is
+    one slice, so group g of row n is entry 16 n + g of every plane, and the two 64-wide
+    block scales of row n are scales[2 n], scales[2 n + 1]."""
+    N, K = 3, 128
+    lay, n16, n8 = _hand_ladder(N, K, bpw, 64, seed=bpw)
+    f = lambda b: b.view(np.float16).astype(np.float64)  # noqa: E731
+    NG = N * 16
+    W = np.zeros((N, K))
+    for n in range(N):
+        for g in range(16):
+            e = 16 * n + g
+            c = f(lay["cb1"][lay["idx16"][e]])
+            for t in range(1, n16):
+                c = c + float(lay["mult"][t - 1]) * f(lay["cbr"][t - 1][lay["idx16"][t * NG + e]])
+            if n8:
+                c = c + float(lay["mult"][n16 - 1]) * f(lay["cb8"][lay["idx8"][e]])
+            W[n, 8 * g:8 * g + 8] = f(lay["scales"][2 * n + g // 8]) * c
+    w, _ = oracle.dequant(lay)
+    assert np.allclose(w, W, rtol=1e-14, atol=1e-15)
+    x = make_x(2, K, DT_F16, cfg_id=97)
+    xd = x.view(np.float16).astype(np.float64)
+    assert np.allclose(oracle.forward(lay, x, DT_F16), xd @ W.T, rtol=1e-12, atol=1e-12)
+
+
+def test_ladder_two_bits_is_the_16bit_format(oracle):
+    """bpw = 2 is the primary stage alone: the same weights as the single-stage 16-bit
+    format on the same plane, codebook and scales, bit for bit."""
+    lay, _, _ = _hand_ladder(40, 384, 2, 64, seed=5)
+    plain = {"spec": LayerSpec(40, 384, FMT_VQ16, 64), "cb1": lay["cb1"], "idx16": lay["idx16"],
+             "scales": lay["scales"]}
+    for wdt in (DT_F16, DT_BF16):
+        w1, b1 = oracle.dequant(lay, wdt)
+        w2, b2 = oracle.dequant(plain, wdt)
+        assert np.array_equal(w1, w2) and np.array_equal(b1, b2)
+
+
+@pytest.mark.parametrize("bpw", [3, 5, 8])
+def test_ladder_is_a_sum_of_single_stage_layers(oracle, bpw):
+    """Linearity in the stages: the ladder equals the sum, over its stages, of multiplier x the
+    single-stage 16-bit decode of that stage's plane and codebook (the 8-bit stage as a
+    16-bit layer whose codebook starts with the 256 entries), several slices, ragged tail."""
+    N, K = 24, 448  # 3 full slices + a 64-wide tail
+    lay, n16, n8 = _hand_ladder(N, K, bpw, 64, seed=10 + bpw)
+    NG = N * K // 8
+    def single(plane, cb):
+        return oracle.dequant({"spec": LayerSpec(N, K, FMT_VQ16, 64), "cb1": cb, "idx16": plane,
+                               "scales": lay["scales"]})[0]
+    ref = single(lay["idx16"][:NG], lay["cb1"])
+    for t in range(1, n16):
+        ref += float(lay["mult"][t - 1]) * single(lay["idx16"][t * NG:(t + 1) * NG], lay["cbr"][t - 1])
+    if n8:
+        cb = np.zeros((65536, 8), np.uint16)
+        cb[:256] = lay["cb8"]
+        ref += float(lay["mult"][n16 - 1]) * single(lay["idx8"].astype(np.uint16), cb)
+    w, _ = oracle.dequant(lay)
+    assert np.allclose(w, ref, rtol=1e-13, atol=1e-13 * np.abs(ref).max())
+
+
+@pytest.mark.parametrize("wdt", [DT_F16, DT_BF16])
+def test_ladder_materialised_bits(oracle, wdt):
+    """Materialised weights: v = c1, v = fl32(mult * c + v) per stage, RN(fl32(s * v)), checked
+    against numpy float32 arithmetic (the product mult * c is exact in float64)."""
+    N, K = 16, 256
+    lay, n16, n8 = _hand_ladder(N, K, 7, 64, seed=21)
+    _, wb = oracle.dequant(lay, wdt)
+    f = lambda b: b.view(np.float16).astype(np.float64)  # noqa: E731
+    NG = N * K // 8
+    G = K // 8
+    v = np.zeros((N, K), np.float32)
+    s = np.zeros((N, K), np.float32)
+    for n in range(N):
+        for g in range(G):
+            sl, o = g // 16, g % 16
+            e = 16 * sl * N + n * 16 + o
+            vv = f(lay["cb1"][lay["idx16"][e]]).astype(np.float32)
+            for t in range(1, n16):
+                vv = (float(lay["mult"][t - 1]) * f(lay["cbr"][t - 1][lay["idx16"][t * NG + e]])
+                      + vv.astype(np.float64)).astype(np.float32)
+            vv = (float(lay["mult"][n16 - 1]) * f(lay["cb8"][lay["idx8"][e]]) + vv.astype(np.float64)).astype(np.float32)
+            v[n, 8 * g:8 * g + 8] = vv
+            s[n, 8 * g:8 * g + 8] = f(lay["scales"][2 * sl * N + 2 * n + o // 8])  # two 64-wide blocks per slice
+    p = (s.astype(np.float64) * v.astype(np.float64)).astype(np.float32)
+    ref = _f16(p) if wdt == DT_F16 else f32_to_bf16_bits(p)
+    assert np.array_equal(wb, ref), f"{np.sum(wb != ref)} weights differ"
+
+
+def test_ladder_stage_sum_rounds_once(oracle):
+    """A tie the fp64 sum alone would get wrong: v = 1 + 2^-11 after stage 2, then
+    mult * c = 2^-24 + 2^-57 (mult = 14245331 * 2^-48, c = 1206 / 1024; 14245331 * 1206 =
+    2^34 + 2).  The exact stage sum is just above the binary32 midpoint 1 + 2^-11 + 2^-24, so
+    one rounding gives 1 + 2^-11 + 2^-23, which is above the fp16 midpoint 1 + 2^-11: the
+    weight is fp16 1 + 2^-10 (0x3C01).  Rounding the fp64 sum instead lands on the midpoint,
+    ties to 1 + 2^-11 and then to fp16 1.0 (0x3C00)."""
+    assert 14245331 * 1206 == 2 ** 34 + 2
+    lay = {"spec": LayerSpec(1, 16, FMT_VQ16_RVQ, 16, bpw=6),
+           "cb1": np.zeros((65536, 8), np.uint16), "cbr": np.zeros((2, 65536, 8), np.uint16),
+           "cb8": np.zeros((256, 8), np.uint16), "idx16": np.zeros(6, np.uint16), "idx8": None,
+           "mult": np.array([2.0 ** -11, 14245331 * 2.0 ** -48], np.float32),
+           "scales": _f16([1.0])}
+    assert float(lay["mult"][1]) == 14245331 * 2.0 ** -48  # exact in binary32
+    lay["cb1"][0] = _f16([1.0] * 8)
+    lay["cbr"][0][0] = _f16([1.0] * 8)
+    lay["cbr"][1][0] = _f16([1206 / 1024] * 8)
+    w, wb = oracle.dequant(lay, DT_F16)
+    assert np.all(wb[0, :8] == 0x3C01), wb[0, :8]
+    assert np.allclose(w[0, :8], 1 + 2.0 ** -11 + 2.0 ** -24 + 2.0 ** -57, rtol=0, atol=1e-16)
 
 
 # ------------------------------------------------- block-diagonal rotation (K not 2^p)
