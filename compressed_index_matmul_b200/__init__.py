@@ -15,6 +15,8 @@ from ._binding import (  # noqa: F401
     VQ_FMT_RVQ12,
     VQ_FMT_RVQ12_4,
     VQ_FMT_VQ16,
+    VQ_FMT_VQ16_RVQ,
+    LADDER_STAGES,
     VQ_PATH_AUTO,
     VQ_PATH_GATHER,
     VQ_PATH_GEMV,

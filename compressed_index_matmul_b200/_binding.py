@@ -17,7 +17,11 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libvqlinear.so")
 
 VQ_OK, VQ_ERR_INVALID_ARG, VQ_ERR_UNSUPPORTED, VQ_ERR_CUDA, VQ_ERR_NOMEM, VQ_ERR_TIMEOUT = range(6)
-VQ_FMT_RVQ12, VQ_FMT_RVQ12_4, VQ_FMT_VQ16 = 1, 2, 3
+VQ_FMT_RVQ12, VQ_FMT_RVQ12_4, VQ_FMT_VQ16, VQ_FMT_VQ16_RVQ = 1, 2, 3, 4
+
+# GLQ README, "Bit widths": bits per weight of the residual ladder -> (16-bit stages
+# including the primary, 8-bit stages after them).
+LADDER_STAGES = {2: (1, 0), 3: (1, 1), 4: (2, 0), 5: (2, 1), 6: (3, 0), 7: (3, 1), 8: (4, 0)}
 VQ_F16, VQ_BF16 = 0, 1
 VQ_PATH_AUTO, VQ_PATH_LUT, VQ_PATH_GEMV, VQ_PATH_TC, VQ_PATH_GATHER = 0, 1, 2, 3, 4
 
@@ -40,16 +44,18 @@ class VQError(RuntimeError):
 class vq_linear_desc(ctypes.Structure):
     _fields_ = [("N", ctypes.c_int32), ("K", ctypes.c_int32), ("fmt", ctypes.c_int32),
                 ("scale_group", ctypes.c_int32), ("act_dtype", ctypes.c_int32), ("max_M", ctypes.c_int32),
-                ("rht", ctypes.c_int32)]
+                ("rht", ctypes.c_int32), ("n16", ctypes.c_int32), ("n8", ctypes.c_int32),
+                ("mult", ctypes.c_float * 3)]
 
 
 class vq_planes(ctypes.Structure):
     _fields_ = [("lo", ctypes.c_void_p), ("hi4", ctypes.c_void_p), ("s2", ctypes.c_void_p),
-                ("idx16", ctypes.c_void_p)]
+                ("idx16", ctypes.c_void_p), ("idx8", ctypes.c_void_p)]
 
 
 class vq_codebooks(ctypes.Structure):
-    _fields_ = [("cb1", ctypes.c_void_p), ("cb2", ctypes.c_void_p)]
+    _fields_ = [("cb1", ctypes.c_void_p), ("cb2", ctypes.c_void_p), ("cbr", ctypes.c_void_p * 3),
+                ("cb8", ctypes.c_void_p)]
 
 
 _lock = threading.Lock()
@@ -131,20 +137,28 @@ def _stream(stream) -> int | None:
     return stream.cuda_stream
 
 
-def make_planes(lo=None, hi4=None, s2=None, idx16=None) -> vq_planes:
-    return vq_planes(_ptr(lo), _ptr(hi4), _ptr(s2), _ptr(idx16))
+def make_planes(lo=None, hi4=None, s2=None, idx16=None, idx8=None) -> vq_planes:
+    return vq_planes(_ptr(lo), _ptr(hi4), _ptr(s2), _ptr(idx16), _ptr(idx8))
 
 
-def make_codebooks(cb1, cb2=None) -> vq_codebooks:
-    return vq_codebooks(_ptr(cb1), _ptr(cb2))
+def make_codebooks(cb1, cb2=None, cbr=(), cb8=None) -> vq_codebooks:
+    """cbr: up to three codebooks (tensors or raw device addresses) of the ladder's 16-bit
+    residual stages."""
+    cbr = list(cbr) + [None] * (3 - len(cbr))
+    return vq_codebooks(_ptr(cb1), _ptr(cb2), (ctypes.c_void_p * 3)(*[_ptr(c) for c in cbr]), _ptr(cb8))
+
+
+def make_desc(N, K, fmt, scale_group, act_dtype, max_M, rht=0, n16=0, n8=0, mult=()) -> vq_linear_desc:
+    m = list(mult) + [0.0] * (3 - len(mult))
+    return vq_linear_desc(N, K, fmt, scale_group, act_dtype, max_M, rht, n16, n8, (ctypes.c_float * 3)(*m))
 
 
 def vq_abi_version() -> int:
     return load().vq_abi_version()
 
 
-def vq_linear_create(N, K, fmt, scale_group, act_dtype, max_M, rht=0) -> int:
-    d = vq_linear_desc(N, K, fmt, scale_group, act_dtype, max_M, rht)
+def vq_linear_create(N, K, fmt, scale_group, act_dtype, max_M, rht=0, n16=0, n8=0, mult=()) -> int:
+    d = make_desc(N, K, fmt, scale_group, act_dtype, max_M, rht, n16, n8, mult)
     h = ctypes.c_void_p()
     _check(load().vq_linear_create(ctypes.byref(d), ctypes.byref(h)))
     return h.value
@@ -179,9 +193,9 @@ def vq_linear_forward_rotated(h, x, signs, planes: vq_planes, codebooks: vq_code
 
 
 def vq_linear_forward_noalloc(N, K, fmt, scale_group, act_dtype, x, planes: vq_planes, codebooks: vq_codebooks,
-                              scales, y, M, stream=None, rht=0) -> None:
+                              scales, y, M, stream=None, rht=0, n16=0, n8=0, mult=()) -> None:
     """Handle-free forward of 0 <= M <= 16 tokens that allocates nothing (fixed in-library scratch)."""
-    d = vq_linear_desc(N, K, fmt, scale_group, act_dtype, max(M, 1), rht)
+    d = make_desc(N, K, fmt, scale_group, act_dtype, max(M, 1), rht, n16, n8, mult)
     _check(load().vq_linear_forward_noalloc(ctypes.byref(d), _ptr(x), ctypes.byref(planes), ctypes.byref(codebooks),
                                             _ptr(scales), _ptr(y), M, _stream(stream)))
 

@@ -71,8 +71,14 @@ vq_status validate_desc(const vq_linear_desc* d) {
   if (d->K % 64 != 0) return fail(VQ_ERR_UNSUPPORTED, "K=%d: this library needs K to be a multiple of 64", d->K);
   if (d->N > (1 << 24) || d->K > (1 << 24))
     return fail(VQ_ERR_UNSUPPORTED, "N=%d / K=%d exceed the supported 2^24", d->N, d->K);
-  if (d->fmt != VQ_FMT_RVQ12 && d->fmt != VQ_FMT_RVQ12_4 && d->fmt != VQ_FMT_VQ16)
+  if (d->fmt != VQ_FMT_RVQ12 && d->fmt != VQ_FMT_RVQ12_4 && d->fmt != VQ_FMT_VQ16 && d->fmt != VQ_FMT_VQ16_RVQ)
     return fail(VQ_ERR_INVALID_ARG, "fmt=%d is not a VQ_FMT_* value", d->fmt);
+  if (d->fmt == VQ_FMT_VQ16_RVQ) {
+    if (d->n16 < 1 || d->n16 > 4 || d->n8 < 0 || d->n8 > 1 || d->n16 + d->n8 > 4)
+      return fail(VQ_ERR_INVALID_ARG, "n16=%d, n8=%d: need 1 <= n16, 0 <= n8 <= 1, n16 + n8 <= 4", d->n16, d->n8);
+    for (int t = 0; t < d->n16 + d->n8 - 1; ++t)
+      if (!std::isfinite(d->mult[t])) return fail(VQ_ERR_INVALID_ARG, "mult[%d] is not finite", t);
+  }
   if (d->scale_group <= 0 || d->scale_group % 8 != 0 || d->K % d->scale_group != 0)
     return fail(VQ_ERR_INVALID_ARG, "scale_group=%d must be a positive multiple of 8 dividing K", d->scale_group);
   if (d->scale_group != 64 && d->scale_group != d->K)
@@ -87,8 +93,9 @@ vq_status validate_desc(const vq_linear_desc* d) {
 vq_status validate_planes(const vq_linear_desc& d, const vq_planes* p) {
   if (p == nullptr) return fail(VQ_ERR_INVALID_ARG, "planes is NULL");
   vq_status st;
-  if (d.fmt == VQ_FMT_VQ16) {
+  if (d.fmt == VQ_FMT_VQ16 || d.fmt == VQ_FMT_VQ16_RVQ) {
     if ((st = check_ptr(p->idx16, "planes->idx16"))) return st;
+    if (d.fmt == VQ_FMT_VQ16_RVQ && d.n8 && (st = check_ptr(p->idx8, "planes->idx8"))) return st;
   } else {
     if ((st = check_ptr(p->lo, "planes->lo"))) return st;
     if ((st = check_ptr(p->hi4, "planes->hi4"))) return st;
@@ -102,6 +109,11 @@ vq_status validate_codebooks(const vq_linear_desc& d, const vq_codebooks* cb, co
   vq_status st;
   if ((st = check_ptr(cb->cb1, "codebooks->cb1"))) return st;
   if (d.fmt == VQ_FMT_RVQ12_4 && (st = check_ptr(cb->cb2, "codebooks->cb2"))) return st;
+  if (d.fmt == VQ_FMT_VQ16_RVQ) {
+    for (int t = 0; t < d.n16 - 1; ++t)
+      if ((st = check_ptr(cb->cbr[t], "codebooks->cbr[t]"))) return st;
+    if (d.n8 && (st = check_ptr(cb->cb8, "codebooks->cb8"))) return st;
+  }
   if ((st = check_ptr(scales, "scales"))) return st;
   return VQ_OK;
 }
@@ -129,6 +141,18 @@ vq::LayerArgs make_args(const vq_linear_desc& d, const vq_planes* p, const vq_co
   a.fmt = d.fmt;
   a.scale_group = d.scale_group;
   a.act = d.act_dtype;
+  a.n16 = 1;
+  a.n8 = 0;
+  if (d.fmt == VQ_FMT_VQ16_RVQ) {  // only the entries the stage counts use are read
+    a.n16 = d.n16;
+    a.n8 = d.n8;
+    a.idx8 = (p && d.n8) ? p->idx8 : nullptr;
+    for (int t = 0; t < 3; ++t) {
+      a.cbr[t] = (cb && t < d.n16 - 1) ? static_cast<const uint16_t*>(cb->cbr[t]) : nullptr;
+      a.mult[t] = t < d.n16 + d.n8 - 1 ? d.mult[t] : 0.f;
+    }
+    a.cb8 = (cb && d.n8) ? static_cast<const uint16_t*>(cb->cb8) : nullptr;
+  }
   return a;
 }
 
@@ -145,7 +169,7 @@ bool plan_forward(const vq_linear_desc& d, const DeviceInfo& dev, int M, int for
     path = (M == 1) ? VQ_PATH_LUT : ((M <= 16 && !large) ? VQ_PATH_GEMV : VQ_PATH_TC);
     // 16-bit indices, up to 4 tokens: the gather kernel where it applies (measured on
     // B200, 4096 x 4096: faster than the tensor-core path up to M = 4, slower at 8)
-    if (d.fmt == VQ_FMT_VQ16 && M <= 4 && plan_vq16(d, dev, M, out)) return true;
+    if ((d.fmt == VQ_FMT_VQ16 || d.fmt == VQ_FMT_VQ16_RVQ) && M <= 4 && plan_vq16(d, dev, M, out)) return true;
   }
   switch (path) {
     case VQ_PATH_GATHER:
@@ -174,7 +198,7 @@ bool plan_forward(const vq_linear_desc& d, const DeviceInfo& dev, int M, int for
 
 }  // namespace vq
 
-VQ_API int32_t vq_abi_version(void) { return 1; }
+VQ_API int32_t vq_abi_version(void) { return 2; }
 
 VQ_API const char* vq_last_error(void) { return t_err.c_str(); }
 

@@ -4,6 +4,7 @@
 #include "common.cuh"
 #include "rotate.cuh"
 #include "internal.h"
+#include "ladder.cuh"
 #include "tc_ptx.cuh"
 
 namespace vq {
@@ -94,7 +95,7 @@ cudaError_t launch_rht_output(const void* y, void* y_out, const int8_t* signs, i
 __device__ __forceinline__ void unpack_one(const LayerArgs& a, int n, int g, uint32_t* i1, uint32_t* i2) {
   const int G = a.K / 8;
   const int64_t e = slice_entry(n, g, a.N, G);  // even for even g (slice widths are even)
-  if (a.fmt == kFmtVq16) {
+  if (a.fmt == kFmtVq16 || a.fmt == kFmtVq16Rvq) {  // the primary stage's plane
     *i1 = a.idx16[e];
     *i2 = 0;
     return;
@@ -131,7 +132,27 @@ __global__ void debug_dequant_kernel(LayerArgs a, uint16_t* __restrict__ w) {
     const float s = f16_bits_to_f32(a.scales[scale_index(n, 8 * g, a.N, a.K, a.scale_group)]);
     const uint4 c1 = reinterpret_cast<const uint4*>(a.cb1)[i1];
     uint32_t out[4];
-    if (a.fmt == kFmtRvq12_4) {
+    if (a.fmt == kFmtVq16Rvq) {  // the residual ladder, stage by stage (ladder.cuh)
+      const int64_t e = slice_entry(n, g, a.N, G), NG = (int64_t)a.N * G;
+      float v[8];
+      const uint32_t w1[4] = {c1.x, c1.y, c1.z, c1.w};
+      for (int p = 0; p < 4; ++p) {
+        const float2 f = f16x2_to_f32x2(w1[p]);
+        v[2 * p] = f.x;
+        v[2 * p + 1] = f.y;
+      }
+      for (int t = 2; t <= a.n16; ++t) {
+        const uint16_t* cb = t == 2 ? a.cbr[0] : (t == 3 ? a.cbr[1] : a.cbr[2]);
+        const float m = t == 2 ? a.mult[0] : (t == 3 ? a.mult[1] : a.mult[2]);
+        fma_codeword(m, reinterpret_cast<const uint4*>(cb)[a.idx16[(int64_t)(t - 1) * NG + e]], v);
+      }
+      if (a.n8) {
+        const int t = a.n16 + 1;
+        const float m = t == 2 ? a.mult[0] : (t == 3 ? a.mult[1] : a.mult[2]);
+        fma_codeword(m, reinterpret_cast<const uint4*>(a.cb8)[a.idx8[e]], v);
+      }
+      pack_scaled<W>(v, s, out);
+    } else if (a.fmt == kFmtRvq12_4) {
       const uint4 c2 = reinterpret_cast<const uint4*>(a.cb2)[i2];
       decode_group_packed<W, true>(c1, c2, s, out);
     } else {

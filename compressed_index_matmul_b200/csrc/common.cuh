@@ -17,6 +17,7 @@ namespace vq {
 constexpr int kFmtRvq12 = 1;
 constexpr int kFmtRvq12_4 = 2;
 constexpr int kFmtVq16 = 3;
+constexpr int kFmtVq16Rvq = 4;  // residual ladder: 16-bit stages, then at most one 8-bit stage
 
 // Device error flag bits (written by bounded waits that gave up).
 constexpr uint32_t kErrTimeout = 1u;

@@ -21,7 +21,8 @@
 // shared-memory load -- no shuffles on either operand.
 //
 // Decoded weights use the materialised-weight rounding (stage sum and scaled
-// value rounded to fp32, then to the activation type), so every product the MMA
+// value rounded to fp32, then to the activation type; for the residual ladder one
+// fused multiply-add per residual stage, ladder.cuh), so every product the MMA
 // forms is of exactly the weights vq_debug_dequant exports.
 //
 // Split-K reduction: each split writes fp32 partials; the CTA that completes a
@@ -32,6 +33,7 @@
 // kernel in the stream, and reads x / writes y only after that wait.
 #include "common.cuh"
 #include "internal.h"
+#include "ladder.cuh"
 #include "tc_ptx.cuh"
 
 namespace vq {
@@ -51,6 +53,12 @@ struct BlockIdx {
   uint32_t w[2][4];  // per row: lo (2 words) + hi4 (1) + s2 (1), or idx16 (4 words)
   uint32_t sc;       // two fp16 scales (rows g, g+8)
 };
+template <>
+struct BlockIdx<kFmtVq16Rvq> {
+  uint32_t w[2][4];  // per row: the primary stage's idx16 words
+  uint32_t sc;
+  LadderIdx res[2];  // per row: the residual stages' index words
+};
 
 // Index bytes of one 64-wide k block (8 groups, starting at group gbase) for rows
 // g and g+8 of the lane, plus their scales.
@@ -63,9 +71,11 @@ __device__ __forceinline__ void load_block(const LayerArgs& a, const int rows[2]
 #pragma unroll
   for (int r = 0; r < 2; ++r) {
     b.w[r][0] = b.w[r][1] = b.w[r][2] = b.w[r][3] = 0;
+    if constexpr (FMT == kFmtVq16Rvq) b.res[r] = LadderIdx{};
     if (!valid[r]) continue;
     const int64_t e = (int64_t)16 * s * a.N + (int64_t)rows[r] * w + o;
-    if (FMT == kFmtVq16) {
+    if constexpr (FMT == kFmtVq16Rvq) load_ladder_block(a, e, b.res[r]);
+    if (FMT == kFmtVq16 || FMT == kFmtVq16Rvq) {
       const uint4 v = *reinterpret_cast<const uint4*>(a.idx16 + e);
       b.w[r][0] = v.x; b.w[r][1] = v.y; b.w[r][2] = v.z; b.w[r][3] = v.w;
     } else {
@@ -84,7 +94,8 @@ template <int FMT, typename T, int NT>
 __global__ void __launch_bounds__(256) gemv_kernel(LayerArgs a, int k_per_split, int splits, float* __restrict__ partial,
                                                    uint32_t* __restrict__ tickets) {
   extern __shared__ __align__(128) unsigned char smem[];
-  constexpr bool kSmemCb = (FMT != kFmtVq16);
+  constexpr bool k16 = (FMT == kFmtVq16 || FMT == kFmtVq16Rvq);
+  constexpr bool kSmemCb = !k16;
   constexpr bool kTwo = (FMT == kFmtRvq12_4);
   uint4* cb1s = reinterpret_cast<uint4*>(smem);                                // 4096 entries
   uint4* cb2s = cb1s + (kSmemCb ? 4096 : 0);                                   // 16 entries
@@ -157,15 +168,21 @@ __global__ void __launch_bounds__(256) gemv_kernel(LayerArgs a, int k_per_split,
 #pragma unroll
       for (int r = 0; r < 2; ++r) {
         uint32_t i1, i2 = 0;
-        if (FMT == kFmtVq16) {
+        if (k16) {
           i1 = (cur.w[r][q >> 1] >> (16 * (q & 1))) & 0xFFFFu;
         } else {
           i1 = ((cur.w[r][q >> 2] >> (8 * (q & 3))) & 0xFFu) | (((cur.w[r][2] >> (4 * q)) & 15u) << 8);
           if (kTwo) i2 = (cur.w[r][3] >> (4 * q)) & 15u;
         }
         const uint4 c1 = kSmemCb ? cb1s[i1] : __ldg(reinterpret_cast<const uint4*>(a.cb1) + i1);
-        const uint4 c2 = kTwo ? cb2s[i2] : c1;
-        decode_group_packed<T, kTwo>(c1, c2, active ? s[r] : 0.f, wq[r]);
+        if constexpr (FMT == kFmtVq16Rvq) {
+          float v[8];
+          ladder_sum(a, cur.res[r], q, c1, v);
+          pack_scaled<T>(v, active ? s[r] : 0.f, wq[r]);
+        } else {
+          const uint4 c2 = kTwo ? cb2s[i2] : c1;
+          decode_group_packed<T, kTwo>(c1, c2, active ? s[r] : 0.f, wq[r]);
+        }
       }
 #pragma unroll
       for (int t = 0; t < NT; ++t) {
@@ -222,7 +239,8 @@ __global__ void __launch_bounds__(256) gemv_kernel(LayerArgs a, int k_per_split,
 template <int FMT, typename T, int NT>
 static cudaError_t launch_one(const LayerArgs& a, const Plan& p, float* scratch, uint32_t* tickets, cudaStream_t s) {
   const int kc = p.k_per_split;
-  const size_t smem = (FMT != kFmtVq16 ? 4096 * 16 : 0) + (FMT == kFmtRvq12_4 ? 256 : 0) + 16 +
+  const bool k16 = (FMT == kFmtVq16 || FMT == kFmtVq16Rvq);
+  const size_t smem = (!k16 ? 4096 * 16 : 0) + (FMT == kFmtRvq12_4 ? 256 : 0) + 16 +
                       (size_t)8 * NT * (kc + 8) * 2;
   auto kern = gemv_kernel<FMT, T, NT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -251,6 +269,7 @@ static cudaError_t launch_fmt(const LayerArgs& a, const Plan& p, float* scratch,
   switch (a.fmt) {
     case kFmtRvq12: return launch_nt<kFmtRvq12, T>(a, p, scratch, tickets, s);
     case kFmtRvq12_4: return launch_nt<kFmtRvq12_4, T>(a, p, scratch, tickets, s);
+    case kFmtVq16Rvq: return launch_nt<kFmtVq16Rvq, T>(a, p, scratch, tickets, s);
     default: return launch_nt<kFmtVq16, T>(a, p, scratch, tickets, s);
   }
 }

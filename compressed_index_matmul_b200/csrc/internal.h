@@ -17,14 +17,19 @@ struct LayerArgs {
   const uint8_t* lo;    // [N][G]
   const uint8_t* hi4;   // [N][G/2]
   const uint8_t* s2;    // [N][G/2]
-  const uint16_t* idx16;
-  const uint16_t* cb1;  // fp16 bits
+  const uint16_t* idx16;  // [n16][N][G] (one plane per 16-bit stage)
+  const uint8_t* idx8;    // [N][G] (the ladder's 8-bit stage)
+  const uint16_t* cb1;    // fp16 bits
   const uint16_t* cb2;
+  const uint16_t* cbr[3]; // the ladder's codebooks of 16-bit stages 2..n16
+  const uint16_t* cb8;    // the ladder's 8-bit codebook
   const uint16_t* scales;
   int M, N, K;
   int fmt;
   int scale_group;
-  int act;              // VQ_F16 / VQ_BF16
+  int act;                // VQ_F16 / VQ_BF16
+  int n16, n8;            // stages of the 16-bit formats (1, 0 for VQ_FMT_VQ16)
+  float mult[3];          // multipliers of residual stages 2..n16 + n8
 };
 
 // Work split chosen for one forward.
@@ -58,8 +63,8 @@ cudaError_t launch_gemv(const LayerArgs& a, const Plan& p, float* scratch, uint3
 // sizes other launches of the handle used).
 cudaError_t launch_lut(const LayerArgs& a, const Plan& p, float* scratch, uint32_t* gbar, uint32_t* err,
                        cudaStream_t s);
-// The batch-1 kernel of the 16-bit format (VQ_PATH_GATHER, clusters of 8 CTAs,
-// no scratch); `signs` (may be NULL) makes it rotate x itself
+// The few-token kernel of the 16-bit formats (VQ_PATH_GATHER, clusters of 2
+// CTAs, no scratch); `signs` (may be NULL, M == 1 only) makes it rotate x itself
 // (vq_linear_forward_rotated).
 cudaError_t launch_vq16(const LayerArgs& a, const Plan& p, const int8_t* signs, cudaStream_t s);
 cudaError_t launch_tc(const LayerArgs& a, const Plan& p, float* scratch, uint32_t* tickets, uint32_t* err_flag,

@@ -501,7 +501,7 @@ static LutGeom lut_geom(int N, int K, int num_sms) {
 }
 
 bool plan_lut(const vq_linear_desc& d, const DeviceInfo& dev, int M, Plan* p) {
-  if (M != 1 || d.fmt == VQ_FMT_VQ16 || d.K % (8 * kLutGroups) != 0 || d.N % 4 != 0 || dev.smem_optin < kLutSmem)
+  if (M != 1 || d.fmt == VQ_FMT_VQ16 || d.fmt == VQ_FMT_VQ16_RVQ || d.K % (8 * kLutGroups) != 0 || d.N % 4 != 0 || dev.smem_optin < kLutSmem)
     return false;
   const LutGeom g = lut_geom(d.N, d.K, dev.num_sms);
   p->path = VQ_PATH_LUT;

@@ -36,6 +36,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "ladder.cuh"
 #include "tc_ptx.cuh"
 
 namespace vq {
@@ -119,8 +120,11 @@ template <int FMT, typename T, bool kStaged>
 __global__ void __launch_bounds__(kTcThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap ymap, TcArgs p) {
   extern __shared__ unsigned char smem_raw[];
-  constexpr bool kSmemCb = (FMT != kFmtVq16);
+  constexpr bool k16 = (FMT == kFmtVq16 || FMT == kFmtVq16Rvq);
+  constexpr bool kLadder = (FMT == kFmtVq16Rvq);
+  constexpr bool kSmemCb = !k16;
   constexpr bool kTwo = (FMT == kFmtRvq12_4);
+  static_assert(!(kLadder && kStaged), "the residual ladder reads its indices directly");
   const LayerArgs& a = p.a;
   // 1024-byte aligned base (the swizzle pattern of the x tiles is taken from address bits).
   const uint32_t raw = smem_u32(smem_raw);
@@ -306,6 +310,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       uint2 lo8 = make_uint2(0, 0);
       uint32_t hi4w = 0, s24w = 0;
       uint4 v16 = make_uint4(0, 0, 0, 0);
+      LadderIdx res{};
       unsigned short sc = row_scale;
       if (valid) {
         if (kStaged) {
@@ -320,7 +325,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           if (block_scales) sc = *reinterpret_cast<const uint16_t*>(slot + kTcIdxSc + (dr * (w / 8) + h) * 2);
         } else {
           const int64_t e = (int64_t)16 * sl * N + (int64_t)r * w + 8 * h;
-          if (FMT == kFmtVq16) {
+          if constexpr (kLadder) load_ladder_block(a, e, res);
+          if (k16) {
             v16 = *reinterpret_cast<const uint4*>(a.idx16 + e);
           } else {
             lo8 = *reinterpret_cast<const uint2*>(a.lo + e);
@@ -334,23 +340,27 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(idx_empty(j % kTcIdxSlots));
       }
-      const float scf = kTwo ? __half2float(__ushort_as_half(sc)) : 0.f;
+      const float scf = (kTwo || kLadder) ? __half2float(__ushort_as_half(sc)) : 0.f;
       ptx::tc_fence_after();
 #pragma unroll
       for (int c = 0; c < 2; ++c) {  // 4 groups (16 TMEM columns) at a time
         uint32_t out[16];
         const uint32_t low = c ? lo8.y : lo8.x;
-        const uint32_t v0 = FMT == kFmtVq16 ? (c ? v16.z : v16.x) : 0u, v1 = FMT == kFmtVq16 ? (c ? v16.w : v16.y) : 0u;
+        const uint32_t v0 = k16 ? (c ? v16.z : v16.x) : 0u, v1 = k16 ? (c ? v16.w : v16.y) : 0u;
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
           const int g = 4 * c + t;
           uint32_t i1;
-          if (FMT == kFmtVq16)
+          if (k16)
             i1 = ((t < 2 ? v0 : v1) >> (16 * (t & 1))) & 0xFFFFu;
           else
             i1 = ((low >> (8 * t)) & 0xFFu) | (((hi4w >> (4 * g)) & 15u) << 8);
           const uint4 c1 = kSmemCb ? cb1s[i1] : __ldg(cbg + i1);
-          if (kTwo) {
+          if constexpr (kLadder) {
+            float v[8];
+            ladder_sum(a, res, g, c1, v);
+            pack_scaled<T>(v, scf, out + 4 * t);
+          } else if (kTwo) {
             const int i2 = (int)((s24w >> (4 * g)) & 15u);
             uint32_t c2[4];
 #pragma unroll
@@ -631,6 +641,9 @@ cudaError_t launch_tc(const LayerArgs& a, const Plan& pl, float* scratch, uint32
     case kFmtRvq12_4:
       return bf ? launch_tc_s<kFmtRvq12_4, __nv_bfloat16>(a, g, scratch, tickets, err, s)
                 : launch_tc_s<kFmtRvq12_4, __half>(a, g, scratch, tickets, err, s);
+    case kFmtVq16Rvq:  // the ladder's indices are read directly (no staging ring)
+      return bf ? launch_tc_t<kFmtVq16Rvq, __nv_bfloat16, false>(a, g, scratch, tickets, err, s)
+                : launch_tc_t<kFmtVq16Rvq, __half, false>(a, g, scratch, tickets, err, s);
     default:
       return bf ? launch_tc_s<kFmtVq16, __nv_bfloat16>(a, g, scratch, tickets, err, s)
                 : launch_tc_s<kFmtVq16, __half>(a, g, scratch, tickets, err, s);

@@ -1,4 +1,5 @@
-// Small-batch GEMV for the single-stage 16-bit format (1 <= M <= 8, VQ_FMT_VQ16,
+// Small-batch GEMV for the 16-bit formats (1 <= M <= 8, VQ_FMT_VQ16 and the residual
+// ladder VQ_FMT_VQ16_RVQ,
 // K % 128 == 0, K <= 16384, M K <= 32768, N % 4 == 0), with the input rotation
 // optionally applied inside the kernel at M == 1.
 //
@@ -93,7 +94,11 @@ struct V16Pos {
 };
 
 // MT: tokens rounded up to 1, 2, 4 or 8 (the x of tokens M .. MT-1 is zero).
-template <typename T, int MT>
+// kLadder: the residual ladder (GLQ README, "Bit widths"): after the primary stage,
+// each residual stage t of the position is gathered the same way (its 16 indices
+// loaded then, from plane t or the 8-bit plane) and its dot products are added as
+// mult_t * (x . c_t) before the block scales.
+template <typename T, int MT, bool kLadder>
 __global__ void __launch_bounds__(kV16Consumers, 1)
     vq16_gemv_kernel(LayerArgs a, const int8_t* __restrict__ signs, float xscale, int S, int blocks_per_cluster,
                      int rblk) {
@@ -168,6 +173,51 @@ __global__ void __launch_bounds__(kV16Consumers, 1)
           for (int m = 0; m < MT; ++m) {
             const float4* xv = reinterpret_cast<const float4*>(xsl + m * K + 8 * g);
             blk[m][g >> 3] = dot8(c[g], xv[0], xv[1], blk[m][g >> 3]);
+          }
+        }
+        if constexpr (kLadder) {
+          const int64_t e = (int64_t)16 * ((int64_t)(sa + p / nrows) * N + r0 + p % nrows);
+          const int64_t NG = (int64_t)N * (K / 8);
+          const int nst = a.n16 + a.n8;
+#pragma unroll 1
+          for (int t = 2; t <= nst; ++t) {
+            const bool is8 = t > a.n16;
+            const float mt = t == 2 ? a.mult[0] : (t == 3 ? a.mult[1] : a.mult[2]);
+            const uint4* cbt = reinterpret_cast<const uint4*>(
+                is8 ? a.cb8 : (t == 2 ? a.cbr[0] : (t == 3 ? a.cbr[1] : a.cbr[2])));
+            uint32_t jw[8];
+            if (is8) {  // 16 one-byte indices
+              const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.idx8 + e));
+              jw[0] = v.x; jw[1] = v.y; jw[2] = v.z; jw[3] = v.w;
+              jw[4] = jw[5] = jw[6] = jw[7] = 0u;
+            } else {
+              const uint4* src = reinterpret_cast<const uint4*>(a.idx16 + (int64_t)(t - 1) * NG + e);
+              const uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
+              jw[0] = v0.x; jw[1] = v0.y; jw[2] = v0.z; jw[3] = v0.w;
+              jw[4] = v1.x; jw[5] = v1.y; jw[6] = v1.z; jw[7] = v1.w;
+            }
+            uint4 cr[16];
+#pragma unroll
+            for (int g = 0; g < 16; ++g) {
+              const uint32_t i = is8 ? (jw[g >> 2] >> (8 * (g & 3))) & 0xFFu : (jw[g >> 1] >> (16 * (g & 1))) & 0xFFFFu;
+              cr[g] = __ldg(cbt + i);
+            }
+            float tb[MT][2];
+#pragma unroll
+            for (int m = 0; m < MT; ++m) tb[m][0] = tb[m][1] = 0.f;
+#pragma unroll
+            for (int g = 0; g < 16; ++g) {
+#pragma unroll
+              for (int m = 0; m < MT; ++m) {
+                const float4* xv = reinterpret_cast<const float4*>(xsl + m * K + 8 * g);
+                tb[m][g >> 3] = dot8(cr[g], xv[0], xv[1], tb[m][g >> 3]);
+              }
+            }
+#pragma unroll
+            for (int m = 0; m < MT; ++m) {
+              blk[m][0] = fmaf(mt, tb[m][0], blk[m][0]);
+              blk[m][1] = fmaf(mt, tb[m][1], blk[m][1]);
+            }
           }
         }
         const float2 sc = block_scales ? f16x2_to_f32x2(cur.sc) : make_float2(1.f, 1.f);
@@ -270,9 +320,9 @@ static int v16_max_clusters(int num_sms) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaFuncSetAttribute(vq16_gemv_kernel<__half, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+  if (cudaFuncSetAttribute(vq16_gemv_kernel<__half, 8, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
           cudaSuccess ||
-      cudaOccupancyMaxActiveClusters(&n, vq16_gemv_kernel<__half, 8>, &cfg) != cudaSuccess || n < 1) {
+      cudaOccupancyMaxActiveClusters(&n, vq16_gemv_kernel<__half, 8, false>, &cfg) != cudaSuccess || n < 1) {
     cudaGetLastError();
     n = num_sms / kV16Cluster;
   }
@@ -281,7 +331,7 @@ static int v16_max_clusters(int num_sms) {
 }
 
 bool plan_vq16(const vq_linear_desc& d, const DeviceInfo& dev, int M, Plan* p) {
-  if (M < 1 || M > kV16MaxM || d.fmt != VQ_FMT_VQ16 || d.K % 128 != 0 || d.K > kV16MaxK ||
+  if (M < 1 || M > kV16MaxM || (d.fmt != VQ_FMT_VQ16 && d.fmt != VQ_FMT_VQ16_RVQ) || d.K % 128 != 0 || d.K > kV16MaxK ||
       v16_mt(M) * d.K > kV16MaxMK || d.N % 4 != 0 || dev.smem_optin < v16_max_smem())
     return false;
   const V16Geom g = v16_geom(d.N, v16_max_clusters(dev.num_sms), d.K / 128, v16_mt(M));
@@ -295,10 +345,10 @@ bool plan_vq16(const vq_linear_desc& d, const DeviceInfo& dev, int M, Plan* p) {
   return true;
 }
 
-template <typename T, int MT>
+template <typename T, int MT, bool kLadder>
 static cudaError_t launch_vq16_t(const LayerArgs& a, int grid, const int8_t* signs, cudaStream_t s) {
   const int S = a.K / 128;
-  auto kern = vq16_gemv_kernel<T, MT>;
+  auto kern = vq16_gemv_kernel<T, MT, kLadder>;
   static std::atomic<uint64_t> opted{0};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -317,9 +367,9 @@ static cudaError_t launch_vq16_t(const LayerArgs& a, int grid, const int8_t* sig
   if (ncl < 1) ncl = 1;
   const V16Geom g = v16_geom(a.N, ncl, S, MT);
   const int smem = v16_smem(S, MT, g.rblk, a.K).bytes;
-  // Orthonormal factor of the rotation, rounded once from double precision.
-  // a power-of-two K takes its orthonormal factor at the store; otherwise each block
-  // was scaled in shared memory
+  // Orthonormal factor of the rotation, rounded once from double precision: a
+  // power-of-two K takes it at the store; otherwise each block was scaled in shared
+  // memory
   const bool pow2 = (a.K & (a.K - 1)) == 0;
   const float xscale = signs && pow2 ? (float)(1.0 / std::sqrt((double)a.K)) : 1.f;
   cudaLaunchConfig_t cfg = {};
@@ -339,19 +389,22 @@ static cudaError_t launch_vq16_t(const LayerArgs& a, int grid, const int8_t* sig
   return cudaLaunchKernelEx(&cfg, kern, a, signs, xscale, S, g.blocks_per_cluster, g.rblk);
 }
 
-template <typename T>
+template <typename T, bool kLadder>
 static cudaError_t launch_vq16_m(const LayerArgs& a, int grid, const int8_t* signs, cudaStream_t s) {
   switch (v16_mt(a.M)) {
-    case 1: return launch_vq16_t<T, 1>(a, grid, signs, s);
-    case 2: return launch_vq16_t<T, 2>(a, grid, nullptr, s);
-    case 4: return launch_vq16_t<T, 4>(a, grid, nullptr, s);
-    default: return launch_vq16_t<T, 8>(a, grid, nullptr, s);
+    case 1: return launch_vq16_t<T, 1, kLadder>(a, grid, signs, s);
+    case 2: return launch_vq16_t<T, 2, kLadder>(a, grid, nullptr, s);
+    case 4: return launch_vq16_t<T, 4, kLadder>(a, grid, nullptr, s);
+    default: return launch_vq16_t<T, 8, kLadder>(a, grid, nullptr, s);
   }
 }
 
 cudaError_t launch_vq16(const LayerArgs& a, const Plan& p, const int8_t* signs, cudaStream_t s) {
-  return a.act == VQ_BF16 ? launch_vq16_m<__nv_bfloat16>(a, p.grid, signs, s)
-                          : launch_vq16_m<__half>(a, p.grid, signs, s);
+  const bool lad = a.fmt == kFmtVq16Rvq;
+  if (a.act == VQ_BF16)
+    return lad ? launch_vq16_m<__nv_bfloat16, true>(a, p.grid, signs, s)
+               : launch_vq16_m<__nv_bfloat16, false>(a, p.grid, signs, s);
+  return lad ? launch_vq16_m<__half, true>(a, p.grid, signs, s) : launch_vq16_m<__half, false>(a, p.grid, signs, s);
 }
 
 }  // namespace vq

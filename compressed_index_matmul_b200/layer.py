@@ -20,8 +20,11 @@ class VQLinear:
     """Holds the planes, codebooks and scales of one layer in device memory.
 
     ``arrays`` is a dict with numpy arrays named as in include/vqlinear.h
-    (lo, hi4, s2, idx16, cb1, cb2, scales; fp16 as uint16 bits) and the layer shape
-    (N, K, fmt, scale_group).  ``forward(x)`` calls vq_linear_forward.
+    (lo, hi4, s2, idx16, idx8, cb1, cb2, cbr, cb8, scales; fp16 as uint16 bits) and the
+    layer shape (N, K, fmt, scale_group).  For the residual ladder (VQ_FMT_VQ16_RVQ)
+    idx16 holds one plane per 16-bit stage, cbr is [n16 - 1, 65536, 8] and ``mult``
+    the float32 multipliers of the residual stages; the stage counts follow from the
+    arrays.  ``forward(x)`` calls vq_linear_forward.
     """
 
     def __init__(self, N, K, fmt, scale_group, act_dtype, max_M, arrays: dict, device="cuda", rht=0):
@@ -30,11 +33,23 @@ class VQLinear:
         self.N, self.K, self.fmt, self.scale_group, self.act_dtype, self.max_M = N, K, fmt, scale_group, act_dtype, max_M
         self.device = torch.device(device)
         self.t = {k: _dev(v, self.device) for k, v in arrays.items() if v is not None and k in
-                  ("lo", "hi4", "s2", "idx16", "cb1", "cb2", "scales")}
-        self.planes = B.make_planes(self.t.get("lo"), self.t.get("hi4"), self.t.get("s2"), self.t.get("idx16"))
-        self.codebooks = B.make_codebooks(self.t["cb1"], self.t.get("cb2"))
+                  ("lo", "hi4", "s2", "idx16", "idx8", "cb1", "cb2", "cbr", "cb8", "scales")}
+        self.n16, self.n8, self.mult = 0, 0, ()
+        cbr = ()
+        if fmt == B.VQ_FMT_VQ16_RVQ:
+            ng = N * (K // 8)
+            self.n16 = int(np.asarray(arrays["idx16"]).size // ng)
+            self.n8 = 1 if arrays.get("idx8") is not None else 0
+            self.mult = tuple(float(m) for m in np.asarray(arrays["mult"], dtype=np.float32))
+            if "cbr" in self.t:
+                stride = 65536 * 8 * 2
+                cbr = tuple(self.t["cbr"].data_ptr() + i * stride for i in range(self.n16 - 1))
+        self.planes = B.make_planes(self.t.get("lo"), self.t.get("hi4"), self.t.get("s2"), self.t.get("idx16"),
+                                    self.t.get("idx8"))
+        self.codebooks = B.make_codebooks(self.t["cb1"], self.t.get("cb2"), cbr, self.t.get("cb8"))
         with torch.cuda.device(self.device):
-            self.handle = B.vq_linear_create(N, K, fmt, scale_group, act_dtype, max_M, rht)
+            self.handle = B.vq_linear_create(N, K, fmt, scale_group, act_dtype, max_M, rht, self.n16, self.n8,
+                                             self.mult)
 
     @property
     def torch_dtype(self):

@@ -12,6 +12,10 @@
  *   - GLQ README, "How it works" (E8 lattice codebooks): one 16-bit index per
  *     8-weight group into a 65,536-entry codebook; "Randomized Hadamard Transform":
  *     random sign flips followed by a fast Walsh-Hadamard transform.
+ *   - GLQ README, "Bit widths": the residual ladder -- a 16-bit primary stage,
+ *     16-bit residual stages, and for an odd bit width one final 8-bit stage
+ *     (3 bpw = 16 + 8, 4 = 16 + 16, ..., 8 = four 16-bit stages); "Direct kernel
+ *     access": each residual stage has its own codebook and inverse residual scale.
  *   - GLQ README, "Inference kernels": Y = X . dequant(W)^T computed against the
  *     compressed indices; partial sums reduced in a fixed order (no atomics), so
  *     results are bit-identical from run to run.
@@ -28,16 +32,30 @@
  *                          within a row's slice entries group 2t is in bits 0..3 of
  *                          byte t and group 2t+1 in bits 4..7
  *   s2    uint8  [N*G/2]   4-bit stage-2 index, packed like hi4 (VQ_FMT_RVQ12_4 only)
- *   idx16 uint16 [N*G]     16-bit index, one entry per group (VQ_FMT_VQ16 only)
+ *   idx16 uint16 [N*G]     16-bit index, one entry per group (VQ_FMT_VQ16); for
+ *                          VQ_FMT_VQ16_RVQ [n16][N*G], one such plane per 16-bit
+ *                          stage, stage after stage
+ *   idx8  uint8  [N*G]     8-bit stage index, one byte per group, laid out like lo
+ *                          (VQ_FMT_VQ16_RVQ with n8 == 1 only)
  *   scales fp16            scale_group == 64: one per 64 inputs, in the same
  *                          K-slice-major order (2 entries per row per full slice,
  *                          1 in a 64-wide last slice); scale_group == K: [N]
  *   cb1   fp16   [4096][8]  stage-1 codebook (or [65536][8] for VQ_FMT_VQ16)
  *   cb2   fp16   [16][8]    stage-2 codebook (VQ_FMT_RVQ12_4 only)
+ *   cbr[t] fp16  [65536][8] codebook of 16-bit stage t+2 (VQ_FMT_VQ16_RVQ; may be
+ *                          cb1 or each other); cb8 fp16 [256][8] the 8-bit stage's
+ *                          codebook (n8 == 1)
  *   x     fp16 or bf16 [M][K] row-major;   y  same dtype [M][N] row-major
  * Weight (n, k) with g = k/8, j = k%8 decodes to
  *   scale(n, k) * (cb1[i1(n,g)][j] + cb2[i2(n,g)][j]),
  * with i1 = lo byte | hi nibble << 8 and i2 the s2 nibble (or i1 = idx16 entry).
+ * VQ_FMT_VQ16_RVQ decodes to
+ *   scale(n, k) * (cb1[i_1][j] + sum_{t=2..n16} mult[t-2] * cbr[t-2][i_t][j]
+ *                  + [n8 == 1] mult[n16-1] * cb8[i_8][j])
+ * with i_t the entry of 16-bit plane t and i_8 that of the 8-bit plane.  Paths
+ * that materialise weights (VQ_PATH_GEMV, VQ_PATH_TC, vq_debug_dequant) form the
+ * stage sum in fp32 with one fused multiply-add per residual stage, in stage
+ * order, then round scale * sum to fp32 and to the activation type.
  *
  * Conventions shared by every entry point:
  *   - Errors: every call returns a vq_status.  Argument problems are detected on
@@ -79,14 +97,17 @@ typedef enum {
 enum {
   VQ_FMT_RVQ12 = 1,   /* one 12-bit stage: lo + hi4 planes, 4096 x 8 codebook */
   VQ_FMT_RVQ12_4 = 2, /* 12-bit stage 1 + 4-bit stage 2: lo + hi4 + s2, cb1 + cb2 */
-  VQ_FMT_VQ16 = 3     /* one 16-bit stage: idx16 plane, 65,536 x 8 codebook */
+  VQ_FMT_VQ16 = 3,    /* one 16-bit stage: idx16 plane, 65,536 x 8 codebook */
+  VQ_FMT_VQ16_RVQ = 4 /* residual ladder: n16 16-bit stages (idx16 planes, cb1 and
+                         cbr codebooks), then n8 8-bit stages (idx8, cb8), each
+                         residual stage weighted by its mult (desc) */
 };
 
 /* Element types of x / y / materialised weights. */
 enum { VQ_F16 = 0, VQ_BF16 = 1 };
 
 /* Kernel choice for vq_linear_set_path.  VQ_PATH_AUTO picks by format, M and layer
- * size: VQ_FMT_VQ16 with M <= 4 -> VQ_PATH_GATHER where it applies (K % 128 == 0,
+ * size: VQ_FMT_VQ16 / VQ_FMT_VQ16_RVQ with M <= 4 -> VQ_PATH_GATHER where it applies (K % 128 == 0,
  * K <= 16384, M' K <= 32768 with M' = M rounded up to 1, 2, 4 or 8, N % 4 == 0);
  * otherwise M == 1 -> VQ_PATH_LUT where it applies (12-bit formats, K % 128 == 0,
  * N % 4 == 0), else VQ_PATH_GEMV; 2 <= M <= 16 -> VQ_PATH_TC for layers of at least
@@ -96,7 +117,7 @@ enum {
   VQ_PATH_LUT = 1,    /* M == 1 only: per-group x.codebook tables in shared memory */
   VQ_PATH_GEMV = 2,   /* 1 <= M <= 16: decode to registers, warp MMA, split-K */
   VQ_PATH_TC = 3,     /* any M: decode into tensor memory, tcgen05 MMA (fp32 in TMEM) */
-  VQ_PATH_GATHER = 4  /* 1 <= M <= 8, VQ_FMT_VQ16 only: codewords gathered from L2
+  VQ_PATH_GATHER = 4  /* 1 <= M <= 8, 16-bit formats only: codewords gathered from L2
                          into fp32 dot products; at M == 1 it can apply the input
                          rotation itself */
 };
@@ -113,18 +134,29 @@ typedef struct {
                           vq_linear_forward, or calls vq_linear_forward_rotated
                           (create then also allocates a max_M x K rotation buffer
                           for the shapes whose rotation is not fused) */
+  int32_t n16;         /* VQ_FMT_VQ16_RVQ: 16-bit stages including the primary, 1..4 */
+  int32_t n8;          /* VQ_FMT_VQ16_RVQ: 8-bit stages after them, 0 or 1; n16 + n8 <= 4
+                          (bits per weight 2 n16 + n8).  Both ignored for other formats */
+  float mult[3];       /* VQ_FMT_VQ16_RVQ: multiplier of residual stage 2, 3, 4 (the
+                          inverse residual scales; the 16-bit stages first, the 8-bit
+                          one last); finite; entries past n16 + n8 - 1 are ignored */
 } vq_linear_desc;
 
 typedef struct {
   const uint8_t* lo;     /* N*K/8 bytes, K-slice-major (RVQ12, RVQ12_4), else NULL */
   const uint8_t* hi4;    /* N*K/16 bytes, K-slice-major (RVQ12, RVQ12_4), else NULL */
   const uint8_t* s2;     /* N*K/16 bytes, K-slice-major (RVQ12_4), else NULL */
-  const uint16_t* idx16; /* N*K/8 entries, K-slice-major (VQ16), else NULL */
+  const uint16_t* idx16; /* N*K/8 entries, K-slice-major (VQ16); n16*N*K/8 entries,
+                            stage-major (VQ16_RVQ); else NULL */
+  const uint8_t* idx8;   /* N*K/8 bytes, K-slice-major (VQ16_RVQ with n8 == 1), else NULL */
 } vq_planes;
 
 typedef struct {
   const void* cb1; /* fp16 [4096][8], or [65536][8] for VQ_FMT_VQ16 */
   const void* cb2; /* fp16 [16][8] for VQ_FMT_RVQ12_4, else NULL */
+  const void* cbr[3]; /* VQ_FMT_VQ16_RVQ: fp16 [65536][8] codebooks of 16-bit stages 2..n16
+                         (entries past n16 - 1 ignored), else ignored */
+  const void* cb8;    /* VQ_FMT_VQ16_RVQ with n8 == 1: fp16 [256][8], else ignored */
 } vq_codebooks;
 
 typedef struct vq_linear_s* vq_linear_t;

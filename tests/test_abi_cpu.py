@@ -34,7 +34,7 @@ def test_header_declares_the_binding_exports():
 def test_library_exports_every_declared_symbol(lib):
     for name in declared_functions():
         assert hasattr(lib, name), name
-    assert lib.vq_abi_version() == 1
+    assert lib.vq_abi_version() == 2
 
 
 def test_no_symbols_beyond_the_abi(lib):
@@ -62,12 +62,34 @@ def _create(**kw):
     (dict(scale_group=128), B.VQ_ERR_UNSUPPORTED),
     (dict(act_dtype=5), B.VQ_ERR_INVALID_ARG),
     (dict(max_M=0), B.VQ_ERR_INVALID_ARG),
+    # residual ladder: stage counts and multipliers
+    (dict(fmt=B.VQ_FMT_VQ16_RVQ, n16=0, n8=0), B.VQ_ERR_INVALID_ARG),
+    (dict(fmt=B.VQ_FMT_VQ16_RVQ, n16=5, n8=0), B.VQ_ERR_INVALID_ARG),
+    (dict(fmt=B.VQ_FMT_VQ16_RVQ, n16=2, n8=2), B.VQ_ERR_INVALID_ARG),
+    (dict(fmt=B.VQ_FMT_VQ16_RVQ, n16=4, n8=1), B.VQ_ERR_INVALID_ARG),  # 9 bpw: not in the table
+    (dict(fmt=B.VQ_FMT_VQ16_RVQ, n16=2, n8=1, mult=(0.1, float("nan"))), B.VQ_ERR_INVALID_ARG),
+    (dict(fmt=B.VQ_FMT_VQ16_RVQ, n16=3, n8=0, mult=(float("inf"), 0.1)), B.VQ_ERR_INVALID_ARG),
 ])
 def test_create_rejects_bad_descriptors(lib, kw, status):
     with pytest.raises(B.VQError) as ei:
         _create(**kw)
     assert ei.value.status == status
     assert lib.vq_last_error()
+
+
+def test_ladder_struct_layout_matches_the_header():
+    """The ctypes mirrors of the three ABI structs have the C layout: the ladder fields
+    follow the original ones."""
+    assert ctypes.sizeof(B.vq_linear_desc) == 7 * 4 + 2 * 4 + 3 * 4
+    assert B.vq_linear_desc.n16.offset == 28 and B.vq_linear_desc.mult.offset == 36
+    assert ctypes.sizeof(B.vq_planes) == 5 * 8 and B.vq_planes.idx8.offset == 32
+    assert ctypes.sizeof(B.vq_codebooks) == 6 * 8 and B.vq_codebooks.cb8.offset == 40
+
+
+def test_ladder_stage_table():
+    """GLQ README, "Bit widths": bits per weight = 2 n16 + n8, at most four stages."""
+    for bpw, (n16, n8) in B.LADDER_STAGES.items():
+        assert 2 * n16 + n8 == bpw and n16 + n8 <= 4 and n8 <= 1
 
 
 def test_null_arguments_are_rejected(lib):
