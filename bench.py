@@ -44,7 +44,8 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from synth import CONFIGS, DT_BF16, DT_F16, FMT_VQ16, make_layer, make_signs, make_x  # noqa: E402
+from synth import (CONFIGS, DT_BF16, DT_F16, FMT_VQ16, FMT_VQ16_RVQ, LayerSpec, make_layer, make_signs,  # noqa: E402
+                   make_x)
 
 METRIC = "vq_linear µs/layer & achieved HBM GB/s (% of roofline) at batch 1/16; TFLOP/s at M=256"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -56,6 +57,20 @@ WORKLOADS = {
     "prefill-8192": dict(cfg=5, layers=1),
     "single-256": dict(cfg=1, layers=1),
 }
+# The residual bit-width ladder (GLQ README, "Bit widths": 3 bpw = 16 + 8, 4 = 16 + 16,
+# 5 = 16 + 16 + 8) on a 4096 x 4096 layer with one scale per row, like the 16-bit
+# workload; seeded with its own id.
+for _bpw in (3, 4, 5):
+    WORKLOADS[f"vq16-ladder-4096-{_bpw}bpw"] = dict(
+        cfg=100 + _bpw, layers=1,
+        config=dict(name=f"vq16-ladder-4096x4096-{_bpw}bpw", layers=1, act=DT_F16, Ms=(1, 8), rht=False,
+                    tensors=[("w", LayerSpec(4096, 4096, FMT_VQ16_RVQ, 4096, bpw=_bpw))]))
+_16BIT = (FMT_VQ16, FMT_VQ16_RVQ)
+
+
+def _workload_config(name):
+    w = WORKLOADS[name]
+    return w["config"] if "config" in w else CONFIGS[w["cfg"]]
 
 
 def load_peaks():
@@ -72,6 +87,9 @@ def layer_bytes(spec, M, act_bytes=2):
     G = spec.K // 8
     if spec.fmt == FMT_VQ16:
         planes, cb = spec.N * G * 2, 65536 * 16
+    elif spec.fmt == FMT_VQ16_RVQ:  # one 16-bit plane and codebook per 16-bit stage, the 8-bit ones
+        n16, n8 = spec.bpw // 2, spec.bpw % 2
+        planes, cb = spec.N * G * (2 * n16 + n8), 65536 * 16 * n16 + 256 * 16 * n8
     else:
         planes = spec.N * G + spec.N * G // 2 + (spec.N * G // 2 if spec.fmt == 2 else 0)
         cb = 4096 * 16 + (256 if spec.fmt == 2 else 0)
@@ -147,7 +165,7 @@ class Workload:
 
         self.name = name
         w = WORKLOADS[name]
-        self.cfg = CONFIGS[w["cfg"]]
+        self.cfg = w["config"] if "config" in w else CONFIGS[w["cfg"]]
         self.act = self.cfg["act"]
         self.tdtype = torch.bfloat16 if self.act == DT_BF16 else torch.float16
         self.max_M = max_M
@@ -254,7 +272,7 @@ class Workload:
 
     def rotation_fused(self, spec, M):
         """True where vq_linear_forward_rotated is one kernel (the batch-1 gather kernel)."""
-        return M == 1 and spec.fmt == FMT_VQ16 and spec.K % 128 == 0 and spec.K <= 16384 and spec.N % 4 == 0
+        return M == 1 and spec.fmt in _16BIT and spec.K % 128 == 0 and spec.K <= 16384 and spec.N % 4 == 0
 
     def launches_per_step(self, M):
         n = 0
@@ -278,13 +296,14 @@ def _clone_layer(L):
     from compressed_index_matmul_b200 import _binding as B
 
     c = copy.copy(L)
-    # The 65,536-entry codebook of the 16-bit format is one table shared by every
-    # copy: GLQ's lattice codebook is shared by all layers and served from L2.  The
-    # index planes, scales and 4096-entry codebooks are copied.
-    shared = ("cb1",) if L.fmt == FMT_VQ16 else ()
+    # The 65,536-entry codebooks of the 16-bit formats are tables shared by every
+    # copy: GLQ's lattice codebook is shared by all layers and served from L2 (the
+    # ladder's residual and 8-bit codebooks likewise).  The index planes, scales and
+    # 4096-entry codebooks are copied.
+    shared = ("cb1", "cbr", "cb8") if L.fmt in _16BIT else ()
     c.t = {k: (v if k in shared else v.clone()) for k, v in L.t.items()}
-    c.planes = B.make_planes(c.t.get("lo"), c.t.get("hi4"), c.t.get("s2"), c.t.get("idx16"))
-    c.codebooks = B.make_codebooks(c.t["cb1"], c.t.get("cb2"))
+    c.planes = B.make_planes(c.t.get("lo"), c.t.get("hi4"), c.t.get("s2"), c.t.get("idx16"), c.t.get("idx8"))
+    c.codebooks = L.codebooks if L.fmt in _16BIT else B.make_codebooks(c.t["cb1"], c.t.get("cb2"))
     c.close = lambda: None  # the handle belongs to L
     return c
 
@@ -486,7 +505,7 @@ def gpu_arm(args):
     per_fwd_eff = [fwd_ms] * len(wl.layers) if uniform else list(per_fwd)
     achieved = sum(bytes_per_fwd) / (sum(per_fwd_eff) * 1e-3) / 1e9
     fmt0 = wl.layers[0][1].fmt
-    dominant = ("lut_gemv_kernel" if M == 1 and fmt0 != FMT_VQ16 else
+    dominant = ("lut_gemv_kernel" if M == 1 and fmt0 not in _16BIT else
                 "vq16_gemv_kernel" if M == 1 else "gemv_kernel" if M <= 16 else "tc_gemm_kernel")
     traffic = lookup_traffic(dominant, args.workload, M)
     avg_launch_us = round(1e3 * float(np.mean(per_fwd_eff)), 3)
@@ -536,7 +555,7 @@ def gpu_arm(args):
                    "parallelism": f"replicas x{world}",
                    "l2": L2_NOTE.format(r=R, mb=R * wl.weight_bytes() / 1e6) + (
                        "; the 65,536-entry codebook is one table shared by the copies (L2-resident)"
-                       if fmt0 == FMT_VQ16 else ""),
+                       if fmt0 in _16BIT else ""),
                    "layer": ("MLP step / 3 weight matrices: gate and up (same x) run concurrently on two "
                              "streams, half of the SMs each (vq_linear_set_sm_budget), then down"
                              if wl.concurrent_gate_up else "one vq_linear_forward (one weight matrix)"),
@@ -627,6 +646,14 @@ def detail(args, peaks, main_wl):
         res["prefill-8192 M=256"] = {"error": str(exc)[:300]}
     for M in (1, 8):
         res[f"rotation 4096 M={M}"] = time_rotations(4096, M, steps)
+    for bpw in (3, 4, 5):  # the residual ladder
+        name = f"vq16-ladder-4096-{bpw}bpw"
+        if name == args.workload:
+            continue
+        wl = Workload(name, max_M=8)
+        for M in (1, 8):
+            res[f"{name} M={M}"] = measure(wl, M, steps, 3, peaks)
+        del wl
     for v in res.values():
         for k in list(v):
             if isinstance(v[k], float):
@@ -697,7 +724,7 @@ def cpu_baseline(workload, M, budget_s=15.0, threads=None):
     orc.build()
     threads = threads or _host_cores()
     w = WORKLOADS[workload]
-    cfg = CONFIGS[w["cfg"]]
+    cfg = w["config"] if "config" in w else CONFIGS[w["cfg"]]
     tensors = cfg["tensors"]
     x_cache = {}
     per_layer_s = []
@@ -740,8 +767,7 @@ def reference_arm(args):
             per_step.append(cb["value"])
     v = float(np.mean(per_step))
     out = {"metric": METRIC, "value": round(v, 1), "unit": "us/layer", "n_gpus": world, "steps": args.steps,
-           "warmup": args.warmup, "ms_per_step": round(v * 1e-3 * len(CONFIGS[WORKLOADS[args.workload]["cfg"]]
-                                                                      ["tensors"]), 3),
+           "warmup": args.warmup, "ms_per_step": round(v * 1e-3 * len(_workload_config(args.workload)["tensors"]), 3),
            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
            "data": "synthetic (seeded)", "impl": "reference",
            "config": {"workload": args.workload, "M": args.batch, "layer": "one weight matrix"},
