@@ -121,7 +121,15 @@ __device__ __forceinline__ void hadamard_to_smem(const uint16_t* x, const int8_t
 // and signs into its slice of xs.  With scale_blocks each block is multiplied in
 // place by its orthonormal factor 1/sqrt(b) (where K is not a power of two no single
 // factor applies to the whole vector); otherwise the caller applies 1/sqrt(K).
-__device__ __forceinline__ float block_scale(int b) { return (float)(1.0 / sqrt((double)b)); }
+// fl32(1/sqrt(b)) for b = 2^p, built exactly in single precision: 2^-(p/2) for even p,
+// 2^-((p-1)/2) times fl32(1/sqrt(2)) = 0x3F3504F3 for odd p (a power-of-two scaling, so
+// the product is the correctly rounded value), the same bits as rounding the
+// double-precision quotient.
+__device__ __forceinline__ float block_scale(int b) {
+  const int p = 31 - __clz(b);
+  const float base = __int_as_float((127 - (p >> 1)) << 23);
+  return (p & 1) ? base * __int_as_float(0x3F3504F3) : base;
+}
 
 template <typename T, int NT, int kMaxK, bool kSignsFirst = true>
 __device__ __forceinline__ void hadamard_blocks_to_smem(const uint16_t* x, const int8_t* signs, float* xs, int K,

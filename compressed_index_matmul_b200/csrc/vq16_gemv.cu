@@ -87,6 +87,21 @@ __device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
   return v;
 }
 
+// The 16 indices of residual stage t of the ladder at plane entry e (a multiple of
+// 16): two 16-byte loads from 16-bit plane t, or one from the 8-bit plane.
+__device__ __forceinline__ void load_ladder_stage(const LayerArgs& a, int t, int64_t e, int64_t NG, uint32_t (&w)[8]) {
+  if (t > a.n16) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.idx8 + e));
+    w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+    w[4] = w[5] = w[6] = w[7] = 0u;
+  } else {
+    const uint4* src = reinterpret_cast<const uint4*>(a.idx16 + (int64_t)(t - 1) * NG + e);
+    const uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
+    w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w;
+    w[4] = v1.x; w[5] = v1.y; w[6] = v1.z; w[7] = v1.w;
+  }
+}
+
 // Index words (16 x uint16) and block scales of one (slice, row) position.
 struct V16Pos {
   uint4 i0, i1;
@@ -159,6 +174,15 @@ __global__ void __launch_bounds__(kV16Consumers, 1)
         if (pn < ns * nrn) load_pos(pn, r0n, nrn, nxt);
       }
       if (p < npos) {
+        // the ladder's next residual stage's indices are always loaded one stage ahead,
+        // so their latency overlaps the current stage's gathers
+        uint32_t nw[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+        int64_t e_pos = 0, NG = 0;
+        if constexpr (kLadder) {
+          e_pos = (int64_t)16 * ((int64_t)(sa + p / nrows) * N + r0 + p % nrows);
+          NG = (int64_t)N * (K / 8);
+          if (a.n16 + a.n8 >= 2) load_ladder_stage(a, 2, e_pos, NG, nw);
+        }
         const uint32_t iw[8] = {cur.i0.x, cur.i0.y, cur.i0.z, cur.i0.w, cur.i1.x, cur.i1.y, cur.i1.z, cur.i1.w};
         uint4 c[16];
 #pragma unroll
@@ -176,8 +200,6 @@ __global__ void __launch_bounds__(kV16Consumers, 1)
           }
         }
         if constexpr (kLadder) {
-          const int64_t e = (int64_t)16 * ((int64_t)(sa + p / nrows) * N + r0 + p % nrows);
-          const int64_t NG = (int64_t)N * (K / 8);
           const int nst = a.n16 + a.n8;
 #pragma unroll 1
           for (int t = 2; t <= nst; ++t) {
@@ -186,16 +208,9 @@ __global__ void __launch_bounds__(kV16Consumers, 1)
             const uint4* cbt = reinterpret_cast<const uint4*>(
                 is8 ? a.cb8 : (t == 2 ? a.cbr[0] : (t == 3 ? a.cbr[1] : a.cbr[2])));
             uint32_t jw[8];
-            if (is8) {  // 16 one-byte indices
-              const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.idx8 + e));
-              jw[0] = v.x; jw[1] = v.y; jw[2] = v.z; jw[3] = v.w;
-              jw[4] = jw[5] = jw[6] = jw[7] = 0u;
-            } else {
-              const uint4* src = reinterpret_cast<const uint4*>(a.idx16 + (int64_t)(t - 1) * NG + e);
-              const uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
-              jw[0] = v0.x; jw[1] = v0.y; jw[2] = v0.z; jw[3] = v0.w;
-              jw[4] = v1.x; jw[5] = v1.y; jw[6] = v1.z; jw[7] = v1.w;
-            }
+#pragma unroll
+            for (int q = 0; q < 8; ++q) jw[q] = nw[q];
+            if (t < nst) load_ladder_stage(a, t + 1, e_pos, NG, nw);
             uint4 cr[16];
 #pragma unroll
             for (int g = 0; g < 16; ++g) {
