@@ -599,6 +599,10 @@ def aggregate_over_ranks(total_ms_local: float, steps: int, layers_per_step: int
     return ms_per_step, 1e3 * ms_per_step / (layers_per_step * world)
 
 
+KERNEL_UNITS = {"lut_gemv_kernel": "lut_gemv.cu", "vq16_gemv_kernel": "vq16_gemv.cu", "tc_gemm_kernel": "tc_gemm.cu",
+                "gemv_kernel": "gemv.cu"}
+
+
 def lookup_traffic(kernel, workload, M):
     """DRAM bytes per launch from a committed ncu capture, if it matches the current kernel source."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
@@ -614,7 +618,8 @@ def lookup_traffic(kernel, workload, M):
         return None
     from compressed_index_matmul_b200.build import source_digest
 
-    if e.get("source_digest") != source_digest():
+    # the digest of the kernel's own translation unit, every header and the flags
+    if e.get("source_digest") != source_digest(KERNEL_UNITS.get(kernel)):
         return None
     return e.get("dram_bytes_per_launch")
 

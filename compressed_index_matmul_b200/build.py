@@ -40,9 +40,10 @@ def _sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
-def _deps_hash() -> str:
+def _deps_hash(unit: str | None = None) -> str:
     h = hashlib.sha256()
-    files = _sources() + sorted(glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h")))
+    units = _sources() if unit is None else [os.path.join(CSRC, unit)]
+    files = units + sorted(glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h")))
     files.append(os.path.join(INCLUDE, "vqlinear.h"))
     for f in files:
         h.update(f.encode())
@@ -52,9 +53,11 @@ def _deps_hash() -> str:
     return h.hexdigest()
 
 
-def source_digest() -> str:
-    """Hash of every kernel/ABI source and the compile flags (identifies a build of the kernels)."""
-    return _deps_hash()[:16]
+def source_digest(unit: str | None = None) -> str:
+    """Hash of every kernel/ABI source and the compile flags (identifies a build of the kernels);
+    with `unit` (a file name under csrc/), of that translation unit, every header and the flags
+    (identifies a build of the kernels defined in it)."""
+    return _deps_hash(unit)[:16]
 
 
 def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) -> str:

@@ -59,6 +59,13 @@ __global__ void __launch_bounds__(kRhtThreads) rht_kernel(const uint16_t* __rest
   const int64_t row = blockIdx.x;
   const uint16_t* xrow = x + row * K;
   uint16_t* orow = xo + row * K;
+  if ((K & (K - 1)) == 0) {  // one block: the whole row, with no offsets
+    hadamard_to_smem<T, kRhtThreads, 32768, !kOutput>(xrow, signs, buf, K, threadIdx.x);
+    const float scale = block_scale(K);
+    for (int i = threadIdx.x; i < K; i += kRhtThreads)
+      orow[i] = Elt<T>::from_f32(kOutput ? buf[i] * scale * (float)signs[i] : buf[i] * scale);
+    return;
+  }
   for (int o = 0, rest = K; rest > 0;) {
     const int b = 1 << (31 - __clz(rest));  // the largest power of two left
     hadamard_to_smem<T, kRhtThreads, 32768, !kOutput>(xrow + o, signs + o, buf + o, b, threadIdx.x);
