@@ -41,5 +41,6 @@ from ._binding import (  # noqa: F401
     vq_linear_set_sm_budget,
     vq_rht_apply,
     vq_rht_apply_output,
+    vq_rht_apply_output_sharded,
 )
 from .layer import VQLinear  # noqa: F401

@@ -435,6 +435,36 @@ VQ_API vq_status vq_rht_apply_output(const void* y, void* y_out, const int8_t* s
   return VQ_OK;
 }
 
+VQ_API vq_status vq_rht_apply_output_sharded(const void* y, void* y_out, const int8_t* signs, int32_t M, int32_t N,
+                                             const int32_t* shard_n, int32_t nshards, int32_t dtype, void* stream) {
+  if (shard_n == nullptr) return fail(VQ_ERR_INVALID_ARG, "shard_n is NULL");
+  if (nshards < 1 || nshards > vq::kRhtMaxShards)
+    return fail(VQ_ERR_INVALID_ARG, "nshards=%d outside [1, %d]", nshards, vq::kRhtMaxShards);
+  vq::RhtShards sh{};
+  sh.n = nshards;
+  int64_t total = 0;
+  for (int i = 0; i < nshards; ++i) {
+    const int w = shard_n[i];
+    if (w < 64 || w > 32768 || w % 64 != 0)
+      return fail(VQ_ERR_INVALID_ARG, "shard_n[%d]=%d must be a multiple of 64 in [64, 32768]", i, w);
+    sh.off[i] = (int)total;
+    total += w;
+  }
+  if (total != N) return fail(VQ_ERR_INVALID_ARG, "the shards add up to %lld columns, N=%d", (long long)total, N);
+  sh.off[nshards] = N;
+  if (M < 0) return fail(VQ_ERR_INVALID_ARG, "M=%d is negative", M);
+  if (dtype != VQ_F16 && dtype != VQ_BF16) return fail(VQ_ERR_INVALID_ARG, "dtype=%d", dtype);
+  vq_status st;
+  if ((st = check_ptr(y, "y")) || (st = check_ptr(y_out, "y_out")) || (st = check_ptr(signs, "signs"))) return st;
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(y), b0 = reinterpret_cast<uintptr_t>(y_out);
+  const uintptr_t bytes = (uintptr_t)M * N * 2;
+  if (a0 != b0 && a0 < b0 + bytes && b0 < a0 + bytes) return fail(VQ_ERR_INVALID_ARG, "y_out partially overlaps y");
+  if (M == 0) return VQ_OK;
+  cudaError_t e = vq::launch_rht_output_shards(y, y_out, signs, M, N, sh, dtype, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "vq_rht_apply_output_sharded launch");
+  return VQ_OK;
+}
+
 VQ_API vq_status vq_linear_check(vq_linear_t h, void* stream) {
   if (h == nullptr) return fail(VQ_ERR_INVALID_ARG, "handle is NULL");
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));

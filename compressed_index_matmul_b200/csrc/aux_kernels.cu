@@ -51,14 +51,11 @@ constexpr int kRhtThreads = 512;
 
 // kOutput: the output-side rotation signs / sqrt(b) * H_b x (GLQ README, "Bit
 // widths": the fused linear ends with an output RHT), the transpose of the input
-// rotation: the transform first, the signs at the store.
+// rotation: the transform first, the signs at the store.  One row of K elements by
+// the whole CTA (buf: K floats of shared memory).
 template <typename T, bool kOutput>
-__global__ void __launch_bounds__(kRhtThreads) rht_kernel(const uint16_t* __restrict__ x, uint16_t* __restrict__ xo,
-                                                          const int8_t* __restrict__ signs, int K) {
-  extern __shared__ float buf[];
-  const int64_t row = blockIdx.x;
-  const uint16_t* xrow = x + row * K;
-  uint16_t* orow = xo + row * K;
+__device__ __forceinline__ void rotate_row(const uint16_t* __restrict__ xrow, uint16_t* __restrict__ orow,
+                                           const int8_t* __restrict__ signs, int K, float* buf) {
   if ((K & (K - 1)) == 0) {  // one block: the whole row, with no offsets
     hadamard_to_smem<T, kRhtThreads, 32768, !kOutput>(xrow, signs, buf, K, threadIdx.x);
     const float scale = block_scale(K);
@@ -78,12 +75,54 @@ __global__ void __launch_bounds__(kRhtThreads) rht_kernel(const uint16_t* __rest
 }
 
 template <typename T, bool kOutput>
+__global__ void __launch_bounds__(kRhtThreads) rht_kernel(const uint16_t* __restrict__ x, uint16_t* __restrict__ xo,
+                                                          const int8_t* __restrict__ signs, int K) {
+  extern __shared__ float buf[];
+  const int64_t row = blockIdx.x;
+  rotate_row<T, kOutput>(x + row * K, xo + row * K, signs, K, buf);
+}
+
+// Shard-batched output rotation (GLQ README, "Inference kernels": per-shard output
+// transforms of a fused QKV / gate-up projection in one launch over grid.y): CTA
+// (row, shard) applies the output rotation to columns [off[s], off[s+1]) of row `row`
+// of y [M][N], with signs[off[s] ..].
+template <typename T>
+__global__ void __launch_bounds__(kRhtThreads) rht_shard_kernel(const uint16_t* __restrict__ y,
+                                                                uint16_t* __restrict__ yo,
+                                                                const int8_t* __restrict__ signs, int N,
+                                                                RhtShards sh) {
+  extern __shared__ float buf[];
+  const int64_t row = blockIdx.x;
+  const int s = blockIdx.y;
+  const int o = sh.off[s], w = sh.off[s + 1] - sh.off[s];
+  rotate_row<T, true>(y + row * N + o, yo + row * N + o, signs + o, w, buf);
+}
+
+template <typename T, bool kOutput>
 static cudaError_t launch_rht_t(const void* x, void* x_out, const int8_t* signs, int M, int K, cudaStream_t s) {
   const size_t smem = (size_t)K * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(rht_kernel<T, kOutput>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   rht_kernel<T, kOutput><<<M, kRhtThreads, smem, s>>>((const uint16_t*)x, (uint16_t*)x_out, signs, K);
   return cudaGetLastError();
+}
+
+template <typename T>
+static cudaError_t launch_rht_shards_t(const void* y, void* y_out, const int8_t* signs, int M, int N,
+                                       const RhtShards& sh, cudaStream_t s) {
+  int wmax = 0;
+  for (int i = 0; i < sh.n; ++i) wmax = sh.off[i + 1] - sh.off[i] > wmax ? sh.off[i + 1] - sh.off[i] : wmax;
+  const size_t smem = (size_t)wmax * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(rht_shard_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  rht_shard_kernel<T><<<dim3(M, sh.n), kRhtThreads, smem, s>>>((const uint16_t*)y, (uint16_t*)y_out, signs, N, sh);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rht_output_shards(const void* y, void* y_out, const int8_t* signs, int M, int N,
+                                     const RhtShards& sh, int dtype, cudaStream_t s) {
+  return dtype == VQ_BF16 ? launch_rht_shards_t<__nv_bfloat16>(y, y_out, signs, M, N, sh, s)
+                          : launch_rht_shards_t<__half>(y, y_out, signs, M, N, sh, s);
 }
 
 cudaError_t launch_rht(const void* x, void* x_out, const int8_t* signs, int M, int K, int dtype, cudaStream_t s) {

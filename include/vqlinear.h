@@ -295,6 +295,20 @@ vq_status vq_rht_apply(const void* x, void* x_out, const int8_t* signs, int32_t 
 vq_status vq_rht_apply_output(const void* y, void* y_out, const int8_t* signs, int32_t M, int32_t N,
                               int32_t dtype, void* stream);
 
+/* Shard-batched output rotation (GLQ README, "Inference kernels": per-shard output
+ * transforms of a fused QKV or gate-up projection in one launch).  y is [M][N] whose
+ * columns are nshards shards laid side by side: shard s has shard_n[s] columns and
+ * starts at column o_s = shard_n[0] + ... + shard_n[s-1]; the shard sizes add up to N.
+ * Every shard of every row gets vq_rht_apply_output's rotation (block-diagonal for a
+ * size that is not a power of two) with its own signs, signs[o_s .. o_s + shard_n[s]),
+ * exactly as separate vq_rht_apply_output calls on the shards would give them.
+ * shard_n is a HOST array of nshards values, each a multiple of 64 in [64, 32768];
+ * 1 <= nshards <= 16.  signs is a device int8 array of +1/-1 [N], 16-byte aligned;
+ * dtype is VQ_F16 or VQ_BF16 for both y and y_out; y_out may be y (in place), partial
+ * overlap is invalid.  One kernel launch (grid M x nshards) on `stream`. */
+vq_status vq_rht_apply_output_sharded(const void* y, void* y_out, const int8_t* signs, int32_t M, int32_t N,
+                                      const int32_t* shard_n, int32_t nshards, int32_t dtype, void* stream);
+
 /* Synchronise `stream` and report (then clear) any error flag a bounded
  * device-side wait of this handle's kernels raised: VQ_ERR_TIMEOUT if one gave
  * up, else VQ_OK.  Synchronous. */

@@ -120,6 +120,25 @@ def test_rht_rejects_bad_arguments_without_a_gpu(lib, M, K, dt, x, xo, signs):
     assert lib.vq_rht_apply_output(x or None, xo or None, signs or None, M, K, dt, None) == B.VQ_ERR_INVALID_ARG
 
 
+@pytest.mark.parametrize("shards,N,signs,xo", [
+    (None, 64, 16, 16),              # NULL shard sizes
+    ((), 64, 16, 16),                # no shard
+    ((64,) * 17, 64 * 17, 16, 16),   # more than 16 shards
+    ((96,), 96, 16, 16),             # not a multiple of 64
+    ((65536,), 65536, 16, 16),       # above 32768
+    ((64, 128), 256, 16, 16),        # the shards do not add up to N
+    ((64, 128), 192, 24, 16),        # misaligned signs
+    ((64, 128), 192, 16, 16 + 64),   # y_out partially overlaps y (M = 2)
+])
+def test_rht_sharded_rejects_bad_arguments_without_a_gpu(lib, shards, N, signs, xo):
+    if shards is None:
+        rc = lib.vq_rht_apply_output_sharded(16, xo, signs, 2, N, None, 1, 0, None)
+    else:
+        arr = (ctypes.c_int32 * max(1, len(shards)))(*shards)
+        rc = lib.vq_rht_apply_output_sharded(16, xo, signs, 2, N, arr, len(shards), 0, None)
+    assert rc == B.VQ_ERR_INVALID_ARG
+
+
 def test_python_binding_raises_with_message(lib):
     with pytest.raises(B.VQError, match="multiple of 64"):
         B.vq_rht_apply(16, 16, 16, 1, 100, 0, stream=0)

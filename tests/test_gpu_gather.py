@@ -240,6 +240,38 @@ def test_rht_output_matches_oracle(oracle, N, dt):
     assert np.array_equal(host_bits(yt), host_bits(out))
 
 
+@pytest.mark.parametrize("shards", [(4096, 1024, 1024), (14336, 14336), (64,), (2688, 192, 64)],
+                         ids=lambda s: "+".join(map(str, s)))
+@pytest.mark.parametrize("dt", [DT_F16, DT_BF16])
+def test_rht_output_sharded(oracle, shards, dt):
+    """Fused QKV / gate-up shards rotated in one launch: every shard bit-identical to a
+    separate vq_rht_apply_output call on it, within the oracle's bound, and in place."""
+    M, N = 3, sum(shards)
+    y = make_x(M, N, dt, cfg_id=89)
+    signs = make_signs(N, cfg_id=89)
+    yt, st = dev(y), dev(signs)
+    out = torch.empty_like(yt)
+    vq.vq_rht_apply_output_sharded(yt, out, st, M, N, shards, dt)
+    torch.cuda.synchronize()
+    got_all = host_bits(out)
+    o = 0
+    for w in shards:
+        part = yt[:, o:o + w].contiguous()
+        alone = torch.empty_like(part)
+        vq.vq_rht_apply_output(part, alone, st[o:o + w].contiguous(), M, w, dt)
+        torch.cuda.synchronize()
+        assert np.array_equal(host_bits(alone), got_all[:, o:o + w]), f"shard at {o}"
+        ref = oracle.rht_out_f64(widen(y[:, o:o + w], dt), signs[o:o + w])
+        ulp = np.spacing(np.abs(ref).astype(np.float16)).astype(np.float64) if dt == DT_F16 else np.abs(ref) * 2.0 ** -7
+        atol = 2 * np.log2(w) * 2.0 ** -24 * np.linalg.norm(widen(y[:, o:o + w], dt), axis=1, keepdims=True)
+        err = np.abs(widen(got_all[:, o:o + w], dt) - ref)
+        assert np.all(err <= ulp + atol), f"shard at {o}: max err/(ulp+atol) = {np.max(err / (ulp + atol))}"
+        o += w
+    vq.vq_rht_apply_output_sharded(yt, yt, st, M, N, shards, dt)
+    torch.cuda.synchronize()
+    assert np.array_equal(host_bits(yt), got_all)
+
+
 def test_two_sided_rotation(oracle):
     """A layer stored as W_hat = R_out W R_in^T: forward_rotated with the input signs, then
     the output rotation, against the oracle's rotations around the exact W_hat product.
