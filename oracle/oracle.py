@@ -75,6 +75,8 @@ def _load():
             lib.vqo_forward.argtypes = [I, I, I, I, P, I, P, P, P, P, P, P, P, I, P, I, P]
             lib.vqo_rht.restype = I
             lib.vqo_rht.argtypes = [I, I, P, I, P, P]
+            lib.vqo_encode.restype = I
+            lib.vqo_encode.argtypes = [I, I, I, P, P, I, P, P, P, P, P, P]
             lib.vqo_ladder_dequant.restype = I
             lib.vqo_ladder_dequant.argtypes = [I, I, I, I, P, P, P, P, P, P, P, I, P, I, P, P, I]
             lib.vqo_ladder_forward.restype = I
@@ -186,6 +188,34 @@ def dequant(layer, wdt: int = DT_F16, rows=None) -> tuple[np.ndarray, np.ndarray
     if rc:
         raise ValueError(f"vqo_dequant failed rc={rc}")
     return w, wb
+
+
+def encode(spec, w, scales, cb1, cb2=None) -> dict:
+    """Nearest-entry encode of a dense W [N,K] (orka README, "How it works") into the
+    planes of `spec.fmt`, with the given scales (fp16 bits, storage order) and codebooks.
+    Returns a layer dict like ``synth.make_layer``'s."""
+    lib = _load()
+    N, K, G = spec.N, spec.K, spec.K // 8
+    wd = _c(w, np.float64)
+    if wd.shape != (N, K):
+        raise ValueError("w has the wrong shape")
+    sc, c1, c2 = _c(scales, np.uint16), _c(cb1, np.uint16), _c(cb2, np.uint16)
+    out = {"spec": spec, "cb1": c1, "scales": sc}
+    lo = hi4 = s2 = idx16 = None
+    if spec.fmt == FMT_VQ16:
+        idx16 = np.zeros(N * G, np.uint16)
+        out["idx16"] = idx16
+    else:
+        lo, hi4 = np.zeros(N * G, np.uint8), np.zeros(N * G // 2, np.uint8)
+        out["lo"], out["hi4"] = lo, hi4
+        if spec.fmt == FMT_RVQ12_4:
+            s2 = np.zeros(N * G // 2, np.uint8)
+            out["s2"], out["cb2"] = s2, c2
+    rc = lib.vqo_encode(spec.fmt, N, K, _p(wd), _p(sc), spec.scale_group, _p(c1), _p(c2), _p(lo), _p(hi4), _p(s2),
+                        _p(idx16))
+    if rc:
+        raise ValueError(f"vqo_encode failed rc={rc}")
+    return out
 
 
 def forward(layer, x_bits, xdt: int, rows=None) -> np.ndarray:

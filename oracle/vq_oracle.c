@@ -17,6 +17,7 @@
  *   - GLQ README, "Inference kernels": Y = X . dequant(W)^T without materialising W.
  *   - GLQ README, "Bit widths": the residual ladder (16-bit primary, 16-bit
  *     residual stages, one 8-bit stage for odd bit widths), vqo_ladder_*.
+ *   - orka README, "How it works": encode = nearest entry per group, vqo_encode.
  *
  * Readings taken where the pages are silent (all fixed here, by construction):
  *   - groups run along K (the input dimension), G = K/8 groups per row;
@@ -294,6 +295,68 @@ int vqo_forward(int fmt, int M, int N, int K, const uint16_t* x, int xdt, const 
   free(wrow);
   free(xd);
   return rc;
+}
+
+/* ---------------------------------------------------------------------------
+ * Encode (orka README, "How it works": "encode -> nearest-entry index per group",
+ * then "indices as 12-bit BIT-PLANES (lo byte + packed hi)"; the two-stage format
+ * adds a 4-bit residual stage).  For group g of row n with scale s (one scale
+ * covers the whole group), stage 1 takes the entry nearest to the group's weights:
+ *   i1 = argmin_i sum_j (w[n][8g+j] - s * cb1[i][j])^2,
+ * and, for VQO_FMT_RVQ12_4, stage 2 the entry nearest to what stage 1 leaves:
+ *   i2 = argmin_t sum_j (w[n][8g+j] - s * (cb1[i1][j] + cb2[t][j]))^2.
+ * Distances in fp64; equal distances go to the smaller index (reading).  The
+ * indices are written in the storage layout the decoder reads (vqo_unpack is its
+ * inverse).  w is [N][K] fp64, scales fp16 bits in their storage order.
+ * ------------------------------------------------------------------------- */
+static uint32_t vqo_nearest(const double* w8, double s, const uint16_t* cb, uint32_t entries,
+                            const double* base8) {
+  uint32_t best = 0;
+  double bestd = INFINITY;
+  for (uint32_t i = 0; i < entries; ++i) {
+    double d = 0.0;
+    for (int j = 0; j < 8; ++j) {
+      const double c = (base8 ? base8[j] : 0.0) + vqo_f16_to_f64(cb[(int64_t)i * 8 + j]);
+      const double e = w8[j] - s * c;
+      d += e * e;
+    }
+    if (d < bestd) { bestd = d; best = i; }
+  }
+  return best;
+}
+
+int vqo_encode(int fmt, int N, int K, const double* w, const uint16_t* scales, int scale_group,
+               const uint16_t* cb1, const uint16_t* cb2, uint8_t* lo, uint8_t* hi4, uint8_t* s2,
+               uint16_t* idx16) {
+  int rc = vqo_check(fmt, N, K, scale_group);
+  if (rc) return rc;
+  const int G = K / 8;
+  const uint32_t entries = fmt == VQO_FMT_VQ16 ? 65536u : 4096u;
+  if (fmt != VQO_FMT_VQ16) {  /* the packed planes are filled nibble by nibble */
+    memset(hi4, 0, (size_t)N * G / 2);
+    if (fmt == VQO_FMT_RVQ12_4) memset(s2, 0, (size_t)N * G / 2);
+  }
+  for (int n = 0; n < N; ++n) {
+    for (int g = 0; g < G; ++g) {
+      const double* w8 = w + (int64_t)n * K + 8 * g;
+      const double s = vqo_f16_to_f64(scales[vqo_scale_index(n, 8 * g, N, K, scale_group)]);
+      const uint32_t i1 = vqo_nearest(w8, s, cb1, entries, NULL);
+      const int64_t e = vqo_slice_entry(n, g, N, G);
+      if (fmt == VQO_FMT_VQ16) {
+        idx16[e] = (uint16_t)i1;
+        continue;
+      }
+      lo[e] = (uint8_t)(i1 & 0xFFu);
+      hi4[e / 2] |= (uint8_t)(((i1 >> 8) & 15u) << ((g & 1) ? 4 : 0));
+      if (fmt == VQO_FMT_RVQ12_4) {
+        double b1[8];
+        for (int j = 0; j < 8; ++j) b1[j] = vqo_f16_to_f64(cb1[(int64_t)i1 * 8 + j]);
+        const uint32_t i2 = vqo_nearest(w8, s, cb2, 16u, b1);
+        s2[e / 2] |= (uint8_t)((i2 & 15u) << ((g & 1) ? 4 : 0));
+      }
+    }
+  }
+  return 0;
 }
 
 /* ---------------------------------------------------------------------------

@@ -381,6 +381,76 @@ def test_rht_bits_entry_matches_f64(oracle):
     assert np.array_equal(oracle.rht(x, DT_BF16, signs), oracle.rht_f64(xd, signs))
 
 
+# ------------------------------------------------------------------- encode (F4)
+
+@pytest.mark.parametrize("fmt,N,K", [(FMT_RVQ12, 24, 448), (FMT_VQ16, 8, 256)])
+def test_encode_round_trips_exact_codewords(oracle, fmt, N, K):
+    """W made exactly of scaled codewords encodes back to its own indices (orka README, "How it
+    works": encode = nearest entry; the true entry is at distance 0 and the codewords are
+    distinct)."""
+    layer = make_layer(LayerSpec(N, K, fmt, 64), cfg_id=120, tensor_id=fmt)
+    assert np.unique(layer["cb1"], axis=0).shape[0] == layer["cb1"].shape[0]
+    w, _ = oracle.dequant(layer)
+    enc = oracle.encode(layer["spec"], w, layer["scales"], layer["cb1"])
+    for k in ("lo", "hi4", "idx16"):
+        if k in layer:
+            assert np.array_equal(enc[k], layer[k]), k
+
+
+def test_encode_two_stage_round_trip(oracle):
+    """With a stage-2 codebook much smaller than the spacing of stage 1, W = s (c1 + c2) encodes
+    back to both indices (stage 2 takes the residual stage 1 leaves)."""
+    N, K = 16, 320
+    layer = make_layer(LayerSpec(N, K, FMT_RVQ12_4, 64), cfg_id=121)
+    small = (layer["cb2"].view(np.float16).astype(np.float32) * np.float32(1e-3)).astype(np.float16)
+    layer["cb2"] = small.view(np.uint16)
+    assert np.unique(layer["cb2"], axis=0).shape[0] == 16
+    w, _ = oracle.dequant(layer)
+    enc = oracle.encode(layer["spec"], w, layer["scales"], layer["cb1"], layer["cb2"])
+    for k in ("lo", "hi4", "s2"):
+        assert np.array_equal(enc[k], layer[k]), k
+
+
+@pytest.mark.parametrize("fmt", [FMT_RVQ12, FMT_RVQ12_4])
+def test_encode_matches_numpy_brute_force(oracle, fmt):
+    """Arbitrary W (not made of codewords): numpy argmin over every entry, stage by stage, read
+    back through the pinned unpack."""
+    N, K = 5, 192
+    rng = np.random.default_rng(122 + fmt)
+    layer = make_layer(LayerSpec(N, K, fmt, 64), cfg_id=122, tensor_id=fmt)
+    w = rng.standard_normal((N, K)) * 0.02
+    enc = oracle.encode(layer["spec"], w, layer["scales"], layer["cb1"], layer.get("cb2"))
+    i1, i2 = oracle.unpack(enc)
+    f = lambda b: b.view(np.float16).astype(np.float64)  # noqa: E731
+    c1 = f(layer["cb1"])
+    G = K // 8
+    for n in range(N):
+        for g in range(G):
+            sl, o = g // 16, g % 16
+            wsl = min(16, G - 16 * sl)
+            s = f(layer["scales"][2 * sl * N + n * (wsl // 8) + o // 8])
+            v = w[n, 8 * g:8 * g + 8]
+            a = int(np.argmin(((v[None, :] - s * c1) ** 2).sum(axis=1)))
+            assert i1[n, g] == a, (n, g)
+            if fmt == FMT_RVQ12_4:
+                c2 = f(layer["cb2"])
+                b = int(np.argmin(((v[None, :] - s * (c1[a][None, :] + c2)) ** 2).sum(axis=1)))
+                assert i2[n, g] == b, (n, g)
+
+
+def test_encode_ties_go_to_the_smaller_index(oracle):
+    N, K = 1, 16
+    cb1 = np.full((4096, 8), np.float16(30.0)).view(np.uint16).copy()
+    target = np.array([0.5, -1, 2, 0.25, -0.5, 1, 1.5, -2], np.float16)
+    cb1[9] = target.view(np.uint16)
+    cb1[5] = target.view(np.uint16)
+    sc = np.array([np.float16(0.5)], np.float16).view(np.uint16)
+    w = np.tile(0.5 * target.astype(np.float64), 2)[None, :]
+    enc = oracle.encode(LayerSpec(N, K, FMT_RVQ12, K), w, sc, cb1)
+    i1, _ = oracle.unpack(enc)
+    assert i1.tolist() == [[5, 5]]
+
+
 # ------------------------------------------------------------ residual ladder (F3)
 
 def _f16(a):
