@@ -60,3 +60,22 @@ def test_layer_bytes_match_the_format_arithmetic():
     # the headline workload's three tensors have equal byte counts
     sizes = {bench.layer_bytes(s, 1) for _, s in CONFIGS[4]["tensors"]}
     assert len(sizes) == 1
+
+
+def test_ladder_bytes_and_workloads():
+    """The residual ladder's algorithmic bytes: one 2-byte index per group per 16-bit stage and
+    one byte for the 8-bit stage, a 1 MiB codebook per 16-bit stage and 4 KiB for the 8-bit one
+    (GLQ README, "Bit widths": 5 bpw = 16 + 16 + 8)."""
+    from synth import FMT_VQ16_RVQ
+
+    spec = LayerSpec(4096, 4096, FMT_VQ16_RVQ, 4096, bpw=5)
+    G = 512
+    assert bench.layer_bytes(spec, 1) == 4096 * G * 5 + 4096 * 2 + 2 * 65536 * 16 + 256 * 16 + 4096 * 2 * 2
+    # bits per weight of the planes alone
+    planes = bench.layer_bytes(spec, 0) - 4096 * 2 - 2 * 65536 * 16 - 256 * 16
+    assert planes * 8 / (4096 * 4096) == 5.0
+    for bpw in (3, 4, 5):
+        cfg = bench._workload_config(f"vq16-ladder-4096-{bpw}bpw")
+        (_, s), = cfg["tensors"]
+        assert (s.fmt, s.bpw, s.N, s.K) == (FMT_VQ16_RVQ, bpw, 4096, 4096)
+    assert bench._workload_config("llama3-8b-mlp") is CONFIGS[4]
