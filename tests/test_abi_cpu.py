@@ -142,3 +142,12 @@ def test_rht_sharded_rejects_bad_arguments_without_a_gpu(lib, shards, N, signs, 
 def test_python_binding_raises_with_message(lib):
     with pytest.raises(B.VQError, match="multiple of 64"):
         B.vq_rht_apply(16, 16, 16, 1, 100, 0, stream=0)
+
+
+def test_zero_rows_return_before_touching_the_device(lib):
+    """M = 0 is valid for every rotation entry point and returns VQ_OK after the host-side
+    checks, without a launch (so without a GPU)."""
+    assert lib.vq_rht_apply(16, 16, 16, 0, 2688, 0, None) == B.VQ_OK
+    assert lib.vq_rht_apply_output(16, 16, 16, 0, 192, 1, None) == B.VQ_OK
+    arr = (ctypes.c_int32 * 3)(4096, 1024, 1024)
+    assert lib.vq_rht_apply_output_sharded(16, 16, 16, 0, 6144, arr, 3, 0, None) == B.VQ_OK
