@@ -732,13 +732,15 @@ def cpu_baseline(workload, M, budget_s=15.0, threads=None):
     cfg = w["config"] if "config" in w else CONFIGS[w["cfg"]]
     tensors = cfg["tensors"]
     x_cache = {}
-    per_layer_s = []
+    per_layer_s, single_s = [], []
     t_start = time.perf_counter()
     sample_desc = []
     for ti, (label, spec) in enumerate(tensors):
         layer = make_layer(spec, cfg_id=w["cfg"], layer=0, tensor_id=ti)
         if spec.K not in x_cache:
             x_cache[spec.K] = make_x(M, spec.K, cfg["act"], cfg_id=w["cfg"])
+        if ti == 0:  # untimed: loads the oracle library and starts the threads once
+            _oracle_rows(orc, layer, x_cache[spec.K], cfg["act"], min(spec.N, threads), threads)
         rows = max(8, min(spec.N, int(threads * 2048 * 4096 / spec.K)))
         # shrink the sample until one tensor fits its share of the budget
         while True:
@@ -749,13 +751,19 @@ def cpu_baseline(workload, M, budget_s=15.0, threads=None):
                 break
             rows = max(8, rows // 4)
         per_layer_s.append(dt * spec.N / rows)
-        sample_desc.append(f"{label}: {rows}/{spec.N} rows")
+        # the same oracle on one thread, on a 1/threads share of the sample (about the same wall time)
+        rows1 = max(8, rows // threads)
+        t0 = time.perf_counter()
+        _oracle_rows(orc, layer, x_cache[spec.K], cfg["act"], rows1, 1)
+        single_s.append((time.perf_counter() - t0) * spec.N / rows1)
+        sample_desc.append(f"{label}: {rows}/{spec.N} rows ({rows1} on one thread)")
         if time.perf_counter() - t_start > budget_s:
             break
     us = 1e6 * float(np.mean(per_layer_s))
     return {"value": round(us, 1), "unit": "us/layer", "cores": threads, "kind": "oracle",
-            "sample": f"M={M}; " + ", ".join(sample_desc) + f"; {threads} threads over row subsets; "
-                      "time scaled by N/rows (rows are independent)"}
+            "single_thread_value": round(1e6 * float(np.mean(single_s)), 1),
+            "sample": f"M={M}; " + ", ".join(sample_desc) + f"; {threads} threads over row subsets "
+                      "(single_thread_value: one thread); time scaled by N/rows (rows are independent)"}
 
 
 def reference_arm(args):
@@ -764,12 +772,13 @@ def reference_arm(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    per_step = []
+    per_step, single = [], []
     budget = max(1.0, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
     for k in range(args.warmup + args.steps):
         cb = cpu_baseline(args.workload, args.batch, budget_s=budget)
         if k >= args.warmup:
             per_step.append(cb["value"])
+            single.append(cb["single_thread_value"])
     v = float(np.mean(per_step))
     out = {"metric": METRIC, "value": round(v, 1), "unit": "us/layer", "n_gpus": world, "steps": args.steps,
            "warmup": args.warmup, "ms_per_step": round(v * 1e-3 * len(_workload_config(args.workload)["tensors"]), 3),
@@ -777,7 +786,7 @@ def reference_arm(args):
            "data": "synthetic (seeded)", "impl": "reference",
            "config": {"workload": args.workload, "M": args.batch, "layer": "one weight matrix"},
            "cpu_baseline": {"value": round(v, 1), "unit": "us/layer", "cores": cb["cores"], "kind": "oracle",
-                            "sample": cb["sample"]},
+                            "single_thread_value": round(float(np.mean(single)), 1), "sample": cb["sample"]},
            "e2e": {"value": round(v, 1), "unit": "us/layer", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
 
