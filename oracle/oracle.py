@@ -77,6 +77,10 @@ def _load():
             lib.vqo_rht.argtypes = [I, I, P, I, P, P]
             lib.vqo_encode.restype = I
             lib.vqo_encode.argtypes = [I, I, I, P, P, I, P, P, P, P, P, P]
+            lib.vqo_dist32.restype = ctypes.c_double
+            lib.vqo_dist32.argtypes = [P, ctypes.c_double, P]
+            lib.vqo_encode32.restype = I
+            lib.vqo_encode32.argtypes = [I, I, I, P, P, I, P, P, P, P, P, P]
             lib.vqo_ladder_dequant.restype = I
             lib.vqo_ladder_dequant.argtypes = [I, I, I, I, P, P, P, P, P, P, P, I, P, I, P, P, I]
             lib.vqo_ladder_forward.restype = I
@@ -190,11 +194,20 @@ def dequant(layer, wdt: int = DT_F16, rows=None) -> tuple[np.ndarray, np.ndarray
     return w, wb
 
 
-def encode(spec, w, scales, cb1, cb2=None) -> dict:
+def dist32(w8, s, c8) -> float:
+    """The binary32 distance the GPU encoder decides with (binary32 inputs)."""
+    w8, c8 = _c(w8, np.float64), _c(c8, np.float64)
+    return _load().vqo_dist32(_p(w8), float(s), _p(c8))
+
+
+def encode(spec, w, scales, cb1, cb2=None, precision: str = "f64") -> dict:
     """Nearest-entry encode of a dense W [N,K] (orka README, "How it works") into the
     planes of `spec.fmt`, with the given scales (fp16 bits, storage order) and codebooks.
-    Returns a layer dict like ``synth.make_layer``'s."""
+    precision "f64": the definition, distances in fp64; "f32": the same decisions taken
+    with binary32 distances in a fixed operation order (W must hold binary32 values), the
+    precision of the GPU encoder.  Returns a layer dict like ``synth.make_layer``'s."""
     lib = _load()
+    fn = {"f64": lib.vqo_encode, "f32": lib.vqo_encode32}[precision]
     N, K, G = spec.N, spec.K, spec.K // 8
     wd = _c(w, np.float64)
     if wd.shape != (N, K):
@@ -211,8 +224,7 @@ def encode(spec, w, scales, cb1, cb2=None) -> dict:
         if spec.fmt == FMT_RVQ12_4:
             s2 = np.zeros(N * G // 2, np.uint8)
             out["s2"], out["cb2"] = s2, c2
-    rc = lib.vqo_encode(spec.fmt, N, K, _p(wd), _p(sc), spec.scale_group, _p(c1), _p(c2), _p(lo), _p(hi4), _p(s2),
-                        _p(idx16))
+    rc = fn(spec.fmt, N, K, _p(wd), _p(sc), spec.scale_group, _p(c1), _p(c2), _p(lo), _p(hi4), _p(s2), _p(idx16))
     if rc:
         raise ValueError(f"vqo_encode failed rc={rc}")
     return out

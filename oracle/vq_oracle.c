@@ -359,6 +359,75 @@ int vqo_encode(int fmt, int N, int K, const double* w, const uint16_t* scales, i
   return 0;
 }
 
+/* The same encode with the distances in binary32, the precision the GPU encoder
+ * decides in (reading: where floating point decides an integer, both sides decide in
+ * the same precision).  For group values w_j (binary32) and scale s:
+ *   d = (((e_0^2 + e_1^2) + e_2^2) + ... + e_7^2),  e_j = w_j - s * c_j,
+ * every product, difference and sum rounded to binary32 in that order, with
+ * c_j = cb1[i][j] for stage 1 and c_j = cb1[i1][j] + cb2[t][j] (rounded) for stage 2.
+ * Each operation is on binary32 values, so the fp64 result rounded once is the
+ * binary32 result.  w is [N][K] binary32 values held in doubles. */
+/* The binary32 distance of 8 values to 8 codeword values (all binary32 values held
+ * in doubles), in the order above. */
+double vqo_dist32(const double* w8, double s, const double* c8) {
+  double d = 0.0;
+  for (int j = 0; j < 8; ++j) {
+    const double e = vqo_fl32(w8[j] - vqo_fl32(s * c8[j]));
+    d = vqo_fl32(d + vqo_fl32(e * e));
+  }
+  return d;
+}
+
+static uint32_t vqo_nearest32(const double* w8, double s, const uint16_t* cb, uint32_t entries,
+                              const double* base8) {
+  uint32_t best = 0;
+  double bestd = INFINITY;
+  for (uint32_t i = 0; i < entries; ++i) {
+    double c[8];
+    for (int j = 0; j < 8; ++j) {
+      c[j] = vqo_f16_to_f64(cb[(int64_t)i * 8 + j]);
+      if (base8) c[j] = vqo_fl32(base8[j] + c[j]);
+    }
+    const double d = vqo_dist32(w8, s, c);
+    if (d < bestd) { bestd = d; best = i; }
+  }
+  return best;
+}
+
+int vqo_encode32(int fmt, int N, int K, const double* w, const uint16_t* scales, int scale_group,
+                 const uint16_t* cb1, const uint16_t* cb2, uint8_t* lo, uint8_t* hi4, uint8_t* s2,
+                 uint16_t* idx16) {
+  int rc = vqo_check(fmt, N, K, scale_group);
+  if (rc) return rc;
+  const int G = K / 8;
+  const uint32_t entries = fmt == VQO_FMT_VQ16 ? 65536u : 4096u;
+  if (fmt != VQO_FMT_VQ16) {
+    memset(hi4, 0, (size_t)N * G / 2);
+    if (fmt == VQO_FMT_RVQ12_4) memset(s2, 0, (size_t)N * G / 2);
+  }
+  for (int n = 0; n < N; ++n) {
+    for (int g = 0; g < G; ++g) {
+      const double* w8 = w + (int64_t)n * K + 8 * g;
+      const double s = vqo_f16_to_f64(scales[vqo_scale_index(n, 8 * g, N, K, scale_group)]);
+      const uint32_t i1 = vqo_nearest32(w8, s, cb1, entries, NULL);
+      const int64_t e = vqo_slice_entry(n, g, N, G);
+      if (fmt == VQO_FMT_VQ16) {
+        idx16[e] = (uint16_t)i1;
+        continue;
+      }
+      lo[e] = (uint8_t)(i1 & 0xFFu);
+      hi4[e / 2] |= (uint8_t)(((i1 >> 8) & 15u) << ((g & 1) ? 4 : 0));
+      if (fmt == VQO_FMT_RVQ12_4) {
+        double b1[8];
+        for (int j = 0; j < 8; ++j) b1[j] = vqo_f16_to_f64(cb1[(int64_t)i1 * 8 + j]);
+        const uint32_t i2 = vqo_nearest32(w8, s, cb2, 16u, b1);
+        s2[e / 2] |= (uint8_t)((i2 & 15u) << ((g & 1) ? 4 : 0));
+      }
+    }
+  }
+  return 0;
+}
+
 /* ---------------------------------------------------------------------------
  * Residual ladder (GLQ README, "Bit widths": a 16-bit primary stage, then 16-bit
  * residual stages, and for an odd bit width one final 8-bit stage -- 3 bpw is

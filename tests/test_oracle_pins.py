@@ -438,6 +438,78 @@ def test_encode_matches_numpy_brute_force(oracle, fmt):
                 assert i2[n, g] == b, (n, g)
 
 
+@pytest.mark.parametrize("fmt", [FMT_RVQ12, FMT_RVQ12_4])
+def test_encode32_matches_numpy_float32(oracle, fmt):
+    """The binary32 decision (the GPU encoder's precision) against numpy float32 arithmetic in
+    the same order: e_j = w_j - s * c_j, d = ((e_0^2 + e_1^2) + ...) + e_7^2, argmin first."""
+    N, K = 4, 192
+    rng = np.random.default_rng(130 + fmt)
+    layer = make_layer(LayerSpec(N, K, fmt, 64), cfg_id=130, tensor_id=fmt)
+    w = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    enc = oracle.encode(layer["spec"], w.astype(np.float64), layer["scales"], layer["cb1"], layer.get("cb2"),
+                        precision="f32")
+    i1, i2 = oracle.unpack(enc)
+    c1 = layer["cb1"].view(np.float16).astype(np.float32)
+    G = K // 8
+
+    def nearest(v, s, c):
+        d = np.zeros(c.shape[0], np.float32)
+        for j in range(8):
+            e = v[j] - s * c[:, j]
+            d = d + e * e
+        return int(np.argmin(d))
+
+    for n in range(N):
+        for g in range(G):
+            sl, o = g // 16, g % 16
+            s = layer["scales"][2 * sl * N + n * (min(16, G - 16 * sl) // 8) + o // 8].view(np.float16).astype(np.float32)
+            v = w[n, 8 * g:8 * g + 8]
+            a = nearest(v, s, c1)
+            assert i1[n, g] == a, (n, g)
+            if fmt == FMT_RVQ12_4:
+                c2 = c1[a][None, :] + layer["cb2"].view(np.float16).astype(np.float32)
+                assert i2[n, g] == nearest(v, s, c2), (n, g)
+
+
+def test_dist32_is_bit_exact_binary32(oracle):
+    """Every product, difference and sum rounded to binary32, in the stated order: the value
+    equals numpy float32 arithmetic bit for bit (an fma, another order or fp64 accumulation
+    changes some of these)."""
+    rng = np.random.default_rng(132)
+    for _ in range(3000):
+        w = (rng.standard_normal(8) * 10.0 ** rng.uniform(-3, 1)).astype(np.float32)
+        c = rng.standard_normal(8).astype(np.float16).astype(np.float32)
+        s = np.float32(np.float16(rng.lognormal(-4, 1)))
+        d = np.float32(0)
+        for j in range(8):
+            e = np.float32(w[j] - np.float32(s * c[j]))
+            d = np.float32(d + np.float32(e * e))
+        assert oracle.dist32(w.astype(np.float64), float(s), c.astype(np.float64)) == float(d)
+
+
+def test_encode32_agrees_with_the_definition(oracle):
+    """binary32 and fp64 decisions agree except where the two candidates' exact distances
+    are within the binary32 error of each other; exact codewords round trip in both."""
+    N, K = 32, 256
+    layer = make_layer(LayerSpec(N, K, FMT_RVQ12, 64), cfg_id=131)
+    w = (np.random.default_rng(131).standard_normal((N, K)) * 0.02).astype(np.float32).astype(np.float64)
+    a64, _ = oracle.unpack(oracle.encode(layer["spec"], w, layer["scales"], layer["cb1"]))
+    a32, _ = oracle.unpack(oracle.encode(layer["spec"], w, layer["scales"], layer["cb1"], precision="f32"))
+    c1 = layer["cb1"].view(np.float16).astype(np.float64)
+    G = K // 8
+    differ = np.argwhere(a64 != a32)
+    assert len(differ) <= 0.01 * N * G
+    for n, g in differ:
+        sl, o = g // 16, g % 16
+        s = layer["scales"][2 * sl * N + n * 2 + o // 8].view(np.float16).astype(np.float64)
+        v = w[n, 8 * g:8 * g + 8]
+        d = lambda i: float(((v - s * c1[i]) ** 2).sum())  # noqa: E731
+        assert d(a32[n, g]) - d(a64[n, g]) <= 1e-5 * d(a64[n, g]), (n, g)
+    wx, _ = oracle.dequant(layer)
+    rt = oracle.encode(layer["spec"], wx, layer["scales"], layer["cb1"], precision="f32")
+    assert np.array_equal(rt["lo"], layer["lo"]) and np.array_equal(rt["hi4"], layer["hi4"])
+
+
 def test_encode_ties_go_to_the_smaller_index(oracle):
     N, K = 1, 16
     cb1 = np.full((4096, 8), np.float16(30.0)).view(np.uint16).copy()
