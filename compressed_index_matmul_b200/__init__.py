@@ -30,6 +30,7 @@ from ._binding import (  # noqa: F401
     vq_debug_dequant,
     vq_debug_unpack,
     vq_debug_wait_timeout,
+    vq_encode,
     vq_linear_check,
     vq_linear_create,
     vq_linear_destroy,

@@ -31,7 +31,7 @@ STATUS_NAMES = {0: "VQ_OK", 1: "VQ_ERR_INVALID_ARG", 2: "VQ_ERR_UNSUPPORTED", 3:
 # Every entry point the header declares (checked by the tests against the .so).
 EXPORTS = ("vq_abi_version", "vq_linear_create", "vq_linear_destroy", "vq_linear_set_path", "vq_linear_set_sm_budget",
            "vq_linear_forward",
-           "vq_linear_forward_noalloc", "vq_linear_forward_rotated", "vq_linear_launches", "vq_rht_apply", "vq_rht_apply_output", "vq_rht_apply_output_sharded", "vq_linear_check", "vq_last_error",
+           "vq_linear_forward_noalloc", "vq_linear_forward_rotated", "vq_linear_launches", "vq_rht_apply", "vq_rht_apply_output", "vq_rht_apply_output_sharded", "vq_encode", "vq_linear_check", "vq_last_error",
            "vq_debug_unpack", "vq_debug_dequant", "vq_debug_wait_timeout")
 
 
@@ -103,6 +103,8 @@ def load(path: str | None = None):
         lib.vq_rht_apply.argtypes = [P, P, P, I32, I32, I32, P]
         lib.vq_rht_apply_output.restype = st
         lib.vq_rht_apply_output.argtypes = [P, P, P, I32, I32, I32, P]
+        lib.vq_encode.restype = st
+        lib.vq_encode.argtypes = [ctypes.POINTER(vq_linear_desc), P, P, ctypes.POINTER(vq_codebooks), P, P, P, P, P]
         lib.vq_rht_apply_output_sharded.restype = st
         lib.vq_rht_apply_output_sharded.argtypes = [P, P, P, I32, I32, ctypes.POINTER(I32), I32, I32, P]
         lib.vq_linear_check.restype = st
@@ -208,6 +210,14 @@ def vq_rht_apply(x, x_out, signs, M, K, dtype, stream=None) -> None:
 
 def vq_rht_apply_output(y, y_out, signs, M, N, dtype, stream=None) -> None:
     _check(load().vq_rht_apply_output(_ptr(y), _ptr(y_out), _ptr(signs), M, N, dtype, _stream(stream)))
+
+
+def vq_encode(N, K, fmt, scale_group, w, scales, codebooks: vq_codebooks, lo=None, hi4=None, s2=None, idx16=None,
+              stream=None) -> None:
+    """Nearest-entry encode of fp32 W [N, K] (device) into the index planes (device outputs)."""
+    d = make_desc(N, K, fmt, scale_group, VQ_F16, 1)
+    _check(load().vq_encode(ctypes.byref(d), _ptr(w), _ptr(scales), ctypes.byref(codebooks), _ptr(lo), _ptr(hi4),
+                            _ptr(s2), _ptr(idx16), _stream(stream)))
 
 
 def vq_rht_apply_output_sharded(y, y_out, signs, M, N, shard_n, dtype, stream=None) -> None:

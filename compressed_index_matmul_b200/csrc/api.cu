@@ -465,6 +465,42 @@ VQ_API vq_status vq_rht_apply_output_sharded(const void* y, void* y_out, const i
   return VQ_OK;
 }
 
+VQ_API vq_status vq_encode(const vq_linear_desc* desc, const float* w, const void* scales,
+                           const vq_codebooks* codebooks, uint8_t* lo, uint8_t* hi4, uint8_t* s2, uint16_t* idx16,
+                           void* stream) {
+  if (desc == nullptr) return fail(VQ_ERR_INVALID_ARG, "desc is NULL");
+  vq_linear_desc d = *desc;  // the fields a forward needs but the encoder does not use
+  d.act_dtype = VQ_F16;
+  d.max_M = 1;
+  d.rht = 0;
+  vq_status st;
+  if ((st = validate_desc(&d))) return st;
+  if (d.fmt == VQ_FMT_VQ16_RVQ) return fail(VQ_ERR_UNSUPPORTED, "the encoder takes the single-plane formats only");
+  if ((st = check_ptr(w, "w")) || (st = validate_codebooks(d, codebooks, scales))) return st;
+  if (d.fmt == VQ_FMT_VQ16) {
+    if ((st = check_ptr(idx16, "idx16"))) return st;
+  } else {
+    if ((st = check_ptr(lo, "lo")) || (st = check_ptr(hi4, "hi4"))) return st;
+    if (d.fmt == VQ_FMT_RVQ12_4 && (st = check_ptr(s2, "s2"))) return st;
+  }
+  vq::EncodeArgs a{};
+  a.w = w;
+  a.scales = static_cast<const uint16_t*>(scales);
+  a.cb1 = static_cast<const uint16_t*>(codebooks->cb1);
+  a.cb2 = d.fmt == VQ_FMT_RVQ12_4 ? static_cast<const uint16_t*>(codebooks->cb2) : nullptr;
+  a.lo = lo;
+  a.hi4 = hi4;
+  a.s2 = s2;
+  a.idx16 = idx16;
+  a.N = d.N;
+  a.K = d.K;
+  a.fmt = d.fmt;
+  a.scale_group = d.scale_group;
+  cudaError_t e = vq::launch_encode(a, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "vq_encode launch");
+  return VQ_OK;
+}
+
 VQ_API vq_status vq_linear_check(vq_linear_t h, void* stream) {
   if (h == nullptr) return fail(VQ_ERR_INVALID_ARG, "handle is NULL");
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));

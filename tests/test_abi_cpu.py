@@ -151,3 +151,21 @@ def test_zero_rows_return_before_touching_the_device(lib):
     assert lib.vq_rht_apply_output(16, 16, 16, 0, 192, 1, None) == B.VQ_OK
     arr = (ctypes.c_int32 * 3)(4096, 1024, 1024)
     assert lib.vq_rht_apply_output_sharded(16, 16, 16, 0, 6144, arr, 3, 0, None) == B.VQ_OK
+
+
+def test_encode_rejects_bad_arguments_without_a_gpu(lib):
+    cbs = B.make_codebooks(16, 16)
+    def enc(**kw):
+        a = dict(N=8, K=128, fmt=B.VQ_FMT_RVQ12_4, scale_group=64, w=16, scales=16, lo=16, hi4=16, s2=16, idx16=None)
+        a.update(kw)
+        d = B.make_desc(a["N"], a["K"], a["fmt"], a["scale_group"], B.VQ_F16, 1)
+        return lib.vq_encode(ctypes.byref(d), a["w"], a["scales"], ctypes.byref(cbs), a["lo"], a["hi4"], a["s2"],
+                             a["idx16"], None)
+    assert lib.vq_encode(None, 16, 16, ctypes.byref(cbs), 16, 16, 16, None, None) == B.VQ_ERR_INVALID_ARG
+    assert enc(w=None) == B.VQ_ERR_INVALID_ARG
+    assert enc(w=24) == B.VQ_ERR_INVALID_ARG          # misaligned
+    assert enc(s2=None) == B.VQ_ERR_INVALID_ARG       # the two-stage format writes s2
+    assert enc(fmt=B.VQ_FMT_VQ16, idx16=None) == B.VQ_ERR_INVALID_ARG
+    assert enc(K=72) == B.VQ_ERR_INVALID_ARG
+    assert enc(K=256, scale_group=128) == B.VQ_ERR_UNSUPPORTED
+    assert enc(fmt=B.VQ_FMT_VQ16_RVQ) == B.VQ_ERR_INVALID_ARG  # ladder stage counts of zero
