@@ -169,3 +169,25 @@ def test_encode_rejects_bad_arguments_without_a_gpu(lib):
     assert enc(K=72) == B.VQ_ERR_INVALID_ARG
     assert enc(K=256, scale_group=128) == B.VQ_ERR_UNSUPPORTED
     assert enc(fmt=B.VQ_FMT_VQ16_RVQ) == B.VQ_ERR_INVALID_ARG  # ladder stage counts of zero
+
+
+def test_missing_library_fails_loudly():
+    """No CPU fallback: loading a library that is not there raises ImportError."""
+    import subprocess
+    import sys
+
+    code = ("from compressed_index_matmul_b200 import _binding as B\n"
+            "try:\n    B.load('/nonexistent/libvqlinear.so')\nexcept ImportError:\n    raise SystemExit(7)\n")
+    r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True)
+    assert r.returncode == 7, r.stderr
+
+
+def test_product_package_never_uses_the_oracle():
+    """The oracle is test infrastructure: nothing in the product package imports, loads or
+    names its module or library."""
+    pkg = os.path.join(ROOT, "compressed_index_matmul_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                src = open(os.path.join(dirpath, f)).read()
+                assert not re.search(r"\boracle\b|vq_oracle|vqo_", src), os.path.join(dirpath, f)
