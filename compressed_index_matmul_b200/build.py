@@ -12,6 +12,7 @@ from __future__ import annotations
 import concurrent.futures as cf
 import glob
 import hashlib
+import re
 import os
 import shutil
 import subprocess
@@ -40,23 +41,49 @@ def _sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
+_INCLUDE_RE = re.compile(r'^\s*#\s*include\s+"([^"]+)"', re.M)
+
+
+def _unit_files(unit: str) -> list:
+    """A translation unit under csrc/ and every header it includes, transitively (quoted
+    includes, looked up in csrc/ and include/ as the compile flags do)."""
+    seen, todo = set(), [os.path.join(CSRC, unit)]
+    while todo:
+        f = todo.pop()
+        if f in seen:
+            continue
+        seen.add(f)
+        with open(f) as fh:
+            for name in _INCLUDE_RE.findall(fh.read()):
+                for d in (CSRC, INCLUDE):
+                    cand = os.path.join(d, name)
+                    if os.path.exists(cand):
+                        todo.append(cand)
+                        break
+    return sorted(seen)
+
+
 def _deps_hash(unit: str | None = None) -> str:
     h = hashlib.sha256()
-    units = _sources() if unit is None else [os.path.join(CSRC, unit)]
-    files = units + sorted(glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h")))
-    files.append(os.path.join(INCLUDE, "vqlinear.h"))
+    if unit is None:
+        files = _sources() + sorted(glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h")) +
+                                    glob.glob(os.path.join(INCLUDE, "*.h")))
+    else:
+        files = _unit_files(unit)
+    # paths relative to the repository root, so the same sources hash the same wherever
+    # the repository is checked out
     for f in files:
-        h.update(f.encode())
+        h.update(os.path.relpath(f, ROOT).encode())
         with open(f, "rb") as fh:
             h.update(fh.read())
-    h.update(" ".join(NVCC_FLAGS).encode())
+    h.update(" ".join(NVCC_FLAGS).replace(ROOT, "<root>").encode())
     return h.hexdigest()
 
 
 def source_digest(unit: str | None = None) -> str:
     """Hash of every kernel/ABI source and the compile flags (identifies a build of the kernels);
-    with `unit` (a file name under csrc/), of that translation unit, every header and the flags
-    (identifies a build of the kernels defined in it)."""
+    with `unit` (a file name under csrc/), of that translation unit, the headers it includes
+    (transitively) and the flags (identifies a build of the kernels defined in it)."""
     return _deps_hash(unit)[:16]
 
 

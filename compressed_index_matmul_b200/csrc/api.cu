@@ -12,7 +12,9 @@
 #include <string>
 
 #include "internal.h"
+#include "tools.h"
 #include "vqlinear.h"
+#include "vqlinear_tools.h"
 
 #define VQ_API extern "C" __attribute__((visibility("default")))
 

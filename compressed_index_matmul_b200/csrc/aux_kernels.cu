@@ -4,6 +4,7 @@
 #include "common.cuh"
 #include "rotate.cuh"
 #include "internal.h"
+#include "tools.h"
 #include "ladder.cuh"
 #include "tc_ptx.cuh"
 

@@ -20,6 +20,7 @@
 // the forward path.
 #include "common.cuh"
 #include "internal.h"
+#include "tools.h"
 
 namespace vq {
 

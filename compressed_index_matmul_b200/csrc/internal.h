@@ -74,28 +74,6 @@ cudaError_t launch_rht(const void* x, void* x_out, const int8_t* signs, int M, i
                        cudaStream_t s);
 cudaError_t launch_rht_output(const void* y, void* y_out, const int8_t* signs, int M, int N, int dtype,
                               cudaStream_t s);
-// Column shards of y for the shard-batched output rotation: shard s is columns
-// [off[s], off[s+1]), n <= kRhtMaxShards.
-constexpr int kRhtMaxShards = 16;
-struct RhtShards {
-  int n;
-  int off[kRhtMaxShards + 1];
-};
-cudaError_t launch_rht_output_shards(const void* y, void* y_out, const int8_t* signs, int M, int N,
-                                     const RhtShards& sh, int dtype, cudaStream_t s);
-// The nearest-entry encoder (encode.cu): W [N][K] fp32 -> index planes.
-struct EncodeArgs {
-  const float* w;
-  const uint16_t* scales;
-  const uint16_t* cb1;
-  const uint16_t* cb2;
-  uint8_t* lo;
-  uint8_t* hi4;
-  uint8_t* s2;
-  uint16_t* idx16;
-  int N, K, fmt, scale_group;
-};
-cudaError_t launch_encode(const EncodeArgs& a, cudaStream_t s);
 cudaError_t launch_debug_unpack(const LayerArgs& a, uint16_t* i1, uint8_t* i2, cudaStream_t s);
 cudaError_t launch_debug_dequant(const LayerArgs& a, void* w, int wdt, cudaStream_t s);
 cudaError_t launch_debug_wait_timeout(uint32_t* err, cudaStream_t s);

@@ -22,7 +22,9 @@ def lib():
 
 
 def declared_functions():
-    src = open(HEADER).read()
+    import glob
+
+    src = "".join(open(h).read() for h in sorted(glob.glob(os.path.join(ROOT, "include", "*.h"))))
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
     return sorted(set(re.findall(r"\b(vq_[a-z0-9_]+)\s*\(", src)))
 

@@ -79,3 +79,25 @@ def test_ladder_bytes_and_workloads():
         (_, s), = cfg["tensors"]
         assert (s.fmt, s.bpw, s.N, s.K) == (FMT_VQ16_RVQ, bpw, 4096, 4096)
     assert bench._workload_config("llama3-8b-mlp") is CONFIGS[4]
+
+
+def test_source_digest_does_not_depend_on_the_checkout_path(tmp_path):
+    """The traffic figures are keyed by a digest of each kernel's translation unit and the
+    headers it includes; a copy of the sources elsewhere (as on a GPU machine) hashes the same."""
+    import importlib.util
+    import shutil
+
+    from compressed_index_matmul_b200 import build as b
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    pkg = tmp_path / "compressed_index_matmul_b200"
+    shutil.copytree(os.path.join(root, "compressed_index_matmul_b200", "csrc"), pkg / "csrc")
+    shutil.copy(os.path.join(root, "compressed_index_matmul_b200", "build.py"), pkg / "build.py")
+    shutil.copytree(os.path.join(root, "include"), tmp_path / "include")
+    spec = importlib.util.spec_from_file_location("build_copy", pkg / "build.py")
+    copy = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(copy)
+    for unit in ("lut_gemv.cu", "vq16_gemv.cu", "tc_gemm.cu"):
+        assert copy.source_digest(unit) == b.source_digest(unit)
+        assert [os.path.relpath(f, tmp_path) for f in copy._unit_files(unit)] == \
+               [os.path.relpath(f, root) for f in b._unit_files(unit)]
