@@ -707,17 +707,23 @@ def _host_cores():
         return os.cpu_count() or 1
 
 
+_POOLS = {}
+
+
 def _oracle_rows(orc, layer, x, act, rows, threads):
     """The oracle on rows 0..rows-1 of the full layer, split over `threads` threads
-    (ctypes releases the GIL during the C call, so the row subsets run in parallel)."""
+    (ctypes releases the GIL during the C call, so the row subsets run in parallel; the
+    thread pool is made once per thread count)."""
     import concurrent.futures as cf
 
     parts = [p for p in np.array_split(np.arange(rows, dtype=np.int32), threads) if len(p)]
     if len(parts) == 1:
         orc.forward(layer, x, act, rows=parts[0])
         return
-    with cf.ThreadPoolExecutor(len(parts)) as ex:
-        list(ex.map(lambda r: orc.forward(layer, x, act, rows=r), parts))
+    ex = _POOLS.get(threads)
+    if ex is None:
+        ex = _POOLS[threads] = cf.ThreadPoolExecutor(threads)
+    list(ex.map(lambda r: orc.forward(layer, x, act, rows=r), parts))
 
 
 def cpu_baseline(workload, M, budget_s=15.0, threads=None):
@@ -766,27 +772,62 @@ def cpu_baseline(workload, M, budget_s=15.0, threads=None):
                       "(single_thread_value: one thread); time scaled by N/rows (rows are independent)"}
 
 
+REFERENCE_SECONDS = 150.0  # the whole --impl reference run, warm-up included
+
+
 def reference_arm(args):
-    """--impl reference: the oracle on the host cores, same workload/metric; rank 0 only."""
+    """--impl reference: the oracle on the host cores, same workload/metric; rank 0 only.
+
+    Each of the W + K steps times the oracle on a row sample of one tensor of the
+    workload (the tensors in turn), sized so that the whole run takes about
+    REFERENCE_SECONDS; a step's result is its sample time scaled to the whole tensor
+    (rows are independent) and the line reports the mean over the K timed steps."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    per_step, single = [], []
-    budget = max(1.0, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
+    from oracle import oracle as orc
+
+    orc.build()
+    threads = _host_cores()
+    w = WORKLOADS[args.workload]
+    cfg = _workload_config(args.workload)
+    layers, xs = [], {}
+    for ti, (label, spec) in enumerate(cfg["tensors"]):
+        layers.append((label, spec, make_layer(spec, cfg_id=w["cfg"], layer=0, tensor_id=ti)))
+        if spec.K not in xs:
+            xs[spec.K] = make_x(args.batch, spec.K, cfg["act"], cfg_id=w["cfg"])
+    # calibration (untimed): seconds per row of each tensor on all threads
+    row_s = []
+    for label, spec, layer in layers:
+        r0 = min(spec.N, 64 * threads)
+        _oracle_rows(orc, layer, xs[spec.K], cfg["act"], r0, threads)
+        t0 = time.perf_counter()
+        _oracle_rows(orc, layer, xs[spec.K], cfg["act"], r0, threads)
+        row_s.append(max(1e-9, (time.perf_counter() - t0) / r0))
+    per_step = REFERENCE_SECONDS / max(1, args.steps + args.warmup)
+    per_layer, rows_used = [], set()
     for k in range(args.warmup + args.steps):
-        cb = cpu_baseline(args.workload, args.batch, budget_s=budget)
+        ti = k % len(layers)
+        label, spec, layer = layers[ti]
+        rows = int(max(8, min(spec.N, per_step / row_s[ti])))
+        t0 = time.perf_counter()
+        _oracle_rows(orc, layer, xs[spec.K], cfg["act"], rows, threads)
+        dt = time.perf_counter() - t0
         if k >= args.warmup:
-            per_step.append(cb["value"])
-            single.append(cb["single_thread_value"])
-    v = float(np.mean(per_step))
+            per_layer.append(1e6 * dt * spec.N / rows)
+            rows_used.add((label, rows, spec.N))
+    v = float(np.mean(per_layer))
+    sample = (f"M={args.batch}; each step one tensor in turn, rows 0..r-1 of the full layer on {threads} threads, "
+              "time scaled by N/r (rows are independent): " +
+              ", ".join(f"{lb} {r}/{n} rows" for lb, r, n in sorted(rows_used)))
     out = {"metric": METRIC, "value": round(v, 1), "unit": "us/layer", "n_gpus": world, "steps": args.steps,
-           "warmup": args.warmup, "ms_per_step": round(v * 1e-3 * len(_workload_config(args.workload)["tensors"]), 3),
+           "warmup": args.warmup, "ms_per_step": round(v * 1e-3 * len(cfg["tensors"]), 3),
            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
            "data": "synthetic (seeded)", "impl": "reference",
            "config": {"workload": args.workload, "M": args.batch, "layer": "one weight matrix"},
-           "cpu_baseline": {"value": round(v, 1), "unit": "us/layer", "cores": cb["cores"], "kind": "oracle",
-                            "single_thread_value": round(float(np.mean(single)), 1), "sample": cb["sample"]},
+           "cpu_baseline": {"value": round(v, 1), "unit": "us/layer", "cores": threads, "kind": "oracle",
+                            "sample": sample},
            "e2e": {"value": round(v, 1), "unit": "us/layer", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
 
