@@ -33,8 +33,8 @@ struct vq_linear_s {
   size_t scratch_bytes;
   uint32_t* tickets;  // completion counters, zeroed at create, left zero by every forward
   int num_tickets;
-  uint32_t* gbar;     // grid-barrier arrival counters, one 64-bit word per grid size 0..num_sms
-                      // (8-byte aligned; each only ever grows by whole grids)
+  uint32_t* sync;     // the table kernel's cross-CTA words (zeroed at create)
+  int num_sync;
   uint32_t* err;      // device word, set by bounded waits that gave up
   int sm_budget;      // CTAs of the table kernel (0: every SM)
   void* xrot;         // rotated-x buffer [max_M][K] (desc.rht == 1), for the unfused rotated forward
@@ -223,7 +223,7 @@ VQ_API vq_status vq_linear_create(const vq_linear_desc* desc, vq_linear_t* out) 
 
   // Scratch: the largest any path may need for any M <= max_M.
   size_t need = 0;
-  int tickets = 0;
+  int tickets = 0, sync_words = 0;
   for (int M = 1; M <= desc->max_M; ++M) {
     const int paths[4] = {VQ_PATH_LUT, VQ_PATH_GEMV, VQ_PATH_TC, VQ_PATH_GATHER};
     for (int pth : paths) {
@@ -231,6 +231,7 @@ VQ_API vq_status vq_linear_create(const vq_linear_desc* desc, vq_linear_t* out) 
       if (!vq::plan_forward(*desc, dev, M, pth, &p)) continue;
       if (p.scratch_bytes > need) need = p.scratch_bytes;
       if (p.tickets > tickets) tickets = p.tickets;
+      if (p.sync_words > sync_words) sync_words = p.sync_words;
     }
   }
   // Test hook: VQ_TEST_FAIL_ALLOC=1 makes the device allocations fail, so callers'
@@ -263,16 +264,16 @@ VQ_API vq_status vq_linear_create(const vq_linear_desc* desc, vq_linear_t* out) 
     }
   }
   h->num_tickets = tickets;
-  // words: [0] error flag, [1] pad, then (num_sms + 1) 64-bit barrier counters, then tickets
-  const size_t bar_words = 2 * ((size_t)dev.num_sms + 1);
-  const size_t small = sizeof(uint32_t) * (2 + bar_words + (size_t)tickets);
+  h->num_sync = sync_words;
+  // words: [0] error flag, [1] pad, then the tickets, then the table kernel's sync words
+  const size_t small = sizeof(uint32_t) * (2 + (size_t)tickets + (size_t)sync_words);
   uint32_t* words = nullptr;
   e = cudaMalloc(&words, small);
   if (e == cudaSuccess) e = cudaMemset(words, 0, small);
   if (e == cudaSuccess) e = cudaDeviceSynchronize();  // the zeroing is complete before any forward
   h->err = words;
-  h->gbar = words ? words + 2 : nullptr;
-  h->tickets = (words && tickets) ? words + 2 + bar_words : nullptr;
+  h->tickets = (words && tickets) ? words + 2 : nullptr;
+  h->sync = (words && sync_words) ? words + 2 + tickets : nullptr;
   if (e != cudaSuccess) {
     cudaFree(h->scratch);
     cudaFree(h->xrot);
@@ -288,9 +289,21 @@ VQ_API vq_status vq_linear_create(const vq_linear_desc* desc, vq_linear_t* out) 
 VQ_API vq_status vq_linear_destroy(vq_linear_t h) {
   if (h == nullptr) return VQ_OK;
   cudaError_t e1 = cudaSuccess, e2 = cudaSuccess;
+  // Wait for the handle's device to finish all enqueued work (a forward still in
+  // flight may read the scratch or the counters freed below), on that device.
+  int prev = -1;
+  e1 = cudaGetDevice(&prev);
+  if (e1 == cudaSuccess && prev != h->dev.device) e1 = cudaSetDevice(h->dev.device);
+  if (e1 == cudaSuccess) e1 = cudaDeviceSynchronize();
+  if (e1 != cudaSuccess) {
+    if (prev >= 0 && prev != h->dev.device) cudaSetDevice(prev);
+    delete h;  // the device memory is unreachable now; report the error
+    return cuda_fail(e1, "vq_linear_destroy: synchronising the handle's device");
+  }
   if (h->scratch) e1 = cudaFree(h->scratch);
   if (h->xrot && e1 == cudaSuccess) e1 = cudaFree(h->xrot);
-  if (h->err) e2 = cudaFree(h->err);  // also frees the barrier words and tickets (one allocation)
+  if (h->err) e2 = cudaFree(h->err);  // also frees the tickets and sync words (one allocation)
+  if (prev >= 0 && prev != h->dev.device) cudaSetDevice(prev);
   delete h;
   if (e1 != cudaSuccess) return cuda_fail(e1, "cudaFree(scratch)");
   if (e2 != cudaSuccess) return cuda_fail(e2, "cudaFree(err)");
@@ -340,9 +353,9 @@ VQ_API vq_status vq_linear_forward(vq_linear_t h, const void* x, const vq_planes
     return fail(VQ_ERR_UNSUPPORTED, "path %d cannot run M=%d", h->path, M);
   if ((p.path == VQ_PATH_LUT || p.path == VQ_PATH_GATHER) && h->sm_budget > 0 && p.grid > h->sm_budget)
     p.grid = h->sm_budget;
-  if (p.scratch_bytes > h->scratch_bytes || p.tickets > h->num_tickets)
-    return fail(VQ_ERR_UNSUPPORTED, "plan needs %zu scratch bytes / %d tickets, handle has %zu / %d",
-                p.scratch_bytes, p.tickets, h->scratch_bytes, h->num_tickets);
+  if (p.scratch_bytes > h->scratch_bytes || p.tickets > h->num_tickets || p.sync_words > h->num_sync)
+    return fail(VQ_ERR_UNSUPPORTED, "plan needs %zu scratch bytes / %d tickets / %d sync words, handle has %zu / %d / %d",
+                p.scratch_bytes, p.tickets, p.sync_words, h->scratch_bytes, h->num_tickets, h->num_sync);
   vq::LayerArgs a = make_args(d, planes, codebooks, scales);
   a.x = x;
   a.y = y;
@@ -350,7 +363,7 @@ VQ_API vq_status vq_linear_forward(vq_linear_t h, const void* x, const vq_planes
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e;
   switch (p.path) {
-    case VQ_PATH_LUT: e = vq::launch_lut(a, p, h->scratch, h->gbar, h->err, s); break;  // p.grid CTAs
+    case VQ_PATH_LUT: e = vq::launch_lut(a, p, h->scratch, h->sync, h->err, s); break;  // p.grid CTAs
     case VQ_PATH_GATHER: e = vq::launch_vq16(a, p, nullptr, s); break;
     case VQ_PATH_TC: e = vq::launch_tc(a, p, h->scratch, h->tickets, h->err, s); break;
     default: e = vq::launch_gemv(a, p, h->scratch, h->tickets, s); break;

@@ -40,6 +40,7 @@ struct Plan {
   int launches;      // kernels enqueued
   size_t scratch_bytes;
   int tickets;       // completion counters needed (zero between forwards)
+  int sync_words;    // words of the batch-1 table kernel's cross-CTA protocol (kept apart from the tickets)
   int grid;          // CTAs of the persistent batch-1 kernels (VQ_PATH_LUT / GATHER), else 0
 };
 
@@ -56,12 +57,11 @@ bool plan_forward(const vq_linear_desc& d, const DeviceInfo& dev, int M, int for
 // `tickets` are per-launch completion counters: zero before every forward, and
 // every forward leaves them zero again.
 cudaError_t launch_gemv(const LayerArgs& a, const Plan& p, float* scratch, uint32_t* tickets, cudaStream_t s);
-// `gbar` is the handle's array of grid-barrier arrival counters, one 64-bit word
-// per grid size (index = the launch's grid, up to the SM count): zero at create
-// and only ever incremented (each launch adds its grid size to its own word, so
-// every word stays a multiple of its grid size between launches, whatever grid
-// sizes other launches of the handle used).
-cudaError_t launch_lut(const LayerArgs& a, const Plan& p, float* scratch, uint32_t* gbar, uint32_t* err,
+// The batch-1 table kernel (p.grid CTAs).  `sync` is the handle's array of
+// p.sync_words words for its end-of-kernel protocol (an arrival counter, a
+// generation word and one claim word per 32-row unit): zero at create; every
+// forward leaves the counter at zero and every claim word equal to the generation.
+cudaError_t launch_lut(const LayerArgs& a, const Plan& p, float* scratch, uint32_t* sync, uint32_t* err,
                        cudaStream_t s);
 // The few-token kernel of the 16-bit formats (VQ_PATH_GATHER, clusters of 2
 // CTAs, no scratch); `signs` (may be NULL, M == 1 only) makes it rotate x itself

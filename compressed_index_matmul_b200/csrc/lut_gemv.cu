@@ -27,8 +27,8 @@
 // writes one fp32 partial sum per row and slice.
 //
 // Split-K reduction: after the last chunk every CTA meets at a grid-wide barrier
-// (all CTAs are resident: the grid never exceeds the SM count and a CTA takes a
-// whole SM's shared memory); then each CTA sums the partials of its own share
+// (the launch is cooperative, so all CTAs are resident together: the grid never
+// exceeds the SM count); then each CTA sums the partials of its own share
 // of the rows with a fixed tree (GLQ README, "Inference kernels": fixed-order
 // split-K reduction, no floating-point atomics), so y does not depend on
 // scheduling.  One launch per forward.
@@ -154,7 +154,7 @@ __device__ __forceinline__ void lookup_row(const uint4& lo4, const uint2& h, con
 
 template <int FMT, typename T>
 __global__ void __launch_bounds__(kLutThreads, 1)
-    lut_gemv_kernel(LayerArgs a, float* __restrict__ partial, uint32_t* __restrict__ gbar, uint32_t* __restrict__ err,
+    lut_gemv_kernel(LayerArgs a, float* __restrict__ partial, uint32_t* __restrict__ sync, uint32_t* __restrict__ err,
                     int S) {
   extern __shared__ __align__(128) unsigned char smem[];
   constexpr bool kTwo = (FMT == kFmtRvq12_4);
@@ -164,7 +164,6 @@ __global__ void __launch_bounds__(kLutThreads, 1)
   const uint32_t empty0 = smem_u32(smem + kLutOffMisc + 96);        // [kLutStages] mbarriers: chunk consumed
   volatile int* abortf = reinterpret_cast<volatile int*>(smem + kLutOffMisc + 128);  // a bounded wait gave up
   const uint32_t cb_bar = smem_u32(smem + kLutOffMisc + 136);       // codebook copy landed
-  volatile unsigned long long* bar_base = reinterpret_cast<volatile unsigned long long*>(smem + kLutOffMisc + 144);
   const uint32_t t1_base = smem_u32(t1), ring_base = smem_u32(smem + kLutOffRing);
 
   const int N = a.N;
@@ -236,16 +235,6 @@ __global__ void __launch_bounds__(kLutThreads, 1)
     // before the wait for the codebook copy, so the two latencies overlap.  Every
     // warp holds a whole x slice: lane l has inputs 4l .. 4l+3 of it.
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    if (tid == 0 && S > 1) {
-      // The grid-barrier counter of this grid size before any CTA of this launch
-      // arrives: the previous launch of this handle has completed.
-      unsigned long long v;
-      asm volatile("ld.relaxed.gpu.u64 %0, [%1];"
-                   : "=l"(v)
-                   : "l"(reinterpret_cast<unsigned long long*>(gbar) + gridDim.x)
-                   : "memory");
-      *bar_base = v;
-    }
     uint2 xpre[kLutMaxX];
 #pragma unroll
     for (int i = 0; i < kLutMaxX; ++i) {
@@ -399,28 +388,39 @@ __global__ void __launch_bounds__(kLutThreads, 1)
   }
 
   // --------------------------------------------------- grid barrier + reduce
-  // Each grid size has its own arrival counter, which only grows by whole grids:
-  // this launch's CTAs take it from `base` (read after the previous kernel
-  // completed) to base + grid.  The CTA barrier orders every thread's partial
-  // stores before thread 0's release add; thread 0's acquire load and the second
-  // CTA barrier order them before every thread's reads below.
+  // A self-resetting barrier on two handle words: an arrival counter and a
+  // generation.  Each CTA reads the generation before it arrives (it cannot
+  // change before every CTA of this launch, this one included, has arrived); the
+  // CTA whose arrival completes the grid zeroes the counter and advances the
+  // generation, and the others wait for that.  No CTA reads a count that other
+  // CTAs of the same launch may already have changed, whenever it started.  The
+  // CTA barrier orders every thread's partial stores before thread 0's arrival
+  // (release); thread 0's acquire and the second CTA barrier order all CTAs'
+  // partial stores before every thread's reads below.
   __syncthreads();
   if (tid == 0) {
-    unsigned long long* cnt = reinterpret_cast<unsigned long long*>(gbar) + gridDim.x;
-    const unsigned long long target = *bar_base + gridDim.x;
-    asm volatile("red.release.gpu.global.add.u64 [%0], 1;" ::"l"(cnt) : "memory");
-    const uint64_t t0 = ptx::globaltimer_ns();
-    bool released = false;
-    for (uint32_t i = 0; i < kWaitSpinLimit; ++i) {
-      unsigned long long v;
-      asm volatile("ld.acquire.gpu.u64 %0, [%1];" : "=l"(v) : "l"(cnt) : "memory");
-      if (v >= target) {
-        released = true;
-        break;
+    uint32_t* cnt = sync;
+    uint32_t* gen = sync + 1;
+    uint32_t g0, old;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(g0) : "l"(gen) : "memory");
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(cnt) : "memory");
+    if (old == gridDim.x - 1) {
+      *cnt = 0;  // every CTA has arrived: nothing else touches it in this launch
+      asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(gen), "r"(g0 + 1) : "memory");
+    } else {
+      const uint64_t t0 = ptx::globaltimer_ns();
+      bool released = false;
+      for (uint32_t i = 0; i < kWaitSpinLimit; ++i) {
+        uint32_t g;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(g) : "l"(gen) : "memory");
+        if (g != g0) {
+          released = true;
+          break;
+        }
+        if ((i & 63u) == 63u && ptx::globaltimer_ns() - t0 > 1000000000ull) break;
       }
-      if ((i & 63u) == 63u && ptx::globaltimer_ns() - t0 > 1000000000ull) break;
+      if (!released) atomicOr(err, kErrTimeout);
     }
-    if (!released) atomicOr(err, kErrTimeout);
   }
   __syncthreads();
   // Every CTA of this grid has passed the barrier, so all of them are resident:
@@ -509,13 +509,14 @@ bool plan_lut(const vq_linear_desc& d, const DeviceInfo& dev, int M, Plan* p) {
   p->k_per_split = kLutGroups * 8;
   p->launches = 1;
   p->scratch_bytes = g.S > 1 ? (size_t)g.S * d.N * sizeof(float) : 0;
-  p->tickets = 0;  // uses the handle's grid-barrier words instead
+  p->tickets = 0;
+  p->sync_words = g.S > 1 ? 2 : 0;  // the grid barrier's arrival counter and generation
   p->grid = g.grid;
   return true;
 }
 
 template <int FMT, typename T>
-static cudaError_t launch_lut_t(const LayerArgs& a, int grid, float* scratch, uint32_t* tickets, uint32_t* err,
+static cudaError_t launch_lut_t(const LayerArgs& a, int grid, float* scratch, uint32_t* sync, uint32_t* err,
                                 cudaStream_t s) {
   const int S = a.K / (8 * kLutGroups);
   auto kern = lut_gemv_kernel<FMT, T>;
@@ -536,21 +537,26 @@ static cudaError_t launch_lut_t(const LayerArgs& a, int grid, float* scratch, ui
   cfg.blockDim = dim3(kLutThreads);
   cfg.dynamicSmemBytes = kLutSmem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // prologue overlaps the previous kernel
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  // The CTAs meet at a grid barrier: a cooperative launch makes them all resident
+  // together even beside other work on the GPU (the grid never exceeds the SM
+  // count and a CTA takes a whole SM's shared memory).
+  attr[1].id = cudaLaunchAttributeCooperative;
+  attr[1].val.cooperative = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, a, S > 1 ? scratch : nullptr, tickets, err, S);
+  cfg.numAttrs = S > 1 ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, kern, a, S > 1 ? scratch : nullptr, sync, err, S);
 }
 
-cudaError_t launch_lut(const LayerArgs& a, const Plan& p, float* scratch, uint32_t* gbar, uint32_t* err,
+cudaError_t launch_lut(const LayerArgs& a, const Plan& p, float* scratch, uint32_t* sync, uint32_t* err,
                        cudaStream_t s) {
   if (a.fmt == kFmtRvq12_4)
-    return a.act == VQ_BF16 ? launch_lut_t<kFmtRvq12_4, __nv_bfloat16>(a, p.grid, scratch, gbar, err, s)
-                            : launch_lut_t<kFmtRvq12_4, __half>(a, p.grid, scratch, gbar, err, s);
-  return a.act == VQ_BF16 ? launch_lut_t<kFmtRvq12, __nv_bfloat16>(a, p.grid, scratch, gbar, err, s)
-                          : launch_lut_t<kFmtRvq12, __half>(a, p.grid, scratch, gbar, err, s);
+    return a.act == VQ_BF16 ? launch_lut_t<kFmtRvq12_4, __nv_bfloat16>(a, p.grid, scratch, sync, err, s)
+                            : launch_lut_t<kFmtRvq12_4, __half>(a, p.grid, scratch, sync, err, s);
+  return a.act == VQ_BF16 ? launch_lut_t<kFmtRvq12, __nv_bfloat16>(a, p.grid, scratch, sync, err, s)
+                          : launch_lut_t<kFmtRvq12, __half>(a, p.grid, scratch, sync, err, s);
 }
 
 }  // namespace vq

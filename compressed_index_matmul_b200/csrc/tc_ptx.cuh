@@ -66,6 +66,16 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
                : "memory");
 }
 
+// Prefetch [src, src + bytes) into L2 (bulk prefetches of at most 32 KiB; src
+// and bytes multiples of 16).  Nothing waits for them.
+__device__ __forceinline__ void prefetch_l2_range(const void* src, int64_t bytes) {
+  const char* p = static_cast<const char*>(src);
+  for (int64_t off = 0; off < bytes; off += 32768) {
+    const uint32_t n = (uint32_t)(bytes - off < 32768 ? bytes - off : 32768);
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p + off), "r"(n) : "memory");
+  }
+}
+
 // 2-D tiled tensor load (coordinates in elements, innermost first).
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int c0, int c1, uint32_t bar) {
   asm volatile(

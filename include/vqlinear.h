@@ -169,8 +169,11 @@ int32_t vq_abi_version(void);
  * Synchronous.  On error *out is set to NULL. */
 vq_status vq_linear_create(const vq_linear_desc* desc, vq_linear_t* out);
 
-/* Free the handle and its scratch.  Synchronises the device first so that no
- * enqueued forward still uses the scratch.  NULL is accepted (no-op). */
+/* Free the handle and its scratch.  Synchronises the handle's device first
+ * (cudaDeviceSynchronize with that device current; the caller's current device is
+ * restored) so that no enqueued forward still uses the scratch.  If that
+ * synchronisation fails the handle is released without freeing its device memory
+ * and VQ_ERR_CUDA is returned.  NULL is accepted (no-op). */
 vq_status vq_linear_destroy(vq_linear_t h);
 
 /* Force a kernel (VQ_PATH_*) for later forwards of this handle; VQ_PATH_AUTO
@@ -178,16 +181,14 @@ vq_status vq_linear_destroy(vq_linear_t h);
  * returns VQ_ERR_UNSUPPORTED. */
 vq_status vq_linear_set_path(vq_linear_t h, int32_t path);
 
-/* Limit the batch-1 table kernel (VQ_PATH_LUT) of this handle to `sms` CTAs, one
- * per SM; 0 restores the default (every SM).  That kernel keeps all of its CTAs
- * resident and meets them at a grid barrier, so it can share the GPU with another
- * forward only on disjoint SMs: two independent forwards (say the gate and up
- * projections of an MLP, both reading the same x) may run concurrently on two
- * streams when the sum of their budgets does not exceed the SM count.  With a
- * larger sum the barrier's bounded wait can give up (VQ_ERR_TIMEOUT from
- * vq_linear_check; y is then not valid).  The other kernels are not persistent
- * and ignore the budget.  Returns VQ_ERR_INVALID_ARG when `sms` is negative or
- * above the device's SM count. */
+/* Limit the persistent batch-1 kernels (VQ_PATH_LUT, VQ_PATH_GATHER) of this
+ * handle to `sms` CTAs, one per SM; 0 restores the default (every SM).  Two
+ * independent forwards (say the gate and up projections of an MLP, both reading
+ * the same x) can then run concurrently on two streams on about disjoint SMs.  No
+ * CTA of these kernels waits for another, so any budgets are correct; budgets
+ * that add up to more than the SM count only serialise part of the work.  The
+ * other kernels are not persistent and ignore the budget.  Returns
+ * VQ_ERR_INVALID_ARG when `sms` is negative or above the device's SM count. */
 vq_status vq_linear_set_sm_budget(vq_linear_t h, int32_t sms);
 
 /* y = x . W^T with W decoded on the fly from planes / codebooks / scales
