@@ -311,7 +311,7 @@ def _clone_layer(L):
 L2_NOTE = "inputs larger than L2: the step's weights are cycled over {r} copies ({mb:.0f} MB, >= 4x L2)"
 
 
-def capture_steps(wl, M, stream, evs=None):
+def capture_steps(wl, M, stream, evs=None, concurrent=True):
     """One CUDA graph per weight copy, each holding one step's forwards."""
     import torch
 
@@ -319,16 +319,16 @@ def capture_steps(wl, M, stream, evs=None):
     for r in range(len(wl.replicas)):
         calls = wl.plan(M, r)
         with torch.cuda.stream(stream):
-            wl.enqueue(calls, M)  # plain run: every call validated outside capture
+            wl.enqueue(calls, M, concurrent=concurrent)  # plain run: every call validated outside capture
         stream.synchronize()
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream, capture_error_mode="relaxed"):
-            wl.enqueue(calls, M, evs)
+            wl.enqueue(calls, M, evs, concurrent=concurrent)
         graphs.append(g)
     return graphs
 
 
-def capture_cycle(wl, M, stream):
+def capture_cycle(wl, M, stream, concurrent=True):
     """One CUDA graph holding one step on each weight copy in turn (R steps back to back)."""
     import torch
 
@@ -336,7 +336,7 @@ def capture_cycle(wl, M, stream):
     plans = [wl.plan(M, r) for r in range(len(wl.replicas))]
     with torch.cuda.graph(g, stream=stream, capture_error_mode="relaxed"):
         for calls in plans:
-            wl.enqueue(calls, M)
+            wl.enqueue(calls, M, concurrent=concurrent)
     return g
 
 
@@ -355,14 +355,54 @@ def run_steps(graphs, cycle, first, steps, stream):
             k += 1
 
 
-def time_graph(wl, M, steps, warmup, per_kernel=False):
+WARMUP_SECONDS = 0.5  # replays before any timed region, whatever --warmup is
+REGIONS = 5           # timed regions of exactly K steps each; the line reports their median
+
+
+def warm_up(graphs, cycle, stream, steps, seconds=WARMUP_SECONDS):
+    """`steps` untimed steps, then more whole cycles until `seconds` of wall time have passed
+    (clocks, L2 and TLB state settle before the first timed region).  Returns the next step index."""
+    import torch
+
+    with torch.cuda.stream(stream):
+        run_steps(graphs, cycle, 0, steps, stream)
+    stream.synchronize()
+    k = steps
+    R = len(graphs)
+    t_end = time.perf_counter() + seconds
+    while time.perf_counter() < t_end:
+        with torch.cuda.stream(stream):
+            start = -(-k // R) * R  # next cycle boundary
+            run_steps(graphs, cycle, k, start - k + R, stream)
+            k = start + R
+        stream.synchronize()
+    return k
+
+
+def timed_regions(graphs, cycle, stream, first, steps, regions):
+    """`regions` back-to-back event regions of exactly `steps` steps each; ms per region."""
+    import torch
+
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(regions + 1)]
+    with torch.cuda.stream(stream):
+        evs[0].record(stream)
+        k = first
+        for i in range(regions):
+            run_steps(graphs, cycle, k, steps, stream)
+            k += steps
+            evs[i + 1].record(stream)
+    stream.synchronize()
+    return [evs[i].elapsed_time(evs[i + 1]) for i in range(regions)]
+
+
+def time_graph(wl, M, steps, warmup, per_kernel=False, concurrent=True):
     """Replay the step graphs `steps` times (cycling the weight copies); per-step ms (and per-forward ms)."""
     import torch
 
     stream = torch.cuda.Stream()
     n = len(wl.plan(M))
     evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n + 1)] if per_kernel else None
-    graphs = capture_steps(wl, M, stream, evs)
+    graphs = capture_steps(wl, M, stream, evs, concurrent=concurrent)
     R = len(graphs)
     per_fwd = np.zeros(n) if per_kernel else None
     if per_kernel:  # one step at a time, events between the forwards
@@ -376,18 +416,11 @@ def time_graph(wl, M, steps, warmup, per_kernel=False):
                 per_fwd += np.array([evs[i].elapsed_time(evs[i + 1]) for i in range(n)])
         del graphs
         return None, per_fwd / steps
-    cycle = capture_cycle(wl, M, stream)
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        run_steps(graphs, cycle, 0, warmup, stream)
-        stream.synchronize()
-        t0.record(stream)
-        run_steps(graphs, cycle, warmup, steps, stream)
-        t1.record(stream)
-    stream.synchronize()
-    total = t0.elapsed_time(t1)
+    cycle = capture_cycle(wl, M, stream, concurrent=concurrent)
+    k = warm_up(graphs, cycle, stream, warmup, seconds=0.2)
+    region_ms = timed_regions(graphs, cycle, stream, k, steps, 3)
     del graphs, cycle
-    return [total / steps] * steps, None
+    return [statistics.median(region_ms) / steps] * steps, None
 
 
 def time_e2e(wl, M, steps, warmup):
@@ -461,14 +494,11 @@ def gpu_arm(args):
     wl = Workload(args.workload, max_M=max(M, 16))
     R = len(wl.replicas)
 
-    # ------------------------------------------------ timed region (exactly K steps)
+    # ------------------------------------------------ timed regions (exactly K steps each)
     stream = torch.cuda.Stream()
     graphs = capture_steps(wl, M, stream)
     cycle = capture_cycle(wl, M, stream)
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        run_steps(graphs, cycle, 0, args.warmup, stream)
-    stream.synchronize()
+    first = warm_up(graphs, cycle, stream, args.warmup)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -476,49 +506,44 @@ def gpu_arm(args):
     ids = [v for v in vis.split(",") if v.strip()]
     smi_index = int(ids[local]) if local < len(ids) and ids[local].strip().isdigit() else local
     with ClockSampler(smi_index) as clk:
-        with torch.cuda.stream(stream):
-            t0.record(stream)
-            run_steps(graphs, cycle, args.warmup, args.steps, stream)
-            t1.record(stream)
+        region_ms = timed_regions(graphs, cycle, stream, first, args.steps, args.regions)
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     del graphs, cycle
-    step_ms = [t0.elapsed_time(t1) / args.steps] * args.steps
     layers = len(wl.layers)
-    ms_per_step, us_per_layer = aggregate_over_ranks(float(sum(step_ms)), args.steps, layers, world)
+    ms_per_step, us_per_layer = aggregate_over_ranks(float(statistics.median(region_ms)), args.steps, layers, world)
 
-    # ------------------------------------------------ per-kernel roofline (same stream, graph nodes)
-    _, per_fwd = time_graph(wl, M, min(args.steps, 200), 3, per_kernel=True)
+    # ------------------------------------------------ per-launch roofline (same stream)
+    _, per_fwd = time_graph(wl, M, min(args.steps, 200), 3, per_kernel=True)  # event nodes between forwards
     launches_per_fwd = [L.launches(M) for _, _, L in wl.layers]
     bytes_per_fwd = [layer_bytes(spec, M) for _, spec, _ in wl.layers]
-    # When every forward of the timed region runs the same kernels (no rotation
-    # launch), the region's time per forward is a forward's average duration; else
-    # use the event nodes captured between the forwards (which include the gaps).
-    # The batch-1 table path is two kernels per forward (lookups, then the split-K
-    # reduction) that overlap by programmatic dependent launch, so the forward,
-    # not either kernel alone, is the unit its bytes are divided by.
+    # When every forward runs the same single kernel (no rotation launch), a region's
+    # time per launch is that kernel's average duration; else use the event nodes
+    # captured between the forwards (which include the gaps).  A step that overlaps
+    # gate and up has no such per-launch time, so the same forwards are timed one after
+    # another (each with every SM) in a region of their own for the roofline.
     fused = all(wl.rotation_fused(spec, M) for _, spec, _ in wl.layers)
     uniform = (not wl.rht or fused) and len(set(launches_per_fwd)) == 1
-    fwd_ms = ms_per_step / len(wl.layers) if uniform else float(np.mean(per_fwd))
-    per_fwd_eff = [fwd_ms] * len(wl.layers) if uniform else list(per_fwd)
+    if uniform and wl.concurrent_gate_up:
+        fwd_ms = time_graph(wl, M, args.steps, args.warmup, concurrent=False)[0][0] / len(wl.layers)
+        launch_source = ("a separate region of K steps with the forwards one after another on one stream, every "
+                         "SM each (every launch is this kernel) / launches")
+    elif uniform:
+        fwd_ms = ms_per_step / len(wl.layers)
+        launch_source = ("timed region / launches (every launch is this kernel)" if launches_per_fwd[0] == 1 else
+                         "timed region / forwards")
+    else:
+        fwd_ms = float(np.mean(per_fwd))
+        launch_source = "CUDA event nodes between the forwards"
+    per_fwd_eff = [fwd_ms / max(1, launches_per_fwd[0]) if uniform else fwd_ms] * len(wl.layers)
     achieved = sum(bytes_per_fwd) / (sum(per_fwd_eff) * 1e-3) / 1e9
     fmt0 = wl.layers[0][1].fmt
     dominant = ("lut_gemv_kernel" if M == 1 and fmt0 not in _16BIT else
                 "vq16_gemv_kernel" if M == 1 else "gemv_kernel" if M <= 16 else "tc_gemm_kernel")
     traffic = lookup_traffic(dominant, args.workload, M)
     avg_launch_us = round(1e3 * float(np.mean(per_fwd_eff)), 3)
-    if not uniform:
-        launch_source = "CUDA event nodes between the forwards"
-    elif launches_per_fwd[0] == 1 and wl.concurrent_gate_up:
-        launch_source = ("timed region / forwards (every launch is this kernel; gate and up overlap on two "
-                         "streams, so this is the step's time per weight matrix)")
-    elif launches_per_fwd[0] == 1:
-        launch_source = "timed region / launches (every launch is this kernel)"
-    else:
-        launch_source = ("timed region / forwards (one forward = lut_gemv_kernel + lut_reduce_kernel, "
-                         "overlapped by programmatic dependent launch)")
     if dominant == "tc_gemm_kernel":
         # a dense contraction: 2*M*N*K flops per forward against the bf16 tensor peak
         flops_per_fwd = [2.0 * M * spec.N * spec.K for _, spec, _ in wl.layers]
@@ -542,11 +567,18 @@ def gpu_arm(args):
     # ------------------------------------------------ end to end through the public API
     e2e_ms, h2d, d2h = time_e2e(wl, M, min(args.steps, 200), 3)
     e2e = {"value": round(1e3 * statistics.fmean(e2e_ms) / layers, 3), "unit": "us/layer",
-           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+           "how": "per step: pinned-host x -> device copy, the forwards as eager C-ABI calls one after another "
+                  "on one stream, y -> pinned host; timed by CUDA events on that stream"}
 
     out = {
         "metric": METRIC, "value": round(us_per_layer, 3), "unit": "us/layer", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+        "timing": {"regions": args.regions, "steps_per_region": args.steps,
+                   "region_ms_per_step": [round(v / args.steps, 5) for v in region_ms],
+                   "spread": round((max(region_ms) - min(region_ms)) / statistics.median(region_ms), 4),
+                   "warmup": f"{args.warmup} steps, then whole weight-copy cycles until {WARMUP_SECONDS} s of "
+                             "replays; value = the median region"},
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded; uniform indices, N(0,1) codebooks and activations, lognormal scales)",
         "config": {"workload": args.workload, "M": M, "layers_per_step": layers,
@@ -625,12 +657,13 @@ def lookup_traffic(kernel, workload, M):
 
 
 def detail(args, peaks, main_wl):
-    """The rest of the metric: batch 16 of the headline workload and the other workloads."""
+    """The rest of the metric: the other batch sizes of the headline workload and every
+    other workload at each of its M, the rotations and the encoder."""
     steps = max(10, min(args.steps, 300))
     res = {}
-    r = measure(main_wl, 16, steps, 3, peaks)
-    res[f"{args.workload} M=16"] = r
-    for name, Ms in (("smollm-135m-stack", (1, 16)), ("vq16-4096-rht", (1, 8))):
+    for M in (4, 16):
+        res[f"{args.workload} M={M}"] = measure(main_wl, M, steps, 3, peaks)
+    for name, Ms in (("single-256", (1,)), ("smollm-135m-stack", (1, 4, 16)), ("vq16-4096-rht", (1, 8))):
         if name == args.workload:
             continue
         wl = Workload(name, max_M=16)
@@ -640,17 +673,21 @@ def detail(args, peaks, main_wl):
                 r["us_per_transformer_layer"] = 1e3 * r["ms_per_step"] / 30
             res[f"{name} M={M}"] = r
         del wl
-    try:
-        wl = Workload("prefill-8192", max_M=256)
-        wl.plan(256)
-        r = measure(wl, 256, max(5, steps // 10), 2, peaks, with_kernels=False)
-        r["tensor_frac"] = r["tflops"] / peaks["bf16_tflops"]
-        r["tensor_frac_sustained"] = r["tflops"] / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
-        res["prefill-8192 M=256"] = r
-    except Exception as exc:  # the tensor-core path reports why it could not run
-        res["prefill-8192 M=256"] = {"error": str(exc)[:300]}
+    if args.workload != "prefill-8192":
+        try:
+            wl = Workload("prefill-8192", max_M=1024)
+            for M in (64, 256, 1024):
+                r = measure(wl, M, max(5, steps // 10), 3, peaks, with_kernels=False)
+                r["tensor_frac"] = r["tflops"] / peaks["bf16_tflops"]
+                r["tensor_frac_sustained"] = r["tflops"] / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+                res[f"prefill-8192 M={M}"] = r
+            del wl
+        except Exception as exc:  # the tensor-core path reports why it could not run
+            res["prefill-8192"] = {"error": str(exc)[:300]}
     for M in (1, 8):
         res[f"rotation 4096 M={M}"] = time_rotations(4096, M, steps)
+        for label, shards in (("qkv 4096+1024+1024", (4096, 1024, 1024)), ("gate-up 14336+14336", (14336, 14336))):
+            res[f"sharded output rotation {label} M={M}"] = time_sharded_rotation(shards, M, steps)
     for bpw in (3, 4, 5):  # the residual ladder
         name = f"vq16-ladder-4096-{bpw}bpw"
         if name == args.workload:
@@ -659,11 +696,92 @@ def detail(args, peaks, main_wl):
         for M in (1, 8):
             res[f"{name} M={M}"] = measure(wl, M, steps, 3, peaks)
         del wl
+    from synth import FMT_RVQ12_4
+    for fmt, sg, label in ((FMT_RVQ12_4, 64, "rvq12_4 block-64"), (FMT_VQ16, 4096, "vq16 per-row")):
+        res[f"encode 4096x4096 {label}"] = time_encoder(LayerSpec(4096, 4096, fmt, sg))
     for v in res.values():
         for k in list(v):
             if isinstance(v[k], float):
                 v[k] = round(v[k], 4)
     return res
+
+
+def time_sharded_rotation(shards, M, steps):
+    """Device time per launch of the shard-batched output rotation (vq_rht_apply_output_sharded):
+    every column shard of an [M, sum(shards)] fp16 output rotated with its own signs."""
+    import torch
+
+    import compressed_index_matmul_b200 as vq
+
+    N = int(sum(shards))
+    y = torch.from_numpy(make_x(M, N, DT_F16, cfg_id=3).view(np.int16)).cuda().view(torch.float16)
+    sg = torch.from_numpy(make_signs(N, cfg_id=3)).cuda()
+    out = torch.empty_like(y)
+    stream = torch.cuda.Stream()
+    reps = 20
+    with torch.cuda.stream(stream):
+        vq.vq_rht_apply_output_sharded(y, out, sg, M, N, shards, DT_F16, stream.cuda_stream)
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for _ in range(reps):
+                vq.vq_rht_apply_output_sharded(y, out, sg, M, N, shards, DT_F16, stream.cuda_stream)
+        g.replay()
+        stream.synchronize()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(max(1, steps // reps)):
+            g.replay()
+        t1.record(stream)
+    torch.cuda.synchronize()
+    us = 1e3 * t0.elapsed_time(t1) / (reps * max(1, steps // reps))
+    return {"M": M, "shards": list(shards), "us_per_launch": us, "launches": 1}
+
+
+def time_encoder(spec, calls=5):
+    """Device time of one nearest-entry encode (vq_encode) of a dense binary32 N x K matrix into
+    the planes of `spec` (an encoder runs once per layer, off the forward path)."""
+    import torch
+
+    import compressed_index_matmul_b200 as vq
+
+    layer = make_layer(spec, cfg_id=143, tensor_id=spec.fmt)
+    N, K, G = spec.N, spec.K, spec.K // 8
+    w = (torch.randn((N, K), generator=torch.Generator().manual_seed(143), dtype=torch.float32) * 0.02).cuda()
+    out = {}
+    if spec.fmt == FMT_VQ16:
+        out["idx16"] = torch.zeros(N * G, dtype=torch.int16, device="cuda")
+    else:
+        out["lo"] = torch.zeros(N * G, dtype=torch.uint8, device="cuda")
+        out["hi4"] = torch.zeros(N * G // 2, dtype=torch.uint8, device="cuda")
+        if "cb2" in layer:
+            out["s2"] = torch.zeros(N * G // 2, dtype=torch.uint8, device="cuda")
+
+    def dev(a):
+        a = np.ascontiguousarray(a)
+        return torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a).cuda()
+
+    cb1, cb2 = dev(layer["cb1"]), (dev(layer["cb2"]) if "cb2" in layer else None)
+    sc = dev(layer["scales"])
+    cbs = vq.make_codebooks(cb1, cb2)
+
+    def once():
+        vq.vq_encode(N, K, spec.fmt, spec.scale_group, w, sc, cbs, out.get("lo"), out.get("hi4"), out.get("s2"),
+                     out.get("idx16"))
+
+    once()
+    torch.cuda.synchronize()
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(calls + 1)]
+    evs[0].record()
+    for i in range(calls):
+        once()
+        evs[i + 1].record()
+    torch.cuda.synchronize()
+    ms = [evs[i].elapsed_time(evs[i + 1]) for i in range(calls)]
+    med = statistics.median(ms)
+    entries = 65536 if spec.fmt == FMT_VQ16 else 4096 + (16 if "cb2" in layer else 0)
+    return {"N": N, "K": K, "ms_per_encode": med, "groups_per_s": N * G / (med * 1e-3),
+            "distances_per_s": N * G * entries / (med * 1e-3), "calls": calls}
 
 
 def time_rotations(K, M, steps):
@@ -843,6 +961,8 @@ def main():
     ap.add_argument("--no-detail", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--regions", type=int, default=REGIONS,
+                    help="timed regions of exactly K steps each (the line reports their median)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
