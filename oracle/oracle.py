@@ -75,6 +75,12 @@ def _load():
             lib.vqo_forward.argtypes = [I, I, I, I, P, I, P, P, P, P, P, P, P, I, P, I, P]
             lib.vqo_rht.restype = I
             lib.vqo_rht.argtypes = [I, I, P, I, P, P]
+            lib.vqo_corr_check.restype = I
+            lib.vqo_corr_check.argtypes = [I, I, P, P]
+            lib.vqo_dequant_corr.restype = I
+            lib.vqo_dequant_corr.argtypes = [I, I, I, P, P, P, P, P, P, P, I, P, P, P, P, I, P, P, I]
+            lib.vqo_forward_corr.restype = I
+            lib.vqo_forward_corr.argtypes = [I, I, I, I, P, I, P, P, P, P, P, P, P, I, P, P, P, P, I, P]
             lib.vqo_encode.restype = I
             lib.vqo_encode.argtypes = [I, I, I, P, P, I, P, P, P, P, P, P]
             lib.vqo_dist32.restype = ctypes.c_double
@@ -187,11 +193,29 @@ def dequant(layer, wdt: int = DT_F16, rows=None) -> tuple[np.ndarray, np.ndarray
     n = spec.N if r is None else nr
     w = np.empty((n, spec.K), dtype=np.float64)
     wb = np.empty((n, spec.K), dtype=np.uint16)
-    rc = lib.vqo_dequant(spec.fmt, spec.N, spec.K, _p(lo), _p(hi4), _p(s2), _p(idx16), _p(cb1), _p(cb2),
-                         _p(sc), spec.scale_group, _p(r), nr, _p(w), _p(wb), wdt)
+    if "corr" in layer:  # the sparse correction (orka README, "How it works")
+        rp, cl, vl = _corr(layer)
+        rc = lib.vqo_dequant_corr(spec.fmt, spec.N, spec.K, _p(lo), _p(hi4), _p(s2), _p(idx16), _p(cb1), _p(cb2),
+                                  _p(sc), spec.scale_group, _p(rp), _p(cl), _p(vl), _p(r), nr, _p(w), _p(wb), wdt)
+    else:
+        rc = lib.vqo_dequant(spec.fmt, spec.N, spec.K, _p(lo), _p(hi4), _p(s2), _p(idx16), _p(cb1), _p(cb2),
+                             _p(sc), spec.scale_group, _p(r), nr, _p(w), _p(wb), wdt)
     if rc:
         raise ValueError(f"vqo_dequant failed rc={rc}")
     return w, wb
+
+
+def _corr(layer):
+    """The sparse correction of a layer dict in the oracle's calling form (CSR by output row)."""
+    c = layer["corr"]
+    if layer["spec"].fmt == FMT_VQ16_RVQ:
+        raise ValueError("the sparse correction is defined for the 12-bit and 16-bit formats only")
+    return _c(c["row_ptr"], np.int32), _c(c["col"], np.int32), _c(c["val"], np.uint16)
+
+
+def corr_check(N: int, K: int, row_ptr, col) -> int:
+    """0 if (row_ptr, col) is a valid correction layout for an N x K layer, else nonzero."""
+    return _load().vqo_corr_check(N, K, _p(_c(row_ptr, np.int32)), _p(_c(col, np.int32)))
 
 
 def dist32(w8, s, c8) -> float:
@@ -252,8 +276,14 @@ def forward(layer, x_bits, xdt: int, rows=None) -> np.ndarray:
         return y
     lo, hi4, s2, idx16 = _planes(layer)
     cb1, cb2, sc = _c(layer["cb1"], np.uint16), _c(layer.get("cb2"), np.uint16), _c(layer["scales"], np.uint16)
-    rc = lib.vqo_forward(spec.fmt, M, spec.N, spec.K, _p(x), xdt, _p(lo), _p(hi4), _p(s2), _p(idx16), _p(cb1),
-                         _p(cb2), _p(sc), spec.scale_group, _p(r), nr, _p(y))
+    if "corr" in layer:  # y = x (W + C)^T with the sparse correction C
+        rp, cl, vl = _corr(layer)
+        rc = lib.vqo_forward_corr(spec.fmt, M, spec.N, spec.K, _p(x), xdt, _p(lo), _p(hi4), _p(s2), _p(idx16),
+                                  _p(cb1), _p(cb2), _p(sc), spec.scale_group, _p(rp), _p(cl), _p(vl), _p(r), nr,
+                                  _p(y))
+    else:
+        rc = lib.vqo_forward(spec.fmt, M, spec.N, spec.K, _p(x), xdt, _p(lo), _p(hi4), _p(s2), _p(idx16),
+                             _p(cb1), _p(cb2), _p(sc), spec.scale_group, _p(r), nr, _p(y))
     if rc:
         raise ValueError(f"vqo_forward failed rc={rc}")
     return y

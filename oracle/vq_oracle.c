@@ -18,6 +18,8 @@
  *   - GLQ README, "Bit widths": the residual ladder (16-bit primary, 16-bit
  *     residual stages, one 8-bit stage for odd bit widths), vqo_ladder_*.
  *   - orka README, "How it works": encode = nearest entry per group, vqo_encode.
+ *   - orka README, "How it works": the decode's "(+ sparse correction)", a sparse
+ *     matrix added to the decoded weights, vqo_dequant_corr / vqo_forward_corr.
  *
  * Readings taken where the pages are silent (all fixed here, by construction):
  *   - groups run along K (the input dimension), G = K/8 groups per row;
@@ -225,35 +227,82 @@ static int vqo_check(int fmt, int N, int K, int scale_group) {
   return 0;
 }
 
+/* ---------------------------------------------------------------------------
+ * Sparse correction (orka README, "How it works": the decode line is
+ * "scale x sum(codebook[index]) (+ sparse correction)"; the CLI's `correct`
+ * adds a sparse correction to an artifact).  Reading: a sparse N x K matrix C
+ * added to the decoded weights, W' = s * (c1 + c2) + C, stored by output row:
+ * the entries of row n are j = row_ptr[n] .. row_ptr[n+1] - 1, at columns
+ * col[j] in [0, K), strictly increasing within a row, with fp16 values val[j].
+ * The materialised weight takes one more fp32 rounding:
+ * RN(fl32(fl32(s * fl32(c1 + c2)) + C[n][k])).  row_ptr == NULL: no correction.
+ * ------------------------------------------------------------------------- */
+int vqo_corr_check(int N, int K, const int32_t* row_ptr, const int32_t* col) {
+  if (!row_ptr) return 0;
+  if (row_ptr[0] != 0) return 1;
+  for (int n = 0; n < N; ++n) {
+    if (row_ptr[n + 1] < row_ptr[n]) return 1;
+    for (int32_t j = row_ptr[n]; j < row_ptr[n + 1]; ++j) {
+      if (col[j] < 0 || col[j] >= K) return 1;
+      if (j > row_ptr[n] && col[j] <= col[j - 1]) return 1;
+    }
+  }
+  return 0;
+}
+
 /* rows: the output rows to decode (NULL = all N); outputs are [nrows][K]. */
-int vqo_dequant(int fmt, int N, int K, const uint8_t* lo, const uint8_t* hi4, const uint8_t* s2,
-                const uint16_t* idx16, const uint16_t* cb1, const uint16_t* cb2, const uint16_t* scales,
-                int scale_group, const int32_t* rows, int nrows, double* w_exact, uint16_t* w_bits, int wdt) {
+static int vqo_dequant_impl(int fmt, int N, int K, const uint8_t* lo, const uint8_t* hi4, const uint8_t* s2,
+                            const uint16_t* idx16, const uint16_t* cb1, const uint16_t* cb2, const uint16_t* scales,
+                            int scale_group, const int32_t* row_ptr, const int32_t* col, const uint16_t* val,
+                            const int32_t* rows, int nrows, double* w_exact, uint16_t* w_bits, int wdt) {
   int rc = vqo_check(fmt, N, K, scale_group);
   if (rc) return rc;
+  if ((rc = vqo_corr_check(N, K, row_ptr, col))) return rc;
   if (!rows) nrows = N;
   const int G = K / 8;
   uint32_t* i1 = (uint32_t*)malloc(sizeof(uint32_t) * (size_t)G);
   uint8_t* i2 = (uint8_t*)malloc((size_t)G);
-  if (!i1 || !i2) { free(i1); free(i2); return 3; }
+  double* corr = (double*)calloc((size_t)K, sizeof(double));
+  if (!i1 || !i2 || !corr) { free(i1); free(i2); free(corr); return 3; }
   for (int t = 0; rc == 0 && t < nrows; ++t) {
     const int n = rows ? rows[t] : t;
     if (n < 0 || n >= N) { rc = 1; break; }
     rc = vqo_unpack_row(fmt, n, N, K, lo, hi4, s2, idx16, i1, i2);
+    if (row_ptr)
+      for (int32_t j = row_ptr[n]; j < row_ptr[n + 1]; ++j) corr[col[j]] = vqo_f16_to_f64(val[j]);
     for (int k = 0; rc == 0 && k < K; ++k) {
       double c, s;
       double w = vqo_weight_exact(fmt, n, k, N, K, i1, i2, cb1, cb2, scales, scale_group, &c, &s);
-      if (w_exact) w_exact[(int64_t)t * K + k] = w;
+      if (w_exact) w_exact[(int64_t)t * K + k] = w + corr[k];
       if (w_bits) {
         double c32 = vqo_fl32(c);       /* stage sum rounded to fp32 */
         double p32 = vqo_fl32(s * c32); /* exact product of two fp32-representable values, rounded */
+        if (corr[k] != 0.0) p32 = vqo_fl32(p32 + corr[k]); /* the correction, one more fp32 rounding */
         w_bits[(int64_t)t * K + k] = wdt == VQO_DT_BF16 ? vqo_f64_to_bf16(p32) : vqo_f64_to_f16(p32);
       }
     }
+    if (row_ptr)
+      for (int32_t j = row_ptr[n]; j < row_ptr[n + 1]; ++j) corr[col[j]] = 0.0;
   }
   free(i1);
   free(i2);
+  free(corr);
   return rc;
+}
+
+int vqo_dequant(int fmt, int N, int K, const uint8_t* lo, const uint8_t* hi4, const uint8_t* s2,
+                const uint16_t* idx16, const uint16_t* cb1, const uint16_t* cb2, const uint16_t* scales,
+                int scale_group, const int32_t* rows, int nrows, double* w_exact, uint16_t* w_bits, int wdt) {
+  return vqo_dequant_impl(fmt, N, K, lo, hi4, s2, idx16, cb1, cb2, scales, scale_group, NULL, NULL, NULL, rows,
+                          nrows, w_exact, w_bits, wdt);
+}
+
+int vqo_dequant_corr(int fmt, int N, int K, const uint8_t* lo, const uint8_t* hi4, const uint8_t* s2,
+                     const uint16_t* idx16, const uint16_t* cb1, const uint16_t* cb2, const uint16_t* scales,
+                     int scale_group, const int32_t* row_ptr, const int32_t* col, const uint16_t* val,
+                     const int32_t* rows, int nrows, double* w_exact, uint16_t* w_bits, int wdt) {
+  return vqo_dequant_impl(fmt, N, K, lo, hi4, s2, idx16, cb1, cb2, scales, scale_group, row_ptr, col, val, rows,
+                          nrows, w_exact, w_bits, wdt);
 }
 
 /* ---------------------------------------------------------------------------
@@ -262,12 +311,13 @@ int vqo_dequant(int fmt, int N, int K, const uint8_t* lo, const uint8_t* hi4, co
  * exactly from its fp16/bf16 bits, a naive loop over k in order.  rows == NULL
  * means every row (nrows = N); y is [M][nrows].
  * ------------------------------------------------------------------------- */
-int vqo_forward(int fmt, int M, int N, int K, const uint16_t* x, int xdt, const uint8_t* lo,
-                const uint8_t* hi4, const uint8_t* s2, const uint16_t* idx16, const uint16_t* cb1,
-                const uint16_t* cb2, const uint16_t* scales, int scale_group, const int32_t* rows, int nrows,
-                double* y) {
+static int vqo_forward_impl(int fmt, int M, int N, int K, const uint16_t* x, int xdt, const uint8_t* lo,
+                            const uint8_t* hi4, const uint8_t* s2, const uint16_t* idx16, const uint16_t* cb1,
+                            const uint16_t* cb2, const uint16_t* scales, int scale_group, const int32_t* row_ptr,
+                            const int32_t* col, const uint16_t* val, const int32_t* rows, int nrows, double* y) {
   int rc = vqo_check(fmt, N, K, scale_group);
   if (rc || M < 0) return rc ? rc : 1;
+  if ((rc = vqo_corr_check(N, K, row_ptr, col))) return rc;
   if (!rows) nrows = N;
   const int G = K / 8;
   uint32_t* i1 = (uint32_t*)malloc(sizeof(uint32_t) * (size_t)G);
@@ -284,6 +334,8 @@ int vqo_forward(int fmt, int M, int N, int K, const uint16_t* x, int xdt, const 
       double c, s;
       wrow[k] = vqo_weight_exact(fmt, n, k, N, K, i1, i2, cb1, cb2, scales, scale_group, &c, &s);
     }
+    if (row_ptr) /* W' = W + C on this row */
+      for (int32_t j = row_ptr[n]; j < row_ptr[n + 1]; ++j) wrow[col[j]] += vqo_f16_to_f64(val[j]);
     for (int m = 0; rc == 0 && m < M; ++m) {
       double acc = 0.0;
       for (int k = 0; k < K; ++k) acc += xd[(int64_t)m * K + k] * wrow[k];
@@ -295,6 +347,21 @@ int vqo_forward(int fmt, int M, int N, int K, const uint16_t* x, int xdt, const 
   free(wrow);
   free(xd);
   return rc;
+}
+
+int vqo_forward(int fmt, int M, int N, int K, const uint16_t* x, int xdt, const uint8_t* lo, const uint8_t* hi4,
+                const uint8_t* s2, const uint16_t* idx16, const uint16_t* cb1, const uint16_t* cb2,
+                const uint16_t* scales, int scale_group, const int32_t* rows, int nrows, double* y) {
+  return vqo_forward_impl(fmt, M, N, K, x, xdt, lo, hi4, s2, idx16, cb1, cb2, scales, scale_group, NULL, NULL, NULL,
+                          rows, nrows, y);
+}
+
+int vqo_forward_corr(int fmt, int M, int N, int K, const uint16_t* x, int xdt, const uint8_t* lo,
+                     const uint8_t* hi4, const uint8_t* s2, const uint16_t* idx16, const uint16_t* cb1,
+                     const uint16_t* cb2, const uint16_t* scales, int scale_group, const int32_t* row_ptr,
+                     const int32_t* col, const uint16_t* val, const int32_t* rows, int nrows, double* y) {
+  return vqo_forward_impl(fmt, M, N, K, x, xdt, lo, hi4, s2, idx16, cb1, cb2, scales, scale_group, row_ptr, col,
+                          val, rows, nrows, y);
 }
 
 /* ---------------------------------------------------------------------------

@@ -29,6 +29,9 @@ Storage format (the encoder's output, consumed by both implementations):
   in K-slice-major order like the planes (a row's scales of one slice are
   adjacent); ``scale_group == K`` is one scale per row, [N]
 * ``x`` fp16 or bf16 [M, K]; ``signs`` int8 [K] of +-1 for the input rotation
+* ``corr`` (optional, ``make_correction``): a sparse correction by output row,
+  ``row_ptr`` int32 [N+1], ``col`` int32 [nnz] (increasing within a row),
+  ``val`` fp16 [nnz] (orka README, "How it works": "(+ sparse correction)")
 
 fp16/bf16 arrays are returned as raw uint16 bit patterns.
 """
@@ -42,6 +45,7 @@ from .layers import (  # noqa: F401
     DT_BF16,
     LayerSpec,
     make_layer,
+    make_correction,
     make_x,
     make_signs,
     f32_to_bf16_bits,

@@ -109,6 +109,23 @@ def make_layer(spec: LayerSpec, cfg_id: int = 0, layer: int = 0, tensor_id: int 
     return out
 
 
+def make_correction(N: int, K: int, density: float = 0.002, cfg_id: int = 0, layer: int = 0, tensor_id: int = 0,
+                    seed: int = 0, scale: float = 0.05) -> dict:
+    """A sparse correction sidecar for an N x K layer (orka README, "How it works": the
+    decode's "(+ sparse correction)"), by output row: row n's entries are
+    row_ptr[n] .. row_ptr[n+1]-1, with distinct columns in increasing order and fp16
+    values.  Each weight is corrected with probability `density`; values ~ N(0, scale^2),
+    a few times the synthetic layers' decoded weights, as corrections of outliers are."""
+    r = _rng(cfg_id, layer, tensor_id, seed, stream=7)
+    counts = r.binomial(K, density, size=N).astype(np.int64)
+    row_ptr = np.zeros(N + 1, dtype=np.int32)
+    row_ptr[1:] = np.cumsum(counts)
+    cols = [np.sort(r.choice(K, size=int(c), replace=False)) for c in counts]
+    col = (np.concatenate(cols) if N else np.zeros(0)).astype(np.int32)
+    val = f32_to_f16_bits((r.standard_normal(int(row_ptr[-1])) * scale).astype(np.float32))
+    return {"row_ptr": row_ptr, "col": col, "val": val}
+
+
 def make_x(M: int, K: int, dtype: int, cfg_id: int = 0, seed: int = 0, stream: int = 1) -> np.ndarray:
     """Activations [M, K] ~ N(0, 1) as fp16 or bf16 bits."""
     r = _rng(cfg_id, 1_000_000, M, seed, stream)

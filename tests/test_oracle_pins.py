@@ -15,6 +15,7 @@ import scipy.linalg
 import torch
 
 from synth import (FMT_RVQ12, FMT_RVQ12_4, FMT_VQ16, FMT_VQ16_RVQ, DT_BF16, DT_F16, LayerSpec, f32_to_bf16_bits,
+                   make_correction,
                    make_layer, make_x)
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
@@ -752,3 +753,104 @@ def test_two_sided_rotation_end_to_end(oracle):
     W_hat = R_out @ W @ R_in.T
     y = oracle.rht_out_f64(oracle.rht_f64(x, s_in) @ W_hat.T, s_out)
     assert np.allclose(y, x @ W.T, atol=1e-12)
+
+
+# --------------------------------------------------------------------------- sparse correction
+# orka README, "How it works": decode = scale x sum(codebook[index]) (+ sparse correction).
+# Reading: W' = W + C with C sparse, by output row (CSR); materialised weights take one more
+# fp32 rounding, RN(fl32(fl32(s * fl32(c1 + c2)) + C)).
+
+def _csr(N, entries):
+    """(row, col, value) triples -> the CSR arrays, rows in order."""
+    entries = sorted(entries)
+    row_ptr = np.zeros(N + 1, np.int32)
+    for n, _, _ in entries:
+        row_ptr[n + 1:] += 1
+    col = np.array([c for _, c, _ in entries], np.int32)
+    val = np.array([v for _, _, v in entries], np.float16).view(np.uint16)
+    return {"row_ptr": row_ptr, "col": col, "val": val}
+
+
+def _dense_corr(corr, N, K):
+    C = np.zeros((N, K))
+    for n in range(N):
+        for j in range(corr["row_ptr"][n], corr["row_ptr"][n + 1]):
+            C[n, corr["col"][j]] += float(corr["val"][j:j + 1].view(np.float16)[0])
+    return C
+
+
+def test_correction_by_hand(oracle):
+    """Two rows of 16 weights, every codeword 1.0 except entry 0 (dims 0..7 = 0..7), scale 0.5;
+    corrections (0, 3, +0.25), (1, 0, -2.0), (1, 15, +0.5)."""
+    cb1 = np.ones((4096, 8), np.float16)
+    cb1[0] = np.arange(8)
+    i1 = np.array([[0, 1], [1, 0]], np.uint32)  # row 0: groups (entry 0, entry 1); row 1: (entry 1, entry 0)
+    layer = {"spec": LayerSpec(2, 16, FMT_RVQ12, 16), "cb1": cb1.view(np.uint16),
+             "scales": np.array([0.5, 0.5], np.float16).view(np.uint16), **_pack12(i1, np.zeros_like(i1))}
+    layer["corr"] = _csr(2, [(0, 3, 0.25), (1, 0, -2.0), (1, 15, 0.5)])
+    want = np.array([[0, .5, 1, 1.5 + .25, 2, 2.5, 3, 3.5] + [.5] * 8,
+                     [.5 - 2.0] + [.5] * 7 + [0, .5, 1, 1.5, 2, 2.5, 3, 3.5 + .5]])
+    w, wb = oracle.dequant(layer, DT_F16)
+    assert w.tolist() == want.tolist()
+    assert wb.view(np.float16).astype(np.float64).tolist() == want.tolist()  # all exact in fp16
+    x = np.ones((1, 16), np.float16).view(np.uint16)
+    assert oracle.forward(layer, x, DT_F16).tolist() == [want.sum(axis=1).tolist()]
+
+
+@pytest.mark.parametrize("p,v,dt,expect", [
+    (1.0, 2.0 ** -11, DT_F16, 0x3C00),       # 1 + 2^-11 is exact in fp32, then ties to even in fp16
+    (1.0, 3 * 2.0 ** -11, DT_F16, 0x3C02),   # ... and rounds up to 1 + 2^-9
+    (2048.0, 2.0 ** -14, DT_F16, 0x6800),    # fl32(2048 + 2^-14) = 2048 (below half an fp32 ulp)
+    (1.0, 2.0 ** -8, DT_BF16, 0x3F80),       # bf16 tie to even
+    (-3.0, 0.5, DT_BF16, 0xC020),            # -2.5 exactly
+])
+def test_correction_rounding_points_by_hand(oracle, p, v, dt, expect):
+    layer = _one_group_layer(p, 0.0, 1.0, fmt=FMT_RVQ12)
+    layer.pop("cb2")
+    layer["corr"] = _csr(1, [(0, 0, v)])
+    w, wb = oracle.dequant(layer, dt)
+    assert int(wb[0, 0]) == expect
+    assert w[0, 0] == p + v
+    assert int(wb[0, 1]) == int(oracle.dequant(_one_group_layer(p, 0.0, 1.0, fmt=FMT_RVQ12), dt)[1][0, 1])
+
+
+@pytest.mark.parametrize("fmt,sg,K", [(FMT_RVQ12, 64, 384), (FMT_RVQ12_4, 64, 320), (FMT_VQ16, 192, 192)])
+def test_correction_matches_dense_numpy(oracle, fmt, sg, K):
+    """W' = W + C built independently (numpy dense W, dense C from the triples) against the
+    oracle's dequant and forward, on all rows and on a row subset."""
+    N = 24
+    layer = make_layer(LayerSpec(N, K, fmt, sg), cfg_id=96, tensor_id=fmt)
+    layer["corr"] = make_correction(N, K, density=0.05, cfg_id=96, tensor_id=fmt)
+    assert layer["corr"]["row_ptr"][-1] > 0
+    Wc = _dense_numpy(layer) + _dense_corr(layer["corr"], N, K)
+    w, _ = oracle.dequant(layer)
+    assert np.array_equal(w, Wc)
+    x = make_x(3, K, DT_BF16, cfg_id=96)
+    xd = (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    ref = xd @ Wc.T
+    y = oracle.forward(layer, x, DT_BF16)
+    assert np.allclose(y, ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
+    rows = [20, 3, 11]
+    assert np.array_equal(oracle.forward(layer, x, DT_BF16, rows=rows), y[:, rows])
+
+
+def test_correction_of_zeros_is_the_identity(oracle):
+    N, K = 16, 256
+    layer = make_layer(LayerSpec(N, K, FMT_RVQ12_4, 64), cfg_id=95)
+    x = make_x(2, K, DT_F16, cfg_id=95)
+    base_y, (base_w, base_wb) = oracle.forward(layer, x, DT_F16), oracle.dequant(layer, DT_F16)
+    corr = make_correction(N, K, density=0.1, cfg_id=95)
+    corr["val"] = np.zeros_like(corr["val"])
+    layer["corr"] = corr
+    assert np.array_equal(oracle.forward(layer, x, DT_F16), base_y)
+    w, wb = oracle.dequant(layer, DT_F16)
+    assert np.array_equal(w, base_w) and np.array_equal(wb, base_wb)
+
+
+def test_correction_layout_is_checked(oracle):
+    ok = _csr(3, [(0, 1, 1.0), (0, 5, 1.0), (2, 0, 1.0)])
+    assert oracle.corr_check(3, 8, ok["row_ptr"], ok["col"]) == 0
+    assert oracle.corr_check(3, 8, ok["row_ptr"], np.array([5, 1, 0], np.int32)) != 0   # columns not increasing
+    assert oracle.corr_check(3, 8, ok["row_ptr"], np.array([1, 5, 8], np.int32)) != 0   # column beyond K
+    assert oracle.corr_check(3, 8, np.array([0, 2, 1, 3], np.int32), ok["col"]) != 0    # row_ptr decreasing
+    assert oracle.corr_check(3, 8, np.array([1, 2, 2, 3], np.int32), ok["col"]) != 0    # row_ptr[0] != 0
