@@ -44,8 +44,8 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from synth import (CONFIGS, DT_BF16, DT_F16, FMT_VQ16, FMT_VQ16_RVQ, LayerSpec, make_layer, make_signs,  # noqa: E402
-                   make_x)
+from synth import (CONFIGS, DT_BF16, DT_F16, FMT_VQ16, FMT_VQ16_RVQ, LayerSpec, make_correction,  # noqa: E402
+                   make_layer, make_signs, make_x)
 
 METRIC = "vq_linear µs/layer & achieved HBM GB/s (% of roofline) at batch 1/16; TFLOP/s at M=256"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -65,6 +65,9 @@ for _bpw in (3, 4, 5):
         cfg=100 + _bpw, layers=1,
         config=dict(name=f"vq16-ladder-4096x4096-{_bpw}bpw", layers=1, act=DT_F16, Ms=(1, 8), rht=False,
                     tensors=[("w", LayerSpec(4096, 4096, FMT_VQ16_RVQ, 4096, bpw=_bpw))]))
+# The MLP with a sparse correction sidecar on every matrix (orka README, "How it works":
+# "(+ sparse correction)"): 0.1 % of the weights corrected, fp16 values ~ N(0, 0.05^2).
+WORKLOADS["llama3-8b-mlp-corr"] = dict(cfg=4, layers=1, gate_up_concurrent=True, corr_density=0.001)
 _16BIT = (FMT_VQ16, FMT_VQ16_RVQ)
 
 
@@ -80,6 +83,15 @@ def load_peaks():
             d = json.load(f)
         return d, "measured"
     return dict(FALLBACK_PEAKS), "fallback"
+
+
+def corr_bytes(L):
+    """Bytes of a layer's sparse correction sidecar: row pointers, and a column (int32) and
+    a value (fp16) per entry; 0 without one."""
+    if L is None or not getattr(L, "corr", 0):
+        return 0
+    t = L.t
+    return t["corr_rows"].numel() * 4 + (t["corr_cols"].numel() * 6 if "corr_cols" in t else 0)
 
 
 def layer_bytes(spec, M, act_bytes=2):
@@ -173,6 +185,9 @@ class Workload:
         for li in range(w["layers"]):
             for ti, (label, spec) in enumerate(self.cfg["tensors"]):
                 arr = make_layer(spec, cfg_id=w["cfg"], layer=li, tensor_id=ti, seed=seed)
+                if w.get("corr_density"):
+                    arr["corr"] = make_correction(spec.N, spec.K, density=w["corr_density"], cfg_id=w["cfg"],
+                                                  layer=li, tensor_id=ti, seed=seed)
                 L = vq.VQLinear(spec.N, spec.K, spec.fmt, spec.scale_group, self.act, max_M, arr,
                                 rht=int(self.cfg["rht"]))
                 self.layers.append((f"{li}.{label}", spec, L))
@@ -203,7 +218,7 @@ class Workload:
 
     def weight_bytes(self):
         """Bytes of one copy of the step's layer inputs that do not depend on M."""
-        return sum(layer_bytes(spec, 0) for _, spec, _ in self.layers)
+        return sum(layer_bytes(spec, 0) + corr_bytes(L) for _, spec, L in self.layers)
 
     def plan(self, M, replica=0):
         """Forward calls of one step: (layer, input tensor, output tensor) with the stack's chaining."""
@@ -283,7 +298,7 @@ class Workload:
     def bytes_per_step(self, M):
         # an unfused rotation reads and writes x once more (2 + 2 bytes per element)
         extra = sum(4 * M * spec.K for _, spec, _ in self.layers if self.rht and not self.rotation_fused(spec, M))
-        return sum(layer_bytes(spec, M) for _, spec, _ in self.layers) + extra
+        return sum(layer_bytes(spec, M) + corr_bytes(L) for _, spec, L in self.layers) + extra
 
     def flops_per_step(self, M):
         return sum(2.0 * M * spec.N * spec.K for _, spec, _ in self.layers)
@@ -302,7 +317,8 @@ def _clone_layer(L):
     # 4096-entry codebooks are copied.
     shared = ("cb1", "cbr", "cb8") if L.fmt in _16BIT else ()
     c.t = {k: (v if k in shared else v.clone()) for k, v in L.t.items()}
-    c.planes = B.make_planes(c.t.get("lo"), c.t.get("hi4"), c.t.get("s2"), c.t.get("idx16"), c.t.get("idx8"))
+    c.planes = B.make_planes(c.t.get("lo"), c.t.get("hi4"), c.t.get("s2"), c.t.get("idx16"), c.t.get("idx8"),
+                             c.t.get("corr_rows"), c.t.get("corr_cols"), c.t.get("corr_vals"))
     c.codebooks = L.codebooks if L.fmt in _16BIT else B.make_codebooks(c.t["cb1"], c.t.get("cb2"))
     c.close = lambda: None  # the handle belongs to L
     return c
@@ -518,7 +534,7 @@ def gpu_arm(args):
     # ------------------------------------------------ per-launch roofline (same stream)
     _, per_fwd = time_graph(wl, M, min(args.steps, 200), 3, per_kernel=True)  # event nodes between forwards
     launches_per_fwd = [L.launches(M) for _, _, L in wl.layers]
-    bytes_per_fwd = [layer_bytes(spec, M) for _, spec, _ in wl.layers]
+    bytes_per_fwd = [layer_bytes(spec, M) + corr_bytes(L) for _, spec, L in wl.layers]
     # When every forward runs the same single kernel (no rotation launch), a region's
     # time per launch is that kernel's average duration; else use the event nodes
     # captured between the forwards (which include the gaps).  A step that overlaps
@@ -663,7 +679,8 @@ def detail(args, peaks, main_wl):
     res = {}
     for M in (4, 16):
         res[f"{args.workload} M={M}"] = measure(main_wl, M, steps, 3, peaks)
-    for name, Ms in (("single-256", (1,)), ("smollm-135m-stack", (1, 4, 16)), ("vq16-4096-rht", (1, 8))):
+    for name, Ms in (("single-256", (1,)), ("smollm-135m-stack", (1, 4, 16)), ("vq16-4096-rht", (1, 8)),
+                     ("llama3-8b-mlp-corr", (1, 16))):
         if name == args.workload:
             continue
         wl = Workload(name, max_M=16)

@@ -45,12 +45,13 @@ class vq_linear_desc(ctypes.Structure):
     _fields_ = [("N", ctypes.c_int32), ("K", ctypes.c_int32), ("fmt", ctypes.c_int32),
                 ("scale_group", ctypes.c_int32), ("act_dtype", ctypes.c_int32), ("max_M", ctypes.c_int32),
                 ("rht", ctypes.c_int32), ("n16", ctypes.c_int32), ("n8", ctypes.c_int32),
-                ("mult", ctypes.c_float * 3)]
+                ("mult", ctypes.c_float * 3), ("corr", ctypes.c_int32)]
 
 
 class vq_planes(ctypes.Structure):
     _fields_ = [("lo", ctypes.c_void_p), ("hi4", ctypes.c_void_p), ("s2", ctypes.c_void_p),
-                ("idx16", ctypes.c_void_p), ("idx8", ctypes.c_void_p)]
+                ("idx16", ctypes.c_void_p), ("idx8", ctypes.c_void_p),
+                ("corr_rows", ctypes.c_void_p), ("corr_cols", ctypes.c_void_p), ("corr_vals", ctypes.c_void_p)]
 
 
 class vq_codebooks(ctypes.Structure):
@@ -141,8 +142,11 @@ def _stream(stream) -> int | None:
     return stream.cuda_stream
 
 
-def make_planes(lo=None, hi4=None, s2=None, idx16=None, idx8=None) -> vq_planes:
-    return vq_planes(_ptr(lo), _ptr(hi4), _ptr(s2), _ptr(idx16), _ptr(idx8))
+def make_planes(lo=None, hi4=None, s2=None, idx16=None, idx8=None, corr_rows=None, corr_cols=None,
+                corr_vals=None) -> vq_planes:
+    """corr_*: the sparse correction sidecar (CSR by output row), or None."""
+    return vq_planes(_ptr(lo), _ptr(hi4), _ptr(s2), _ptr(idx16), _ptr(idx8), _ptr(corr_rows), _ptr(corr_cols),
+                     _ptr(corr_vals))
 
 
 def make_codebooks(cb1, cb2=None, cbr=(), cb8=None) -> vq_codebooks:
@@ -152,17 +156,17 @@ def make_codebooks(cb1, cb2=None, cbr=(), cb8=None) -> vq_codebooks:
     return vq_codebooks(_ptr(cb1), _ptr(cb2), (ctypes.c_void_p * 3)(*[_ptr(c) for c in cbr]), _ptr(cb8))
 
 
-def make_desc(N, K, fmt, scale_group, act_dtype, max_M, rht=0, n16=0, n8=0, mult=()) -> vq_linear_desc:
+def make_desc(N, K, fmt, scale_group, act_dtype, max_M, rht=0, n16=0, n8=0, mult=(), corr=0) -> vq_linear_desc:
     m = list(mult) + [0.0] * (3 - len(mult))
-    return vq_linear_desc(N, K, fmt, scale_group, act_dtype, max_M, rht, n16, n8, (ctypes.c_float * 3)(*m))
+    return vq_linear_desc(N, K, fmt, scale_group, act_dtype, max_M, rht, n16, n8, (ctypes.c_float * 3)(*m), corr)
 
 
 def vq_abi_version() -> int:
     return load().vq_abi_version()
 
 
-def vq_linear_create(N, K, fmt, scale_group, act_dtype, max_M, rht=0, n16=0, n8=0, mult=()) -> int:
-    d = make_desc(N, K, fmt, scale_group, act_dtype, max_M, rht, n16, n8, mult)
+def vq_linear_create(N, K, fmt, scale_group, act_dtype, max_M, rht=0, n16=0, n8=0, mult=(), corr=0) -> int:
+    d = make_desc(N, K, fmt, scale_group, act_dtype, max_M, rht, n16, n8, mult, corr)
     h = ctypes.c_void_p()
     _check(load().vq_linear_create(ctypes.byref(d), ctypes.byref(h)))
     return h.value
@@ -197,9 +201,9 @@ def vq_linear_forward_rotated(h, x, signs, planes: vq_planes, codebooks: vq_code
 
 
 def vq_linear_forward_noalloc(N, K, fmt, scale_group, act_dtype, x, planes: vq_planes, codebooks: vq_codebooks,
-                              scales, y, M, stream=None, rht=0, n16=0, n8=0, mult=()) -> None:
+                              scales, y, M, stream=None, rht=0, n16=0, n8=0, mult=(), corr=0) -> None:
     """Handle-free forward of 0 <= M <= 16 tokens that allocates nothing (fixed in-library scratch)."""
-    d = make_desc(N, K, fmt, scale_group, act_dtype, max(M, 1), rht, n16, n8, mult)
+    d = make_desc(N, K, fmt, scale_group, act_dtype, max(M, 1), rht, n16, n8, mult, corr)
     _check(load().vq_linear_forward_noalloc(ctypes.byref(d), _ptr(x), ctypes.byref(planes), ctypes.byref(codebooks),
                                             _ptr(scales), _ptr(y), M, _stream(stream)))
 

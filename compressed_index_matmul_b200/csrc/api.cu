@@ -38,6 +38,7 @@ struct vq_linear_s {
   uint32_t* err;      // device word, set by bounded waits that gave up
   int sm_budget;      // CTAs of the table kernel (0: every SM)
   void* xrot;         // rotated-x buffer [max_M][K] (desc.rht == 1), for the unfused rotated forward
+  float* corr_y;      // the sparse correction's x . C^T, fp32 [max_M][N] (desc.corr == 1)
 };
 
 namespace {
@@ -89,6 +90,9 @@ vq_status validate_desc(const vq_linear_desc* d) {
     return fail(VQ_ERR_INVALID_ARG, "act_dtype=%d is not VQ_F16 or VQ_BF16", d->act_dtype);
   if (d->max_M <= 0 || d->max_M > (1 << 20))
     return fail(VQ_ERR_INVALID_ARG, "max_M=%d must be in [1, 2^20]", d->max_M);
+  if (d->corr != 0 && d->corr != 1) return fail(VQ_ERR_INVALID_ARG, "corr=%d must be 0 or 1", d->corr);
+  if (d->corr && d->fmt == VQ_FMT_VQ16_RVQ)
+    return fail(VQ_ERR_UNSUPPORTED, "the sparse correction is defined for the 12-bit and 16-bit formats only");
   return VQ_OK;
 }
 
@@ -102,6 +106,15 @@ vq_status validate_planes(const vq_linear_desc& d, const vq_planes* p) {
     if ((st = check_ptr(p->lo, "planes->lo"))) return st;
     if ((st = check_ptr(p->hi4, "planes->hi4"))) return st;
     if (d.fmt == VQ_FMT_RVQ12_4 && (st = check_ptr(p->s2, "planes->s2"))) return st;
+  }
+  if (d.corr) {
+    if ((st = check_ptr(p->corr_rows, "planes->corr_rows"))) return st;
+    if (p->corr_cols && !aligned16(p->corr_cols)) return fail(VQ_ERR_INVALID_ARG, "planes->corr_cols is not 16-byte aligned");
+    if (p->corr_vals && !aligned16(p->corr_vals)) return fail(VQ_ERR_INVALID_ARG, "planes->corr_vals is not 16-byte aligned");
+    if ((p->corr_cols == nullptr) != (p->corr_vals == nullptr))
+      return fail(VQ_ERR_INVALID_ARG, "planes->corr_cols and corr_vals must both be given (or both NULL: no entries)");
+  } else if (p->corr_rows || p->corr_cols || p->corr_vals) {
+    return fail(VQ_ERR_INVALID_ARG, "planes carry a sparse correction but the handle was created with corr = 0");
   }
   return VQ_OK;
 }
@@ -135,6 +148,11 @@ vq::LayerArgs make_args(const vq_linear_desc& d, const vq_planes* p, const vq_co
   a.hi4 = p ? p->hi4 : nullptr;
   a.s2 = p ? p->s2 : nullptr;
   a.idx16 = p ? p->idx16 : nullptr;
+  if (p && d.corr) {
+    a.corr_rows = p->corr_rows;
+    a.corr_cols = p->corr_cols;
+    a.corr_vals = p->corr_vals;
+  }
   a.cb1 = cb ? static_cast<const uint16_t*>(cb->cb1) : nullptr;
   a.cb2 = cb ? static_cast<const uint16_t*>(cb->cb2) : nullptr;
   a.scales = static_cast<const uint16_t*>(scales);
@@ -200,7 +218,7 @@ bool plan_forward(const vq_linear_desc& d, const DeviceInfo& dev, int M, int for
 
 }  // namespace vq
 
-VQ_API int32_t vq_abi_version(void) { return 2; }
+VQ_API int32_t vq_abi_version(void) { return 3; }
 
 VQ_API const char* vq_last_error(void) { return t_err.c_str(); }
 
@@ -263,6 +281,17 @@ VQ_API vq_status vq_linear_create(const vq_linear_desc* desc, vq_linear_t* out) 
                   cudaGetErrorString(e));
     }
   }
+  if (desc->corr) {
+    e = cudaMalloc(&h->corr_y, (size_t)desc->max_M * desc->N * sizeof(float));
+    if (e != cudaSuccess) {
+      cudaFree(h->scratch);
+      cudaFree(h->xrot);
+      delete h;
+      cudaGetLastError();
+      return fail(VQ_ERR_NOMEM, "cudaMalloc of the %d x %d correction buffer failed: %s", desc->max_M, desc->N,
+                  cudaGetErrorString(e));
+    }
+  }
   h->num_tickets = tickets;
   h->num_sync = sync_words;
   // words: [0] error flag, [1] pad, then the tickets, then the table kernel's sync words
@@ -277,6 +306,7 @@ VQ_API vq_status vq_linear_create(const vq_linear_desc* desc, vq_linear_t* out) 
   if (e != cudaSuccess) {
     cudaFree(h->scratch);
     cudaFree(h->xrot);
+    cudaFree(h->corr_y);
     cudaFree(words);
     delete h;
     cudaGetLastError();
@@ -302,6 +332,7 @@ VQ_API vq_status vq_linear_destroy(vq_linear_t h) {
   }
   if (h->scratch) e1 = cudaFree(h->scratch);
   if (h->xrot && e1 == cudaSuccess) e1 = cudaFree(h->xrot);
+  if (h->corr_y && e1 == cudaSuccess) e1 = cudaFree(h->corr_y);
   if (h->err) e2 = cudaFree(h->err);  // also frees the tickets and sync words (one allocation)
   if (prev >= 0 && prev != h->dev.device) cudaSetDevice(prev);
   delete h;
@@ -330,7 +361,7 @@ VQ_API int32_t vq_linear_launches(vq_linear_t h, int32_t M) {
   if (M == 0) return 0;
   vq::Plan p{};
   if (!vq::plan_forward(h->d, h->dev, M, h->path, &p)) return -1;
-  return p.launches;
+  return p.launches + (h->d.corr ? 1 : 0);  // the sparse correction's kernel
 }
 
 VQ_API vq_status vq_linear_forward(vq_linear_t h, const void* x, const vq_planes* planes,
@@ -362,6 +393,11 @@ VQ_API vq_status vq_linear_forward(vq_linear_t h, const void* x, const vq_planes
   a.M = M;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e;
+  if (d.corr) {  // x . C^T first, in fp32; the forward kernel adds it before rounding
+    e = vq::launch_corr(a, h->corr_y, s);
+    if (e != cudaSuccess) return cuda_fail(e, "vq_linear_forward correction launch");
+    a.addend = h->corr_y;
+  }
   switch (p.path) {
     case VQ_PATH_LUT: e = vq::launch_lut(a, p, h->scratch, h->sync, h->err, s); break;  // p.grid CTAs
     case VQ_PATH_GATHER: e = vq::launch_vq16(a, p, nullptr, s); break;
@@ -393,7 +429,8 @@ VQ_API vq_status vq_linear_forward_rotated(vq_linear_t h, const void* x, const i
   if (!vq::plan_forward(d, h->dev, M, h->path, &p))
     return fail(VQ_ERR_UNSUPPORTED, "path %d cannot run M=%d", h->path, M);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (p.path == VQ_PATH_GATHER && M == 1) {  // the kernel rotates x itself
+  if (p.path == VQ_PATH_GATHER && M == 1 && !d.corr) {  // the kernel rotates x itself
+    // (a sparse correction needs the rotated x too: that layer takes the route below)
     if (h->sm_budget > 0 && p.grid > h->sm_budget) p.grid = h->sm_budget;
     if (p.scratch_bytes > h->scratch_bytes)
       return fail(VQ_ERR_UNSUPPORTED, "plan needs %zu scratch bytes, handle has %zu", p.scratch_bytes,
@@ -634,6 +671,8 @@ VQ_API vq_status vq_linear_forward_noalloc(const vq_linear_desc* desc, const voi
                                            const vq_codebooks* codebooks, const void* scales, void* y, int32_t M,
                                            void* stream) {
   vq_status st = validate_desc(desc);
+  if (st == VQ_OK && desc->corr)
+    return fail(VQ_ERR_UNSUPPORTED, "the sparse correction needs a handle's buffer: use vq_linear_forward");
   if (st) return st;
   const vq_linear_desc& d = *desc;
   if (M < 0 || M > 16) return fail(VQ_ERR_INVALID_ARG, "M=%d outside [0, 16] (the no-allocation path)", M);

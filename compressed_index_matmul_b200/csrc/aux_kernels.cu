@@ -199,6 +199,34 @@ __global__ void debug_dequant_kernel(LayerArgs a, uint16_t* __restrict__ w) {
         fma_codeword(m, reinterpret_cast<const uint4*>(a.cb8)[a.idx8[e]], v);
       }
       pack_scaled<W>(v, s, out);
+    } else if (a.corr_rows) {
+      // With the sparse correction: the same fp32 weights, then fl32(p + C) for the
+      // corrected ones (the row's entries are in increasing column order).
+      const uint32_t w1[4] = {c1.x, c1.y, c1.z, c1.w};
+      uint4 c2 = c1;
+      if (a.fmt == kFmtRvq12_4) c2 = reinterpret_cast<const uint4*>(a.cb2)[i2];
+      const uint32_t w2[4] = {c2.x, c2.y, c2.z, c2.w};
+      float p[8];
+      for (int q = 0; q < 4; ++q) {
+        float2 c = f16x2_to_f32x2(w1[q]);
+        if (a.fmt == kFmtRvq12_4) {
+          const float2 d = f16x2_to_f32x2(w2[q]);
+          c.x = __fadd_rn(c.x, d.x);
+          c.y = __fadd_rn(c.y, d.y);
+        }
+        p[2 * q] = __fmul_rn(s, c.x);
+        p[2 * q + 1] = __fmul_rn(s, c.y);
+      }
+      int lo = a.corr_rows[n], hi = a.corr_rows[n + 1];
+      while (lo < hi) {  // first entry at column >= 8g
+        const int mid = (lo + hi) >> 1;
+        if (a.corr_cols[mid] < 8 * g) lo = mid + 1; else hi = mid;
+      }
+      for (int j = lo; j < a.corr_rows[n + 1] && a.corr_cols[j] < 8 * g + 8; ++j) {
+        const int d = a.corr_cols[j] - 8 * g;
+        if (d >= 0) p[d] = __fadd_rn(p[d], f16_bits_to_f32(a.corr_vals[j]));  // d < 0 only for unsorted columns
+      }
+      for (int q = 0; q < 4; ++q) out[q] = Elt<W>::pack(p[2 * q], p[2 * q + 1]);
     } else if (a.fmt == kFmtRvq12_4) {
       const uint4 c2 = reinterpret_cast<const uint4*>(a.cb2)[i2];
       decode_group_packed<W, true>(c1, c2, s, out);
@@ -207,6 +235,35 @@ __global__ void debug_dequant_kernel(LayerArgs a, uint16_t* __restrict__ w) {
     }
     reinterpret_cast<uint4*>(w)[t] = make_uint4(out[0], out[1], out[2], out[3]);
   }
+}
+
+// The sparse correction's contribution (orka README, "How it works": the decode
+// adds a sparse correction): out[m][n] = sum_j x[m][col_j] * val_j over row n's
+// entries in order, fp32, one thread per (m, n) (consecutive threads take
+// consecutive rows of one token, so the stores coalesce and a row's entries are
+// read from L1/L2 by the M threads that share them).  Columns are clamped to
+// [0, K), so a malformed column can give a wrong value but never an out-of-range
+// read.  It reads x (perhaps written by the previous kernel) and overwrites the
+// buffer the previous forward of the handle read, so it waits for the previous
+// kernel.
+template <typename T>
+__global__ void __launch_bounds__(256) corr_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ rows,
+                                                   const int32_t* __restrict__ cols,
+                                                   const uint16_t* __restrict__ vals, float* __restrict__ out, int M,
+                                                   int N, int K) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= (int64_t)M * N) return;
+  const int m = (int)(t / N), n = (int)(t - (int64_t)m * N);
+  const uint16_t* xm = x + (int64_t)m * K;
+  const int j1 = rows[n + 1];
+  float acc = 0.f;
+  for (int j = rows[n]; j < j1; ++j) {
+    const int c = min(max(cols[j], 0), K - 1);
+    acc = fmaf(Elt<T>::to_f32(xm[c]), f16_bits_to_f32(vals[j]), acc);
+  }
+  out[t] = acc;
 }
 
 // Test of the bounded waits: one thread waits on an mbarrier that nothing
@@ -245,6 +302,23 @@ cudaError_t launch_debug_dequant(const LayerArgs& a, void* w, int wdt, cudaStrea
   else
     debug_dequant_kernel<__half><<<grid_for(total, 256), 256, 0, s>>>(a, (uint16_t*)w);
   return cudaGetLastError();
+}
+
+cudaError_t launch_corr(const LayerArgs& a, float* out, cudaStream_t s) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(((int64_t)a.M * a.N + 255) / 256));
+  cfg.blockDim = dim3(256);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const uint16_t* x = static_cast<const uint16_t*>(a.x);
+  if (a.act == VQ_BF16)
+    return cudaLaunchKernelEx(&cfg, corr_kernel<__nv_bfloat16>, x, a.corr_rows, a.corr_cols, a.corr_vals, out, a.M,
+                              a.N, a.K);
+  return cudaLaunchKernelEx(&cfg, corr_kernel<__half>, x, a.corr_rows, a.corr_cols, a.corr_vals, out, a.M, a.N, a.K);
 }
 
 }  // namespace vq

@@ -207,7 +207,8 @@ __global__ void __launch_bounds__(256) gemv_kernel(LayerArgs a, int k_per_split,
       for (int i = 0; i < 4; ++i) {
         const int m = 8 * t + 2 * c + (i & 1);
         const int r = rows[i >> 1];
-        if (m < M && r < N) y[(int64_t)m * N + r] = Elt<T>::from_f32(acc[t][i]);
+        if (m < M && r < N)
+          y[(int64_t)m * N + r] = Elt<T>::from_f32(a.addend ? acc[t][i] + a.addend[(int64_t)m * N + r] : acc[t][i]);
       }
     return;
   }
@@ -231,7 +232,7 @@ __global__ void __launch_bounds__(256) gemv_kernel(LayerArgs a, int k_per_split,
     const int m = i / nrows, r = rbeg + i % nrows;
     float sum = 0.f;
     for (int k = 0; k < splits; ++k) sum += __ldcg(partial + ((int64_t)k * M + m) * N + r);
-    y[(int64_t)m * N + r] = Elt<T>::from_f32(sum);
+    y[(int64_t)m * N + r] = Elt<T>::from_f32(a.addend ? sum + a.addend[(int64_t)m * N + r] : sum);
   }
   if (threadIdx.x == 0) tickets[blockIdx.x] = 0u;  // ready for the next forward
 }

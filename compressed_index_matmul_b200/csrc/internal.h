@@ -30,6 +30,13 @@ struct LayerArgs {
   int act;                // VQ_F16 / VQ_BF16
   int n16, n8;            // stages of the 16-bit formats (1, 0 for VQ_FMT_VQ16)
   float mult[3];          // multipliers of residual stages 2..n16 + n8
+  // The sparse correction (NULL when there is none): CSR by output row, and the
+  // fp32 [M][N] buffer holding x . C^T, which the forward kernels add to their
+  // fp32 result before rounding into y.
+  const int32_t* corr_rows;
+  const int32_t* corr_cols;
+  const uint16_t* corr_vals;
+  const float* addend;
 };
 
 // Work split chosen for one forward.
@@ -76,6 +83,8 @@ cudaError_t launch_rht_output(const void* y, void* y_out, const int8_t* signs, i
                               cudaStream_t s);
 cudaError_t launch_debug_unpack(const LayerArgs& a, uint16_t* i1, uint8_t* i2, cudaStream_t s);
 cudaError_t launch_debug_dequant(const LayerArgs& a, void* w, int wdt, cudaStream_t s);
+// out[m][n] = sum over row n's correction entries j (in order) of x[m][col_j] * val_j, fp32.
+cudaError_t launch_corr(const LayerArgs& a, float* out, cudaStream_t s);
 cudaError_t launch_debug_wait_timeout(uint32_t* err, cudaStream_t s);
 
 }  // namespace vq

@@ -372,6 +372,7 @@ __global__ void __launch_bounds__(kLutThreads, 1)
         }
         if (S == 1) {
           if (!block_scales) acc *= f16_bits_to_f32(a.scales[r]);
+          if (a.addend) acc += a.addend[r];  // the sparse correction's x . C^T term
           static_cast<uint16_t*>(a.y)[r] = Elt<T>::from_f32(acc);
         } else {
           partial[(int64_t)s * N + r] = acc;
@@ -477,6 +478,10 @@ __global__ void __launch_bounds__(kLutThreads, 1)
       if (!block_scales) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) o4[i] *= f16_bits_to_f32(a.scales[r + i]);
+      }
+      if (a.addend) {  // the sparse correction's x . C^T term
+#pragma unroll
+        for (int i = 0; i < 4; ++i) o4[i] += a.addend[r + i];
       }
       uint16_t* yr = static_cast<uint16_t*>(a.y) + r;
       *reinterpret_cast<uint2*>(yr) =

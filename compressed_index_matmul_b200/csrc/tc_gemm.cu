@@ -432,6 +432,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             asm volatile("ld.shared.f32 %0, [%1];" : "=f"(o) : "r"(recv_addr(ci, i)));
             f += o;
           }
+          // the sparse correction's x . C^T term, added before the one rounding
+          if (a.addend && valid && tok0 + 16 * ci + i < M) f += a.addend[(int64_t)(tok0 + 16 * ci + i) * N + r];
           const uint16_t h = Elt<T>::from_f32(f);
           asm volatile("st.shared.u16 [%0], %1;" ::"r"(stage_addr(ci, i)), "h"(h) : "memory");
         }
@@ -462,7 +464,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const int tok = tok0 + c0 + i;
           if (tok >= M || !valid) continue;
           if (p.splits == 1)
-            y[(int64_t)tok * N + r] = Elt<T>::from_f32(__uint_as_float(v[i]));
+            y[(int64_t)tok * N + r] =
+                Elt<T>::from_f32(a.addend ? __uint_as_float(v[i]) + a.addend[(int64_t)tok * N + r] : __uint_as_float(v[i]));
           else
             p.partial[((int64_t)split * M + tok) * N + r] = __uint_as_float(v[i]);
         }
@@ -498,7 +501,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
 #pragma unroll
           for (int i = 0; i < 16; ++i)
-            if (valid && tok0 + c0 + i < M) y[(int64_t)(tok0 + c0 + i) * N + r] = Elt<T>::from_f32(acc[i]);
+            if (valid && tok0 + c0 + i < M)
+              y[(int64_t)(tok0 + c0 + i) * N + r] =
+                  Elt<T>::from_f32(a.addend ? acc[i] + a.addend[(int64_t)(tok0 + c0 + i) * N + r] : acc[i]);
         }
         ptx::tc_fence_before();
         if (threadIdx.x == 64) p.tickets[tile] = 0u;

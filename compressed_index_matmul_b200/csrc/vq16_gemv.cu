@@ -272,7 +272,9 @@ __global__ void __launch_bounds__(kV16Consumers, 1)
         float v = 0.f;
 #pragma unroll
         for (int q = 0; q < kV16Cluster; ++q) v += ld_cluster_f32(ptx::map_shared_rank(local, q));
-        static_cast<uint16_t*>(a.y)[(int64_t)m * N + r0 + r] = Elt<T>::from_f32(v * xscale * row_scale[o]);
+        float out = v * xscale * row_scale[o];
+        if (a.addend) out += a.addend[(int64_t)m * N + r0 + r];  // the sparse correction's x . C^T term
+        static_cast<uint16_t*>(a.y)[(int64_t)m * N + r0 + r] = Elt<T>::from_f32(out);
       }
     }
     ptx::cluster_sync();  // no CTA reuses or releases its csum while another reads it

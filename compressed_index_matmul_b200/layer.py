@@ -24,7 +24,9 @@ class VQLinear:
     layer shape (N, K, fmt, scale_group).  For the residual ladder (VQ_FMT_VQ16_RVQ)
     idx16 holds one plane per 16-bit stage, cbr is [n16 - 1, 65536, 8] and ``mult``
     the float32 multipliers of the residual stages; the stage counts follow from the
-    arrays.  ``forward(x)`` calls vq_linear_forward.
+    arrays.  An optional ``corr`` dict (row_ptr int32 [N+1], col int32, val fp16 bits)
+    is the sparse correction sidecar; the handle is then created with corr = 1 and
+    every forward passes it.  ``forward(x)`` calls vq_linear_forward.
     """
 
     def __init__(self, N, K, fmt, scale_group, act_dtype, max_M, arrays: dict, device="cuda", rht=0):
@@ -44,12 +46,21 @@ class VQLinear:
             if "cbr" in self.t:
                 stride = 65536 * 8 * 2
                 cbr = tuple(self.t["cbr"].data_ptr() + i * stride for i in range(self.n16 - 1))
+        self.corr = 0
+        if arrays.get("corr") is not None:
+            c = arrays["corr"]
+            self.corr = 1
+            self.t["corr_rows"] = _dev(np.asarray(c["row_ptr"], np.int32), self.device)
+            if len(c["col"]):
+                self.t["corr_cols"] = _dev(np.asarray(c["col"], np.int32), self.device)
+                self.t["corr_vals"] = _dev(np.asarray(c["val"], np.uint16), self.device)
         self.planes = B.make_planes(self.t.get("lo"), self.t.get("hi4"), self.t.get("s2"), self.t.get("idx16"),
-                                    self.t.get("idx8"))
+                                    self.t.get("idx8"), self.t.get("corr_rows"), self.t.get("corr_cols"),
+                                    self.t.get("corr_vals"))
         self.codebooks = B.make_codebooks(self.t["cb1"], self.t.get("cb2"), cbr, self.t.get("cb8"))
         with torch.cuda.device(self.device):
             self.handle = B.vq_linear_create(N, K, fmt, scale_group, act_dtype, max_M, rht, self.n16, self.n8,
-                                             self.mult)
+                                             self.mult, self.corr)
 
     @property
     def torch_dtype(self):

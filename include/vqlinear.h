@@ -140,6 +140,10 @@ typedef struct {
   float mult[3];       /* VQ_FMT_VQ16_RVQ: multiplier of residual stage 2, 3, 4 (the
                           inverse residual scales; the 16-bit stages first, the 8-bit
                           one last); finite; entries past n16 + n8 - 1 are ignored */
+  int32_t corr;        /* (ABI 3) 1: every forward of this handle carries a sparse
+                          correction (vq_planes.corr_*), and create allocates an fp32
+                          max_M x N buffer for its contribution; 0: none may be given.
+                          Not for VQ_FMT_VQ16_RVQ. */
 } vq_linear_desc;
 
 typedef struct {
@@ -149,6 +153,17 @@ typedef struct {
   const uint16_t* idx16; /* N*K/8 entries, K-slice-major (VQ16); n16*N*K/8 entries,
                             stage-major (VQ16_RVQ); else NULL */
   const uint8_t* idx8;   /* N*K/8 bytes, K-slice-major (VQ16_RVQ with n8 == 1), else NULL */
+  /* (ABI 3) Sparse correction sidecar (orka README, "How it works": the decode is
+   * scale x sum(codebook[index]) (+ sparse correction)): W' = W + C with C sparse,
+   * by output row.  Row n's entries are j = corr_rows[n] .. corr_rows[n+1] - 1, at
+   * columns corr_cols[j] in [0, K), strictly increasing within a row (not checked
+   * on the device: a caller that breaks this gets a wrong y, never an out-of-range
+   * access), with fp16 values corr_vals[j].  corr_rows[0] == 0.  All three given
+   * exactly when desc.corr == 1, else all NULL.  Device memory, owned by the caller;
+   * corr_cols / corr_vals may be NULL when there are no entries. */
+  const int32_t* corr_rows; /* [N + 1] */
+  const int32_t* corr_cols; /* [nnz] */
+  const uint16_t* corr_vals; /* [nnz], fp16 bits */
 } vq_planes;
 
 typedef struct {
@@ -161,11 +176,13 @@ typedef struct {
 
 typedef struct vq_linear_s* vq_linear_t;
 
-/* Version of this ABI (increments on any incompatible change). */
+/* Version of this ABI (increments on any incompatible change).  3: the sparse
+ * correction fields (vq_linear_desc.corr, vq_planes.corr_*). */
 int32_t vq_abi_version(void);
 
 /* Create a handle for one layer shape.  Validates `desc`, queries the current
- * device and allocates the split-K scratch buffer (sized from max_M and N) on it.
+ * device and allocates the split-K scratch buffer (sized from max_M and N) on it,
+ * and with desc->corr == 1 an fp32 max_M x N buffer for the sparse correction.
  * Synchronous.  On error *out is set to NULL. */
 vq_status vq_linear_create(const vq_linear_desc* desc, vq_linear_t* out);
 
@@ -200,9 +217,14 @@ vq_status vq_linear_set_sm_budget(vq_linear_t h, int32_t sms);
  *   even into y.  For a given handle, path and M the result is bit-identical from
  *   run to run: split-K partials are summed in a fixed order (an integer atomic
  *   only picks which CTA does the sum; no floating-point atomics).
- * Enqueues one kernel on `stream` (see vq_linear_launches) and returns.  The
- * kernel may start its prologue (reading the constant layer inputs) while the
- * previous kernel in the stream finishes; it reads x and writes y only after it. */
+ * With a sparse correction (desc.corr == 1) y = x . (W + C)^T: a first small
+ * kernel computes every x . C^T term in fp32 (entries of a row in order) into the
+ * handle's buffer, and the forward kernel adds it to its fp32 result before the
+ * one rounding into y.
+ * Enqueues one kernel on `stream` (two with a correction; see vq_linear_launches)
+ * and returns.  The kernel may start its prologue (reading the constant layer
+ * inputs) while the previous kernel in the stream finishes; it reads x and
+ * writes y only after it. */
 vq_status vq_linear_forward(vq_linear_t h, const void* x, const vq_planes* planes,
                             const vq_codebooks* codebooks, const void* scales, void* y,
                             int32_t M, int32_t N, int32_t K, void* stream);
@@ -224,8 +246,9 @@ vq_status vq_linear_forward(vq_linear_t h, const void* x, const vq_planes* plane
  * copy per device: 4 MiB of partials and 4096 counters.  A shape whose plan
  * needs more (roughly splits x M x N x 4 bytes, or more than 4096 tiles of 16
  * output rows) returns VQ_ERR_UNSUPPORTED with the sizes in vq_last_error();
- * use a handle for those.  No call allocates memory: neither this library nor
- * any library it calls does.
+ * use a handle for those.  A sparse correction (desc->corr, planes->corr_*) needs
+ * a handle's buffer and is refused here (VQ_ERR_UNSUPPORTED).  No call allocates
+ * memory: neither this library nor any library it calls does.
  *
  * Set-up: the first call on a device (the current one) looks up the buffer's
  * address, clears the counters and synchronises the device.  Make that first
@@ -260,8 +283,8 @@ vq_status vq_linear_forward_rotated(vq_linear_t h, const void* x, const int8_t* 
                                     const vq_codebooks* codebooks, const void* scales, void* y, int32_t M,
                                     int32_t N, int32_t K, void* stream);
 
-/* Number of kernels vq_linear_forward enqueues for this M (0 for M == 0), or -1
- * if M is out of range. */
+/* Number of kernels vq_linear_forward enqueues for this M (0 for M == 0; one
+ * more when the handle carries a sparse correction), or -1 if M is out of range. */
 int32_t vq_linear_launches(vq_linear_t h, int32_t M);
 
 /* Randomised Hadamard rotation of the input (GLQ README, "How it works",
@@ -315,7 +338,8 @@ vq_status vq_debug_unpack(vq_linear_t h, const vq_planes* planes, uint16_t* i1_o
 
 /* Materialised weights w_out [N][K] in fp16 (wdt = VQ_F16) or bf16 (VQ_BF16),
  * each rounded exactly as  RN(fl32(fl32(s) * fl32(cb1 + cb2)))  -- the stage sum
- * and the scaled value are rounded to fp32, then to nearest even in wdt.
+ * and the scaled value are rounded to fp32, then to nearest even in wdt.  With a
+ * sparse correction, a corrected weight is RN(fl32(fl32(s * fl32(cb1 + cb2)) + C)).
  * One kernel launch.  The forward path never calls this. */
 vq_status vq_debug_dequant(vq_linear_t h, const vq_planes* planes, const vq_codebooks* codebooks,
                            const void* scales, void* w_out, int32_t wdt, void* stream);

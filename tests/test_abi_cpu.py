@@ -36,7 +36,7 @@ def test_header_declares_the_binding_exports():
 def test_library_exports_every_declared_symbol(lib):
     for name in declared_functions():
         assert hasattr(lib, name), name
-    assert lib.vq_abi_version() == 2
+    assert lib.vq_abi_version() == 3
 
 
 def test_no_symbols_beyond_the_abi(lib):
@@ -71,6 +71,9 @@ def _create(**kw):
     (dict(fmt=B.VQ_FMT_VQ16_RVQ, n16=4, n8=1), B.VQ_ERR_INVALID_ARG),  # 9 bpw: not in the table
     (dict(fmt=B.VQ_FMT_VQ16_RVQ, n16=2, n8=1, mult=(0.1, float("nan"))), B.VQ_ERR_INVALID_ARG),
     (dict(fmt=B.VQ_FMT_VQ16_RVQ, n16=3, n8=0, mult=(float("inf"), 0.1)), B.VQ_ERR_INVALID_ARG),
+    # sparse correction: a flag, and not defined for the residual ladder
+    (dict(corr=2), B.VQ_ERR_INVALID_ARG),
+    (dict(fmt=B.VQ_FMT_VQ16_RVQ, n16=2, n8=0, mult=(0.1,), corr=1), B.VQ_ERR_UNSUPPORTED),
 ])
 def test_create_rejects_bad_descriptors(lib, kw, status):
     with pytest.raises(B.VQError) as ei:
@@ -81,10 +84,12 @@ def test_create_rejects_bad_descriptors(lib, kw, status):
 
 def test_ladder_struct_layout_matches_the_header():
     """The ctypes mirrors of the three ABI structs have the C layout: the ladder fields
-    follow the original ones."""
-    assert ctypes.sizeof(B.vq_linear_desc) == 7 * 4 + 2 * 4 + 3 * 4
+    follow the original ones, the sparse correction's fields follow those (ABI 3)."""
+    assert ctypes.sizeof(B.vq_linear_desc) == 7 * 4 + 2 * 4 + 3 * 4 + 4
     assert B.vq_linear_desc.n16.offset == 28 and B.vq_linear_desc.mult.offset == 36
-    assert ctypes.sizeof(B.vq_planes) == 5 * 8 and B.vq_planes.idx8.offset == 32
+    assert B.vq_linear_desc.corr.offset == 48
+    assert ctypes.sizeof(B.vq_planes) == 8 * 8 and B.vq_planes.idx8.offset == 32
+    assert B.vq_planes.corr_rows.offset == 40 and B.vq_planes.corr_vals.offset == 56
     assert ctypes.sizeof(B.vq_codebooks) == 6 * 8 and B.vq_codebooks.cb8.offset == 40
 
 
@@ -193,3 +198,34 @@ def test_product_package_never_uses_the_oracle():
             if f.endswith((".py", ".cu", ".cuh", ".h")):
                 src = open(os.path.join(dirpath, f)).read()
                 assert not re.search(r"\boracle\b|vq_oracle|vqo_", src), os.path.join(dirpath, f)
+
+
+def test_struct_offsets_match_the_c_header(tmp_path):
+    """The ctypes mirrors against the real header: a C program built with gcc prints every
+    field's offsetof and each struct's sizeof."""
+    import subprocess
+
+    fields = {"vq_linear_desc": [f for f, _ in B.vq_linear_desc._fields_],
+              "vq_planes": [f for f, _ in B.vq_planes._fields_],
+              "vq_codebooks": [f for f, _ in B.vq_codebooks._fields_]}
+    src = ["#include <stddef.h>", "#include <stdio.h>", '#include "vqlinear.h"', "int main(void) {"]
+    for st, fs in fields.items():
+        src.append(f'  printf("{st} sizeof %zu\\n", sizeof({st}));')
+        for f in fs:
+            src.append(f'  printf("{st} {f} %zu\\n", offsetof({st}, {f}));')
+    src.append("  return 0;\n}")
+    c = tmp_path / "offsets.c"
+    c.write_text("\n".join(src))
+    exe = tmp_path / "offsets"
+    inc = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
+    subprocess.run(["gcc", "-std=c11", "-I", inc, "-I", "/usr/local/cuda/include", str(c), "-o", str(exe)],
+                   check=True)
+    got = {}
+    for ln in subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.splitlines():
+        st, f, v = ln.split()
+        got[(st, f)] = int(v)
+    for st, fs in fields.items():
+        cls = getattr(B, st)
+        assert got[(st, "sizeof")] == ctypes.sizeof(cls), st
+        for f in fs:
+            assert got[(st, f)] == getattr(cls, f).offset, (st, f)
