@@ -470,8 +470,14 @@ def time_e2e(wl, M, steps, warmup):
     return ms, host_x.numel() * host_x.element_size(), host_y.numel() * host_y.element_size()
 
 
-def measure(wl, M, steps, warmup, peaks, with_kernels=True):
-    ms, per_fwd = time_graph(wl, M, steps, warmup, per_kernel=False)
+def measure(wl, M, steps, warmup, peaks, with_kernels=True, gpu_index=None):
+    if gpu_index is not None:  # clocks and throttle reasons while this row is timed
+        with ClockSampler(gpu_index) as clk:
+            ms, per_fwd = time_graph(wl, M, steps, warmup, per_kernel=False)
+        clocks = clk.summary()
+    else:
+        ms, per_fwd = time_graph(wl, M, steps, warmup, per_kernel=False)
+        clocks = None
     res = {"M": M, "ms_per_step": statistics.fmean(ms), "layers_per_step": len(wl.layers)}
     res["us_per_layer"] = 1e3 * res["ms_per_step"] / len(wl.layers)
     b = wl.bytes_per_step(M)
@@ -479,6 +485,8 @@ def measure(wl, M, steps, warmup, peaks, with_kernels=True):
     res["hbm_gbs"] = b / (res["ms_per_step"] * 1e-3) / 1e9
     res["hbm_frac"] = res["hbm_gbs"] / peaks["hbm_gbs"]
     res["tflops"] = wl.flops_per_step(M) / (res["ms_per_step"] * 1e-3) / 1e12
+    if clocks is not None:
+        res["clocks"] = clocks
     if with_kernels:
         _, per_fwd = time_graph(wl, M, max(5, min(steps, 50)), 2, per_kernel=True)
         res["per_forward_us"] = [float(1e3 * v) for v in per_fwd]
@@ -616,7 +624,7 @@ def gpu_arm(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(args.workload, M, budget_s=args.cpu_seconds)
     if rank == 0 and not args.no_detail:
-        out["detail"] = detail(args, peaks, wl)
+        out["detail"] = detail(args, peaks, wl, gpu_index=smi_index)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -672,35 +680,37 @@ def lookup_traffic(kernel, workload, M):
     return e.get("dram_bytes_per_launch")
 
 
-def detail(args, peaks, main_wl):
+def detail(args, peaks, main_wl, gpu_index=None):
     """The rest of the metric: the other batch sizes of the headline workload and every
-    other workload at each of its M, the rotations and the encoder."""
+    other workload at each of its M, the rotations and the encoder.  The compute-bound
+    prefill rows come first (before the GPU has run minutes of other work, which can put
+    it under its power cap); every row carries the clocks sampled while it was timed."""
     steps = max(10, min(args.steps, 300))
     res = {}
-    for M in (4, 16):
-        res[f"{args.workload} M={M}"] = measure(main_wl, M, steps, 3, peaks)
-    for name, Ms in (("single-256", (1,)), ("smollm-135m-stack", (1, 4, 16)), ("vq16-4096-rht", (1, 8)),
-                     ("llama3-8b-mlp-corr", (1, 16))):
-        if name == args.workload:
-            continue
-        wl = Workload(name, max_M=16)
-        for M in Ms:
-            r = measure(wl, M, steps, 3, peaks, with_kernels=(name != "smollm-135m-stack"))
-            if name == "smollm-135m-stack":
-                r["us_per_transformer_layer"] = 1e3 * r["ms_per_step"] / 30
-            res[f"{name} M={M}"] = r
-        del wl
     if args.workload != "prefill-8192":
         try:
             wl = Workload("prefill-8192", max_M=1024)
             for M in (64, 256, 1024):
-                r = measure(wl, M, max(5, steps // 10), 3, peaks, with_kernels=False)
+                r = measure(wl, M, max(20, steps // 4), 3, peaks, with_kernels=False, gpu_index=gpu_index)
                 r["tensor_frac"] = r["tflops"] / peaks["bf16_tflops"]
                 r["tensor_frac_sustained"] = r["tflops"] / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
                 res[f"prefill-8192 M={M}"] = r
             del wl
         except Exception as exc:  # the tensor-core path reports why it could not run
             res["prefill-8192"] = {"error": str(exc)[:300]}
+    for M in (4, 16):
+        res[f"{args.workload} M={M}"] = measure(main_wl, M, steps, 3, peaks, gpu_index=gpu_index)
+    for name, Ms in (("single-256", (1,)), ("smollm-135m-stack", (1, 4, 16)), ("vq16-4096-rht", (1, 8)),
+                     ("llama3-8b-mlp-corr", (1, 16))):
+        if name == args.workload:
+            continue
+        wl = Workload(name, max_M=16)
+        for M in Ms:
+            r = measure(wl, M, steps, 3, peaks, with_kernels=(name != "smollm-135m-stack"), gpu_index=gpu_index)
+            if name == "smollm-135m-stack":
+                r["us_per_transformer_layer"] = 1e3 * r["ms_per_step"] / 30
+            res[f"{name} M={M}"] = r
+        del wl
     for M in (1, 8):
         res[f"rotation 4096 M={M}"] = time_rotations(4096, M, steps)
         for label, shards in (("qkv 4096+1024+1024", (4096, 1024, 1024)), ("gate-up 14336+14336", (14336, 14336))):
@@ -711,7 +721,7 @@ def detail(args, peaks, main_wl):
             continue
         wl = Workload(name, max_M=8)
         for M in (1, 8):
-            res[f"{name} M={M}"] = measure(wl, M, steps, 3, peaks)
+            res[f"{name} M={M}"] = measure(wl, M, steps, 3, peaks, gpu_index=gpu_index)
         del wl
     from synth import FMT_RVQ12_4
     for fmt, sg, label in ((FMT_RVQ12_4, 64, "rvq12_4 block-64"), (FMT_VQ16, 4096, "vq16 per-row")):

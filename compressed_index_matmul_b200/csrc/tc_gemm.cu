@@ -13,10 +13,14 @@
 //              x 64, 128-byte swizzle) into a 4-stage ring.
 //   warp 1     allocates TMEM; lane 0 issues tcgen05.mma (M=128, N=T, K=16, four
 //              per k block, A read from TMEM) and commits each stage back.
-//   warps 2-17 decode: four warps per TMEM lane quarter; thread = one row of the
-//              tile (its TMEM lane); warp `part` of a quarter decodes every 4th k
-//              block (kb % 4 == part), all 8 groups of it, so A stage `part` is
-//              always written by the same 4 warps.  Per block a thread reads its 8
+//   warps 2.. decode: P warps per TMEM lane quarter (P = 3 for token tiles of 64
+//              and more, 4 for narrower ones); thread = one row of the tile (its
+//              TMEM lane); warp `part` of a quarter decodes every P-th k block
+//              (kb % P == part), all 8 groups of it, into A stage kb % 4.  With P = 3
+//              the CTA has 14 warps, at most four share an SM sub-partition and each
+//              thread may hold 128 registers (no spills); with P = 4, 18 warps and
+//              96 registers (the decode loop spills a little, but more warps hide
+//              its latency when each block's MMA is short).  Per block a thread reads its 8
 //              index bytes (plus nibbles and scale) from the staged slice, gathers
 //              the stage-1 codewords from shared memory and the stage-2 codewords
 //              from the warp's registers (shuffle), decodes with the
@@ -43,8 +47,9 @@ namespace vq {
 
 constexpr int kTcRows = 128;
 constexpr int kTcStages = 4;        // x tiles in shared memory and A tiles in TMEM
-constexpr int kTcDecodeWarps = 16;
-constexpr int kTcThreads = 64 + 32 * kTcDecodeWarps;
+// Decode warps per TMEM lane quarter (kParts, a template parameter): 3 for token
+// tiles of 64 and more, 4 for smaller ones (see the launch).
+__host__ __device__ constexpr int tc_threads(int parts) { return 64 + 32 * 4 * parts; }
 constexpr int kTcMaxT = 256;
 constexpr uint32_t kTcACols = 32;   // TMEM columns of one A stage (64 k of 16-bit pairs)
 // index-slice ring slot: lo 16 B, hi4 8 B, s2 8 B, scales 4 B per row (idx16: 32 B per row)
@@ -116,8 +121,8 @@ __device__ __forceinline__ void decode_two_stage(const uint4& c1, const uint32_t
   }
 }
 
-template <int FMT, typename T, bool kStaged>
-__global__ void __launch_bounds__(kTcThreads, 1)
+template <int FMT, typename T, bool kStaged, int kTcParts>
+__global__ void __launch_bounds__(tc_threads(kTcParts), 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap ymap, TcArgs p) {
   extern __shared__ unsigned char smem_raw[];
   constexpr bool k16 = (FMT == kFmtVq16 || FMT == kFmtVq16Rvq);
@@ -170,7 +175,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     for (int s = 0; s < kTcIdxSlots; ++s) {
       ptx::mbar_init(idx_full(s), 1);
-      ptx::mbar_init(idx_empty(s), kTcDecodeWarps / 2);  // the 8 warps that decode the slice's two blocks
+      ptx::mbar_init(idx_empty(s), 8);  // the 8 warps (two parts x four quarters) that decode the slice's two blocks
     }
     ptx::mbar_init(accum_bar, 1);
     ptx::mbar_init(cb_bar, 1);
@@ -277,11 +282,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ decode
-    // Warp (quarter q, part) decodes every 4th k block, kb = part, part+4, ...: all
-    // 8 groups of the block for its 32 rows, i.e. the whole A stage kb % 4 == part
+    // Warp (quarter q, part) decodes every P-th k block, kb = part, part+P, ...: all
+    // 8 groups of the block for its 32 rows, i.e. the whole A stage kb % 4
     // for its TMEM lane quarter.
     const int q = warp & 3;            // TMEM lane quarter of this warp
-    const int part = (warp - 2) >> 2;  // 0..3 == the A stage this warp writes
+    const int part = (warp - 2) >> 2;  // 0..kTcParts-1: this warp decodes blocks kb == part (mod kTcParts)
     const int dr = 32 * q + lane;      // row within the tile == TMEM lane
     const int r = row0 + dr;
     const bool valid = r < N;
@@ -292,16 +297,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       cb2r[0] = v.x; cb2r[1] = v.y; cb2r[2] = v.z; cb2r[3] = v.w;
     }
     const unsigned short row_scale = (!block_scales && valid) ? a.scales[r] : (unsigned short)0;
-    const uint32_t tlane = tmem + ((uint32_t)(32 * q) << 16) + acol0 + kTcACols * (uint32_t)part;
+    const uint32_t tlane0 = tmem + ((uint32_t)(32 * q) << 16) + acol0;  // + the A stage's columns
     bool ok = true;
     if (kSmemCb && !ptx::mbar_wait(cb_bar, 0, p.err)) {
       *abort_flag = 1;
       ok = false;
     }
-    for (int kb = part; ok && kb < nkb; kb += 4) {
+    for (int kb = part; ok && kb < nkb; kb += kTcParts) {
       const int j = kb >> 1, h = kb & 1;
       const int sl = s_first + j, w = slice_width(sl, G);
-      if (*abort_flag || (kb >= kTcStages && !ptx::mbar_wait(empty(part), ((kb / kTcStages) - 1) & 1, p.err)) ||
+      // A stage kb % kTcStages; the MMA of block kb - kTcStages must be done with it.
+      // (This warp's previous block, kb - kTcParts, already needed the MMA of block
+      // kb - kTcParts - kTcStages, so the stage's barrier is at most one phase behind.)
+      const int st = kb % kTcStages;
+      const uint32_t tlane = tlane0 + kTcACols * (uint32_t)st;
+      if (*abort_flag || (kb >= kTcStages && !ptx::mbar_wait(empty(st), ((kb / kTcStages) - 1) & 1, p.err)) ||
           (kStaged && !ptx::mbar_wait(idx_full(j % kTcIdxSlots), (j / kTcIdxSlots) & 1, p.err))) {
         *abort_flag = 1;
         ok = false;
@@ -375,7 +385,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(full_a(part));
+      if (lane == 0) ptx::mbar_arrive(full_a(st));
     }
     if (ok && !ptx::mbar_wait(accum_bar, 0, p.err)) *abort_flag = 1;
   }
@@ -390,7 +400,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int dr = 32 * q + lane, r = row0 + dr;
   const bool valid = r < N;
   const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16);
-  const int nch = p.T / 16;  // 16-token chunks; thread (row dr, part) handles chunks part, part+4, ...
+  const int nch = p.T / 16;  // 16-token chunks; thread (row dr, part) handles chunks part, part+P, ...
   if (p.epi != kEpiGlobal) {
     // y through a shared-memory staging tile ([chunk][16 tokens][128 rows] in the
     // codebook area, free now) and TMA tensor stores, which also clip the ragged
@@ -405,7 +415,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       ptx::cluster_sync();  // both CTAs are done with their x stages
       if (dec && fine) {
         ptx::tc_fence_after();
-        for (int ci = part; ci < nch; ci += 4) {
+        for (int ci = part; ci < nch; ci += kTcParts) {
           if ((uint32_t)(ci & 1) == rank || tok0 + 16 * ci >= M) continue;
           uint32_t v[16];
           ptx::tmem_ld16(taddr + 16 * ci, v);
@@ -419,7 +429,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     if (dec && fine) {
       ptx::tc_fence_after();
-      for (int ci = part; ci < nch; ci += 4) {
+      for (int ci = part; ci < nch; ci += kTcParts) {
         if ((pair && (uint32_t)(ci & 1) != rank) || tok0 + 16 * ci >= M) continue;
         uint32_t v[16];
         ptx::tmem_ld16(taddr + 16 * ci, v);
@@ -455,7 +465,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint16_t* y = static_cast<uint16_t*>(a.y);
     if (fine) {
       ptx::tc_fence_after();
-      for (int c0 = 16 * part; c0 < p.T; c0 += 64) {
+      for (int c0 = 16 * part; c0 < p.T; c0 += 16 * kTcParts) {
         uint32_t v[16];
         ptx::tmem_ld16(taddr + c0, v);
         ptx::tmem_wait_ld();
@@ -474,16 +484,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     if (fine && p.splits > 1) {
       __threadfence();
-      asm volatile("bar.sync 1, %0;" ::"n"(32 * kTcDecodeWarps) : "memory");
+      asm volatile("bar.sync 1, %0;" ::"n"(32 * 4 * kTcParts) : "memory");
       const int tile = blockIdx.y * gridDim.x + blockIdx.x;
       if (threadIdx.x == 64) *last_flag = (atomicAdd(&p.tickets[tile], 1u) == (uint32_t)(p.splits - 1));
-      asm volatile("bar.sync 1, %0;" ::"n"(32 * kTcDecodeWarps) : "memory");
+      asm volatile("bar.sync 1, %0;" ::"n"(32 * 4 * kTcParts) : "memory");
       if (*last_flag) {
         __threadfence();
         ptx::tc_fence_after();
         // Sixteen tokens per step, so each split's loads are all in flight at
         // once; this CTA's own split comes from its accumulator.
-        for (int c0 = 16 * part; c0 < p.T; c0 += 64) {
+        for (int c0 = 16 * part; c0 < p.T; c0 += 16 * kTcParts) {
           float acc[16];
           for (int k = 0; k < p.splits; ++k) {
             uint32_t t[16];
@@ -573,7 +583,7 @@ bool plan_tc(const vq_linear_desc& d, const DeviceInfo& dev, int M, Plan* p) {
   return true;
 }
 
-template <int FMT, typename T, bool kStaged>
+template <int FMT, typename T, bool kStaged, int kParts>
 static cudaError_t launch_tc_t(const LayerArgs& a, const TcGeom& g, float* scratch, uint32_t* tickets,
                                uint32_t* err, cudaStream_t s) {
   EncodeTiledFn enc = encode_fn();
@@ -599,14 +609,14 @@ static cudaError_t launch_tc_t(const LayerArgs& a, const TcGeom& g, float* scrat
     if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
   }
   const uint32_t smem = kTcTilesOffset + kTcStages * ((uint32_t)g.T * 128u) + 1024u;
-  auto kern = tc_gemm_kernel<FMT, T, kStaged>;
+  auto kern = tc_gemm_kernel<FMT, T, kStaged, kParts>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const bool partials = g.S > 1 && g.epi == kEpiGlobal;
   TcArgs p{a, g.epi, g.T, g.kps, g.S, partials ? scratch : nullptr, partials ? tickets : nullptr, err};
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(g.RT, g.TT, g.S);
-  cfg.blockDim = dim3(kTcThreads);
+  cfg.blockDim = dim3(tc_threads(kParts));
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -627,8 +637,17 @@ template <int FMT, typename T>
 static cudaError_t launch_tc_s(const LayerArgs& a, const TcGeom& g, float* scratch, uint32_t* tickets,
                                uint32_t* err, cudaStream_t s) {
   // Bulk copies need 16-byte sizes: N % 8 == 0 makes every per-slice run one.
-  return (a.N % 8 == 0) ? launch_tc_t<FMT, T, true>(a, g, scratch, tickets, err, s)
-                        : launch_tc_t<FMT, T, false>(a, g, scratch, tickets, err, s);
+  // Token tiles of 64 and more: 3 decode warps per quarter (14 warps, 128 registers
+  // each, no spills: the decode keeps up with the longer MMAs of a wide tile);
+  // narrower tiles: 4 (18 warps, 96 registers), more warps to hide the decode's
+  // latency when each block's MMA is short.  Measured on B200 (8192 x 8192 M = 256:
+  // 39.5 vs 43.1 us; Llama-3-8B gate M = 16 and the residual ladder at M = 8 are
+  // 3-18 % faster with 4).
+  if (g.T >= 64)
+    return (a.N % 8 == 0) ? launch_tc_t<FMT, T, true, 3>(a, g, scratch, tickets, err, s)
+                          : launch_tc_t<FMT, T, false, 3>(a, g, scratch, tickets, err, s);
+  return (a.N % 8 == 0) ? launch_tc_t<FMT, T, true, 4>(a, g, scratch, tickets, err, s)
+                        : launch_tc_t<FMT, T, false, 4>(a, g, scratch, tickets, err, s);
 }
 
 cudaError_t launch_tc(const LayerArgs& a, const Plan& pl, float* scratch, uint32_t* tickets, uint32_t* err,
@@ -647,8 +666,11 @@ cudaError_t launch_tc(const LayerArgs& a, const Plan& pl, float* scratch, uint32
       return bf ? launch_tc_s<kFmtRvq12_4, __nv_bfloat16>(a, g, scratch, tickets, err, s)
                 : launch_tc_s<kFmtRvq12_4, __half>(a, g, scratch, tickets, err, s);
     case kFmtVq16Rvq:  // the ladder's indices are read directly (no staging ring)
-      return bf ? launch_tc_t<kFmtVq16Rvq, __nv_bfloat16, false>(a, g, scratch, tickets, err, s)
-                : launch_tc_t<kFmtVq16Rvq, __half, false>(a, g, scratch, tickets, err, s);
+      if (g.T >= 64)
+        return bf ? launch_tc_t<kFmtVq16Rvq, __nv_bfloat16, false, 3>(a, g, scratch, tickets, err, s)
+                  : launch_tc_t<kFmtVq16Rvq, __half, false, 3>(a, g, scratch, tickets, err, s);
+      return bf ? launch_tc_t<kFmtVq16Rvq, __nv_bfloat16, false, 4>(a, g, scratch, tickets, err, s)
+                : launch_tc_t<kFmtVq16Rvq, __half, false, 4>(a, g, scratch, tickets, err, s);
     default:
       return bf ? launch_tc_s<kFmtVq16, __nv_bfloat16>(a, g, scratch, tickets, err, s)
                 : launch_tc_s<kFmtVq16, __half>(a, g, scratch, tickets, err, s);
