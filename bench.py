@@ -286,8 +286,11 @@ class Workload:
             events[len(calls)].record()
 
     def rotation_fused(self, spec, M):
-        """True where vq_linear_forward_rotated is one kernel (the batch-1 gather kernel)."""
-        return M == 1 and spec.fmt in _16BIT and spec.K % 128 == 0 and spec.K <= 16384 and spec.N % 4 == 0
+        """True where vq_linear_forward_rotated is one kernel: the automatic choice is the
+        16-bit gather kernel (M <= 4), which rotates x itself."""
+        mt = 1 if M <= 1 else 2 if M <= 2 else 4
+        return (M <= 4 and spec.fmt in _16BIT and spec.K % 128 == 0 and spec.K <= 16384 and mt * spec.K <= 32768
+                and spec.N % 4 == 0)
 
     def launches_per_step(self, M):
         n = 0
@@ -563,12 +566,11 @@ def gpu_arm(args):
         launch_source = "CUDA event nodes between the forwards"
     per_fwd_eff = [fwd_ms / max(1, launches_per_fwd[0]) if uniform else fwd_ms] * len(wl.layers)
     achieved = sum(bytes_per_fwd) / (sum(per_fwd_eff) * 1e-3) / 1e9
-    fmt0 = wl.layers[0][1].fmt
-    dominant = ("lut_gemv_kernel" if M == 1 and fmt0 not in _16BIT else
-                "vq16_gemv_kernel" if M == 1 else "gemv_kernel" if M <= 16 else "tc_gemm_kernel")
+    # the kernel the library plans for the first weight matrix (the step's largest)
+    dominant = kernel_of_path(wl.layers[0][2].plan(M)["path"])
     traffic = lookup_traffic(dominant, args.workload, M)
     avg_launch_us = round(1e3 * float(np.mean(per_fwd_eff)), 3)
-    if dominant == "tc_gemm_kernel":
+    if M > 16:
         # a dense contraction: 2*M*N*K flops per forward against the bf16 tensor peak
         flops_per_fwd = [2.0 * M * spec.N * spec.K for _, spec, _ in wl.layers]
         tflops = sum(flops_per_fwd) / (sum(per_fwd_eff) * 1e-3) / 1e12
@@ -611,7 +613,7 @@ def gpu_arm(args):
                    "parallelism": f"replicas x{world}",
                    "l2": L2_NOTE.format(r=R, mb=R * wl.weight_bytes() / 1e6) + (
                        "; the 65,536-entry codebook is one table shared by the copies (L2-resident)"
-                       if fmt0 in _16BIT else ""),
+                       if wl.layers[0][1].fmt in _16BIT else ""),
                    "layer": ("MLP step / 3 weight matrices: gate and up (same x) run concurrently on two "
                              "streams, half of the SMs each (vq_linear_set_sm_budget), then down"
                              if wl.concurrent_gate_up else "one vq_linear_forward (one weight matrix)"),
@@ -653,6 +655,14 @@ def aggregate_over_ranks(total_ms_local: float, steps: int, layers_per_step: int
     total_ms = max_over_ranks(total_ms_local, world)
     ms_per_step = total_ms / steps
     return ms_per_step, 1e3 * ms_per_step / (layers_per_step * world)
+
+
+
+def kernel_of_path(path):
+    import compressed_index_matmul_b200 as vq
+
+    return {vq.VQ_PATH_LUT: "lut_gemv_kernel", vq.VQ_PATH_GATHER: "vq16_gemv_kernel",
+            vq.VQ_PATH_GEMV: "gemv_kernel", vq.VQ_PATH_TC: "tc_gemm_kernel"}[path]
 
 
 KERNEL_UNITS = {"lut_gemv_kernel": "lut_gemv.cu", "vq16_gemv_kernel": "vq16_gemv.cu", "tc_gemm_kernel": "tc_gemm.cu",

@@ -38,6 +38,7 @@ from ._binding import (  # noqa: F401
     vq_linear_forward_noalloc,
     vq_linear_forward_rotated,
     vq_linear_launches,
+    vq_linear_plan,
     vq_linear_set_path,
     vq_linear_set_sm_budget,
     vq_rht_apply,

@@ -31,7 +31,7 @@ STATUS_NAMES = {0: "VQ_OK", 1: "VQ_ERR_INVALID_ARG", 2: "VQ_ERR_UNSUPPORTED", 3:
 # Every entry point the header declares (checked by the tests against the .so).
 EXPORTS = ("vq_abi_version", "vq_linear_create", "vq_linear_destroy", "vq_linear_set_path", "vq_linear_set_sm_budget",
            "vq_linear_forward",
-           "vq_linear_forward_noalloc", "vq_linear_forward_rotated", "vq_linear_launches", "vq_rht_apply", "vq_rht_apply_output", "vq_rht_apply_output_sharded", "vq_encode", "vq_linear_check", "vq_last_error",
+           "vq_linear_forward_noalloc", "vq_linear_forward_rotated", "vq_linear_launches", "vq_linear_plan", "vq_rht_apply", "vq_rht_apply_output", "vq_rht_apply_output_sharded", "vq_encode", "vq_linear_check", "vq_last_error",
            "vq_debug_unpack", "vq_debug_dequant", "vq_debug_wait_timeout")
 
 
@@ -52,6 +52,11 @@ class vq_planes(ctypes.Structure):
     _fields_ = [("lo", ctypes.c_void_p), ("hi4", ctypes.c_void_p), ("s2", ctypes.c_void_p),
                 ("idx16", ctypes.c_void_p), ("idx8", ctypes.c_void_p),
                 ("corr_rows", ctypes.c_void_p), ("corr_cols", ctypes.c_void_p), ("corr_vals", ctypes.c_void_p)]
+
+
+class vq_plan_info(ctypes.Structure):
+    _fields_ = [("path", ctypes.c_int32), ("launches", ctypes.c_int32), ("ctas", ctypes.c_int32),
+                ("splits", ctypes.c_int32)]
 
 
 class vq_codebooks(ctypes.Structure):
@@ -97,6 +102,8 @@ def load(path: str | None = None):
         lib.vq_debug_wait_timeout.argtypes = [P, P]
         lib.vq_linear_launches.restype = I32
         lib.vq_linear_launches.argtypes = [P, I32]
+        lib.vq_linear_plan.restype = st
+        lib.vq_linear_plan.argtypes = [P, I32, ctypes.POINTER(vq_plan_info)]
         lib.vq_linear_forward_rotated.restype = st
         lib.vq_linear_forward_rotated.argtypes = [P, P, P, ctypes.POINTER(vq_planes), ctypes.POINTER(vq_codebooks), P,
                                                   P, I32, I32, I32, P]
@@ -186,6 +193,13 @@ def vq_linear_set_sm_budget(h, sms: int) -> None:
 
 def vq_linear_launches(h, M: int) -> int:
     return load().vq_linear_launches(h, M)
+
+
+def vq_linear_plan(h, M: int) -> dict:
+    """How vq_linear_forward runs this M: path, launches, ctas, splits."""
+    info = vq_plan_info()
+    _check(load().vq_linear_plan(h, M, ctypes.byref(info)))
+    return {name: getattr(info, name) for name, _ in vq_plan_info._fields_}
 
 
 def vq_linear_forward(h, x, planes: vq_planes, codebooks: vq_codebooks, scales, y, M, N, K, stream=None) -> None:

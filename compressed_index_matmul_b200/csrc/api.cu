@@ -364,6 +364,21 @@ VQ_API int32_t vq_linear_launches(vq_linear_t h, int32_t M) {
   return p.launches + (h->d.corr ? 1 : 0);  // the sparse correction's kernel
 }
 
+VQ_API vq_status vq_linear_plan(vq_linear_t h, int32_t M, vq_plan_info* out) {
+  if (h == nullptr || out == nullptr) return fail(VQ_ERR_INVALID_ARG, "handle or out is NULL");
+  if (M < 1 || M > h->d.max_M) return fail(VQ_ERR_INVALID_ARG, "M=%d outside [1, max_M=%d]", M, h->d.max_M);
+  vq::Plan p{};
+  if (!vq::plan_forward(h->d, h->dev, M, h->path, &p))
+    return fail(VQ_ERR_UNSUPPORTED, "path %d cannot run M=%d for this layer", h->path, M);
+  if ((p.path == VQ_PATH_LUT || p.path == VQ_PATH_GATHER) && h->sm_budget > 0 && p.grid > h->sm_budget)
+    p.ctas = h->sm_budget;  // as the forward clamps its grid
+  out->path = p.path;
+  out->launches = p.launches + (h->d.corr ? 1 : 0);
+  out->ctas = p.ctas;
+  out->splits = p.splits;
+  return VQ_OK;
+}
+
 VQ_API vq_status vq_linear_forward(vq_linear_t h, const void* x, const vq_planes* planes,
                                    const vq_codebooks* codebooks, const void* scales, void* y, int32_t M,
                                    int32_t N, int32_t K, void* stream) {
@@ -429,8 +444,11 @@ VQ_API vq_status vq_linear_forward_rotated(vq_linear_t h, const void* x, const i
   if (!vq::plan_forward(d, h->dev, M, h->path, &p))
     return fail(VQ_ERR_UNSUPPORTED, "path %d cannot run M=%d", h->path, M);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (p.path == VQ_PATH_GATHER && M == 1 && !d.corr) {  // the kernel rotates x itself
-    // (a sparse correction needs the rotated x too: that layer takes the route below)
+  // Where the forward runs the 16-bit gather kernel (automatically up to M = 4, or
+  // forced up to M = 8) that kernel rotates x itself: one launch, no rotated copy of
+  // x in memory.  (A sparse correction needs the rotated x too: that layer takes the
+  // route below.)
+  if (p.path == VQ_PATH_GATHER && !d.corr) {
     if (h->sm_budget > 0 && p.grid > h->sm_budget) p.grid = h->sm_budget;
     if (p.scratch_bytes > h->scratch_bytes)
       return fail(VQ_ERR_UNSUPPORTED, "plan needs %zu scratch bytes, handle has %zu", p.scratch_bytes,

@@ -97,8 +97,9 @@ __global__ void __launch_bounds__(256) gemv_kernel(LayerArgs a, int k_per_split,
   constexpr bool k16 = (FMT == kFmtVq16 || FMT == kFmtVq16Rvq);
   constexpr bool kSmemCb = !k16;
   constexpr bool kTwo = (FMT == kFmtRvq12_4);
-  uint4* cb1s = reinterpret_cast<uint4*>(smem);                                // 4096 entries
-  uint4* cb2s = cb1s + (kSmemCb ? 4096 : 0);                                   // 16 entries
+  constexpr bool kLadder = (FMT == kFmtVq16Rvq);
+  uint4* cb1s = reinterpret_cast<uint4*>(smem);  // 4096 entries (12-bit formats); the ladder's 8-bit codebook
+  uint4* cb2s = cb1s + (kSmemCb ? 4096 : (kLadder ? 256 : 0));                 // 16 entries
   uint64_t* bar = reinterpret_cast<uint64_t*>(cb2s + (kTwo ? 16 : 0));         // codebook barrier
   int* flag = reinterpret_cast<int*>(bar + 1);
   uint16_t* xs = reinterpret_cast<uint16_t*>(bar + 2);
@@ -123,6 +124,7 @@ __global__ void __launch_bounds__(256) gemv_kernel(LayerArgs a, int k_per_split,
     ptx::bulk_load(smem_u32(cb1s), a.cb1, 65536u, b);
     if (kTwo) ptx::bulk_load(smem_u32(cb2s), a.cb2, 256u, b);
   }
+  if (kLadder) stage_cb8(a, cb1s, threadIdx.x, blockDim.x);
   BlockIdx<FMT> cur, nxt;
   {
     const int kb = 0, kblock = k0 + kb + 64 * c;
@@ -177,7 +179,7 @@ __global__ void __launch_bounds__(256) gemv_kernel(LayerArgs a, int k_per_split,
         const uint4 c1 = kSmemCb ? cb1s[i1] : __ldg(reinterpret_cast<const uint4*>(a.cb1) + i1);
         if constexpr (FMT == kFmtVq16Rvq) {
           float v[8];
-          ladder_sum(a, cur.res[r], q, c1, v);
+          ladder_sum(a, cur.res[r], q, c1, cb1s, v);
           pack_scaled<T>(v, active ? s[r] : 0.f, wq[r]);
         } else {
           const uint4 c2 = kTwo ? cb2s[i2] : c1;
@@ -241,7 +243,7 @@ template <int FMT, typename T, int NT>
 static cudaError_t launch_one(const LayerArgs& a, const Plan& p, float* scratch, uint32_t* tickets, cudaStream_t s) {
   const int kc = p.k_per_split;
   const bool k16 = (FMT == kFmtVq16 || FMT == kFmtVq16Rvq);
-  const size_t smem = (!k16 ? 4096 * 16 : 0) + (FMT == kFmtRvq12_4 ? 256 : 0) + 16 +
+  const size_t smem = (!k16 ? 4096 * 16 : 0) + (FMT == kFmtVq16Rvq ? 256 * 16 : 0) + (FMT == kFmtRvq12_4 ? 256 : 0) + 16 +
                       (size_t)8 * NT * (kc + 8) * 2;
   auto kern = gemv_kernel<FMT, T, NT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -298,6 +300,7 @@ void plan_gemv(const vq_linear_desc& d, const DeviceInfo& dev, int M, Plan* p) {
   p->launches = 1;
   p->scratch_bytes = S > 1 ? (size_t)S * M * d.N * sizeof(float) : 0;
   p->tickets = S > 1 ? row_tiles : 0;
+  p->ctas = row_tiles * S;
 }
 
 }  // namespace vq

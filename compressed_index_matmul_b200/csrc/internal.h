@@ -49,6 +49,7 @@ struct Plan {
   int tickets;       // completion counters needed (zero between forwards)
   int sync_words;    // words of the batch-1 table kernel's cross-CTA protocol (kept apart from the tickets)
   int grid;          // CTAs of the persistent batch-1 kernels (VQ_PATH_LUT / GATHER), else 0
+  int ctas;          // CTAs of the main kernel (vq_linear_plan)
 };
 
 struct DeviceInfo {
@@ -65,9 +66,8 @@ bool plan_forward(const vq_linear_desc& d, const DeviceInfo& dev, int M, int for
 // every forward leaves them zero again.
 cudaError_t launch_gemv(const LayerArgs& a, const Plan& p, float* scratch, uint32_t* tickets, cudaStream_t s);
 // The batch-1 table kernel (p.grid CTAs).  `sync` is the handle's array of
-// p.sync_words words for its end-of-kernel protocol (an arrival counter, a
-// generation word and one claim word per 32-row unit): zero at create; every
-// forward leaves the counter at zero and every claim word equal to the generation.
+// p.sync_words words for its grid barrier (an arrival counter and a generation
+// word): zero at create; every forward leaves the counter at zero.
 cudaError_t launch_lut(const LayerArgs& a, const Plan& p, float* scratch, uint32_t* sync, uint32_t* err,
                        cudaStream_t s);
 // The few-token kernel of the 16-bit formats (VQ_PATH_GATHER, clusters of 2

@@ -54,9 +54,10 @@ __device__ __forceinline__ void fma_codeword(float m, const uint4& c, float (&v)
   }
 }
 
-// Stage sum of group g (0..7) of a block whose primary codeword is c1.
+// Stage sum of group g (0..7) of a block whose primary codeword is c1; cb8s is the
+// 8-bit codebook staged in shared memory.
 __device__ __forceinline__ void ladder_sum(const LayerArgs& a, const LadderIdx& q, int g, const uint4& c1,
-                                           float (&v)[8]) {
+                                           const uint4* cb8s, float (&v)[8]) {
   const uint32_t w1[4] = {c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
   for (int p = 0; p < 4; ++p) {
@@ -71,9 +72,16 @@ __device__ __forceinline__ void ladder_sum(const LayerArgs& a, const LadderIdx& 
       fma_codeword(a.mult[t - 2], __ldg(reinterpret_cast<const uint4*>(a.cbr[t - 2]) + i), v);
     } else if (t == a.n16 + 1 && a.n8) {
       const uint32_t i = (q.r[t - 2][g >> 2] >> (8 * (g & 3))) & 0xFFu;
-      fma_codeword(a.mult[t - 2], __ldg(reinterpret_cast<const uint4*>(a.cb8) + i), v);
+      fma_codeword(a.mult[t - 2], cb8s[i], v);
     }
   }
+}
+
+// Copies the 8-bit codebook (256 entries) into shared memory, thread `tid` of
+// `nthreads`; the caller's next CTA barrier makes it visible.
+__device__ __forceinline__ void stage_cb8(const LayerArgs& a, uint4* cb8s, int tid, int nthreads) {
+  if (!a.n8) return;
+  for (int i = tid; i < 256; i += nthreads) cb8s[i] = __ldg(reinterpret_cast<const uint4*>(a.cb8) + i);
 }
 
 // Eight materialised weights RN_T(fl32(s * v)) as four packed pairs.

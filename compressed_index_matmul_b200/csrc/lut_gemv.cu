@@ -517,6 +517,7 @@ bool plan_lut(const vq_linear_desc& d, const DeviceInfo& dev, int M, Plan* p) {
   p->tickets = 0;
   p->sync_words = g.S > 1 ? 2 : 0;  // the grid barrier's arrival counter and generation
   p->grid = g.grid;
+  p->ctas = g.grid;
   return true;
 }
 

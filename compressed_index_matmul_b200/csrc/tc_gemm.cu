@@ -186,6 +186,8 @@ __global__ void __launch_bounds__(tc_threads(kTcParts), 1)
     ptx::tmem_alloc(smem_u32(tmem_slot), tcols);
     ptx::tmem_relinquish();
   }
+  // The ladder's 8-bit codebook into the (otherwise unused) codebook area.
+  if (kLadder) stage_cb8(a, const_cast<uint4*>(cb1s), threadIdx.x, blockDim.x);
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
@@ -368,7 +370,7 @@ __global__ void __launch_bounds__(tc_threads(kTcParts), 1)
           const uint4 c1 = kSmemCb ? cb1s[i1] : __ldg(cbg + i1);
           if constexpr (kLadder) {
             float v[8];
-            ladder_sum(a, res, g, c1, v);
+            ladder_sum(a, res, g, c1, cb1s, v);
             pack_scaled<T>(v, scf, out + 4 * t);
           } else if (kTwo) {
             const int i2 = (int)((s24w >> (4 * g)) & 15u);
@@ -580,6 +582,7 @@ bool plan_tc(const vq_linear_desc& d, const DeviceInfo& dev, int M, Plan* p) {
   const bool partials = g.S > 1 && g.epi == kEpiGlobal;
   p->scratch_bytes = partials ? (size_t)g.S * M * d.N * sizeof(float) : 0;
   p->tickets = partials ? g.RT * g.TT : 0;
+  p->ctas = g.RT * g.TT * g.S;
   return true;
 }
 

@@ -1,7 +1,7 @@
 // Small-batch GEMV for the 16-bit formats (1 <= M <= 8, VQ_FMT_VQ16 and the residual
 // ladder VQ_FMT_VQ16_RVQ,
 // K % 128 == 0, K <= 16384, M K <= 32768, N % 4 == 0), with the input rotation
-// optionally applied inside the kernel at M == 1.
+// optionally applied inside the kernel.
 //
 // GLQ README, "How it works": one 16-bit index per group of 8 weights selects a
 // codeword of a 65,536 x 8 codebook (1 MiB of fp16), too large for shared memory;
@@ -13,8 +13,8 @@
 // codeword serves all M tokens.
 //
 // Rotated input (GLQ README, "How it works": random sign flips followed by a fast
-// Walsh-Hadamard transform): when `signs` is given (M == 1), every CTA computes the
-// whole rotated vector x' = H (signs . x) in fp32 in shared memory
+// Walsh-Hadamard transform): when `signs` is given, every CTA computes the whole
+// rotated input x'_m = H (signs . x_m) of every token in fp32 in shared memory
 // (hadamard_blocks_to_smem, rotate.cuh); for a power-of-two K the orthonormal factor
 // 1/sqrt(K) multiplies every partial sum, otherwise ("Bit widths": block-diagonal
 // transform over the binary expansion of K) each block of x' is scaled by its own
@@ -52,17 +52,21 @@ constexpr int kV16MaxM = 8;           // tokens
 constexpr int kV16MaxMK = 32768;      // tokens x K (the fp32 x of all tokens is in shared memory)
 constexpr int kV16PartBytes = 65536;  // partial sums of one block
 
+constexpr int kV16Cb8Bytes = 256 * 16;  // the ladder's 8-bit codebook
+
 // Shared memory of one CTA: partials [ceil(S / C)][MT][rblk], row sums [MT][rblk],
-// fp32 x [MT][K] (byte offsets, 16-byte aligned; rblk is a multiple of 4).
+// fp32 x [MT][K], and for the residual ladder its 8-bit codebook (byte offsets,
+// 16-byte aligned; rblk is a multiple of 4).
 struct V16Smem {
-  int off_sum, off_x, bytes;
+  int off_sum, off_x, off_cb8, bytes;
 };
-__host__ __device__ inline V16Smem v16_smem(int S, int MT, int rblk, int K) {
+__host__ __device__ inline V16Smem v16_smem(int S, int MT, int rblk, int K, bool ladder) {
   V16Smem m;
   const int spc = (S + kV16Cluster - 1) / kV16Cluster;
   m.off_sum = spc * MT * rblk * 4;
   m.off_x = m.off_sum + MT * rblk * 4;
-  m.bytes = m.off_x + 4 * MT * K;
+  m.off_cb8 = m.off_x + 4 * MT * K;
+  m.bytes = m.off_cb8 + (ladder ? kV16Cb8Bytes : 0);
   return m;
 }
 
@@ -119,7 +123,7 @@ __global__ void __launch_bounds__(kV16Consumers, 1)
                      int rblk) {
   extern __shared__ __align__(128) unsigned char smem[];
   const int N = a.N, K = a.K, M = a.M;
-  const V16Smem lay = v16_smem(S, MT, rblk, K);
+  const V16Smem lay = v16_smem(S, MT, rblk, K, kLadder);
   float* part = reinterpret_cast<float*>(smem);                 // [ceil(S / C)][MT][rblk]
   float* csum = reinterpret_cast<float*>(smem + lay.off_sum);  // [MT][rblk]
   float* xs = reinterpret_cast<float*>(smem + lay.off_x);      // [MT][K]
@@ -148,11 +152,21 @@ __global__ void __launch_bounds__(kV16Consumers, 1)
   V16Pos cur{}, nxt{};
   int bi = 0, p0 = 0, r0 = 0, nrows = block_rows(0, r0);
   if (tid < ns * nrows) load_pos(tid, r0, nrows, cur);
+  // The ladder's 8-bit codebook (4 KiB) is gathered from shared memory: an L1 gather
+  // of 32 random entries touches up to 32 different lines, a shared one at most 32
+  // bank quads.  Visible to all threads after the barrier that ends the x staging.
+  const uint4* cb8s = reinterpret_cast<const uint4*>(smem + lay.off_cb8);
+  if (kLadder && a.n8 && tid < kV16Cb8Bytes / 16)
+    reinterpret_cast<uint4*>(smem + lay.off_cb8)[tid] = __ldg(reinterpret_cast<const uint4*>(a.cb8) + tid);
 
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  if (MT == 1 && signs) {
-    hadamard_blocks_to_smem<T, kV16Consumers, kV16MaxK>(static_cast<const uint16_t*>(a.x), signs, xs, K, tid,
-                                                        (K & (K - 1)) != 0);
+  if (signs) {
+    // every token's rotation (the padding tokens M .. MT-1 are zero; the rotations'
+    // barriers order those stores before any read)
+    for (int i = M * K + tid; i < MT * K; i += kV16Consumers) xs[i] = 0.f;
+    for (int m = 0; m < M; ++m)
+      hadamard_blocks_to_smem<T, kV16Consumers, kV16MaxK>(static_cast<const uint16_t*>(a.x) + (int64_t)m * K, signs,
+                                                          xs + m * K, K, tid, (K & (K - 1)) != 0);
   } else {
     const uint16_t* xg = static_cast<const uint16_t*>(a.x);
     for (int i = tid; i < MT * K; i += kV16Consumers) xs[i] = i < M * K ? Elt<T>::to_f32(xg[i]) : 0.f;
@@ -205,8 +219,7 @@ __global__ void __launch_bounds__(kV16Consumers, 1)
           for (int t = 2; t <= nst; ++t) {
             const bool is8 = t > a.n16;
             const float mt = t == 2 ? a.mult[0] : (t == 3 ? a.mult[1] : a.mult[2]);
-            const uint4* cbt = reinterpret_cast<const uint4*>(
-                is8 ? a.cb8 : (t == 2 ? a.cbr[0] : (t == 3 ? a.cbr[1] : a.cbr[2])));
+            const uint4* cbt = reinterpret_cast<const uint4*>(t == 2 ? a.cbr[0] : (t == 3 ? a.cbr[1] : a.cbr[2]));
             uint32_t jw[8];
 #pragma unroll
             for (int q = 0; q < 8; ++q) jw[q] = nw[q];
@@ -214,8 +227,10 @@ __global__ void __launch_bounds__(kV16Consumers, 1)
             uint4 cr[16];
 #pragma unroll
             for (int g = 0; g < 16; ++g) {
-              const uint32_t i = is8 ? (jw[g >> 2] >> (8 * (g & 3))) & 0xFFu : (jw[g >> 1] >> (16 * (g & 1))) & 0xFFFFu;
-              cr[g] = __ldg(cbt + i);
+              if (is8)
+                cr[g] = cb8s[(jw[g >> 2] >> (8 * (g & 3))) & 0xFFu];
+              else
+                cr[g] = __ldg(cbt + ((jw[g >> 1] >> (16 * (g & 1))) & 0xFFFFu));
             }
             float tb[MT][2];
 #pragma unroll
@@ -315,8 +330,8 @@ static V16Geom v16_geom(int N, int clusters, int S, int MT) {
 }
 
 // Largest shared-memory size of any launch: capped partials, row sums of 8 tokens x
-// 512 rows, fp32 x of M K <= kV16MaxMK inputs.
-static int v16_max_smem() { return kV16PartBytes + kV16MaxM * kV16MaxBlk * 4 + 4 * kV16MaxMK; }
+// 512 rows, fp32 x of M K <= kV16MaxMK inputs, the ladder's 8-bit codebook.
+static int v16_max_smem() { return kV16PartBytes + kV16MaxM * kV16MaxBlk * 4 + 4 * kV16MaxMK + kV16Cb8Bytes; }
 
 static int v16_max_clusters(int num_sms) {
   static std::atomic<int> cached[64];
@@ -359,6 +374,7 @@ bool plan_vq16(const vq_linear_desc& d, const DeviceInfo& dev, int M, Plan* p) {
   p->scratch_bytes = 0;  // partial sums stay in shared memory
   p->tickets = 0;
   p->grid = g.ncl * kV16Cluster;
+  p->ctas = p->grid;
   return true;
 }
 
@@ -383,7 +399,7 @@ static cudaError_t launch_vq16_t(const LayerArgs& a, int grid, const int8_t* sig
   int ncl = grid / kV16Cluster;
   if (ncl < 1) ncl = 1;
   const V16Geom g = v16_geom(a.N, ncl, S, MT);
-  const int smem = v16_smem(S, MT, g.rblk, a.K).bytes;
+  const int smem = v16_smem(S, MT, g.rblk, a.K, kLadder).bytes;
   // Orthonormal factor of the rotation, rounded once from double precision: a
   // power-of-two K takes it at the store; otherwise each block was scaled in shared
   // memory
@@ -410,9 +426,9 @@ template <typename T, bool kLadder>
 static cudaError_t launch_vq16_m(const LayerArgs& a, int grid, const int8_t* signs, cudaStream_t s) {
   switch (v16_mt(a.M)) {
     case 1: return launch_vq16_t<T, 1, kLadder>(a, grid, signs, s);
-    case 2: return launch_vq16_t<T, 2, kLadder>(a, grid, nullptr, s);
-    case 4: return launch_vq16_t<T, 4, kLadder>(a, grid, nullptr, s);
-    default: return launch_vq16_t<T, 8, kLadder>(a, grid, nullptr, s);
+    case 2: return launch_vq16_t<T, 2, kLadder>(a, grid, signs, s);
+    case 4: return launch_vq16_t<T, 4, kLadder>(a, grid, signs, s);
+    default: return launch_vq16_t<T, 8, kLadder>(a, grid, signs, s);
   }
 }
 

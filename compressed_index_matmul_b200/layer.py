@@ -101,6 +101,10 @@ class VQLinear:
     def launches(self, M: int) -> int:
         return B.vq_linear_launches(self.handle, M)
 
+    def plan(self, M: int) -> dict:
+        """How a forward of M tokens runs (path, launches, ctas, splits)."""
+        return B.vq_linear_plan(self.handle, M)
+
     def close(self):
         if getattr(self, "handle", None):
             B.vq_linear_destroy(self.handle)

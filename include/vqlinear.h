@@ -118,7 +118,7 @@ enum {
   VQ_PATH_GEMV = 2,   /* 1 <= M <= 16: decode to registers, warp MMA, split-K */
   VQ_PATH_TC = 3,     /* any M: decode into tensor memory, tcgen05 MMA (fp32 in TMEM) */
   VQ_PATH_GATHER = 4  /* 1 <= M <= 8, 16-bit formats only: codewords gathered from L2
-                         into fp32 dot products; at M == 1 it can apply the input
+                         into fp32 dot products; it can apply the input
                          rotation itself */
 };
 
@@ -201,11 +201,13 @@ vq_status vq_linear_set_path(vq_linear_t h, int32_t path);
 /* Limit the persistent batch-1 kernels (VQ_PATH_LUT, VQ_PATH_GATHER) of this
  * handle to `sms` CTAs, one per SM; 0 restores the default (every SM).  Two
  * independent forwards (say the gate and up projections of an MLP, both reading
- * the same x) can then run concurrently on two streams on about disjoint SMs.  No
- * CTA of these kernels waits for another, so any budgets are correct; budgets
- * that add up to more than the SM count only serialise part of the work.  The
- * other kernels are not persistent and ignore the budget.  Returns
- * VQ_ERR_INVALID_ARG when `sms` is negative or above the device's SM count. */
+ * the same x) can then run concurrently on two streams on about disjoint SMs.
+ * The table kernel's CTAs meet at a grid barrier, and its launch is cooperative:
+ * it starts only when all of its CTAs can be resident, so budgets that add up to
+ * more than the SM count serialise part of the work instead of deadlocking.  The
+ * gather kernel's CTAs wait only for the partner CTA of their cluster.  The other
+ * kernels are not persistent and ignore the budget.  Returns VQ_ERR_INVALID_ARG
+ * when `sms` is negative or above the device's SM count. */
 vq_status vq_linear_set_sm_budget(vq_linear_t h, int32_t sms);
 
 /* y = x . W^T with W decoded on the fly from planes / codebooks / scales
@@ -270,9 +272,11 @@ vq_status vq_linear_forward_noalloc(const vq_linear_desc* desc, const void* x, c
  * a device int8 array of +1/-1 [K] (16-byte aligned, like every pointer); K must
  * be a multiple of 64, 64 <= K <= 32768 (block-diagonal when not a power of two,
  * as in vq_rht_apply).
- *   - Where VQ_PATH_GATHER runs with M == 1 (VQ_FMT_VQ16, K <= 16384) this is one
- *     kernel: every CTA rotates x in fp32 in shared memory and uses it unrounded;
- *     nothing else is written.
+ *   - Where vq_linear_forward would run VQ_PATH_GATHER (by the automatic choice,
+ *     1 <= M <= 4, or forced with vq_linear_set_path, 1 <= M <= 8) and the layer
+ *     has no sparse correction, this is one kernel: every CTA rotates each token
+ *     of x in fp32 in shared memory and uses it unrounded; nothing else is
+ *     written.
  *   - Otherwise it enqueues vq_rht_apply into a buffer of the handle (allocated
  *     by vq_linear_create when desc->rht == 1: max_M x K elements) followed by
  *     vq_linear_forward on it, so the rotated x is rounded to the activation type
@@ -286,6 +290,23 @@ vq_status vq_linear_forward_rotated(vq_linear_t h, const void* x, const int8_t* 
 /* Number of kernels vq_linear_forward enqueues for this M (0 for M == 0; one
  * more when the handle carries a sparse correction), or -1 if M is out of range. */
 int32_t vq_linear_launches(vq_linear_t h, int32_t M);
+
+/* How vq_linear_forward runs this M, with the handle's forced path and SM
+ * budget; nothing is launched.
+ *   path      the kernel family (VQ_PATH_*, never VQ_PATH_AUTO);
+ *   launches  as vq_linear_launches;
+ *   ctas      CTAs of the main kernel;
+ *   splits    K splits per output tile (1: none; the table kernel's 128-input
+ *             slices; the gather kernel's slices).
+ * VQ_ERR_INVALID_ARG for a NULL handle or `out`, or M outside [1, max_M];
+ * VQ_ERR_UNSUPPORTED when the forced path cannot take this M. */
+typedef struct {
+  int32_t path;
+  int32_t launches;
+  int32_t ctas;
+  int32_t splits;
+} vq_plan_info;
+vq_status vq_linear_plan(vq_linear_t h, int32_t M, vq_plan_info* out);
 
 /* Randomised Hadamard rotation of the input (GLQ README, "How it works",
  * Randomized Hadamard Transform): for every row m,

@@ -105,6 +105,7 @@ def test_null_arguments_are_rejected(lib):
     assert lib.vq_linear_set_path(None, 0) == B.VQ_ERR_INVALID_ARG
     assert lib.vq_linear_set_sm_budget(None, 0) == B.VQ_ERR_INVALID_ARG
     assert lib.vq_linear_launches(None, 1) == -1
+    assert lib.vq_linear_plan(None, 1, None) == B.VQ_ERR_INVALID_ARG
     assert lib.vq_linear_destroy(None) == B.VQ_OK
     assert lib.vq_linear_check(None, None) == B.VQ_ERR_INVALID_ARG
 
@@ -207,7 +208,8 @@ def test_struct_offsets_match_the_c_header(tmp_path):
 
     fields = {"vq_linear_desc": [f for f, _ in B.vq_linear_desc._fields_],
               "vq_planes": [f for f, _ in B.vq_planes._fields_],
-              "vq_codebooks": [f for f, _ in B.vq_codebooks._fields_]}
+              "vq_codebooks": [f for f, _ in B.vq_codebooks._fields_],
+              "vq_plan_info": [f for f, _ in B.vq_plan_info._fields_]}
     src = ["#include <stddef.h>", "#include <stdio.h>", '#include "vqlinear.h"', "int main(void) {"]
     for st, fs in fields.items():
         src.append(f'  printf("{st} sizeof %zu\\n", sizeof({st}));')

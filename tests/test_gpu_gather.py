@@ -12,7 +12,8 @@ import pytest
 import torch
 
 import compressed_index_matmul_b200 as vq
-from synth import CONFIGS, DT_BF16, DT_F16, FMT_RVQ12_4, FMT_VQ16, LayerSpec, make_layer, make_signs, make_x
+from synth import (CONFIGS, DT_BF16, DT_F16, FMT_RVQ12_4, FMT_VQ16, FMT_VQ16_RVQ, LayerSpec, make_layer, make_signs,
+                   make_x)
 from tests.gpu_util import assert_y_within, dev, host_bits, layer_on_gpu, require_gpu, run_forward, widen
 
 pytestmark = pytest.mark.gpu
@@ -152,10 +153,10 @@ def test_rotated_fused_matches_oracle(oracle, shape):
     assert np.array_equal(y1, y2), "not bit-identical run to run"
 
 
-@pytest.mark.parametrize("M", [1, 8])
+@pytest.mark.parametrize("M", [1, 4, 8])
 def test_rotated_config3(oracle, M):
-    """Config 3: M = 1 runs the fused kernel, M = 8 the rotation into the handle's
-    buffer followed by the forward (the handle is created with rht = 1)."""
+    """Config 3: M <= 4 runs the fused kernel, M = 8 the rotation into the handle's
+    buffer followed by the tensor-core forward (the handle is created with rht = 1)."""
     spec = CONFIGS[3]["tensors"][0][1]
     layer = make_layer(spec, cfg_id=3)
     L = vq.VQLinear(spec.N, spec.K, spec.fmt, spec.scale_group, DT_F16, 8, layer, rht=1)
@@ -165,7 +166,7 @@ def test_rotated_config3(oracle, M):
     torch.cuda.synchronize()
     vq.vq_linear_check(L.handle)
     rows = np.sort(np.random.default_rng(M).choice(spec.N, size=512, replace=False))
-    if M == 1:
+    if M <= 4:
         y_ref, tol = _rotated_reference(oracle, layer, x, DT_F16, signs, rows)
     else:
         x_rot = oracle.round_to(oracle.rht(x, DT_F16, signs), DT_F16)
@@ -175,14 +176,45 @@ def test_rotated_config3(oracle, M):
     assert_y_within(y[:, rows], DT_F16, y_ref, tol, what=f"cfg3 rotated M={M}")
 
 
+@pytest.mark.parametrize("N, K, sg, act, M, bpw", [
+    (256, 256, 256, DT_F16, 2, 0), (520, 2048, 64, DT_BF16, 3, 0), (128, 1024, 64, DT_F16, 4, 0),
+    (256, 2688, 64, DT_BF16, 5, 0),      # block-diagonal rotation, 2048 + 512 + 128
+    (384, 4096, 4096, DT_F16, 8, 0),     # M' K = 32768, the largest x the kernel holds
+    (256, 1024, 1024, DT_F16, 3, 3),     # the residual ladder (16 + 8 bits)
+], ids=lambda v: str(v))
+def test_rotated_fused_several_tokens(oracle, N, K, sg, act, M, bpw):
+    """1 < M <= 8 on the gather kernel (forced beyond M = 4): one kernel rotates every
+    token in fp32 (the handle has no rotation buffer, so the unfused route would be
+    refused) and matches the oracle's unrounded rotation."""
+    spec = LayerSpec(N, K, FMT_VQ16_RVQ, sg, bpw=bpw) if bpw else LayerSpec(N, K, FMT_VQ16, sg)
+    layer = make_layer(spec, cfg_id=77, tensor_id=N + M)
+    L = layer_on_gpu(layer, act, M)
+    L.set_path(vq.VQ_PATH_GATHER)
+    x = make_x(M, K, act, cfg_id=77, seed=M)
+    signs = make_signs(K, cfg_id=77)
+    xt, st = dev(x).view(_tdt(act)), dev(signs)
+    y1 = host_bits(L.forward_rotated(xt, st))
+    y2 = host_bits(L.forward_rotated(xt, st))
+    torch.cuda.synchronize()
+    vq.vq_linear_check(L.handle)
+    y_ref, tol = _rotated_reference(oracle, layer, x, act, signs, None)
+    assert_y_within(y1, act, y_ref, tol, what=f"fused rotation M={M}")
+    assert np.array_equal(y1, y2), "not bit-identical run to run"
+
+
 def test_rotated_argument_errors():
     layer = make_layer(LayerSpec(256, 256, FMT_VQ16, 256), cfg_id=75)
     L = layer_on_gpu(layer, DT_F16, 8)  # rht = 0: no rotation buffer
     signs = dev(make_signs(256, cfg_id=75))
     x8 = torch.zeros((8, 256), dtype=torch.float16, device="cuda")
-    with pytest.raises(vq.VQError) as ei:  # M = 8 is not fused and the handle has no buffer
+    with pytest.raises(vq.VQError) as ei:  # M = 8 is not fused by default and the handle has no buffer
         L.forward_rotated(x8, signs)
     assert ei.value.status == vq._binding.VQ_ERR_INVALID_ARG
+    L.set_path(vq.VQ_PATH_TC)
+    with pytest.raises(vq.VQError) as ei:  # a forced path other than the gather kernel is not fused
+        L.forward_rotated(x8[:1], signs)
+    assert ei.value.status == vq._binding.VQ_ERR_INVALID_ARG
+    L.set_path(vq.VQ_PATH_AUTO)
     y = torch.empty((1, 256), dtype=torch.float16, device="cuda")
     with pytest.raises(vq.VQError) as ei:
         vq.vq_linear_forward_rotated(L.handle, x8[:1], None, L.planes, L.codebooks, L.t["scales"], y, 1, 256, 256)
@@ -199,11 +231,13 @@ def test_rotated_argument_errors():
 
 
 def test_rotated_block_diagonal_unfused(oracle):
-    """K = 2688 = 2048 + 512 + 128 at M = 8: the rotation kernel into the handle's buffer,
-    then the forward, against the oracle's block-diagonal rotation rounded the same way."""
+    """K = 2688 = 2048 + 512 + 128 at M = 8 on the tensor-core path (forced): the rotation
+    kernel into the handle's buffer, then the forward, against the oracle's
+    block-diagonal rotation rounded the same way."""
     N, K, M = 384, 2688, 8
     layer = make_layer(LayerSpec(N, K, FMT_VQ16, 64), cfg_id=76)
     L = vq.VQLinear(N, K, FMT_VQ16, 64, DT_BF16, M, layer, rht=1)
+    L.set_path(vq.VQ_PATH_TC)
     x = make_x(M, K, DT_BF16, cfg_id=76)
     signs = make_signs(K, cfg_id=76)
     y = host_bits(L.forward_rotated(dev(x).view(torch.bfloat16), dev(signs)))

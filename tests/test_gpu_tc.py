@@ -2,6 +2,7 @@
 
 import numpy as np
 import pytest
+import torch
 
 import compressed_index_matmul_b200 as vq
 from synth import DT_BF16, DT_F16, FMT_RVQ12, FMT_RVQ12_4, FMT_VQ16, CONFIGS, LayerSpec, make_layer, make_x
@@ -82,6 +83,68 @@ def test_single_split_many_slices(oracle):
     assert_y_within(y[:, rows], DT_F16, y_ref, oracle.tolerance(x, DT_F16, w, TOL), what="tc single split")
 
 
+# Layer-sized cases, checked element by element (or on sampled rows): up to eight
+# K splits with the last-CTA reduction, ragged rows and tokens, both index widths.
+LARGE_CASES = [
+    # (N, K, fmt, scale_group, act, M, rows sampled or None)
+    (2048, 4096, FMT_RVQ12_4, 64, DT_BF16, 16, None),    # 16 row tiles x 8 K splits
+    (2040, 4096, FMT_RVQ12_4, 64, DT_F16, 20, None),     # N % 8 != 0 (indices from global), ragged tokens
+    (2048, 4096, FMT_RVQ12, 4096, DT_BF16, 16, None),    # one stage, one scale per row
+    (1024, 8192, FMT_VQ16, 8192, DT_F16, 48, None),      # 16-bit indices, 8 splits of 8 slices
+    (5120, 512, FMT_RVQ12_4, 64, DT_BF16, 1024, 160),    # 160 tiles in two waves, one split
+    (8192, 1024, FMT_RVQ12_4, 64, DT_BF16, 300, 160),    # two token tiles, the second ragged
+]
+
+
+@pytest.mark.parametrize("case", LARGE_CASES, ids=lambda c: f"{c[0]}x{c[1]}f{c[2]}a{c[4]}M{c[5]}")
+def test_tc_layer_sized_match_oracle(oracle, case):
+    N, K, fmt, sg, act, M, nrows = case
+    layer = make_layer(LayerSpec(N, K, fmt, sg), cfg_id=84, tensor_id=N + M)
+    L = layer_on_gpu(layer, act, M)
+    L.set_path(vq.VQ_PATH_TC)
+    plan = L.plan(M)
+    assert plan["path"] == vq.VQ_PATH_TC and plan["launches"] == 1 and plan["ctas"] >= 1, plan
+    x = make_x(M, K, act, cfg_id=84, seed=M)
+    y = run_forward(L, x, act, vq.VQ_PATH_TC)
+    vq.vq_linear_check(L.handle)
+    y2 = run_forward(L, x, act, vq.VQ_PATH_TC)
+    assert np.array_equal(y, y2), "not bit-identical run to run"
+    rows = None if nrows is None else np.sort(np.random.default_rng(N).choice(N, size=nrows, replace=False))
+    y_ref = oracle.forward(layer, x, act, rows=rows)
+    w, _ = oracle.dequant(layer, rows=rows)
+    got = y if rows is None else y[:, rows]
+    assert_y_within(got, act, y_ref, oracle.tolerance(x, act, w, TOL), what=f"layer-sized M={M}")
+
+
+def test_plan_reports_the_kernel():
+    """vq_linear_plan: the kernel family, launches, CTAs and K splits of a forward."""
+    handles = []
+
+    def plan_of(spec, M, max_M=1024, corr=0):
+        h = vq.vq_linear_create(spec.N, spec.K, spec.fmt, spec.scale_group, DT_BF16, max_M, corr=corr)
+        handles.append(h)
+        return vq.vq_linear_plan(h, M)
+
+    try:
+        gate = CONFIGS[4]["tensors"][0][1]
+        p1 = plan_of(gate, 1)
+        assert p1["path"] == vq.VQ_PATH_LUT and p1["launches"] == 1 and p1["splits"] == gate.K // 128
+        assert p1["ctas"] == torch.cuda.get_device_properties(0).multi_processor_count
+        p16 = plan_of(gate, 16)
+        assert p16["path"] == vq.VQ_PATH_TC and p16["launches"] == 1
+        assert p16["ctas"] == (gate.N // 128) * p16["splits"]
+        assert plan_of(gate, 16, corr=1)["launches"] == 2  # the correction's kernel first
+        ps = plan_of(LayerSpec(256, 512, FMT_RVQ12_4, 64), 64)
+        assert ps["path"] == vq.VQ_PATH_TC and ps["ctas"] == 2 * ps["splits"]
+        pg = plan_of(LayerSpec(256, 512, FMT_RVQ12_4, 64), 4)
+        assert pg["path"] == vq.VQ_PATH_GEMV
+        with pytest.raises(vq.VQError):
+            vq.vq_linear_plan(handles[0], 0)
+    finally:
+        for h in handles:
+            vq.vq_linear_destroy(h)
+
+
 ONE_HOT_CASES = [
     (200, 576, FMT_RVQ12_4, 64, DT_F16),    # staged slices, 64-wide last slice
     (200, 576, FMT_RVQ12_4, 64, DT_BF16),
@@ -90,6 +153,7 @@ ONE_HOT_CASES = [
     (136, 1024, FMT_VQ16, 64, DT_BF16),
     (8192, 256, FMT_RVQ12_4, 64, DT_BF16),  # 64 row tiles: K-split pair over a 2-CTA cluster
     (9600, 256, FMT_RVQ12, 256, DT_F16),    # 75 row tiles: one split, TMA-stored y
+    (2048, 4096, FMT_RVQ12_4, 64, DT_BF16), # 8 K splits: the last CTA of a tile adds the partial sums
 ]
 
 
