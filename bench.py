@@ -245,11 +245,13 @@ class Workload:
                 x = y
         return calls
 
-    def _forward(self, L, inp, y):
+    def _forward(self, L, inp, y, stream):
+        """One forward on `stream` (a raw cudaStream_t: the caller looks the stream up once
+        per step instead of once per call)."""
         if self.rht:  # the layer rotates its input (vq_linear_forward_rotated)
-            L.forward_rotated(inp, self.signs, y)
+            L.forward_rotated(inp, self.signs, y, stream)
         else:
-            L.forward(inp, y)
+            L.forward(inp, y, stream)
 
     def _pair(self, a, b):
         return (self.concurrent_gate_up and self.role[id(a[0])] == "gate" and self.role[id(b[0])] == "up"
@@ -262,6 +264,7 @@ class Workload:
         import torch
 
         cur = torch.cuda.current_stream()
+        cur_s = cur.cuda_stream
         i = 0
         while i < len(calls):
             if concurrent and events is None and i + 1 < len(calls) and self._pair(calls[i], calls[i + 1]):
@@ -270,9 +273,8 @@ class Workload:
                 g.set_sm_budget(half)
                 u.set_sm_budget(self.sms - half)
                 self.side.wait_stream(cur)
-                with torch.cuda.stream(self.side):
-                    self._forward(u, ui, uy)
-                self._forward(g, gi, gy)
+                self._forward(u, ui, uy, self.side.cuda_stream)
+                self._forward(g, gi, gy, cur_s)
                 cur.wait_stream(self.side)
                 g.set_sm_budget(0)
                 u.set_sm_budget(0)
@@ -280,7 +282,7 @@ class Workload:
                 continue
             if events is not None:
                 events[i].record()
-            self._forward(*calls[i])
+            self._forward(*calls[i], cur_s)
             i += 1
         if events is not None:
             events[len(calls)].record()
