@@ -579,7 +579,12 @@ VQ_API vq_status vq_linear_check(vq_linear_t h, void* stream) {
   e = cudaMemcpy(&flag, h->err, sizeof flag, cudaMemcpyDeviceToHost);
   if (e != cudaSuccess) return cuda_fail(e, "reading the error word");
   if (flag) {
-    cudaMemset(h->err, 0, sizeof(uint32_t));
+    // A forward that gave up may have left completion counters or the table
+    // kernel's arrival counter part-way: clear them with the flag (one
+    // allocation), so the handle is usable again.
+    e = cudaMemset(h->err, 0, sizeof(uint32_t) * (2 + (size_t)h->num_tickets + (size_t)h->num_sync));
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the error word and the counters");
     return fail(VQ_ERR_TIMEOUT, "a bounded device wait gave up (flag 0x%x)", flag);
   }
   return VQ_OK;
