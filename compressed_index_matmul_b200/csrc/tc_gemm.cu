@@ -48,7 +48,7 @@ namespace vq {
 constexpr int kTcRows = 128;
 constexpr int kTcStages = 4;        // x tiles in shared memory and A tiles in TMEM
 // Decode warps per TMEM lane quarter (kParts, a template parameter): 3 for token
-// tiles of 64 and more, 4 for smaller ones (see the launch).
+// tiles of 64 and more, 2 for tiles of 16 to 48 (two CTAs per SM), see the launch.
 __host__ __device__ constexpr int tc_threads(int parts) { return 64 + 32 * 4 * parts; }
 constexpr int kTcMaxT = 256;
 constexpr uint32_t kTcACols = 32;   // TMEM columns of one A stage (64 k of 16-bit pairs)
@@ -122,7 +122,7 @@ __device__ __forceinline__ void decode_two_stage(const uint4& c1, const uint32_t
 }
 
 template <int FMT, typename T, bool kStaged, int kTcParts>
-__global__ void __launch_bounds__(tc_threads(kTcParts), 1)
+__global__ void __launch_bounds__(tc_threads(kTcParts), kTcParts == 2 ? 2 : 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap ymap, TcArgs p) {
   extern __shared__ unsigned char smem_raw[];
   constexpr bool k16 = (FMT == kFmtVq16 || FMT == kFmtVq16Rvq);
@@ -560,7 +560,9 @@ static TcGeom tc_geom(int M, int N, int K, int num_sms) {
   g.RT = (N + kTcRows - 1) / kTcRows;
   const int tiles = g.RT * g.TT;
   const int nsl = (K + 127) / 128;  // splits start on 128-input slice boundaries
-  int S = num_sms / tiles;
+  // Token tiles of 48 and less run two CTAs per SM (2 decode warps per lane quarter).
+  const int slots = g.T <= 48 ? 2 * num_sms : num_sms;
+  int S = slots / tiles;
   if (S < 1) S = 1;
   if (S > 8) S = 8;
   if (S > nsl) S = nsl;
@@ -615,6 +617,10 @@ static cudaError_t launch_tc_t(const LayerArgs& a, const TcGeom& g, float* scrat
   auto kern = tc_gemm_kernel<FMT, T, kStaged, kParts>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
+  if (kParts == 2) {  // two CTAs per SM: the whole carve-out as shared memory
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    if (e != cudaSuccess) return e;
+  }
   const bool partials = g.S > 1 && g.epi == kEpiGlobal;
   TcArgs p{a, g.epi, g.T, g.kps, g.S, partials ? scratch : nullptr, partials ? tickets : nullptr, err};
   cudaLaunchConfig_t cfg = {};
@@ -641,16 +647,17 @@ static cudaError_t launch_tc_s(const LayerArgs& a, const TcGeom& g, float* scrat
                                uint32_t* err, cudaStream_t s) {
   // Bulk copies need 16-byte sizes: N % 8 == 0 makes every per-slice run one.
   // Token tiles of 64 and more: 3 decode warps per quarter (14 warps, 128 registers
-  // each, no spills: the decode keeps up with the longer MMAs of a wide tile);
-  // narrower tiles: 4 (18 warps, 96 registers), more warps to hide the decode's
-  // latency when each block's MMA is short.  Measured on B200 (8192 x 8192 M = 256:
-  // 39.5 vs 43.1 us; Llama-3-8B gate M = 16 and the residual ladder at M = 8 are
-  // 3-18 % faster with 4).
+  // each, no spills: the decode keeps up with the longer MMAs of a wide tile;
+  // 8192 x 8192 M = 256: 39.5 vs 43.1 us with 4).  Narrower tiles: 2 per quarter
+  // (10 warps, 96 registers) and two CTAs per SM, each with its own decode -> MMA
+  // pipeline; tc_geom counts two slots per SM, so the Llama-3-8B gate at M = 16
+  // splits K over a cluster pair and fills every SM (27.4 vs 31.3 us with one
+  // CTA of 4 decode warps per quarter per SM; down 31.2 vs 32.5).
   if (g.T >= 64)
     return (a.N % 8 == 0) ? launch_tc_t<FMT, T, true, 3>(a, g, scratch, tickets, err, s)
                           : launch_tc_t<FMT, T, false, 3>(a, g, scratch, tickets, err, s);
-  return (a.N % 8 == 0) ? launch_tc_t<FMT, T, true, 4>(a, g, scratch, tickets, err, s)
-                        : launch_tc_t<FMT, T, false, 4>(a, g, scratch, tickets, err, s);
+  return (a.N % 8 == 0) ? launch_tc_t<FMT, T, true, 2>(a, g, scratch, tickets, err, s)
+                        : launch_tc_t<FMT, T, false, 2>(a, g, scratch, tickets, err, s);
 }
 
 cudaError_t launch_tc(const LayerArgs& a, const Plan& pl, float* scratch, uint32_t* tickets, uint32_t* err,
@@ -672,8 +679,8 @@ cudaError_t launch_tc(const LayerArgs& a, const Plan& pl, float* scratch, uint32
       if (g.T >= 64)
         return bf ? launch_tc_t<kFmtVq16Rvq, __nv_bfloat16, false, 3>(a, g, scratch, tickets, err, s)
                   : launch_tc_t<kFmtVq16Rvq, __half, false, 3>(a, g, scratch, tickets, err, s);
-      return bf ? launch_tc_t<kFmtVq16Rvq, __nv_bfloat16, false, 4>(a, g, scratch, tickets, err, s)
-                : launch_tc_t<kFmtVq16Rvq, __half, false, 4>(a, g, scratch, tickets, err, s);
+      return bf ? launch_tc_t<kFmtVq16Rvq, __nv_bfloat16, false, 2>(a, g, scratch, tickets, err, s)
+                : launch_tc_t<kFmtVq16Rvq, __half, false, 2>(a, g, scratch, tickets, err, s);
     default:
       return bf ? launch_tc_s<kFmtVq16, __nv_bfloat16>(a, g, scratch, tickets, err, s)
                 : launch_tc_s<kFmtVq16, __half>(a, g, scratch, tickets, err, s);
