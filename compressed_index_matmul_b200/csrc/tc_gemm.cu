@@ -48,7 +48,9 @@ namespace vq {
 constexpr int kTcRows = 128;
 constexpr int kTcStages = 4;        // x tiles in shared memory and A tiles in TMEM
 // Decode warps per TMEM lane quarter (kParts, a template parameter): 3 for token
-// tiles of 64 and more, 2 for tiles of 16 to 48 (two CTAs per SM), see the launch.
+// tiles of 64 and more; for tiles of 16 to 48, 2 with two CTAs per SM (12-bit
+// formats) or 4 with one (16-bit formats, whose codeword gathers need the L1
+// cache that a second CTA's shared memory would take); see the launch.
 __host__ __device__ constexpr int tc_threads(int parts) { return 64 + 32 * 4 * parts; }
 constexpr int kTcMaxT = 256;
 constexpr uint32_t kTcACols = 32;   // TMEM columns of one A stage (64 k of 16-bit pairs)
@@ -550,18 +552,20 @@ static EncodeTiledFn encode_fn() {
 
 struct TcGeom {
   int T, TT, RT, S, kps, epi;
+  bool dual;  // two CTAs per SM (2 decode warps per lane quarter)
 };
 
-static TcGeom tc_geom(int M, int N, int K, int num_sms) {
+// fmt: kFmt*.
+static TcGeom tc_geom(int fmt, int M, int N, int K, int num_sms) {
   TcGeom g;
   const int m16 = (M + 15) / 16 * 16;
   g.T = m16 < kTcMaxT ? m16 : kTcMaxT;
   g.TT = (M + g.T - 1) / g.T;
+  g.dual = g.T <= 48 && fmt != kFmtVq16 && fmt != kFmtVq16Rvq;
   g.RT = (N + kTcRows - 1) / kTcRows;
   const int tiles = g.RT * g.TT;
   const int nsl = (K + 127) / 128;  // splits start on 128-input slice boundaries
-  // Token tiles of 48 and less run two CTAs per SM (2 decode warps per lane quarter).
-  const int slots = g.T <= 48 ? 2 * num_sms : num_sms;
+  const int slots = g.dual ? 2 * num_sms : num_sms;
   int S = slots / tiles;
   if (S < 1) S = 1;
   if (S > 8) S = 8;
@@ -576,7 +580,7 @@ static TcGeom tc_geom(int M, int N, int K, int num_sms) {
 
 bool plan_tc(const vq_linear_desc& d, const DeviceInfo& dev, int M, Plan* p) {
   if (M < 1 || dev.smem_optin < (int)kTcSmemMax) return false;
-  const TcGeom g = tc_geom(M, d.N, d.K, dev.num_sms);
+  const TcGeom g = tc_geom(d.fmt, M, d.N, d.K, dev.num_sms);
   p->path = VQ_PATH_TC;
   p->splits = g.S;
   p->k_per_split = g.kps;
@@ -652,12 +656,20 @@ static cudaError_t launch_tc_s(const LayerArgs& a, const TcGeom& g, float* scrat
   // (10 warps, 96 registers) and two CTAs per SM, each with its own decode -> MMA
   // pipeline; tc_geom counts two slots per SM, so the Llama-3-8B gate at M = 16
   // splits K over a cluster pair and fills every SM (27.4 vs 31.3 us with one
-  // CTA of 4 decode warps per quarter per SM; down 31.2 vs 32.5).
+  // CTA of 4 decode warps per quarter per SM; down 31.2 vs 32.5).  The 16-bit
+  // formats keep one CTA of 4 per quarter (18 warps, 96 registers): two CTAs'
+  // shared memory leaves too little L1 for their codeword gathers from the
+  // 1 MiB codebook (4096 x 4096 M = 8: 29.2 vs 18 us).
   if (g.T >= 64)
     return (a.N % 8 == 0) ? launch_tc_t<FMT, T, true, 3>(a, g, scratch, tickets, err, s)
                           : launch_tc_t<FMT, T, false, 3>(a, g, scratch, tickets, err, s);
-  return (a.N % 8 == 0) ? launch_tc_t<FMT, T, true, 2>(a, g, scratch, tickets, err, s)
-                        : launch_tc_t<FMT, T, false, 2>(a, g, scratch, tickets, err, s);
+  if constexpr (FMT != kFmtVq16) {
+    if (g.dual)
+      return (a.N % 8 == 0) ? launch_tc_t<FMT, T, true, 2>(a, g, scratch, tickets, err, s)
+                            : launch_tc_t<FMT, T, false, 2>(a, g, scratch, tickets, err, s);
+  }
+  return (a.N % 8 == 0) ? launch_tc_t<FMT, T, true, 4>(a, g, scratch, tickets, err, s)
+                        : launch_tc_t<FMT, T, false, 4>(a, g, scratch, tickets, err, s);
 }
 
 cudaError_t launch_tc(const LayerArgs& a, const Plan& pl, float* scratch, uint32_t* tickets, uint32_t* err,
@@ -665,7 +677,7 @@ cudaError_t launch_tc(const LayerArgs& a, const Plan& pl, float* scratch, uint32
   int dev = 0, sms = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const TcGeom g = tc_geom(a.M, a.N, a.K, sms);
+  const TcGeom g = tc_geom(a.fmt, a.M, a.N, a.K, sms);
   if (g.S != pl.splits) return cudaErrorInvalidValue;
   const bool bf = a.act == VQ_BF16;
   switch (a.fmt) {
@@ -679,8 +691,8 @@ cudaError_t launch_tc(const LayerArgs& a, const Plan& pl, float* scratch, uint32
       if (g.T >= 64)
         return bf ? launch_tc_t<kFmtVq16Rvq, __nv_bfloat16, false, 3>(a, g, scratch, tickets, err, s)
                   : launch_tc_t<kFmtVq16Rvq, __half, false, 3>(a, g, scratch, tickets, err, s);
-      return bf ? launch_tc_t<kFmtVq16Rvq, __nv_bfloat16, false, 2>(a, g, scratch, tickets, err, s)
-                : launch_tc_t<kFmtVq16Rvq, __half, false, 2>(a, g, scratch, tickets, err, s);
+      return bf ? launch_tc_t<kFmtVq16Rvq, __nv_bfloat16, false, 4>(a, g, scratch, tickets, err, s)
+                : launch_tc_t<kFmtVq16Rvq, __half, false, 4>(a, g, scratch, tickets, err, s);
     default:
       return bf ? launch_tc_s<kFmtVq16, __nv_bfloat16>(a, g, scratch, tickets, err, s)
                 : launch_tc_s<kFmtVq16, __half>(a, g, scratch, tickets, err, s);
