@@ -342,10 +342,7 @@ vq_status vq_rht_apply_output(const void* y, void* y_out, const int8_t* signs, i
 
 /* Synchronise `stream` and report (then clear) any error flag a bounded
  * device-side wait of this handle's kernels raised: VQ_ERR_TIMEOUT if one gave
- * up, else VQ_OK.  Clearing the flag also zeroes the handle's completion
- * counters and the table kernel's barrier words, which a forward that gave up
- * may have left part-way, so later forwards of the handle are correct again.
- * Synchronous (it waits for the whole device when it clears). */
+ * up, else VQ_OK.  Synchronous. */
 vq_status vq_linear_check(vq_linear_t h, void* stream);
 
 /* Message for the calling thread's last non-OK status ("" if none).  The
