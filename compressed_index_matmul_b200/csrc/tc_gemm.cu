@@ -10,17 +10,21 @@
 //              per 128-input slice, bulk-copies the tile's index bytes (the
 //              K-slice-major planes make them one contiguous run per plane) into
 //              a 4-slot ring; per 64-wide k block, TMA-loads the x tile (T tokens
-//              x 64, 128-byte swizzle) into a 4-stage ring.
+//              x 64, 128-byte swizzle) into a ring of S stages (S = 4; 3 when two
+//              64-token CTAs share an SM).
 //   warp 1     allocates TMEM; lane 0 issues tcgen05.mma (M=128, N=T, K=16, four
 //              per k block, A read from TMEM) and commits each stage back.
 //   warps 2.. decode: P warps per TMEM lane quarter (P = 3 for token tiles of 64
-//              and more, 4 for narrower ones); thread = one row of the tile (its
-//              TMEM lane); warp `part` of a quarter decodes every P-th k block
-//              (kb % P == part), all 8 groups of it, into A stage kb % 4.  With P = 3
-//              the CTA has 14 warps, at most four share an SM sub-partition and each
-//              thread may hold 128 registers (no spills); with P = 4, 18 warps and
-//              96 registers (the decode loop spills a little, but more warps hide
-//              its latency when each block's MMA is short).  Per block a thread reads its 8
+//              and more; 2 with two CTAs per SM for the 12-bit formats' tiles of
+//              16 to 64; 4 for the 16-bit formats' narrower tiles); thread = one
+//              row of the tile (its TMEM lane); warp `part` of a quarter decodes
+//              every P-th k block (kb % P == part), all 8 groups of it, into A
+//              stage kb % S.  With P = 3 the CTA has 14 warps, at most four share
+//              an SM sub-partition and each thread may hold 128 registers (no
+//              spills); with P = 2, 10 warps and 96 registers, two CTAs per SM;
+//              with P = 4, 18 warps and 96 registers (the decode loop spills a
+//              little, but more warps hide its latency when each block's MMA is
+//              short).  Per block a thread reads its 8
 //              index bytes (plus nibbles and scale) from the staged slice, gathers
 //              the stage-1 codewords from shared memory and the stage-2 codewords
 //              from the warp's registers (shuffle), decodes with the
@@ -46,7 +50,7 @@
 namespace vq {
 
 constexpr int kTcRows = 128;
-constexpr int kTcStages = 4;        // x tiles in shared memory and A tiles in TMEM
+constexpr int kTcStages = 4;        // x tiles in shared memory and A tiles in TMEM (3 for two 64-token CTAs per SM)
 // Decode warps per TMEM lane quarter (kParts, a template parameter): 3 for token
 // tiles of 64 and more; for tiles of 16 to 48, 2 with two CTAs per SM (12-bit
 // formats) or 4 with one (16-bit formats, whose codeword gathers need the L1
@@ -123,7 +127,7 @@ __device__ __forceinline__ void decode_two_stage(const uint4& c1, const uint32_t
   }
 }
 
-template <int FMT, typename T, bool kStaged, int kTcParts>
+template <int FMT, typename T, bool kStaged, int kTcParts, int kSt>
 __global__ void __launch_bounds__(tc_threads(kTcParts), kTcParts == 2 ? 2 : 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap ymap, TcArgs p) {
   extern __shared__ unsigned char smem_raw[];
@@ -132,6 +136,7 @@ __global__ void __launch_bounds__(tc_threads(kTcParts), kTcParts == 2 ? 2 : 1)
   constexpr bool kSmemCb = !k16;
   constexpr bool kTwo = (FMT == kFmtRvq12_4);
   static_assert(!(kLadder && kStaged), "the residual ladder reads its indices directly");
+  static_assert(kSt >= kTcParts && kSt <= kTcStages, "a stage barrier may be at most one phase behind");
   const LayerArgs& a = p.a;
   // 1024-byte aligned base (the swizzle pattern of the x tiles is taken from address bits).
   const uint32_t raw = smem_u32(smem_raw);
@@ -140,13 +145,13 @@ __global__ void __launch_bounds__(tc_threads(kTcParts), kTcParts == 2 ? 2 : 1)
   const uint4* cb1s = reinterpret_cast<const uint4*>(sm);
   const uint32_t bar0 = base + kTcOffBars;
   auto full_a = [&](int s) { return bar0 + 8u * s; };
-  auto full_b = [&](int s) { return bar0 + 8u * (kTcStages + s); };
-  auto empty = [&](int s) { return bar0 + 8u * (2 * kTcStages + s); };
-  const uint32_t accum_bar = bar0 + 8u * (3 * kTcStages);
+  auto full_b = [&](int s) { return bar0 + 8u * (kSt + s); };
+  auto empty = [&](int s) { return bar0 + 8u * (2 * kSt + s); };
+  const uint32_t accum_bar = bar0 + 8u * (3 * kSt);
   const uint32_t cb_bar = accum_bar + 8u;
   auto idx_full = [&](int s) { return cb_bar + 8u + 8u * s; };
   auto idx_empty = [&](int s) { return cb_bar + 8u + 8u * kTcIdxSlots + 8u * s; };
-  static_assert(8 * (3 * kTcStages + 2 + 2 * kTcIdxSlots) <= 192, "barriers overlap the flags");
+  static_assert(8 * (3 * kSt + 2 + 2 * kTcIdxSlots) <= 192, "barriers overlap the flags");
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kTcOffBars + 192);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + kTcOffBars + 196);
   volatile int* last_flag = reinterpret_cast<volatile int*>(sm + kTcOffBars + 200);
@@ -164,13 +169,13 @@ __global__ void __launch_bounds__(tc_threads(kTcParts), kTcParts == 2 ? 2 : 1)
   const int nsl = (nkb + 1) / 2;  // 128-input slices of this split (the last may be 64 wide)
   const int s_first = kbeg / 128;
   const bool block_scales = (a.scale_group == 64);
-  // TMEM: the accumulator in columns [0, T), then kTcStages A stages of 32 columns.
+  // TMEM: the accumulator in columns [0, T), then kSt A stages of 32 columns.
   const uint32_t acol0 = ((uint32_t)p.T + 31u) & ~31u;
-  const uint32_t tneed = acol0 + kTcStages * kTcACols;
+  const uint32_t tneed = acol0 + kSt * kTcACols;
   const uint32_t tcols = tneed <= 32 ? 32u : (tneed <= 64 ? 64u : (tneed <= 128 ? 128u : (tneed <= 256 ? 256u : 512u)));
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kTcStages; ++s) {
+    for (int s = 0; s < kSt; ++s) {
       ptx::mbar_init(full_a(s), 4);  // one decode warp per TMEM lane quarter
       ptx::mbar_init(full_b(s), 1);               // the producer's expect_tx arrival (+ bytes)
       ptx::mbar_init(empty(s), 1);                // one tcgen05.commit
@@ -224,8 +229,8 @@ __global__ void __launch_bounds__(tc_threads(kTcParts), kTcParts == 2 ? 2 : 1)
       if (kStaged)
         for (; issued_idx < kTcIdxSlots && issued_idx < nsl; ++issued_idx) issue_idx(issued_idx);
       for (int kb = 0; kb < nkb && !*abort_flag; ++kb) {
-        const int s = kb % kTcStages;
-        if (kb >= kTcStages && !ptx::mbar_wait(empty(s), ((kb / kTcStages) - 1) & 1, p.err)) {
+        const int s = kb % kSt;
+        if (kb >= kSt && !ptx::mbar_wait(empty(s), ((kb / kSt) - 1) & 1, p.err)) {
           *abort_flag = 1;
           break;
         }
@@ -235,8 +240,8 @@ __global__ void __launch_bounds__(tc_threads(kTcParts), kTcParts == 2 ? 2 : 1)
         // After x of block kb (odd, >= 5) is issued, refill with slice (kb+3)/2.
         // Its slot held slice (kb-5)/2, which the warps decoding blocks kb - 5 and
         // kb - 4 released before decoding them; the stage-empty wait above already
-        // saw MMA kb - 4 (and so every earlier block) complete, so this wait never
-        // holds back the x loads.
+        // saw MMA kb - kSt >= kb - 4 (and so every earlier block) complete, so this
+        // wait never holds back the x loads.
         if (kStaged && (kb & 1) == 1 && kb >= 5 && (kb + 3) / 2 == issued_idx && issued_idx < nsl) {
           const int j = issued_idx;
           if (!ptx::mbar_wait(idx_empty(j % kTcIdxSlots), ((j / kTcIdxSlots) - 1) & 1, p.err)) {
@@ -248,8 +253,8 @@ __global__ void __launch_bounds__(tc_threads(kTcParts), kTcParts == 2 ? 2 : 1)
         }
       }
       // Do not leave while a copy into this CTA's shared memory may be in flight.
-      for (int kb = (issued > kTcStages ? issued - kTcStages : 0); kb < issued; ++kb)
-        ptx::mbar_wait(full_b(kb % kTcStages), (kb / kTcStages) & 1, p.err);
+      for (int kb = (issued > kSt ? issued - kSt : 0); kb < issued; ++kb)
+        ptx::mbar_wait(full_b(kb % kSt), (kb / kSt) & 1, p.err);
       if (kStaged)
         for (int j = (issued_idx > kTcIdxSlots ? issued_idx - kTcIdxSlots : 0); j < issued_idx; ++j)
           ptx::mbar_wait(idx_full(j % kTcIdxSlots), (j / kTcIdxSlots) & 1, p.err);
@@ -263,8 +268,8 @@ __global__ void __launch_bounds__(tc_threads(kTcParts), kTcParts == 2 ? 2 : 1)
       bool ok = true;
       int issued = 0;
       for (int kb = 0; kb < nkb; ++kb) {
-        const int s = kb % kTcStages;
-        const uint32_t par = (kb / kTcStages) & 1;
+        const int s = kb % kSt;
+        const uint32_t par = (kb / kSt) & 1;
         if (*abort_flag || !ptx::mbar_wait(full_b(s), par, p.err) || !ptx::mbar_wait(full_a(s), par, p.err)) {
           *abort_flag = 1;
           ok = false;
@@ -287,7 +292,7 @@ __global__ void __launch_bounds__(tc_threads(kTcParts), kTcParts == 2 ? 2 : 1)
   } else {
     // ------------------------------------------------------------ decode
     // Warp (quarter q, part) decodes every P-th k block, kb = part, part+P, ...: all
-    // 8 groups of the block for its 32 rows, i.e. the whole A stage kb % 4
+    // 8 groups of the block for its 32 rows, i.e. the whole A stage kb % kSt
     // for its TMEM lane quarter.
     const int q = warp & 3;            // TMEM lane quarter of this warp
     const int part = (warp - 2) >> 2;  // 0..kTcParts-1: this warp decodes blocks kb == part (mod kTcParts)
@@ -310,12 +315,12 @@ __global__ void __launch_bounds__(tc_threads(kTcParts), kTcParts == 2 ? 2 : 1)
     for (int kb = part; ok && kb < nkb; kb += kTcParts) {
       const int j = kb >> 1, h = kb & 1;
       const int sl = s_first + j, w = slice_width(sl, G);
-      // A stage kb % kTcStages; the MMA of block kb - kTcStages must be done with it.
+      // A stage kb % kSt; the MMA of block kb - kSt must be done with it.
       // (This warp's previous block, kb - kTcParts, already needed the MMA of block
-      // kb - kTcParts - kTcStages, so the stage's barrier is at most one phase behind.)
-      const int st = kb % kTcStages;
+      // kb - kTcParts - kSt, so the stage's barrier is at most one phase behind.)
+      const int st = kb % kSt;
       const uint32_t tlane = tlane0 + kTcACols * (uint32_t)st;
-      if (*abort_flag || (kb >= kTcStages && !ptx::mbar_wait(empty(st), ((kb / kTcStages) - 1) & 1, p.err)) ||
+      if (*abort_flag || (kb >= kSt && !ptx::mbar_wait(empty(st), ((kb / kSt) - 1) & 1, p.err)) ||
           (kStaged && !ptx::mbar_wait(idx_full(j % kTcIdxSlots), (j / kTcIdxSlots) & 1, p.err))) {
         *abort_flag = 1;
         ok = false;
@@ -552,7 +557,7 @@ static EncodeTiledFn encode_fn() {
 
 struct TcGeom {
   int T, TT, RT, S, kps, epi;
-  bool dual;  // two CTAs per SM (2 decode warps per lane quarter)
+  bool dual;  // two CTAs per SM (2 decode warps per lane quarter; 3 stages for 64-token tiles)
 };
 
 // fmt: kFmt*.
@@ -561,15 +566,24 @@ static TcGeom tc_geom(int fmt, int M, int N, int K, int num_sms) {
   const int m16 = (M + 15) / 16 * 16;
   g.T = m16 < kTcMaxT ? m16 : kTcMaxT;
   g.TT = (M + g.T - 1) / g.T;
-  g.dual = g.T <= 48 && fmt != kFmtVq16 && fmt != kFmtVq16Rvq;
+  g.dual = g.T <= 64 && fmt != kFmtVq16 && fmt != kFmtVq16Rvq;
   g.RT = (N + kTcRows - 1) / kTcRows;
   const int tiles = g.RT * g.TT;
   const int nsl = (K + 127) / 128;  // splits start on 128-input slice boundaries
-  const int slots = g.dual ? 2 * num_sms : num_sms;
-  int S = slots / tiles;
-  if (S < 1) S = 1;
-  if (S > 8) S = 8;
-  if (S > nsl) S = nsl;
+  auto splits = [&](int slots) {
+    int S = slots / tiles;
+    if (S < 1) S = 1;
+    if (S > 8) S = 8;
+    return S > nsl ? nsl : S;
+  };
+  int S = splits(g.dual ? 2 * num_sms : num_sms);
+  // 64-token tiles: two CTAs per SM only while the K split stays a cluster pair
+  // (Llama-3-8B gate M = 64: 28.3 vs 32.7 us; 8192 x 8192 M = 64, where it would
+  // take four splits with partial sums in global memory: 36.6 vs 33.5 us).
+  if (g.dual && g.T == 64 && S > 2) {
+    g.dual = false;
+    S = splits(num_sms);
+  }
   const int sps = (nsl + S - 1) / S;
   g.S = (nsl + sps - 1) / sps;
   g.kps = sps * 128;
@@ -592,7 +606,7 @@ bool plan_tc(const vq_linear_desc& d, const DeviceInfo& dev, int M, Plan* p) {
   return true;
 }
 
-template <int FMT, typename T, bool kStaged, int kParts>
+template <int FMT, typename T, bool kStaged, int kParts, int kSt = kTcStages>
 static cudaError_t launch_tc_t(const LayerArgs& a, const TcGeom& g, float* scratch, uint32_t* tickets,
                                uint32_t* err, cudaStream_t s) {
   EncodeTiledFn enc = encode_fn();
@@ -617,8 +631,8 @@ static cudaError_t launch_tc_t(const LayerArgs& a, const TcGeom& g, float* scrat
             CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
   }
-  const uint32_t smem = kTcTilesOffset + kTcStages * ((uint32_t)g.T * 128u) + 1024u;
-  auto kern = tc_gemm_kernel<FMT, T, kStaged, kParts>;
+  const uint32_t smem = kTcTilesOffset + kSt * ((uint32_t)g.T * 128u) + 1024u;
+  auto kern = tc_gemm_kernel<FMT, T, kStaged, kParts, kSt>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   if (kParts == 2) {  // two CTAs per SM: the whole carve-out as shared memory
@@ -652,22 +666,28 @@ static cudaError_t launch_tc_s(const LayerArgs& a, const TcGeom& g, float* scrat
   // Bulk copies need 16-byte sizes: N % 8 == 0 makes every per-slice run one.
   // Token tiles of 64 and more: 3 decode warps per quarter (14 warps, 128 registers
   // each, no spills: the decode keeps up with the longer MMAs of a wide tile;
-  // 8192 x 8192 M = 256: 39.5 vs 43.1 us with 4).  Narrower tiles: 2 per quarter
-  // (10 warps, 96 registers) and two CTAs per SM, each with its own decode -> MMA
-  // pipeline; tc_geom counts two slots per SM, so the Llama-3-8B gate at M = 16
+  // 8192 x 8192 M = 256: 39.5 vs 43.1 us with 4).  The 12-bit formats' tiles of 16
+  // to 48 tokens, and of 64 when the split stays a cluster pair (tc_geom): 2 per
+  // quarter (10 warps, 96 registers) and two CTAs per SM, each with its own decode
+  // -> MMA pipeline (64-token tiles with three x stages, so that two fit in shared
+  // memory); tc_geom counts two slots per SM, so the Llama-3-8B gate at M = 16
   // splits K over a cluster pair and fills every SM (27.4 vs 31.3 us with one
-  // CTA of 4 decode warps per quarter per SM; down 31.2 vs 32.5).  The 16-bit
+  // CTA of 4 decode warps per quarter per SM; down 31.2 vs 32.5; the gate at
+  // M = 64 28.3 vs 32.7 with one CTA of 3).  The 16-bit
   // formats keep one CTA of 4 per quarter (18 warps, 96 registers): two CTAs'
   // shared memory leaves too little L1 for their codeword gathers from the
   // 1 MiB codebook (4096 x 4096 M = 8: 29.2 vs 18 us).
-  if (g.T >= 64)
-    return (a.N % 8 == 0) ? launch_tc_t<FMT, T, true, 3>(a, g, scratch, tickets, err, s)
-                          : launch_tc_t<FMT, T, false, 3>(a, g, scratch, tickets, err, s);
   if constexpr (FMT != kFmtVq16) {
+    if (g.dual && g.T == 64)  // two 64-token CTAs fit in shared memory with three x stages
+      return (a.N % 8 == 0) ? launch_tc_t<FMT, T, true, 2, 3>(a, g, scratch, tickets, err, s)
+                            : launch_tc_t<FMT, T, false, 2, 3>(a, g, scratch, tickets, err, s);
     if (g.dual)
       return (a.N % 8 == 0) ? launch_tc_t<FMT, T, true, 2>(a, g, scratch, tickets, err, s)
                             : launch_tc_t<FMT, T, false, 2>(a, g, scratch, tickets, err, s);
   }
+  if (g.T >= 64)
+    return (a.N % 8 == 0) ? launch_tc_t<FMT, T, true, 3>(a, g, scratch, tickets, err, s)
+                          : launch_tc_t<FMT, T, false, 3>(a, g, scratch, tickets, err, s);
   return (a.N % 8 == 0) ? launch_tc_t<FMT, T, true, 4>(a, g, scratch, tickets, err, s)
                         : launch_tc_t<FMT, T, false, 4>(a, g, scratch, tickets, err, s);
 }

@@ -93,6 +93,8 @@ LARGE_CASES = [
     (1024, 8192, FMT_VQ16, 8192, DT_F16, 48, None),      # 16-bit indices, 8 splits of 8 slices
     (5120, 512, FMT_RVQ12_4, 64, DT_BF16, 1024, 160),    # 160 tiles in two waves, one split
     (8192, 1024, FMT_RVQ12_4, 64, DT_BF16, 300, 160),    # two token tiles, the second ragged
+    (14336, 1024, FMT_RVQ12_4, 64, DT_BF16, 16, 160),    # two CTAs per SM, K-split cluster pairs
+    (14336, 1024, FMT_RVQ12_4, 64, DT_F16, 64, 160),     # the same with 64-token tiles (three x stages)
 ]
 
 
