@@ -41,6 +41,7 @@ from ._binding import (  # noqa: F401
     vq_linear_plan,
     vq_linear_set_path,
     vq_linear_set_sm_budget,
+    vq_plan_for_device,
     vq_rht_apply,
     vq_rht_apply_output,
     vq_rht_apply_output_sharded,

@@ -31,7 +31,7 @@ STATUS_NAMES = {0: "VQ_OK", 1: "VQ_ERR_INVALID_ARG", 2: "VQ_ERR_UNSUPPORTED", 3:
 # Every entry point the header declares (checked by the tests against the .so).
 EXPORTS = ("vq_abi_version", "vq_linear_create", "vq_linear_destroy", "vq_linear_set_path", "vq_linear_set_sm_budget",
            "vq_linear_forward",
-           "vq_linear_forward_noalloc", "vq_linear_forward_rotated", "vq_linear_launches", "vq_linear_plan", "vq_rht_apply", "vq_rht_apply_output", "vq_rht_apply_output_sharded", "vq_encode", "vq_linear_check", "vq_last_error",
+           "vq_linear_forward_noalloc", "vq_linear_forward_rotated", "vq_linear_launches", "vq_linear_plan", "vq_plan_for_device", "vq_rht_apply", "vq_rht_apply_output", "vq_rht_apply_output_sharded", "vq_encode", "vq_linear_check", "vq_last_error",
            "vq_debug_unpack", "vq_debug_dequant", "vq_debug_wait_timeout")
 
 
@@ -104,6 +104,9 @@ def load(path: str | None = None):
         lib.vq_linear_launches.argtypes = [P, I32]
         lib.vq_linear_plan.restype = st
         lib.vq_linear_plan.argtypes = [P, I32, ctypes.POINTER(vq_plan_info)]
+        lib.vq_plan_for_device.restype = st
+        lib.vq_plan_for_device.argtypes = [ctypes.POINTER(vq_linear_desc), I32, I32, I32, I32,
+                                           ctypes.POINTER(vq_plan_info)]
         lib.vq_linear_forward_rotated.restype = st
         lib.vq_linear_forward_rotated.argtypes = [P, P, P, ctypes.POINTER(vq_planes), ctypes.POINTER(vq_codebooks), P,
                                                   P, I32, I32, I32, P]
@@ -199,6 +202,19 @@ def vq_linear_plan(h, M: int) -> dict:
     """How vq_linear_forward runs this M: path, launches, ctas, splits."""
     info = vq_plan_info()
     _check(load().vq_linear_plan(h, M, ctypes.byref(info)))
+    return {name: getattr(info, name) for name, _ in vq_plan_info._fields_}
+
+
+B200_SMS, B200_SMEM_OPTIN = 148, 232448
+
+
+def vq_plan_for_device(N, K, fmt, scale_group, act_dtype, max_M, M, path=0, num_sms=B200_SMS,
+                       smem_optin=B200_SMEM_OPTIN, rht=0, n16=0, n8=0, mult=(), corr=0) -> dict:
+    """The plan of a forward of M tokens for such a layer on such a device (path 0 =
+    automatic choice), computed on the host without a handle or a GPU."""
+    d = make_desc(N, K, fmt, scale_group, act_dtype, max_M, rht, n16, n8, mult, corr)
+    info = vq_plan_info()
+    _check(load().vq_plan_for_device(ctypes.byref(d), M, path, num_sms, smem_optin, ctypes.byref(info)))
     return {name: getattr(info, name) for name, _ in vq_plan_info._fields_}
 
 

@@ -379,6 +379,30 @@ VQ_API vq_status vq_linear_plan(vq_linear_t h, int32_t M, vq_plan_info* out) {
   return VQ_OK;
 }
 
+VQ_API vq_status vq_plan_for_device(const vq_linear_desc* desc, int32_t M, int32_t path, int32_t num_sms,
+                                    int32_t smem_optin, vq_plan_info* out) {
+  vq_status st = validate_desc(desc);
+  if (st) return st;
+  if (out == nullptr) return fail(VQ_ERR_INVALID_ARG, "out is NULL");
+  if (M < 1 || M > desc->max_M) return fail(VQ_ERR_INVALID_ARG, "M=%d outside [1, max_M=%d]", M, desc->max_M);
+  if (num_sms < 1 || smem_optin < 0)
+    return fail(VQ_ERR_INVALID_ARG, "num_sms=%d and smem_optin=%d: need num_sms >= 1, smem_optin >= 0", num_sms,
+                smem_optin);
+  if (path < VQ_PATH_AUTO || path > VQ_PATH_GATHER) return fail(VQ_ERR_INVALID_ARG, "path=%d is not a VQ_PATH_*", path);
+  vq::DeviceInfo dev{};
+  dev.device = -1;
+  dev.num_sms = num_sms;
+  dev.smem_optin = smem_optin;
+  vq::Plan p{};
+  if (!vq::plan_forward(*desc, dev, M, path, &p))
+    return fail(VQ_ERR_UNSUPPORTED, "path %d cannot run M=%d for this layer on this device", path, M);
+  out->path = p.path;
+  out->launches = p.launches + (desc->corr ? 1 : 0);
+  out->ctas = p.ctas;
+  out->splits = p.splits;
+  return VQ_OK;
+}
+
 VQ_API vq_status vq_linear_forward(vq_linear_t h, const void* x, const vq_planes* planes,
                                    const vq_codebooks* codebooks, const void* scales, void* y, int32_t M,
                                    int32_t N, int32_t K, void* stream) {
