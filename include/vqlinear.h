@@ -308,19 +308,6 @@ typedef struct {
 } vq_plan_info;
 vq_status vq_linear_plan(vq_linear_t h, int32_t M, vq_plan_info* out);
 
-/* The plan vq_linear_plan would report for a handle created from `desc` and given
- * the kernel choice `path` (VQ_PATH_AUTO, or a path as vq_linear_set_path forces
- * it), on a device with `num_sms` SMs and `smem_optin` bytes of opt-in shared
- * memory per block (a B200: 148 and 232448), with no SM budget.  Host arithmetic
- * only: no handle, no device, no CUDA call, so it runs on any machine (capacity
- * planning; tests of the path and tiling policy).
- * VQ_ERR_INVALID_ARG for a NULL `desc` or `out`, an invalid `desc` (as
- * vq_linear_create checks it), M outside [1, desc->max_M], num_sms < 1,
- * smem_optin < 0 or `path` not a VQ_PATH_*; VQ_ERR_UNSUPPORTED when the path
- * cannot take this M on such a device. */
-vq_status vq_plan_for_device(const vq_linear_desc* desc, int32_t M, int32_t path, int32_t num_sms,
-                             int32_t smem_optin, vq_plan_info* out);
-
 /* Randomised Hadamard rotation of the input (GLQ README, "How it works",
  * Randomized Hadamard Transform): for every row m,
  *   x_out[m][k] = (1/sqrt K) * sum_j (-1)^popcount(k & j) * signs[j] * x[m][j],

@@ -1,6 +1,6 @@
 /*
  * vqlinear_tools.h -- entry points of libvqlinear beside the forward: the shard-batched
- * output rotation and the nearest-entry encoder.  The storage format, the element
+ * output rotation, the nearest-entry encoder and the host-side plan query.  The storage format, the element
  * types and the conventions shared by every entry point (status codes and
  * vq_last_error, streams, ownership, 16-byte alignment of device pointers) are those
  * stated in vqlinear.h.
@@ -27,6 +27,19 @@ extern "C" {
  * overlap is invalid.  One kernel launch (grid M x nshards) on `stream`. */
 vq_status vq_rht_apply_output_sharded(const void* y, void* y_out, const int8_t* signs, int32_t M, int32_t N,
                                       const int32_t* shard_n, int32_t nshards, int32_t dtype, void* stream);
+
+/* The plan vq_linear_plan would report for a handle created from `desc` and given
+ * the kernel choice `path` (VQ_PATH_AUTO, or a path as vq_linear_set_path forces
+ * it), on a device with `num_sms` SMs and `smem_optin` bytes of opt-in shared
+ * memory per block (a B200: 148 and 232448), with no SM budget.  Host arithmetic
+ * only: no handle, no device, no CUDA call, so it runs on any machine (capacity
+ * planning; tests of the path and tiling policy).
+ * VQ_ERR_INVALID_ARG for a NULL `desc` or `out`, an invalid `desc` (as
+ * vq_linear_create checks it), M outside [1, desc->max_M], num_sms < 1,
+ * smem_optin < 0 or `path` not a VQ_PATH_*; VQ_ERR_UNSUPPORTED when the path
+ * cannot take this M on such a device. */
+vq_status vq_plan_for_device(const vq_linear_desc* desc, int32_t M, int32_t path, int32_t num_sms,
+                             int32_t smem_optin, vq_plan_info* out);
 
 /* Nearest-entry encode of a dense weight matrix into index planes (orka README, "How
  * it works": "encode -> nearest-entry index per group", stored as bit-planes; the
