@@ -52,9 +52,10 @@ namespace vq {
 constexpr int kTcRows = 128;
 constexpr int kTcStages = 4;        // x tiles in shared memory and A tiles in TMEM (3 for two 64-token CTAs per SM)
 // Decode warps per TMEM lane quarter (kParts, a template parameter): 3 for token
-// tiles of 64 and more; for tiles of 16 to 48, 2 with two CTAs per SM (12-bit
-// formats) or 4 with one (16-bit formats, whose codeword gathers need the L1
-// cache that a second CTA's shared memory would take); see the launch.
+// tiles of 64 and more; 2 with two CTAs per SM for the 12-bit formats' tiles of
+// 16 to 48 tokens (and of 64 when the K split stays a cluster pair); 4 with one
+// CTA per SM for the 16-bit formats' narrower tiles, whose codeword gathers need
+// the L1 cache that a second CTA's shared memory would take; see the launch.
 __host__ __device__ constexpr int tc_threads(int parts) { return 64 + 32 * 4 * parts; }
 constexpr int kTcMaxT = 256;
 constexpr uint32_t kTcACols = 32;   // TMEM columns of one A stage (64 k of 16-bit pairs)
@@ -560,7 +561,7 @@ struct TcGeom {
   bool dual;  // two CTAs per SM (2 decode warps per lane quarter; 3 stages for 64-token tiles)
 };
 
-// fmt: kFmt*.
+// fmt: kFmt* (the same values as VQ_FMT_*).
 static TcGeom tc_geom(int fmt, int M, int N, int K, int num_sms) {
   TcGeom g;
   const int m16 = (M + 15) / 16 * 16;
